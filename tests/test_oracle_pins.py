@@ -1,0 +1,380 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+* the worked example of "Sparse Attention의 Indexer" (ai-systems-engineering.com),
+  Fig. 1-3, and a PIVOT example derived from those keys by hand;
+* hand-computed closed forms (ReLU, head weights, ties, padding);
+* special cases that reduce to library routines (numpy matmul + lexsort;
+  torch's float8 / bfloat16 casts; numpy mean on exact values);
+* invariants the abstract of arXiv 2607.24593 implies (g = 1 is the dense
+  indexer; Refine over every prefix position is the dense indexer; Reuse and
+  Refine pick from the candidate set; Refine's recall identity; decode equals
+  the last prefill group).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from top_token_selection_b200 import inputs as gen
+
+F32, BF16, E4M3 = oracle.F32, oracle.BF16, oracle.E4M3
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+def _tutorial_seq(ex):
+    keys = np.stack([ex["keys_first_component"], ex["keys_second_component"]], axis=1)
+    k = keys.astype(np.float32)
+    q = np.zeros((8, 1, 2), dtype=np.float32)
+    w = np.ones((8, 1), dtype=np.float32)
+    return q, w, k
+
+
+# ---------------------------------------------------------------------------
+# worked example
+# ---------------------------------------------------------------------------
+
+def test_tutorial_selection_scores_and_top3(golden_dir):
+    ex = _load(golden_dir, "indexer_tutorial_example.json")
+    q, w, k = _tutorial_seq(ex)
+    for case in ex["cases"]:
+        t = case["position"]
+        q[t, 0] = case["query"]
+        lo, hi = case["prefix"]
+        sc = oracle.score_positions(F32, q, None, w, k, None, t, np.arange(lo, hi + 1))
+        np.testing.assert_allclose(sc, case["scores"], rtol=0, atol=1e-6)
+        idx, _ = oracle.dense_index(F32, q, None, w, k, None, 3, rows=[t])
+        assert sorted(idx[0].tolist()) == case["top3_set"], case["figure"]
+
+
+def test_tutorial_window_union(golden_dir):
+    ex = _load(golden_dir, "indexer_tutorial_example.json")["window_union"]
+    u = oracle.window_union(ex["selected"], ex["position"], ex["window"])
+    assert u.tolist() == ex["union"]
+
+
+def _derived(golden_dir):
+    ex = _load(golden_dir, "pivot_derived_example.json")
+    k = np.array(ex["keys_x10"], dtype=np.float32)
+    return ex, k
+
+
+def test_derived_example_decode(golden_dir):
+    ex, k = _derived(golden_dir)
+    q = np.array([[m["query"] for m in ex["members"]]], dtype=np.float32)[:, :, None, :]
+    w = np.ones((1, 2, 1), dtype=np.float32)
+    kc = k[None]
+    cl = np.array([ex["cache_len"]], dtype=np.int32)
+    for mode, key, C in [(oracle.REUSE, "reuse", 3), (oracle.REFINE, "refine", 3),
+                         (oracle.REFINE, "refine_C8", 8), (oracle.DENSE, "dense", 3)]:
+        idx, cand, _ = oracle.decode(F32, q, None, w, kc, None, cl, mode, C, ex["topk"])
+        assert idx[0, 0].tolist() == ex[key]["6"], key
+        assert idx[0, 1].tolist() == ex[key]["7"], key
+        if mode != oracle.DENSE and C == ex["C"]:
+            assert cand[0].tolist() == ex["candidates"]
+
+
+def test_derived_example_prefill(golden_dir):
+    """Same example as a prefill with g = 2: group 3 holds positions 6 and 7."""
+    ex, k = _derived(golden_dir)
+    L, g = 8, 2
+    q = np.zeros((L, 1, 2), dtype=np.float32)
+    for m in ex["members"]:
+        q[m["position"], 0] = m["query"]
+    w = np.ones((L, 1), dtype=np.float32)
+    pq, _, pw = oracle.proxy_reduce(F32, q, None, w, g)
+    assert pq[3, 0].tolist() == ex["proxy_query"]
+    sc = oracle.score_positions(F32, pq, None, pw, k, None, 3, np.arange(8))
+    assert sc.tolist() == ex["proxy_scores"]
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, ex["C"])
+    assert cand[3].tolist() == ex["candidates"]
+    reuse = oracle.reuse(L, g, cand, 3, rows=[6, 7])
+    assert reuse.tolist() == [ex["reuse"]["6"], ex["reuse"]["7"]]
+    ref, _ = oracle.refine(F32, q, None, w, k, None, g, cand, 3, rows=[6, 7])
+    assert ref.tolist() == [ex["refine"]["6"], ex["refine"]["7"]]
+
+
+# ---------------------------------------------------------------------------
+# closed forms
+# ---------------------------------------------------------------------------
+
+def test_relu_and_head_weights_closed_form():
+    # q[t] has two heads: [1, 0] and [-1, 0]; w = [1, 2].
+    # key 0 = [2, 0]: 1*relu(2) + 2*relu(-2) = 2
+    # key 1 = [-3, 0]: 1*relu(-3) + 2*relu(3) = 6
+    # key 2 = [0, 5]: both dots 0 -> 0
+    q = np.zeros((3, 2, 2), dtype=np.float32)
+    q[2, 0] = [1, 0]
+    q[2, 1] = [-1, 0]
+    w = np.zeros((3, 2), dtype=np.float32)
+    w[2] = [1, 2]
+    k = np.array([[2, 0], [-3, 0], [0, 5]], dtype=np.float32)
+    sc = oracle.score_positions(F32, q, None, w, k, None, 2, [0, 1, 2])
+    assert sc.tolist() == [2.0, 6.0, 0.0]
+    idx, s = oracle.dense_index(F32, q, None, w, k, None, 3, rows=[2])
+    assert idx[0].tolist() == [1, 0, 2]
+    assert s[0].tolist() == [6.0, 2.0, 0.0]
+
+
+def test_scales_multiply_the_dot_product():
+    # e4m3 codes 0x38 = 1.0; q scale 3, k scale 0.5: I = w * relu(3 * 0.5 * D)
+    D = 4
+    q = np.full((2, 1, D), 0x38, dtype=np.uint8)
+    k = np.full((2, D), 0x38, dtype=np.uint8)
+    w = np.array([[1.0], [2.0]], dtype=np.float32)
+    sc = oracle.score_positions(E4M3, q, np.array([1.0, 3.0], np.float32), w, k,
+                                np.array([0.5, 0.25], np.float32), 1, [0, 1])
+    assert sc.tolist() == [2.0 * 3 * 0.5 * D, 2.0 * 3 * 0.25 * D]
+
+
+def test_ties_break_by_lower_position_and_short_prefix_pads():
+    L, H, D = 10, 1, 3
+    q = np.zeros((L, H, D), dtype=np.float32)   # every score is 0
+    k = np.ones((L, D), dtype=np.float32)
+    w = np.ones((L, H), dtype=np.float32)
+    idx, s = oracle.dense_index(F32, q, None, w, k, None, 4, rows=[9, 2])
+    assert idx[0].tolist() == [0, 1, 2, 3]
+    assert idx[1].tolist() == [0, 1, 2, -1]          # prefix 0..2 has 3 positions
+    assert np.isneginf(s[1, 3])
+    # negative weights give negative scores: the highest is still first
+    w[:] = -1.0
+    q[5, 0] = [1, 0, 0]
+    k[:, 0] = np.arange(L)
+    idx, _ = oracle.dense_index(F32, q, None, w, k, None, 3, rows=[5])
+    assert idx[0].tolist() == [0, 1, 2]              # scores 0, -1, -2, ...
+
+
+# ---------------------------------------------------------------------------
+# special case reducing to library routines
+# ---------------------------------------------------------------------------
+
+def test_single_head_nonnegative_is_plain_inner_product_topk():
+    rng = np.random.default_rng(7)
+    L, D, kk = 64, 5, 7
+    q = rng.random((L, 1, D), dtype=np.float32)
+    k = rng.random((L, D), dtype=np.float32)
+    w = np.ones((L, 1), dtype=np.float32)
+    idx, s = oracle.dense_index(F32, q, None, w, k, None, kk)
+    S = q[:, 0, :].astype(np.float64) @ k.astype(np.float64).T     # [t, s]
+    for t in range(L):
+        pos = np.arange(t + 1)
+        order = np.lexsort((pos, -S[t, : t + 1]))[:kk]
+        want = list(pos[order]) + [-1] * (kk - len(order))
+        assert idx[t].tolist() == want, t
+        np.testing.assert_allclose(s[t, : len(order)], S[t, order], rtol=1e-12)
+
+
+def test_topk_definition_brute_force():
+    """Every selected score >= every unselected one; ties resolved low-first."""
+    p = gen.make_prefill(24, 3, 4, F32, kind="int", seed=3)
+    q, qs, w, k, ks = p.codes()
+    kk = 6
+    idx, s = oracle.dense_index(F32, q, qs, w, k, ks, kk)
+    for t in range(24):
+        allsc = oracle.score_positions(F32, q, qs, w, k, ks, t, np.arange(t + 1))
+        sel = [i for i in idx[t] if i >= 0]
+        assert len(sel) == min(kk, t + 1)
+        rest = [i for i in range(t + 1) if i not in sel]
+        if rest:
+            lo = min(allsc[sel])
+            assert lo >= max(allsc[rest])
+            for i in rest:       # an unselected tie must sit at a higher position
+                if allsc[i] == lo:
+                    assert all(j < i for j in sel if allsc[j] == lo)
+
+
+# ---------------------------------------------------------------------------
+# formats against torch's casts
+# ---------------------------------------------------------------------------
+
+def test_e4m3_decode_all_codes_vs_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle.e4m3_to_float(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().double().numpy()
+    nan = np.isnan(ref)
+    assert (np.isnan(mine) == nan).all()
+    assert (mine[~nan] == ref[~nan]).all()
+
+
+def test_e4m3_encode_vs_torch_including_ties():
+    rng = np.random.default_rng(1)
+    vals = [rng.uniform(-448, 448, 4000), rng.uniform(-1, 1, 2000) * 2.0 ** -6,
+            rng.standard_normal(2000)]
+    # exact midpoints between neighbouring codes (round-half-even cases)
+    finite = oracle.e4m3_to_float(np.arange(0, 0x7F, dtype=np.uint8))
+    mids = (finite[:-1] + finite[1:]) / 2
+    vals += [mids, -mids]
+    x = np.concatenate(vals).astype(np.float32)
+    mine = oracle.float_to_e4m3(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert (mine == ref).all()
+    # saturation
+    assert oracle.float_to_e4m3(np.array([1e6, -1e6, 470.0])).tolist() == [0x7E, 0xFE, 0x7E]
+
+
+def test_bf16_codecs_vs_torch():
+    rng = np.random.default_rng(2)
+    x = np.concatenate([rng.standard_normal(5000) * 10.0 ** rng.integers(-30, 30, 5000),
+                        rng.standard_normal(100)]).astype(np.float32)
+    # exact ties: bf16 value + half an ulp
+    b = torch.from_numpy(rng.standard_normal(500).astype(np.float32)).to(torch.bfloat16).float()
+    ties = (b.view(torch.int32) + (1 << 15)).view(torch.float32).numpy()
+    x = np.concatenate([x, ties])
+    mine = oracle.float_to_bf16(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert (mine == ref).all()
+    dec = oracle.bf16_to_float(ref)
+    assert (dec == torch.from_numpy(ref.view(np.int16)).view(torch.bfloat16).double().numpy()).all()
+
+
+# ---------------------------------------------------------------------------
+# proxy
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", [F32, BF16, E4M3])
+def test_proxy_of_one_member_is_the_member(dtype):
+    p = gen.make_prefill(16, 2, 8, dtype, kind="dsa", seed=5)
+    q, qs, w, k, ks = p.codes()
+    pq, pqs, pw = oracle.proxy_reduce(dtype, q, qs, w, 1)
+    assert (pq == q).all() and (pw == w).all()
+    if dtype == E4M3:
+        assert (pqs == qs).all()
+
+
+def test_proxy_integer_mean_is_exact_and_partial_group_uses_member_count():
+    p = gen.make_prefill(10, 3, 5, F32, kind="int", seed=11)
+    q, _, w, _, _ = p.codes()
+    pq, _, pw = oracle.proxy_reduce(F32, q, None, w, 4)
+    assert pq.shape[0] == 3
+    for j, (a, b) in enumerate([(0, 4), (4, 8), (8, 10)]):
+        assert (pq[j] == q[a:b].astype(np.float64).mean(axis=0)).all()
+        assert (pw[j] == w[a:b].astype(np.float64).mean(axis=0)).all()
+
+
+def test_proxy_e4m3_requantisation():
+    p = gen.make_prefill(64, 4, 16, E4M3, kind="dsa", seed=12)
+    q, qs, w, _, _ = p.codes()
+    g = 8
+    pq, pqs, pw = oracle.proxy_reduce(E4M3, q, qs, w, g)
+    deq = oracle.e4m3_to_float(q) * qs[:, None, None]
+    for j in range(8):
+        mean = deq[j * g:(j + 1) * g].mean(axis=0)
+        amax = np.abs(mean).max()
+        assert abs(pqs[j] - amax / 448.0) <= 1e-6 * amax / 448.0
+        # codes are the saturating round-to-nearest-even of mean / scale
+        y = torch.from_numpy((mean / pqs[j]).astype(np.float32))
+        ref = y.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        mism = (pq[j] != ref)
+        # fp32 vs fp64 summation can move a value across a rounding midpoint
+        assert mism.mean() < 0.01
+        assert (pq[j] & 0x7F).max() == 0x7E            # the largest magnitude maps to 448
+
+
+def test_proxy_bf16_rounds_to_nearest():
+    p = gen.make_prefill(32, 4, 16, BF16, kind="dsa", seed=13)
+    q, _, w, _, _ = p.codes()
+    g = 8
+    pq, _, _ = oracle.proxy_reduce(BF16, q, None, w, g)
+    dq = oracle.bf16_to_float(q)
+    got = oracle.bf16_to_float(pq)
+    for j in range(4):
+        mean = dq[j * g:(j + 1) * g].mean(axis=0)
+        ulp = 2.0 ** (np.floor(np.log2(np.abs(mean) + 1e-30)) - 7)
+        assert (np.abs(got[j] - mean) <= 0.5 * ulp * 1.0001 + 1e-6 * np.abs(mean)).all()
+
+
+# ---------------------------------------------------------------------------
+# invariants of the method
+# ---------------------------------------------------------------------------
+
+def _int_case(L=48, H=3, D=6, seed=21):
+    p = gen.make_prefill(L, H, D, F32, kind="int", seed=seed)
+    return p.codes()
+
+
+def test_proxy_scan_is_dense_on_the_proxies_at_group_ends():
+    L, g, C = 45, 4, 9
+    q, _, w, k, _ = _int_case(L)
+    pq, _, pw = oracle.proxy_reduce(F32, q, None, w, g)
+    cand, cs = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, C)
+    # a sequence whose row e_j is proxy j
+    q2, w2 = q.copy(), w.copy()
+    ends = [min(L, (j + 1) * g) - 1 for j in range(pq.shape[0])]
+    for j, e in enumerate(ends):
+        q2[e], w2[e] = pq[j], pw[j]
+    dense, ds = oracle.dense_index(F32, q2, None, w2, k, None, C, rows=ends)
+    assert (cand == dense).all() and (cs == ds).all()
+
+
+def test_group_of_one_is_dense():
+    L, kk = 40, 5
+    q, _, w, k, _ = _int_case(L)
+    dense, _ = oracle.dense_index(F32, q, None, w, k, None, kk)
+    pq, _, pw = oracle.proxy_reduce(F32, q, None, w, 1)
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, 1, kk + 3)
+    assert (oracle.reuse(L, 1, cand, kk) == dense).all()
+    ref, _ = oracle.refine(F32, q, None, w, k, None, 1, cand, kk)
+    assert (ref == dense).all()
+
+
+def test_refine_over_the_whole_prefix_is_dense():
+    L, g, kk = 40, 4, 6
+    q, _, w, k, _ = _int_case(L)
+    dense, ds = oracle.dense_index(F32, q, None, w, k, None, kk)
+    pq, _, pw = oracle.proxy_reduce(F32, q, None, w, g)
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, L)
+    ref, rs = oracle.refine(F32, q, None, w, k, None, g, cand, kk)
+    assert (ref == dense).all() and (rs == ds).all()
+
+
+def test_reuse_refine_inside_candidates_and_recall_identity():
+    L, g, C, kk = 64, 8, 12, 6
+    q, _, w, k, _ = _int_case(L, H=4, D=8, seed=33)
+    dense, _ = oracle.dense_index(F32, q, None, w, k, None, kk)
+    pq, _, pw = oracle.proxy_reduce(F32, q, None, w, g)
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, C)
+    reu = oracle.reuse(L, g, cand, kk)
+    ref, _ = oracle.refine(F32, q, None, w, k, None, g, cand, kk)
+    for t in range(L):
+        cset = set(x for x in cand[t // g] if 0 <= x <= t)
+        rs = set(x for x in reu[t] if x >= 0)
+        fs = set(x for x in ref[t] if x >= 0)
+        ds = set(x for x in dense[t] if x >= 0)
+        assert rs <= cset and fs <= cset
+        assert all(x <= t for x in rs | fs)
+        # reuse keeps the proxy's rank order
+        assert [x for x in reu[t] if x >= 0] == [x for x in cand[t // g][:kk] if 0 <= x <= t]
+        # Refine keeps exactly the dense picks that are candidates (unique scores
+        # are not guaranteed on integer inputs, so compare through the scores)
+        assert len(fs) == min(kk, len(cset))
+        if len(ds & cset) == len(ds) and len(cset) >= kk:
+            sc = dict(zip(range(t + 1), oracle.score_positions(F32, q, None, w, k, None, t,
+                                                               np.arange(t + 1))))
+            assert sorted(sc[x] for x in fs) == sorted(sc[x] for x in ds)
+
+
+def test_decode_equals_last_prefill_group():
+    H, D, C, kk, n = 3, 6, 10, 5, 30
+    q, _, w, k, _ = _int_case(n, H, D, seed=44)
+    dq = q[n - 2:][None]
+    dw = w[n - 2:][None]
+    kc = k[None]
+    cl = np.array([n], dtype=np.int32)
+    pq, _, pw = oracle.proxy_reduce(F32, q, None, w, 2)
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, n, 2, C)
+    want = {
+        oracle.DENSE: oracle.dense_index(F32, q, None, w, k, None, kk, rows=[n - 2, n - 1])[0],
+        oracle.REUSE: oracle.reuse(n, 2, cand, kk, rows=[n - 2, n - 1]),
+        oracle.REFINE: oracle.refine(F32, q, None, w, k, None, 2, cand, kk, rows=[n - 2, n - 1])[0],
+    }
+    for mode, ref in want.items():
+        idx, dc, _ = oracle.decode(F32, dq, None, dw, kc, None, cl, mode, C, kk)
+        assert (idx[0] == ref).all(), mode
+        if dc is not None:
+            assert (dc[0] == cand[(n - 1) // 2]).all()
