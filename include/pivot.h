@@ -1,0 +1,193 @@
+/*
+ * pivot.h -- C ABI of libpivot, a B200 (sm_100a) implementation of the PIVOT
+ * proxy-query indexer for token-level sparse attention.
+ *
+ * What the library computes (cited by page title and section):
+ *  - The dense indexer ("Sparse Attention의 Indexer: 내용에 따라 읽을 위치
+ *    고르기", ai-systems-engineering.com, Fig. 1-2, and the abstract of
+ *    arXiv 2607.24593): for every query t, score each key s of its causal
+ *    prefix (0 <= s <= t, t included) and return the positions of the k
+ *    highest scores.  The score is the multi-head lightning-indexer form
+ *        I(t,s) = sum_h w[t,h] * ReLU(q[t,h] . k[s])
+ *    (times q_scale[t] * k_scale[s] for FP8 inputs).
+ *  - PIVOT (abstract of arXiv 2607.24593; "PIVOT 설명 ... 10분 만에
+ *    구현하기", molayo1419.me, section "How It Works"): group g nearby
+ *    queries, average them into one proxy query, run one full-prefix scan
+ *    per group to get a top-C candidate set, then either share the proxy's
+ *    top-k with every member (PIVOT-Reuse) or re-score the candidates with
+ *    each member's own query and take a per-member top-k (PIVOT-Refine).
+ *    Prefill groups are runs of g consecutive queries; decode groups are the
+ *    tokens decoded together in one MTP step.
+ *
+ * Conventions shared by every call:
+ *  - Every pointer argument is a DEVICE pointer owned by the caller, except
+ *    the pivot_seq_t / pivot_decode_t structs themselves (host memory, read
+ *    during the call only).  The library allocates no device memory on any
+ *    call; scratch space is the caller's workspace `ws` of `ws_bytes` bytes
+ *    (query the size with the matching *_workspace_size call).  `ws` must be
+ *    256-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Calls enqueue work and return; results are ready when the
+ *    stream reaches them.  Calls on distinct streams with distinct outputs
+ *    and workspaces may run concurrently.
+ *  - Layouts are row-major.  dtype PIVOT_F32: q, k are float32.  PIVOT_BF16:
+ *    bfloat16.  PIVOT_E4M3: OCP FP8 e4m3 codes with one float32 scale per
+ *    token (value = code * scale).  w is float32 in every dtype.
+ *  - Output index rows hold positions in rank order -- higher score first,
+ *    equal scores by lower position, -0 equal to +0 -- padded with -1 when
+ *    fewer positions are eligible.  Optional score outputs are float32 with
+ *    -inf padding.
+ *  - Argument errors are found before anything is enqueued and return
+ *    PIVOT_ERR_INVALID_ARG / _UNSUPPORTED / _WORKSPACE; a failed launch
+ *    returns PIVOT_ERR_CUDA.  Faults found by the kernels themselves (a
+ *    bounded wait that ran out, a bad cache length) set a per-device error
+ *    word read by pivot_get_device_error().
+ *  - FP8 and bf16 scoring runs on the tensor cores with fp32 accumulation;
+ *    PIVOT_F32 inputs are consumed at TF32 precision by the tensor cores
+ *    (exact for integer-valued inputs of magnitude < 2048).
+ */
+#ifndef PIVOT_H
+#define PIVOT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PIVOT_VERSION 100
+
+typedef enum {
+    PIVOT_OK = 0,
+    PIVOT_ERR_INVALID_ARG = 1,   /* null pointer, bad size, C < k, misaligned ... */
+    PIVOT_ERR_UNSUPPORTED = 2,   /* a shape this build does not implement       */
+    PIVOT_ERR_WORKSPACE = 3,     /* ws_bytes below the minimum for the call      */
+    PIVOT_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed         */
+    PIVOT_ERR_TIMEOUT = 5,       /* a kernel's bounded wait ran out              */
+    PIVOT_ERR_DEVICE = 6         /* a kernel found bad device-side data          */
+} pivot_status_t;
+
+typedef enum { PIVOT_F32 = 0, PIVOT_BF16 = 1, PIVOT_E4M3 = 2 } pivot_dtype_t;
+
+typedef enum {
+    PIVOT_MODE_DENSE = 0,        /* per-query full-prefix scan                   */
+    PIVOT_MODE_REUSE = 1,        /* the proxy's top-k shared by the group        */
+    PIVOT_MODE_REFINE = 2        /* candidates re-scored per member              */
+} pivot_mode_t;
+
+/* One prefill sequence.  Keys cover the whole sequence [0, L); the call
+ * indexes the query rows [t_begin, t_end) (t_end = 0 means L), so a long
+ * sequence can be split across calls or GPUs.  For the PIVOT calls t_begin
+ * must be a multiple of g.  Output rows are relative to t_begin (and group
+ * rows to t_begin / g). */
+typedef struct {
+    int32_t dtype;               /* pivot_dtype_t                                */
+    int32_t L, H, D;             /* sequence length, indexer heads, head dim     */
+    const void* q;               /* [L, H, D]                                    */
+    const float* q_scale;        /* [L] for PIVOT_E4M3, else NULL                */
+    const float* w;              /* [L, H] head weights                          */
+    const void* k;               /* [L, D] one shared indexer key per token      */
+    const float* k_scale;        /* [L] for PIVOT_E4M3, else NULL                */
+    int32_t t_begin, t_end;      /* query rows of this call                      */
+} pivot_seq_t;
+
+/* One MTP decode step over a batch of cached sequences.  cache_len[b]
+ * counts the keys of sequence b including the Gm new tokens' keys, which
+ * are already appended; member m (0-based) of sequence b is the token at
+ * position cache_len[b] - Gm + m and sees keys [0, cache_len[b] - Gm + m]. */
+typedef struct {
+    int32_t dtype;
+    int32_t B, Gm, H, D;         /* batch, MTP tokens per step (= group size)    */
+    int32_t maxlen;              /* key-cache capacity per sequence              */
+    const void* q;               /* [B, Gm, H, D]                                */
+    const float* q_scale;        /* [B, Gm] for PIVOT_E4M3, else NULL            */
+    const float* w;              /* [B, Gm, H]                                   */
+    const void* kc;              /* [B, maxlen, D]                               */
+    const float* kc_scale;       /* [B, maxlen] for PIVOT_E4M3, else NULL        */
+    const int32_t* cache_len;    /* [B] on the device, Gm <= cache_len <= maxlen */
+} pivot_decode_t;
+
+/* Dense indexer (Fig. 1-2 of the indexer tutorial; the baseline the PIVOT
+ * abstract compares with).  idx [rows, topk] int32; score [rows, topk] or
+ * NULL.  rows = t_end - t_begin.  topk >= 1. */
+pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* idx,
+                                 float* score, void* ws, size_t ws_bytes, void* stream);
+size_t pivot_dense_index_workspace_size(const pivot_seq_t* seq, int32_t topk);
+
+/* Proxy queries (PIVOT abstract: a group is aggregated into one proxy
+ * query; "How It Works": the proxy is the mean of the group).  For each
+ * group j of the call's rows (members [j*g, min(L,(j+1)*g))):
+ *   pq[j,h,d] = (sum over members of q value * q scale) / members   (fp32,
+ *               left to right in member order, no fused multiply-add)
+ *   pw[j,h]   = (sum over members of w) / members
+ * stored in seq->dtype: f32 as is, bf16 rounded to nearest even, e4m3 with
+ * pq_scale[j] = amax/448 (1 if amax = 0) and codes = e4m3(pq / pq_scale),
+ * rounded to nearest even and saturated.  A one-member group is copied
+ * unchanged (codes, scale and weights).  pq [G, H, D], pq_scale [G]
+ * (PIVOT_E4M3, else NULL), pw [G, H]; G = ceil(rows / g).  pq must be
+ * 16-byte aligned. */
+pivot_status_t pivot_proxy_reduce(const pivot_seq_t* seq, int32_t g, void* pq,
+                                  float* pq_scale, float* pw, void* stream);
+
+/* One full-prefix scan per group (PIVOT abstract): proxy j scores keys
+ * [0, e_j], e_j = min(L, (j+1)*g) - 1, with the dense score formula and
+ * keeps its top-C.  cand [G, C] int32 in rank order (its first k entries
+ * are the proxy's top-k); cand_score [G, C] or NULL.  1 <= C. */
+pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* pq,
+                                 const float* pq_scale, const float* pw, int32_t C,
+                                 int32_t* cand, float* cand_score, void* ws,
+                                 size_t ws_bytes, void* stream);
+size_t pivot_proxy_scan_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C);
+
+/* PIVOT-Reuse (PIVOT abstract): member t of group j takes the first topk
+ * entries of cand[j], keeps those <= t in their order and pads with -1.
+ * Rows [t_begin, t_end) with t_begin a multiple of g; cand rows relative to
+ * t_begin / g.  idx [rows, topk].  1 <= topk <= C. */
+pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int32_t* cand,
+                           int32_t C, int32_t topk, int32_t* idx, void* stream);
+
+/* PIVOT-Refine (PIVOT abstract): member t of group j scores every candidate
+ * s in cand[j] with 0 <= s <= t using its own q[t], w[t] (the dense score
+ * formula) and keeps the top-k.  idx [rows, topk], score [rows, topk] or
+ * NULL.  1 <= topk <= C. */
+pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* cand,
+                            int32_t C, int32_t topk, int32_t* idx, float* score, void* ws,
+                            size_t ws_bytes, void* stream);
+size_t pivot_refine_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C, int32_t topk);
+
+/* One MTP decode step (PIVOT abstract: the tokens decoded together form the
+ * group).  PIVOT_MODE_DENSE: each member scans its own prefix.  REUSE /
+ * REFINE: the Gm members' proxy scans [0, cache_len[b] - 1] for its top-C,
+ * then Reuse or Refine as in prefill.  idx [B, Gm, topk]; cand [B, C] or
+ * NULL (the candidates, PIVOT modes only). */
+pivot_status_t pivot_decode(const pivot_decode_t* batch, int32_t mode, int32_t C,
+                            int32_t topk, int32_t* idx, int32_t* cand, void* ws,
+                            size_t ws_bytes, void* stream);
+size_t pivot_decode_workspace_size(const pivot_decode_t* batch, int32_t mode, int32_t C,
+                                   int32_t topk);
+
+/* Waits for `stream`, then returns and clears the current device's error
+ * word: PIVOT_OK, PIVOT_ERR_TIMEOUT or PIVOT_ERR_DEVICE (PIVOT_ERR_CUDA if
+ * the wait itself failed). */
+pivot_status_t pivot_get_device_error(void* stream);
+
+/* Test hook: bounded waits give up after `ns` nanoseconds of waiting on the
+ * current device (0 restores the default of 4 s).  Used to prove that a
+ * wait that runs out returns an error instead of hanging. */
+pivot_status_t pivot_set_wait_limit_ns(uint64_t ns);
+
+/* Test hook: enqueue one kernel whose single wait is on a barrier nothing
+ * arrives on.  With the wait limit lowered, a following
+ * pivot_get_device_error() returns PIVOT_ERR_TIMEOUT and the device stays
+ * usable.  Not needed in normal use. */
+pivot_status_t pivot_selftest_wait_timeout(void* stream);
+
+const char* pivot_status_string(pivot_status_t status);
+int32_t pivot_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PIVOT_H */

@@ -1,0 +1,114 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, and rejects bad arguments before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from top_token_selection_b200 import build as pbuild
+from top_token_selection_b200 import pivot as pv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pivot.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pbuild.build()
+    return pv.load()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pivot_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert header_functions() == sorted(pv.ABI_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", pv.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (pivot_\w+)", out))
+    missing = [f for f in header_functions() if f not in exported]
+    assert not missing, missing
+    for f in header_functions():
+        assert hasattr(lib, f)
+
+
+def test_version_and_status_strings(lib):
+    assert pv.pivot_version() == 100
+    assert pv.pivot_status_string(0) == "ok"
+    assert pv.pivot_status_string(3) == "workspace too small"
+
+
+FAKE = 0x10000   # never dereferenced: every call below fails validation first
+
+
+def _seq(**kw):
+    base = dict(dtype=pv.F32, L=64, H=4, D=32, q=FAKE, q_scale=None, w=FAKE, k=FAKE,
+                k_scale=None, t_begin=0, t_end=0)
+    base.update(kw)
+    return pv.PivotSeq(**base)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(dtype=7), dict(L=0), dict(H=0), dict(q=None), dict(w=None), dict(k=None),
+    dict(q_scale=FAKE),                       # f32 takes no scales
+    dict(dtype=pv.E4M3, D=128),               # e4m3 needs both scales
+    dict(t_begin=10, t_end=5), dict(t_end=65), dict(q=FAKE + 4),
+])
+def test_dense_rejects_bad_sequences(lib, bad):
+    seq = _seq(**bad)
+    st = pv.pivot_dense_index(seq, 8, FAKE, None, FAKE, 1 << 20, None)
+    assert st == 1, bad
+
+
+def test_dense_rejects_bad_topk_and_workspace(lib):
+    seq = _seq()
+    assert pv.pivot_dense_index(seq, 0, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_dense_index(seq, 8, None, None, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_dense_index(seq, 8, FAKE, None, None, 1 << 20, None) == 1
+    assert pv.pivot_dense_index(seq, 8, FAKE, None, FAKE + 16, 1 << 20, None) == 1  # alignment
+    assert pv.pivot_dense_index(seq, 8, FAKE, None, FAKE, 64, None) == 3            # too small
+    assert pv.pivot_dense_index(seq, 1 << 20, FAKE, None, FAKE, 1 << 20, None) == 2
+
+
+def test_group_and_candidate_checks(lib):
+    seq = _seq(t_begin=3)
+    assert pv.pivot_proxy_reduce(seq, 4, FAKE, None, FAKE, None) == 1      # t_begin % g
+    seq = _seq()
+    assert pv.pivot_proxy_reduce(seq, 0, FAKE, None, FAKE, None) == 1      # g >= 1
+    assert pv.pivot_proxy_reduce(seq, 4, FAKE, FAKE, FAKE, None) == 1      # no pq_scale for f32
+    assert pv.pivot_proxy_scan(seq, 4, FAKE, None, FAKE, 0, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_reuse(0, 64, 4, FAKE, 8, 16, FAKE, None) == 1           # C < k
+    assert pv.pivot_reuse(1, 64, 4, FAKE, 16, 8, FAKE, None) == 1           # t_begin % g
+    assert pv.pivot_refine(seq, 4, FAKE, 8, 16, FAKE, None, FAKE, 1 << 20, None) == 1
+
+
+def test_workspace_sizes(lib):
+    seq = _seq(L=1000, H=4, D=32)
+    n = pv.pivot_dense_index_workspace_size(seq, 64)
+    assert n >= 1000 * 1024 * 4 and n % 256 == 0
+    assert pv.pivot_proxy_scan_workspace_size(seq, 4, 256) >= 250 * 1024 * 4
+    assert pv.pivot_refine_workspace_size(seq, 4, 256, 64) >= 1000 * 256 * 4
+    assert pv.pivot_dense_index_workspace_size(_seq(L=0), 64) == 0
+    dec = pv.PivotDecode(pv.E4M3, 4, 2, 64, 128, 4096, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert pv.pivot_decode_workspace_size(dec, pv.DENSE, 0, 64) >= 8 * 4096 * 4
+    assert pv.pivot_decode_workspace_size(dec, pv.REFINE, 256, 64) > \
+        pv.pivot_decode_workspace_size(dec, pv.REUSE, 256, 64)
+    assert pv.pivot_decode_workspace_size(dec, pv.REUSE, 32, 64) == 0      # C < k
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = pv._lib
+    try:
+        pv._lib = None
+        with pytest.raises(ImportError):
+            pv.load(str(tmp_path / "nope.so"))
+    finally:
+        pv._lib = saved

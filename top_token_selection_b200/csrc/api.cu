@@ -1,0 +1,622 @@
+// api.cu -- the libpivot C ABI: argument checks, workspace carving, TMA
+// descriptors and kernel launches.  See include/pivot.h for the contract.
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pivot {
+
+__device__ uint32_t g_error_word = 0;
+__device__ uint64_t g_wait_limit_ns = 4000000000ull;
+
+namespace {
+
+constexpr size_t WS_ALIGN = 256;
+constexpr size_t SCORE_BUF_CAP = size_t(4) << 30;   // preferred score buffer, 4 GiB
+constexpr int MAX_K = 16384;
+constexpr int TAIL_CAP = 4096;
+constexpr int MAX_SMS = 1024;
+
+int esize_of(int dtype) { return dtype == PIVOT_F32 ? 4 : (dtype == PIVOT_BF16 ? 2 : 1); }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (cache[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? (n < MAX_SMS ? n : MAX_SMS) : 148;
+    }
+    return cache[dev];
+}
+
+// ------------------------------------------------------------------ TMA maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D map over rows x cols elements (row stride = cols * esize), box of
+// 128 bytes x box_rows, 128-byte swizzle, zero fill out of bounds.
+bool make_tmap(CUtensorMap* map, int dtype, const void* base, long long rows, int cols,
+               int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const int es = esize_of(dtype);
+    CUtensorMapDataType dt = dtype == PIVOT_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                             : dtype == PIVOT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t gstride[1] = {(cuuint64_t)cols * es};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / es), (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void*>(base), gdim, gstride, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- validation
+bool dtype_ok(int dt) { return dt == PIVOT_F32 || dt == PIVOT_BF16 || dt == PIVOT_E4M3; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Tensor-core tiling: N = P*H <= 256 with H in {4..64}; key rows of 128 or
+// 256 bytes (two 128-byte swizzle atoms).
+bool umma_shape_ok(int H, int D, int dtype) {
+    const int rb = D * esize_of(dtype);
+    return (H == 4 || H == 8 || H == 16 || H == 32 || H == 64) && (rb == 128 || rb == 256);
+}
+
+bool simt_shape_ok(int H, int D) {
+    const size_t smem = ((size_t)D * 128 + (size_t)H * D + H) * 4;
+    return smem <= 200 * 1024;
+}
+
+pivot_status_t check_seq(const pivot_seq_t* s, int* t0, int* t1) {
+    if (!s || !dtype_ok(s->dtype)) return PIVOT_ERR_INVALID_ARG;
+    if (s->L < 1 || s->H < 1 || s->D < 1) return PIVOT_ERR_INVALID_ARG;
+    if (!s->q || !s->w || !s->k) return PIVOT_ERR_INVALID_ARG;
+    const bool fp8 = s->dtype == PIVOT_E4M3;
+    if (fp8 != (s->q_scale != nullptr) || fp8 != (s->k_scale != nullptr))
+        return PIVOT_ERR_INVALID_ARG;
+    *t0 = s->t_begin;
+    *t1 = s->t_end == 0 ? s->L : s->t_end;
+    if (*t0 < 0 || *t1 > s->L || *t0 >= *t1) return PIVOT_ERR_INVALID_ARG;
+    if (!aligned16(s->q) || !aligned16(s->k)) return PIVOT_ERR_INVALID_ARG;
+    if ((s->D * esize_of(s->dtype)) % 16) return PIVOT_ERR_UNSUPPORTED;
+    if (!umma_shape_ok(s->H, s->D, s->dtype) && !simt_shape_ok(s->H, s->D))
+        return PIVOT_ERR_UNSUPPORTED;
+    return PIVOT_OK;
+}
+
+pivot_status_t check_group_range(const pivot_seq_t* s, int g, int t0, int t1) {
+    if (g < 1) return PIVOT_ERR_INVALID_ARG;
+    if (t0 % g) return PIVOT_ERR_INVALID_ARG;
+    if (t1 != s->L && t1 % g) return PIVOT_ERR_INVALID_ARG;
+    return PIVOT_OK;
+}
+
+pivot_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? PIVOT_OK : PIVOT_ERR_CUDA; }
+
+long long score_stride(int nkeys) { return (long long)align_up((size_t)nkeys, 32); }
+
+// Rows of scores that fit in `bytes`, a multiple of `unit`, at least one unit.
+long long rows_fitting(size_t bytes, long long stride, int unit) {
+    long long r = (long long)(bytes / ((size_t)stride * 4));
+    return r / unit * unit;
+}
+
+// ------------------------------------------------------------------ scans
+// Rows [r0, r1) of kind `kind` into S (row r at S + (r - r0)*stride).
+pivot_status_t run_scan(int kind, int dtype, int H, int D, const void* qbase, long long q_rows,
+                        int qrow_base, const float* w, const float* q_scale, const void* kbase,
+                        long long k_rows, const float* k_scale, int L, int g, int Gm, int maxlen,
+                        const int32_t* cache_len, int P, int r0, int r1, int maxlim_total,
+                        float* S, long long stride, cudaStream_t st) {
+    ScanParams p{};
+    p.kind = kind;
+    p.dtype = dtype;
+    p.esize = esize_of(dtype);
+    p.H = H;
+    p.D = D;
+    p.P = P;
+    p.row0 = r0;
+    p.nrows = r1 - r0;
+    p.qrow_base = qrow_base;
+    p.L = L;
+    p.g = g;
+    p.Gm = Gm;
+    p.maxlen = maxlen;
+    p.cache_len = cache_len;
+    p.w = w;
+    p.q_scale = q_scale;
+    p.k_scale = k_scale;
+    p.S = S;
+    p.S_stride = stride;
+    const int nblocks = ceil_div(p.nrows, P);
+    const int nt = ceil_div(maxlim_total + 1, 128);
+    const int N = P * H;
+    if (umma_shape_ok(H, D, dtype) && N >= 16 && N <= 256 && N % 16 == 0) {
+        const bool decode = kind == SCAN_DECODE_DENSE || kind == SCAN_DECODE_PROXY;
+        p.tiles_per_item = decode ? 8 : 32;
+        p.items_per_block = ceil_div(nt, p.tiles_per_item);
+        p.nitems = nblocks * p.items_per_block;
+        CUtensorMap tk, tq;
+        if (!make_tmap(&tk, dtype, kbase, k_rows, D, 128)) return PIVOT_ERR_CUDA;
+        if (!make_tmap(&tq, dtype, qbase, q_rows * H, D, P * H)) return PIVOT_ERR_CUDA;
+        const int grid = p.nitems < num_sms() ? p.nitems : num_sms();
+        return from_cuda(launch_scan_umma(tk, tq, p, grid, st));
+    }
+    p.tiles_per_item = 1;
+    p.items_per_block = nt;
+    p.nitems = nblocks * nt;
+    return from_cuda(launch_scan_simt(qbase, kbase, p, st));
+}
+
+int rows_per_block(int H, int D, int dtype) {
+    return umma_shape_ok(H, D, dtype) ? 256 / H : 8;
+}
+
+pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, int Gm, int maxlen,
+                                 const int32_t* cache_len, const float* S, long long stride,
+                                 int K, int32_t* out, float* out_score, int out_base,
+                                 cudaStream_t st) {
+    SelectParams sp{};
+    sp.kind = SEL_PREFIX;
+    sp.scan_kind = scan_kind;
+    sp.row0 = r0;
+    sp.nrows = r1 - r0;
+    sp.L = L;
+    sp.g = g;
+    sp.Gm = Gm;
+    sp.maxlen = maxlen;
+    sp.cache_len = cache_len;
+    sp.S = S;
+    sp.S_stride = stride;
+    sp.K = K;
+    sp.out_idx = out;
+    sp.out_score = out_score;
+    sp.out_base = out_base;
+    sp.tail_cap = TAIL_CAP;
+    return from_cuda(launch_select(sp, st));
+}
+
+pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int Gm, int maxlen,
+                               const int32_t* cache_len, const float* S, const int32_t* cand,
+                               int cand_base, int C, int K, int32_t* out, float* out_score,
+                               int out_base, cudaStream_t st) {
+    SelectParams sp{};
+    sp.kind = SEL_CANDIDATES;
+    sp.scan_kind = scan_kind;
+    sp.row0 = r0;
+    sp.nrows = r1 - r0;
+    sp.L = L;
+    sp.g = g;
+    sp.Gm = Gm;
+    sp.maxlen = maxlen;
+    sp.cache_len = cache_len;
+    sp.S = S;
+    sp.S_stride = C;
+    sp.cand = cand;
+    sp.cand_base = cand_base;
+    sp.C = C;
+    sp.K = K;
+    sp.out_idx = out;
+    sp.out_score = out_score;
+    sp.out_base = out_base;
+    sp.tail_cap = TAIL_CAP;
+    return from_cuda(launch_select(sp, st));
+}
+
+pivot_status_t run_refine_scores(int kind, int dtype, int H, int D, const void* q,
+                                 int qrow_base, const float* q_scale, const float* w,
+                                 const void* k, const float* k_scale, int L, int g, int Gm,
+                                 int maxlen, const int32_t* cache_len, const int32_t* cand,
+                                 int cand_base, int C, int r0, int r1, float* S, cudaStream_t st) {
+    RefineParams rp{};
+    rp.dtype = dtype;
+    rp.esize = esize_of(dtype);
+    rp.H = H;
+    rp.D = D;
+    rp.kind = kind;
+    rp.row0 = r0;
+    rp.nrows = r1 - r0;
+    rp.qrow_base = qrow_base;
+    rp.L = L;
+    rp.g = g;
+    rp.Gm = Gm;
+    rp.maxlen = maxlen;
+    rp.cache_len = cache_len;
+    rp.q = q;
+    rp.q_scale = q_scale;
+    rp.w = w;
+    rp.k = k;
+    rp.k_scale = k_scale;
+    rp.cand = cand;
+    rp.cand_base = cand_base;
+    rp.C = C;
+    rp.S = S;
+    return from_cuda(launch_refine_simt(rp, st));
+}
+
+// Carve `bytes` (256-aligned) from the workspace cursor.
+struct Carver {
+    uint8_t* base;
+    size_t cap, off = 0;
+    bool ok = true;
+    void* take(size_t bytes) {
+        off = align_up(off, WS_ALIGN);
+        if (off + bytes > cap) { ok = false; return nullptr; }
+        void* p = base + off;
+        off += bytes;
+        return p;
+    }
+};
+
+size_t dense_rowbytes(int L) { return (size_t)score_stride(L) * 4; }
+
+// One thread waits on an mbarrier that nothing arrives on: the bounded wait
+// must run out, raise the timeout bit and let the kernel return.
+__global__ void wait_selftest_kernel() {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0);
+}
+
+}  // namespace
+
+cudaError_t launch_wait_selftest(cudaStream_t stream) {
+    wait_selftest_kernel<<<1, 32, 0, stream>>>();
+    return cudaGetLastError();
+}
+
+}  // namespace pivot
+
+using namespace pivot;
+
+extern "C" {
+
+int32_t pivot_version(void) { return PIVOT_VERSION; }
+
+const char* pivot_status_string(pivot_status_t s) {
+    switch (s) {
+        case PIVOT_OK: return "ok";
+        case PIVOT_ERR_INVALID_ARG: return "invalid argument";
+        case PIVOT_ERR_UNSUPPORTED: return "unsupported shape";
+        case PIVOT_ERR_WORKSPACE: return "workspace too small";
+        case PIVOT_ERR_CUDA: return "CUDA error";
+        case PIVOT_ERR_TIMEOUT: return "a kernel wait timed out";
+        case PIVOT_ERR_DEVICE: return "bad device-side data";
+    }
+    return "unknown status";
+}
+
+pivot_status_t pivot_get_device_error(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return PIVOT_ERR_CUDA;
+    uint32_t w = 0;
+    if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return PIVOT_ERR_CUDA;
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return PIVOT_ERR_CUDA;
+    if (w & ERRBIT_TIMEOUT) return PIVOT_ERR_TIMEOUT;
+    if (w & ERRBIT_DATA) return PIVOT_ERR_DEVICE;
+    return PIVOT_OK;
+}
+
+pivot_status_t pivot_set_wait_limit_ns(uint64_t ns) {
+    const uint64_t v = ns ? ns : 4000000000ull;
+    return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? PIVOT_OK
+                                                                            : PIVOT_ERR_CUDA;
+}
+
+pivot_status_t pivot_selftest_wait_timeout(void* stream) {
+    return launch_wait_selftest(static_cast<cudaStream_t>(stream)) == cudaSuccess ? PIVOT_OK
+                                                                                  : PIVOT_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ dense
+size_t pivot_dense_index_workspace_size(const pivot_seq_t* seq, int32_t topk) {
+    int t0, t1;
+    if (check_seq(seq, &t0, &t1) != PIVOT_OK || topk < 1) return 0;
+    const int P = rows_per_block(seq->H, seq->D, seq->dtype);
+    const size_t rb = dense_rowbytes(seq->L);
+    long long rows = t1 - t0;
+    long long cap = (long long)(SCORE_BUF_CAP / rb) / P * P;
+    if (cap < P) cap = P;
+    if (rows > cap) rows = cap;
+    return align_up((size_t)rows * rb, WS_ALIGN);
+}
+
+pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* idx, float* score,
+                                 void* ws, size_t ws_bytes, void* stream) {
+    int t0, t1;
+    pivot_status_t st = check_seq(seq, &t0, &t1);
+    if (st != PIVOT_OK) return st;
+    if (topk < 1 || !idx) return PIVOT_ERR_INVALID_ARG;
+    if (topk > MAX_K) return PIVOT_ERR_UNSUPPORTED;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
+    const int P = rows_per_block(seq->H, seq->D, seq->dtype);
+    const long long stride = score_stride(seq->L);
+    long long chunk = rows_fitting(ws_bytes, stride, P);
+    if (chunk < P) return PIVOT_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* S = static_cast<float*>(ws);
+    for (long long c0 = t0; c0 < t1; c0 += chunk) {
+        const int r0 = (int)c0;
+        const int r1 = (int)(c0 + chunk < t1 ? c0 + chunk : t1);
+        st = run_scan(SCAN_PREFILL_DENSE, seq->dtype, seq->H, seq->D, seq->q, seq->L, 0, seq->w,
+                      seq->q_scale, seq->k, seq->L, seq->k_scale, seq->L, 1, 1, 0, nullptr, P, r0,
+                      r1, r1 - 1, S, stride, s);
+        if (st != PIVOT_OK) return st;
+        st = run_select_prefix(SCAN_PREFILL_DENSE, r0, r1, seq->L, 1, 1, 0, nullptr, S, stride,
+                               topk, idx, score, t0, s);
+        if (st != PIVOT_OK) return st;
+    }
+    return PIVOT_OK;
+}
+
+// ------------------------------------------------------------ proxy reduce
+pivot_status_t pivot_proxy_reduce(const pivot_seq_t* seq, int32_t g, void* pq, float* pq_scale,
+                                  float* pw, void* stream) {
+    int t0, t1;
+    pivot_status_t st = check_seq(seq, &t0, &t1);
+    if (st != PIVOT_OK) return st;
+    if ((st = check_group_range(seq, g, t0, t1)) != PIVOT_OK) return st;
+    if (!pq || !pw || !aligned16(pq)) return PIVOT_ERR_INVALID_ARG;
+    if ((seq->dtype == PIVOT_E4M3) != (pq_scale != nullptr)) return PIVOT_ERR_INVALID_ARG;
+    ReduceParams rp{};
+    rp.dtype = seq->dtype;
+    rp.esize = esize_of(seq->dtype);
+    rp.H = seq->H;
+    rp.D = seq->D;
+    rp.nmembers_total = t1 - t0;
+    rp.g = g;
+    rp.ngroups = ceil_div(t1 - t0, g);
+    rp.q = static_cast<const uint8_t*>(seq->q) + (size_t)t0 * seq->H * seq->D * rp.esize;
+    rp.q_scale = seq->q_scale ? seq->q_scale + t0 : nullptr;
+    rp.w = seq->w + (size_t)t0 * seq->H;
+    rp.pq = pq;
+    rp.pq_scale = pq_scale;
+    rp.pw = pw;
+    rp.group_stride_members = g;
+    return from_cuda(launch_proxy_reduce(rp, static_cast<cudaStream_t>(stream)));
+}
+
+// -------------------------------------------------------------- proxy scan
+size_t pivot_proxy_scan_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C) {
+    int t0, t1;
+    if (check_seq(seq, &t0, &t1) != PIVOT_OK || g < 1 || C < 1) return 0;
+    const int P = rows_per_block(seq->H, seq->D, seq->dtype);
+    const size_t rb = dense_rowbytes(seq->L);
+    long long rows = ceil_div(t1 - t0, g);
+    long long cap = (long long)(SCORE_BUF_CAP / rb) / P * P;
+    if (cap < P) cap = P;
+    if (rows > cap) rows = cap;
+    return align_up((size_t)rows * rb, WS_ALIGN);
+}
+
+pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* pq,
+                                 const float* pq_scale, const float* pw, int32_t C, int32_t* cand,
+                                 float* cand_score, void* ws, size_t ws_bytes, void* stream) {
+    int t0, t1;
+    pivot_status_t st = check_seq(seq, &t0, &t1);
+    if (st != PIVOT_OK) return st;
+    if ((st = check_group_range(seq, g, t0, t1)) != PIVOT_OK) return st;
+    if (!pq || !pw || !cand || !aligned16(pq) || C < 1) return PIVOT_ERR_INVALID_ARG;
+    if ((seq->dtype == PIVOT_E4M3) != (pq_scale != nullptr)) return PIVOT_ERR_INVALID_ARG;
+    if (C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
+    const int P = rows_per_block(seq->H, seq->D, seq->dtype);
+    const long long stride = score_stride(seq->L);
+    long long chunk = rows_fitting(ws_bytes, stride, P);
+    if (chunk < P) return PIVOT_ERR_WORKSPACE;
+    const int j0 = t0 / g, j1 = ceil_div(t1, g);
+    const int G = j1 - j0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* S = static_cast<float*>(ws);
+    for (long long c0 = j0; c0 < j1; c0 += chunk) {
+        const int r0 = (int)c0;
+        const int r1 = (int)(c0 + chunk < j1 ? c0 + chunk : j1);
+        const int e_last = (r1 * g < seq->L ? r1 * g : seq->L) - 1;
+        st = run_scan(SCAN_PREFILL_PROXY, seq->dtype, seq->H, seq->D, pq, G, j0, pw, pq_scale,
+                      seq->k, seq->L, seq->k_scale, seq->L, g, 1, 0, nullptr, P, r0, r1, e_last, S,
+                      stride, s);
+        if (st != PIVOT_OK) return st;
+        st = run_select_prefix(SCAN_PREFILL_PROXY, r0, r1, seq->L, g, 1, 0, nullptr, S, stride, C,
+                               cand, cand_score, j0, s);
+        if (st != PIVOT_OK) return st;
+    }
+    return PIVOT_OK;
+}
+
+// ------------------------------------------------------------------- reuse
+pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int32_t* cand,
+                           int32_t C, int32_t topk, int32_t* idx, void* stream) {
+    if (g < 1 || t_begin < 0 || t_end <= t_begin || t_begin % g) return PIVOT_ERR_INVALID_ARG;
+    if (!cand || !idx || topk < 1 || C < topk) return PIVOT_ERR_INVALID_ARG;
+    return from_cuda(
+        launch_reuse(t_begin, t_end, g, cand, C, topk, idx, static_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------------------------------ refine
+size_t pivot_refine_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C, int32_t topk) {
+    int t0, t1;
+    if (check_seq(seq, &t0, &t1) != PIVOT_OK || g < 1 || C < 1 || topk < 1) return 0;
+    long long rows = t1 - t0;
+    const size_t rb = (size_t)C * 4;
+    long long cap = (long long)(SCORE_BUF_CAP / rb) / g * g;
+    if (cap < g) cap = g;
+    if (rows > cap) rows = cap;
+    return align_up((size_t)rows * rb, WS_ALIGN);
+}
+
+pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* cand, int32_t C,
+                            int32_t topk, int32_t* idx, float* score, void* ws, size_t ws_bytes,
+                            void* stream) {
+    int t0, t1;
+    pivot_status_t st = check_seq(seq, &t0, &t1);
+    if (st != PIVOT_OK) return st;
+    if ((st = check_group_range(seq, g, t0, t1)) != PIVOT_OK) return st;
+    if (!cand || !idx || topk < 1 || C < topk) return PIVOT_ERR_INVALID_ARG;
+    if (C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
+    long long chunk = (long long)(ws_bytes / ((size_t)C * 4)) / g * g;
+    if (chunk < g) return PIVOT_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* S = static_cast<float*>(ws);
+    const int j0 = t0 / g;
+    for (long long c0 = t0; c0 < t1; c0 += chunk) {
+        const int r0 = (int)c0;
+        const int r1 = (int)(c0 + chunk < t1 ? c0 + chunk : t1);
+        const int jc = r0 / g;
+        st = run_refine_scores(SCAN_PREFILL_DENSE, seq->dtype, seq->H, seq->D, seq->q, 0,
+                               seq->q_scale, seq->w, seq->k, seq->k_scale, seq->L, g, 1, 0,
+                               nullptr, cand + (size_t)(jc - j0) * C, jc, C, r0, r1, S, s);
+        if (st != PIVOT_OK) return st;
+        st = run_select_cand(SCAN_PREFILL_DENSE, r0, r1, seq->L, g, 1, 0, nullptr, S,
+                             cand + (size_t)(jc - j0) * C, jc, C, topk, idx, score, t0, s);
+        if (st != PIVOT_OK) return st;
+    }
+    return PIVOT_OK;
+}
+
+// ------------------------------------------------------------------ decode
+static pivot_status_t check_decode(const pivot_decode_t* b) {
+    if (!b || !dtype_ok(b->dtype)) return PIVOT_ERR_INVALID_ARG;
+    if (b->B < 1 || b->Gm < 1 || b->H < 1 || b->D < 1 || b->maxlen < b->Gm)
+        return PIVOT_ERR_INVALID_ARG;
+    if (!b->q || !b->w || !b->kc || !b->cache_len) return PIVOT_ERR_INVALID_ARG;
+    const bool fp8 = b->dtype == PIVOT_E4M3;
+    if (fp8 != (b->q_scale != nullptr) || fp8 != (b->kc_scale != nullptr))
+        return PIVOT_ERR_INVALID_ARG;
+    if (!aligned16(b->q) || !aligned16(b->kc)) return PIVOT_ERR_INVALID_ARG;
+    if ((b->D * esize_of(b->dtype)) % 16) return PIVOT_ERR_UNSUPPORTED;
+    if (!umma_shape_ok(b->H, b->D, b->dtype) && !simt_shape_ok(b->H, b->D))
+        return PIVOT_ERR_UNSUPPORTED;
+    if (b->Gm * b->H > 256 && !simt_shape_ok(b->H, b->D)) return PIVOT_ERR_UNSUPPORTED;
+    return PIVOT_OK;
+}
+
+struct DecodeWs {
+    float* S;       // [B*Gm or B, stride]
+    void* pq;       // [B, H, D]
+    float* pqs;     // [B]
+    float* pw;      // [B, H]
+    int32_t* cand;  // [B, C]
+    float* R;       // [B*Gm, C]
+};
+
+static size_t decode_layout(const pivot_decode_t* b, int mode, int C, DecodeWs* out, void* base,
+                            size_t cap) {
+    Carver c{static_cast<uint8_t*>(base), base ? cap : ~size_t(0) / 2};
+    if (!base) c.base = reinterpret_cast<uint8_t*>(WS_ALIGN);   // size query only
+    const long long stride = score_stride(b->maxlen);
+    const int rows = mode == PIVOT_MODE_DENSE ? b->B * b->Gm : b->B;
+    DecodeWs w{};
+    w.S = static_cast<float*>(c.take((size_t)rows * stride * 4));
+    if (mode != PIVOT_MODE_DENSE) {
+        w.pq = c.take((size_t)b->B * b->H * b->D * esize_of(b->dtype));
+        w.pqs = static_cast<float*>(c.take((size_t)b->B * 4));
+        w.pw = static_cast<float*>(c.take((size_t)b->B * b->H * 4));
+        w.cand = static_cast<int32_t*>(c.take((size_t)b->B * C * 4));
+        if (mode == PIVOT_MODE_REFINE)
+            w.R = static_cast<float*>(c.take((size_t)b->B * b->Gm * C * 4));
+    }
+    if (out) *out = w;
+    return c.ok ? align_up(c.off, WS_ALIGN) : 0;
+}
+
+size_t pivot_decode_workspace_size(const pivot_decode_t* b, int32_t mode, int32_t C, int32_t topk) {
+    if (check_decode(b) != PIVOT_OK || mode < 0 || mode > 2 || topk < 1) return 0;
+    if (mode != PIVOT_MODE_DENSE && C < topk) return 0;
+    return decode_layout(b, mode, C, nullptr, nullptr, 0);
+}
+
+pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, int32_t topk,
+                            int32_t* idx, int32_t* cand, void* ws, size_t ws_bytes, void* stream) {
+    pivot_status_t st = check_decode(b);
+    if (st != PIVOT_OK) return st;
+    if (mode < 0 || mode > 2 || topk < 1 || !idx) return PIVOT_ERR_INVALID_ARG;
+    if (mode != PIVOT_MODE_DENSE && C < topk) return PIVOT_ERR_INVALID_ARG;
+    if (topk > MAX_K || C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
+    DecodeWs w;
+    if (decode_layout(b, mode, C, &w, ws, ws_bytes) == 0) return PIVOT_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long stride = score_stride(b->maxlen);
+    const long long krows = (long long)b->B * b->maxlen;
+    if (mode == PIVOT_MODE_DENSE) {
+        const int rows = b->B * b->Gm;
+        const int P = b->Gm;   // one sequence's members share a row block
+        st = run_scan(SCAN_DECODE_DENSE, b->dtype, b->H, b->D, b->q, rows, 0, b->w, b->q_scale,
+                      b->kc, krows, b->kc_scale, 0, 1, b->Gm, b->maxlen, b->cache_len, P, 0, rows,
+                      b->maxlen - 1, w.S, stride, s);
+        if (st != PIVOT_OK) return st;
+        return run_select_prefix(SCAN_DECODE_DENSE, 0, rows, 0, 1, b->Gm, b->maxlen, b->cache_len,
+                                 w.S, stride, topk, idx, nullptr, 0, s);
+    }
+    // proxy of each sequence's Gm new tokens
+    ReduceParams rp{};
+    rp.dtype = b->dtype;
+    rp.esize = esize_of(b->dtype);
+    rp.H = b->H;
+    rp.D = b->D;
+    rp.nmembers_total = b->B * b->Gm;
+    rp.g = b->Gm;
+    rp.ngroups = b->B;
+    rp.q = b->q;
+    rp.q_scale = b->q_scale;
+    rp.w = b->w;
+    rp.pq = w.pq;
+    rp.pq_scale = b->dtype == PIVOT_E4M3 ? w.pqs : nullptr;
+    rp.pw = w.pw;
+    rp.group_stride_members = b->Gm;
+    if ((st = from_cuda(launch_proxy_reduce(rp, s))) != PIVOT_OK) return st;
+    st = run_scan(SCAN_DECODE_PROXY, b->dtype, b->H, b->D, w.pq, b->B, 0, w.pw,
+                  b->dtype == PIVOT_E4M3 ? w.pqs : nullptr, b->kc, krows, b->kc_scale, 0, 1, b->Gm,
+                  b->maxlen, b->cache_len, 1, 0, b->B, b->maxlen - 1, w.S, stride, s);
+    if (st != PIVOT_OK) return st;
+    st = run_select_prefix(SCAN_DECODE_PROXY, 0, b->B, 0, 1, b->Gm, b->maxlen, b->cache_len, w.S,
+                           stride, C, w.cand, nullptr, 0, s);
+    if (st != PIVOT_OK) return st;
+    if (cand)
+        if (cudaMemcpyAsync(cand, w.cand, (size_t)b->B * C * 4, cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
+            return PIVOT_ERR_CUDA;
+    if (mode == PIVOT_MODE_REUSE)
+        return from_cuda(launch_decode_reuse(b->B, b->Gm, b->maxlen, b->cache_len, w.cand, C, topk,
+                                             idx, s));
+    const int rows = b->B * b->Gm;
+    st = run_refine_scores(SCAN_DECODE_DENSE, b->dtype, b->H, b->D, b->q, 0, b->q_scale, b->w,
+                           b->kc, b->kc_scale, 0, 1, b->Gm, b->maxlen, b->cache_len, w.cand, 0, C,
+                           0, rows, w.R, s);
+    if (st != PIVOT_OK) return st;
+    return run_select_cand(SCAN_DECODE_DENSE, 0, rows, 0, 1, b->Gm, b->maxlen, b->cache_len, w.R,
+                           w.cand, 0, C, topk, idx, nullptr, 0, s);
+}
+
+}  // extern "C"

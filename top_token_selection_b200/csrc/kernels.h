@@ -1,0 +1,114 @@
+// kernels.h -- internal launch interfaces of libpivot (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pivot {
+
+// Which rows a scan launch scores and how their causal limit is found.
+enum ScanKind {
+    SCAN_PREFILL_DENSE = 0,   // row r = query t, keys [0, t]
+    SCAN_PREFILL_PROXY = 1,   // row r = group j, keys [0, min(L,(j+1)g) - 1]
+    SCAN_DECODE_DENSE = 2,    // row r = b*Gm + m, keys [0, cache_len[b] - Gm + m] of seq b
+    SCAN_DECODE_PROXY = 3,    // row r = b, keys [0, cache_len[b] - 1] of seq b
+};
+
+struct ScanParams {
+    int kind;            // ScanKind
+    int dtype;           // pivot_dtype_t
+    int esize;           // bytes per q/k element
+    int H, D;
+    int P;               // rows per row block; N = P*H <= 256
+    int row0, nrows;     // global rows of this launch
+    int qrow_base;       // per-row arrays (q, w, q_scale) are indexed by r - qrow_base
+    int L, g;            // prefill
+    int Gm, maxlen;      // decode
+    const int32_t* cache_len;
+    const float* w;
+    const float* q_scale;
+    const float* k_scale;   // indexed by key row (decode: b*maxlen + s)
+    float* S;               // scores of row r at S + (r - row0)*S_stride + s
+    long long S_stride;
+    int tiles_per_item, items_per_block, nitems;
+};
+
+int scan_smem_bytes(int row_bytes);
+cudaError_t launch_scan_umma(const CUtensorMap& tk, const CUtensorMap& tq, const ScanParams& p,
+                             int grid, cudaStream_t stream);
+cudaError_t launch_scan_simt(const void* q, const void* k, const ScanParams& p,
+                             cudaStream_t stream);
+
+// Row selection: for each row, the top-K entries by (score desc, position
+// asc) among the row's valid entries, written in rank order with -1 / -inf
+// padding.
+enum SelectKind {
+    SEL_PREFIX = 0,      // row r: entries 0..lim(r) of S, position = entry index
+    SEL_CANDIDATES = 1,  // row r: C entries, position = cand[grp(r)][i], valid iff 0 <= pos <= lim(r)
+};
+
+struct SelectParams {
+    int kind;             // SelectKind
+    int scan_kind;        // ScanKind giving lim(r) (SEL_PREFIX and SEL_CANDIDATES)
+    int row0, nrows;
+    int L, g, Gm, maxlen;
+    const int32_t* cache_len;
+    const float* S;       // row r at S + (r - row0)*S_stride
+    long long S_stride;
+    const int32_t* cand;  // SEL_CANDIDATES: group rows at cand + (grp - cand_base)*C
+    int cand_base, C;
+    int K;
+    int32_t* out_idx;     // row r at out_idx + (r - out_base)*K
+    float* out_score;     // or NULL
+    int out_base;
+    int tail_cap;         // capacity of the boundary buffer (entries)
+};
+
+cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
+size_t select_smem_bytes(int K, int tail_cap);
+
+struct ReduceParams {
+    int dtype, esize, H, D;
+    int nmembers_total;    // rows available from member 0 of the first group
+    int g;                 // members per group
+    int ngroups;
+    const void* q;         // member rows, q + m*H*D*esize for member m (relative)
+    const float* q_scale;
+    const float* w;
+    void* pq;
+    float* pq_scale;
+    float* pw;
+    long long group_stride_members;  // members between consecutive groups
+};
+cudaError_t launch_proxy_reduce(const ReduceParams& p, cudaStream_t stream);
+
+cudaError_t launch_reuse(int t_begin, int t_end, int g, const int32_t* cand, int C, int topk,
+                         int32_t* idx, cudaStream_t stream);
+cudaError_t launch_decode_reuse(int B, int Gm, int maxlen, const int32_t* cache_len,
+                                const int32_t* cand, int C, int topk, int32_t* idx,
+                                cudaStream_t stream);
+
+// Refine scores: member r of group grp(r) against C candidate keys.
+struct RefineParams {
+    int dtype, esize, H, D;
+    int kind;              // ScanKind for the member rows (PREFILL_DENSE or DECODE_DENSE)
+    int row0, nrows;       // member rows
+    int qrow_base;
+    int L, g, Gm, maxlen;
+    const int32_t* cache_len;
+    const void* q;
+    const float* q_scale;
+    const float* w;
+    const void* k;
+    const float* k_scale;
+    const int32_t* cand;   // group rows at cand + (grp - cand_base)*C
+    int cand_base, C;
+    float* S;              // row r at S + (r - row0)*C
+};
+cudaError_t launch_refine_simt(const RefineParams& p, cudaStream_t stream);
+
+cudaError_t launch_wait_selftest(cudaStream_t stream);
+
+}  // namespace pivot

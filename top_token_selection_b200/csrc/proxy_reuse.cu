@@ -1,0 +1,173 @@
+// proxy_reuse.cu -- the proxy query of a group and PIVOT-Reuse.
+//
+// Proxy (abstract of arXiv 2607.24593: a group is aggregated into one proxy
+// query; "PIVOT 설명 ... 10분 만에 구현하기", section "How It Works": the
+// proxy is the mean of the group).  Per element, in fp32 and in member
+// order, without fused multiply-add:
+//     x_m = q value * q scale;   pq = (x_0 + x_1 + ... + x_{n-1}) / n
+// and the same for the head weights; then stored in the input format (bf16
+// round-to-nearest-even; e4m3 with one scale amax/448, saturating RNE).  A
+// one-member group is copied unchanged.
+//
+// Reuse (same abstract): every member takes the proxy's top-k, i.e. the
+// first k candidates in rank order, minus the positions after itself.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pivot {
+
+namespace {
+
+constexpr int RED_THREADS = 256;
+
+template <int DT>
+__device__ __forceinline__ float member_value(const void* q, const float* q_scale, size_t row,
+                                              size_t HD, size_t i) {
+    if constexpr (DT == PIVOT_F32) {
+        return static_cast<const float*>(q)[row * HD + i];
+    } else if constexpr (DT == PIVOT_BF16) {
+        return bf16_to_f32(static_cast<const uint16_t*>(q)[row * HD + i]);
+    } else {
+        return __fmul_rn(e4m3_to_f32(static_cast<const uint8_t*>(q)[row * HD + i]), q_scale[row]);
+    }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(RED_THREADS) proxy_reduce_kernel(const ReduceParams p) {
+    extern __shared__ float qbar_s[];          // H*D (e4m3 only)
+    __shared__ float red_s[RED_THREADS / 32];
+    const int j = blockIdx.x;
+    const size_t HD = (size_t)p.H * p.D;
+    const long long m0 = (long long)j * p.group_stride_members;
+    const int n = (int)min((long long)p.g, (long long)p.nmembers_total - m0);
+    if (n <= 0) return;
+
+    if (n == 1) {   // a group of one is its member
+        const size_t esz = DT == PIVOT_F32 ? 4 : (DT == PIVOT_BF16 ? 2 : 1);
+        const uint8_t* src = static_cast<const uint8_t*>(p.q) + (size_t)m0 * HD * esz;
+        uint8_t* dst = static_cast<uint8_t*>(p.pq) + (size_t)j * HD * esz;
+        for (size_t i = threadIdx.x; i < HD * esz; i += RED_THREADS) dst[i] = src[i];
+        for (int h = threadIdx.x; h < p.H; h += RED_THREADS)
+            p.pw[(size_t)j * p.H + h] = p.w[(size_t)m0 * p.H + h];
+        if (DT == PIVOT_E4M3 && threadIdx.x == 0) p.pq_scale[j] = p.q_scale[m0];
+        return;
+    }
+
+    const float fn = (float)n;
+    float amax = 0.0f;
+    for (size_t i = threadIdx.x; i < HD; i += RED_THREADS) {
+        float acc = member_value<DT>(p.q, p.q_scale, (size_t)m0, HD, i);
+        for (int m = 1; m < n; ++m)
+            acc = __fadd_rn(acc, member_value<DT>(p.q, p.q_scale, (size_t)(m0 + m), HD, i));
+        const float qb = __fdiv_rn(acc, fn);
+        if constexpr (DT == PIVOT_F32) {
+            static_cast<float*>(p.pq)[(size_t)j * HD + i] = qb;
+        } else if constexpr (DT == PIVOT_BF16) {
+            const __nv_bfloat16 b = __float2bfloat16_rn(qb);
+            static_cast<__nv_bfloat16*>(p.pq)[(size_t)j * HD + i] = b;
+        } else {
+            qbar_s[i] = qb;
+            amax = fmaxf(amax, fabsf(qb));
+        }
+    }
+    for (int h = threadIdx.x; h < p.H; h += RED_THREADS) {
+        float acc = p.w[(size_t)m0 * p.H + h];
+        for (int m = 1; m < n; ++m) acc = __fadd_rn(acc, p.w[(size_t)(m0 + m) * p.H + h]);
+        p.pw[(size_t)j * p.H + h] = __fdiv_rn(acc, fn);
+    }
+    if constexpr (DT == PIVOT_E4M3) {
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if ((threadIdx.x & 31) == 0) red_s[threadIdx.x >> 5] = amax;
+        __syncthreads();
+        float a = 0.0f;
+        for (int w = 0; w < RED_THREADS / 32; ++w) a = fmaxf(a, red_s[w]);
+        const float s = a > 0.0f ? __fdiv_rn(a, 448.0f) : 1.0f;
+        uint8_t* dst = static_cast<uint8_t*>(p.pq) + (size_t)j * HD;
+        for (size_t i = threadIdx.x; i < HD; i += RED_THREADS)
+            dst[i] = f32_to_e4m3_satfinite(__fdiv_rn(qbar_s[i], s));
+        if (threadIdx.x == 0) p.pq_scale[j] = s;
+    }
+}
+
+// One warp per member row: compact the first topk candidates to those <= lim.
+__device__ __forceinline__ void reuse_row(const int32_t* c, int topk, int lim, int32_t* o) {
+    const int lane = threadIdx.x & 31;
+    int n = 0;
+    for (int i0 = 0; i0 < topk; i0 += 32) {
+        const int i = i0 + lane;
+        const int32_t s = i < topk ? c[i] : -1;
+        const bool ok = s >= 0 && s <= lim;
+        const unsigned bal = __ballot_sync(0xffffffffu, ok);
+        if (ok) o[n + __popc(bal & ((1u << lane) - 1u))] = s;
+        n += __popc(bal);
+    }
+    for (int i = n + lane; i < topk; i += 32) o[i] = -1;
+}
+
+__global__ void reuse_kernel(int t_begin, int t_end, int g, const int32_t* cand, int C, int topk,
+                             int32_t* idx) {
+    const int t = t_begin + blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (t >= t_end) return;
+    const int j = t / g - t_begin / g;
+    reuse_row(cand + (size_t)j * C, topk, t, idx + (size_t)(t - t_begin) * topk);
+}
+
+__global__ void decode_reuse_kernel(int B, int Gm, int maxlen, const int32_t* cache_len,
+                                    const int32_t* cand, int C, int topk, int32_t* idx) {
+    const int r = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (r >= B * Gm) return;
+    const int b = r / Gm, m = r % Gm;
+    const int n = cache_len[b];
+    int lim = n - Gm + m;
+    if (n < Gm || n > maxlen) {
+        if ((threadIdx.x & 31) == 0) raise_error(ERRBIT_DATA);
+        lim = -1;
+    }
+    reuse_row(cand + (size_t)b * C, topk, lim, idx + (size_t)r * topk);
+}
+
+}  // namespace
+
+cudaError_t launch_proxy_reduce(const ReduceParams& p, cudaStream_t stream) {
+    if (p.ngroups <= 0) return cudaSuccess;
+    const size_t smem = p.dtype == PIVOT_E4M3 ? (size_t)p.H * p.D * 4 : 0;
+    switch (p.dtype) {
+        case PIVOT_F32:
+            proxy_reduce_kernel<PIVOT_F32><<<p.ngroups, RED_THREADS, 0, stream>>>(p);
+            break;
+        case PIVOT_BF16:
+            proxy_reduce_kernel<PIVOT_BF16><<<p.ngroups, RED_THREADS, 0, stream>>>(p);
+            break;
+        default: {
+            cudaError_t e = cudaFuncSetAttribute(proxy_reduce_kernel<PIVOT_E4M3>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+            if (e != cudaSuccess) return e;
+            proxy_reduce_kernel<PIVOT_E4M3><<<p.ngroups, RED_THREADS, smem, stream>>>(p);
+        }
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reuse(int t_begin, int t_end, int g, const int32_t* cand, int C, int topk,
+                         int32_t* idx, cudaStream_t stream) {
+    const int rows = t_end - t_begin;
+    if (rows <= 0) return cudaSuccess;
+    const int wpb = 8;
+    reuse_kernel<<<ceil_div(rows, wpb), wpb * 32, 0, stream>>>(t_begin, t_end, g, cand, C, topk,
+                                                                idx);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_reuse(int B, int Gm, int maxlen, const int32_t* cache_len,
+                                const int32_t* cand, int C, int topk, int32_t* idx,
+                                cudaStream_t stream) {
+    const int rows = B * Gm;
+    if (rows <= 0) return cudaSuccess;
+    const int wpb = 8;
+    decode_reuse_kernel<<<ceil_div(rows, wpb), wpb * 32, 0, stream>>>(B, Gm, maxlen, cache_len,
+                                                                       cand, C, topk, idx);
+    return cudaGetLastError();
+}
+
+}  // namespace pivot

@@ -1,0 +1,280 @@
+"""Python binding of libpivot (ctypes).
+
+The functions named ``pivot_*`` mirror the C ABI of ``include/pivot.h`` one
+to one (argument marshalling only).  The lower-case helpers below them
+(``dense_index``, ``proxy_reduce``, ...) allocate outputs and workspaces
+with torch on the caller's device and stream and then call the same entry
+points; every step of the indexer runs in the library's CUDA kernels.
+
+There is no fallback: if ``libpivot.so`` is missing or cannot be loaded,
+``load()`` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpivot.so")
+
+F32, BF16, E4M3 = 0, 1, 2
+DENSE, REUSE, REFINE = 0, 1, 2
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "workspace too small",
+          4: "CUDA error", 5: "a kernel wait timed out", 6: "bad device-side data"}
+
+ABI_SYMBOLS = [
+    "pivot_dense_index", "pivot_dense_index_workspace_size", "pivot_proxy_reduce",
+    "pivot_proxy_scan", "pivot_proxy_scan_workspace_size", "pivot_reuse", "pivot_refine",
+    "pivot_refine_workspace_size", "pivot_decode", "pivot_decode_workspace_size",
+    "pivot_get_device_error", "pivot_set_wait_limit_ns", "pivot_selftest_wait_timeout",
+    "pivot_status_string", "pivot_version",
+]
+
+
+class PivotError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} (status {status})")
+
+
+class PivotSeq(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int32), ("L", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("q", ctypes.c_void_p), ("q_scale", ctypes.c_void_p),
+                ("w", ctypes.c_void_p), ("k", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
+                ("t_begin", ctypes.c_int32), ("t_end", ctypes.c_int32)]
+
+
+class PivotDecode(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int32), ("B", ctypes.c_int32), ("Gm", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("D", ctypes.c_int32), ("maxlen", ctypes.c_int32),
+                ("q", ctypes.c_void_p), ("q_scale", ctypes.c_void_p), ("w", ctypes.c_void_p),
+                ("kc", ctypes.c_void_p), ("kc_scale", ctypes.c_void_p),
+                ("cache_len", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libpivot.so (raises if it is missing: there is no other path)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libpivot.so not built at {path}; run "
+                          "`python -m top_token_selection_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    sig = {
+        "pivot_dense_index": ([P, I32, P, P, P, SZ, P], I32),
+        "pivot_dense_index_workspace_size": ([P, I32], SZ),
+        "pivot_proxy_reduce": ([P, I32, P, P, P, P], I32),
+        "pivot_proxy_scan": ([P, I32, P, P, P, I32, P, P, P, SZ, P], I32),
+        "pivot_proxy_scan_workspace_size": ([P, I32, I32], SZ),
+        "pivot_reuse": ([I32, I32, I32, P, I32, I32, P, P], I32),
+        "pivot_refine": ([P, I32, P, I32, I32, P, P, P, SZ, P], I32),
+        "pivot_refine_workspace_size": ([P, I32, I32, I32], SZ),
+        "pivot_decode": ([P, I32, I32, I32, P, P, P, SZ, P], I32),
+        "pivot_decode_workspace_size": ([P, I32, I32, I32], SZ),
+        "pivot_get_device_error": ([P], I32),
+        "pivot_set_wait_limit_ns": ([ctypes.c_uint64], I32),
+        "pivot_selftest_wait_timeout": ([P], I32),
+        "pivot_status_string": ([I32], ctypes.c_char_p),
+        "pivot_version": ([], I32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+# ---------------------------------------------------------------------------
+# C ABI mirrors (same names, same arguments)
+# ---------------------------------------------------------------------------
+
+def pivot_dense_index(seq, topk, idx, score, ws, ws_bytes, stream):
+    return load().pivot_dense_index(ctypes.byref(seq), topk, idx, score, ws, ws_bytes, stream)
+
+
+def pivot_dense_index_workspace_size(seq, topk):
+    return load().pivot_dense_index_workspace_size(ctypes.byref(seq), topk)
+
+
+def pivot_proxy_reduce(seq, g, pq, pq_scale, pw, stream):
+    return load().pivot_proxy_reduce(ctypes.byref(seq), g, pq, pq_scale, pw, stream)
+
+
+def pivot_proxy_scan(seq, g, pq, pq_scale, pw, C, cand, cand_score, ws, ws_bytes, stream):
+    return load().pivot_proxy_scan(ctypes.byref(seq), g, pq, pq_scale, pw, C, cand, cand_score,
+                                   ws, ws_bytes, stream)
+
+
+def pivot_proxy_scan_workspace_size(seq, g, C):
+    return load().pivot_proxy_scan_workspace_size(ctypes.byref(seq), g, C)
+
+
+def pivot_reuse(t_begin, t_end, g, cand, C, topk, idx, stream):
+    return load().pivot_reuse(t_begin, t_end, g, cand, C, topk, idx, stream)
+
+
+def pivot_refine(seq, g, cand, C, topk, idx, score, ws, ws_bytes, stream):
+    return load().pivot_refine(ctypes.byref(seq), g, cand, C, topk, idx, score, ws, ws_bytes,
+                               stream)
+
+
+def pivot_refine_workspace_size(seq, g, C, topk):
+    return load().pivot_refine_workspace_size(ctypes.byref(seq), g, C, topk)
+
+
+def pivot_decode(batch, mode, C, topk, idx, cand, ws, ws_bytes, stream):
+    return load().pivot_decode(ctypes.byref(batch), mode, C, topk, idx, cand, ws, ws_bytes,
+                               stream)
+
+
+def pivot_decode_workspace_size(batch, mode, C, topk):
+    return load().pivot_decode_workspace_size(ctypes.byref(batch), mode, C, topk)
+
+
+def pivot_get_device_error(stream):
+    return load().pivot_get_device_error(stream)
+
+
+def pivot_set_wait_limit_ns(ns):
+    return load().pivot_set_wait_limit_ns(ns)
+
+
+def pivot_selftest_wait_timeout(stream):
+    return load().pivot_selftest_wait_timeout(stream)
+
+
+def pivot_status_string(status):
+    return load().pivot_status_string(status).decode()
+
+
+def pivot_version():
+    return load().pivot_version()
+
+
+# ---------------------------------------------------------------------------
+# torch marshalling helpers
+# ---------------------------------------------------------------------------
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype in (torch.float8_e4m3fn, torch.uint8):
+        return E4M3
+    raise TypeError(f"unsupported indexer dtype {t.dtype}")
+
+
+def _p(t):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "libpivot takes contiguous CUDA tensors"
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status, what):
+    if status != 0:
+        raise PivotError(status, what)
+
+
+def _workspace(nbytes, device):
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def make_seq(q, q_scale, w, k, k_scale, t_begin=0, t_end=0) -> PivotSeq:
+    L, H, D = q.shape
+    return PivotSeq(_dtype_code(q), L, H, D, _p(q), _p(q_scale), _p(w), _p(k), _p(k_scale),
+                    t_begin, t_end)
+
+
+def make_decode(q, q_scale, w, kc, kc_scale, cache_len) -> PivotDecode:
+    B, Gm, H, D = q.shape
+    return PivotDecode(_dtype_code(q), B, Gm, H, D, kc.shape[1], _p(q), _p(q_scale), _p(w),
+                       _p(kc), _p(kc_scale), _p(cache_len))
+
+
+def _rows(seq):
+    return (seq.t_end or seq.L) - seq.t_begin
+
+
+def dense_index(seq: PivotSeq, topk, with_score=False, ws=None, stream=None, device="cuda"):
+    n = _rows(seq)
+    idx = torch.empty(n, topk, dtype=torch.int32, device=device)
+    score = torch.empty(n, topk, dtype=torch.float32, device=device) if with_score else None
+    if ws is None:
+        ws = _workspace(pivot_dense_index_workspace_size(seq, topk), device)
+    _check(pivot_dense_index(seq, topk, _p(idx), _p(score), _p(ws), ws.numel(), _stream(stream)),
+           "pivot_dense_index")
+    return idx, score
+
+
+def proxy_reduce(seq: PivotSeq, g, stream=None, device="cuda"):
+    G = -(-_rows(seq) // g)
+    store = {F32: torch.float32, BF16: torch.bfloat16, E4M3: torch.float8_e4m3fn}[seq.dtype]
+    pq = torch.empty(G, seq.H, seq.D, dtype=store, device=device)
+    pqs = torch.empty(G, dtype=torch.float32, device=device) if seq.dtype == E4M3 else None
+    pw = torch.empty(G, seq.H, dtype=torch.float32, device=device)
+    _check(pivot_proxy_reduce(seq, g, _p(pq), _p(pqs), _p(pw), _stream(stream)),
+           "pivot_proxy_reduce")
+    return pq, pqs, pw
+
+
+def proxy_scan(seq: PivotSeq, g, pq, pqs, pw, C, with_score=False, ws=None, stream=None,
+               device="cuda"):
+    G = pq.shape[0]
+    cand = torch.empty(G, C, dtype=torch.int32, device=device)
+    cs = torch.empty(G, C, dtype=torch.float32, device=device) if with_score else None
+    if ws is None:
+        ws = _workspace(pivot_proxy_scan_workspace_size(seq, g, C), device)
+    _check(pivot_proxy_scan(seq, g, _p(pq), _p(pqs), _p(pw), C, _p(cand), _p(cs), _p(ws),
+                            ws.numel(), _stream(stream)), "pivot_proxy_scan")
+    return cand, cs
+
+
+def reuse(t_begin, t_end, g, cand, topk, stream=None, device="cuda"):
+    idx = torch.empty(t_end - t_begin, topk, dtype=torch.int32, device=device)
+    _check(pivot_reuse(t_begin, t_end, g, _p(cand), cand.shape[1], topk, _p(idx),
+                       _stream(stream)), "pivot_reuse")
+    return idx
+
+
+def refine(seq: PivotSeq, g, cand, topk, with_score=False, ws=None, stream=None, device="cuda"):
+    n = _rows(seq)
+    C = cand.shape[1]
+    idx = torch.empty(n, topk, dtype=torch.int32, device=device)
+    score = torch.empty(n, topk, dtype=torch.float32, device=device) if with_score else None
+    if ws is None:
+        ws = _workspace(pivot_refine_workspace_size(seq, g, C, topk), device)
+    _check(pivot_refine(seq, g, _p(cand), C, topk, _p(idx), _p(score), _p(ws), ws.numel(),
+                        _stream(stream)), "pivot_refine")
+    return idx, score
+
+
+def decode(batch: PivotDecode, mode, C, topk, want_cand=False, ws=None, stream=None,
+           device="cuda"):
+    idx = torch.empty(batch.B, batch.Gm, topk, dtype=torch.int32, device=device)
+    cand = (torch.empty(batch.B, C, dtype=torch.int32, device=device)
+            if (want_cand and mode != DENSE) else None)
+    if ws is None:
+        ws = _workspace(pivot_decode_workspace_size(batch, mode, C, topk), device)
+    _check(pivot_decode(batch, mode, C, topk, _p(idx), _p(cand), _p(ws), ws.numel(),
+                        _stream(stream)), "pivot_decode")
+    return idx, cand
+
+
+def device_error(stream=None) -> int:
+    return pivot_get_device_error(_stream(stream))
