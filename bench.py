@@ -1,0 +1,562 @@
+"""Benchmark of the PIVOT indexer on B200 (libpivot, through its C ABI).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--seed S]
+
+One step is one pass of the whole hot path over one synthetic sequence:
+the dense indexer (every query scans its full causal prefix, keeps top-k),
+then PIVOT -- proxy reduce, one proxy scan per group (top-C candidates),
+PIVOT-Reuse and PIVOT-Refine -- so each step produces the dense, Reuse and
+Refine index sets of all L queries.  ``value`` = L * n_gpus / step time
+(queries/s, whole job).  Per-mode times, Reuse/Refine recall against dense
+and the neighbour overlap of dense are reported beside it.
+
+Timing: W untimed warm-up steps, then K steps between CUDA events on the
+launching stream, bracketed by a barrier and a device synchronize; the max
+over ranks is reported.  The inputs (q alone is 1 GiB at L=128K) and the
+score buffers are far larger than L2, so no flush is needed.
+
+``--impl reference`` times the CPU oracle (``oracle/``, plain C, fp64) on a
+bounded sample of the same workload and extrapolates to the full step; it
+is the reference arm (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from top_token_selection_b200 import inputs as gen  # noqa: E402
+
+METRIC = "indexer queries/s at L=128K (dense vs PIVOT-Reuse/Refine), % roofline; recall"
+DEFAULT_WORKLOAD = "long_prefill_128k_fp8"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (host logic, testable on CPU with gloo)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Weak scaling: every rank indexes its own independent sequence."""
+    return base_seed + 1000003 * rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(queries_per_rank: int, world: int, ms_max: float, steps: int) -> float:
+    """Whole-job queries/s: all ranks' queries over the slowest rank's time."""
+    return queries_per_rank * world * steps / (ms_max / 1e3)
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [v for v in vis.split(",") if v.strip()]
+        self.dev = ids[local_rank] if local_rank < len(ids) else str(local_rank)
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.dev, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def make_inputs(wl, seed):
+    return gen.make_prefill(wl["L"], wl["H"], wl["D"], wl["dtype"], kind=wl["kind"], seed=seed)
+
+
+class Runner:
+    """Device buffers and one step of the hot path through the C ABI."""
+
+    def __init__(self, p, wl, device):
+        from top_token_selection_b200 import pivot as pv
+        self.pv = pv
+        pv.load()
+        self.wl = wl
+        self.L, self.H, self.D = p.L, p.H, p.D
+        self.g, self.C, self.k = wl["g"], wl["C"], wl["topk"]
+        self.G = -(-self.L // self.g)
+        d = device
+        self.host = {"q": p.q, "q_scale": p.q_scale, "w": p.w, "k": p.k, "k_scale": p.k_scale}
+        self.dev = {n: (None if t is None else torch.empty_like(t, device=d))
+                    for n, t in self.host.items()}
+        for n, t in self.host.items():
+            if t is not None:
+                self.dev[n].copy_(t)
+        self.seq = pv.make_seq(self.dev["q"], self.dev["q_scale"], self.dev["w"], self.dev["k"],
+                               self.dev["k_scale"])
+        store = {gen.F32: torch.float32, gen.BF16: torch.bfloat16,
+                 gen.E4M3: torch.float8_e4m3fn}[wl["dtype"]]
+        self.dense = torch.empty(self.L, self.k, dtype=torch.int32, device=d)
+        self.reu = torch.empty(self.L, self.k, dtype=torch.int32, device=d)
+        self.ref = torch.empty(self.L, self.k, dtype=torch.int32, device=d)
+        self.cand = torch.empty(self.G, self.C, dtype=torch.int32, device=d)
+        self.pq = torch.empty(self.G, self.H, self.D, dtype=store, device=d)
+        self.pqs = (torch.empty(self.G, dtype=torch.float32, device=d)
+                    if wl["dtype"] == gen.E4M3 else None)
+        self.pw = torch.empty(self.G, self.H, dtype=torch.float32, device=d)
+        wsb = max(pv.pivot_dense_index_workspace_size(self.seq, self.k),
+                  pv.pivot_proxy_scan_workspace_size(self.seq, self.g, self.C),
+                  pv.pivot_refine_workspace_size(self.seq, self.g, self.C, self.k))
+        self.ws = torch.empty(wsb, dtype=torch.uint8, device=d)
+        self.stream = torch.cuda.current_stream()
+
+    def _ptr(self, t):
+        return None if t is None else t.data_ptr()
+
+    def step(self, events=None):
+        pv, s = self.pv, self.stream
+        sp = pv._stream(s)
+        ws, wsn = self.ws.data_ptr(), self.ws.numel()
+
+        def mark(i):
+            if events is not None:
+                events[i].record(s)
+        mark(0)
+        pv._check(pv.pivot_dense_index(self.seq, self.k, self.dense.data_ptr(), None, ws, wsn, sp),
+                  "dense")
+        mark(1)
+        pv._check(pv.pivot_proxy_reduce(self.seq, self.g, self.pq.data_ptr(), self._ptr(self.pqs),
+                                        self.pw.data_ptr(), sp), "reduce")
+        mark(2)
+        pv._check(pv.pivot_proxy_scan(self.seq, self.g, self.pq.data_ptr(), self._ptr(self.pqs),
+                                      self.pw.data_ptr(), self.C, self.cand.data_ptr(), None, ws,
+                                      wsn, sp), "scan")
+        mark(3)
+        pv._check(pv.pivot_reuse(0, self.L, self.g, self.cand.data_ptr(), self.C, self.k,
+                                 self.reu.data_ptr(), sp), "reuse")
+        mark(4)
+        pv._check(pv.pivot_refine(self.seq, self.g, self.cand.data_ptr(), self.C, self.k,
+                                  self.ref.data_ptr(), None, ws, wsn, sp), "refine")
+        mark(5)
+
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.host.values() if t is not None)
+
+    def d2h_bytes(self):
+        return 3 * self.L * self.k * 4
+
+
+def recall_stats(dense, other, rows_per_chunk=4096):
+    """Mean over rows of |other ∩ dense| / |dense| (both -1 padded)."""
+    tot, n = 0.0, 0
+    for r0 in range(0, dense.shape[0], rows_per_chunk):
+        a = dense[r0:r0 + rows_per_chunk].long()
+        b = other[r0:r0 + rows_per_chunk].long()
+        big = torch.iinfo(torch.int64).max
+        a_s, _ = torch.sort(torch.where(a >= 0, a, big), dim=1)
+        pos = torch.searchsorted(a_s, b.contiguous())
+        hit = (pos < a.shape[1]) & (torch.gather(a_s, 1, pos.clamp(max=a.shape[1] - 1)) == b)
+        hit &= b >= 0
+        cnt = (a >= 0).sum(1).clamp(min=1)
+        tot += (hit.sum(1).double() / cnt.double()).sum().item()
+        n += a.shape[0]
+    return tot / max(n, 1)
+
+
+def neighbour_overlap(dense, rows_per_chunk=4096):
+    k = dense.shape[1]
+    tot, n = 0.0, 0
+    for r0 in range(0, dense.shape[0] - 1, rows_per_chunk):
+        r1 = min(dense.shape[0] - 1, r0 + rows_per_chunk)
+        a = dense[r0:r1]
+        b = dense[r0 + 1:r1 + 1]
+        full = (a >= 0).all(1) & (b >= 0).all(1)
+        if full.any():
+            tot += recall_stats(a[full], b[full]) * int(full.sum())
+            n += int(full.sum())
+    return tot / max(n, 1) if k else 0.0
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_time(p, wl, budget_rows=None, seed=0):
+    """Time the oracle on a stratified sample of the step and extrapolate.
+
+    Dense rows, proxy-scan groups and Refine rows are sampled evenly over
+    positions; each part's time is scaled by (work of all rows) / (work of
+    the sampled rows), work being the causal pairs the oracle scores.  The
+    proxy reduce and Reuse run on sampled groups/rows and scale by count.
+    Returns (seconds for one full step, description, threads)."""
+    import oracle
+    L, H, D, g, C, k = p.L, p.H, p.D, wl["g"], wl["C"], wl["topk"]
+    G = -(-L // g)
+    q, qs, w, kk, ks = p.codes()
+    nd, ns, nr = budget_rows or (48, 24, 192)
+    rng = np.random.default_rng(seed)
+    dense_rows = np.unique(np.linspace(0, L - 1, nd).astype(np.int64) +
+                           rng.integers(0, max(1, L // nd), nd)).clip(0, L - 1).astype(np.int32)
+    groups = np.unique(np.linspace(0, G - 1, ns).astype(np.int64)).astype(np.int32)
+    ref_rows = np.unique(np.linspace(0, L - 1, nr).astype(np.int64)).astype(np.int32)
+    threads = oracle.max_threads()
+
+    t0 = time.perf_counter()
+    oracle.dense_index(p.dtype, q, qs, w, kk, ks, k, rows=dense_rows)
+    t_dense = time.perf_counter() - t0
+    all_pairs = L * (L + 1) / 2
+    dense_full = t_dense * all_pairs / float(np.sum(dense_rows.astype(np.float64) + 1))
+
+    t0 = time.perf_counter()
+    pq, pqs, pw = oracle.proxy_reduce(p.dtype, q, qs, w, g, groups=groups)
+    t_red = time.perf_counter() - t0
+    red_full = t_red * G / len(groups)
+
+    # proxy scan on the sampled groups: the oracle scan indexes pq by group id,
+    # so place the sampled proxies in a full-size table
+    store = pq.dtype
+    pq_full = np.zeros((G, H, D), dtype=store)
+    pw_full = np.zeros((G, H), dtype=np.float32)
+    pqs_full = np.ones(G, dtype=np.float32) if pqs is not None else None
+    pq_full[groups], pw_full[groups] = pq, pw
+    if pqs is not None:
+        pqs_full[groups] = pqs
+    t0 = time.perf_counter()
+    cand, _ = oracle.proxy_scan(p.dtype, pq_full, pqs_full, pw_full, kk, ks, L, g, C,
+                                groups=groups)
+    t_scan = time.perf_counter() - t0
+    e = np.minimum(L, (groups.astype(np.float64) + 1) * g)
+    scan_all = sum(min(L, (j + 1) * g) for j in range(G))
+    scan_full = t_scan * scan_all / float(np.sum(e))
+
+    # Refine and Reuse for the sampled rows, against candidates of their groups
+    cand_full = np.full((G, C), -1, dtype=np.int32)
+    cand_full[groups] = cand
+    need = np.unique(ref_rows // g)
+    missing = np.setdiff1d(need, groups).astype(np.int32)
+    if len(missing):
+        pq2, pqs2, pw2 = oracle.proxy_reduce(p.dtype, q, qs, w, g, groups=missing)
+        pq_full[missing], pw_full[missing] = pq2, pw2
+        if pqs2 is not None:
+            pqs_full[missing] = pqs2
+        c2, _ = oracle.proxy_scan(p.dtype, pq_full, pqs_full, pw_full, kk, ks, L, g, C,
+                                  groups=missing)
+        cand_full[missing] = c2
+    t0 = time.perf_counter()
+    oracle.refine(p.dtype, q, qs, w, kk, ks, g, cand_full, k, rows=ref_rows)
+    t_ref = time.perf_counter() - t0
+    m = min(C, L)
+    ref_all = m * (m + 1) / 2 + (L - m) * C          # sum over t of min(C, t + 1)
+    ref_full = t_ref * ref_all / float(np.sum(np.minimum(C, ref_rows.astype(np.float64) + 1)))
+    t0 = time.perf_counter()
+    oracle.reuse(L, g, cand_full, k, rows=ref_rows)
+    t_reu = time.perf_counter() - t0
+    reu_full = t_reu * L / len(ref_rows)
+
+    total = dense_full + red_full + scan_full + ref_full + reu_full
+    desc = (f"{len(dense_rows)} dense rows, {len(groups)} proxy-scan groups, {len(ref_rows)} "
+            f"Refine/Reuse rows, {len(groups)} proxy groups, sampled evenly over positions; "
+            f"each part scaled to the full step by causal pairs (dense, scan, Refine) or by "
+            f"count (reduce, Reuse); sample CPU time {t_dense + t_red + t_scan + t_ref + t_reu:.1f}s")
+    parts = {"dense_s": dense_full, "reduce_s": red_full, "scan_s": scan_full,
+             "refine_s": ref_full, "reuse_s": reu_full}
+    return total, desc, threads, parts
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args, wl):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    p = make_inputs(wl, rank_seed(args.seed, 0))
+    times = []
+    desc, threads = "", 0
+    for i in range(args.warmup + args.steps):
+        total, desc, threads, _ = oracle_sample_time(p, wl, seed=i)
+        if i >= args.warmup:
+            times.append(total)
+    t = float(np.mean(times))
+    value = p.L / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": gen.DTYPE_NAMES[wl["dtype"]], "data": "synthetic",
+            "config": config_of(wl, args),
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": threads,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl, args):
+    return {"workload": args.workload, "L": wl["L"], "H": wl["H"], "D": wl["D"],
+            "g": wl["g"], "C": wl["C"], "topk": wl["topk"],
+            "q_k_format": gen.DTYPE_NAMES[wl["dtype"]] + (" + fp32 per-token scale"
+                                                         if wl["dtype"] == gen.E4M3 else ""),
+            "step": "dense index + proxy reduce + proxy scan + Reuse + Refine, all L queries",
+            "parallelism": f"replicas{dist_env()[2]}",
+            "l2": "no flush: inputs and score buffers larger than L2 (q alone 1 GiB)"}
+
+
+def run_ours(args, wl):
+    import torch.distributed as dist
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+    p = make_inputs(wl, rank_seed(args.seed, rank))
+    run = Runner(p, wl, device)
+    pv = run.pv
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        run.step()
+    barrier()
+    assert pv.device_error() == 0, "a kernel reported an error during warm-up"
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    pv.pivot_profile_enable(1)
+    n0 = pv.pivot_launch_count()
+    barrier()
+    start.record(run.stream)
+    for i in range(args.steps):
+        run.step(ev[i])
+    stop.record(run.stream)
+    barrier()
+    n1 = pv.pivot_launch_count()
+    pv.pivot_profile_enable(0)
+    clk = clocks.stop()
+    ms = start.elapsed_time(stop)
+    ms_max = max_over_ranks(ms, device)
+    assert pv.device_error() == 0, "a kernel reported an error in the timed region"
+
+    stage = np.zeros(5)
+    for e in ev:
+        for j in range(5):
+            stage[j] += e[j].elapsed_time(e[j + 1])
+    stage /= args.steps
+    dense_ms, red_ms, scan_ms, reu_ms, ref_ms = stage
+    L = run.L
+    modes = {
+        "dense": {"ms": dense_ms, "queries_per_s": L / (dense_ms / 1e3)},
+        "reuse": {"ms": red_ms + scan_ms + reu_ms,
+                  "queries_per_s": L / ((red_ms + scan_ms + reu_ms) / 1e3)},
+        "refine": {"ms": red_ms + scan_ms + ref_ms,
+                   "queries_per_s": L / ((red_ms + scan_ms + ref_ms) / 1e3)},
+        "stages_ms": {"dense": dense_ms, "proxy_reduce": red_ms, "proxy_scan": scan_ms,
+                      "reuse": reu_ms, "refine": ref_ms},
+    }
+    modes["reuse"]["speedup_vs_dense"] = dense_ms / modes["reuse"]["ms"]
+    modes["refine"]["speedup_vs_dense"] = dense_ms / modes["refine"]["ms"]
+
+    # kernels, roofline of the dominant one
+    peaks, peak_src = load_peaks()
+    kern = {}
+    for kid, name in pv.KERNELS.items():
+        n, kms, work = pv.profile_read(kid)
+        kern[name] = {"launches": n, "ms": kms, "work": work}
+    total_k = sum(v["ms"] for v in kern.values()) or 1.0
+    for v in kern.values():
+        v["share"] = v["ms"] / total_k
+    flop_pair = 2.0 * run.H * run.D
+    fp8 = wl["dtype"] == gen.E4M3
+    tc_peak_burst = peaks["bf16_tflops"] * (FP8_OVER_BF16 if fp8 else 1.0)
+    tc_peak = peaks["bf16_tflops_sustained"] * (FP8_OVER_BF16 if fp8 else 1.0)
+    for name in ("scan", "refine"):
+        v = kern[name]
+        if v["ms"] > 0:
+            v["tflops"] = v["work"] * flop_pair / (v["ms"] / 1e3) / 1e12
+    for name in ("select",):
+        v = kern[name]
+        if v["ms"] > 0:
+            v["gbs_scores"] = v["work"] * 4 / (v["ms"] / 1e3) / 1e9
+    for name in ("reduce", "reuse"):
+        v = kern[name]
+        if v["ms"] > 0:
+            v["gbs"] = v["work"] / (v["ms"] / 1e3) / 1e9
+    dom = max(kern, key=lambda n: kern[n]["ms"])
+    dv = kern[dom]
+    if dom in ("scan", "refine"):
+        ach = dv["tflops"]
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": ach / tc_peak, "traffic": None,
+                "peak_source": f"{peak_src} bf16 sustained x {FP8_OVER_BF16 if fp8 else 1.0} "
+                               f"({'fp8' if fp8 else 'bf16'} nominal ratio)",
+                "frac_of_burst": ach / tc_peak_burst,
+                "per_launch": {"work_pairs": dv["work"] / max(dv["launches"], 1),
+                               "ms": dv["ms"] / max(dv["launches"], 1)}}
+    else:
+        key = "gbs_scores" if dom == "select" else "gbs"
+        ach = dv[key]
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peak_src} hbm"}
+
+    # quality
+    rec = {"reuse_vs_dense": recall_stats(run.dense, run.reu),
+           "refine_vs_dense": recall_stats(run.dense, run.ref),
+           "dense_neighbour_overlap": neighbour_overlap(run.dense)}
+
+    # end to end through host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        pinned = {n: (None if t is None else t.pin_memory()) for n, t in run.host.items()}
+        outs = [torch.empty(run.L, run.k, dtype=torch.int32).pin_memory() for _ in range(3)]
+
+        def e2e_step():
+            for n, t in pinned.items():
+                if t is not None:
+                    run.dev[n].copy_(t, non_blocking=True)
+            run.step()
+            for o, dsrc in zip(outs, (run.dense, run.reu, run.ref)):
+                o.copy_(dsrc, non_blocking=True)
+        e2e_step()
+        barrier()
+        k_e2e = max(1, min(args.steps, 3))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(run.stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        b.record(run.stream)
+        barrier()
+        e_ms = max_over_ranks(a.elapsed_time(b), device)
+        e2e = {"value": aggregate_value(L, world, e_ms, k_e2e), "unit": "queries/s",
+               "h2d_bytes_per_step": run.h2d_bytes(), "d2h_bytes_per_step": run.d2h_bytes(),
+               "ms_per_step": e_ms / k_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        total, desc, threads, parts = oracle_sample_time(p, wl)
+        cpu = {"value": L / total, "unit": "queries/s", "cores": threads, "kind": "oracle",
+               "sample": desc, "extrapolated_step_s": total, "parts_s": parts}
+
+    value = aggregate_value(L, world, ms_max, args.steps)
+    line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": gen.DTYPE_NAMES[wl["dtype"]], "data": "synthetic",
+            "config": config_of(wl, args), "modes": modes, "recall": rec,
+            "roofline": roof, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(n1 - n0), "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=[k for k in gen.WORKLOADS if "decode" not in k])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = dict(gen.WORKLOADS[args.workload])
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -183,6 +183,25 @@ pivot_status_t pivot_set_wait_limit_ns(uint64_t ns);
  * usable.  Not needed in normal use. */
 pivot_status_t pivot_selftest_wait_timeout(void* stream);
 
+/* Kernel timing, off by default.  pivot_profile_enable(1) clears the
+ * counters and, from then on, brackets every kernel launch of the library
+ * with two CUDA events on the launch's stream and records the launch's
+ * algorithmic work; pivot_profile_enable(0) stops recording.
+ * pivot_profile_read(kernel, ...) waits for the recorded events and returns,
+ * for one kernel class, the launches, the summed event time in ms and the
+ * summed work.  Kernel classes and their work units:
+ *   0 scan    causal (query or proxy row, key) pairs scored
+ *   1 select  score entries examined by the top-k selection
+ *   2 refine  (member, candidate) pairs, sum over members of min(C, t+1)
+ *   3 reduce  bytes of the proxy reduce (member rows in, proxy rows out)
+ *   4 reuse   bytes of Reuse (index rows out, candidate prefixes in)
+ * Work is 0 for decode launches, whose sizes live on the device. */
+pivot_status_t pivot_profile_enable(int32_t on);
+pivot_status_t pivot_profile_read(int32_t kernel, int64_t* launches, double* total_ms,
+                                  double* work);
+/* Kernels launched by this library in this process so far. */
+int64_t pivot_launch_count(void);
+
 const char* pivot_status_string(pivot_status_t status);
 int32_t pivot_version(void);
 

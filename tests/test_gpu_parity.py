@@ -113,12 +113,14 @@ def test_tiny_invariants_on_gpu(tiny):
 
 
 @pytest.mark.parametrize("L,g,C,kk", [
-    (37, 4, 16, 8),          # fewer keys than a tile; prefixes shorter than k
-    (300, 5, 64, 64),        # C == k; g not a power of two; ragged group
-    (129, 3, 300, 7),        # C larger than every prefix
-    (515, 8, 40, 1),         # k = 1
+    (37, 4, 16, 8),          # fewer keys than a tile; prefixes shorter than k; 1-member tail
+    (300, 4, 64, 64),        # C == k
+    (129, 2, 300, 7),        # C larger than every prefix
+    (514, 8, 40, 1),         # k = 1; 2-member tail group
 ])
 def test_edge_shapes_exact(L, g, C, kk):
+    """Every group has a power-of-two member count, so the proxy mean of
+    integers is exact at TF32 and every comparison is bit for bit."""
     p = gen.make_prefill(L, 4, 32, F32, kind="int", seed=L)
     dev = to_device(p)
     q, qs, w, k, ks = p.codes()
@@ -130,6 +132,26 @@ def test_edge_shapes_exact(L, g, C, kk):
     assert_rows_exact(cand.cpu(), ocand, "cand")
     assert_rows_exact(reu.cpu(), oracle.reuse(L, g, ocand, kk), "reuse")
     assert_rows_exact(ref.cpu(), oracle.refine(F32, q, qs, w, k, ks, g, ocand, kk)[0], "refine")
+
+
+@pytest.mark.parametrize("L,g,C,kk", [(300, 5, 64, 64), (515, 3, 40, 9)])
+def test_edge_shapes_odd_groups(L, g, C, kk):
+    """g not a power of two: the proxy mean is not dyadic, the TF32 scan
+    rounds it, so candidates compare within tolerance; Reuse and Refine on
+    the GPU's own candidates stay exact (members' own integer queries)."""
+    p = gen.make_prefill(L, 4, 32, F32, kind="int", seed=L + 1)
+    dev = to_device(p)
+    q, qs, w, k, ks = p.codes()
+    pq, pqs, pw, cand, cs, reu, ref, _ = _pivot_gpu(p, dev, g, C, kk)
+    opq, opqs, opw = oracle.proxy_reduce(F32, q, qs, w, g)
+    assert (pq.cpu().numpy() == opq).all() and (pw.cpu().numpy() == opw).all()
+    groups = np.arange(opq.shape[0])
+    ocand, ocs = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, L, g, C)
+    assert_rows_close(cand.cpu().numpy(), ocand, ocs, proxy_score_fn(p, opq, opqs, opw), groups,
+                      "cand", gpu_scores=cs.cpu().numpy())
+    gc = cand.cpu().numpy()
+    assert_rows_exact(reu.cpu(), oracle.reuse(L, g, gc, kk), "reuse")
+    assert_rows_exact(ref.cpu(), oracle.refine(F32, q, qs, w, k, ks, g, gc, kk)[0], "refine")
 
 
 def test_row_ranges_and_small_workspace_match_one_call(tiny):

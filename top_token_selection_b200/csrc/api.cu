@@ -4,6 +4,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "profile.h"
 
 namespace pivot {
 
@@ -120,10 +121,37 @@ pivot_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? PIVOT_OK : P
 
 long long score_stride(int nkeys) { return (long long)align_up((size_t)nkeys, 32); }
 
-// Rows of scores that fit in `bytes`, a multiple of `unit`, at least one unit.
-long long rows_fitting(size_t bytes, long long stride, int unit) {
-    long long r = (long long)(bytes / ((size_t)stride * 4));
-    return r / unit * unit;
+// Rows per chunk for `total` rows of `rowbytes` each in `bytes` of
+// workspace: all of them if they fit, else a multiple of `unit` when at
+// least one unit fits, else as many as fit (0 if not even one row fits).
+long long chunk_rows(size_t bytes, size_t rowbytes, long long total, int unit) {
+    const long long fit = (long long)(bytes / rowbytes);
+    if (fit >= total) return total;
+    if (fit >= unit) return fit / unit * unit;
+    return fit;
+}
+
+// Causal (row, key) pairs of rows [r0, r1): the algorithmic work of a scan.
+// Decode rows depend on device-side cache lengths: reported as 0.
+double scan_pairs(int kind, int r0, int r1, int L, int g) {
+    double s = 0.0;
+    if (kind == SCAN_PREFILL_DENSE) {
+        s = 0.5 * ((double)r1 * (r1 + 1) - (double)r0 * (r0 + 1));
+    } else if (kind == SCAN_PREFILL_PROXY) {
+        for (int j = r0; j < r1; ++j) s += (double)((j + 1) * (long long)g < L ? (j + 1) * g : L);
+    }
+    return s;
+}
+
+// (member, candidate) pairs of prefill Refine rows [r0, r1): sum of min(C, t+1).
+double refine_pairs(int r0, int r1, int C) {
+    double s = 0.0;
+    const int knee = C - 1;   // rows t >= knee see C candidates
+    const int a_end = r1 < knee ? r1 : knee;
+    if (r0 < a_end) s += 0.5 * ((double)a_end * (a_end + 1) - (double)r0 * (r0 + 1));
+    const int b0 = r0 > knee ? r0 : knee;
+    if (b0 < r1) s += (double)(r1 - b0) * C;
+    return s;
 }
 
 // ------------------------------------------------------------------ scans
@@ -165,12 +193,14 @@ pivot_status_t run_scan(int kind, int dtype, int H, int D, const void* qbase, lo
         if (!make_tmap(&tk, dtype, kbase, k_rows, D, 128)) return PIVOT_ERR_CUDA;
         if (!make_tmap(&tq, dtype, qbase, q_rows * H, D, P * H)) return PIVOT_ERR_CUDA;
         const int grid = p.nitems < num_sms() ? p.nitems : num_sms();
-        return from_cuda(launch_scan_umma(tk, tq, p, grid, st));
+        return from_cuda(profiled(PK_SCAN, scan_pairs(kind, r0, r1, L, g), st,
+                                  [&] { return launch_scan_umma(tk, tq, p, grid, st); }));
     }
     p.tiles_per_item = 1;
     p.items_per_block = nt;
     p.nitems = nblocks * nt;
-    return from_cuda(launch_scan_simt(qbase, kbase, p, st));
+    return from_cuda(profiled(PK_SCAN, scan_pairs(kind, r0, r1, L, g), st,
+                              [&] { return launch_scan_simt(qbase, kbase, p, st); }));
 }
 
 int rows_per_block(int H, int D, int dtype) {
@@ -198,7 +228,8 @@ pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, in
     sp.out_score = out_score;
     sp.out_base = out_base;
     sp.tail_cap = TAIL_CAP;
-    return from_cuda(launch_select(sp, st));
+    return from_cuda(profiled(PK_SELECT, scan_pairs(scan_kind, r0, r1, L, g), st,
+                              [&] { return launch_select(sp, st); }));
 }
 
 pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int Gm, int maxlen,
@@ -225,7 +256,8 @@ pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int 
     sp.out_score = out_score;
     sp.out_base = out_base;
     sp.tail_cap = TAIL_CAP;
-    return from_cuda(launch_select(sp, st));
+    return from_cuda(profiled(PK_SELECT, (double)(r1 - r0) * C, st,
+                              [&] { return launch_select(sp, st); }));
 }
 
 pivot_status_t run_refine_scores(int kind, int dtype, int H, int D, const void* q,
@@ -256,7 +288,8 @@ pivot_status_t run_refine_scores(int kind, int dtype, int H, int D, const void* 
     rp.cand_base = cand_base;
     rp.C = C;
     rp.S = S;
-    return from_cuda(launch_refine_simt(rp, st));
+    const double work = kind == SCAN_PREFILL_DENSE ? refine_pairs(r0, r1, C) : 0.0;
+    return from_cuda(profiled(PK_REFINE, work, st, [&] { return launch_refine_simt(rp, st); }));
 }
 
 // Carve `bytes` (256-aligned) from the workspace cursor.
@@ -346,7 +379,7 @@ size_t pivot_dense_index_workspace_size(const pivot_seq_t* seq, int32_t topk) {
     const size_t rb = dense_rowbytes(seq->L);
     long long rows = t1 - t0;
     long long cap = (long long)(SCORE_BUF_CAP / rb) / P * P;
-    if (cap < P) cap = P;
+    if (cap < 1) cap = 1;
     if (rows > cap) rows = cap;
     return align_up((size_t)rows * rb, WS_ALIGN);
 }
@@ -361,8 +394,8 @@ pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* 
     if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
     const int P = rows_per_block(seq->H, seq->D, seq->dtype);
     const long long stride = score_stride(seq->L);
-    long long chunk = rows_fitting(ws_bytes, stride, P);
-    if (chunk < P) return PIVOT_ERR_WORKSPACE;
+    const long long chunk = chunk_rows(ws_bytes, (size_t)stride * 4, t1 - t0, P);
+    if (chunk < 1) return PIVOT_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* S = static_cast<float*>(ws);
     for (long long c0 = t0; c0 < t1; c0 += chunk) {
@@ -403,7 +436,9 @@ pivot_status_t pivot_proxy_reduce(const pivot_seq_t* seq, int32_t g, void* pq, f
     rp.pq_scale = pq_scale;
     rp.pw = pw;
     rp.group_stride_members = g;
-    return from_cuda(launch_proxy_reduce(rp, static_cast<cudaStream_t>(stream)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const double bytes = ((double)(t1 - t0) + rp.ngroups) * seq->H * (seq->D * rp.esize + 4.0);
+    return from_cuda(profiled(PK_REDUCE, bytes, s, [&] { return launch_proxy_reduce(rp, s); }));
 }
 
 // -------------------------------------------------------------- proxy scan
@@ -414,7 +449,7 @@ size_t pivot_proxy_scan_workspace_size(const pivot_seq_t* seq, int32_t g, int32_
     const size_t rb = dense_rowbytes(seq->L);
     long long rows = ceil_div(t1 - t0, g);
     long long cap = (long long)(SCORE_BUF_CAP / rb) / P * P;
-    if (cap < P) cap = P;
+    if (cap < 1) cap = 1;
     if (rows > cap) rows = cap;
     return align_up((size_t)rows * rb, WS_ALIGN);
 }
@@ -432,9 +467,9 @@ pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* p
     if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
     const int P = rows_per_block(seq->H, seq->D, seq->dtype);
     const long long stride = score_stride(seq->L);
-    long long chunk = rows_fitting(ws_bytes, stride, P);
-    if (chunk < P) return PIVOT_ERR_WORKSPACE;
     const int j0 = t0 / g, j1 = ceil_div(t1, g);
+    const long long chunk = chunk_rows(ws_bytes, (size_t)stride * 4, j1 - j0, P);
+    if (chunk < 1) return PIVOT_ERR_WORKSPACE;
     const int G = j1 - j0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* S = static_cast<float*>(ws);
@@ -458,8 +493,11 @@ pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int3
                            int32_t C, int32_t topk, int32_t* idx, void* stream) {
     if (g < 1 || t_begin < 0 || t_end <= t_begin || t_begin % g) return PIVOT_ERR_INVALID_ARG;
     if (!cand || !idx || topk < 1 || C < topk) return PIVOT_ERR_INVALID_ARG;
-    return from_cuda(
-        launch_reuse(t_begin, t_end, g, cand, C, topk, idx, static_cast<cudaStream_t>(stream)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const double bytes = 4.0 * topk * ((double)(t_end - t_begin) + ceil_div(t_end - t_begin, g));
+    return from_cuda(profiled(PK_REUSE, bytes, s, [&] {
+        return launch_reuse(t_begin, t_end, g, cand, C, topk, idx, s);
+    }));
 }
 
 // ------------------------------------------------------------------ refine
@@ -469,7 +507,7 @@ size_t pivot_refine_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C,
     long long rows = t1 - t0;
     const size_t rb = (size_t)C * 4;
     long long cap = (long long)(SCORE_BUF_CAP / rb) / g * g;
-    if (cap < g) cap = g;
+    if (cap < 1) cap = 1;
     if (rows > cap) rows = cap;
     return align_up((size_t)rows * rb, WS_ALIGN);
 }
@@ -484,8 +522,8 @@ pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* ca
     if (!cand || !idx || topk < 1 || C < topk) return PIVOT_ERR_INVALID_ARG;
     if (C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
-    long long chunk = (long long)(ws_bytes / ((size_t)C * 4)) / g * g;
-    if (chunk < g) return PIVOT_ERR_WORKSPACE;
+    const long long chunk = chunk_rows(ws_bytes, (size_t)C * 4, t1 - t0, g);
+    if (chunk < 1) return PIVOT_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* S = static_cast<float*>(ws);
     const int j0 = t0 / g;
@@ -595,7 +633,9 @@ pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, in
     rp.pq_scale = b->dtype == PIVOT_E4M3 ? w.pqs : nullptr;
     rp.pw = w.pw;
     rp.group_stride_members = b->Gm;
-    if ((st = from_cuda(launch_proxy_reduce(rp, s))) != PIVOT_OK) return st;
+    if ((st = from_cuda(profiled(PK_REDUCE, 0.0, s, [&] { return launch_proxy_reduce(rp, s); }))) !=
+        PIVOT_OK)
+        return st;
     st = run_scan(SCAN_DECODE_PROXY, b->dtype, b->H, b->D, w.pq, b->B, 0, w.pw,
                   b->dtype == PIVOT_E4M3 ? w.pqs : nullptr, b->kc, krows, b->kc_scale, 0, 1, b->Gm,
                   b->maxlen, b->cache_len, 1, 0, b->B, b->maxlen - 1, w.S, stride, s);
@@ -608,8 +648,9 @@ pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, in
             cudaSuccess)
             return PIVOT_ERR_CUDA;
     if (mode == PIVOT_MODE_REUSE)
-        return from_cuda(launch_decode_reuse(b->B, b->Gm, b->maxlen, b->cache_len, w.cand, C, topk,
-                                             idx, s));
+        return from_cuda(profiled(PK_REUSE, 0.0, s, [&] {
+            return launch_decode_reuse(b->B, b->Gm, b->maxlen, b->cache_len, w.cand, C, topk, idx, s);
+        }));
     const int rows = b->B * b->Gm;
     st = run_refine_scores(SCAN_DECODE_DENSE, b->dtype, b->H, b->D, b->q, 0, b->q_scale, b->w,
                            b->kc, b->kc_scale, 0, 1, b->Gm, b->maxlen, b->cache_len, w.cand, 0, C,

@@ -29,8 +29,10 @@ ABI_SYMBOLS = [
     "pivot_proxy_scan", "pivot_proxy_scan_workspace_size", "pivot_reuse", "pivot_refine",
     "pivot_refine_workspace_size", "pivot_decode", "pivot_decode_workspace_size",
     "pivot_get_device_error", "pivot_set_wait_limit_ns", "pivot_selftest_wait_timeout",
-    "pivot_status_string", "pivot_version",
+    "pivot_status_string", "pivot_version", "pivot_profile_enable", "pivot_profile_read",
+    "pivot_launch_count",
 ]
+KERNELS = {0: "scan", 1: "select", 2: "refine", 3: "reduce", 4: "reuse"}
 
 
 class PivotError(RuntimeError):
@@ -83,6 +85,9 @@ def load(path: str = LIB_PATH):
         "pivot_selftest_wait_timeout": ([P], I32),
         "pivot_status_string": ([I32], ctypes.c_char_p),
         "pivot_version": ([], I32),
+        "pivot_profile_enable": ([I32], I32),
+        "pivot_profile_read": ([I32, P, P, P], I32),
+        "pivot_launch_count": ([], ctypes.c_int64),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -151,6 +156,28 @@ def pivot_selftest_wait_timeout(stream):
     return load().pivot_selftest_wait_timeout(stream)
 
 
+def pivot_profile_enable(on):
+    return load().pivot_profile_enable(on)
+
+
+def pivot_profile_read(kernel, launches, total_ms, work):
+    return load().pivot_profile_read(kernel, launches, total_ms, work)
+
+
+def pivot_launch_count():
+    return load().pivot_launch_count()
+
+
+def profile_read(kernel):
+    """(launches, total_ms, work) of one kernel class since profiling began."""
+    n = ctypes.c_int64(0)
+    ms = ctypes.c_double(0.0)
+    wk = ctypes.c_double(0.0)
+    _check(pivot_profile_read(kernel, ctypes.byref(n), ctypes.byref(ms), ctypes.byref(wk)),
+           "pivot_profile_read")
+    return n.value, ms.value, wk.value
+
+
 def pivot_status_string(status):
     return load().pivot_status_string(status).decode()
 
@@ -196,15 +223,21 @@ def _workspace(nbytes, device):
 
 
 def make_seq(q, q_scale, w, k, k_scale, t_begin=0, t_end=0) -> PivotSeq:
+    """Describe one prefill sequence; the struct keeps the tensors alive."""
     L, H, D = q.shape
-    return PivotSeq(_dtype_code(q), L, H, D, _p(q), _p(q_scale), _p(w), _p(k), _p(k_scale),
-                    t_begin, t_end)
+    s = PivotSeq(_dtype_code(q), L, H, D, _p(q), _p(q_scale), _p(w), _p(k), _p(k_scale),
+                 t_begin, t_end)
+    s._keep = (q, q_scale, w, k, k_scale)
+    return s
 
 
 def make_decode(q, q_scale, w, kc, kc_scale, cache_len) -> PivotDecode:
+    """Describe one decode batch; the struct keeps the tensors alive."""
     B, Gm, H, D = q.shape
-    return PivotDecode(_dtype_code(q), B, Gm, H, D, kc.shape[1], _p(q), _p(q_scale), _p(w),
-                       _p(kc), _p(kc_scale), _p(cache_len))
+    s = PivotDecode(_dtype_code(q), B, Gm, H, D, kc.shape[1], _p(q), _p(q_scale), _p(w),
+                    _p(kc), _p(kc_scale), _p(cache_len))
+    s._keep = (q, q_scale, w, kc, kc_scale, cache_len)
+    return s
 
 
 def _rows(seq):
