@@ -468,7 +468,9 @@ def run_ours(args, wl):
             v["gbs"] = v["work"] / (v["ms"] / 1e3) / 1e9
     dom = max(kern, key=lambda n: kern[n]["ms"])
     dv = kern[dom]
-    if dom in ("scan", "refine"):
+    if dv["ms"] <= 0:
+        roof = None
+    elif dom in ("scan", "refine"):
         ach = dv["tflops"]
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": tc_peak,
                 "unit": "TFLOP/s", "frac": ach / tc_peak, "traffic": None,

@@ -186,7 +186,8 @@ pivot_status_t pivot_selftest_wait_timeout(void* stream);
 /* Kernel timing, off by default.  pivot_profile_enable(1) clears the
  * counters and, from then on, brackets every kernel launch of the library
  * with two CUDA events on the launch's stream and records the launch's
- * algorithmic work; pivot_profile_enable(0) stops recording.
+ * algorithmic work; pivot_profile_enable(0) stops recording and keeps the
+ * totals for reading.
  * pivot_profile_read(kernel, ...) waits for the recorded events and returns,
  * for one kernel class, the launches, the summed event time in ms and the
  * summed work.  Kernel classes and their work units:

@@ -13,7 +13,7 @@ from top_token_selection_b200 import inputs as gen
 from top_token_selection_b200 import pivot as pv
 
 from parity import (assert_rows_close, assert_rows_exact, proxy_score_fn, score_fn_for, seq_of,
-                    to_device)
+                    tf32_abs_tol, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -136,9 +136,10 @@ def test_edge_shapes_exact(L, g, C, kk):
 
 @pytest.mark.parametrize("L,g,C,kk", [(300, 5, 64, 64), (515, 3, 40, 9)])
 def test_edge_shapes_odd_groups(L, g, C, kk):
-    """g not a power of two: the proxy mean is not dyadic, the TF32 scan
-    rounds it, so candidates compare within tolerance; Reuse and Refine on
-    the GPU's own candidates stay exact (members' own integer queries)."""
+    """g not a power of two: the proxy mean is not dyadic and the tensor
+    cores consume fp32 at TF32, so candidates compare within the TF32 error
+    bound; Reuse and Refine on the GPU's own candidates stay exact (members'
+    own integer queries)."""
     p = gen.make_prefill(L, 4, 32, F32, kind="int", seed=L + 1)
     dev = to_device(p)
     q, qs, w, k, ks = p.codes()
@@ -148,7 +149,7 @@ def test_edge_shapes_odd_groups(L, g, C, kk):
     groups = np.arange(opq.shape[0])
     ocand, ocs = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, L, g, C)
     assert_rows_close(cand.cpu().numpy(), ocand, ocs, proxy_score_fn(p, opq, opqs, opw), groups,
-                      "cand", gpu_scores=cs.cpu().numpy())
+                      "cand", gpu_scores=cs.cpu().numpy(), abs_tol=tf32_abs_tol(opq, opw, k))
     gc = cand.cpu().numpy()
     assert_rows_exact(reu.cpu(), oracle.reuse(L, g, gc, kk), "reuse")
     assert_rows_exact(ref.cpu(), oracle.refine(F32, q, qs, w, k, ks, g, gc, kk)[0], "refine")
@@ -174,6 +175,28 @@ def test_row_ranges_and_small_workspace_match_one_call(tiny):
     ref2, _ = pv.refine(seq2, g, cand2, kk)
     assert torch.equal(ref2, ref[512:])
     assert torch.equal(pv.reuse(512, 1024, g, cand2, kk), reu[512:])
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_zigzag_sharded_calls_match_one_call(tiny, world):
+    """Each rank's zig-zag row ranges, run as separate calls (as separate
+    GPUs would), reassemble the single-call result exactly."""
+    from top_token_selection_b200.sharding import zigzag_ranges
+    p, dev, cfg = tiny
+    g, C, kk = cfg["g"], cfg["C"], cfg["topk"]
+    full_dense, _ = pv.dense_index(seq_of(dev), kk)
+    _, _, _, full_cand, _, full_reu, full_ref, _ = _pivot_gpu(p, dev, g, C, kk, with_score=False)
+    for rank in range(world):
+        for a, b in zigzag_ranges(p.L, g, world, rank):
+            seq = seq_of(dev, a, b)
+            d, _ = pv.dense_index(seq, kk)
+            assert torch.equal(d, full_dense[a:b])
+            pq, pqs, pw = pv.proxy_reduce(seq, g)
+            cand, _ = pv.proxy_scan(seq, g, pq, pqs, pw, C)
+            assert torch.equal(cand, full_cand[a // g:-(-b // g)])
+            assert torch.equal(pv.reuse(a, b, g, cand, kk), full_reu[a:b])
+            r, _ = pv.refine(seq, g, cand, kk)
+            assert torch.equal(r, full_ref[a:b])
 
 
 # ---------------------------------------------------------------------------

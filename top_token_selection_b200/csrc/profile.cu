@@ -86,10 +86,12 @@ extern "C" {
 pivot_status_t pivot_profile_enable(int32_t on) {
     std::lock_guard<std::mutex> lk(g_mu);
     resolve_pending();
-    for (int k = 0; k < PK_COUNT; ++k) {
-        g_count[k] = 0;
-        g_ms[k] = 0.0;
-        g_work[k] = 0.0;
+    if (on) {   // a new measurement starts from zero; turning off keeps the totals
+        for (int k = 0; k < PK_COUNT; ++k) {
+            g_count[k] = 0;
+            g_ms[k] = 0.0;
+            g_work[k] = 0.0;
+        }
     }
     g_on = on != 0;
     return PIVOT_OK;
