@@ -167,6 +167,26 @@ pivot_status_t pivot_decode(const pivot_decode_t* batch, int32_t mode, int32_t C
 size_t pivot_decode_workspace_size(const pivot_decode_t* batch, int32_t mode, int32_t C,
                                    int32_t topk);
 
+/* pivot_decode without a caller workspace, for callers that cannot allocate
+ * device memory at the call site -- e.g. a plugin inside an inference engine
+ * whose memory planner owns the whole device, or a per-token decode loop
+ * that may not add an allocation mid-step.  This entry point has no
+ * counterpart on the pages; it is a packaging of pivot_decode.
+ *
+ * Arguments and results are those of pivot_decode (inputs and outputs are
+ * still the caller's device buffers).  The scratch space is a fixed 64 MiB
+ * array inside the library, one per device, held from when the library is
+ * loaded until the process exits; the call allocates nothing.  A batch
+ * whose pivot_decode_workspace_size() exceeds 64 MiB is rejected with
+ * PIVOT_ERR_WORKSPACE before anything is enqueued.  The first call on each
+ * device looks up that device's array address (with the device current);
+ * make that first call before any stream capture.  Every call on a device
+ * uses the same array and leaves its contents behind: calls that can
+ * overlap on the GPU (different streams without ordering) race on it and
+ * must be serialised by the caller. */
+pivot_status_t pivot_decode_noalloc(const pivot_decode_t* batch, int32_t mode, int32_t C,
+                                    int32_t topk, int32_t* idx, int32_t* cand, void* stream);
+
 /* Waits for `stream`, then returns and clears the current device's error
  * word: PIVOT_OK, PIVOT_ERR_TIMEOUT or PIVOT_ERR_DEVICE (PIVOT_ERR_CUDA if
  * the wait itself failed). */

@@ -30,7 +30,7 @@ ABI_SYMBOLS = [
     "pivot_refine_workspace_size", "pivot_decode", "pivot_decode_workspace_size",
     "pivot_get_device_error", "pivot_set_wait_limit_ns", "pivot_selftest_wait_timeout",
     "pivot_status_string", "pivot_version", "pivot_profile_enable", "pivot_profile_read",
-    "pivot_launch_count",
+    "pivot_launch_count", "pivot_decode_noalloc",
 ]
 KERNELS = {0: "scan", 1: "select", 2: "refine", 3: "reduce", 4: "reuse"}
 
@@ -88,6 +88,7 @@ def load(path: str = LIB_PATH):
         "pivot_profile_enable": ([I32], I32),
         "pivot_profile_read": ([I32, P, P, P], I32),
         "pivot_launch_count": ([], ctypes.c_int64),
+        "pivot_decode_noalloc": ([P, I32, I32, I32, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -142,6 +143,10 @@ def pivot_decode(batch, mode, C, topk, idx, cand, ws, ws_bytes, stream):
 
 def pivot_decode_workspace_size(batch, mode, C, topk):
     return load().pivot_decode_workspace_size(ctypes.byref(batch), mode, C, topk)
+
+
+def pivot_decode_noalloc(batch, mode, C, topk, idx, cand, stream):
+    return load().pivot_decode_noalloc(ctypes.byref(batch), mode, C, topk, idx, cand, stream)
 
 
 def pivot_get_device_error(stream):
