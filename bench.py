@@ -207,8 +207,8 @@ class Runner:
                                         self.pw.data_ptr(), sp), "reduce")
         mark(2)
         pv._check(pv.pivot_proxy_scan(self.seq, self.g, self.pq.data_ptr(), self._ptr(self.pqs),
-                                      self.pw.data_ptr(), self.C, self.cand.data_ptr(), None, ws,
-                                      wsn, sp), "scan")
+                                      self.pw.data_ptr(), self.C, self.k, self.cand.data_ptr(),
+                                      None, ws, wsn, sp), "scan")
         mark(3)
         pv._check(pv.pivot_reuse(0, self.L, self.g, self.cand.data_ptr(), self.C, self.k,
                                  self.reu.data_ptr(), sp), "reuse")
@@ -300,7 +300,7 @@ def oracle_sample_time(p, wl, budget_rows=None, seed=0):
     if pqs is not None:
         pqs_full[groups] = pqs
     t0 = time.perf_counter()
-    cand, _ = oracle.proxy_scan(p.dtype, pq_full, pqs_full, pw_full, kk, ks, L, g, C,
+    cand, _ = oracle.proxy_scan(p.dtype, pq_full, pqs_full, pw_full, kk, ks, L, g, C, k,
                                 groups=groups)
     t_scan = time.perf_counter() - t0
     e = np.minimum(L, (groups.astype(np.float64) + 1) * g)
@@ -317,7 +317,7 @@ def oracle_sample_time(p, wl, budget_rows=None, seed=0):
         pq_full[missing], pw_full[missing] = pq2, pw2
         if pqs2 is not None:
             pqs_full[missing] = pqs2
-        c2, _ = oracle.proxy_scan(p.dtype, pq_full, pqs_full, pw_full, kk, ks, L, g, C,
+        c2, _ = oracle.proxy_scan(p.dtype, pq_full, pqs_full, pw_full, kk, ks, L, g, C, k,
                                   groups=missing)
         cand_full[missing] = c2
     t0 = time.perf_counter()

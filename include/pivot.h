@@ -33,10 +33,12 @@
  *  - Layouts are row-major.  dtype PIVOT_F32: q, k are float32.  PIVOT_BF16:
  *    bfloat16.  PIVOT_E4M3: OCP FP8 e4m3 codes with one float32 scale per
  *    token (value = code * scale).  w is float32 in every dtype.
- *  - Output index rows hold positions in rank order -- higher score first,
- *    equal scores by lower position, -0 equal to +0 -- padded with -1 when
- *    fewer positions are eligible.  Optional score outputs are float32 with
- *    -inf padding.
+ *  - Selection keeps the k highest scores; equal scores are taken lower
+ *    position first; -0 equals +0.  Output index rows list the selected
+ *    positions in ascending order (the indexer hands on a set of positions;
+ *    the indexer tutorial's Fig. 1 lists them by position), padded with -1
+ *    when fewer positions are eligible.  Optional score outputs are float32,
+ *    aligned with the positions, -inf padding.
  *  - Argument errors are found before anything is enqueued and return
  *    PIVOT_ERR_INVALID_ARG / _UNSUPPORTED / _WORKSPACE; a failed launch
  *    returns PIVOT_ERR_CUDA.  Faults found by the kernels themselves (a
@@ -132,16 +134,19 @@ pivot_status_t pivot_proxy_reduce(const pivot_seq_t* seq, int32_t g, void* pq,
 
 /* One full-prefix scan per group (PIVOT abstract): proxy j scores keys
  * [0, e_j], e_j = min(L, (j+1)*g) - 1, with the dense score formula and
- * keeps its top-C.  cand [G, C] int32 in rank order (its first k entries
- * are the proxy's top-k); cand_score [G, C] or NULL.  1 <= C. */
+ * keeps its top-C.  cand [G, C] int32: the proxy's top-`topk` positions
+ * (ascending), then the rest of its top-C (ascending) -- so the first topk
+ * entries are what PIVOT-Reuse shares.  cand_score [G, C] or NULL.
+ * 1 <= topk <= C. */
 pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* pq,
                                  const float* pq_scale, const float* pw, int32_t C,
-                                 int32_t* cand, float* cand_score, void* ws,
+                                 int32_t topk, int32_t* cand, float* cand_score, void* ws,
                                  size_t ws_bytes, void* stream);
 size_t pivot_proxy_scan_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C);
 
 /* PIVOT-Reuse (PIVOT abstract): member t of group j takes the first topk
- * entries of cand[j], keeps those <= t in their order and pads with -1.
+ * entries of cand[j] (the proxy's top-k), keeps those <= t in their order
+ * (ascending) and pads with -1.
  * Rows [t_begin, t_end) with t_begin a multiple of g; cand rows relative to
  * t_begin / g.  idx [rows, topk].  1 <= topk <= C. */
 pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int32_t* cand,
@@ -160,7 +165,7 @@ size_t pivot_refine_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C,
  * group).  PIVOT_MODE_DENSE: each member scans its own prefix.  REUSE /
  * REFINE: the Gm members' proxy scans [0, cache_len[b] - 1] for its top-C,
  * then Reuse or Refine as in prefill.  idx [B, Gm, topk]; cand [B, C] or
- * NULL (the candidates, PIVOT modes only). */
+ * NULL (the candidates, laid out as in pivot_proxy_scan with topk). */
 pivot_status_t pivot_decode(const pivot_decode_t* batch, int32_t mode, int32_t C,
                             int32_t topk, int32_t* idx, int32_t* cand, void* ws,
                             size_t ws_bytes, void* stream);

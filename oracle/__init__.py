@@ -63,7 +63,7 @@ def _load():
             lib.oracle_score_positions.argtypes = [I, I, I, I, P, P, P, P, P, I, I, P, P]
             lib.oracle_dense_index.argtypes = [I, I, I, I, P, P, P, P, P, I, I, P, P, P, I]
             lib.oracle_proxy_reduce.argtypes = [I, I, I, I, P, P, P, I, I, P, P, P, P]
-            lib.oracle_proxy_scan.argtypes = [I, I, I, I, P, P, P, P, P, I, I, I, P, P, P, I]
+            lib.oracle_proxy_scan.argtypes = [I, I, I, I, P, P, P, P, P, I, I, I, I, P, P, P, I]
             lib.oracle_reuse.argtypes = [I, I, P, I, I, I, P, P]
             lib.oracle_refine.argtypes = [I, I, I, I, P, P, P, P, P, I, P, I, I, I, P, P, P, I]
             lib.oracle_decode.argtypes = [I, I, I, I, I, P, P, P, P, P, I, P, I, I, I, P, P, P, I]
@@ -156,7 +156,8 @@ def score_positions(dtype, q, q_scale, w, k, k_scale, row, positions):
 
 
 def dense_index(dtype, q, q_scale, w, k, k_scale, topk, rows=None, nthreads=0):
-    """Dense indexer: top-k positions (and fp64 scores) of each listed row."""
+    """Dense indexer: top-k positions, ascending (and their fp64 scores), of
+    each listed row."""
     lib = _load()
     L, H, D = q.shape
     q, k = _codes(q, dtype), _codes(k, dtype)
@@ -187,8 +188,9 @@ def proxy_reduce(dtype, q, q_scale, w, g, groups=None):
     return pq, pqs, pw
 
 
-def proxy_scan(dtype, pq, pq_scale, pw, k, k_scale, L, g, C, groups=None, nthreads=0):
-    """Top-C candidates of each listed group's proxy over [0, e_j]."""
+def proxy_scan(dtype, pq, pq_scale, pw, k, k_scale, L, g, C, topk, groups=None, nthreads=0):
+    """Top-C candidates of each listed group's proxy over [0, e_j]: the
+    top-`topk` positions ascending, then the rest ascending."""
     lib = _load()
     G, H, D = pq.shape
     pq, k = _codes(pq, dtype), _codes(k, dtype)
@@ -197,7 +199,7 @@ def proxy_scan(dtype, pq, pq_scale, pw, k, k_scale, L, g, C, groups=None, nthrea
     cand = np.empty((len(groups), C), dtype=np.int32)
     sc = np.empty((len(groups), C), dtype=np.float64)
     lib.oracle_proxy_scan(dtype, L, H, D, _ptr(pq), _ptr(pq_scale), _ptr(pw), _ptr(k),
-                          _ptr(k_scale), g, C, len(groups), _ptr(groups), _ptr(cand),
+                          _ptr(k_scale), g, C, topk, len(groups), _ptr(groups), _ptr(cand),
                           _ptr(sc), nthreads)
     return cand, sc
 

@@ -31,7 +31,11 @@
  *
  * Readings where the pages are silent (each listed in the design doc):
  *  - causal prefix is inclusive: query t sees s in [0, t]        ([TUT] Fig. 2)
- *  - order: higher score first, ties by lower position; -0 == +0
+ *  - selection: the k highest scores, equal scores lower position first;
+ *    -0 == +0; the selected positions are listed in ascending order (the
+ *    tutorial's Fig. 1 lists the picked positions by position)
+ *  - a candidate row lists the proxy's top-k first, then the rest of its
+ *    top-C, each ascending (Reuse shares the proxy's top-k)
  *  - fewer eligible positions than k: return them all, pad with -1
  *  - a group's full prefix runs through its last member e_j
  *  - the proxy averages both q and w, per head; a last partial group
@@ -174,10 +178,28 @@ static int entry_cmp(const void* a, const void* b) {
     return (x->pos < y->pos) ? -1 : (x->pos > y->pos);
 }
 
-/* Sort n entries and write the first min(k, n) positions (and scores);
- * pad the rest of the k slots with -1 (and -inf). */
-static void take_topk(entry_t* e, int n, int k, int32_t* out_idx, double* out_score) {
+/* Ascending position. */
+static int pos_cmp(const void* a, const void* b) {
+    const entry_t* x = (const entry_t*)a;
+    const entry_t* y = (const entry_t*)b;
+    return (x->pos < y->pos) ? -1 : (x->pos > y->pos);
+}
+
+/* Select the min(k, n) best entries (rank order: higher score, then lower
+ * position) and write their positions (and scores) in ascending position
+ * order -- the first min(split, k, n) best first, then the rest, when split
+ * is in (0, k); pad the rest of the k slots with -1 (and -inf). */
+static void take_topk_split(entry_t* e, int n, int k, int split, int32_t* out_idx,
+                            double* out_score) {
     qsort(e, (size_t)n, sizeof(entry_t), entry_cmp);
+    int m = n < k ? n : k;
+    int s = (split > 0 && split < m) ? split : 0;
+    if (s) {
+        qsort(e, (size_t)s, sizeof(entry_t), pos_cmp);
+        qsort(e + s, (size_t)(m - s), sizeof(entry_t), pos_cmp);
+    } else {
+        qsort(e, (size_t)m, sizeof(entry_t), pos_cmp);
+    }
     for (int i = 0; i < k; ++i) {
         if (i < n) {
             out_idx[i] = e[i].pos;
@@ -187,6 +209,10 @@ static void take_topk(entry_t* e, int n, int k, int32_t* out_idx, double* out_sc
             if (out_score) out_score[i] = -INFINITY;
         }
     }
+}
+
+static void take_topk(entry_t* e, int n, int k, int32_t* out_idx, double* out_score) {
+    take_topk_split(e, n, k, 0, out_idx, out_score);
 }
 
 /* Decode a query row (H*D values, times its scale) into qd. */
@@ -208,9 +234,10 @@ static double* decode_keys(int dtype, const void* k, const float* k_scale, int n
     return kd;
 }
 
-/* Top-k of one query row over keys [0, lim] (lim inclusive). */
+/* Top-k of one query row over keys [0, lim] (lim inclusive); with split in
+ * (0, k) the best `split` are listed first. */
 static void row_topk_prefix(int H, int D, const double* qd, const float* wrow,
-                            const double* kd, int lim, int k,
+                            const double* kd, int lim, int k, int split,
                             int32_t* out_idx, double* out_score) {
     int n = lim + 1;
     entry_t* e = (entry_t*)malloc(sizeof(entry_t) * (size_t)(n > 0 ? n : 1));
@@ -218,7 +245,7 @@ static void row_topk_prefix(int H, int D, const double* qd, const float* wrow,
         e[s].pos = s;
         e[s].score = indexer_score(H, D, qd, wrow, kd + (size_t)s * D);
     }
-    take_topk(e, n, k, out_idx, out_score);
+    take_topk_split(e, n, k, split, out_idx, out_score);
     free(e);
 }
 
@@ -274,7 +301,7 @@ int oracle_dense_index(int dtype, int L, int H, int D, const void* q,
         int t = rows[r];
         double* qd = (double*)malloc(sizeof(double) * (size_t)H * D);
         decode_qrow(dtype, q, q_scale, (size_t)t, H, D, qd);
-        row_topk_prefix(H, D, qd, w + (size_t)t * H, kd, t, topk,
+        row_topk_prefix(H, D, qd, w + (size_t)t * H, kd, t, topk, 0,
                         out_idx + (size_t)r * topk,
                         out_score ? out_score + (size_t)r * topk : NULL);
         free(qd);
@@ -369,10 +396,11 @@ int oracle_proxy_reduce(int dtype, int L, int H, int D, const void* q,
 
 /* For each listed group j: the indexer score of proxy j (rows of pq / pw /
  * pq_scale indexed by j, full [G, ...] arrays) over the prefix [0, e_j],
- * e_j = min(L, (j+1)g) - 1, and its top-C -> cand [ngroups, C]. */
+ * e_j = min(L, (j+1)g) - 1, and its top-C -> cand [ngroups, C]: the top
+ * `topk` by position, then the rest by position. */
 int oracle_proxy_scan(int dtype, int L, int H, int D, const void* pq,
                       const float* pq_scale, const float* pw, const void* k,
-                      const float* k_scale, int g, int C, int ngroups,
+                      const float* k_scale, int g, int C, int topk, int ngroups,
                       const int32_t* groups, int32_t* cand, double* cand_score,
                       int nthreads) {
     set_threads(nthreads);
@@ -383,7 +411,7 @@ int oracle_proxy_scan(int dtype, int L, int H, int D, const void* pq,
         int e = ((j + 1) * g < L ? (j + 1) * g : L) - 1;
         double* qd = (double*)malloc(sizeof(double) * (size_t)H * D);
         decode_qrow(dtype, pq, pq_scale, (size_t)j, H, D, qd);
-        row_topk_prefix(H, D, qd, pw + (size_t)j * H, kd, e, C,
+        row_topk_prefix(H, D, qd, pw + (size_t)j * H, kd, e, C, topk,
                         cand + (size_t)r * C, cand_score ? cand_score + (size_t)r * C : NULL);
         free(qd);
     }
@@ -396,8 +424,8 @@ int oracle_proxy_scan(int dtype, int L, int H, int D, const void* pq,
 /* ------------------------------------------------------------------------ */
 
 /* Member t of group j = t / g: the first k entries of cand[j] (the proxy's
- * top-k in rank order), keeping only positions <= t in their order, padded
- * with -1.  cand is the full [G, C]; out is [nrows, k]. */
+ * top-k), keeping only positions <= t in their order, padded with -1.
+ * cand is the full [G, C]; out is [nrows, k]. */
 int oracle_reuse(int L, int g, const int32_t* cand, int C, int topk, int nrows,
                  const int32_t* rows, int32_t* out_idx) {
     (void)L;
@@ -463,7 +491,7 @@ int oracle_refine(int dtype, int L, int H, int D, const void* q,
  * cache_len [B] counts the Gm new tokens' keys, already appended.
  * Member m sees [0, cache_len - Gm + m]; the proxy sees [0, cache_len - 1].
  * mode 0 = dense, 1 = Reuse, 2 = Refine.  out_idx [B, Gm, k]; cand_out
- * [B, C] (modes 1, 2; may be NULL).  Sequences are processed one at a time
+ * [B, C] (modes 1, 2; may be NULL), laid out as in the proxy scan.  Sequences are processed one at a time
  * with the same steps as prefill. */
 int oracle_decode(int dtype, int B, int Gm, int H, int D, const void* q,
                   const float* q_scale, const float* w, const void* kc,
@@ -488,7 +516,7 @@ int oracle_decode(int dtype, int B, int Gm, int H, int D, const void* q,
         if (mode == 0) {
             for (int m = 0; m < Gm; ++m) {
                 decode_qrow(dtype, qb, qbs, (size_t)m, H, D, qd);
-                row_topk_prefix(H, D, qd, wb + (size_t)m * H, kd, n - Gm + m, topk,
+                row_topk_prefix(H, D, qd, wb + (size_t)m * H, kd, n - Gm + m, topk, 0,
                                 ob + (size_t)m * topk, osb ? osb + (size_t)m * topk : NULL);
             }
         } else {
@@ -498,7 +526,7 @@ int oracle_decode(int dtype, int B, int Gm, int H, int D, const void* q,
             int32_t* cand = (int32_t*)malloc(sizeof(int32_t) * C);
             proxy_one(dtype, H, D, qb, qbs, wb, 0, Gm, pq, &pqs, pw);
             decode_qrow(dtype, pq, dtype == OR_E4M3 ? &pqs : NULL, 0, H, D, qd);
-            row_topk_prefix(H, D, qd, pw, kd, n - 1, C, cand, NULL);
+            row_topk_prefix(H, D, qd, pw, kd, n - 1, C, topk, cand, NULL);
             if (cand_out) memcpy(cand_out + (size_t)b * C, cand, sizeof(int32_t) * C);
             for (int m = 0; m < Gm; ++m) {
                 int lim = n - Gm + m;

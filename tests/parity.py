@@ -6,7 +6,8 @@ Comparison rules (the indexer returns positions in rank order):
   rows must be identical, order and -1 padding included;
 * real-valued inputs: GPU scores accumulate in fp32 (tensor cores) while the
   oracle is fp64, so rows may differ only at the selection boundary.  With
-  s_k the oracle's k-th score and tol = 1e-3 * |s_k|: every position the GPU
+  s_k the oracle's k-th score (the lowest selected one; rows list positions
+  in ascending order) and tol = 1e-3 * |s_k|: every position the GPU
   picked that the oracle did not must score >= s_k - tol (by the oracle),
   and every position the oracle picked that the GPU did not must score
   <= s_k + tol; GPU scores must be within tol of the oracle's.
@@ -56,7 +57,7 @@ def assert_rows_close(gpu_idx, ref_idx, ref_scores, score_fn, rows, what="", gpu
         assert len(g) == len(o), f"{what} row {r}: gpu picked {len(g)}, oracle {len(o)}"
         if not o:
             continue
-        sk = ref_scores[i][len(o) - 1]
+        sk = float(np.min(ref_scores[i][:len(o)]))     # the k-th score: rows are listed by position
         tol = REL_TOL * max(abs(sk), 1e-30) if abs_tol is None else abs_tol(r)
         gs, os_ = set(g), set(o)
         only_g = sorted(gs - os_)

@@ -84,7 +84,9 @@ def test_group_and_candidate_checks(lib):
     seq = _seq()
     assert pv.pivot_proxy_reduce(seq, 0, FAKE, None, FAKE, None) == 1      # g >= 1
     assert pv.pivot_proxy_reduce(seq, 4, FAKE, FAKE, FAKE, None) == 1      # no pq_scale for f32
-    assert pv.pivot_proxy_scan(seq, 4, FAKE, None, FAKE, 0, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_proxy_scan(seq, 4, FAKE, None, FAKE, 0, 1, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_proxy_scan(seq, 4, FAKE, None, FAKE, 8, 9, FAKE, None, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_proxy_scan(seq, 4, FAKE, None, FAKE, 8, 0, FAKE, None, FAKE, 1 << 20, None) == 1
     assert pv.pivot_reuse(0, 64, 4, FAKE, 8, 16, FAKE, None) == 1           # C < k
     assert pv.pivot_reuse(1, 64, 4, FAKE, 16, 8, FAKE, None) == 1           # t_begin % g
     assert pv.pivot_refine(seq, 4, FAKE, 8, 16, FAKE, None, FAKE, 1 << 20, None) == 1

@@ -30,7 +30,7 @@ def _lib():
 def _pivot_gpu(p, dev, g, C, topk, with_score=True):
     seq = seq_of(dev)
     pq, pqs, pw = pv.proxy_reduce(seq, g)
-    cand, cs = pv.proxy_scan(seq, g, pq, pqs, pw, C, with_score=with_score)
+    cand, cs = pv.proxy_scan(seq, g, pq, pqs, pw, C, topk, with_score=with_score)
     reu = pv.reuse(0, p.L, g, cand, topk)
     ref, rs = pv.refine(seq, g, cand, topk, with_score=with_score)
     torch.cuda.synchronize()
@@ -89,7 +89,7 @@ def test_tiny_pivot_exact(tiny):
     pq, pqs, pw, cand, cs, reu, ref, rs = _pivot_gpu(p, dev, g, C, kk)
     q, qs, w, k, ks = p.codes()
     opq, opqs, opw = oracle.proxy_reduce(F32, q, qs, w, g)
-    ocand, ocs = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, p.L, g, C)
+    ocand, ocs = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, p.L, g, C, kk)
     assert_rows_exact(cand.cpu(), ocand, "proxy scan")
     ok = ocand >= 0
     assert (cs.cpu().numpy()[ok] == ocs[ok]).all()
@@ -128,10 +128,52 @@ def test_edge_shapes_exact(L, g, C, kk):
     assert_rows_exact(idx.cpu(), oracle.dense_index(F32, q, qs, w, k, ks, kk)[0], "dense")
     _, _, _, cand, _, reu, ref, _ = _pivot_gpu(p, dev, g, C, kk, with_score=False)
     opq, opqs, opw = oracle.proxy_reduce(F32, q, qs, w, g)
-    ocand, _ = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, L, g, C)
+    ocand, _ = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, L, g, C, kk)
     assert_rows_exact(cand.cpu(), ocand, "cand")
     assert_rows_exact(reu.cpu(), oracle.reuse(L, g, ocand, kk), "reuse")
     assert_rows_exact(ref.cpu(), oracle.refine(F32, q, qs, w, k, ks, g, ocand, kk)[0], "refine")
+
+
+def test_long_rows_exact():
+    """Rows longer than the selection's kept-entry buffer (2048 for k <= 1024)
+    take the sampled-threshold path; integer scores keep it bit-exact, ties
+    included."""
+    L, g, C, kk = 6000, 4, 1100, 100
+    p = gen.make_prefill(L, 4, 32, F32, kind="int", seed=77)
+    dev = to_device(p)
+    q, qs, w, k, ks = p.codes()
+    rows = np.array(sorted(set(np.linspace(2048, L - 1, 48).astype(int)) | {L - 1}))
+    idx, sc = pv.dense_index(seq_of(dev), kk, with_score=True)
+    oidx, osc = oracle.dense_index(F32, q, qs, w, k, ks, kk, rows=rows)
+    assert_rows_exact(idx.cpu().numpy()[rows], oidx, "dense long rows")
+    assert (sc.cpu().numpy()[rows] == osc).all()
+    _, _, _, cand, _, reu, ref, _ = _pivot_gpu(p, dev, g, C, kk, with_score=False)
+    opq, opqs, opw = oracle.proxy_reduce(F32, q, qs, w, g)
+    groups = np.array(sorted(set(np.linspace(600, L // g - 1, 32).astype(int))))
+    ocand, _ = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, L, g, C, kk, groups=groups)
+    assert_rows_exact(cand.cpu().numpy()[groups], ocand, "cand long rows")
+    gc = cand.cpu().numpy()
+    assert_rows_exact(ref.cpu().numpy()[rows], oracle.refine(F32, q, qs, w, k, ks, g, gc, kk,
+                                                             rows=rows)[0], "refine")
+
+
+@pytest.mark.parametrize("dtype", [BF16, E4M3])
+def test_dsa_long_rows_within_tolerance(dtype):
+    L, H, D, g, C, kk = 9000, 64, 128, 8, 2600, 300
+    p = gen.make_prefill(L, H, D, dtype, kind="dsa", seed=8)
+    dev = to_device(p)
+    q, qs, w, k, ks = p.codes()
+    rows = np.array(sorted(set(np.linspace(2100, L - 1, 24).astype(int))))
+    idx, sc = pv.dense_index(seq_of(dev), kk, with_score=True)
+    oidx, osc = oracle.dense_index(dtype, q, qs, w, k, ks, kk, rows=rows)
+    assert_rows_close(idx.cpu().numpy()[rows], oidx, osc, score_fn_for(p), rows, "dense",
+                      gpu_scores=sc.cpu().numpy()[rows])
+    pq, pqs, pw, cand, cs, reu, ref, rs = _pivot_gpu(p, dev, g, C, kk)
+    opq, opqs, opw = oracle.proxy_reduce(dtype, q, qs, w, g)
+    groups = np.array(sorted(set(np.linspace(700, L // g - 1, 16).astype(int))))
+    ocand, ocs = oracle.proxy_scan(dtype, opq, opqs, opw, k, ks, L, g, C, kk, groups=groups)
+    assert_rows_close(cand.cpu().numpy()[groups], ocand, ocs, proxy_score_fn(p, opq, opqs, opw),
+                      groups, "cand", gpu_scores=cs.cpu().numpy()[groups])
 
 
 @pytest.mark.parametrize("L,g,C,kk", [(300, 5, 64, 64), (515, 3, 40, 9)])
@@ -147,7 +189,7 @@ def test_edge_shapes_odd_groups(L, g, C, kk):
     opq, opqs, opw = oracle.proxy_reduce(F32, q, qs, w, g)
     assert (pq.cpu().numpy() == opq).all() and (pw.cpu().numpy() == opw).all()
     groups = np.arange(opq.shape[0])
-    ocand, ocs = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, L, g, C)
+    ocand, ocs = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, L, g, C, kk)
     assert_rows_close(cand.cpu().numpy(), ocand, ocs, proxy_score_fn(p, opq, opqs, opw), groups,
                       "cand", gpu_scores=cs.cpu().numpy(), abs_tol=tf32_abs_tol(opq, opw, k))
     gc = cand.cpu().numpy()
@@ -170,7 +212,7 @@ def test_row_ranges_and_small_workspace_match_one_call(tiny):
     _, _, _, cand, _, reu, ref, _ = _pivot_gpu(p, dev, g, C, kk, with_score=False)
     seq2 = seq_of(dev, 512, 1024)
     pq, pqs, pw = pv.proxy_reduce(seq2, g)
-    cand2, _ = pv.proxy_scan(seq2, g, pq, pqs, pw, C)
+    cand2, _ = pv.proxy_scan(seq2, g, pq, pqs, pw, C, kk)
     assert torch.equal(cand2, cand[512 // g:])
     ref2, _ = pv.refine(seq2, g, cand2, kk)
     assert torch.equal(ref2, ref[512:])
@@ -192,7 +234,7 @@ def test_zigzag_sharded_calls_match_one_call(tiny, world):
             d, _ = pv.dense_index(seq, kk)
             assert torch.equal(d, full_dense[a:b])
             pq, pqs, pw = pv.proxy_reduce(seq, g)
-            cand, _ = pv.proxy_scan(seq, g, pq, pqs, pw, C)
+            cand, _ = pv.proxy_scan(seq, g, pq, pqs, pw, C, kk)
             assert torch.equal(cand, full_cand[a // g:-(-b // g)])
             assert torch.equal(pv.reuse(a, b, g, cand, kk), full_reu[a:b])
             r, _ = pv.refine(seq, g, cand, kk)
@@ -220,7 +262,7 @@ def test_dsa_small_within_tolerance(dtype):
     opq, opqs, opw = oracle.proxy_reduce(dtype, q, qs, w, g)
     G = opq.shape[0]
     groups = np.array(sorted(set(np.linspace(0, G - 1, 24).astype(int))))
-    ocand, ocs = oracle.proxy_scan(dtype, opq, opqs, opw, k, ks, L, g, C, groups=groups)
+    ocand, ocs = oracle.proxy_scan(dtype, opq, opqs, opw, k, ks, L, g, C, kk, groups=groups)
     pfn = proxy_score_fn(p, opq, opqs, opw)
     assert_rows_close(cand.cpu().numpy()[groups], ocand, ocs, pfn, groups, "cand",
                       gpu_scores=cs.cpu().numpy()[groups])

@@ -78,6 +78,11 @@ def test_derived_example_decode(golden_dir):
         assert idx[0, 1].tolist() == ex[key]["7"], key
         if mode != oracle.DENSE and C == ex["C"]:
             assert cand[0].tolist() == ex["candidates"]
+    sp = ex["split_case"]
+    for mode, key in [(oracle.REUSE, "reuse"), (oracle.REFINE, "refine")]:
+        idx, cand, _ = oracle.decode(F32, q, None, w, kc, None, cl, mode, sp["C"], sp["topk"])
+        assert cand[0].tolist() == sp["candidates"]
+        assert idx[0, 0].tolist() == sp[key]["6"] and idx[0, 1].tolist() == sp[key]["7"], key
 
 
 def test_derived_example_prefill(golden_dir):
@@ -92,12 +97,19 @@ def test_derived_example_prefill(golden_dir):
     assert pq[3, 0].tolist() == ex["proxy_query"]
     sc = oracle.score_positions(F32, pq, None, pw, k, None, 3, np.arange(8))
     assert sc.tolist() == ex["proxy_scores"]
-    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, ex["C"])
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, ex["C"], ex["topk"])
     assert cand[3].tolist() == ex["candidates"]
     reuse = oracle.reuse(L, g, cand, 3, rows=[6, 7])
     assert reuse.tolist() == [ex["reuse"]["6"], ex["reuse"]["7"]]
     ref, _ = oracle.refine(F32, q, None, w, k, None, g, cand, 3, rows=[6, 7])
     assert ref.tolist() == [ex["refine"]["6"], ex["refine"]["7"]]
+    sp = ex["split_case"]
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, sp["C"], sp["topk"])
+    assert cand[3].tolist() == sp["candidates"]
+    assert oracle.reuse(L, g, cand, sp["topk"], rows=[6, 7]).tolist() == \
+        [sp["reuse"]["6"], sp["reuse"]["7"]]
+    ref, _ = oracle.refine(F32, q, None, w, k, None, g, cand, sp["topk"], rows=[6, 7])
+    assert ref.tolist() == [sp["refine"]["6"], sp["refine"]["7"]]
 
 
 # ---------------------------------------------------------------------------
@@ -117,9 +129,9 @@ def test_relu_and_head_weights_closed_form():
     k = np.array([[2, 0], [-3, 0], [0, 5]], dtype=np.float32)
     sc = oracle.score_positions(F32, q, None, w, k, None, 2, [0, 1, 2])
     assert sc.tolist() == [2.0, 6.0, 0.0]
-    idx, s = oracle.dense_index(F32, q, None, w, k, None, 3, rows=[2])
-    assert idx[0].tolist() == [1, 0, 2]
-    assert s[0].tolist() == [6.0, 2.0, 0.0]
+    idx, s = oracle.dense_index(F32, q, None, w, k, None, 2, rows=[2])
+    assert idx[0].tolist() == [0, 1]                 # the two best, listed by position
+    assert s[0].tolist() == [2.0, 6.0]
 
 
 def test_scales_multiply_the_dot_product():
@@ -164,7 +176,7 @@ def test_single_head_nonnegative_is_plain_inner_product_topk():
     S = q[:, 0, :].astype(np.float64) @ k.astype(np.float64).T     # [t, s]
     for t in range(L):
         pos = np.arange(t + 1)
-        order = np.lexsort((pos, -S[t, : t + 1]))[:kk]
+        order = np.sort(np.lexsort((pos, -S[t, : t + 1]))[:kk])   # top-k, listed by position
         want = list(pos[order]) + [-1] * (kk - len(order))
         assert idx[t].tolist() == want, t
         np.testing.assert_allclose(s[t, : len(order)], S[t, order], rtol=1e-12)
@@ -302,7 +314,7 @@ def test_proxy_scan_is_dense_on_the_proxies_at_group_ends():
     L, g, C = 45, 4, 9
     q, _, w, k, _ = _int_case(L)
     pq, _, pw = oracle.proxy_reduce(F32, q, None, w, g)
-    cand, cs = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, C)
+    cand, cs = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, C, C)
     # a sequence whose row e_j is proxy j
     q2, w2 = q.copy(), w.copy()
     ends = [min(L, (j + 1) * g) - 1 for j in range(pq.shape[0])]
@@ -317,7 +329,7 @@ def test_group_of_one_is_dense():
     q, _, w, k, _ = _int_case(L)
     dense, _ = oracle.dense_index(F32, q, None, w, k, None, kk)
     pq, _, pw = oracle.proxy_reduce(F32, q, None, w, 1)
-    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, 1, kk + 3)
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, 1, kk + 3, kk)
     assert (oracle.reuse(L, 1, cand, kk) == dense).all()
     ref, _ = oracle.refine(F32, q, None, w, k, None, 1, cand, kk)
     assert (ref == dense).all()
@@ -328,7 +340,7 @@ def test_refine_over_the_whole_prefix_is_dense():
     q, _, w, k, _ = _int_case(L)
     dense, ds = oracle.dense_index(F32, q, None, w, k, None, kk)
     pq, _, pw = oracle.proxy_reduce(F32, q, None, w, g)
-    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, L)
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, L, kk)
     ref, rs = oracle.refine(F32, q, None, w, k, None, g, cand, kk)
     assert (ref == dense).all() and (rs == ds).all()
 
@@ -338,7 +350,7 @@ def test_reuse_refine_inside_candidates_and_recall_identity():
     q, _, w, k, _ = _int_case(L, H=4, D=8, seed=33)
     dense, _ = oracle.dense_index(F32, q, None, w, k, None, kk)
     pq, _, pw = oracle.proxy_reduce(F32, q, None, w, g)
-    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, C)
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, C, kk)
     reu = oracle.reuse(L, g, cand, kk)
     ref, _ = oracle.refine(F32, q, None, w, k, None, g, cand, kk)
     for t in range(L):
@@ -348,8 +360,15 @@ def test_reuse_refine_inside_candidates_and_recall_identity():
         ds = set(x for x in dense[t] if x >= 0)
         assert rs <= cset and fs <= cset
         assert all(x <= t for x in rs | fs)
-        # reuse keeps the proxy's rank order
+        # Reuse keeps the proxy's top-k (the candidate row's first k) in order
         assert [x for x in reu[t] if x >= 0] == [x for x in cand[t // g][:kk] if 0 <= x <= t]
+        # every index row is listed by position
+        for row in (reu[t], ref[t], dense[t]):
+            vals = [x for x in row if x >= 0]
+            assert vals == sorted(vals)
+        # the candidate row: the proxy's top-k ascending, then the rest ascending
+        cj = [x for x in cand[t // g] if x >= 0]
+        assert cj[:kk] == sorted(cj[:kk]) and cj[kk:] == sorted(cj[kk:])
         # Refine keeps exactly the dense picks that are candidates (unique scores
         # are not guaranteed on integer inputs, so compare through the scores)
         assert len(fs) == min(kk, len(cset))
@@ -367,7 +386,7 @@ def test_decode_equals_last_prefill_group():
     kc = k[None]
     cl = np.array([n], dtype=np.int32)
     pq, _, pw = oracle.proxy_reduce(F32, q, None, w, 2)
-    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, n, 2, C)
+    cand, _ = oracle.proxy_scan(F32, pq, None, pw, k, None, n, 2, C, kk)
     want = {
         oracle.DENSE: oracle.dense_index(F32, q, None, w, k, None, kk, rows=[n - 2, n - 1])[0],
         oracle.REUSE: oracle.reuse(n, 2, cand, kk, rows=[n - 2, n - 1]),

@@ -209,9 +209,11 @@ int rows_per_block(int H, int D, int dtype) {
 
 pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, int Gm, int maxlen,
                                  const int32_t* cache_len, const float* S, long long stride,
-                                 int K, int32_t* out, float* out_score, int out_base,
-                                 cudaStream_t st) {
+                                 int K, int split, int npos, int32_t* out, float* out_score,
+                                 int out_base, cudaStream_t st) {
     SelectParams sp{};
+    sp.split = split;
+    sp.npos = npos;
     sp.kind = SEL_PREFIX;
     sp.scan_kind = scan_kind;
     sp.row0 = r0;
@@ -234,9 +236,10 @@ pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, in
 
 pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int Gm, int maxlen,
                                const int32_t* cache_len, const float* S, const int32_t* cand,
-                               int cand_base, int C, int K, int32_t* out, float* out_score,
-                               int out_base, cudaStream_t st) {
+                               int cand_base, int C, int K, int npos, int32_t* out,
+                               float* out_score, int out_base, cudaStream_t st) {
     SelectParams sp{};
+    sp.npos = npos;
     sp.kind = SEL_CANDIDATES;
     sp.scan_kind = scan_kind;
     sp.row0 = r0;
@@ -261,10 +264,55 @@ pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int 
 }
 
 pivot_status_t run_refine_scores(int kind, int dtype, int H, int D, const void* q,
-                                 int qrow_base, const float* q_scale, const float* w,
-                                 const void* k, const float* k_scale, int L, int g, int Gm,
-                                 int maxlen, const int32_t* cache_len, const int32_t* cand,
-                                 int cand_base, int C, int r0, int r1, float* S, cudaStream_t st) {
+                                 long long q_rows, int qrow_base, const float* q_scale,
+                                 const float* w, const void* k, long long k_rows,
+                                 const float* k_scale, int L, int g, int Gm, int maxlen,
+                                 const int32_t* cache_len, const int32_t* cand, int cand_base,
+                                 int C, int r0, int r1, float* S, cudaStream_t st) {
+    const double work = kind == SCAN_PREFILL_DENSE ? refine_pairs(r0, r1, C) : 0.0;
+    const int gsize = kind == SCAN_DECODE_DENSE ? Gm : g;
+    int P = umma_shape_ok(H, D, dtype) ? 256 / H : 0;
+    if (P > gsize) P = gsize;
+    const int N = P * H;
+    if (P > 0 && N >= 16 && N <= 256 && N % 16 == 0) {
+        // tensor cores: candidate keys gathered with TMA
+        ScanParams p{};
+        p.kind = kind;
+        p.dtype = dtype;
+        p.esize = esize_of(dtype);
+        p.H = H;
+        p.D = D;
+        p.P = P;
+        p.row0 = r0;
+        p.nrows = r1 - r0;
+        p.qrow_base = qrow_base;
+        p.L = L;
+        p.g = g;
+        p.Gm = Gm;
+        p.maxlen = maxlen;
+        p.cache_len = cache_len;
+        p.w = w;
+        p.q_scale = q_scale;
+        p.k_scale = k_scale;
+        p.S = S;
+        p.S_stride = C;
+        p.cand = cand;
+        p.cand_base = cand_base;
+        p.C = C;
+        p.gsize = gsize;
+        p.nkeys = kind == SCAN_DECODE_DENSE ? maxlen : L;
+        p.tiles_per_item = ceil_div(C, 128);
+        p.items_per_block = ceil_div(gsize, P);
+        const int ngroups = (r1 - 1) / gsize - cand_base + 1;
+        p.nitems = ngroups * p.items_per_block;
+        p.kbase = k;
+        (void)k_rows;
+        CUtensorMap tq;
+        if (!make_tmap(&tq, dtype, q, q_rows * H, D, N)) return PIVOT_ERR_CUDA;
+        const int grid = p.nitems < num_sms() ? p.nitems : num_sms();
+        return from_cuda(profiled(PK_REFINE, work, st,
+                                  [&] { return launch_refine_umma(tq, p, grid, st); }));
+    }
     RefineParams rp{};
     rp.dtype = dtype;
     rp.esize = esize_of(dtype);
@@ -288,7 +336,6 @@ pivot_status_t run_refine_scores(int kind, int dtype, int H, int D, const void* 
     rp.cand_base = cand_base;
     rp.C = C;
     rp.S = S;
-    const double work = kind == SCAN_PREFILL_DENSE ? refine_pairs(r0, r1, C) : 0.0;
     return from_cuda(profiled(PK_REFINE, work, st, [&] { return launch_refine_simt(rp, st); }));
 }
 
@@ -406,7 +453,7 @@ pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* 
                       r1, r1 - 1, S, stride, s);
         if (st != PIVOT_OK) return st;
         st = run_select_prefix(SCAN_PREFILL_DENSE, r0, r1, seq->L, 1, 1, 0, nullptr, S, stride,
-                               topk, idx, score, t0, s);
+                               topk, 0, seq->L, idx, score, t0, s);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;
@@ -455,13 +502,15 @@ size_t pivot_proxy_scan_workspace_size(const pivot_seq_t* seq, int32_t g, int32_
 }
 
 pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* pq,
-                                 const float* pq_scale, const float* pw, int32_t C, int32_t* cand,
-                                 float* cand_score, void* ws, size_t ws_bytes, void* stream) {
+                                 const float* pq_scale, const float* pw, int32_t C, int32_t topk,
+                                 int32_t* cand, float* cand_score, void* ws, size_t ws_bytes,
+                                 void* stream) {
     int t0, t1;
     pivot_status_t st = check_seq(seq, &t0, &t1);
     if (st != PIVOT_OK) return st;
     if ((st = check_group_range(seq, g, t0, t1)) != PIVOT_OK) return st;
     if (!pq || !pw || !cand || !aligned16(pq) || C < 1) return PIVOT_ERR_INVALID_ARG;
+    if (topk < 1 || topk > C) return PIVOT_ERR_INVALID_ARG;
     if ((seq->dtype == PIVOT_E4M3) != (pq_scale != nullptr)) return PIVOT_ERR_INVALID_ARG;
     if (C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
@@ -482,7 +531,7 @@ pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* p
                       stride, s);
         if (st != PIVOT_OK) return st;
         st = run_select_prefix(SCAN_PREFILL_PROXY, r0, r1, seq->L, g, 1, 0, nullptr, S, stride, C,
-                               cand, cand_score, j0, s);
+                               topk, seq->L, cand, cand_score, j0, s);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;
@@ -531,12 +580,12 @@ pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* ca
         const int r0 = (int)c0;
         const int r1 = (int)(c0 + chunk < t1 ? c0 + chunk : t1);
         const int jc = r0 / g;
-        st = run_refine_scores(SCAN_PREFILL_DENSE, seq->dtype, seq->H, seq->D, seq->q, 0,
-                               seq->q_scale, seq->w, seq->k, seq->k_scale, seq->L, g, 1, 0,
-                               nullptr, cand + (size_t)(jc - j0) * C, jc, C, r0, r1, S, s);
+        st = run_refine_scores(SCAN_PREFILL_DENSE, seq->dtype, seq->H, seq->D, seq->q, seq->L, 0,
+                               seq->q_scale, seq->w, seq->k, seq->L, seq->k_scale, seq->L, g, 1,
+                               0, nullptr, cand + (size_t)(jc - j0) * C, jc, C, r0, r1, S, s);
         if (st != PIVOT_OK) return st;
         st = run_select_cand(SCAN_PREFILL_DENSE, r0, r1, seq->L, g, 1, 0, nullptr, S,
-                             cand + (size_t)(jc - j0) * C, jc, C, topk, idx, score, t0, s);
+                             cand + (size_t)(jc - j0) * C, jc, C, topk, seq->L, idx, score, t0, s);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;
@@ -615,7 +664,7 @@ pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, in
                       b->maxlen - 1, w.S, stride, s);
         if (st != PIVOT_OK) return st;
         return run_select_prefix(SCAN_DECODE_DENSE, 0, rows, 0, 1, b->Gm, b->maxlen, b->cache_len,
-                                 w.S, stride, topk, idx, nullptr, 0, s);
+                                 w.S, stride, topk, 0, b->maxlen, idx, nullptr, 0, s);
     }
     // proxy of each sequence's Gm new tokens
     ReduceParams rp{};
@@ -641,7 +690,7 @@ pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, in
                   b->maxlen, b->cache_len, 1, 0, b->B, b->maxlen - 1, w.S, stride, s);
     if (st != PIVOT_OK) return st;
     st = run_select_prefix(SCAN_DECODE_PROXY, 0, b->B, 0, 1, b->Gm, b->maxlen, b->cache_len, w.S,
-                           stride, C, w.cand, nullptr, 0, s);
+                           stride, C, topk, b->maxlen, w.cand, nullptr, 0, s);
     if (st != PIVOT_OK) return st;
     if (cand)
         if (cudaMemcpyAsync(cand, w.cand, (size_t)b->B * C * 4, cudaMemcpyDeviceToDevice, s) !=
@@ -652,12 +701,12 @@ pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, in
             return launch_decode_reuse(b->B, b->Gm, b->maxlen, b->cache_len, w.cand, C, topk, idx, s);
         }));
     const int rows = b->B * b->Gm;
-    st = run_refine_scores(SCAN_DECODE_DENSE, b->dtype, b->H, b->D, b->q, 0, b->q_scale, b->w,
-                           b->kc, b->kc_scale, 0, 1, b->Gm, b->maxlen, b->cache_len, w.cand, 0, C,
-                           0, rows, w.R, s);
+    st = run_refine_scores(SCAN_DECODE_DENSE, b->dtype, b->H, b->D, b->q, rows, 0, b->q_scale,
+                           b->w, b->kc, krows, b->kc_scale, 0, 1, b->Gm, b->maxlen, b->cache_len,
+                           w.cand, 0, C, 0, rows, w.R, s);
     if (st != PIVOT_OK) return st;
     return run_select_cand(SCAN_DECODE_DENSE, 0, rows, 0, 1, b->Gm, b->maxlen, b->cache_len, w.R,
-                           w.cand, 0, C, topk, idx, nullptr, 0, s);
+                           w.cand, 0, C, topk, b->maxlen, idx, nullptr, 0, s);
 }
 
 }  // extern "C"

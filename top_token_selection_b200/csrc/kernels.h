@@ -33,6 +33,12 @@ struct ScanParams {
     float* S;               // scores of row r at S + (r - row0)*S_stride + s
     long long S_stride;
     int tiles_per_item, items_per_block, nitems;
+    // gather mode (Refine): member rows score the candidate keys of their group
+    const int32_t* cand;    // group rows at cand + (grp - cand_base)*C
+    int cand_base, C;
+    int gsize;              // members per group (g in prefill, Gm in decode)
+    int nkeys;              // key positions per sequence (L, or maxlen in decode)
+    const void* kbase;      // gather mode: key rows (stored format), row stride D*esize
 };
 
 int scan_smem_bytes(int row_bytes);
@@ -42,8 +48,8 @@ cudaError_t launch_scan_simt(const void* q, const void* k, const ScanParams& p,
                              cudaStream_t stream);
 
 // Row selection: for each row, the top-K entries by (score desc, position
-// asc) among the row's valid entries, written in rank order with -1 / -inf
-// padding.
+// asc) among the row's valid entries, written in ascending position order
+// (with `split`, the top `split` first, then the rest) with -1 / -inf padding.
 enum SelectKind {
     SEL_PREFIX = 0,      // row r: entries 0..lim(r) of S, position = entry index
     SEL_CANDIDATES = 1,  // row r: C entries, position = cand[grp(r)][i], valid iff 0 <= pos <= lim(r)
@@ -64,6 +70,10 @@ struct SelectParams {
     float* out_score;     // or NULL
     int out_base;
     int tail_cap;         // capacity of the boundary buffer (entries)
+    int split;            // > 0: list the top `split` first, then the rest (each by position)
+    int npos;             // positions are < npos (bitmap size)
+    int fast_cap;         // set by launch_select: kept-entry capacity of the fast path
+    int bitmap_words;     // set by launch_select
 };
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
@@ -108,6 +118,11 @@ struct RefineParams {
     float* S;              // row r at S + (r - row0)*C
 };
 cudaError_t launch_refine_simt(const RefineParams& p, cudaStream_t stream);
+// Refine scores on the tensor cores: candidate keys gathered from p.kbase
+// with cp.async, member queries from tmap_q.  p.kind is SCAN_PREFILL_DENSE
+// or SCAN_DECODE_DENSE (member rows); S rows have C entries.
+cudaError_t launch_refine_umma(const CUtensorMap& tmap_q, const ScanParams& p, int grid,
+                               cudaStream_t stream);
 
 cudaError_t launch_wait_selftest(cudaStream_t stream);
 

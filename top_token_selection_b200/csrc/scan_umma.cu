@@ -1,12 +1,18 @@
 // scan_umma.cu -- indexer scores on the 5th-generation tensor cores.
 //
-// Computes, for a block of P query rows (queries, or proxy queries) that
-// share one key sequence, the indexer score of every key of the causal
-// prefix:
+// Computes, for a block of P query rows (queries, proxy queries, or the
+// members of one group) the indexer score against a stream of keys:
 //     I(r, s) = sum_h w[r,h] * ReLU(q[r,h] . k[s])      (x q_scale * k_scale)
-// (dense indexer of "Sparse Attention의 Indexer", Fig. 1-2, in the multi-head
-// form; the same scan serves the PIVOT proxy scan of the abstract of arXiv
-// 2607.24593, run once per group with the proxy as the query).
+// (the dense indexer of "Sparse Attention의 Indexer", Fig. 1-2, in its
+// multi-head form).  Two modes share one kernel:
+//  * scan   -- keys 0..lim of the causal prefix, contiguous, loaded with tiled
+//              TMA: the dense indexer, and the PIVOT proxy scan (abstract of
+//              arXiv 2607.24593: one full-prefix scan per group, run with the
+//              proxy as the query);
+//  * gather -- the C candidate keys of the group, gathered row by row with
+//              16-byte cp.async into the swizzled tile: PIVOT-Refine (same
+//              abstract: every member re-scores the candidate set with its
+//              own query).
 //
 // Mapping: keys on the MMA M axis (128 TMEM lanes), the P*H query heads on
 // N (<= 256 columns).  Each epilogue thread owns one key and reduces its
@@ -15,8 +21,9 @@
 // through a TMA ring.  Accumulators are double-buffered in TMEM (2 x 256
 // columns) so the epilogue of tile i overlaps the MMAs of tile i+1.
 //
-// Warp roles (192 threads): warp 0 issues TMA, warp 1 allocates TMEM and
-// issues tcgen05.mma, warps 2-5 run the epilogue.
+// Warp roles (192 threads): warp 0 loads (one lane issuing TMA in scan mode;
+// all 32 lanes copying in gather mode), warp 1 allocates TMEM and issues
+// tcgen05.mma, warps 2-5 run the epilogue.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -52,35 +59,58 @@ __device__ __forceinline__ int scan_key_base(const ScanParams& p, int r) {
 }
 
 struct ItemInfo {
-    int blk, rows, row_first, t0, t1, keybase, maxlim;
+    int rows, row_first, t0, t1, keybase, maxlim;
+    const int32_t* cand;   // gather mode: this group's candidate row
     bool valid;
 };
 
-// Work item i = (row block, chunk of key tiles).  Items whose chunk starts
-// beyond the block's causal extent are empty.  Every role walks the same
-// item sequence.
+// Scan mode: item i = (row block, chunk of key tiles); items whose chunk
+// starts beyond the block's causal extent are empty.
+// Gather mode: item i = (group, block of that group's member rows); the
+// tiles cover the C candidates.  Every role walks the same item sequence.
+template <bool GATHER>
 __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
     ItemInfo it;
-    it.blk = item / p.items_per_block;
-    int chunk = item % p.items_per_block;
-    it.row_first = p.row0 + it.blk * p.P;
-    int rows = p.row0 + p.nrows - it.row_first;
-    it.rows = rows < p.P ? rows : p.P;
-    bool ok;
-    int maxlim = scan_row_lim(p, it.row_first + it.rows - 1, ok);
-    it.maxlim = ok ? maxlim : -1;
-    it.keybase = scan_key_base(p, it.row_first);
-    int nt = ok ? (maxlim + 1 + 127) / 128 : 0;
-    it.t0 = chunk * p.tiles_per_item;
-    it.t1 = it.t0 + p.tiles_per_item < nt ? it.t0 + p.tiles_per_item : nt;
-    it.valid = it.t0 < nt;
+    if constexpr (!GATHER) {
+        const int blk = item / p.items_per_block;
+        const int chunk = item % p.items_per_block;
+        it.row_first = p.row0 + blk * p.P;
+        const int rows = p.row0 + p.nrows - it.row_first;
+        it.rows = rows < p.P ? rows : p.P;
+        bool ok;
+        const int maxlim = scan_row_lim(p, it.row_first + it.rows - 1, ok);
+        it.maxlim = ok ? maxlim : -1;
+        it.keybase = scan_key_base(p, it.row_first);
+        const int nt = ok ? (maxlim + 1 + 127) / 128 : 0;
+        it.t0 = chunk * p.tiles_per_item;
+        it.t1 = it.t0 + p.tiles_per_item < nt ? it.t0 + p.tiles_per_item : nt;
+        it.valid = it.t0 < nt;
+        it.cand = nullptr;
+    } else {
+        const int grp = p.cand_base + item / p.items_per_block;
+        const int mb = item % p.items_per_block;
+        const int gstart = grp * p.gsize;
+        int first = gstart + mb * p.P;
+        int end = first + p.P;
+        if (end > gstart + p.gsize) end = gstart + p.gsize;
+        if (first < p.row0) first = p.row0;
+        if (end > p.row0 + p.nrows) end = p.row0 + p.nrows;
+        it.row_first = first;
+        it.rows = end - first;
+        it.keybase = p.kind == SCAN_DECODE_DENSE ? grp * p.maxlen : 0;
+        it.maxlim = p.nkeys - 1;
+        it.t0 = 0;
+        it.t1 = (p.C + 127) / 128;
+        it.valid = it.rows > 0;
+        it.cand = p.cand + (size_t)(grp - p.cand_base) * p.C;
+    }
     return it;
 }
 
-template <int KIND, int HEADS, int ROWB>
+template <int KIND, int HEADS, int ROWB, bool GATHER>
 __global__ void __launch_bounds__(192, 1)
-    scan_umma_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                     const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
+    index_umma_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                      const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
     constexpr int KBLK = ROWB / 128;           // 128-byte K blocks per row
     constexpr int KSTEPS = ROWB / 32;          // one MMA consumes 32 bytes of K
     constexpr int A_BYTES = 128 * ROWB;        // one key tile
@@ -137,45 +167,124 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem_base = *tmem_holder;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA
-        if (lane == 0) {
+        // ------------------------------------------------------- producer
+        if constexpr (!GATHER) {
+            // Scan mode: lane 0 streams contiguous key tiles with tiled TMA.
+            if (lane == 0) {
+                int stage = 0;
+                uint32_t phase = 0;
+                int nit = 0;
+                // parity of the last load issued per stage / query slot (-1:
+                // none), so every load can be waited for before the CTA exits
+                int last_a[STAGES], last_b[2] = {-1, -1};
+                for (int i = 0; i < STAGES; ++i) last_a[i] = -1;
+                bool aborted = false;
+                for (int item = blockIdx.x; item < p.nitems && !aborted; item += gridDim.x) {
+                    ItemInfo it = scan_item<GATHER>(p, item);
+                    if (!it.valid) continue;
+                    const int slot = nit & 1;
+                    const uint32_t bph = (nit >> 1) & 1;
+                    if (!mbar_wait(&bempty[slot], bph ^ 1)) { aborted = true; break; }
+                    mbar_arrive_expect_tx(&bfull[slot], (uint32_t)(N * ROWB));
+                    last_b[slot] = (int)bph;
+                    const int qrow = (it.row_first - p.qrow_base) * HEADS;
+                    for (int kb = 0; kb < KBLK; ++kb)
+                        tma_load_2d(sB + slot * B_SLOT + kb * (N * 128), &tmap_q, &bfull[slot],
+                                    kb * (128 / p.esize), qrow);
+                    for (int t = it.t0; t < it.t1; ++t) {
+                        if (!mbar_wait(&empty[stage], phase ^ 1)) { aborted = true; break; }
+                        mbar_arrive_expect_tx(&full[stage], (uint32_t)A_BYTES);
+                        last_a[stage] = (int)phase;
+                        for (int kb = 0; kb < KBLK; ++kb)
+                            tma_load_2d(sA + stage * A_BYTES + kb * (128 * 128), &tmap_k,
+                                        &full[stage], kb * (128 / p.esize), it.keybase + t * 128);
+                        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    }
+                    ++nit;
+                }
+                // Every load issued lands before the CTA may exit (only the
+                // producer arrives on these barriers, so the last phase stays).
+                for (int i = 0; i < STAGES; ++i)
+                    if (last_a[i] >= 0) mbar_wait(&full[i], (uint32_t)last_a[i]);
+                for (int i = 0; i < 2; ++i)
+                    if (last_b[i] >= 0) mbar_wait(&bfull[i], (uint32_t)last_b[i]);
+            }
+        } else {
+            // Gather mode: the whole warp copies each tile's 128 candidate
+            // key rows with 16-byte cp.async straight into the swizzled tile
+            // layout.  A tile is published (full[stage] arrive) once its
+            // copies have landed and been fenced for the tensor cores; up to
+            // GDEPTH tiles are in flight.
+            constexpr int GDEPTH = STAGES > 3 ? 3 : STAGES - 1;
+            static_assert(STAGES > GDEPTH && GDEPTH >= 1, "the ring must outrun the copies");
+            const uint8_t* kbytes = static_cast<const uint8_t*>(p.kbase);
             int stage = 0;
             uint32_t phase = 0;
             int nit = 0;
-            // parity of the last load issued per stage / query slot (-1: none),
-            // so every load can be waited for before the CTA exits
-            int last_a[STAGES], last_b[2] = {-1, -1};
-            for (int i = 0; i < STAGES; ++i) last_a[i] = -1;
+            int pend[GDEPTH] = {0};
+            int npend = 0;
+            int last_b[2] = {-1, -1};
             bool aborted = false;
+            auto publish_oldest = [&]() {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[pend[0]]);
+                for (int i = 1; i < npend; ++i) pend[i - 1] = pend[i];
+                --npend;
+            };
             for (int item = blockIdx.x; item < p.nitems && !aborted; item += gridDim.x) {
-                ItemInfo it = scan_item(p, item);
+                ItemInfo it = scan_item<GATHER>(p, item);
                 if (!it.valid) continue;
                 const int slot = nit & 1;
                 const uint32_t bph = (nit >> 1) & 1;
-                if (!mbar_wait(&bempty[slot], bph ^ 1)) { aborted = true; break; }
-                mbar_arrive_expect_tx(&bfull[slot], (uint32_t)(N * ROWB));
-                last_b[slot] = (int)bph;
-                const int qrow = (it.row_first - p.qrow_base) * HEADS;
-                for (int kb = 0; kb < KBLK; ++kb)
-                    tma_load_2d(sB + slot * B_SLOT + kb * (N * 128), &tmap_q, &bfull[slot],
-                                kb * (128 / p.esize), qrow);
-                for (int t = it.t0; t < it.t1; ++t) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1)) { aborted = true; break; }
-                    mbar_arrive_expect_tx(&full[stage], (uint32_t)A_BYTES);
-                    last_a[stage] = (int)phase;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bempty[slot], bph ^ 1))) {
+                    aborted = true;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bfull[slot], (uint32_t)(N * ROWB));
+                    const int qrow = (it.row_first - p.qrow_base) * HEADS;
                     for (int kb = 0; kb < KBLK; ++kb)
-                        tma_load_2d(sA + stage * A_BYTES + kb * (128 * 128), &tmap_k,
-                                    &full[stage], kb * (128 / p.esize), it.keybase + t * 128);
+                        tma_load_2d(sB + slot * B_SLOT + kb * (N * 128), &tmap_q, &bfull[slot],
+                                    kb * (128 / p.esize), qrow);
+                }
+                last_b[slot] = (int)bph;
+                for (int t = it.t0; t < it.t1; ++t) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1))) {
+                        aborted = true;
+                        break;
+                    }
+                    const uint32_t dst = smem_u32(sA + stage * A_BYTES);
+                    // 32 lanes cover 4 rows x 8 chunks per step; a 128-row
+                    // tile of one 128-byte K block takes 32 steps
+#pragma unroll 4
+                    for (int step = 0; step < 32; ++step) {
+                        const int r = step * 4 + (lane >> 3);
+                        const int c = lane & 7;
+                        const int slot_r = t * 128 + r;
+                        const int pos = slot_r < p.C ? it.cand[slot_r] : -1;
+                        const size_t row = (size_t)(it.keybase + ((pos >= 0 && pos < p.nkeys) ? pos : 0));
+                        const uint8_t* src = kbytes + row * ROWB + c * 16;
+#pragma unroll
+                        for (int kb = 0; kb < KBLK; ++kb)
+                            cp_async16(dst + kb * (128 * 128) + sw128_offset(r, c), src + kb * 128);
+                    }
+                    cp_async_commit();
+                    pend[npend++] = stage;
+                    if (npend == GDEPTH) {
+                        cp_async_wait<GDEPTH - 1>();
+                        publish_oldest();
+                    }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 ++nit;
             }
-            // Every load issued lands before the CTA may exit (only the
-            // producer arrives on these barriers, so the last phase stays).
-            for (int i = 0; i < STAGES; ++i)
-                if (last_a[i] >= 0) mbar_wait(&full[i], (uint32_t)last_a[i]);
-            for (int i = 0; i < 2; ++i)
-                if (last_b[i] >= 0) mbar_wait(&bfull[i], (uint32_t)last_b[i]);
+            // publish (or, after an abort, just land) every tile still in flight
+            cp_async_wait<0>();
+            while (npend > 0) publish_oldest();
+            if (lane == 0)
+                for (int i = 0; i < 2; ++i)
+                    if (last_b[i] >= 0) mbar_wait(&bfull[i], (uint32_t)last_b[i]);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
@@ -186,7 +295,7 @@ __global__ void __launch_bounds__(192, 1)
             int nit = 0, ntile = 0;
             bool aborted = false;
             for (int item = blockIdx.x; item < p.nitems && !aborted; item += gridDim.x) {
-                ItemInfo it = scan_item(p, item);
+                ItemInfo it = scan_item<GATHER>(p, item);
                 if (!it.valid) continue;
                 const int slot = nit & 1;
                 const uint32_t bph = (nit >> 1) & 1;
@@ -231,18 +340,24 @@ __global__ void __launch_bounds__(192, 1)
         // epilogue warps are always reached.
         bool aborted = false;
         for (int item = blockIdx.x; item < p.nitems; item += gridDim.x) {
-            ItemInfo it = scan_item(p, item);
+            ItemInfo it = scan_item<GATHER>(p, item);
             if (!it.valid) continue;
             named_bar_sync(1, 128);
-            for (int i = et; i < N; i += 128) {
+            // The tables span all 256 columns / PMAX rows: a TMEM load covers
+            // 32 columns even when N is 16, and the columns past N must map
+            // to masked rows (lim -1) with zero weights.
+            for (int i = et; i < 256; i += 128) {
                 const int pr = i / HEADS;
-                w_s[i] = pr < it.rows
+                w_s[i] = (i < N && pr < it.rows)
                              ? p.w[(size_t)(it.row_first + pr - p.qrow_base) * HEADS + i % HEADS]
                              : 0.0f;
             }
-            for (int pr = et; pr < p.P; pr += 128) {
+            for (int pr = et; pr < PMAX; pr += 128) {
                 bool ok = true;
-                int lim = pr < it.rows ? scan_row_lim(p, it.row_first + pr, ok) : -1;
+                int lim = -1;
+                // gather mode: every candidate slot is written (the selection
+                // drops empty slots and positions after the member)
+                if (pr < it.rows) lim = GATHER ? 0x7fffffff : scan_row_lim(p, it.row_first + pr, ok);
                 lim_s[pr] = ok ? lim : -1;
                 sq_s[pr] = (p.q_scale && pr < it.rows)
                                ? p.q_scale[it.row_first + pr - p.qrow_base]
@@ -257,9 +372,18 @@ __global__ void __launch_bounds__(192, 1)
                 const bool got = mbar_wait(&accfull[acc], aph);
                 if (!__all_sync(0xffffffffu, got)) { aborted = true; continue; }
                 tc_fence_after();
-                const int s = t * 128 + key_in_tile;                 // key position
-                const float sk =
-                    (p.k_scale && s <= it.maxlim) ? p.k_scale[it.keybase + s] : 1.0f;
+                // s: the output column (key position in scan mode, candidate
+                // slot in gather mode); keyrow: the key's row for its scale
+                const int s = t * 128 + key_in_tile;
+                int keyrow = -1;
+                if constexpr (GATHER) {
+                    const int pos = s < p.C ? it.cand[s] : -1;
+                    if (pos >= 0 && pos < p.nkeys) keyrow = it.keybase + pos;
+                } else {
+                    if (s <= it.maxlim) keyrow = it.keybase + s;
+                }
+                const bool col_ok = GATHER ? (s < p.C) : true;
+                const float sk = (p.k_scale && keyrow >= 0) ? p.k_scale[keyrow] : 1.0f;
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * 256);
                 float rowacc = 0.0f;
@@ -274,7 +398,7 @@ __global__ void __launch_bounds__(192, 1)
                             rowacc = fmaf(w_s[c0 + i], fmaxf(v[i], 0.0f), rowacc);
                             if ((i + 1) % HEADS == 0) {
                                 const int pr = (c0 + i) / HEADS;
-                                if (s <= lim_s[pr])
+                                if (col_ok && s <= lim_s[pr])
                                     p.S[(size_t)(it.row_first + pr - p.row0) * p.S_stride + s] =
                                         rowacc * sq_s[pr] * sk;
                                 rowacc = 0.0f;
@@ -286,7 +410,7 @@ __global__ void __launch_bounds__(192, 1)
                             rowacc = fmaf(w_s[c0 + i], fmaxf(v[i], 0.0f), rowacc);
                         if ((c0 + 32) % HEADS == 0) {
                             const int pr = c0 / HEADS;
-                            if (s <= lim_s[pr])
+                            if (col_ok && s <= lim_s[pr])
                                 p.S[(size_t)(it.row_first + pr - p.row0) * p.S_stride + s] =
                                     rowacc * sq_s[pr] * sk;
                             rowacc = 0.0f;
@@ -308,18 +432,24 @@ __global__ void __launch_bounds__(192, 1)
     }
 }
 
-template <int KIND, int HEADS>
-static cudaError_t launch_scan_heads(const CUtensorMap& tk, const CUtensorMap& tq,
-                                     const ScanParams& p, int row_bytes, int grid,
-                                     cudaStream_t stream) {
+int scan_smem_bytes(int row_bytes) {
+    const int stages = row_bytes == 128 ? 6 : 3;
+    const int pmax = 64;
+    return 1024 /*align slack*/ + 2 * 256 * row_bytes + stages * 128 * row_bytes +
+           (2 * stages + 9) * 8 + 16 + 256 * 4 + pmax * 8;
+}
+
+template <int KIND, int HEADS, bool GATHER>
+static cudaError_t launch_heads(const CUtensorMap& tk, const CUtensorMap& tq, const ScanParams& p,
+                                int row_bytes, int grid, cudaStream_t stream) {
     if (row_bytes == 128) {
-        auto kfn = scan_umma_kernel<KIND, HEADS, 128>;
+        auto kfn = index_umma_kernel<KIND, HEADS, 128, GATHER>;
         const int smem = scan_smem_bytes(128);
         cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         kfn<<<grid, 192, smem, stream>>>(tk, tq, p);
     } else {
-        auto kfn = scan_umma_kernel<KIND, HEADS, 256>;
+        auto kfn = index_umma_kernel<KIND, HEADS, 256, GATHER>;
         const int smem = scan_smem_bytes(256);
         cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
@@ -328,36 +458,41 @@ static cudaError_t launch_scan_heads(const CUtensorMap& tk, const CUtensorMap& t
     return cudaGetLastError();
 }
 
-int scan_smem_bytes(int row_bytes) {
-    const int stages = row_bytes == 128 ? 6 : 3;
-    const int pmax = 64;
-    return 1024 /*align slack*/ + 2 * 256 * row_bytes + stages * 128 * row_bytes +
-           (2 * stages + 9) * 8 + 16 + 256 * 4 + pmax * 8;
+template <int KIND, bool GATHER>
+static cudaError_t launch_kind(const CUtensorMap& tk, const CUtensorMap& tq, const ScanParams& p,
+                               int row_bytes, int grid, cudaStream_t stream) {
+    switch (p.H) {
+        case 4: return launch_heads<KIND, 4, GATHER>(tk, tq, p, row_bytes, grid, stream);
+        case 8: return launch_heads<KIND, 8, GATHER>(tk, tq, p, row_bytes, grid, stream);
+        case 16: return launch_heads<KIND, 16, GATHER>(tk, tq, p, row_bytes, grid, stream);
+        case 32: return launch_heads<KIND, 32, GATHER>(tk, tq, p, row_bytes, grid, stream);
+        case 64: return launch_heads<KIND, 64, GATHER>(tk, tq, p, row_bytes, grid, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
-template <int KIND>
-static cudaError_t launch_scan_kind(const CUtensorMap& tk, const CUtensorMap& tq,
-                                    const ScanParams& p, int row_bytes, int grid,
-                                    cudaStream_t stream) {
-    switch (p.H) {
-        case 4: return launch_scan_heads<KIND, 4>(tk, tq, p, row_bytes, grid, stream);
-        case 8: return launch_scan_heads<KIND, 8>(tk, tq, p, row_bytes, grid, stream);
-        case 16: return launch_scan_heads<KIND, 16>(tk, tq, p, row_bytes, grid, stream);
-        case 32: return launch_scan_heads<KIND, 32>(tk, tq, p, row_bytes, grid, stream);
-        case 64: return launch_scan_heads<KIND, 64>(tk, tq, p, row_bytes, grid, stream);
-        default: return cudaErrorInvalidValue;
+template <bool GATHER>
+static cudaError_t launch_any(const CUtensorMap& tk, const CUtensorMap& tq, const ScanParams& p,
+                              int grid, cudaStream_t stream) {
+    if (p.nitems <= 0 || grid <= 0) return cudaSuccess;
+    const int row_bytes = p.D * p.esize;
+    switch (p.dtype) {
+        case PIVOT_E4M3: return launch_kind<KIND_F8, GATHER>(tk, tq, p, row_bytes, grid, stream);
+        case PIVOT_BF16: return launch_kind<KIND_F16, GATHER>(tk, tq, p, row_bytes, grid, stream);
+        default: return launch_kind<KIND_TF32, GATHER>(tk, tq, p, row_bytes, grid, stream);
     }
 }
 
 cudaError_t launch_scan_umma(const CUtensorMap& tk, const CUtensorMap& tq, const ScanParams& p,
                              int grid, cudaStream_t stream) {
-    if (p.nitems <= 0 || grid <= 0) return cudaSuccess;
-    const int row_bytes = p.D * p.esize;
-    switch (p.dtype) {
-        case PIVOT_E4M3: return launch_scan_kind<KIND_F8>(tk, tq, p, row_bytes, grid, stream);
-        case PIVOT_BF16: return launch_scan_kind<KIND_F16>(tk, tq, p, row_bytes, grid, stream);
-        default: return launch_scan_kind<KIND_TF32>(tk, tq, p, row_bytes, grid, stream);
-    }
+    return launch_any<false>(tk, tq, p, grid, stream);
+}
+
+cudaError_t launch_refine_umma(const CUtensorMap& tmap_q, const ScanParams& p, int grid,
+                               cudaStream_t stream) {
+    // the key operand is gathered with cp.async from p.kbase; its tensor-map
+    // slot is unused, so the query map fills it
+    return launch_any<true>(tmap_q, tmap_q, p, grid, stream);
 }
 
 }  // namespace pivot

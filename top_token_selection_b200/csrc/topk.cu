@@ -1,20 +1,31 @@
-// topk.cu -- exact per-row top-K selection with the indexer's tie-break.
+// topk.cu -- exact per-row top-K selection.
 //
-// The indexer returns positions only, the k highest scores of the row
-// ("Sparse Attention의 Indexer", Fig. 1: top-k keeps the k largest selection
-// scores).  Order: higher score first, equal scores by lower position, -0
-// equal to +0.  Each entry gets a 64-bit key
+// The indexer returns positions only: the k highest scores of the row
+// ("Sparse Attention의 Indexer", Fig. 1 -- top-k keeps the k largest
+// selection scores and hands their positions on, listed by position).
+// Equal scores are taken lower position first; -0 equals +0.  Output rows
+// list the selected positions in ascending order (a candidate row lists the
+// proxy's top-`split` first, then the rest of the top-C, each ascending).
+//
+// Every entry has a 64-bit key
 //     key = ordered(score) << 32 | (0xFFFFFFFF - position)
-// which is unique per row, so "the K largest keys" is exactly the answer.
+// (ordered(): order-preserving uint32 of the float), unique per row, so "the
+// K largest keys" is exactly the answer.
 //
-// One CTA per row:
-//   1. histogram of the top 12 key bits over the row (warp-aggregated
-//      shared-memory atomics);
-//   2. the bin B holding the K-th largest; entries of higher bins are in;
-//   3. entries of bin B go to a shared-memory boundary buffer (or, if it
-//      overflows, are re-read from global memory), where an 8-bit-digit
-//      radix select over the remaining 52 key bits picks the exact rest;
-//   4. the K winners are sorted in shared memory (bitonic) and written.
+// One CTA per row.  Fast path:
+//   1. a lower bound T for the kept scores: the m-th largest of 4096 evenly
+//      spaced sampled scores, m chosen so about 1.4 K entries of the row
+//      should lie at or above it (all entries when the row is short);
+//   2. one vectorised pass appends every eligible entry >= T to shared
+//      memory (warp-aggregated);
+//   3. if between K and the buffer capacity entries were kept, they hold the
+//      top K exactly; the exact K-th score is found by radix passes over
+//      linear bins (no sort); ties at it are resolved by position rank;
+//   4. positions go into a bitmap; prefix popcounts give every selected
+//      entry its output slot, so rows come out in position order unsorted.
+// Otherwise (threshold missed, K > 8192, rows too long for the bitmaps) the
+// exact path: histogram of the top 12 key bits, radix select inside the
+// boundary bin, then a sort by position.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -23,7 +34,10 @@ namespace pivot {
 namespace {
 
 constexpr int SEL_THREADS = 512;
-constexpr int HIST_BINS = 4096;     // top 12 bits of the ordered score
+constexpr int HIST_BINS = 4096;     // top 12 bits of the ordered score; also sample/bin space
+constexpr int SAMPLES = 4096;
+constexpr int LBINS = 4096;         // linear bins of one threshold-search pass
+constexpr float SAMPLE_MARGIN = 1.4f;
 
 __device__ __forceinline__ int row_limit(int kind, int r, int L, int g, int Gm, int maxlen,
                                          const int32_t* cache_len, bool& ok) {
@@ -55,6 +69,18 @@ struct RowView {
     int lim;               // valid positions are <= lim
 };
 
+__device__ __forceinline__ uint64_t make_key(uint32_t u, int pos) {
+    return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)pos);
+}
+__device__ __forceinline__ uint32_t key_u(uint64_t k) { return (uint32_t)(k >> 32); }
+__device__ __forceinline__ int key_pos(uint64_t k) {
+    return (int)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFu));
+}
+// Position as an unsigned value in which a zero (padding) key sorts last.
+__device__ __forceinline__ uint32_t key_upos(uint64_t k) {
+    return 0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFu);
+}
+
 // Key of entry i, or 0 when the entry is not eligible.
 __device__ __forceinline__ uint64_t entry_key(const RowView& v, int i) {
     int pos = i;
@@ -62,8 +88,66 @@ __device__ __forceinline__ uint64_t entry_key(const RowView& v, int i) {
         pos = v.cand[i];
         if (pos < 0 || pos > v.lim) return 0;
     }
-    const uint32_t u = ordered_key(v.S[i]);
-    return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)pos);
+    return make_key(ordered_key(v.S[i]), pos);
+}
+__device__ __forceinline__ uint32_t entry_key32(const RowView& v, int i) {
+    if (v.cand) {
+        const int pos = v.cand[i];
+        if (pos < 0 || pos > v.lim) return 0;
+    }
+    return ordered_key(v.S[i]);
+}
+
+// ------------------------------------------------------------ block helpers
+
+__device__ uint32_t block_sum_u32(uint32_t x, uint32_t* scratch) {
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = x;
+    __syncthreads();
+    uint32_t t = 0;
+    for (int w = 0; w < SEL_THREADS / 32; ++w) t += scratch[w];
+    __syncthreads();
+    return t;
+}
+
+__device__ uint32_t block_min_u32(uint32_t x, uint32_t* scratch) {
+    for (int o = 16; o > 0; o >>= 1) x = min(x, __shfl_xor_sync(0xffffffffu, x, o));
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = x;
+    __syncthreads();
+    uint32_t t = 0xFFFFFFFFu;
+    for (int w = 0; w < SEL_THREADS / 32; ++w) t = min(t, scratch[w]);
+    __syncthreads();
+    return t;
+}
+
+__device__ uint32_t block_max_u32(uint32_t x, uint32_t* scratch) {
+    for (int o = 16; o > 0; o >>= 1) x = max(x, __shfl_xor_sync(0xffffffffu, x, o));
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = x;
+    __syncthreads();
+    uint32_t t = 0;
+    for (int w = 0; w < SEL_THREADS / 32; ++w) t = max(t, scratch[w]);
+    __syncthreads();
+    return t;
+}
+
+// Exclusive prefix sum over threads (in thread order).
+__device__ uint32_t block_excl_scan(uint32_t x, uint32_t* scratch) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint32_t inc = x;
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    __syncthreads();
+    if (lane == 31) scratch[wid] = inc;
+    __syncthreads();
+    uint32_t base = 0;
+    for (int w = 0; w < wid; ++w) base += scratch[w];
+    __syncthreads();
+    return base + inc - x;
 }
 
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
@@ -74,43 +158,22 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool acti
     if ((threadIdx.x & 31) == leader) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
 }
 
-// Block-wide: find the largest bin b with sum_{bins >= b} hist >= need, over
-// `nbins` bins.  Returns b and the count strictly above it in *above.
-// Requires nbins % SEL_THREADS == 0 or nbins <= SEL_THREADS.
+// Block-wide: the largest bin b with sum_{bins >= b} hist >= need, over
+// `nbins` bins (nbins a multiple of SEL_THREADS, or <= SEL_THREADS).
+// Returns b and the count strictly above it in *above.
 __device__ int find_threshold_bin(const uint32_t* hist, int nbins, uint32_t need,
                                   uint32_t* scratch, uint32_t* above) {
     __shared__ int s_bin;
     __shared__ uint32_t s_above;
     const int per = nbins >= SEL_THREADS ? nbins / SEL_THREADS : 1;
     const int t = threadIdx.x;
-    // thread t owns bins [nbins - (t+1)*per, nbins - t*per) (descending order)
     uint32_t local = 0;
-    const int hi = nbins - t * per;        // exclusive
+    const int hi = nbins - t * per;        // thread t owns bins [hi - per, hi), descending
     const int lo = hi - per;
     if (lo >= 0)
         for (int b = lo; b < hi; ++b) local += hist[b];
-    // inclusive scan over threads (descending bins)
-    const int lane = t & 31, wid = t >> 5;
-    uint32_t x = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) scratch[wid] = x;
     if (t == 0) { s_bin = -1; s_above = 0; }
-    __syncthreads();
-    if (wid == 0) {
-        uint32_t w = lane < SEL_THREADS / 32 ? scratch[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += y;
-        }
-        if (lane < SEL_THREADS / 32) scratch[32 + lane] = w;   // inclusive warp totals
-    }
-    __syncthreads();
-    const uint32_t before = (wid > 0 ? scratch[32 + wid - 1] : 0) + x - local;  // exclusive
+    const uint32_t before = block_excl_scan(local, scratch);
     if (lo >= 0 && before < need && before + local >= need) {
         uint32_t acc = before;
         for (int b = hi - 1; b >= lo; --b) {
@@ -124,7 +187,281 @@ __device__ int find_threshold_bin(const uint32_t* hist, int nbins, uint32_t need
     }
     __syncthreads();
     *above = s_above;
-    return s_bin;
+    const int r = s_bin;
+    __syncthreads();
+    return r;
+}
+
+// The m-th largest value among n uint32 values >= 1 (values 0 are ignored),
+// 1 <= m <= the count of such values: repeated histograms over LBINS linear
+// bins of the remaining value range.  *above_out = the count of values
+// strictly greater than the result.  `vals(i)` yields value i.
+template <class F>
+__device__ uint32_t kth_largest_linear(F vals, int n, uint32_t m, uint32_t* hist,
+                                       uint32_t* scratch, uint32_t* above_out) {
+    uint32_t lo_l = 0xFFFFFFFFu, hi_l = 0;
+    for (int i = threadIdx.x; i < n; i += SEL_THREADS) {
+        const uint32_t u = vals(i);
+        if (u) { lo_l = min(lo_l, u); hi_l = max(hi_l, u); }
+    }
+    uint32_t lo = block_min_u32(lo_l, scratch);
+    uint32_t hi = block_max_u32(hi_l, scratch);
+    uint32_t remaining = m, above_total = 0;
+    while (lo < hi) {
+        const uint64_t range = (uint64_t)hi - lo + 1;
+        for (int b = threadIdx.x; b < LBINS; b += SEL_THREADS) hist[b] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += SEL_THREADS) {
+            const uint32_t u = vals(i);
+            if (u && u >= lo && u <= hi) {
+                const uint32_t b = (uint32_t)(((uint64_t)(u - lo) * LBINS) / range);
+                atomicAdd(&hist[b], 1u);
+            }
+        }
+        __syncthreads();
+        uint32_t above;
+        const int b = find_threshold_bin(hist, LBINS, remaining, scratch, &above);
+        remaining -= above;
+        above_total += above;
+        // bin b holds the u with floor((u - lo) * LBINS / range) == b
+        const uint32_t nlo = lo + (uint32_t)(((uint64_t)b * range + LBINS - 1) / LBINS);
+        const uint32_t nhi = lo + (uint32_t)(((uint64_t)(b + 1) * range + LBINS - 1) / LBINS) - 1;
+        lo = nlo;
+        hi = nhi;
+    }
+    *above_out = above_total;
+    return lo;
+}
+
+// Warp-aggregated append of `key` (where pred) to buf[*cnt++]; entries past
+// `cap` are counted but not stored.  All 32 lanes must call it together.
+__device__ __forceinline__ void warp_append(uint64_t* buf, uint32_t* cnt, uint32_t cap,
+                                            uint64_t key, bool pred) {
+    const unsigned m = __ballot_sync(0xffffffffu, pred);
+    if (m == 0) return;
+    const int lane = threadIdx.x & 31;
+    const int leader = __ffs(m) - 1;
+    uint32_t base = 0;
+    if (lane == leader) base = atomicAdd(cnt, (uint32_t)__popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (pred) {
+        const uint32_t idx = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
+        if (idx < cap) buf[idx] = key;
+    }
+}
+
+// Per-word exclusive prefix popcounts of a bitmap of W words.
+__device__ void bitmap_prefix(const uint32_t* bm, uint32_t* pref, int W, uint32_t* scratch) {
+    const int per = (W + SEL_THREADS - 1) / SEL_THREADS;
+    const int w0 = threadIdx.x * per;
+    const int w1 = min(W, w0 + per);
+    uint32_t local = 0;
+    for (int w = w0; w < w1; ++w) local += __popc(bm[w]);
+    uint32_t acc = block_excl_scan(local, scratch);
+    for (int w = w0; w < w1; ++w) {
+        pref[w] = acc;
+        acc += __popc(bm[w]);
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ bool bit_of(const uint32_t* bm, int pos) {
+    return (bm[pos >> 5] >> (pos & 31)) & 1u;
+}
+__device__ __forceinline__ uint32_t rank_of(const uint32_t* bm, const uint32_t* pref, int pos) {
+    return pref[pos >> 5] + __popc(bm[pos >> 5] & ((1u << (pos & 31)) - 1u));
+}
+
+// Mark in `bm` the kept entries with u > Tu, plus the `need` lowest-position
+// entries with u == Tu.  `tie` is a scratch bitmap, `pref` scratch prefixes.
+__device__ void mark_top(const uint64_t* buf, int cnt, uint32_t Tu, uint32_t need, uint32_t* bm,
+                         uint32_t* tie, uint32_t* pref, int W, uint32_t* scratch) {
+    for (int w = threadIdx.x; w < W; w += SEL_THREADS) tie[w] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
+        const uint64_t k = buf[i];
+        const uint32_t u = key_u(k);
+        const int pos = key_pos(k);
+        if (u > Tu) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+        else if (u == Tu) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
+    }
+    __syncthreads();
+    bitmap_prefix(tie, pref, W, scratch);
+    for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
+        const uint64_t k = buf[i];
+        if (key_u(k) == Tu) {
+            const int pos = key_pos(k);
+            if (rank_of(tie, pref, pos) < need) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+        }
+    }
+    __syncthreads();
+}
+
+// Write every kept entry whose position is marked in `bm` at slot
+// base + (its rank among the marked positions).
+__device__ void write_marked(const uint64_t* buf, int cnt, const uint32_t* bm, uint32_t* pref,
+                             int W, uint32_t base, uint32_t* scratch, int32_t* out, float* outs) {
+    bitmap_prefix(bm, pref, W, scratch);
+    for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
+        const uint64_t k = buf[i];
+        const int pos = key_pos(k);
+        if (bit_of(bm, pos)) {
+            const uint32_t slot = base + rank_of(bm, pref, pos);
+            out[slot] = pos;
+            if (outs) outs[slot] = key_to_float(key_u(k));
+        }
+    }
+    __syncthreads();
+}
+
+__device__ void pad_row(uint32_t from, int K, int32_t* out, float* outs) {
+    for (int i = (int)from + threadIdx.x; i < K; i += SEL_THREADS) {
+        out[i] = -1;
+        if (outs) outs[i] = -INFINITY;
+    }
+}
+
+struct FastSmem {
+    uint32_t* hist;     // HIST_BINS: samples, then linear bins
+    uint32_t* scratch;  // 64
+    uint64_t* buf;      // fast_cap kept entries
+    uint32_t* bmS;      // selected positions (W words)
+    uint32_t* bmT;      // ties / class-B scratch (W words)
+    uint32_t* bmA;      // class A, only when split (W words)
+    uint32_t* pref;     // W prefix counts (aliases hist when W <= HIST_BINS)
+};
+
+// Fast path; returns false (block-uniformly) when the threshold kept fewer
+// than K eligible entries or more than the buffer holds.
+__device__ bool select_fast(const SelectParams& p, const RowView& v, const FastSmem& sm,
+                            uint32_t* s_cnt, uint32_t* s_valid, int32_t* out, float* outs) {
+    const int K = p.K, cap = p.fast_cap, W = p.bitmap_words;
+    uint32_t* hist = sm.hist;
+    uint32_t* scratch = sm.scratch;
+    uint64_t* buf = sm.buf;
+    if (threadIdx.x == 0) { *s_cnt = 0; *s_valid = 0; }
+    uint32_t T = 1;
+    if (v.n > cap) {
+        for (int j = threadIdx.x; j < SAMPLES; j += SEL_THREADS)
+            hist[j] = entry_key32(v, (int)(((long long)j * v.n) / SAMPLES));
+        __syncthreads();
+        uint32_t elig = 0;
+        for (int j = threadIdx.x; j < SAMPLES; j += SEL_THREADS) elig += hist[j] != 0;
+        elig = block_sum_u32(elig, scratch);
+        long long m = (long long)ceilf(SAMPLE_MARGIN * (float)K * (float)SAMPLES / (float)v.n);
+        if (m < 1) m = 1;
+        if (m <= (long long)elig) {
+            // move the samples out of the bins' way (the buffer is still free)
+            uint32_t* samp = reinterpret_cast<uint32_t*>(buf);
+            for (int j = threadIdx.x; j < SAMPLES; j += SEL_THREADS) samp[j] = hist[j];
+            __syncthreads();
+            uint32_t above;
+            T = kth_largest_linear([&](int i) { return samp[i]; }, SAMPLES, (uint32_t)m, hist,
+                                   scratch, &above);
+        }
+    }
+    __syncthreads();
+    // filtering pass
+    uint32_t nvalid_local = 0;
+    const bool vec = (v.cand == nullptr) && ((reinterpret_cast<uintptr_t>(v.S) & 15) == 0);
+    if (vec) {
+        const int n4 = v.n / 4;
+        const float4* S4 = reinterpret_cast<const float4*>(v.S);
+#pragma unroll 2
+        for (int i0 = 0; i0 < n4; i0 += SEL_THREADS) {
+            const int i = i0 + threadIdx.x;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            const bool a = i < n4;
+            if (a) x = __ldcs(S4 + i);
+            const uint32_t u0 = ordered_key(x.x), u1 = ordered_key(x.y);
+            const uint32_t u2 = ordered_key(x.z), u3 = ordered_key(x.w);
+            warp_append(buf, s_cnt, cap, make_key(u0, 4 * i + 0), a && u0 >= T);
+            warp_append(buf, s_cnt, cap, make_key(u1, 4 * i + 1), a && u1 >= T);
+            warp_append(buf, s_cnt, cap, make_key(u2, 4 * i + 2), a && u2 >= T);
+            warp_append(buf, s_cnt, cap, make_key(u3, 4 * i + 3), a && u3 >= T);
+        }
+        const int i = n4 * 4 + threadIdx.x;
+        const bool a = threadIdx.x < 4 && i < v.n;
+        const uint32_t u = a ? ordered_key(v.S[i]) : 0u;
+        warp_append(buf, s_cnt, cap, make_key(u, i), a && u >= T);
+    } else {
+        for (int i0 = 0; i0 < v.n; i0 += SEL_THREADS) {
+            const int i = i0 + threadIdx.x;
+            uint32_t u = 0;
+            int pos = i;
+            if (i < v.n) {
+                u = entry_key32(v, i);
+                if (v.cand) pos = v.cand[i];
+            }
+            nvalid_local += (u != 0);
+            warp_append(buf, s_cnt, cap, make_key(u, pos), u != 0 && u >= T);
+        }
+    }
+    if (v.cand) {
+        for (int o = 16; o > 0; o >>= 1) nvalid_local += __shfl_xor_sync(0xffffffffu, nvalid_local, o);
+        if ((threadIdx.x & 31) == 0 && nvalid_local) atomicAdd(s_valid, nvalid_local);
+    }
+    __syncthreads();
+    const uint32_t cnt = *s_cnt;
+    const uint32_t nvalid = v.cand ? *s_valid : (uint32_t)v.n;
+    const uint32_t Kp = nvalid < (uint32_t)K ? nvalid : (uint32_t)K;
+    __syncthreads();
+    if (cnt > (uint32_t)cap || cnt < Kp) return false;
+    if (Kp == 0) {
+        pad_row(0, K, out, outs);
+        return true;
+    }
+    const int n = (int)cnt;
+    auto uval = [&](int i) { return key_u(buf[i]); };
+    uint32_t aboveK, aboveS = 0;
+    const uint32_t TuK = kth_largest_linear(uval, n, Kp, hist, scratch, &aboveK);
+    const int split = (p.split > 0 && (uint32_t)p.split < Kp) ? p.split : 0;
+    uint32_t TuS = 0;
+    if (split) TuS = kth_largest_linear(uval, n, (uint32_t)split, hist, scratch, &aboveS);
+    // selected set (the linear bins are no longer needed, so pref may alias them)
+    for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmS[w] = 0;
+    __syncthreads();
+    mark_top(buf, n, TuK, Kp - aboveK, sm.bmS, sm.bmT, sm.pref, W, scratch);
+    if (!split) {
+        write_marked(buf, n, sm.bmS, sm.pref, W, 0, scratch, out, outs);
+    } else {
+        // class A: the top `split`; class B: the rest of the selected set
+        for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmA[w] = 0;
+        __syncthreads();
+        mark_top(buf, n, TuS, (uint32_t)split - aboveS, sm.bmA, sm.bmT, sm.pref, W, scratch);
+        write_marked(buf, n, sm.bmA, sm.pref, W, 0, scratch, out, outs);
+        for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmT[w] = sm.bmS[w] & ~sm.bmA[w];
+        __syncthreads();
+        write_marked(buf, n, sm.bmT, sm.pref, W, (uint32_t)split, scratch, out, outs);
+    }
+    pad_row(Kp, K, out, outs);
+    return true;
+}
+
+// Sort buf[0, n) ascending by `less` (bitonic, pads to a power of two with
+// `pad`, which must sort last).
+template <class Less>
+__device__ void bitonic_sort(uint64_t* buf, int n, uint64_t pad, Less less) {
+    int M = 1;
+    while (M < n) M <<= 1;
+    for (int i = n + threadIdx.x; i < M; i += SEL_THREADS) buf[i] = pad;
+    __syncthreads();
+    for (int kk = 2; kk <= M; kk <<= 1) {
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < M; i += SEL_THREADS) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const uint64_t a = buf[i], b = buf[ixj];
+                    const bool up = (i & kk) == 0;
+                    if (up ? less(b, a) : less(a, b)) {
+                        buf[i] = b;
+                        buf[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
 }
 
 // Radix select among keys k with (k >> 52) == bin0: the `need` largest.
@@ -170,16 +507,146 @@ __device__ void radix_select_tail(const RowView& v, const uint64_t* tail, int nt
     *out_prefix = prefix;
 }
 
-__global__ void __launch_bounds__(SEL_THREADS)
-    select_kernel(const SelectParams p) {
+
+// Exact path: histogram of the top 12 key bits over the whole row, exact
+// radix select inside the boundary bin, then the selected keys sorted by
+// position (the top `split` first when requested).  `sel` has room for
+// 2 * pow2(K) keys, `tail` for tail_cap keys.
+__device__ void select_exact(const SelectParams& p, const RowView& v, uint32_t* hist,
+                             uint32_t* scratch, uint32_t* hist256, uint64_t* sel, uint64_t* tail,
+                             int M2, uint32_t* s_nsel, uint32_t* s_ntail, int32_t* out,
+                             float* outs) {
+    // 1. histogram of the top 12 bits
+    for (int b = threadIdx.x; b < HIST_BINS; b += SEL_THREADS) hist[b] = 0;
+    if (threadIdx.x == 0) { *s_nsel = 0; *s_ntail = 0; }
+    __syncthreads();
+    for (int i0 = 0; i0 < v.n; i0 += SEL_THREADS) {
+        const int i = i0 + threadIdx.x;
+        const uint32_t u = i < v.n ? entry_key32(v, i) : 0;
+        hist_add(hist, u >> 20, u != 0);
+    }
+    __syncthreads();
+    uint32_t total_local = 0;
+    for (int b = threadIdx.x; b < HIST_BINS; b += SEL_THREADS) total_local += hist[b];
+    const uint32_t total = block_sum_u32(total_local, scratch);
+    const uint32_t Kp = total < (uint32_t)p.K ? total : (uint32_t)p.K;
+
+    // 2. threshold bin
+    int bin = -1;
+    uint32_t above = 0;
+    if (Kp > 0 && Kp < total) bin = find_threshold_bin(hist, HIST_BINS, Kp, scratch, &above);
+    const uint32_t need = Kp - above;
+
+    // 3. collect
+    for (int i0 = 0; i0 < v.n; i0 += SEL_THREADS) {
+        const int i = i0 + threadIdx.x;
+        if (i >= v.n) break;
+        const uint64_t k = entry_key(v, i);
+        if (k == 0) continue;
+        const int b = (int)(k >> 52);
+        if (b > bin) {
+            sel[atomicAdd(s_nsel, 1u)] = k;
+        } else if (b == bin) {
+            const uint32_t slot = atomicAdd(s_ntail, 1u);
+            if (slot < (uint32_t)p.tail_cap) tail[slot] = k;
+        }
+    }
+    __syncthreads();
+
+    // 4. resolve the boundary bin
+    if (bin >= 0 && need > 0) {
+        const uint32_t ntail = *s_ntail;
+        uint64_t mask, prefix;
+        if (ntail == need) {
+            mask = 0; prefix = 0;   // take all of them
+        } else if (ntail <= (uint32_t)p.tail_cap) {
+            radix_select_tail<true>(v, tail, (int)ntail, (uint32_t)bin, need, hist256, scratch,
+                                    &mask, &prefix);
+        } else {
+            radix_select_tail<false>(v, nullptr, 0, (uint32_t)bin, need, hist256, scratch, &mask,
+                                     &prefix);
+        }
+        if (ntail <= (uint32_t)p.tail_cap) {
+            for (uint32_t i = threadIdx.x; i < ntail; i += SEL_THREADS) {
+                const uint64_t k = tail[i];
+                if ((k & mask) >= prefix) sel[atomicAdd(s_nsel, 1u)] = k;
+            }
+        } else {
+            for (int i = threadIdx.x; i < v.n; i += SEL_THREADS) {
+                const uint64_t k = entry_key(v, i);
+                if (k != 0 && (int)(k >> 52) == bin && (k & mask) >= prefix)
+                    sel[atomicAdd(s_nsel, 1u)] = k;
+            }
+        }
+        __syncthreads();
+    }
+
+    // 5. order: by key (to split off the top `split`), then by position
+    auto by_pos = [](uint64_t a, uint64_t b) { return key_upos(a) < key_upos(b); };
+    const int split = (p.split > 0 && (uint32_t)p.split < Kp) ? p.split : 0;
+    if (split) {
+        bitonic_sort(sel, (int)Kp, 0ull, [](uint64_t a, uint64_t b) { return a > b; });
+        uint64_t* rest = sel + M2;
+        for (int i = threadIdx.x; i < (int)Kp - split; i += SEL_THREADS) rest[i] = sel[split + i];
+        __syncthreads();
+        bitonic_sort(sel, split, 0ull, by_pos);
+        bitonic_sort(rest, (int)Kp - split, 0ull, by_pos);
+        for (int i = threadIdx.x; i < (int)Kp - split; i += SEL_THREADS) sel[split + i] = rest[i];
+        __syncthreads();
+    } else {
+        bitonic_sort(sel, (int)Kp, 0ull, by_pos);
+    }
+    for (int i = threadIdx.x; i < p.K; i += SEL_THREADS) {
+        if ((uint32_t)i < Kp) {
+            const uint64_t k = sel[i];
+            out[i] = key_pos(k);
+            if (outs) outs[i] = key_to_float(key_u(k));
+        } else {
+            out[i] = -1;
+            if (outs) outs[i] = -INFINITY;
+        }
+    }
+}
+
+__host__ __device__ int pow2_at_least(int x) {
+    int m = 1;
+    while (m < x) m <<= 1;
+    return m;
+}
+
+}  // namespace
+
+// Shared-memory layout, in bytes from the start of the dynamic buffer:
+//   hist [HIST_BINS] u32 | scratch [64] u32 | hist256 [256] u32 | region
+// region (8-byte aligned) is either the exact path's sel [2 * pow2(K)] +
+// tail [tail_cap] keys, or the fast path's buf [fast_cap] keys followed by
+// the bitmaps bmS, bmT (and bmA when split) and, when W > HIST_BINS, pref.
+struct SelectLayout {
+    size_t region_off, exact_bytes, fast_bytes, total;
+};
+
+static SelectLayout select_layout(int K, int tail_cap, int fast_cap, int W, bool split) {
+    SelectLayout L{};
+    L.region_off = (size_t)(HIST_BINS + 64 + 256) * 4;
+    const size_t m2 = (size_t)pow2_at_least(K);
+    L.exact_bytes = (2 * m2 + (size_t)tail_cap) * 8;
+    L.fast_bytes = 0;
+    if (fast_cap > 0) {
+        const int nbm = split ? 3 : 2;
+        L.fast_bytes = (size_t)fast_cap * 8 + (size_t)(nbm + (W > HIST_BINS ? 1 : 0)) * W * 4;
+    }
+    L.total = L.region_off + (L.exact_bytes > L.fast_bytes ? L.exact_bytes : L.fast_bytes);
+    return L;
+}
+
+__global__ void __launch_bounds__(SEL_THREADS) select_kernel(const SelectParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t* hist = reinterpret_cast<uint32_t*>(smem);                   // HIST_BINS
-    uint32_t* scratch = hist + HIST_BINS;                                  // 64
-    uint64_t* sel = reinterpret_cast<uint64_t*>(scratch + 64);             // pow2(K)
-    int M2 = 1;
-    while (M2 < p.K) M2 <<= 1;
-    uint64_t* tail = sel + M2;                                             // tail_cap
-    __shared__ uint32_t s_nsel, s_ntail;
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem);
+    uint32_t* scratch = hist + HIST_BINS;
+    uint32_t* hist256 = scratch + 64;
+    uint64_t* region = reinterpret_cast<uint64_t*>(hist256 + 256);
+    const int M2 = pow2_at_least(p.K);
+    __shared__ uint32_t s_a, s_b;
 
     const int r = p.row0 + blockIdx.x;
     int32_t* out = p.out_idx + (size_t)(r - p.out_base) * p.K;
@@ -200,147 +667,54 @@ __global__ void __launch_bounds__(SEL_THREADS)
     }
     if (!ok && threadIdx.x == 0) raise_error(ERRBIT_DATA);
 
-    // 1. histogram of the top 12 bits
-    for (int b = threadIdx.x; b < HIST_BINS; b += SEL_THREADS) hist[b] = 0;
-    if (threadIdx.x == 0) { s_nsel = 0; s_ntail = 0; }
-    __syncthreads();
-    const bool vec = (v.cand == nullptr) && ((reinterpret_cast<uintptr_t>(v.S) & 15) == 0);
-    if (vec) {
-        const int n4 = v.n / 4;
-        const float4* S4 = reinterpret_cast<const float4*>(v.S);
-        for (int i0 = 0; i0 < n4; i0 += SEL_THREADS) {
-            const int i = i0 + threadIdx.x;
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < n4) x = S4[i];
-            const bool a = i < n4;
-            hist_add(hist, ordered_key(x.x) >> 20, a);
-            hist_add(hist, ordered_key(x.y) >> 20, a);
-            hist_add(hist, ordered_key(x.z) >> 20, a);
-            hist_add(hist, ordered_key(x.w) >> 20, a);
-        }
-        const int i = n4 * 4 + threadIdx.x;
-        const bool a = i < v.n;
-        hist_add(hist, a ? ordered_key(v.S[i]) >> 20 : 0u, a);
-    } else {
-        for (int i0 = 0; i0 < v.n; i0 += SEL_THREADS) {
-            const int i = i0 + threadIdx.x;
-            uint64_t k = i < v.n ? entry_key(v, i) : 0;
-            hist_add(hist, (uint32_t)(k >> 52), k != 0);
-        }
-    }
-    __syncthreads();
-
-    // total eligible
-    uint32_t total_local = 0;
-    for (int b = threadIdx.x; b < HIST_BINS; b += SEL_THREADS) total_local += hist[b];
-    for (int o = 16; o > 0; o >>= 1) total_local += __shfl_xor_sync(0xffffffffu, total_local, o);
-    if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = total_local;
-    __syncthreads();
-    uint32_t total = 0;
-    for (int w = 0; w < SEL_THREADS / 32; ++w) total += scratch[w];
-    __syncthreads();
-    const uint32_t Kp = total < (uint32_t)p.K ? total : (uint32_t)p.K;
-
-    // 2. threshold bin
-    int bin = -1;
-    uint32_t above = 0;
-    if (Kp > 0 && Kp < total) bin = find_threshold_bin(hist, HIST_BINS, Kp, scratch, &above);
-    const uint32_t need = Kp - above;
-
-    // 3. collect
-    for (int i0 = 0; i0 < v.n; i0 += SEL_THREADS) {
-        const int i = i0 + threadIdx.x;
-        if (i >= v.n) break;
-        const uint64_t k = entry_key(v, i);
-        if (k == 0) continue;
-        const int b = (int)(k >> 52);
-        if (b > bin) {
-            sel[atomicAdd(&s_nsel, 1u)] = k;
-        } else if (b == bin) {
-            const uint32_t slot = atomicAdd(&s_ntail, 1u);
-            if (slot < (uint32_t)p.tail_cap) tail[slot] = k;
-        }
-    }
-    __syncthreads();
-
-    // 4. resolve the boundary bin
-    if (bin >= 0 && need > 0) {
-        const uint32_t ntail = s_ntail;
-        uint64_t mask, prefix;
-        if (ntail == need) {
-            mask = 0; prefix = 0;   // take all of them
-        } else if (ntail <= (uint32_t)p.tail_cap) {
-            radix_select_tail<true>(v, tail, (int)ntail, (uint32_t)bin, need, hist, scratch,
-                                    &mask, &prefix);
-        } else {
-            radix_select_tail<false>(v, nullptr, 0, (uint32_t)bin, need, hist, scratch, &mask,
-                                     &prefix);
-        }
-        if (ntail <= (uint32_t)p.tail_cap) {
-            for (uint32_t i = threadIdx.x; i < ntail; i += SEL_THREADS) {
-                const uint64_t k = tail[i];
-                if ((k & mask) >= prefix) sel[atomicAdd(&s_nsel, 1u)] = k;
-            }
-        } else {
-            for (int i = threadIdx.x; i < v.n; i += SEL_THREADS) {
-                const uint64_t k = entry_key(v, i);
-                if (k != 0 && (int)(k >> 52) == bin && (k & mask) >= prefix)
-                    sel[atomicAdd(&s_nsel, 1u)] = k;
-            }
-        }
+    if (p.fast_cap > 0) {
+        const int W = p.bitmap_words;
+        FastSmem sm;
+        sm.hist = hist;
+        sm.scratch = scratch;
+        sm.buf = region;
+        uint32_t* bms = reinterpret_cast<uint32_t*>(region + p.fast_cap);
+        sm.bmS = bms;
+        sm.bmT = bms + W;
+        sm.bmA = p.split > 0 ? bms + 2 * W : nullptr;
+        sm.pref = W > HIST_BINS ? bms + (p.split > 0 ? 3 : 2) * W : hist;
+        if (select_fast(p, v, sm, &s_a, &s_b, out, outs)) return;
         __syncthreads();
     }
-
-    // 5. rank order: bitonic sort, descending, over the next power of two
-    int M = 1;
-    while ((uint32_t)M < Kp) M <<= 1;
-    for (int i = Kp + threadIdx.x; i < M; i += SEL_THREADS) sel[i] = 0;
-    __syncthreads();
-    for (int kk = 2; kk <= M; kk <<= 1) {
-        for (int j = kk >> 1; j > 0; j >>= 1) {
-            for (int i = threadIdx.x; i < M; i += SEL_THREADS) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const uint64_t a = sel[i], b = sel[ixj];
-                    const bool desc = (i & kk) == 0;
-                    if (desc ? (a < b) : (a > b)) {
-                        sel[i] = b;
-                        sel[ixj] = a;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-    }
-
-    // 6. write
-    for (int i = threadIdx.x; i < p.K; i += SEL_THREADS) {
-        if ((uint32_t)i < Kp) {
-            const uint64_t k = sel[i];
-            out[i] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFu));
-            if (outs) outs[i] = key_to_float((uint32_t)(k >> 32));
-        } else {
-            out[i] = -1;
-            if (outs) outs[i] = -INFINITY;
-        }
-    }
+    select_exact(p, v, hist, scratch, hist256, region, region + 2 * M2, M2, &s_a, &s_b, out,
+                 outs);
 }
 
-}  // namespace
+// Kept-entry capacity of the fast path for top-K: twice K rounded up to a
+// power of two, at least 2048; 0 (exact path only) when K > 8192.
+static int select_fast_cap(int K) {
+    if (K > 8192) return 0;
+    int c = 2048;
+    while (c < 2 * K) c <<= 1;
+    return c;
+}
+
+constexpr size_t SELECT_SMEM_LIMIT = 220 * 1024;
 
 size_t select_smem_bytes(int K, int tail_cap) {
-    size_t m2 = 1;
-    while (m2 < (size_t)K) m2 <<= 1;
-    return HIST_BINS * 4 + 64 * 4 + m2 * 8 + (size_t)tail_cap * 8;
+    return select_layout(K, tail_cap, 0, 0, false).total;
 }
 
-cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
-    if (p.nrows <= 0) return cudaSuccess;
-    const size_t smem = select_smem_bytes(p.K, p.tail_cap);
-    cudaError_t e =
-        cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+cudaError_t launch_select(const SelectParams& p_in, cudaStream_t stream) {
+    if (p_in.nrows <= 0) return cudaSuccess;
+    SelectParams p = p_in;
+    p.bitmap_words = (p.npos + 31) / 32;
+    p.fast_cap = select_fast_cap(p.K);
+    SelectLayout lay = select_layout(p.K, p.tail_cap, p.fast_cap, p.bitmap_words, p.split > 0);
+    if (lay.total > SELECT_SMEM_LIMIT) {   // rows too long for the bitmaps: exact path only
+        p.fast_cap = 0;
+        lay = select_layout(p.K, p.tail_cap, 0, p.bitmap_words, p.split > 0);
+    }
+    if (lay.total > SELECT_SMEM_LIMIT) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)lay.total);
     if (e != cudaSuccess) return e;
-    select_kernel<<<p.nrows, SEL_THREADS, smem, stream>>>(p);
+    select_kernel<<<p.nrows, SEL_THREADS, lay.total, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -73,7 +73,7 @@ def load(path: str = LIB_PATH):
         "pivot_dense_index": ([P, I32, P, P, P, SZ, P], I32),
         "pivot_dense_index_workspace_size": ([P, I32], SZ),
         "pivot_proxy_reduce": ([P, I32, P, P, P, P], I32),
-        "pivot_proxy_scan": ([P, I32, P, P, P, I32, P, P, P, SZ, P], I32),
+        "pivot_proxy_scan": ([P, I32, P, P, P, I32, I32, P, P, P, SZ, P], I32),
         "pivot_proxy_scan_workspace_size": ([P, I32, I32], SZ),
         "pivot_reuse": ([I32, I32, I32, P, I32, I32, P, P], I32),
         "pivot_refine": ([P, I32, P, I32, I32, P, P, P, SZ, P], I32),
@@ -114,9 +114,9 @@ def pivot_proxy_reduce(seq, g, pq, pq_scale, pw, stream):
     return load().pivot_proxy_reduce(ctypes.byref(seq), g, pq, pq_scale, pw, stream)
 
 
-def pivot_proxy_scan(seq, g, pq, pq_scale, pw, C, cand, cand_score, ws, ws_bytes, stream):
-    return load().pivot_proxy_scan(ctypes.byref(seq), g, pq, pq_scale, pw, C, cand, cand_score,
-                                   ws, ws_bytes, stream)
+def pivot_proxy_scan(seq, g, pq, pq_scale, pw, C, topk, cand, cand_score, ws, ws_bytes, stream):
+    return load().pivot_proxy_scan(ctypes.byref(seq), g, pq, pq_scale, pw, C, topk, cand,
+                                   cand_score, ws, ws_bytes, stream)
 
 
 def pivot_proxy_scan_workspace_size(seq, g, C):
@@ -271,14 +271,16 @@ def proxy_reduce(seq: PivotSeq, g, stream=None, device="cuda"):
     return pq, pqs, pw
 
 
-def proxy_scan(seq: PivotSeq, g, pq, pqs, pw, C, with_score=False, ws=None, stream=None,
+def proxy_scan(seq: PivotSeq, g, pq, pqs, pw, C, topk, with_score=False, ws=None, stream=None,
                device="cuda"):
+    """Candidates [G, C]: each proxy's top-topk positions, then the rest of
+    its top-C, each ascending."""
     G = pq.shape[0]
     cand = torch.empty(G, C, dtype=torch.int32, device=device)
     cs = torch.empty(G, C, dtype=torch.float32, device=device) if with_score else None
     if ws is None:
         ws = _workspace(pivot_proxy_scan_workspace_size(seq, g, C), device)
-    _check(pivot_proxy_scan(seq, g, _p(pq), _p(pqs), _p(pw), C, _p(cand), _p(cs), _p(ws),
+    _check(pivot_proxy_scan(seq, g, _p(pq), _p(pqs), _p(pw), C, topk, _p(cand), _p(cs), _p(ws),
                             ws.numel(), _stream(stream)), "pivot_proxy_scan")
     return cand, cs
 
