@@ -21,13 +21,17 @@
 // through a TMA ring.  Accumulators are double-buffered in TMEM (2 x 256
 // columns) so the epilogue of tile i overlaps the MMAs of tile i+1.
 //
-// Warp roles (192 threads): warp 0 loads (one lane issuing TMA in scan mode;
+// Warp roles (320 threads): warp 0 loads (one lane issuing TMA in scan mode;
 // all 32 lanes copying in gather mode), warp 1 allocates TMEM and issues
-// tcgen05.mma, warps 2-5 run the epilogue.
+// tcgen05.mma, warps 2-9 run the epilogue (two warps per TMEM lane quarter,
+// each reducing half of the rows).
 #include "common.cuh"
 #include "kernels.h"
 
 namespace pivot {
+
+constexpr int EPI_WARPS = 8;                        // epilogue warps (2 per TMEM lane quarter)
+constexpr int SCAN_THREADS = 64 + EPI_WARPS * 32;   // + producer warp + MMA warp
 
 __device__ __forceinline__ int scan_row_lim(const ScanParams& p, int r, bool& ok) {
     ok = true;
@@ -108,7 +112,7 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
 }
 
 template <int KIND, int HEADS, int ROWB, bool GATHER>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(SCAN_THREADS, 1)
     index_umma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
     constexpr int KBLK = ROWB / 128;           // 128-byte K blocks per row
@@ -132,8 +136,9 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* accfull = bempty + 2;                       // [2]
     uint64_t* accempty = accfull + 2;                     // [2]
     uint64_t* drain = accempty + 2;                       // [1]
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-    float* w_s = reinterpret_cast<float*>(tmem_holder + 4);   // [256]
+    // barriers take at most 2*6+9 = 21 words of the 256 bytes reserved
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + 256);
+    float* w_s = reinterpret_cast<float*>(tmem_holder + 4);   // [256], 16-byte aligned
     float* sq_s = w_s + 256;                                   // [PMAX]
     int* lim_s = reinterpret_cast<int*>(sq_s + PMAX);          // [PMAX]
 
@@ -150,7 +155,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&bfull[i], 1);
             mbar_init(&bempty[i], 1);
             mbar_init(&accfull[i], 1);
-            mbar_init(&accempty[i], 4);   // one arrive per epilogue warp
+            mbar_init(&accempty[i], EPI_WARPS);   // one arrive per epilogue warp
         }
         mbar_init(drain, 1);
         fence_barrier_init();
@@ -330,29 +335,42 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else {
         // ------------------------------------------------------- epilogue
-        const int ew = warp - 2;                  // 0..3
+        // Eight warps: two per TMEM lane quarter.  With H >= 32 the rows of
+        // the block are split between the two halves (each row's H columns
+        // are reduced by one thread); with H < 32 the first half does all
+        // rows in 32-column chunks and the second half only keeps step.
+        const int e = warp - 2;                   // 0..7
         const int quarter = warp & 3;             // TMEM lane quarter of this warp
+        const int half = e >> 2;
         const int key_in_tile = quarter * 32 + lane;
-        const int et = ew * 32 + lane;            // 0..127
+        const int et = e * 32 + lane;             // 0..255
+        int r_lo = 0, r_hi = 0;
+        if constexpr (HEADS >= 32) {
+            const int Ph = (p.P + 1) / 2;
+            r_lo = half * Ph;
+            r_hi = r_lo + Ph < p.P ? r_lo + Ph : p.P;
+        } else {
+            r_hi = half == 0 ? p.P : 0;
+        }
         int ntile = 0;
         // Once a wait runs out the warp stops touching TMEM and memory but
-        // keeps walking the items, so the named barriers shared by the four
+        // keeps walking the items, so the named barriers shared by the
         // epilogue warps are always reached.
         bool aborted = false;
         for (int item = blockIdx.x; item < p.nitems; item += gridDim.x) {
             ItemInfo it = scan_item<GATHER>(p, item);
             if (!it.valid) continue;
-            named_bar_sync(1, 128);
+            named_bar_sync(1, EPI_WARPS * 32);
             // The tables span all 256 columns / PMAX rows: a TMEM load covers
             // 32 columns even when N is 16, and the columns past N must map
             // to masked rows (lim -1) with zero weights.
-            for (int i = et; i < 256; i += 128) {
+            for (int i = et; i < 256; i += EPI_WARPS * 32) {
                 const int pr = i / HEADS;
                 w_s[i] = (i < N && pr < it.rows)
                              ? p.w[(size_t)(it.row_first + pr - p.qrow_base) * HEADS + i % HEADS]
                              : 0.0f;
             }
-            for (int pr = et; pr < PMAX; pr += 128) {
+            for (int pr = et; pr < PMAX; pr += EPI_WARPS * 32) {
                 bool ok = true;
                 int lim = -1;
                 // gather mode: every candidate slot is written (the selection
@@ -363,57 +381,83 @@ __global__ void __launch_bounds__(192, 1)
                                ? p.q_scale[it.row_first + pr - p.qrow_base]
                                : 1.0f;
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, EPI_WARPS * 32);
+            // key scale of this thread's key in tile t (1 where none)
+            auto key_scale = [&](int t) -> float {
+                if (!p.k_scale) return 1.0f;
+                const int s_t = t * 128 + key_in_tile;
+                int keyrow = -1;
+                if constexpr (GATHER) {
+                    const int pos = s_t < p.C ? it.cand[s_t] : -1;
+                    if (pos >= 0 && pos < p.nkeys) keyrow = it.keybase + pos;
+                } else {
+                    if (s_t <= it.maxlim) keyrow = it.keybase + s_t;
+                }
+                return keyrow >= 0 ? __ldg(p.k_scale + keyrow) : 1.0f;
+            };
+            float sk_next = key_scale(it.t0);
             for (int t = it.t0; t < it.t1; ++t) {
                 const int acc = ntile & 1;
                 const uint32_t aph = (ntile >> 1) & 1;
                 ++ntile;
+                const float sk = sk_next;                  // prefetched a tile ahead
+                if (t + 1 < it.t1) sk_next = key_scale(t + 1);
                 if (aborted) continue;
                 const bool got = mbar_wait(&accfull[acc], aph);
                 if (!__all_sync(0xffffffffu, got)) { aborted = true; continue; }
                 tc_fence_after();
                 // s: the output column (key position in scan mode, candidate
-                // slot in gather mode); keyrow: the key's row for its scale
+                // slot in gather mode)
                 const int s = t * 128 + key_in_tile;
-                int keyrow = -1;
-                if constexpr (GATHER) {
-                    const int pos = s < p.C ? it.cand[s] : -1;
-                    if (pos >= 0 && pos < p.nkeys) keyrow = it.keybase + pos;
-                } else {
-                    if (s <= it.maxlim) keyrow = it.keybase + s;
-                }
                 const bool col_ok = GATHER ? (s < p.C) : true;
-                const float sk = (p.k_scale && keyrow >= 0) ? p.k_scale[keyrow] : 1.0f;
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * 256);
-                float rowacc = 0.0f;
-                float v[32];
-#pragma unroll 1
-                for (int c0 = 0; c0 < N; c0 += 32) {
-                    tmem_ld32(taddr + c0, v);
-                    tmem_ld_wait();
-                    if constexpr (HEADS <= 32) {
+                if constexpr (HEADS >= 32) {
+                    for (int pr = r_lo; pr < r_hi; ++pr) {
+                        float v[HEADS];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            rowacc = fmaf(w_s[c0 + i], fmaxf(v[i], 0.0f), rowacc);
-                            if ((i + 1) % HEADS == 0) {
-                                const int pr = (c0 + i) / HEADS;
-                                if (col_ok && s <= lim_s[pr])
-                                    p.S[(size_t)(it.row_first + pr - p.row0) * p.S_stride + s] =
-                                        rowacc * sq_s[pr] * sk;
-                                rowacc = 0.0f;
-                            }
+                        for (int c = 0; c < HEADS / 32; ++c)
+                            tmem_ld32(taddr + (uint32_t)(pr * HEADS + c * 32), v + c * 32);
+                        tmem_ld_wait();
+                        // eight independent partial sums keep the FMA pipe busy
+                        float a[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) a[j] = 0.0f;
+                        const float4* w4 = reinterpret_cast<const float4*>(w_s + pr * HEADS);
+#pragma unroll
+                        for (int i4 = 0; i4 < HEADS / 4; ++i4) {
+                            const float4 wv = w4[i4];
+                            const int b = (4 * i4) & 7;
+                            a[b + 0] = fmaf(wv.x, fmaxf(v[4 * i4 + 0], 0.0f), a[b + 0]);
+                            a[b + 1] = fmaf(wv.y, fmaxf(v[4 * i4 + 1], 0.0f), a[b + 1]);
+                            a[b + 2] = fmaf(wv.z, fmaxf(v[4 * i4 + 2], 0.0f), a[b + 2]);
+                            a[b + 3] = fmaf(wv.w, fmaxf(v[4 * i4 + 3], 0.0f), a[b + 3]);
                         }
-                    } else {
+                        const float rowsum = ((a[0] + a[1]) + (a[2] + a[3])) +
+                                             ((a[4] + a[5]) + (a[6] + a[7]));
+                        if (col_ok && s <= lim_s[pr])
+                            p.S[(size_t)(it.row_first + pr - p.row0) * p.S_stride + s] =
+                                rowsum * sq_s[pr] * sk;
+                    }
+                } else {
+                    if (r_hi > 0) {
+                        float rowacc = 0.0f;
+                        float v[32];
+#pragma unroll 1
+                        for (int c0 = 0; c0 < N; c0 += 32) {
+                            tmem_ld32(taddr + c0, v);
+                            tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            rowacc = fmaf(w_s[c0 + i], fmaxf(v[i], 0.0f), rowacc);
-                        if ((c0 + 32) % HEADS == 0) {
-                            const int pr = c0 / HEADS;
-                            if (col_ok && s <= lim_s[pr])
-                                p.S[(size_t)(it.row_first + pr - p.row0) * p.S_stride + s] =
-                                    rowacc * sq_s[pr] * sk;
-                            rowacc = 0.0f;
+                            for (int i = 0; i < 32; ++i) {
+                                rowacc = fmaf(w_s[c0 + i], fmaxf(v[i], 0.0f), rowacc);
+                                if ((i + 1) % HEADS == 0) {
+                                    const int pr = (c0 + i) / HEADS;
+                                    if (col_ok && s <= lim_s[pr])
+                                        p.S[(size_t)(it.row_first + pr - p.row0) * p.S_stride +
+                                            s] = rowacc * sq_s[pr] * sk;
+                                    rowacc = 0.0f;
+                                }
+                            }
                         }
                     }
                 }
@@ -436,7 +480,7 @@ int scan_smem_bytes(int row_bytes) {
     const int stages = row_bytes == 128 ? 6 : 3;
     const int pmax = 64;
     return 1024 /*align slack*/ + 2 * 256 * row_bytes + stages * 128 * row_bytes +
-           (2 * stages + 9) * 8 + 16 + 256 * 4 + pmax * 8;
+           256 /*barriers*/ + 16 /*TMEM address*/ + 256 * 4 + pmax * 8;
 }
 
 template <int KIND, int HEADS, bool GATHER>
@@ -447,13 +491,13 @@ static cudaError_t launch_heads(const CUtensorMap& tk, const CUtensorMap& tq, co
         const int smem = scan_smem_bytes(128);
         cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        kfn<<<grid, 192, smem, stream>>>(tk, tq, p);
+        kfn<<<grid, SCAN_THREADS, smem, stream>>>(tk, tq, p);
     } else {
         auto kfn = index_umma_kernel<KIND, HEADS, 256, GATHER>;
         const int smem = scan_smem_bytes(256);
         cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        kfn<<<grid, 192, smem, stream>>>(tk, tq, p);
+        kfn<<<grid, SCAN_THREADS, smem, stream>>>(tk, tq, p);
     }
     return cudaGetLastError();
 }
