@@ -229,6 +229,9 @@ pivot_status_t pivot_profile_read(int32_t kernel, int64_t* launches, double* tot
 int64_t pivot_launch_count(void);
 
 const char* pivot_status_string(pivot_status_t status);
+/* The CUDA error behind the last PIVOT_ERR_CUDA returned on this host
+ * thread ("name: message"). */
+const char* pivot_last_error_detail(void);
 int32_t pivot_version(void);
 
 #ifdef __cplusplus

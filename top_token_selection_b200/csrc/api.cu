@@ -1,5 +1,6 @@
 // api.cu -- the libpivot C ABI: argument checks, workspace carving, TMA
 // descriptors and kernel launches.  See include/pivot.h for the contract.
+#include <cstdio>
 #include <mutex>
 
 #include "common.cuh"
@@ -117,7 +118,14 @@ pivot_status_t check_group_range(const pivot_seq_t* s, int g, int t0, int t1) {
     return PIVOT_OK;
 }
 
-pivot_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? PIVOT_OK : PIVOT_ERR_CUDA; }
+thread_local char g_last_detail[256] = "no CUDA error recorded";
+
+pivot_status_t from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return PIVOT_OK;
+    snprintf(g_last_detail, sizeof(g_last_detail), "%s: %s", cudaGetErrorName(e),
+             cudaGetErrorString(e));
+    return PIVOT_ERR_CUDA;
+}
 
 long long score_stride(int nkeys) { return (long long)align_up((size_t)nkeys, 32); }
 
@@ -203,8 +211,12 @@ pivot_status_t run_scan(int kind, int dtype, int H, int D, const void* qbase, lo
                               [&] { return launch_scan_simt(qbase, kbase, p, st); }));
 }
 
+// Rows of a tensor-core block: N = rows * H columns, 192 for H >= 32 (one
+// row per epilogue warp at H = 64), 256 for smaller H.
+int umma_rows(int H) { return (H >= 32 ? 192 : 256) / H; }
+
 int rows_per_block(int H, int D, int dtype) {
-    return umma_shape_ok(H, D, dtype) ? 256 / H : 8;
+    return umma_shape_ok(H, D, dtype) ? umma_rows(H) : 8;
 }
 
 pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, int Gm, int maxlen,
@@ -271,7 +283,7 @@ pivot_status_t run_refine_scores(int kind, int dtype, int H, int D, const void* 
                                  int C, int r0, int r1, float* S, cudaStream_t st) {
     const double work = kind == SCAN_PREFILL_DENSE ? refine_pairs(r0, r1, C) : 0.0;
     const int gsize = kind == SCAN_DECODE_DENSE ? Gm : g;
-    int P = umma_shape_ok(H, D, dtype) ? 256 / H : 0;
+    int P = umma_shape_ok(H, D, dtype) ? umma_rows(H) : 0;
     if (P > gsize) P = gsize;
     const int N = P * H;
     if (P > 0 && N >= 16 && N <= 256 && N % 16 == 0) {
@@ -381,6 +393,8 @@ using namespace pivot;
 extern "C" {
 
 int32_t pivot_version(void) { return PIVOT_VERSION; }
+
+const char* pivot_last_error_detail(void) { return g_last_detail; }
 
 const char* pivot_status_string(pivot_status_t s) {
     switch (s) {

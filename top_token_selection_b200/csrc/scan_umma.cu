@@ -21,17 +21,24 @@
 // through a TMA ring.  Accumulators are double-buffered in TMEM (2 x 256
 // columns) so the epilogue of tile i overlaps the MMAs of tile i+1.
 //
-// Warp roles (320 threads): warp 0 loads (one lane issuing TMA in scan mode;
+// Warp roles (448 threads): warp 0 loads (one lane issuing TMA in scan mode;
 // all 32 lanes copying in gather mode), warp 1 allocates TMEM and issues
-// tcgen05.mma, warps 2-9 run the epilogue (two warps per TMEM lane quarter,
-// each reducing half of the rows).
+// tcgen05.mma, warps 2-13 run the epilogue (three warps per TMEM lane
+// quarter, each reducing a third of the rows; at H = 64 the block has 3
+// rows, N = 192, and every epilogue warp owns one row whose 64 head weights
+// stay in registers -- reloading them from shared memory every tile competed
+// with the tensor cores' operand reads).
 #include "common.cuh"
 #include "kernels.h"
 
 namespace pivot {
 
-constexpr int EPI_WARPS = 8;                        // epilogue warps (2 per TMEM lane quarter)
-constexpr int SCAN_THREADS = 64 + EPI_WARPS * 32;   // + producer warp + MMA warp
+constexpr int EPI_GROUPS = 3;                       // epilogue warps per TMEM lane quarter
+constexpr int EPI_WARPS = 4 * EPI_GROUPS;           // 12
+constexpr int SCAN_THREADS = 64 + EPI_WARPS * 32;   // + producer warp + MMA warp = 448
+// Register files are per SM sub-partition (16K each); warp w runs on
+// sub-partition w % 4, so 14 warps put at most 4 on one: 128 registers.
+constexpr int SCAN_MAXREG = 128;
 
 __device__ __forceinline__ int scan_row_lim(const ScanParams& p, int r, bool& ok) {
     ok = true;
@@ -112,7 +119,7 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
 }
 
 template <int KIND, int HEADS, int ROWB, bool GATHER>
-__global__ void __launch_bounds__(SCAN_THREADS, 1)
+__global__ void __maxnreg__(SCAN_MAXREG)
     index_umma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
     constexpr int KBLK = ROWB / 128;           // 128-byte K blocks per row
@@ -335,23 +342,28 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
         }
     } else {
         // ------------------------------------------------------- epilogue
-        // Eight warps: two per TMEM lane quarter.  With H >= 32 the rows of
-        // the block are split between the two halves (each row's H columns
-        // are reduced by one thread); with H < 32 the first half does all
-        // rows in 32-column chunks and the second half only keeps step.
-        const int e = warp - 2;                   // 0..7
+        // EPI_GROUPS warps per TMEM lane quarter.  With H >= 32 the rows of
+        // the block are split between the groups (each row's H columns are
+        // reduced by one thread, weights in registers); with H < 32 the first
+        // group does all rows in 32-column chunks (weights from shared
+        // memory) and the others only keep step.
+        const int e = warp - 2;                   // 0..EPI_WARPS-1
         const int quarter = warp & 3;             // TMEM lane quarter of this warp
-        const int half = e >> 2;
+        const int grp = e >> 2;                   // 0..EPI_GROUPS-1
         const int key_in_tile = quarter * 32 + lane;
-        const int et = e * 32 + lane;             // 0..255
+        const int et = e * 32 + lane;
         int r_lo = 0, r_hi = 0;
         if constexpr (HEADS >= 32) {
-            const int Ph = (p.P + 1) / 2;
-            r_lo = half * Ph;
-            r_hi = r_lo + Ph < p.P ? r_lo + Ph : p.P;
+            const int Pg = (p.P + EPI_GROUPS - 1) / EPI_GROUPS;   // <= 64 / HEADS
+            r_lo = grp * Pg < p.P ? grp * Pg : p.P;
+            r_hi = r_lo + Pg < p.P ? r_lo + Pg : p.P;
         } else {
-            r_hi = half == 0 ? p.P : 0;
+            r_hi = grp == 0 ? p.P : 0;
         }
+        constexpr int RROWS = HEADS >= 32 ? 64 / HEADS : 1;      // rows per warp at most
+        float wr[HEADS >= 32 ? 64 : 1];
+        int lim_r[RROWS];
+        float sq_r[RROWS];
         int ntile = 0;
         // Once a wait runs out the warp stops touching TMEM and memory but
         // keeps walking the items, so the named barriers shared by the
@@ -360,28 +372,55 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
         for (int item = blockIdx.x; item < p.nitems; item += gridDim.x) {
             ItemInfo it = scan_item<GATHER>(p, item);
             if (!it.valid) continue;
-            named_bar_sync(1, EPI_WARPS * 32);
-            // The tables span all 256 columns / PMAX rows: a TMEM load covers
-            // 32 columns even when N is 16, and the columns past N must map
-            // to masked rows (lim -1) with zero weights.
-            for (int i = et; i < 256; i += EPI_WARPS * 32) {
-                const int pr = i / HEADS;
-                w_s[i] = (i < N && pr < it.rows)
-                             ? p.w[(size_t)(it.row_first + pr - p.qrow_base) * HEADS + i % HEADS]
-                             : 0.0f;
-            }
-            for (int pr = et; pr < PMAX; pr += EPI_WARPS * 32) {
+            // gather mode: every candidate slot is written (the selection
+            // drops empty slots and positions after the member)
+            auto row_lim = [&](int pr) -> int {
+                if (pr >= it.rows) return -1;
+                if (GATHER) return 0x7fffffff;
                 bool ok = true;
-                int lim = -1;
-                // gather mode: every candidate slot is written (the selection
-                // drops empty slots and positions after the member)
-                if (pr < it.rows) lim = GATHER ? 0x7fffffff : scan_row_lim(p, it.row_first + pr, ok);
-                lim_s[pr] = ok ? lim : -1;
-                sq_s[pr] = (p.q_scale && pr < it.rows)
-                               ? p.q_scale[it.row_first + pr - p.qrow_base]
-                               : 1.0f;
+                const int lim = scan_row_lim(p, it.row_first + pr, ok);
+                return ok ? lim : -1;
+            };
+            auto row_sq = [&](int pr) -> float {
+                return (p.q_scale && pr < it.rows) ? p.q_scale[it.row_first + pr - p.qrow_base]
+                                                   : 1.0f;
+            };
+            if constexpr (HEADS >= 32) {
+                // this warp's rows: weights, limits and query scales in registers
+#pragma unroll
+                for (int lr = 0; lr < RROWS; ++lr) {
+                    const int pr = r_lo + lr;
+                    const bool live = pr < r_hi && pr < it.rows;
+                    const float4* w4 = reinterpret_cast<const float4*>(
+                        p.w + (size_t)(it.row_first + pr - p.qrow_base) * HEADS);
+#pragma unroll
+                    for (int i4 = 0; i4 < HEADS / 4; ++i4) {
+                        const float4 wv = live ? __ldg(w4 + i4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        wr[lr * HEADS + 4 * i4 + 0] = wv.x;
+                        wr[lr * HEADS + 4 * i4 + 1] = wv.y;
+                        wr[lr * HEADS + 4 * i4 + 2] = wv.z;
+                        wr[lr * HEADS + 4 * i4 + 3] = wv.w;
+                    }
+                    lim_r[lr] = pr < r_hi ? row_lim(pr) : -1;
+                    sq_r[lr] = row_sq(pr);
+                }
+            } else {
+                named_bar_sync(1, EPI_WARPS * 32);
+                // The tables span all 256 columns / PMAX rows: a TMEM load
+                // covers 32 columns even when N is 16, and the columns past N
+                // must map to masked rows (lim -1) with zero weights.
+                for (int i = et; i < 256; i += EPI_WARPS * 32) {
+                    const int pr = i / HEADS;
+                    w_s[i] = (i < N && pr < it.rows)
+                                 ? p.w[(size_t)(it.row_first + pr - p.qrow_base) * HEADS + i % HEADS]
+                                 : 0.0f;
+                }
+                for (int pr = et; pr < PMAX; pr += EPI_WARPS * 32) {
+                    lim_s[pr] = row_lim(pr);
+                    sq_s[pr] = row_sq(pr);
+                }
+                named_bar_sync(1, EPI_WARPS * 32);
             }
-            named_bar_sync(1, EPI_WARPS * 32);
             // key scale of this thread's key in tile t (1 where none)
             auto key_scale = [&](int t) -> float {
                 if (!p.k_scale) return 1.0f;
@@ -413,31 +452,34 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * 256);
                 if constexpr (HEADS >= 32) {
-                    for (int pr = r_lo; pr < r_hi; ++pr) {
-                        float v[HEADS];
 #pragma unroll
-                        for (int c = 0; c < HEADS / 32; ++c)
-                            tmem_ld32(taddr + (uint32_t)(pr * HEADS + c * 32), v + c * 32);
-                        tmem_ld_wait();
-                        // eight independent partial sums keep the FMA pipe busy
-                        float a[8];
+                    for (int lr = 0; lr < RROWS; ++lr) {
+                        const int pr = r_lo + lr;
+                        if (pr >= r_hi) break;
+                        // four packed partial sums (two multiply-adds per instruction)
+                        uint64_t a[4];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) a[j] = 0.0f;
-                        const float4* w4 = reinterpret_cast<const float4*>(w_s + pr * HEADS);
+                        for (int j = 0; j < 4; ++j) a[j] = 0ull;
 #pragma unroll
-                        for (int i4 = 0; i4 < HEADS / 4; ++i4) {
-                            const float4 wv = w4[i4];
-                            const int b = (4 * i4) & 7;
-                            a[b + 0] = fmaf(wv.x, fmaxf(v[4 * i4 + 0], 0.0f), a[b + 0]);
-                            a[b + 1] = fmaf(wv.y, fmaxf(v[4 * i4 + 1], 0.0f), a[b + 1]);
-                            a[b + 2] = fmaf(wv.z, fmaxf(v[4 * i4 + 2], 0.0f), a[b + 2]);
-                            a[b + 3] = fmaf(wv.w, fmaxf(v[4 * i4 + 3], 0.0f), a[b + 3]);
+                        for (int c = 0; c < HEADS / 32; ++c) {
+                            float v[32];
+                            tmem_ld32(taddr + (uint32_t)(pr * HEADS + c * 32), v);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int wi = lr * HEADS + c * 32 + 2 * i;
+                                a[i & 3] = ffma2(pack2(fmaxf(v[2 * i], 0.0f), fmaxf(v[2 * i + 1], 0.0f)),
+                                                 pack2(wr[wi], wr[wi + 1]), a[i & 3]);
+                            }
                         }
-                        const float rowsum = ((a[0] + a[1]) + (a[2] + a[3])) +
-                                             ((a[4] + a[5]) + (a[6] + a[7]));
-                        if (col_ok && s <= lim_s[pr])
+                        float lo[4], hi[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) unpack2(a[j], lo[j], hi[j]);
+                        const float rowsum = ((lo[0] + hi[0]) + (lo[1] + hi[1])) +
+                                             ((lo[2] + hi[2]) + (lo[3] + hi[3]));
+                        if (col_ok && s <= lim_r[lr])
                             p.S[(size_t)(it.row_first + pr - p.row0) * p.S_stride + s] =
-                                rowsum * sq_s[pr] * sk;
+                                rowsum * sq_r[lr] * sk;
                     }
                 } else {
                     if (r_hi > 0) {

@@ -30,7 +30,7 @@ ABI_SYMBOLS = [
     "pivot_refine_workspace_size", "pivot_decode", "pivot_decode_workspace_size",
     "pivot_get_device_error", "pivot_set_wait_limit_ns", "pivot_selftest_wait_timeout",
     "pivot_status_string", "pivot_version", "pivot_profile_enable", "pivot_profile_read",
-    "pivot_launch_count", "pivot_decode_noalloc",
+    "pivot_launch_count", "pivot_decode_noalloc", "pivot_last_error_detail",
 ]
 KERNELS = {0: "scan", 1: "select", 2: "refine", 3: "reduce", 4: "reuse"}
 
@@ -89,6 +89,7 @@ def load(path: str = LIB_PATH):
         "pivot_profile_read": ([I32, P, P, P], I32),
         "pivot_launch_count": ([], ctypes.c_int64),
         "pivot_decode_noalloc": ([P, I32, I32, I32, P, P, P], I32),
+        "pivot_last_error_detail": ([], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -191,6 +192,10 @@ def pivot_version():
     return load().pivot_version()
 
 
+def pivot_last_error_detail():
+    return load().pivot_last_error_detail().decode()
+
+
 # ---------------------------------------------------------------------------
 # torch marshalling helpers
 # ---------------------------------------------------------------------------
@@ -220,6 +225,8 @@ def _stream(stream):
 
 def _check(status, what):
     if status != 0:
+        if status == 4:
+            what = f"{what} [{pivot_last_error_detail()}]"
         raise PivotError(status, what)
 
 
