@@ -261,20 +261,35 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                                     kb * (128 / p.esize), qrow);
                 }
                 last_b[slot] = (int)bph;
+                // candidate positions of a tile: lane l holds slots l + 32 j
+                // (j < 4), read one tile ahead so no copy waits on them
+                auto tile_pos = [&](int t, int (&pp)[4]) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int slot_r = t * 128 + j * 32 + lane;
+                        pp[j] = slot_r < p.C ? it.cand[slot_r] : -1;
+                    }
+                };
+                int cur[4], nxt[4];
+                tile_pos(it.t0, nxt);
                 for (int t = it.t0; t < it.t1; ++t) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
+                    if (t + 1 < it.t1) tile_pos(t + 1, nxt);
                     if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1))) {
                         aborted = true;
                         break;
                     }
                     const uint32_t dst = smem_u32(sA + stage * A_BYTES);
                     // 32 lanes cover 4 rows x 8 chunks per step; a 128-row
-                    // tile of one 128-byte K block takes 32 steps
-#pragma unroll 4
+                    // tile of one 128-byte K block takes 32 steps.  Row r of
+                    // step s is slot 4 s + lane / 8, held by lane r % 32 in
+                    // cur[r / 32] (r / 32 = s / 8 for every lane of the step).
+#pragma unroll
                     for (int step = 0; step < 32; ++step) {
                         const int r = step * 4 + (lane >> 3);
                         const int c = lane & 7;
-                        const int slot_r = t * 128 + r;
-                        const int pos = slot_r < p.C ? it.cand[slot_r] : -1;
+                        const int pos = __shfl_sync(0xffffffffu, cur[step >> 3], r & 31);
                         const size_t row = (size_t)(it.keybase + ((pos >= 0 && pos < p.nkeys) ? pos : 0));
                         const uint8_t* src = kbytes + row * ROWB + c * 16;
 #pragma unroll
@@ -421,26 +436,34 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 }
                 named_bar_sync(1, EPI_WARPS * 32);
             }
-            // key scale of this thread's key in tile t (1 where none)
-            auto key_scale = [&](int t) -> float {
-                if (!p.k_scale) return 1.0f;
+            // Key scale of this thread's key in tile t (1 where none).  The
+            // scale is read a tile ahead; in gather mode the key's position
+            // (the candidate slot's entry) is read two tiles ahead, so
+            // neither read waits on the other.
+            auto slot_pos = [&](int t) -> int {
                 const int s_t = t * 128 + key_in_tile;
+                return (GATHER && p.k_scale && t < it.t1 && s_t < p.C) ? it.cand[s_t] : -1;
+            };
+            auto key_scale = [&](int t, int pos) -> float {
+                if (!p.k_scale) return 1.0f;
                 int keyrow = -1;
                 if constexpr (GATHER) {
-                    const int pos = s_t < p.C ? it.cand[s_t] : -1;
                     if (pos >= 0 && pos < p.nkeys) keyrow = it.keybase + pos;
                 } else {
+                    const int s_t = t * 128 + key_in_tile;
                     if (s_t <= it.maxlim) keyrow = it.keybase + s_t;
                 }
                 return keyrow >= 0 ? __ldg(p.k_scale + keyrow) : 1.0f;
             };
-            float sk_next = key_scale(it.t0);
+            float sk_next = key_scale(it.t0, slot_pos(it.t0));
+            int pos_next = slot_pos(it.t0 + 1);            // position for tile t + 1
             for (int t = it.t0; t < it.t1; ++t) {
                 const int acc = ntile & 1;
                 const uint32_t aph = (ntile >> 1) & 1;
                 ++ntile;
                 const float sk = sk_next;                  // prefetched a tile ahead
-                if (t + 1 < it.t1) sk_next = key_scale(t + 1);
+                if (t + 1 < it.t1) sk_next = key_scale(t + 1, pos_next);
+                pos_next = slot_pos(t + 2);
                 if (aborted) continue;
                 const bool got = mbar_wait(&accfull[acc], aph);
                 if (!__all_sync(0xffffffffu, got)) { aborted = true; continue; }
