@@ -411,10 +411,11 @@ __global__ void __maxnreg__(SCAN_MAXREG)
 #pragma unroll
                     for (int i4 = 0; i4 < HEADS / 4; ++i4) {
                         const float4 wv = live ? __ldg(w4 + i4) : make_float4(0.f, 0.f, 0.f, 0.f);
-                        wr[lr * HEADS + 4 * i4 + 0] = wv.x;
-                        wr[lr * HEADS + 4 * i4 + 1] = wv.y;
-                        wr[lr * HEADS + 4 * i4 + 2] = wv.z;
-                        wr[lr * HEADS + 4 * i4 + 3] = wv.w;
+                        // halved: w * max(0, x) == (w / 2) * (x + |x|) exactly
+                        wr[lr * HEADS + 4 * i4 + 0] = 0.5f * wv.x;
+                        wr[lr * HEADS + 4 * i4 + 1] = 0.5f * wv.y;
+                        wr[lr * HEADS + 4 * i4 + 2] = 0.5f * wv.z;
+                        wr[lr * HEADS + 4 * i4 + 3] = 0.5f * wv.w;
                     }
                     lim_r[lr] = pr < r_hi ? row_lim(pr) : -1;
                     sq_r[lr] = row_sq(pr);
@@ -491,7 +492,10 @@ __global__ void __maxnreg__(SCAN_MAXREG)
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
                                 const int wi = lr * HEADS + c * 32 + 2 * i;
-                                a[i & 3] = ffma2(pack2(fmaxf(v[2 * i], 0.0f), fmaxf(v[2 * i + 1], 0.0f)),
+                                // x + |x| = 2 max(0, x): one add on the FMA pipe
+                                // instead of a half-rate max on the ALU pipe
+                                a[i & 3] = ffma2(pack2(v[2 * i] + fabsf(v[2 * i]),
+                                                       v[2 * i + 1] + fabsf(v[2 * i + 1])),
                                                  pack2(wr[wi], wr[wi + 1]), a[i & 3]);
                             }
                         }
