@@ -222,7 +222,7 @@ int rows_per_block(int H, int D, int dtype) {
 pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, int Gm, int maxlen,
                                  const int32_t* cache_len, const float* S, long long stride,
                                  int K, int split, int npos, int32_t* out, float* out_score,
-                                 int out_base, cudaStream_t st) {
+                                 int out_base, cudaStream_t st, uint32_t* thresh = nullptr) {
     SelectParams sp{};
     sp.split = split;
     sp.npos = npos;
@@ -242,6 +242,12 @@ pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, in
     sp.out_score = out_score;
     sp.out_base = out_base;
     sp.tail_cap = TAIL_CAP;
+    sp.thresh = thresh;
+    if (thresh) {   // a launch of its own (no work of its own: the select's bytes count once)
+        const pivot_status_t t = from_cuda(
+            profiled(PK_SELECT, 0.0, st, [&] { return launch_row_threshold(sp, thresh, st); }));
+        if (t != PIVOT_OK) return t;
+    }
     return from_cuda(profiled(PK_SELECT, scan_pairs(scan_kind, r0, r1, L, g), st,
                               [&] { return launch_select(sp, st); }));
 }
@@ -365,7 +371,9 @@ struct Carver {
     }
 };
 
-size_t dense_rowbytes(int L) { return (size_t)score_stride(L) * 4; }
+// A prefill score row in the workspace, plus the row's select bound (4 bytes
+// after all score rows of the chunk).
+size_t dense_rowbytes(int L) { return (size_t)score_stride(L) * 4 + 4; }
 
 // One thread waits on an mbarrier that nothing arrives on: the bounded wait
 // must run out, raise the timeout bit and let the kernel return.
@@ -455,10 +463,11 @@ pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* 
     if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
     const int P = rows_per_block(seq->H, seq->D, seq->dtype);
     const long long stride = score_stride(seq->L);
-    const long long chunk = chunk_rows(ws_bytes, (size_t)stride * 4, t1 - t0, P);
+    const long long chunk = chunk_rows(ws_bytes, dense_rowbytes(seq->L), t1 - t0, P);
     if (chunk < 1) return PIVOT_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* S = static_cast<float*>(ws);
+    uint32_t* thresh = reinterpret_cast<uint32_t*>(S + chunk * stride);
     for (long long c0 = t0; c0 < t1; c0 += chunk) {
         const int r0 = (int)c0;
         const int r1 = (int)(c0 + chunk < t1 ? c0 + chunk : t1);
@@ -467,7 +476,7 @@ pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* 
                       r1, r1 - 1, S, stride, s);
         if (st != PIVOT_OK) return st;
         st = run_select_prefix(SCAN_PREFILL_DENSE, r0, r1, seq->L, 1, 1, 0, nullptr, S, stride,
-                               topk, 0, seq->L, idx, score, t0, s);
+                               topk, 0, seq->L, idx, score, t0, s, thresh);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;
@@ -531,11 +540,12 @@ pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* p
     const int P = rows_per_block(seq->H, seq->D, seq->dtype);
     const long long stride = score_stride(seq->L);
     const int j0 = t0 / g, j1 = ceil_div(t1, g);
-    const long long chunk = chunk_rows(ws_bytes, (size_t)stride * 4, j1 - j0, P);
+    const long long chunk = chunk_rows(ws_bytes, dense_rowbytes(seq->L), j1 - j0, P);
     if (chunk < 1) return PIVOT_ERR_WORKSPACE;
     const int G = j1 - j0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* S = static_cast<float*>(ws);
+    uint32_t* thresh = reinterpret_cast<uint32_t*>(S + chunk * stride);
     for (long long c0 = j0; c0 < j1; c0 += chunk) {
         const int r0 = (int)c0;
         const int r1 = (int)(c0 + chunk < j1 ? c0 + chunk : j1);
@@ -545,7 +555,7 @@ pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* p
                       stride, s);
         if (st != PIVOT_OK) return st;
         st = run_select_prefix(SCAN_PREFILL_PROXY, r0, r1, seq->L, g, 1, 0, nullptr, S, stride, C,
-                               topk, seq->L, cand, cand_score, j0, s);
+                               topk, seq->L, cand, cand_score, j0, s, thresh);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;

@@ -74,9 +74,14 @@ struct SelectParams {
     int npos;             // positions are < npos (bitmap size)
     int fast_cap;         // set by launch_select: kept-entry capacity of the fast path
     int bitmap_words;     // set by launch_select
+    const uint32_t* thresh;   // SEL_PREFIX: row r's lower bound at thresh[r - row0]
+                              // (launch_row_threshold), or NULL: sampled in the select
 };
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
+// SEL_PREFIX rows: per-row lower bound for the select's fast path, written
+// to thresh[r - row0] (one warp per row; p.thresh is ignored).
+cudaError_t launch_row_threshold(const SelectParams& p, uint32_t* thresh, cudaStream_t stream);
 size_t select_smem_bytes(int K, int tail_cap);
 
 struct ReduceParams {

@@ -341,7 +341,9 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
     uint64_t* buf = sm.buf;
     if (threadIdx.x == 0) { *s_cnt = 0; *s_valid = 0; }
     uint32_t T = 1;
-    if (v.n > cap) {
+    if (p.thresh) {
+        T = p.thresh[blockIdx.x];   // row r = row0 + blockIdx.x
+    } else if (v.n > cap) {
         for (int j = threadIdx.x; j < SAMPLES; j += SEL_THREADS)
             hist[j] = entry_key32(v, (int)(((long long)j * v.n) / SAMPLES));
         __syncthreads();
@@ -367,18 +369,40 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
     if (vec) {
         const int n4 = v.n / 4;
         const float4* S4 = reinterpret_cast<const float4*>(v.S);
-#pragma unroll 2
-        for (int i0 = 0; i0 < n4; i0 += SEL_THREADS) {
-            const int i = i0 + threadIdx.x;
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            const bool a = i < n4;
-            if (a) x = __ldcs(S4 + i);
-            const uint32_t u0 = ordered_key(x.x), u1 = ordered_key(x.y);
-            const uint32_t u2 = ordered_key(x.z), u3 = ordered_key(x.w);
-            warp_append(buf, s_cnt, cap, make_key(u0, 4 * i + 0), a && u0 >= T);
-            warp_append(buf, s_cnt, cap, make_key(u1, 4 * i + 1), a && u1 >= T);
-            warp_append(buf, s_cnt, cap, make_key(u2, 4 * i + 2), a && u2 >= T);
-            warp_append(buf, s_cnt, cap, make_key(u3, 4 * i + 3), a && u3 >= T);
+        // Entries are compared as floats: for finite scores, key >= T exactly
+        // when score >= key_to_float(T) (-0 and +0 alike); a bound at or
+        // below the key of -FLT_MAX keeps every finite score.  Each thread
+        // takes two float4 per step and reserves room for all its kept
+        // entries with one shared-memory atomic (a few entries in a hundred
+        // pass, so the atomics rarely collide).
+        const float Tf = T <= 0x00800000u ? -INFINITY : key_to_float(T);
+        for (int i0 = 0; i0 < n4; i0 += 2 * SEL_THREADS) {
+            const int ia = i0 + threadIdx.x, ib = ia + SEL_THREADS;
+            const bool a = ia < n4, b = ib < n4;
+            const float4 xa = a ? __ldcs(S4 + ia) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 xb = b ? __ldcs(S4 + ib) : make_float4(0.f, 0.f, 0.f, 0.f);
+            uint32_t m = 0;
+            if (a) {
+                m |= (xa.x >= Tf ? 1u : 0u) | (xa.y >= Tf ? 2u : 0u) | (xa.z >= Tf ? 4u : 0u) |
+                     (xa.w >= Tf ? 8u : 0u);
+            }
+            if (b) {
+                m |= (xb.x >= Tf ? 16u : 0u) | (xb.y >= Tf ? 32u : 0u) | (xb.z >= Tf ? 64u : 0u) |
+                     (xb.w >= Tf ? 128u : 0u);
+            }
+            if (m) {
+                uint32_t slot = atomicAdd(s_cnt, (uint32_t)__popc(m));
+                do {
+                    const int e = __ffs(m) - 1;
+                    m &= m - 1;
+                    const float4& x = e < 4 ? xa : xb;
+                    const int c = e & 3;
+                    const float f = c == 0 ? x.x : (c == 1 ? x.y : (c == 2 ? x.z : x.w));
+                    const int pos = 4 * (e < 4 ? ia : ib) + c;
+                    if (slot < (uint32_t)cap) buf[slot] = make_key(ordered_key(f), pos);
+                    ++slot;
+                } while (m);
+            }
         }
         const int i = n4 * 4 + threadIdx.x;
         const bool a = threadIdx.x < 4 && i < v.n;
@@ -608,6 +632,134 @@ __device__ void select_exact(const SelectParams& p, const RowView& v, uint32_t* 
     }
 }
 
+// ------------------------------------------------------------ per-row bound
+//
+// The fast path's lower bound T for prefix rows, computed ahead of the
+// select by one warp per row: the m-th largest of 2048 sampled scores (64
+// evenly spread runs of 32 consecutive entries), m set so about
+// SAMPLE_MARGIN K entries of the row should lie at or above it; 1 (keep
+// everything) when the row fits the fast path's buffer.  Exact m-th by
+// histograms over 256 power-of-two-wide bins of the remaining key range.
+
+constexpr int THR_WARPS = 8;           // rows per CTA
+constexpr int THR_RUNS = 64;
+constexpr int THR_SAMPLES = THR_RUNS * 32;
+constexpr int THR_BINS = 256;
+constexpr size_t THR_SMEM_WARP = (size_t)(THR_SAMPLES + THR_BINS) * 4;
+
+__device__ __forceinline__ uint32_t warp_min_u32(uint32_t x) {
+    for (int o = 16; o > 0; o >>= 1) x = min(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t x) {
+    for (int o = 16; o > 0; o >>= 1) x = max(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+// The m-th largest of the nonzero values v[0..n), 1 <= m <= their count, by
+// one warp; v and hist (THR_BINS words) in this warp's shared memory.
+__device__ uint32_t warp_kth_largest(const uint32_t* v, int n, uint32_t m, uint32_t* hist) {
+    const int lane = threadIdx.x & 31;
+    uint32_t lo = 0xFFFFFFFFu, hi = 0;
+    for (int i = lane; i < n; i += 32) {
+        const uint32_t u = v[i];
+        if (u) { lo = min(lo, u); hi = max(hi, u); }
+    }
+    lo = warp_min_u32(lo);
+    hi = warp_max_u32(hi);
+    uint32_t remaining = m;
+    while (lo < hi) {
+        // bins of width 2^sh: the smallest sh with (hi - lo) >> sh < THR_BINS
+        const uint32_t span = hi - lo;
+        int sh = (32 - __clz(span)) - 8;
+        if (sh < 0) sh = 0;
+#pragma unroll
+        for (int b = 0; b < THR_BINS / 32; ++b) hist[b * 32 + lane] = 0;
+        __syncwarp();
+        for (int i = lane; i < n; i += 32) {
+            const uint32_t u = v[i];
+            if (u && u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> sh], 1u);
+        }
+        __syncwarp();
+        // lane l owns the 8 bins [THR_BINS - 8 (l + 1), THR_BINS - 8 l)
+        constexpr int PER = THR_BINS / 32;
+        const int top = THR_BINS - lane * PER;
+        uint32_t c[PER];
+        uint32_t local = 0;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            c[j] = hist[top - 1 - j];
+            local += c[j];
+        }
+        uint32_t inc = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        const uint32_t before = inc - local;
+        const bool mine = before < remaining && inc >= remaining;
+        int b = 0;
+        uint32_t above = 0;
+        if (mine) {
+            uint32_t acc = before;
+#pragma unroll
+            for (int j = 0; j < PER; ++j) {
+                if (acc + c[j] >= remaining) {
+                    b = top - 1 - j;
+                    above = acc;
+                    break;
+                }
+                acc += c[j];
+            }
+        }
+        const unsigned who = __ballot_sync(0xffffffffu, mine);
+        if (who == 0) break;   // m above the count: keep the current lower edge
+        const int src = __ffs(who) - 1;
+        b = __shfl_sync(0xffffffffu, b, src);
+        above = __shfl_sync(0xffffffffu, above, src);
+        remaining -= above;
+        const uint32_t nlo = lo + ((uint32_t)b << sh);
+        const uint64_t ntop = (uint64_t)nlo + ((1ull << sh) - 1);
+        hi = ntop < (uint64_t)hi ? (uint32_t)ntop : hi;
+        lo = nlo;
+        __syncwarp();
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(THR_WARPS * 32) row_threshold_kernel(const SelectParams p,
+                                                                        uint32_t* thresh) {
+    extern __shared__ __align__(16) uint8_t smem_t[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t* samp = reinterpret_cast<uint32_t*>(smem_t + warp * THR_SMEM_WARP);
+    uint32_t* hist = samp + THR_SAMPLES;
+    const int rr = blockIdx.x * THR_WARPS + warp;   // row index within the launch
+    if (rr >= p.nrows) return;
+    const int r = p.row0 + rr;
+    bool ok;
+    const int lim = row_limit(p.scan_kind, r, p.L, p.g, p.Gm, p.maxlen, p.cache_len, ok);
+    const int n = ok ? lim + 1 : 0;
+    uint32_t T = 1;
+    if (n > p.fast_cap) {
+        const float* S = p.S + (size_t)rr * p.S_stride;
+#pragma unroll 8
+        for (int run = 0; run < THR_RUNS; ++run) {
+            long long start = ((long long)run * n) / THR_RUNS;
+            if (start + 32 > n) start = n - 32;
+            samp[run * 32 + lane] = ordered_key(S[start + lane]);
+        }
+        __syncwarp();
+        uint32_t elig = 0;
+        for (int i = lane; i < THR_SAMPLES; i += 32) elig += samp[i] != 0;
+        for (int o = 16; o > 0; o >>= 1) elig += __shfl_xor_sync(0xffffffffu, elig, o);
+        long long m = (long long)ceilf(SAMPLE_MARGIN * (float)p.K * (float)THR_SAMPLES / (float)n);
+        if (m < 1) m = 1;
+        if (m <= (long long)elig) T = warp_kth_largest(samp, THR_SAMPLES, (uint32_t)m, hist);
+    }
+    if (lane == 0) thresh[rr] = T;
+}
+
 __host__ __device__ int pow2_at_least(int x) {
     int m = 1;
     while (m < x) m <<= 1;
@@ -695,6 +847,21 @@ static int select_fast_cap(int K) {
 }
 
 constexpr size_t SELECT_SMEM_LIMIT = 220 * 1024;
+
+cudaError_t launch_row_threshold(const SelectParams& p_in, uint32_t* thresh, cudaStream_t stream) {
+    if (p_in.nrows <= 0) return cudaSuccess;
+    if (p_in.kind != SEL_PREFIX) return cudaErrorInvalidValue;
+    SelectParams p = p_in;
+    p.fast_cap = select_fast_cap(p.K);
+    if (p.fast_cap == 0) p.fast_cap = 0x7fffffff;   // exact path only: no bound needed
+    const size_t smem = THR_WARPS * THR_SMEM_WARP;
+    cudaError_t e = cudaFuncSetAttribute(row_threshold_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (p.nrows + THR_WARPS - 1) / THR_WARPS;
+    row_threshold_kernel<<<grid, THR_WARPS * 32, smem, stream>>>(p, thresh);
+    return cudaGetLastError();
+}
 
 size_t select_smem_bytes(int K, int tail_cap) {
     return select_layout(K, tail_cap, 0, 0, false).total;
