@@ -335,7 +335,8 @@ struct FastSmem {
 // than K eligible entries or more than the buffer holds.
 __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastSmem& sm,
                             uint32_t* s_cnt, uint32_t* s_valid, int32_t* out, float* outs) {
-    const int K = p.K, cap = p.fast_cap, W = p.bitmap_words;
+    // bitmap words this row needs: its positions are <= lim
+    const int K = p.K, cap = p.fast_cap, W = min(p.bitmap_words, (v.lim + 32) >> 5);
     uint32_t* hist = sm.hist;
     uint32_t* scratch = sm.scratch;
     uint64_t* buf = sm.buf;
