@@ -117,6 +117,8 @@ def test_tiny_invariants_on_gpu(tiny):
     (300, 4, 64, 64),        # C == k
     (129, 2, 300, 7),        # C larger than every prefix
     (514, 8, 40, 1),         # k = 1; 2-member tail group
+    (2048, 4, 64, 16),       # one candidate tile per Refine item, several items per CTA
+    (1024, 2, 128, 32),      # the same with full tiles
 ])
 def test_edge_shapes_exact(L, g, C, kk):
     """Every group has a power-of-two member count, so the proxy mean of

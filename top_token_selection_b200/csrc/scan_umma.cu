@@ -233,7 +233,8 @@ __global__ void __maxnreg__(SCAN_MAXREG)
             int stage = 0;
             uint32_t phase = 0;
             int nit = 0;
-            int pend[GDEPTH] = {0};
+            int pend[GDEPTH] = {0};       // stages of the tiles in flight, oldest first
+            int pend_it[GDEPTH] = {0};    // and the item (in this CTA's order) of each
             int npend = 0;
             int last_b[2] = {-1, -1};
             bool aborted = false;
@@ -241,7 +242,10 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[pend[0]]);
-                for (int i = 1; i < npend; ++i) pend[i - 1] = pend[i];
+                for (int i = 1; i < npend; ++i) {
+                    pend[i - 1] = pend[i];
+                    pend_it[i - 1] = pend_it[i];
+                }
                 --npend;
             };
             for (int item = blockIdx.x; item < p.nitems && !aborted; item += gridDim.x) {
@@ -249,6 +253,14 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 if (!it.valid) continue;
                 const int slot = nit & 1;
                 const uint32_t bph = (nit >> 1) & 1;
+                // The query slot frees once the MMAs of item nit - 2 are done,
+                // which needs every tile of that item published: land and
+                // publish what is in flight if any of it is that old (items
+                // shorter than the copy depth).
+                if (npend > 0 && pend_it[0] <= nit - 2) {
+                    cp_async_wait<0>();
+                    while (npend > 0) publish_oldest();
+                }
                 if (!__all_sync(0xffffffffu, mbar_wait(&bempty[slot], bph ^ 1))) {
                     aborted = true;
                     break;
@@ -297,6 +309,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                             cp_async16(dst + kb * (128 * 128) + sw128_offset(r, c), src + kb * 128);
                     }
                     cp_async_commit();
+                    pend_it[npend] = nit;
                     pend[npend++] = stage;
                     if (npend == GDEPTH) {
                         cp_async_wait<GDEPTH - 1>();
