@@ -252,10 +252,13 @@ pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, in
                               [&] { return launch_select(sp, st); }));
 }
 
+// Refine rows: S holds the scores without the key scale, which the
+// selection multiplies in (key_scale, NULL for unscaled formats).
 pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int Gm, int maxlen,
                                const int32_t* cache_len, const float* S, const int32_t* cand,
                                int cand_base, int C, int K, int npos, int32_t* out,
-                               float* out_score, int out_base, cudaStream_t st) {
+                               float* out_score, int out_base, cudaStream_t st,
+                               const float* key_scale) {
     SelectParams sp{};
     sp.npos = npos;
     sp.kind = SEL_CANDIDATES;
@@ -273,6 +276,7 @@ pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int 
     sp.cand_base = cand_base;
     sp.C = C;
     sp.K = K;
+    sp.key_scale = key_scale;
     sp.out_idx = out;
     sp.out_score = out_score;
     sp.out_base = out_base;
@@ -609,7 +613,8 @@ pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* ca
                                0, nullptr, cand + (size_t)(jc - j0) * C, jc, C, r0, r1, S, s);
         if (st != PIVOT_OK) return st;
         st = run_select_cand(SCAN_PREFILL_DENSE, r0, r1, seq->L, g, 1, 0, nullptr, S,
-                             cand + (size_t)(jc - j0) * C, jc, C, topk, seq->L, idx, score, t0, s);
+                             cand + (size_t)(jc - j0) * C, jc, C, topk, seq->L, idx, score, t0, s,
+                             seq->k_scale);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;
@@ -730,7 +735,7 @@ pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, in
                            w.cand, 0, C, 0, rows, w.R, s);
     if (st != PIVOT_OK) return st;
     return run_select_cand(SCAN_DECODE_DENSE, 0, rows, 0, 1, b->Gm, b->maxlen, b->cache_len, w.R,
-                           w.cand, 0, C, topk, b->maxlen, idx, nullptr, 0, s);
+                           w.cand, 0, C, topk, b->maxlen, idx, nullptr, 0, s, b->kc_scale);
 }
 
 }  // extern "C"

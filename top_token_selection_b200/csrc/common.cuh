@@ -138,6 +138,10 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
 __device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
 }
+// The same through L1 (a line fetched for one chunk serves the next ones).
+__device__ __forceinline__ void cp_async16_ca(uint32_t dst_smem, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -288,6 +292,19 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t c) {
 // Saturating round-to-nearest-even fp32 -> e4m3 (cvt.rn.satfinite).
 __device__ __forceinline__ uint8_t f32_to_e4m3_satfinite(float x) {
     return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+
+// Read-only global loads issued where they are written: volatile asm keeps
+// the compiler from sinking a prefetch down to its first use.
+__device__ __forceinline__ int ld_nc_early(const int32_t* p) {
+    int v;
+    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float ld_nc_early(const float* p) {
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
 }
 
 // Order-preserving unsigned key of a finite float; -0 maps like +0.

@@ -74,6 +74,8 @@ struct SelectParams {
     int npos;             // positions are < npos (bitmap size)
     int fast_cap;         // set by launch_select: kept-entry capacity of the fast path
     int bitmap_words;     // set by launch_select
+    const float* key_scale;   // SEL_CANDIDATES: if set, entry i's score is S * key_scale[kb + pos]
+                              // (kb = grp * maxlen for decode rows, else 0)
     const uint32_t* thresh;   // SEL_PREFIX: row r's lower bound at thresh[r - row0]
                               // (launch_row_threshold), or NULL: sampled in the select
 };

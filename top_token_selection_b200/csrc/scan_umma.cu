@@ -227,7 +227,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
             // layout.  A tile is published (full[stage] arrive) once its
             // copies have landed and been fenced for the tensor cores; up to
             // GDEPTH tiles are in flight.
-            constexpr int GDEPTH = STAGES > 3 ? 3 : STAGES - 1;
+            constexpr int GDEPTH = STAGES - 1;
             static_assert(STAGES > GDEPTH && GDEPTH >= 1, "the ring must outrun the copies");
             const uint8_t* kbytes = static_cast<const uint8_t*>(p.kbase);
             int stage = 0;
@@ -279,7 +279,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int slot_r = t * 128 + j * 32 + lane;
-                        pp[j] = slot_r < p.C ? it.cand[slot_r] : -1;
+                        pp[j] = slot_r < p.C ? ld_nc_early(it.cand + slot_r) : -1;
                     }
                 };
                 int cur[4], nxt[4];
@@ -293,20 +293,28 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                         break;
                     }
                     const uint32_t dst = smem_u32(sA + stage * A_BYTES);
-                    // 32 lanes cover 4 rows x 8 chunks per step; a 128-row
-                    // tile of one 128-byte K block takes 32 steps.  Row r of
-                    // step s is slot 4 s + lane / 8, held by lane r % 32 in
-                    // cur[r / 32] (r / 32 = s / 8 for every lane of the step).
+                    // Lane l copies tile rows l + 32 j (j < 4), its own
+                    // positions, 16 bytes at a time.  Chunk c of row r sits at
+                    // (r / 8) 1024 + (r % 8) 128 + ((c ^ r % 8) 16): with the
+                    // tile 1024-byte aligned that is rowbase XOR (c 16), where
+                    // rowbase holds r % 8 in bits 4-6.  The chunks of a row go
+                    // out in consecutive instructions, so after the first the
+                    // line is in L1 (.ca); the loop is two instructions a chunk.
 #pragma unroll
-                    for (int step = 0; step < 32; ++step) {
-                        const int r = step * 4 + (lane >> 3);
-                        const int c = lane & 7;
-                        const int pos = __shfl_sync(0xffffffffu, cur[step >> 3], r & 31);
+                    for (int j = 0; j < 4; ++j) {
+                        const int r = j * 32 + lane;
+                        const int pos = cur[j];
                         const size_t row = (size_t)(it.keybase + ((pos >= 0 && pos < p.nkeys) ? pos : 0));
-                        const uint8_t* src = kbytes + row * ROWB + c * 16;
+                        const uint8_t* src = kbytes + row * ROWB;
+                        const uint32_t x = (uint32_t)(r & 7);
+                        const uint32_t rowbase = dst + (uint32_t)(r >> 3) * 1024u + x * 128u + (x << 4);
 #pragma unroll
-                        for (int kb = 0; kb < KBLK; ++kb)
-                            cp_async16(dst + kb * (128 * 128) + sw128_offset(r, c), src + kb * 128);
+                        for (int c = 0; c < 8; ++c) {
+#pragma unroll
+                            for (int kb = 0; kb < KBLK; ++kb)
+                                cp_async16_ca((rowbase ^ ((uint32_t)c << 4)) + kb * (128 * 128),
+                                              src + kb * 128 + c * 16);
+                        }
                     }
                     cp_async_commit();
                     pend_it[npend] = nit;
@@ -450,34 +458,23 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 }
                 named_bar_sync(1, EPI_WARPS * 32);
             }
-            // Key scale of this thread's key in tile t (1 where none).  The
-            // scale is read a tile ahead; in gather mode the key's position
-            // (the candidate slot's entry) is read two tiles ahead, so
-            // neither read waits on the other.
-            auto slot_pos = [&](int t) -> int {
+            // Key scale of this thread's key in tile t (1 where none), read a
+            // tile ahead.  Gather mode stores its scores without the key
+            // scale (the candidate selection multiplies it in): reading the
+            // candidate's position and then its scale here put two dependent
+            // loads on every tile and halved the rate.
+            auto key_scale = [&](int t) -> float {
+                if (GATHER || !p.k_scale) return 1.0f;
                 const int s_t = t * 128 + key_in_tile;
-                return (GATHER && p.k_scale && t < it.t1 && s_t < p.C) ? it.cand[s_t] : -1;
+                return s_t <= it.maxlim ? ld_nc_early(p.k_scale + it.keybase + s_t) : 1.0f;
             };
-            auto key_scale = [&](int t, int pos) -> float {
-                if (!p.k_scale) return 1.0f;
-                int keyrow = -1;
-                if constexpr (GATHER) {
-                    if (pos >= 0 && pos < p.nkeys) keyrow = it.keybase + pos;
-                } else {
-                    const int s_t = t * 128 + key_in_tile;
-                    if (s_t <= it.maxlim) keyrow = it.keybase + s_t;
-                }
-                return keyrow >= 0 ? __ldg(p.k_scale + keyrow) : 1.0f;
-            };
-            float sk_next = key_scale(it.t0, slot_pos(it.t0));
-            int pos_next = slot_pos(it.t0 + 1);            // position for tile t + 1
+            float sk_next = key_scale(it.t0);
             for (int t = it.t0; t < it.t1; ++t) {
                 const int acc = ntile & 1;
                 const uint32_t aph = (ntile >> 1) & 1;
                 ++ntile;
                 const float sk = sk_next;                  // prefetched a tile ahead
-                if (t + 1 < it.t1) sk_next = key_scale(t + 1, pos_next);
-                pos_next = slot_pos(t + 2);
+                if (t + 1 < it.t1) sk_next = key_scale(t + 1);
                 if (aborted) continue;
                 const bool got = mbar_wait(&accfull[acc], aph);
                 if (!__all_sync(0xffffffffu, got)) { aborted = true; continue; }
@@ -517,9 +514,9 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                         for (int j = 0; j < 4; ++j) unpack2(a[j], lo[j], hi[j]);
                         const float rowsum = ((lo[0] + hi[0]) + (lo[1] + hi[1])) +
                                              ((lo[2] + hi[2]) + (lo[3] + hi[3]));
-                        if (col_ok && s <= lim_r[lr])
-                            p.S[(size_t)(it.row_first + pr - p.row0) * p.S_stride + s] =
-                                rowsum * sq_r[lr] * sk;
+                        if (col_ok && s <= lim_r[lr])   // streaming store: keep L2 for the keys
+                            __stcs(p.S + (size_t)(it.row_first + pr - p.row0) * p.S_stride + s,
+                                   rowsum * sq_r[lr] * sk);
                     }
                 } else {
                     if (r_hi > 0) {
@@ -535,8 +532,9 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                                 if ((i + 1) % HEADS == 0) {
                                     const int pr = (c0 + i) / HEADS;
                                     if (col_ok && s <= lim_s[pr])
-                                        p.S[(size_t)(it.row_first + pr - p.row0) * p.S_stride +
-                                            s] = rowacc * sq_s[pr] * sk;
+                                        __stcs(p.S + (size_t)(it.row_first + pr - p.row0) *
+                                                         p.S_stride + s,
+                                               rowacc * sq_s[pr] * sk);
                                     rowacc = 0.0f;
                                 }
                             }

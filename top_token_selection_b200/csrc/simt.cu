@@ -132,7 +132,10 @@ __global__ void __launch_bounds__(ST) refine_simt_kernel(const RefineParams p) {
     const bool key_ok = keyrow >= 0;
     for (int d = 0; d < p.D; ++d)
         kT[d * ST + threadIdx.x] = key_ok ? load_elem(p.dtype, p.k, (size_t)keyrow * p.D + d) : 0.0f;
-    const float sk = (p.k_scale && key_ok) ? p.k_scale[keyrow] : 1.0f;
+    // Refine scores are stored without the key scale: the candidate
+    // selection multiplies it in, in the same order ((acc * sq) * sk).
+    (void)keyrow;
+    const float sk = 1.0f;
     score_rows(p.dtype, p.H, p.D, p.q, p.q_scale, p.w, p.qrow_base, r_first, r_last - r_first, kT,
                qs, ws, sk, key_ok ? pos : 0x7fffffff, key_ok && c < p.C, p.kind, p.L, p.g, p.Gm,
                p.maxlen, p.cache_len, p.S, p.C, p.row0, c);

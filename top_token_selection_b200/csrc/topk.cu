@@ -65,6 +65,7 @@ __device__ __forceinline__ int row_limit(int kind, int r, int L, int g, int Gm, 
 struct RowView {
     const float* S;
     const int32_t* cand;   // null: position = entry index
+    const float* ksc;      // candidate rows: score = S[i] * ksc[position], or null
     int n;                 // entries
     int lim;               // valid positions are <= lim
 };
@@ -84,18 +85,22 @@ __device__ __forceinline__ uint32_t key_upos(uint64_t k) {
 // Key of entry i, or 0 when the entry is not eligible.
 __device__ __forceinline__ uint64_t entry_key(const RowView& v, int i) {
     int pos = i;
+    float x = v.S[i];
     if (v.cand) {
         pos = v.cand[i];
         if (pos < 0 || pos > v.lim) return 0;
+        if (v.ksc) x = x * v.ksc[pos];
     }
-    return make_key(ordered_key(v.S[i]), pos);
+    return make_key(ordered_key(x), pos);
 }
 __device__ __forceinline__ uint32_t entry_key32(const RowView& v, int i) {
+    float x = v.S[i];
     if (v.cand) {
         const int pos = v.cand[i];
         if (pos < 0 || pos > v.lim) return 0;
+        if (v.ksc) x = x * v.ksc[pos];
     }
-    return ordered_key(v.S[i]);
+    return ordered_key(x);
 }
 
 // ------------------------------------------------------------ block helpers
@@ -810,13 +815,16 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const SelectParams 
     RowView v;
     v.S = p.S + (size_t)(r - p.row0) * p.S_stride;
     v.lim = lim;
+    v.ksc = nullptr;
     if (p.kind == SEL_PREFIX) {
         v.cand = nullptr;
         v.n = ok ? lim + 1 : 0;
     } else {
-        const int grp = (p.scan_kind == SCAN_DECODE_DENSE) ? r / p.Gm : r / p.g;
+        const bool dec = p.scan_kind == SCAN_DECODE_DENSE;
+        const int grp = dec ? r / p.Gm : r / p.g;
         v.cand = p.cand + (size_t)(grp - p.cand_base) * p.C;
         v.n = ok ? p.C : 0;
+        if (p.key_scale) v.ksc = p.key_scale + (dec ? (size_t)grp * p.maxlen : 0);
     }
     if (!ok && threadIdx.x == 0) raise_error(ERRBIT_DATA);
 
