@@ -227,7 +227,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
             // layout.  A tile is published (full[stage] arrive) once its
             // copies have landed and been fenced for the tensor cores; up to
             // GDEPTH tiles are in flight.
-            constexpr int GDEPTH = STAGES - 1;
+            constexpr int GDEPTH = STAGES > 3 ? 3 : STAGES - 1;   // deeper was slower
             static_assert(STAGES > GDEPTH && GDEPTH >= 1, "the ring must outrun the copies");
             const uint8_t* kbytes = static_cast<const uint8_t*>(p.kbase);
             int stage = 0;
