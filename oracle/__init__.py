@@ -68,6 +68,7 @@ def _load():
             lib.oracle_refine.argtypes = [I, I, I, I, P, P, P, P, P, I, P, I, I, I, P, P, P, I]
             lib.oracle_decode.argtypes = [I, I, I, I, I, P, P, P, P, P, I, P, I, I, I, P, P, P, I]
             lib.oracle_window_union.argtypes = [P, I, I, I, P]
+            lib.oracle_reuse_backfill.argtypes = [I, I, P, P, I, I, I, P, P]
             _lib = lib
     return _lib
 
@@ -212,6 +213,34 @@ def reuse(L, g, cand, topk, rows=None):
     rows = _rows(rows, L)
     out = np.empty((len(rows), topk), dtype=np.int32)
     lib.oracle_reuse(L, g, _ptr(cand), C, topk, len(rows), _ptr(rows), _ptr(out))
+    return out
+
+
+def reuse_backfill(L, g, cand, cand_score, topk, rows=None):
+    """Reuse with backfill: per member, the top-k of its group's candidates at
+    positions <= t by proxy score (cand_score, same shape as cand)."""
+    lib = _load()
+    cand = np.ascontiguousarray(cand, dtype=np.int32)
+    cand_score = np.ascontiguousarray(cand_score, dtype=np.float64)
+    assert cand_score.shape == cand.shape
+    G, C = cand.shape
+    rows = _rows(rows, L)
+    out = np.empty((len(rows), topk), dtype=np.int32)
+    lib.oracle_reuse_backfill(L, g, _ptr(cand), _ptr(cand_score), C, topk, len(rows), _ptr(rows),
+                              _ptr(out))
+    return out
+
+
+def window_union_rows(idx, t_first, window):
+    """Each index row (ascending, -1 padded) united with its window
+    [t - window + 1, t], t = t_first + row: [rows, k + window], -1 padded."""
+    idx = np.asarray(idx, dtype=np.int32)
+    rows, k = idx.shape
+    out = np.full((rows, k + window), -1, dtype=np.int32)
+    for r in range(rows):
+        sel = idx[r][idx[r] >= 0]
+        u = window_union(sel, t_first + r, window)
+        out[r, :len(u)] = u
     return out
 
 

@@ -443,6 +443,34 @@ int oracle_reuse(int L, int g, const int32_t* cand, int C, int topk, int nrows,
     return 0;
 }
 
+/* Reuse with backfill (a reading the pages leave open: [BLOG] "How It Works"
+ * says only that members share the proxy's choice).  Member t of group j
+ * takes, among the entries of cand[j] at positions <= t, the k with the
+ * highest proxy score (cand_score[j], lower position first on ties): the
+ * proxy's top-k where none of it is masked, else the next-ranked candidates
+ * fill the masked slots.  Ascending positions, -1 padding. */
+int oracle_reuse_backfill(int L, int g, const int32_t* cand, const double* cand_score, int C,
+                          int topk, int nrows, const int32_t* rows, int32_t* out_idx) {
+    (void)L;
+    entry_t* e = (entry_t*)malloc(sizeof(entry_t) * (size_t)(C > 0 ? C : 1));
+    for (int r = 0; r < nrows; ++r) {
+        int t = rows[r];
+        int j = t / g;
+        int n = 0;
+        for (int i = 0; i < C; ++i) {
+            int32_t s = cand[(size_t)j * C + i];
+            if (s >= 0 && s <= t) {
+                e[n].score = cand_score[(size_t)j * C + i];
+                e[n].pos = s;
+                ++n;
+            }
+        }
+        take_topk(e, n, topk, out_idx + (size_t)r * topk, NULL);
+    }
+    free(e);
+    return 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* PIVOT-Refine ([ABS]): each member re-scores the candidate set.            */
 /* ------------------------------------------------------------------------ */

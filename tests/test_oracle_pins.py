@@ -110,6 +110,9 @@ def test_derived_example_prefill(golden_dir):
         [sp["reuse"]["6"], sp["reuse"]["7"]]
     ref, _ = oracle.refine(F32, q, None, w, k, None, g, cand, sp["topk"], rows=[6, 7])
     assert ref.tolist() == [sp["refine"]["6"], sp["refine"]["7"]]
+    cand, csc = oracle.proxy_scan(F32, pq, None, pw, k, None, L, g, sp["C"], sp["topk"])
+    bf = oracle.reuse_backfill(L, g, cand, csc, sp["topk"], rows=[6, 7])
+    assert bf.tolist() == [sp["reuse_backfill"]["6"], sp["reuse_backfill"]["7"]]
 
 
 # ---------------------------------------------------------------------------
@@ -397,3 +400,42 @@ def test_decode_equals_last_prefill_group():
         assert (idx[0] == ref).all(), mode
         if dc is not None:
             assert (dc[0] == cand[(n - 1) // 2]).all()
+
+
+def test_reuse_backfill_invariants():
+    """Backfill keeps every Reuse entry, is Reuse where nothing of the proxy's
+    top-k is masked, and fills up to min(k, valid candidates) slots with the
+    best-scored valid candidates."""
+    rng = np.random.default_rng(11)
+    L, H, D, g, C, kk = 96, 2, 8, 4, 24, 8
+    q = rng.integers(-3, 4, (L, H, D)).astype(np.float32)
+    k = rng.integers(-3, 4, (L, D)).astype(np.float32)
+    w = rng.integers(1, 4, (L, H)).astype(np.float32)
+    pq, pqs, pw = oracle.proxy_reduce(F32, q, None, w, g)
+    cand, csc = oracle.proxy_scan(F32, pq, pqs, pw, k, None, L, g, C, kk)
+    reu = oracle.reuse(L, g, cand, kk)
+    bf = oracle.reuse_backfill(L, g, cand, csc, kk)
+    for t in range(L):
+        j = t // g
+        r = set(reu[t][reu[t] >= 0].tolist())
+        b = bf[t][bf[t] >= 0].tolist()
+        assert b == sorted(b) and r <= set(b)
+        valid = [i for i in range(C) if 0 <= cand[j, i] <= t]
+        assert len(b) == min(kk, len(valid))
+        if all(0 <= s <= t for s in cand[j, :kk]):
+            assert set(b) == r
+        # nothing left out beats anything taken (score, then position)
+        taken = set(b)
+        worst = min((csc[j, i], -cand[j, i]) for i in valid if cand[j, i] in taken) if b else None
+        for i in valid:
+            if cand[j, i] not in taken:
+                assert (csc[j, i], -cand[j, i]) < worst
+
+
+def test_window_union_rows_matches_the_example(golden_dir):
+    ex = _load(golden_dir, "indexer_tutorial_example.json")["window_union"]
+    row = np.array([ex["selected"] + [-1]], dtype=np.int32)
+    out = oracle.window_union_rows(row, ex["position"], ex["window"])
+    u = out[0][out[0] >= 0].tolist()
+    assert u == ex["union"]
+    assert out.shape == (1, len(ex["selected"]) + 1 + ex["window"])
