@@ -137,7 +137,7 @@ pivot_status_t pivot_proxy_reduce(const pivot_seq_t* seq, int32_t g, void* pq,
  * keeps its top-C.  cand [G, C] int32: the proxy's top-`topk` positions
  * (ascending), then the rest of its top-C (ascending) -- so the first topk
  * entries are what PIVOT-Reuse shares.  cand_score [G, C] or NULL.
- * 1 <= topk <= C. */
+ * 1 <= topk <= C <= 8192. */
 pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* pq,
                                  const float* pq_scale, const float* pw, int32_t C,
                                  int32_t topk, int32_t* cand, float* cand_score, void* ws,
@@ -152,10 +152,39 @@ size_t pivot_proxy_scan_workspace_size(const pivot_seq_t* seq, int32_t g, int32_
 pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int32_t* cand,
                            int32_t C, int32_t topk, int32_t* idx, void* stream);
 
+/* PIVOT-Reuse with backfill.  The pages leave open what a member does when
+ * part of the proxy's top-k lies after it (PIVOT abstract; "How It Works" of
+ * the PIVOT blog post only says the members share the proxy's choice); this
+ * reading refills the masked slots with the next proxy-ranked candidates:
+ * member t of group j takes, among the entries of cand[j] at positions <= t,
+ * the topk with the highest cand_score[j] (lower position first on equal
+ * scores), listed in ascending position, -1 padded.  Where nothing of the
+ * proxy's top-k is masked this is exactly pivot_reuse.
+ * cand, cand_score [G, C] device (rows relative to t_begin / g), as written
+ * by pivot_proxy_scan; rows [t_begin, t_end), t_begin a multiple of g;
+ * idx [rows, topk] device.  1 <= topk <= C <= 8192.  No workspace. */
+pivot_status_t pivot_reuse_backfill(int32_t t_begin, int32_t t_end, int32_t g,
+                                    const int32_t* cand, const float* cand_score, int32_t C,
+                                    int32_t topk, int32_t* idx, void* stream);
+
+/* The selected positions united with a recent window ("Sparse Attention의
+ * Indexer", Fig. 3 and the paragraph after it: a sliding window added to the
+ * indexer's choice, the window's positions counted once).  This is the
+ * variant where the window lies inside the indexer's candidates: row r's
+ * output is its entries of idx below t - window + 1, then every position of
+ * [max(0, t - window + 1), t], ascending, -1 padded.
+ * idx [rows, topk] device, each row ascending with -1 padding (the layout
+ * every index entry point writes); t = positions[r] (device [rows]) or,
+ * when positions is NULL, t_begin + r; out [rows, topk + window] device.
+ * window >= 1.  Rows whose t is negative come out all -1. */
+pivot_status_t pivot_window_union(const int32_t* idx, int32_t rows, int32_t topk, int32_t t_begin,
+                                  const int32_t* positions, int32_t window, int32_t* out,
+                                  void* stream);
+
 /* PIVOT-Refine (PIVOT abstract): member t of group j scores every candidate
  * s in cand[j] with 0 <= s <= t using its own q[t], w[t] (the dense score
  * formula) and keeps the top-k.  idx [rows, topk], score [rows, topk] or
- * NULL.  1 <= topk <= C. */
+ * NULL.  1 <= topk <= C <= 8192. */
 pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* cand,
                             int32_t C, int32_t topk, int32_t* idx, float* score, void* ws,
                             size_t ws_bytes, void* stream);

@@ -114,3 +114,16 @@ def test_missing_library_fails_loudly(tmp_path):
             pv.load(str(tmp_path / "nope.so"))
     finally:
         pv._lib = saved
+
+
+def test_next_steps_reject_bad_arguments(lib):
+    assert pv.pivot_reuse_backfill(0, 64, 0, FAKE, FAKE, 16, 8, FAKE, None) == 1    # g >= 1
+    assert pv.pivot_reuse_backfill(3, 64, 4, FAKE, FAKE, 16, 8, FAKE, None) == 1    # t_begin % g
+    assert pv.pivot_reuse_backfill(0, 64, 4, FAKE, None, 16, 8, FAKE, None) == 1    # scores needed
+    assert pv.pivot_reuse_backfill(0, 64, 4, FAKE, FAKE, 8, 16, FAKE, None) == 1    # C < k
+    assert pv.pivot_reuse_backfill(0, 64, 4, FAKE, FAKE, 1 << 20, 8, FAKE, None) == 2
+    assert pv.pivot_window_union(FAKE, 4, 8, 0, None, 0, FAKE, None) == 1          # window >= 1
+    assert pv.pivot_window_union(FAKE, 4, 0, 0, None, 3, FAKE, None) == 1          # topk >= 1
+    assert pv.pivot_window_union(None, 4, 8, 0, None, 3, FAKE, None) == 1
+    assert pv.pivot_window_union(FAKE, 4, 8, -1, None, 3, FAKE, None) == 1         # no positions
+    assert pv.pivot_window_union(FAKE, 0, 8, 0, None, 3, FAKE, None) == 0          # nothing to do

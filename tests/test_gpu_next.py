@@ -1,0 +1,98 @@
+"""The next steps after the indexer proper, on the GPU through the C ABI:
+Reuse with backfill and the window union, bit for bit against the oracle on
+integer inputs (every score exact, so every choice is the oracle's)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from top_token_selection_b200 import inputs as gen
+from top_token_selection_b200 import pivot as pv
+
+from parity import assert_rows_exact, seq_of, to_device
+
+pytestmark = pytest.mark.gpu
+
+F32 = gen.F32
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    cfg = gen.WORKLOADS["tiny_int_prefill"]
+    p = gen.make_prefill(cfg["L"], cfg["H"], cfg["D"], F32, kind="int", seed=0)
+    return p, to_device(p), cfg
+
+
+@pytest.mark.parametrize("g,C,kk", [(4, 256, 64), (8, 100, 37), (1, 64, 64), (2, 40, 9)])
+def test_reuse_backfill_exact(tiny, g, C, kk):
+    """Power-of-two member counts keep the integer proxy exact at TF32, so
+    candidates and proxy scores are the oracle's bit for bit."""
+    p, dev, _ = tiny
+    seq = seq_of(dev)
+    pq, pqs, pw = pv.proxy_reduce(seq, g)
+    cand, cs = pv.proxy_scan(seq, g, pq, pqs, pw, C, kk, with_score=True)
+    bf = pv.reuse_backfill(0, p.L, g, cand, cs, kk)
+    reu = pv.reuse(0, p.L, g, cand, kk)
+    torch.cuda.synchronize()
+    assert pv.device_error() == 0
+    q, qs, w, k, ks = p.codes()
+    opq, opqs, opw = oracle.proxy_reduce(F32, q, qs, w, g)
+    ocand, ocs = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, p.L, g, C, kk)
+    assert_rows_exact(cand.cpu(), ocand, "cand")
+    assert_rows_exact(bf.cpu(), oracle.reuse_backfill(p.L, g, ocand, ocs, kk), "backfill")
+    # where nothing of the proxy's top-k lies after the member, it is Reuse
+    c = ocand[:, :kk]
+    t = np.arange(p.L)
+    unmasked = (c[t // g] <= t[:, None]).all(axis=1)
+    assert unmasked.any()
+    assert (bf.cpu().numpy()[unmasked] == reu.cpu().numpy()[unmasked]).all()
+
+
+def test_reuse_backfill_row_range(tiny):
+    """Rows [t0, t1) with candidate rows relative to t0 / g match the full call."""
+    p, dev, _ = tiny
+    g, C, kk = 4, 128, 32
+    seq = seq_of(dev)
+    pq, pqs, pw = pv.proxy_reduce(seq, g)
+    cand, cs = pv.proxy_scan(seq, g, pq, pqs, pw, C, kk, with_score=True)
+    full = pv.reuse_backfill(0, p.L, g, cand, cs, kk)
+    t0, t1 = 200, 517
+    part = pv.reuse_backfill(t0, t1, g, cand[t0 // g:], cs[t0 // g:], kk)
+    torch.cuda.synchronize()
+    assert (part.cpu() == full.cpu()[t0:t1]).all()
+
+
+@pytest.mark.parametrize("window", [1, 3, 64, 300])
+def test_window_union_exact(tiny, window):
+    p, dev, cfg = tiny
+    kk = cfg["topk"]
+    idx, _ = pv.dense_index(seq_of(dev), kk)
+    out = pv.window_union(idx, window)
+    torch.cuda.synchronize()
+    q, qs, w, k, ks = p.codes()
+    oidx, _ = oracle.dense_index(F32, q, qs, w, k, ks, kk)
+    assert (out.cpu().numpy() == oracle.window_union_rows(oidx, 0, window)).all()
+
+
+def test_window_union_explicit_positions():
+    """Decode-style rows: positions given per row (one negative: no row)."""
+    rng = np.random.default_rng(4)
+    rows, kk, window = 7, 16, 5
+    pos = np.array([0, 3, 40, 41, 1000, -1, 17], dtype=np.int32)
+    idx = np.full((rows, kk), -1, dtype=np.int32)
+    for r, t in enumerate(pos):
+        if t < 0:
+            continue
+        n = min(kk, t + 1)
+        idx[r, :n] = np.sort(rng.choice(t + 1, n, replace=False))
+    out = pv.window_union(torch.from_numpy(idx).cuda(), window,
+                          positions=torch.from_numpy(pos).cuda())
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    for r, t in enumerate(pos):
+        if t < 0:
+            assert (got[r] == -1).all()
+            continue
+        sel = idx[r][idx[r] >= 0]
+        u = oracle.window_union(sel, int(t), window)
+        assert got[r, :len(u)].tolist() == list(u) and (got[r, len(u):] == -1).all()

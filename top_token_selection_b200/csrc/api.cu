@@ -16,7 +16,7 @@ namespace {
 
 constexpr size_t WS_ALIGN = 256;
 constexpr size_t SCORE_BUF_CAP = size_t(4) << 30;   // preferred score buffer, 4 GiB
-constexpr int MAX_K = 16384;
+constexpr int MAX_K = 8192;   // the select's exact path holds 2 pow2(K) keys in shared memory
 constexpr int TAIL_CAP = 4096;
 constexpr int MAX_SMS = 1024;
 
@@ -574,6 +574,50 @@ pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int3
     const double bytes = 4.0 * topk * ((double)(t_end - t_begin) + ceil_div(t_end - t_begin, g));
     return from_cuda(profiled(PK_REUSE, bytes, s, [&] {
         return launch_reuse(t_begin, t_end, g, cand, C, topk, idx, s);
+    }));
+}
+
+pivot_status_t pivot_reuse_backfill(int32_t t_begin, int32_t t_end, int32_t g,
+                                    const int32_t* cand, const float* cand_score, int32_t C,
+                                    int32_t topk, int32_t* idx, void* stream) {
+    if (g < 1 || t_begin < 0 || t_end <= t_begin || t_begin % g) return PIVOT_ERR_INVALID_ARG;
+    if (!cand || !cand_score || !idx || topk < 1 || C < topk) return PIVOT_ERR_INVALID_ARG;
+    if (C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the candidate selection over each group's proxy scores, per member limit t
+    SelectParams sp{};
+    sp.kind = SEL_CANDIDATES;
+    sp.scan_kind = SCAN_PREFILL_DENSE;   // lim(t) = t
+    sp.row0 = t_begin;
+    sp.nrows = t_end - t_begin;
+    sp.L = t_end;
+    sp.g = g;
+    sp.Gm = 1;
+    sp.S = cand_score;
+    sp.S_stride = C;
+    sp.s_per_group = 1;
+    sp.cand = cand;
+    sp.cand_base = t_begin / g;
+    sp.C = C;
+    sp.K = topk;
+    sp.out_idx = idx;
+    sp.out_base = t_begin;
+    sp.tail_cap = TAIL_CAP;
+    sp.npos = t_end;
+    const double bytes = 8.0 * C * ceil_div(t_end - t_begin, g) + 4.0 * topk * (t_end - t_begin);
+    return from_cuda(profiled(PK_REUSE, bytes, s, [&] { return launch_select(sp, s); }));
+}
+
+pivot_status_t pivot_window_union(const int32_t* idx, int32_t rows, int32_t topk, int32_t t_begin,
+                                  const int32_t* positions, int32_t window, int32_t* out,
+                                  void* stream) {
+    if (rows < 0 || topk < 1 || window < 1 || !idx || !out) return PIVOT_ERR_INVALID_ARG;
+    if (!positions && t_begin < 0) return PIVOT_ERR_INVALID_ARG;
+    if (rows == 0) return PIVOT_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const double bytes = 4.0 * rows * (2.0 * topk + window);
+    return from_cuda(profiled(PK_REUSE, bytes, s, [&] {
+        return launch_window_union(idx, rows, topk, t_begin, positions, window, out, s);
     }));
 }
 

@@ -74,6 +74,7 @@ struct SelectParams {
     int npos;             // positions are < npos (bitmap size)
     int fast_cap;         // set by launch_select: kept-entry capacity of the fast path
     int bitmap_words;     // set by launch_select
+    int s_per_group;          // SEL_CANDIDATES: S rows are per group (grp - cand_base), not per row
     const float* key_scale;   // SEL_CANDIDATES: if set, entry i's score is S * key_scale[kb + pos]
                               // (kb = grp * maxlen for decode rows, else 0)
     const uint32_t* thresh;   // SEL_PREFIX: row r's lower bound at thresh[r - row0]
@@ -103,6 +104,11 @@ cudaError_t launch_proxy_reduce(const ReduceParams& p, cudaStream_t stream);
 
 cudaError_t launch_reuse(int t_begin, int t_end, int g, const int32_t* cand, int C, int topk,
                          int32_t* idx, cudaStream_t stream);
+// Each index row (ascending, -1 padded, k entries) united with the window
+// [t - window + 1, t] (t = positions[r], or t_begin + r): out [rows, k + window].
+cudaError_t launch_window_union(const int32_t* idx, int rows, int k, int t_begin,
+                                const int32_t* positions, int window, int32_t* out,
+                                cudaStream_t stream);
 cudaError_t launch_decode_reuse(int B, int Gm, int maxlen, const int32_t* cache_len,
                                 const int32_t* cand, int C, int topk, int32_t* idx,
                                 cudaStream_t stream);

@@ -126,7 +126,44 @@ __global__ void decode_reuse_kernel(int B, int Gm, int maxlen, const int32_t* ca
     reuse_row(cand + (size_t)b * C, topk, lim, idx + (size_t)r * topk);
 }
 
+// Window union ("Sparse Attention의 Indexer", Fig. 3, the window inside the
+// candidates): an ascending row united with [a, t], a = max(0, t - window + 1),
+// is its entries below a followed by a..t (entries in [a, t] are the window's
+// own).  One warp per row.
+__global__ void window_union_kernel(const int32_t* idx, int rows, int k, int t_begin,
+                                    const int32_t* positions, int window, int32_t* out) {
+    const int r = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    const int lane = threadIdx.x & 31;
+    const int t = positions ? positions[r] : t_begin + r;
+    const int a = t - window + 1 > 0 ? t - window + 1 : 0;
+    const int32_t* in = idx + (size_t)r * k;
+    int32_t* o = out + (size_t)r * (k + window);
+    int n = 0;
+    for (int i0 = 0; i0 < k; i0 += 32) {
+        const int i = i0 + lane;
+        const int32_t s = i < k ? in[i] : -1;
+        const bool keep = s >= 0 && s < a;
+        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) o[n + __popc(bal & ((1u << lane) - 1u))] = s;
+        n += __popc(bal);
+    }
+    const int nw = t >= a ? t - a + 1 : 0;   // t < 0 (no position) leaves the window empty
+    for (int i = lane; i < nw; i += 32) o[n + i] = a + i;
+    for (int i = n + nw + lane; i < k + window; i += 32) o[i] = -1;
+}
+
 }  // namespace
+
+cudaError_t launch_window_union(const int32_t* idx, int rows, int k, int t_begin,
+                                const int32_t* positions, int window, int32_t* out,
+                                cudaStream_t stream) {
+    if (rows <= 0) return cudaSuccess;
+    const int wpb = 8;
+    window_union_kernel<<<ceil_div(rows, wpb), wpb * 32, 0, stream>>>(idx, rows, k, t_begin,
+                                                                       positions, window, out);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_proxy_reduce(const ReduceParams& p, cudaStream_t stream) {
     if (p.ngroups <= 0) return cudaSuccess;

@@ -825,6 +825,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const SelectParams 
         v.cand = p.cand + (size_t)(grp - p.cand_base) * p.C;
         v.n = ok ? p.C : 0;
         if (p.key_scale) v.ksc = p.key_scale + (dec ? (size_t)grp * p.maxlen : 0);
+        if (p.s_per_group) v.S = p.S + (size_t)(grp - p.cand_base) * p.S_stride;
     }
     if (!ok && threadIdx.x == 0) raise_error(ERRBIT_DATA);
 

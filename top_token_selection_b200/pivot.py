@@ -31,6 +31,7 @@ ABI_SYMBOLS = [
     "pivot_get_device_error", "pivot_set_wait_limit_ns", "pivot_selftest_wait_timeout",
     "pivot_status_string", "pivot_version", "pivot_profile_enable", "pivot_profile_read",
     "pivot_launch_count", "pivot_decode_noalloc", "pivot_last_error_detail",
+    "pivot_reuse_backfill", "pivot_window_union",
 ]
 KERNELS = {0: "scan", 1: "select", 2: "refine", 3: "reduce", 4: "reuse"}
 
@@ -90,6 +91,8 @@ def load(path: str = LIB_PATH):
         "pivot_launch_count": ([], ctypes.c_int64),
         "pivot_decode_noalloc": ([P, I32, I32, I32, P, P, P], I32),
         "pivot_last_error_detail": ([], ctypes.c_char_p),
+        "pivot_reuse_backfill": ([I32, I32, I32, P, P, I32, I32, P, P], I32),
+        "pivot_window_union": ([P, I32, I32, I32, P, I32, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -126,6 +129,14 @@ def pivot_proxy_scan_workspace_size(seq, g, C):
 
 def pivot_reuse(t_begin, t_end, g, cand, C, topk, idx, stream):
     return load().pivot_reuse(t_begin, t_end, g, cand, C, topk, idx, stream)
+
+
+def pivot_reuse_backfill(t_begin, t_end, g, cand, cand_score, C, topk, idx, stream):
+    return load().pivot_reuse_backfill(t_begin, t_end, g, cand, cand_score, C, topk, idx, stream)
+
+
+def pivot_window_union(idx, rows, topk, t_begin, positions, window, out, stream):
+    return load().pivot_window_union(idx, rows, topk, t_begin, positions, window, out, stream)
 
 
 def pivot_refine(seq, g, cand, C, topk, idx, score, ws, ws_bytes, stream):
@@ -297,6 +308,21 @@ def reuse(t_begin, t_end, g, cand, topk, stream=None, device="cuda"):
     _check(pivot_reuse(t_begin, t_end, g, _p(cand), cand.shape[1], topk, _p(idx),
                        _stream(stream)), "pivot_reuse")
     return idx
+
+
+def reuse_backfill(t_begin, t_end, g, cand, cand_score, topk, stream=None, device="cuda"):
+    idx = torch.empty(t_end - t_begin, topk, dtype=torch.int32, device=device)
+    _check(pivot_reuse_backfill(t_begin, t_end, g, _p(cand), _p(cand_score), cand.shape[1], topk,
+                                _p(idx), _stream(stream)), "pivot_reuse_backfill")
+    return idx
+
+
+def window_union(idx, window, t_begin=0, positions=None, stream=None):
+    rows, topk = idx.shape
+    out = torch.empty(rows, topk + window, dtype=torch.int32, device=idx.device)
+    _check(pivot_window_union(_p(idx), rows, topk, t_begin, _p(positions), window, _p(out),
+                              _stream(stream)), "pivot_window_union")
+    return out
 
 
 def refine(seq: PivotSeq, g, cand, topk, with_score=False, ws=None, stream=None, device="cuda"):
