@@ -381,6 +381,73 @@ def config_of(wl, args):
             "l2": "no flush: inputs and score buffers larger than L2 (q alone 1 GiB)"}
 
 
+def _event_ms(fn, stream, reps):
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fn()
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def measure_extra(run, wl, device, peaks, seed, reps=3):
+    """Steps outside the headline step, each timed on its own (CUDA events,
+    warm): the MTP decode step on its workload in the three modes, Reuse with
+    backfill and the window union on this prefill.  Not part of `value`."""
+    pv, s = run.pv, run.stream
+    sp = pv._stream(s)
+    hbm = peaks["hbm_gbs"]
+    out = {}
+    # Reuse with backfill needs the proxy scores of the candidates
+    cs = torch.empty(run.G, run.C, dtype=torch.float32, device=device)
+    pv._check(pv.pivot_proxy_scan(run.seq, run.g, run.pq.data_ptr(), run._ptr(run.pqs),
+                                  run.pw.data_ptr(), run.C, run.k, run.cand.data_ptr(),
+                                  cs.data_ptr(), run.ws.data_ptr(), run.ws.numel(), sp), "scan")
+    bf = torch.empty(run.L, run.k, dtype=torch.int32, device=device)
+    ms = _event_ms(lambda: pv._check(pv.pivot_reuse_backfill(
+        0, run.L, run.g, run.cand.data_ptr(), cs.data_ptr(), run.C, run.k, bf.data_ptr(), sp),
+        "backfill"), s, reps)
+    nbytes = run.G * run.C * 8 + run.L * run.k * 4     # candidates + scores read, rows written
+    out["reuse_backfill"] = {"ms": ms, "queries_per_s": run.L / (ms / 1e3),
+                             "gbs": nbytes / (ms / 1e3) / 1e9,
+                             "frac_hbm": nbytes / (ms / 1e3) / 1e9 / hbm,
+                             "bytes": nbytes}
+    window = 128
+    un = torch.empty(run.L, run.k + window, dtype=torch.int32, device=device)
+    ms = _event_ms(lambda: pv._check(pv.pivot_window_union(
+        run.dense.data_ptr(), run.L, run.k, 0, None, window, un.data_ptr(), sp), "union"), s, reps)
+    nbytes = run.L * (2 * run.k + window) * 4
+    out["window_union"] = {"window": window, "ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9,
+                           "frac_hbm": nbytes / (ms / 1e3) / 1e9 / hbm, "bytes": nbytes}
+    # the MTP decode step (its own workload)
+    dw = gen.WORKLOADS["mtp_decode_b32"]
+    d = gen.make_decode(B=dw["B"], Gm=dw["Gm"], H=dw["H"], D=dw["D"], dtype=dw["dtype"],
+                        len_lo=dw["len_lo"], len_hi=dw["len_hi"], seed=seed + 17)
+    dev = [None if t is None else t.to(device) for t in
+           (d.q, d.q_scale, d.w, d.kc, d.kc_scale, d.cache_len)]
+    batch = pv.make_decode(*dev)
+    rows = dw["B"] * dw["Gm"]
+    keys = int(d.cache_len.sum())
+    dec = {"workload": "mtp_decode_b32", "B": dw["B"], "Gm": dw["Gm"], "C": dw["C"],
+           "topk": dw["topk"], "cached_keys": keys}
+    for name, mode in (("dense", pv.DENSE), ("reuse", pv.REUSE), ("refine", pv.REFINE)):
+        wsd = torch.empty(max(1, pv.pivot_decode_workspace_size(batch, mode, dw["C"], dw["topk"])),
+                          dtype=torch.uint8, device=device)
+        idx = torch.empty(dw["B"], dw["Gm"], dw["topk"], dtype=torch.int32, device=device)
+        ms = _event_ms(lambda: pv._check(pv.pivot_decode(
+            batch, mode, dw["C"], dw["topk"], idx.data_ptr(), None, wsd.data_ptr(), wsd.numel(),
+            sp), "decode"), s, reps)
+        dec[name] = {"ms": ms, "tokens_per_s": rows / (ms / 1e3)}
+    dec["reuse"]["speedup_vs_dense"] = dec["dense"]["ms"] / dec["reuse"]["ms"]
+    dec["refine"]["speedup_vs_dense"] = dec["dense"]["ms"] / dec["refine"]["ms"]
+    out["decode"] = dec
+    assert pv.device_error() == 0, "a kernel reported an error in the extra measurements"
+    return out
+
+
 def run_ours(args, wl):
     import torch.distributed as dist
     rank, local_rank, world = dist_env()
@@ -518,6 +585,8 @@ def run_ours(args, wl):
                "h2d_bytes_per_step": run.h2d_bytes(), "d2h_bytes_per_step": run.d2h_bytes(),
                "ms_per_step": e_ms / k_e2e}
 
+    extra = None if args.no_extra else measure_extra(run, wl, device, peaks, args.seed)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         total, desc, threads, parts = oracle_sample_time(p, wl)
@@ -531,7 +600,7 @@ def run_ours(args, wl):
             "dtype": gen.DTYPE_NAMES[wl["dtype"]], "data": "synthetic",
             "config": config_of(wl, args), "modes": modes, "recall": rec,
             "roofline": roof, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": int(n1 - n0), "clocks": clk}
+            "gpu_launches": int(n1 - n0), "clocks": clk, "extra": extra}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -551,6 +620,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the decode / backfill / window-union measurements")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
