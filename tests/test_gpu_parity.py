@@ -287,9 +287,11 @@ def _decode_dev(d):
                           d.cache_len.to(c)), d
 
 
-@pytest.mark.parametrize("dtype,H,D", [(BF16, 64, 128), (E4M3, 64, 128)])
-def test_decode_within_tolerance(dtype, H, D):
-    d = gen.make_decode(B=5, Gm=2, H=H, D=D, dtype=dtype, len_lo=300, len_hi=2200, seed=3)
+@pytest.mark.parametrize("dtype,H,D,Gm", [(BF16, 64, 128, 2), (E4M3, 64, 128, 2),
+                                          (E4M3, 64, 128, 3), (BF16, 64, 128, 4)])
+def test_decode_within_tolerance(dtype, H, D, Gm):
+    """MTP groups of 2 (one draft token) and deeper ones (3, 4 tokens per step)."""
+    d = gen.make_decode(B=5, Gm=Gm, H=H, D=D, dtype=dtype, len_lo=300, len_hi=2200, seed=3)
     batch, d = _decode_dev(d)
     q, qs, w, kc, kcs, cl = d.codes()
     C, kk = 256, 64
@@ -308,19 +310,20 @@ def test_decode_within_tolerance(dtype, H, D):
                 return oracle.score_positions(dtype, q[b], None if qs is None else qs[b], w[b],
                                               kb, kbs, m, positions)
             if mode == pv.DENSE:
-                assert_rows_close(gi[b], oidx[b], osc[b], fn, [0, 1], f"decode dense b={b}")
+                assert_rows_close(gi[b], oidx[b], osc[b], fn, list(range(Gm)),
+                                  f"decode dense b={b}")
             else:
                 gc = cand.cpu().numpy()
                 if mode == pv.REUSE:
-                    for m in range(2):
-                        lim = n - 2 + m
+                    for m in range(Gm):
+                        lim = n - Gm + m
                         want = [x for x in gc[b][:kk] if 0 <= x <= lim]
                         want += [-1] * (kk - len(want))
                         assert list(gi[b][m]) == want
                 else:
                     # refine on the GPU's candidates, member by member
-                    for m in range(2):
-                        lim = n - 2 + m
+                    for m in range(Gm):
+                        lim = n - Gm + m
                         pos = np.array([x for x in gc[b] if 0 <= x <= lim], dtype=np.int32)
                         sc = fn(m, pos)
                         order = np.lexsort((pos, -sc))[:kk]
@@ -330,8 +333,9 @@ def test_decode_within_tolerance(dtype, H, D):
                                           fn, [m], f"decode refine b={b}")
 
 
-def test_decode_integer_exact():
-    d = gen.make_decode(B=3, Gm=2, H=4, D=32, dtype=F32, len_lo=50, len_hi=700, seed=9)
+@pytest.mark.parametrize("Gm", [2, 4])
+def test_decode_integer_exact(Gm):
+    d = gen.make_decode(B=3, Gm=Gm, H=4, D=32, dtype=F32, len_lo=50, len_hi=700, seed=9)
     # integer-valued keys and queries for exact comparison
     gg = torch.Generator().manual_seed(5)
     d.q = torch.randint(-3, 4, d.q.shape, generator=gg).float()

@@ -219,6 +219,19 @@ int rows_per_block(int H, int D, int dtype) {
     return umma_shape_ok(H, D, dtype) ? umma_rows(H) : 8;
 }
 
+// Decode dense rows: a row block must not straddle two sequences (its keys
+// are one sequence's), so its row count divides Gm; on the tensor cores it is
+// also at most umma_rows(H) (the epilogue gives each of its three warp groups
+// at most 64 / H rows at H >= 32).
+int decode_dense_rows(int Gm, int H, int D, int dtype) {
+    if (!umma_shape_ok(H, D, dtype)) return Gm;
+    const int pmax = umma_rows(H);
+    int P = 1;
+    for (int d = 1; d <= Gm && d <= pmax; ++d)
+        if (Gm % d == 0) P = d;
+    return P;
+}
+
 pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, int Gm, int maxlen,
                                  const int32_t* cache_len, const float* S, long long stride,
                                  int K, int split, int npos, int32_t* out, float* out_score,
@@ -731,7 +744,7 @@ pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, in
     const long long krows = (long long)b->B * b->maxlen;
     if (mode == PIVOT_MODE_DENSE) {
         const int rows = b->B * b->Gm;
-        const int P = b->Gm;   // one sequence's members share a row block
+        const int P = decode_dense_rows(b->Gm, b->H, b->D, b->dtype);
         st = run_scan(SCAN_DECODE_DENSE, b->dtype, b->H, b->D, b->q, rows, 0, b->w, b->q_scale,
                       b->kc, krows, b->kc_scale, 0, 1, b->Gm, b->maxlen, b->cache_len, P, 0, rows,
                       b->maxlen - 1, w.S, stride, s);

@@ -563,9 +563,18 @@ int scan_smem_bytes(int row_bytes) {
            256 /*barriers*/ + 16 /*TMEM address*/ + 256 * 4 + pmax * 8;
 }
 
+// The epilogue's three warp groups take ceil(P / 3) rows each, with room
+// for 64 / HEADS rows' weights in registers at HEADS >= 32, and PMAX rows'
+// tables in shared memory below: larger blocks are refused.
+inline bool epilogue_fits(int P, int heads) {
+    if (P < 1 || P * heads > 256) return false;
+    return heads >= 32 ? (P + 2) / 3 <= 64 / heads : true;
+}
+
 template <int KIND, int HEADS, bool GATHER>
 static cudaError_t launch_heads(const CUtensorMap& tk, const CUtensorMap& tq, const ScanParams& p,
                                 int row_bytes, int grid, cudaStream_t stream) {
+    if (!epilogue_fits(p.P, HEADS)) return cudaErrorInvalidValue;
     if (row_bytes == 128) {
         auto kfn = index_umma_kernel<KIND, HEADS, 128, GATHER>;
         const int smem = scan_smem_bytes(128);
