@@ -110,6 +110,23 @@ typedef struct {
     const int32_t* cache_len;    /* [B] on the device, Gm <= cache_len <= maxlen */
 } pivot_decode_t;
 
+/* A batch of prefill sequences packed row after row, the layout of ragged
+ * (variable-length) attention batches: sequence i holds rows
+ * [cu_seqlens[i], cu_seqlens[i+1]) of q, q_scale, w, k and k_scale, and its
+ * positions count from its own first row.  cu_seqlens is a HOST array of
+ * nseq + 1 non-decreasing offsets starting at 0 (the calls plan their
+ * launches from it). */
+typedef struct {
+    int32_t dtype;
+    int32_t nseq, H, D;
+    const int32_t* cu_seqlens;   /* host [nseq + 1]                              */
+    const void* q;               /* [total, H, D]                                */
+    const float* q_scale;        /* [total] for PIVOT_E4M3, else NULL            */
+    const float* w;              /* [total, H]                                   */
+    const void* k;               /* [total, D]                                   */
+    const float* k_scale;        /* [total] for PIVOT_E4M3, else NULL            */
+} pivot_varlen_t;
+
 /* Dense indexer (Fig. 1-2 of the indexer tutorial; the baseline the PIVOT
  * abstract compares with).  idx [rows, topk] int32; score [rows, topk] or
  * NULL.  rows = t_end - t_begin.  topk >= 1. */
@@ -166,6 +183,22 @@ pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int3
 pivot_status_t pivot_reuse_backfill(int32_t t_begin, int32_t t_end, int32_t g,
                                     const int32_t* cand, const float* cand_score, int32_t C,
                                     int32_t topk, int32_t* idx, void* stream);
+
+/* The indexer over a ragged batch (pivot_varlen_t): for every sequence the
+ * dense indexer (mode PIVOT_MODE_DENSE) or PIVOT with Reuse / Refine (its
+ * groups of g consecutive queries never span two sequences), exactly as the
+ * single-sequence calls compute it.  The PIVOT abstract's method per
+ * sequence; the batching itself is not in the pages (the PIVOT blog post
+ * notes batching was left untested).  idx [total, topk] device, row t of
+ * sequence i at cu_seqlens[i] + t, positions within the sequence, -1
+ * padded.  1 <= topk <= C <= 8192 (C unused in dense mode).  ws of at
+ * least pivot_index_varlen_workspace_size bytes, 256-byte aligned.  The
+ * sequences run one after another on the stream. */
+pivot_status_t pivot_index_varlen(const pivot_varlen_t* batch, int32_t mode, int32_t g, int32_t C,
+                                  int32_t topk, int32_t* idx, void* ws, size_t ws_bytes,
+                                  void* stream);
+size_t pivot_index_varlen_workspace_size(const pivot_varlen_t* batch, int32_t mode, int32_t g,
+                                         int32_t C, int32_t topk);
 
 /* The selected positions united with a recent window ("Sparse Attention의
  * Indexer", Fig. 3 and the paragraph after it: a sliding window added to the

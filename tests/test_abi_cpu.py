@@ -127,3 +127,24 @@ def test_next_steps_reject_bad_arguments(lib):
     assert pv.pivot_window_union(None, 4, 8, 0, None, 3, FAKE, None) == 1
     assert pv.pivot_window_union(FAKE, 4, 8, -1, None, 3, FAKE, None) == 1         # no positions
     assert pv.pivot_window_union(FAKE, 0, 8, 0, None, 3, FAKE, None) == 0          # nothing to do
+
+
+def test_ragged_batch_rejects_bad_arguments(lib):
+    import ctypes
+
+    def batch(cu):
+        arr = (ctypes.c_int32 * len(cu))(*cu)
+        b = pv.PivotVarlen(pv.F32, len(cu) - 1, 4, 32, ctypes.addressof(arr), FAKE, None, FAKE,
+                           FAKE, None)
+        b._keep = (arr,)
+        return b
+    good = batch([0, 10, 30])
+    assert pv.pivot_index_varlen_workspace_size(good, 1, 4, 16, 8) > 0
+    assert pv.pivot_index_varlen(batch([0, 10, 5]), 0, 4, 16, 8, FAKE, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_index_varlen(batch([1, 10]), 0, 4, 16, 8, FAKE, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_index_varlen(good, 3, 4, 16, 8, FAKE, FAKE, 1 << 20, None) == 1    # mode
+    assert pv.pivot_index_varlen(good, 1, 4, 8, 16, FAKE, FAKE, 1 << 20, None) == 1    # C < k
+    assert pv.pivot_index_varlen(good, 1, 0, 16, 8, FAKE, FAKE, 1 << 20, None) == 1    # g
+    assert pv.pivot_index_varlen(good, 1, 4, 16, 8, FAKE, FAKE, 64, None) == 3         # workspace
+    assert pv.pivot_index_varlen(good, 1, 4, 16, 8, FAKE, FAKE + 16, 1 << 20, None) == 1
+    assert pv.pivot_index_varlen_workspace_size(batch([0, 10, 5]), 0, 4, 16, 8) == 0

@@ -96,3 +96,29 @@ def test_window_union_explicit_positions():
         sel = idx[r][idx[r] >= 0]
         u = oracle.window_union(sel, int(t), window)
         assert got[r, :len(u)].tolist() == list(u) and (got[r, len(u):] == -1).all()
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_ragged_batch_matches_each_sequence(mode):
+    """A packed batch of ragged sequences: every sequence's rows as the oracle
+    computes that sequence alone (power-of-two member counts, so exact)."""
+    lens = [1, 37, 300, 130, 514, 64]
+    g, C, kk = 4, 64, 16
+    parts = [gen.make_prefill(n, 4, 32, F32, kind="int", seed=100 + i) for i, n in enumerate(lens)]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    cat = lambda name: torch.cat([getattr(p, name) for p in parts]).cuda().contiguous()
+    batch = pv.make_varlen(cu.tolist(), cat("q"), None, cat("w"), cat("k"), None)
+    idx = pv.index_varlen(batch, mode, g, C, kk).cpu().numpy()
+    torch.cuda.synchronize()
+    assert pv.device_error() == 0
+    for i, p in enumerate(parts):
+        q, qs, w, k, ks = p.codes()
+        got = idx[cu[i]:cu[i + 1]]
+        if mode == 0:
+            want, _ = oracle.dense_index(F32, q, qs, w, k, ks, kk)
+        else:
+            opq, opqs, opw = oracle.proxy_reduce(F32, q, qs, w, g)
+            ocand, _ = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, p.L, g, C, kk)
+            want = (oracle.reuse(p.L, g, ocand, kk) if mode == 1 else
+                    oracle.refine(F32, q, qs, w, k, ks, g, ocand, kk)[0])
+        assert_rows_exact(got, want, f"sequence {i} (L={p.L}) mode {mode}")

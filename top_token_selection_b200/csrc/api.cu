@@ -677,6 +677,120 @@ pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* ca
     return PIVOT_OK;
 }
 
+// ------------------------------------------------------------------ ragged batch
+namespace {
+
+// Sequence i of a ragged batch as a single-sequence view (positions from 0).
+pivot_seq_t varlen_seq(const pivot_varlen_t* b, int i) {
+    const long long off = b->cu_seqlens[i];
+    const int es = esize_of(b->dtype);
+    pivot_seq_t s{};
+    s.dtype = b->dtype;
+    s.L = b->cu_seqlens[i + 1] - b->cu_seqlens[i];
+    s.H = b->H;
+    s.D = b->D;
+    s.q = static_cast<const uint8_t*>(b->q) + off * b->H * b->D * es;
+    s.q_scale = b->q_scale ? b->q_scale + off : nullptr;
+    s.w = b->w + off * b->H;
+    s.k = static_cast<const uint8_t*>(b->k) + off * b->D * es;
+    s.k_scale = b->k_scale ? b->k_scale + off : nullptr;
+    return s;
+}
+
+pivot_status_t check_varlen(const pivot_varlen_t* b, int mode, int g, int C, int topk) {
+    if (!b || b->nseq < 1 || !b->cu_seqlens || b->cu_seqlens[0] != 0) return PIVOT_ERR_INVALID_ARG;
+    if (mode < PIVOT_MODE_DENSE || mode > PIVOT_MODE_REFINE || topk < 1) return PIVOT_ERR_INVALID_ARG;
+    if (mode != PIVOT_MODE_DENSE && (g < 1 || C < topk)) return PIVOT_ERR_INVALID_ARG;
+    if (topk > MAX_K || (mode != PIVOT_MODE_DENSE && C > MAX_K)) return PIVOT_ERR_UNSUPPORTED;
+    for (int i = 0; i < b->nseq; ++i)
+        if (b->cu_seqlens[i + 1] < b->cu_seqlens[i]) return PIVOT_ERR_INVALID_ARG;
+    return PIVOT_OK;
+}
+
+// Workspace: proxies and candidates of the longest sequence, then the inner
+// workspace the single-sequence calls need.
+struct VarlenWs {
+    size_t pq, pqs, pw, cand, inner, total;
+};
+
+VarlenWs varlen_layout(const pivot_varlen_t* b, int mode, int g, int C, int topk) {
+    VarlenWs w{};
+    long long maxL = 0;
+    size_t inner = 0;
+    for (int i = 0; i < b->nseq; ++i) {
+        pivot_seq_t s = varlen_seq(b, i);
+        if (s.L < 1) continue;
+        if (s.L > maxL) maxL = s.L;
+        size_t need = mode == PIVOT_MODE_DENSE ? pivot_dense_index_workspace_size(&s, topk)
+                                               : pivot_proxy_scan_workspace_size(&s, g, C);
+        if (mode == PIVOT_MODE_REFINE) {
+            const size_t r = pivot_refine_workspace_size(&s, g, C, topk);
+            if (r > need) need = r;
+        }
+        if (need > inner) inner = need;
+    }
+    size_t off = 0;
+    if (mode != PIVOT_MODE_DENSE && maxL > 0) {
+        const size_t G = (size_t)ceil_div((int)maxL, g);
+        w.pq = off;
+        off = align_up(off + G * b->H * b->D * esize_of(b->dtype), WS_ALIGN);
+        w.pqs = off;
+        off = align_up(off + G * 4, WS_ALIGN);
+        w.pw = off;
+        off = align_up(off + G * b->H * 4, WS_ALIGN);
+        w.cand = off;
+        off = align_up(off + G * C * 4, WS_ALIGN);
+    }
+    w.inner = off;
+    w.total = align_up(off + inner, WS_ALIGN);
+    return w;
+}
+
+}  // namespace
+
+size_t pivot_index_varlen_workspace_size(const pivot_varlen_t* batch, int32_t mode, int32_t g,
+                                         int32_t C, int32_t topk) {
+    if (check_varlen(batch, mode, g, C, topk) != PIVOT_OK) return 0;
+    return varlen_layout(batch, mode, g, C, topk).total;
+}
+
+pivot_status_t pivot_index_varlen(const pivot_varlen_t* batch, int32_t mode, int32_t g, int32_t C,
+                                  int32_t topk, int32_t* idx, void* ws, size_t ws_bytes,
+                                  void* stream) {
+    pivot_status_t st = check_varlen(batch, mode, g, C, topk);
+    if (st != PIVOT_OK) return st;
+    if (!idx || !ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
+    const VarlenWs lay = varlen_layout(batch, mode, g, C, topk);
+    if (ws_bytes < lay.total) return PIVOT_ERR_WORKSPACE;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    const size_t inner_bytes = ws_bytes - lay.inner;
+    for (int i = 0; i < batch->nseq; ++i) {
+        pivot_seq_t s = varlen_seq(batch, i);
+        if (s.L < 1) continue;
+        int32_t* out = idx + (size_t)batch->cu_seqlens[i] * topk;
+        if (mode == PIVOT_MODE_DENSE) {
+            st = pivot_dense_index(&s, topk, out, nullptr, base + lay.inner, inner_bytes, stream);
+        } else {
+            void* pq = base + lay.pq;
+            float* pqs = batch->dtype == PIVOT_E4M3 ? reinterpret_cast<float*>(base + lay.pqs)
+                                                   : nullptr;
+            float* pw = reinterpret_cast<float*>(base + lay.pw);
+            int32_t* cand = reinterpret_cast<int32_t*>(base + lay.cand);
+            st = pivot_proxy_reduce(&s, g, pq, pqs, pw, stream);
+            if (st == PIVOT_OK)
+                st = pivot_proxy_scan(&s, g, pq, pqs, pw, C, topk, cand, nullptr, base + lay.inner,
+                                      inner_bytes, stream);
+            if (st == PIVOT_OK)
+                st = mode == PIVOT_MODE_REUSE
+                         ? pivot_reuse(0, s.L, g, cand, C, topk, out, stream)
+                         : pivot_refine(&s, g, cand, C, topk, out, nullptr, base + lay.inner,
+                                        inner_bytes, stream);
+        }
+        if (st != PIVOT_OK) return st;
+    }
+    return PIVOT_OK;
+}
+
 // ------------------------------------------------------------------ decode
 static pivot_status_t check_decode(const pivot_decode_t* b) {
     if (!b || !dtype_ok(b->dtype)) return PIVOT_ERR_INVALID_ARG;

@@ -31,7 +31,8 @@ ABI_SYMBOLS = [
     "pivot_get_device_error", "pivot_set_wait_limit_ns", "pivot_selftest_wait_timeout",
     "pivot_status_string", "pivot_version", "pivot_profile_enable", "pivot_profile_read",
     "pivot_launch_count", "pivot_decode_noalloc", "pivot_last_error_detail",
-    "pivot_reuse_backfill", "pivot_window_union",
+    "pivot_reuse_backfill", "pivot_window_union", "pivot_index_varlen",
+    "pivot_index_varlen_workspace_size",
 ]
 KERNELS = {0: "scan", 1: "select", 2: "refine", 3: "reduce", 4: "reuse"}
 
@@ -47,6 +48,13 @@ class PivotSeq(ctypes.Structure):
                 ("D", ctypes.c_int32), ("q", ctypes.c_void_p), ("q_scale", ctypes.c_void_p),
                 ("w", ctypes.c_void_p), ("k", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
                 ("t_begin", ctypes.c_int32), ("t_end", ctypes.c_int32)]
+
+
+class PivotVarlen(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int32), ("nseq", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p), ("q", ctypes.c_void_p),
+                ("q_scale", ctypes.c_void_p), ("w", ctypes.c_void_p), ("k", ctypes.c_void_p),
+                ("k_scale", ctypes.c_void_p)]
 
 
 class PivotDecode(ctypes.Structure):
@@ -93,6 +101,8 @@ def load(path: str = LIB_PATH):
         "pivot_last_error_detail": ([], ctypes.c_char_p),
         "pivot_reuse_backfill": ([I32, I32, I32, P, P, I32, I32, P, P], I32),
         "pivot_window_union": ([P, I32, I32, I32, P, I32, P, P], I32),
+        "pivot_index_varlen": ([P, I32, I32, I32, I32, P, P, SZ, P], I32),
+        "pivot_index_varlen_workspace_size": ([P, I32, I32, I32, I32], SZ),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -252,6 +262,36 @@ def make_seq(q, q_scale, w, k, k_scale, t_begin=0, t_end=0) -> PivotSeq:
                  t_begin, t_end)
     s._keep = (q, q_scale, w, k, k_scale)
     return s
+
+
+def make_varlen(cu_seqlens, q, q_scale, w, k, k_scale) -> PivotVarlen:
+    """Describe a ragged batch: cu_seqlens is a host sequence of nseq + 1
+    row offsets; the struct keeps it and the tensors alive."""
+    cu = (ctypes.c_int32 * len(cu_seqlens))(*[int(x) for x in cu_seqlens])
+    _, H, D = q.shape
+    s = PivotVarlen(_dtype_code(q), len(cu_seqlens) - 1, H, D, ctypes.addressof(cu), _p(q),
+                    _p(q_scale), _p(w), _p(k), _p(k_scale))
+    s._keep = (cu, q, q_scale, w, k, k_scale)
+    return s
+
+
+def pivot_index_varlen(batch, mode, g, C, topk, idx, ws, ws_bytes, stream):
+    return load().pivot_index_varlen(ctypes.byref(batch), mode, g, C, topk, idx, ws, ws_bytes,
+                                     stream)
+
+
+def pivot_index_varlen_workspace_size(batch, mode, g, C, topk):
+    return load().pivot_index_varlen_workspace_size(ctypes.byref(batch), mode, g, C, topk)
+
+
+def index_varlen(batch: PivotVarlen, mode, g, C, topk, ws=None, stream=None, device="cuda"):
+    total = batch._keep[0][batch.nseq]
+    idx = torch.empty(total, topk, dtype=torch.int32, device=device)
+    if ws is None:
+        ws = _workspace(pivot_index_varlen_workspace_size(batch, mode, g, C, topk), device)
+    _check(pivot_index_varlen(batch, mode, g, C, topk, _p(idx), _p(ws), ws.numel(),
+                              _stream(stream)), "pivot_index_varlen")
+    return idx
 
 
 def make_decode(q, q_scale, w, kc, kc_scale, cache_len) -> PivotDecode:
