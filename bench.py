@@ -381,6 +381,27 @@ def config_of(wl, args):
             "l2": "no flush: inputs and score buffers larger than L2 (q alone 1 GiB)"}
 
 
+def scan_traffic_per_pair():
+    """DRAM bytes per causal pair of the scan kernel from its committed ncu
+    summary, or None once the kernel sources differ from the captured ones."""
+    import hashlib
+    import re
+    prof = os.path.join(ROOT, "profiles", "index_umma_dense_fp8_L16384.md")
+    try:
+        text = open(prof).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_pair=([0-9.]+) sources=(\S+)", text)
+    if not m:
+        return None
+    for item in m.group(2).split(","):
+        name, digest = item.split(":")
+        src = os.path.join(ROOT, "top_token_selection_b200", "csrc", name)
+        if hashlib.sha1(open(src, "rb").read()).hexdigest()[:len(digest)] != digest:
+            return None
+    return float(m.group(1))
+
+
 def _event_ms(fn, stream, reps):
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     fn()
@@ -539,8 +560,14 @@ def run_ours(args, wl):
         roof = None
     elif dom in ("scan", "refine"):
         ach = dv["tflops"]
+        bpp = scan_traffic_per_pair() if dom == "scan" else None
+        pairs_per_launch = dv["work"] / max(dv["launches"], 1)
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": tc_peak,
-                "unit": "TFLOP/s", "frac": ach / tc_peak, "traffic": None,
+                "unit": "TFLOP/s", "frac": ach / tc_peak,
+                "traffic": None if bpp is None else bpp * pairs_per_launch,
+                "traffic_source": None if bpp is None else
+                    "ncu dram bytes of the dense scan at L=16384 (profiles/), per causal pair, "
+                    "times this run's pairs per launch",
                 "peak_source": f"{peak_src} bf16 sustained x {FP8_OVER_BF16 if fp8 else 1.0} "
                                f"({'fp8' if fp8 else 'bf16'} nominal ratio)",
                 "frac_of_burst": ach / tc_peak_burst,

@@ -211,6 +211,9 @@ WORKLOADS = {
     "dsa_prefill_64k": dict(L=65536, H=64, D=128, dtype=BF16, kind="dsa", topk=2048, g=8, C=4096),
     "long_prefill_128k_fp8": dict(L=131072, H=64, D=128, dtype=E4M3, kind="dsa", topk=2048, g=8,
                                   C=4096),
+    # the long_prefill_128k_fp8 configuration at L=16384: small enough for
+    # full profiler captures, scores still far larger than L2
+    "fp8_prefill_16k": dict(L=16384, H=64, D=128, dtype=E4M3, kind="dsa", topk=2048, g=8, C=4096),
     "mtp_decode_b32": dict(B=32, Gm=2, H=64, D=128, dtype=E4M3, len_lo=32768, len_hi=131072,
                            topk=2048, C=4096),
 }
