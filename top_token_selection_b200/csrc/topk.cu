@@ -309,6 +309,7 @@ __device__ void write_marked(const uint64_t* buf, int cnt, const uint32_t* bm, u
     bitmap_prefix(bm, pref, W, scratch);
     for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
         const uint64_t k = buf[i];
+        if (k == 0) continue;   // an empty slot (candidate rows keep them in place)
         const int pos = key_pos(k);
         if (bit_of(bm, pos)) {
             const uint32_t slot = base + rank_of(bm, pref, pos);
@@ -414,6 +415,35 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
         const bool a = threadIdx.x < 4 && i < v.n;
         const uint32_t u = a ? ordered_key(v.S[i]) : 0u;
         warp_append(buf, s_cnt, cap, make_key(u, i), a && u >= T);
+    } else if (v.cand && v.n <= cap) {
+        // Candidate rows that fit the buffer keep every entry in place
+        // (slot = entry index, key 0 where the candidate is not eligible,
+        // which every later step skips): no compaction, and each thread
+        // issues the loads of eight entries together.
+        constexpr int U = 8;
+        for (int i0 = 0; i0 < v.n; i0 += SEL_THREADS * U) {
+            int pos[U];
+            float x[U];
+#pragma unroll
+            for (int j = 0; j < U; ++j) {
+                const int i = i0 + j * SEL_THREADS + threadIdx.x;
+                pos[j] = i < v.n ? v.cand[i] : -1;
+                x[j] = i < v.n ? v.S[i] : 0.0f;
+            }
+            if (v.ksc) {
+#pragma unroll
+                for (int j = 0; j < U; ++j)
+                    if (pos[j] >= 0 && pos[j] <= v.lim) x[j] = x[j] * v.ksc[pos[j]];
+            }
+#pragma unroll
+            for (int j = 0; j < U; ++j) {
+                const int i = i0 + j * SEL_THREADS + threadIdx.x;
+                const bool ok = pos[j] >= 0 && pos[j] <= v.lim;
+                if (i < v.n) buf[i] = ok ? make_key(ordered_key(x[j]), pos[j]) : 0ull;
+                nvalid_local += ok;
+            }
+        }
+        if (threadIdx.x == 0) *s_cnt = (uint32_t)v.n;
     } else {
         for (int i0 = 0; i0 < v.n; i0 += SEL_THREADS) {
             const int i = i0 + threadIdx.x;
