@@ -279,16 +279,38 @@ __device__ __forceinline__ uint32_t rank_of(const uint32_t* bm, const uint32_t* 
 
 // Mark in `bm` the kept entries with u > Tu, plus the `need` lowest-position
 // entries with u == Tu.  `tie` is a scratch bitmap, `pref` scratch prefixes.
+// When every entry equal to Tu is taken (the usual case: one of them), the
+// ranking of the ties is skipped.
 __device__ void mark_top(const uint64_t* buf, int cnt, uint32_t Tu, uint32_t need, uint32_t* bm,
                          uint32_t* tie, uint32_t* pref, int W, uint32_t* scratch) {
-    for (int w = threadIdx.x; w < W; w += SEL_THREADS) tie[w] = 0;
-    __syncthreads();
+    uint32_t nties = 0;
     for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
         const uint64_t k = buf[i];
         const uint32_t u = key_u(k);
         const int pos = key_pos(k);
         if (u > Tu) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
-        else if (u == Tu) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
+        else if (u == Tu) ++nties;
+    }
+    nties = block_sum_u32(nties, scratch);   // also orders the marks above
+    if (nties <= need) {
+        for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
+            const uint64_t k = buf[i];
+            if (key_u(k) == Tu) {
+                const int pos = key_pos(k);
+                atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+            }
+        }
+        __syncthreads();
+        return;
+    }
+    for (int w = threadIdx.x; w < W; w += SEL_THREADS) tie[w] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
+        const uint64_t k = buf[i];
+        if (key_u(k) == Tu) {
+            const int pos = key_pos(k);
+            atomicOr(&tie[pos >> 5], 1u << (pos & 31));
+        }
     }
     __syncthreads();
     bitmap_prefix(tie, pref, W, scratch);
