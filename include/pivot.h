@@ -200,6 +200,24 @@ pivot_status_t pivot_index_varlen(const pivot_varlen_t* batch, int32_t mode, int
 size_t pivot_index_varlen_workspace_size(const pivot_varlen_t* batch, int32_t mode, int32_t g,
                                          int32_t C, int32_t topk);
 
+/* The other variant of the window section of "Sparse Attention의 Indexer"
+ * (the paragraph after Fig. 3): the recent window [t - window + 1, t] is kept
+ * out of the indexer's candidates, so the whole choice of topk falls outside
+ * it, and the window is read besides.  Row t (t_begin <= t < t_end): the
+ * chosen mode (PIVOT_MODE_DENSE, _REUSE, _REFINE, as pivot_dense_index /
+ * pivot_reuse / pivot_refine compute them) over positions <= t - window
+ * only (the proxy scan still covers its group's whole prefix; its members
+ * drop the later candidates), then every position of
+ * [max(0, t - window + 1), t]; ascending, -1 padded.
+ * idx [rows, topk + window] device.  g, C as for pivot_proxy_scan (unused in
+ * dense mode); window >= 1.  ws of pivot_index_window_outside_workspace_size
+ * bytes, 256-byte aligned. */
+pivot_status_t pivot_index_window_outside(const pivot_seq_t* seq, int32_t mode, int32_t g,
+                                          int32_t C, int32_t topk, int32_t window, int32_t* idx,
+                                          void* ws, size_t ws_bytes, void* stream);
+size_t pivot_index_window_outside_workspace_size(const pivot_seq_t* seq, int32_t mode, int32_t g,
+                                                 int32_t C, int32_t topk, int32_t window);
+
 /* The selected positions united with a recent window ("Sparse Attention의
  * Indexer", Fig. 3 and the paragraph after it: a sliding window added to the
  * indexer's choice, the window's positions counted once).  This is the

@@ -231,6 +231,36 @@ def reuse_backfill(L, g, cand, cand_score, topk, rows=None):
     return out
 
 
+def index_window_outside(dtype, q, q_scale, w, k, k_scale, mode, g, C, topk, window, rows=None):
+    """The window kept out of the candidates: row t chooses by `mode` (DENSE,
+    REUSE, REFINE) among positions <= t - window only, then the window
+    [t - window + 1, t] is added.  [rows, topk + window], ascending, -1 padded.
+    Built from the functions above, row by row (small inputs only)."""
+    L = q.shape[0]
+    rows = _rows(rows, L)
+    out = np.full((len(rows), topk + window), -1, dtype=np.int32)
+    if mode != DENSE:
+        pq, pqs, pw = proxy_reduce(dtype, q, q_scale, w, g)
+        cand, _ = proxy_scan(dtype, pq, pqs, pw, k, k_scale, L, g, C, topk)
+    for r, t in enumerate(rows):
+        lim = t - window
+        if mode == REUSE:
+            sel = [s for s in cand[t // g, :topk] if 0 <= s <= lim]
+        else:
+            if mode == DENSE:
+                pos = np.arange(0, lim + 1, dtype=np.int32)
+            else:
+                pos = np.array([s for s in cand[t // g] if 0 <= s <= lim], dtype=np.int32)
+            sel = []
+            if len(pos):
+                sc = score_positions(dtype, q, q_scale, w, k, k_scale, t, pos)
+                order = np.lexsort((pos, -sc))[:topk]
+                sel = sorted(pos[order].tolist())
+        u = window_union(np.array(sel, dtype=np.int32), int(t), window)
+        out[r, :len(u)] = u
+    return out
+
+
 def window_union_rows(idx, t_first, window):
     """Each index row (ascending, -1 padded) united with its window
     [t - window + 1, t], t = t_first + row: [rows, k + window], -1 padded."""

@@ -148,3 +148,15 @@ def test_ragged_batch_rejects_bad_arguments(lib):
     assert pv.pivot_index_varlen(good, 1, 4, 16, 8, FAKE, FAKE, 64, None) == 3         # workspace
     assert pv.pivot_index_varlen(good, 1, 4, 16, 8, FAKE, FAKE + 16, 1 << 20, None) == 1
     assert pv.pivot_index_varlen_workspace_size(batch([0, 10, 5]), 0, 4, 16, 8) == 0
+
+
+def test_window_outside_rejects_bad_arguments(lib):
+    seq = _seq()
+    assert pv.pivot_index_window_outside(seq, 0, 4, 16, 8, 0, FAKE, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_index_window_outside(seq, 3, 4, 16, 8, 4, FAKE, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_index_window_outside(seq, 1, 4, 8, 16, 4, FAKE, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_index_window_outside(seq, 1, 0, 16, 8, 4, FAKE, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_index_window_outside(seq, 0, 4, 16, 8, 4, None, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_index_window_outside(seq, 0, 4, 16, 8, 4, FAKE, FAKE, 64, None) == 3
+    assert pv.pivot_index_window_outside_workspace_size(seq, 2, 4, 16, 8, 4) > 0
+    assert pv.pivot_index_window_outside_workspace_size(seq, 2, 4, 16, 8, 0) == 0

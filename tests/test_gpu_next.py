@@ -122,3 +122,16 @@ def test_ragged_batch_matches_each_sequence(mode):
             want = (oracle.reuse(p.L, g, ocand, kk) if mode == 1 else
                     oracle.refine(F32, q, qs, w, k, ks, g, ocand, kk)[0])
         assert_rows_exact(got, want, f"sequence {i} (L={p.L}) mode {mode}")
+
+
+@pytest.mark.parametrize("mode,window", [(0, 1), (0, 5), (0, 64), (1, 5), (2, 5), (2, 64)])
+def test_window_outside_exact(tiny, mode, window):
+    """The window kept out of the candidates, then added: bit for bit."""
+    p, dev, cfg = tiny
+    g, C, kk = cfg["g"], cfg["C"], cfg["topk"]
+    out = pv.index_window_outside(seq_of(dev), mode, g, C, kk, window)
+    torch.cuda.synchronize()
+    assert pv.device_error() == 0
+    q, qs, w, k, ks = p.codes()
+    want = oracle.index_window_outside(F32, q, qs, w, k, ks, mode, g, C, kk, window)
+    assert_rows_exact(out.cpu(), want, f"window outside mode {mode} w={window}")

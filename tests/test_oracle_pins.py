@@ -439,3 +439,14 @@ def test_window_union_rows_matches_the_example(golden_dir):
     u = out[0][out[0] >= 0].tolist()
     assert u == ex["union"]
     assert out.shape == (1, len(ex["selected"]) + 1 + ex["window"])
+
+
+def test_window_outside_derived_example(golden_dir):
+    ex = _load(golden_dir, "indexer_tutorial_example.json")
+    q, w, k = _tutorial_seq(ex)
+    case = ex["cases"][0]
+    q[case["position"], 0] = case["query"]
+    wo = ex["window_outside"]
+    out = oracle.index_window_outside(F32, q, None, w, k, None, oracle.DENSE, 1, 8, 3,
+                                      wo["window"], rows=[wo["position"]])
+    assert out[0][out[0] >= 0].tolist() == wo["union"]

@@ -235,8 +235,11 @@ int decode_dense_rows(int Gm, int H, int D, int dtype) {
 pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, int Gm, int maxlen,
                                  const int32_t* cache_len, const float* S, long long stride,
                                  int K, int split, int npos, int32_t* out, float* out_score,
-                                 int out_base, cudaStream_t st, uint32_t* thresh = nullptr) {
+                                 int out_base, cudaStream_t st, uint32_t* thresh = nullptr,
+                                 int lim_shift = 0, int out_stride = 0) {
     SelectParams sp{};
+    sp.lim_shift = lim_shift;
+    sp.out_stride = out_stride;
     sp.split = split;
     sp.npos = npos;
     sp.kind = SEL_PREFIX;
@@ -271,7 +274,7 @@ pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int 
                                const int32_t* cache_len, const float* S, const int32_t* cand,
                                int cand_base, int C, int K, int npos, int32_t* out,
                                float* out_score, int out_base, cudaStream_t st,
-                               const float* key_scale) {
+                               const float* key_scale, int lim_shift = 0, int out_stride = 0) {
     SelectParams sp{};
     sp.npos = npos;
     sp.kind = SEL_CANDIDATES;
@@ -290,6 +293,8 @@ pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int 
     sp.C = C;
     sp.K = K;
     sp.key_scale = key_scale;
+    sp.lim_shift = lim_shift;
+    sp.out_stride = out_stride;
     sp.out_idx = out;
     sp.out_score = out_score;
     sp.out_base = out_base;
@@ -470,8 +475,11 @@ size_t pivot_dense_index_workspace_size(const pivot_seq_t* seq, int32_t topk) {
     return align_up((size_t)rows * rb, WS_ALIGN);
 }
 
-pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* idx, float* score,
-                                 void* ws, size_t ws_bytes, void* stream) {
+// lim_shift > 0 keeps the last lim_shift positions of every row out of the
+// choice; out_stride (0: topk) is the row stride of idx / score.
+static pivot_status_t dense_index_impl(const pivot_seq_t* seq, int32_t topk, int32_t* idx,
+                                       float* score, void* ws, size_t ws_bytes, void* stream,
+                                       int lim_shift, int out_stride) {
     int t0, t1;
     pivot_status_t st = check_seq(seq, &t0, &t1);
     if (st != PIVOT_OK) return st;
@@ -493,10 +501,15 @@ pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* 
                       r1, r1 - 1, S, stride, s);
         if (st != PIVOT_OK) return st;
         st = run_select_prefix(SCAN_PREFILL_DENSE, r0, r1, seq->L, 1, 1, 0, nullptr, S, stride,
-                               topk, 0, seq->L, idx, score, t0, s, thresh);
+                               topk, 0, seq->L, idx, score, t0, s, thresh, lim_shift, out_stride);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;
+}
+
+pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* idx, float* score,
+                                 void* ws, size_t ws_bytes, void* stream) {
+    return dense_index_impl(seq, topk, idx, score, ws, ws_bytes, stream, 0, 0);
 }
 
 // ------------------------------------------------------------ proxy reduce
@@ -646,9 +659,9 @@ size_t pivot_refine_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C,
     return align_up((size_t)rows * rb, WS_ALIGN);
 }
 
-pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* cand, int32_t C,
-                            int32_t topk, int32_t* idx, float* score, void* ws, size_t ws_bytes,
-                            void* stream) {
+static pivot_status_t refine_impl(const pivot_seq_t* seq, int32_t g, const int32_t* cand,
+                                  int32_t C, int32_t topk, int32_t* idx, float* score, void* ws,
+                                  size_t ws_bytes, void* stream, int lim_shift, int out_stride) {
     int t0, t1;
     pivot_status_t st = check_seq(seq, &t0, &t1);
     if (st != PIVOT_OK) return st;
@@ -671,10 +684,16 @@ pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* ca
         if (st != PIVOT_OK) return st;
         st = run_select_cand(SCAN_PREFILL_DENSE, r0, r1, seq->L, g, 1, 0, nullptr, S,
                              cand + (size_t)(jc - j0) * C, jc, C, topk, seq->L, idx, score, t0, s,
-                             seq->k_scale);
+                             seq->k_scale, lim_shift, out_stride);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;
+}
+
+pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* cand, int32_t C,
+                            int32_t topk, int32_t* idx, float* score, void* ws, size_t ws_bytes,
+                            void* stream) {
+    return refine_impl(seq, g, cand, C, topk, idx, score, ws, ws_bytes, stream, 0, 0);
 }
 
 // ------------------------------------------------------------------ ragged batch
@@ -789,6 +808,106 @@ pivot_status_t pivot_index_varlen(const pivot_varlen_t* batch, int32_t mode, int
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;
+}
+
+// ------------------------------------------------------------------ window kept out
+namespace {
+
+struct WinWs {
+    size_t pq, pqs, pw, cand, inner, total;
+};
+
+WinWs window_layout(const pivot_seq_t* seq, int t0, int t1, int mode, int g, int C, int topk) {
+    WinWs w{};
+    size_t off = 0, inner;
+    if (mode == PIVOT_MODE_DENSE) {
+        inner = pivot_dense_index_workspace_size(seq, topk);
+    } else {
+        const size_t G = (size_t)(ceil_div(t1, g) - t0 / g);
+        w.pq = off;
+        off = align_up(off + G * seq->H * seq->D * esize_of(seq->dtype), WS_ALIGN);
+        w.pqs = off;
+        off = align_up(off + G * 4, WS_ALIGN);
+        w.pw = off;
+        off = align_up(off + G * seq->H * 4, WS_ALIGN);
+        w.cand = off;
+        off = align_up(off + G * C * 4, WS_ALIGN);
+        inner = pivot_proxy_scan_workspace_size(seq, g, C);
+        if (mode == PIVOT_MODE_REFINE) {
+            const size_t r = pivot_refine_workspace_size(seq, g, C, topk);
+            if (r > inner) inner = r;
+        }
+    }
+    w.inner = off;
+    w.total = align_up(off + inner, WS_ALIGN);
+    return w;
+}
+
+pivot_status_t check_window(const pivot_seq_t* seq, int mode, int g, int C, int topk,
+                            int window, int* t0, int* t1) {
+    pivot_status_t st = check_seq(seq, t0, t1);
+    if (st != PIVOT_OK) return st;
+    if (mode < PIVOT_MODE_DENSE || mode > PIVOT_MODE_REFINE || topk < 1 || window < 1)
+        return PIVOT_ERR_INVALID_ARG;
+    if (mode != PIVOT_MODE_DENSE) {
+        if ((st = check_group_range(seq, g, *t0, *t1)) != PIVOT_OK) return st;
+        if (C < topk) return PIVOT_ERR_INVALID_ARG;
+        if (C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
+    }
+    if (topk > MAX_K) return PIVOT_ERR_UNSUPPORTED;
+    return PIVOT_OK;
+}
+
+}  // namespace
+
+size_t pivot_index_window_outside_workspace_size(const pivot_seq_t* seq, int32_t mode, int32_t g,
+                                                 int32_t C, int32_t topk, int32_t window) {
+    int t0, t1;
+    if (check_window(seq, mode, g, C, topk, window, &t0, &t1) != PIVOT_OK) return 0;
+    return window_layout(seq, t0, t1, mode, g, C, topk).total;
+}
+
+pivot_status_t pivot_index_window_outside(const pivot_seq_t* seq, int32_t mode, int32_t g,
+                                          int32_t C, int32_t topk, int32_t window, int32_t* idx,
+                                          void* ws, size_t ws_bytes, void* stream) {
+    int t0, t1;
+    pivot_status_t st = check_window(seq, mode, g, C, topk, window, &t0, &t1);
+    if (st != PIVOT_OK) return st;
+    if (!idx || !ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
+    const WinWs lay = window_layout(seq, t0, t1, mode, g, C, topk);
+    if (ws_bytes < lay.total) return PIVOT_ERR_WORKSPACE;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    void* inner = base + lay.inner;
+    const size_t inner_bytes = ws_bytes - lay.inner;
+    const int stride = topk + window;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // 1. the indexer's choice among positions <= t - window, rows at stride topk + window
+    if (mode == PIVOT_MODE_DENSE) {
+        st = dense_index_impl(seq, topk, idx, nullptr, inner, inner_bytes, stream, window, stride);
+    } else {
+        void* pq = base + lay.pq;
+        float* pqs = seq->dtype == PIVOT_E4M3 ? reinterpret_cast<float*>(base + lay.pqs) : nullptr;
+        float* pw = reinterpret_cast<float*>(base + lay.pw);
+        int32_t* cand = reinterpret_cast<int32_t*>(base + lay.cand);
+        st = pivot_proxy_reduce(seq, g, pq, pqs, pw, stream);
+        if (st == PIVOT_OK)
+            st = pivot_proxy_scan(seq, g, pq, pqs, pw, C, topk, cand, nullptr, inner, inner_bytes,
+                                  stream);
+        if (st == PIVOT_OK) {
+            if (mode == PIVOT_MODE_REUSE)
+                st = from_cuda(profiled(PK_REUSE, 0.0, s, [&] {
+                    return launch_reuse(t0, t1, g, cand, C, topk, idx, s, window, stride);
+                }));
+            else
+                st = refine_impl(seq, g, cand, C, topk, idx, nullptr, inner, inner_bytes, stream,
+                                 window, stride);
+        }
+    }
+    if (st != PIVOT_OK) return st;
+    // 2. the window appended after each row's choice, in place
+    return from_cuda(profiled(PK_REUSE, 0.0, s, [&] {
+        return launch_window_union(idx, t1 - t0, topk, t0, nullptr, window, idx, s, stride);
+    }));
 }
 
 // ------------------------------------------------------------------ decode

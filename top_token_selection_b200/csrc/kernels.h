@@ -75,6 +75,8 @@ struct SelectParams {
     int fast_cap;         // set by launch_select: kept-entry capacity of the fast path
     int bitmap_words;     // set by launch_select
     int s_per_group;          // SEL_CANDIDATES: S rows are per group (grp - cand_base), not per row
+    int lim_shift;            // positions considered are <= lim(r) - lim_shift (a window kept out)
+    int out_stride;           // output row stride in entries (0: K)
     const float* key_scale;   // SEL_CANDIDATES: if set, entry i's score is S * key_scale[kb + pos]
                               // (kb = grp * maxlen for decode rows, else 0)
     const uint32_t* thresh;   // SEL_PREFIX: row r's lower bound at thresh[r - row0]
@@ -102,13 +104,16 @@ struct ReduceParams {
 };
 cudaError_t launch_proxy_reduce(const ReduceParams& p, cudaStream_t stream);
 
+// lim_shift: members keep candidates <= t - lim_shift; out_stride 0: topk.
 cudaError_t launch_reuse(int t_begin, int t_end, int g, const int32_t* cand, int C, int topk,
-                         int32_t* idx, cudaStream_t stream);
+                         int32_t* idx, cudaStream_t stream, int lim_shift = 0,
+                         int out_stride = 0);
 // Each index row (ascending, -1 padded, k entries) united with the window
 // [t - window + 1, t] (t = positions[r], or t_begin + r): out [rows, k + window].
+// idx rows at stride in_stride (0: k); out may be idx with in_stride = k + window.
 cudaError_t launch_window_union(const int32_t* idx, int rows, int k, int t_begin,
                                 const int32_t* positions, int window, int32_t* out,
-                                cudaStream_t stream);
+                                cudaStream_t stream, int in_stride = 0);
 cudaError_t launch_decode_reuse(int B, int Gm, int maxlen, const int32_t* cache_len,
                                 const int32_t* cand, int C, int topk, int32_t* idx,
                                 cudaStream_t stream);

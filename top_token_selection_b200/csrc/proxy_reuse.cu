@@ -105,11 +105,11 @@ __device__ __forceinline__ void reuse_row(const int32_t* c, int topk, int lim, i
 }
 
 __global__ void reuse_kernel(int t_begin, int t_end, int g, const int32_t* cand, int C, int topk,
-                             int32_t* idx) {
+                             int32_t* idx, int lim_shift, int out_stride) {
     const int t = t_begin + blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (t >= t_end) return;
     const int j = t / g - t_begin / g;
-    reuse_row(cand + (size_t)j * C, topk, t, idx + (size_t)(t - t_begin) * topk);
+    reuse_row(cand + (size_t)j * C, topk, t - lim_shift, idx + (size_t)(t - t_begin) * out_stride);
 }
 
 __global__ void decode_reuse_kernel(int B, int Gm, int maxlen, const int32_t* cache_len,
@@ -131,13 +131,16 @@ __global__ void decode_reuse_kernel(int B, int Gm, int maxlen, const int32_t* ca
 // is its entries below a followed by a..t (entries in [a, t] are the window's
 // own).  One warp per row.
 __global__ void window_union_kernel(const int32_t* idx, int rows, int k, int t_begin,
-                                    const int32_t* positions, int window, int32_t* out) {
+                                    const int32_t* positions, int window, int32_t* out,
+                                    int in_stride) {
     const int r = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (r >= rows) return;
     const int lane = threadIdx.x & 31;
     const int t = positions ? positions[r] : t_begin + r;
     const int a = t - window + 1 > 0 ? t - window + 1 : 0;
-    const int32_t* in = idx + (size_t)r * k;
+    // in place (out == idx, in_stride == k + window) every read of a chunk
+    // precedes its writes, which never pass the entries read
+    const int32_t* in = idx + (size_t)r * in_stride;
     int32_t* o = out + (size_t)r * (k + window);
     int n = 0;
     for (int i0 = 0; i0 < k; i0 += 32) {
@@ -157,11 +160,11 @@ __global__ void window_union_kernel(const int32_t* idx, int rows, int k, int t_b
 
 cudaError_t launch_window_union(const int32_t* idx, int rows, int k, int t_begin,
                                 const int32_t* positions, int window, int32_t* out,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, int in_stride) {
     if (rows <= 0) return cudaSuccess;
     const int wpb = 8;
-    window_union_kernel<<<ceil_div(rows, wpb), wpb * 32, 0, stream>>>(idx, rows, k, t_begin,
-                                                                       positions, window, out);
+    window_union_kernel<<<ceil_div(rows, wpb), wpb * 32, 0, stream>>>(
+        idx, rows, k, t_begin, positions, window, out, in_stride ? in_stride : k);
     return cudaGetLastError();
 }
 
@@ -187,12 +190,12 @@ cudaError_t launch_proxy_reduce(const ReduceParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_reuse(int t_begin, int t_end, int g, const int32_t* cand, int C, int topk,
-                         int32_t* idx, cudaStream_t stream) {
+                         int32_t* idx, cudaStream_t stream, int lim_shift, int out_stride) {
     const int rows = t_end - t_begin;
     if (rows <= 0) return cudaSuccess;
     const int wpb = 8;
-    reuse_kernel<<<ceil_div(rows, wpb), wpb * 32, 0, stream>>>(t_begin, t_end, g, cand, C, topk,
-                                                                idx);
+    reuse_kernel<<<ceil_div(rows, wpb), wpb * 32, 0, stream>>>(
+        t_begin, t_end, g, cand, C, topk, idx, lim_shift, out_stride ? out_stride : topk);
     return cudaGetLastError();
 }
 

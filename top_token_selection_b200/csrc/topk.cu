@@ -796,8 +796,9 @@ __global__ void __launch_bounds__(THR_WARPS * 32) row_threshold_kernel(const Sel
     if (rr >= p.nrows) return;
     const int r = p.row0 + rr;
     bool ok;
-    const int lim = row_limit(p.scan_kind, r, p.L, p.g, p.Gm, p.maxlen, p.cache_len, ok);
-    const int n = ok ? lim + 1 : 0;
+    const int lim =
+        row_limit(p.scan_kind, r, p.L, p.g, p.Gm, p.maxlen, p.cache_len, ok) - p.lim_shift;
+    const int n = ok && lim >= 0 ? lim + 1 : 0;
     uint32_t T = 1;
     if (n > p.fast_cap) {
         const float* S = p.S + (size_t)rr * p.S_stride;
@@ -859,18 +860,20 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const SelectParams 
     __shared__ uint32_t s_a, s_b;
 
     const int r = p.row0 + blockIdx.x;
-    int32_t* out = p.out_idx + (size_t)(r - p.out_base) * p.K;
-    float* outs = p.out_score ? p.out_score + (size_t)(r - p.out_base) * p.K : nullptr;
+    const size_t ostride = p.out_stride ? (size_t)p.out_stride : (size_t)p.K;
+    int32_t* out = p.out_idx + (size_t)(r - p.out_base) * ostride;
+    float* outs = p.out_score ? p.out_score + (size_t)(r - p.out_base) * ostride : nullptr;
 
     bool ok;
-    const int lim = row_limit(p.scan_kind, r, p.L, p.g, p.Gm, p.maxlen, p.cache_len, ok);
+    const int lim =
+        row_limit(p.scan_kind, r, p.L, p.g, p.Gm, p.maxlen, p.cache_len, ok) - p.lim_shift;
     RowView v;
     v.S = p.S + (size_t)(r - p.row0) * p.S_stride;
     v.lim = lim;
     v.ksc = nullptr;
     if (p.kind == SEL_PREFIX) {
         v.cand = nullptr;
-        v.n = ok ? lim + 1 : 0;
+        v.n = ok && lim >= 0 ? lim + 1 : 0;
     } else {
         const bool dec = p.scan_kind == SCAN_DECODE_DENSE;
         const int grp = dec ? r / p.Gm : r / p.g;

@@ -32,7 +32,8 @@ ABI_SYMBOLS = [
     "pivot_status_string", "pivot_version", "pivot_profile_enable", "pivot_profile_read",
     "pivot_launch_count", "pivot_decode_noalloc", "pivot_last_error_detail",
     "pivot_reuse_backfill", "pivot_window_union", "pivot_index_varlen",
-    "pivot_index_varlen_workspace_size",
+    "pivot_index_varlen_workspace_size", "pivot_index_window_outside",
+    "pivot_index_window_outside_workspace_size",
 ]
 KERNELS = {0: "scan", 1: "select", 2: "refine", 3: "reduce", 4: "reuse"}
 
@@ -103,6 +104,8 @@ def load(path: str = LIB_PATH):
         "pivot_window_union": ([P, I32, I32, I32, P, I32, P, P], I32),
         "pivot_index_varlen": ([P, I32, I32, I32, I32, P, P, SZ, P], I32),
         "pivot_index_varlen_workspace_size": ([P, I32, I32, I32, I32], SZ),
+        "pivot_index_window_outside": ([P, I32, I32, I32, I32, I32, P, P, SZ, P], I32),
+        "pivot_index_window_outside_workspace_size": ([P, I32, I32, I32, I32, I32], SZ),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -282,6 +285,27 @@ def pivot_index_varlen(batch, mode, g, C, topk, idx, ws, ws_bytes, stream):
 
 def pivot_index_varlen_workspace_size(batch, mode, g, C, topk):
     return load().pivot_index_varlen_workspace_size(ctypes.byref(batch), mode, g, C, topk)
+
+
+def pivot_index_window_outside(seq, mode, g, C, topk, window, idx, ws, ws_bytes, stream):
+    return load().pivot_index_window_outside(ctypes.byref(seq), mode, g, C, topk, window, idx, ws,
+                                             ws_bytes, stream)
+
+
+def pivot_index_window_outside_workspace_size(seq, mode, g, C, topk, window):
+    return load().pivot_index_window_outside_workspace_size(ctypes.byref(seq), mode, g, C, topk,
+                                                            window)
+
+
+def index_window_outside(seq: PivotSeq, mode, g, C, topk, window, ws=None, stream=None,
+                         device="cuda"):
+    idx = torch.empty(_rows(seq), topk + window, dtype=torch.int32, device=device)
+    if ws is None:
+        ws = _workspace(pivot_index_window_outside_workspace_size(seq, mode, g, C, topk, window),
+                        device)
+    _check(pivot_index_window_outside(seq, mode, g, C, topk, window, _p(idx), _p(ws), ws.numel(),
+                                      _stream(stream)), "pivot_index_window_outside")
+    return idx
 
 
 def index_varlen(batch: PivotVarlen, mode, g, C, topk, ws=None, stream=None, device="cuda"):
