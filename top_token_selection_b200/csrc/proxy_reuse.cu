@@ -21,18 +21,6 @@ namespace {
 constexpr int RED_THREADS = 256;
 
 template <int DT>
-__device__ __forceinline__ float member_value(const void* q, const float* q_scale, size_t row,
-                                              size_t HD, size_t i) {
-    if constexpr (DT == PIVOT_F32) {
-        return static_cast<const float*>(q)[row * HD + i];
-    } else if constexpr (DT == PIVOT_BF16) {
-        return bf16_to_f32(static_cast<const uint16_t*>(q)[row * HD + i]);
-    } else {
-        return __fmul_rn(e4m3_to_f32(static_cast<const uint8_t*>(q)[row * HD + i]), q_scale[row]);
-    }
-}
-
-template <int DT>
 __global__ void __launch_bounds__(RED_THREADS) proxy_reduce_kernel(const ReduceParams p) {
     extern __shared__ float qbar_s[];          // H*D (e4m3 only)
     __shared__ float red_s[RED_THREADS / 32];
@@ -55,19 +43,58 @@ __global__ void __launch_bounds__(RED_THREADS) proxy_reduce_kernel(const ReduceP
 
     const float fn = (float)n;
     float amax = 0.0f;
-    for (size_t i = threadIdx.x; i < HD; i += RED_THREADS) {
-        float acc = member_value<DT>(p.q, p.q_scale, (size_t)m0, HD, i);
-        for (int m = 1; m < n; ++m)
-            acc = __fadd_rn(acc, member_value<DT>(p.q, p.q_scale, (size_t)(m0 + m), HD, i));
-        const float qb = __fdiv_rn(acc, fn);
+    // 16 bytes of a member row at a time (H*D*esize is a multiple of 16):
+    // the same per-element sums, in member order, as one element at a time
+    constexpr int ESZ = DT == PIVOT_F32 ? 4 : (DT == PIVOT_BF16 ? 2 : 1);
+    constexpr int VE = 16 / ESZ;
+    const size_t nchunks = HD / VE;
+    const uint8_t* qb8 = static_cast<const uint8_t*>(p.q);
+    for (size_t c = threadIdx.x; c < nchunks; c += RED_THREADS) {
+        float acc[VE];
+#pragma unroll 4
+        for (int m = 0; m < n; ++m) {
+            const size_t row = (size_t)(m0 + m);
+            const uint4 raw = *reinterpret_cast<const uint4*>(qb8 + (row * HD + c * VE) * ESZ);
+            const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+            float v[VE];
+            if constexpr (DT == PIVOT_F32) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) v[e] = __uint_as_float(wd[e]);
+            } else if constexpr (DT == PIVOT_BF16) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    v[e] = bf16_to_f32((uint16_t)(wd[e >> 1] >> ((e & 1) * 16)));
+            } else {
+                const float sc = p.q_scale[row];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    v[e] = __fmul_rn(e4m3_to_f32((uint8_t)(wd[e >> 2] >> ((e & 3) * 8))), sc);
+            }
+#pragma unroll
+            for (int e = 0; e < VE; ++e) acc[e] = m == 0 ? v[e] : __fadd_rn(acc[e], v[e]);
+        }
+        float qb[VE];
+#pragma unroll
+        for (int e = 0; e < VE; ++e) qb[e] = __fdiv_rn(acc[e], fn);
         if constexpr (DT == PIVOT_F32) {
-            static_cast<float*>(p.pq)[(size_t)j * HD + i] = qb;
+            *reinterpret_cast<float4*>(static_cast<float*>(p.pq) + (size_t)j * HD + c * VE) =
+                make_float4(qb[0], qb[1], qb[2], qb[3]);
         } else if constexpr (DT == PIVOT_BF16) {
-            const __nv_bfloat16 b = __float2bfloat16_rn(qb);
-            static_cast<__nv_bfloat16*>(p.pq)[(size_t)j * HD + i] = b;
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint16_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(qb[2 * e]));
+                const uint16_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(qb[2 * e + 1]));
+                o[e] = (uint32_t)lo | ((uint32_t)hi << 16);
+            }
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.pq) + (size_t)j * HD + c * VE) =
+                make_uint4(o[0], o[1], o[2], o[3]);
         } else {
-            qbar_s[i] = qb;
-            amax = fmaxf(amax, fabsf(qb));
+#pragma unroll
+            for (int e = 0; e < VE; ++e) {
+                qbar_s[c * VE + e] = qb[e];
+                amax = fmaxf(amax, fabsf(qb[e]));
+            }
         }
     }
     for (int h = threadIdx.x; h < p.H; h += RED_THREADS) {
@@ -83,8 +110,14 @@ __global__ void __launch_bounds__(RED_THREADS) proxy_reduce_kernel(const ReduceP
         for (int w = 0; w < RED_THREADS / 32; ++w) a = fmaxf(a, red_s[w]);
         const float s = a > 0.0f ? __fdiv_rn(a, 448.0f) : 1.0f;
         uint8_t* dst = static_cast<uint8_t*>(p.pq) + (size_t)j * HD;
-        for (size_t i = threadIdx.x; i < HD; i += RED_THREADS)
-            dst[i] = f32_to_e4m3_satfinite(__fdiv_rn(qbar_s[i], s));
+        for (size_t c = threadIdx.x; c < HD / 16; c += RED_THREADS) {
+            uint32_t o[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                o[e >> 2] |= (uint32_t)f32_to_e4m3_satfinite(__fdiv_rn(qbar_s[c * 16 + e], s))
+                             << ((e & 3) * 8);
+            *reinterpret_cast<uint4*>(dst + c * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
         if (threadIdx.x == 0) p.pq_scale[j] = s;
     }
 }
