@@ -191,9 +191,14 @@ pivot_status_t pivot_reuse_backfill(int32_t t_begin, int32_t t_end, int32_t g,
  * sequence; the batching itself is not in the pages (the PIVOT blog post
  * notes batching was left untested).  idx [total, topk] device, row t of
  * sequence i at cu_seqlens[i] + t, positions within the sequence, -1
- * padded.  1 <= topk <= C <= 8192 (C unused in dense mode).  ws of at
- * least pivot_index_varlen_workspace_size bytes, 256-byte aligned.  The
- * sequences run one after another on the stream. */
+ * padded.  1 <= topk <= C <= 8192 (C unused in dense mode).  cu_seqlens is
+ * a host array, read during the call.  ws of at least
+ * pivot_index_varlen_workspace_size bytes, 256-byte aligned.  Shapes the
+ * tensor-core kernels take (H in {4..64}, 128- or 256-byte key rows, 16-byte
+ * aligned q and k) run each step as one launch over all sequences (the
+ * sequence table is passed to the device as launch parameters, so the call
+ * can be captured in a CUDA graph); other shapes run the sequences one after
+ * another. */
 pivot_status_t pivot_index_varlen(const pivot_varlen_t* batch, int32_t mode, int32_t g, int32_t C,
                                   int32_t topk, int32_t* idx, void* ws, size_t ws_bytes,
                                   void* stream);
@@ -281,6 +286,14 @@ pivot_status_t pivot_get_device_error(void* stream);
  * current device (0 restores the default of 4 s).  Used to prove that a
  * wait that runs out returns an error instead of hanging. */
 pivot_status_t pivot_set_wait_limit_ns(uint64_t ns);
+
+/* The score buffer the *_workspace_size functions size for: at most `bytes`
+ * (0 restores the default of 4 GiB; below 4096 is refused).  Scores of more
+ * rows than fit are computed in several launches, one buffer-full at a
+ * time, with the same results.  Process-wide; it changes what later
+ * *_workspace_size calls return, so set it before sizing workspaces.  Not
+ * thread-safe against concurrent calls. */
+pivot_status_t pivot_set_score_buffer_cap(size_t bytes);
 
 /* Test hook: enqueue one kernel whose single wait is on a barrier nothing
  * arrives on.  With the wait limit lowered, a following

@@ -124,6 +124,74 @@ def test_ragged_batch_matches_each_sequence(mode):
         assert_rows_exact(got, want, f"sequence {i} (L={p.L}) mode {mode}")
 
 
+def _ragged(lens, dtype, seed):
+    """A packed batch of sequences of the given lengths (0 allowed), DSA-like
+    inputs at H = 64, D = 128, and each sequence's own device tensors."""
+    parts = {i: gen.make_prefill(n, 64, 128, dtype, kind="dsa", seed=seed + i)
+             for i, n in enumerate(lens) if n > 0}
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+
+    def cat(name):
+        xs = [getattr(parts[i], name) for i in sorted(parts)]
+        return None if xs[0] is None else torch.cat(xs).cuda().contiguous()
+
+    batch = pv.make_varlen(cu.tolist(), cat("q"), cat("q_scale"), cat("w"), cat("k"),
+                           cat("k_scale"))
+    return batch, cu, {i: to_device(p) for i, p in parts.items()}
+
+
+def _alone(dev, mode, g, C, kk):
+    seq = seq_of(dev)
+    if mode == 0:
+        return pv.dense_index(seq, kk)[0]
+    pq, pqs, pw = pv.proxy_reduce(seq, g)
+    cand = pv.proxy_scan(seq, g, pq, pqs, pw, C, kk)[0]
+    if mode == 1:
+        return pv.reuse(0, dev["q"].shape[0], g, cand, kk)
+    return pv.refine(seq, g, cand, kk)[0]
+
+
+@pytest.mark.parametrize("dtype,mode,cap", [(gen.E4M3, 0, 0), (gen.E4M3, 1, 0), (gen.E4M3, 2, 0),
+                                            (gen.E4M3, 0, 1 << 20), (gen.E4M3, 1, 1 << 20),
+                                            (gen.E4M3, 2, 1 << 20), (gen.BF16, 2, 0),
+                                            (gen.BF16, 0, 600 << 10)])
+def test_ragged_one_launch_equals_each_sequence_alone(dtype, mode, cap):
+    """The one-launch ragged batch (tensor-core shapes) against each sequence
+    run alone through the single-sequence calls: bit for bit, with empty and
+    one-token sequences, groups cut by sequence ends, and (cap set) score
+    buffers so small that launches cut row blocks."""
+    lens = [0, 1, 7, 8, 9, 300, 0, 1000, 2049, 130, 64, 3]
+    g, C, kk = 8, 512, 128
+    batch, cu, devs = _ragged(lens, dtype, seed=500)
+    if cap:
+        assert pv.pivot_set_score_buffer_cap(cap) == 0
+    try:
+        idx = pv.index_varlen(batch, mode, g, C, kk)
+        torch.cuda.synchronize()
+        assert pv.device_error() == 0
+        got = idx.cpu().numpy()
+        for i, dev in devs.items():
+            want = _alone(dev, mode, g, C, kk).cpu().numpy()
+            assert_rows_exact(got[cu[i]:cu[i + 1]], want, f"sequence {i} (L={lens[i]}) mode {mode}")
+    finally:
+        pv.pivot_set_score_buffer_cap(0)
+
+
+def test_ragged_one_launch_launch_count():
+    """Many short sequences take a fixed number of launches, not a few per
+    sequence."""
+    lens = [64] * 48
+    batch, _, _ = _ragged(lens, gen.E4M3, seed=900)
+    ws = torch.empty(pv.pivot_index_varlen_workspace_size(batch, 2, 8, 256, 64),
+                     dtype=torch.uint8, device="cuda")
+    pv.index_varlen(batch, 2, 8, 256, 64, ws=ws)
+    torch.cuda.synchronize()
+    n0 = pv.pivot_launch_count()
+    pv.index_varlen(batch, 2, 8, 256, 64, ws=ws)
+    torch.cuda.synchronize()
+    assert pv.pivot_launch_count() - n0 <= 12
+
+
 @pytest.mark.parametrize("mode,window", [(0, 1), (0, 5), (0, 64), (1, 5), (2, 5), (2, 64)])
 def test_window_outside_exact(tiny, mode, window):
     """The window kept out of the candidates, then added: bit for bit."""

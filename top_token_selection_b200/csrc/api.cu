@@ -1,7 +1,9 @@
 // api.cu -- the libpivot C ABI: argument checks, workspace carving, TMA
 // descriptors and kernel launches.  See include/pivot.h for the contract.
+#include <climits>
 #include <cstdio>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -15,7 +17,8 @@ __device__ uint64_t g_wait_limit_ns = 4000000000ull;
 namespace {
 
 constexpr size_t WS_ALIGN = 256;
-constexpr size_t SCORE_BUF_CAP = size_t(4) << 30;   // preferred score buffer, 4 GiB
+constexpr size_t SCORE_BUF_DEFAULT = size_t(4) << 30;   // preferred score buffer, 4 GiB
+size_t g_score_buf_cap = SCORE_BUF_DEFAULT;             // pivot_set_score_buffer_cap
 constexpr int MAX_K = 8192;   // the select's exact path holds 2 pow2(K) keys in shared memory
 constexpr int TAIL_CAP = 4096;
 constexpr int MAX_SMS = 1024;
@@ -236,8 +239,10 @@ pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, in
                                  const int32_t* cache_len, const float* S, long long stride,
                                  int K, int split, int npos, int32_t* out, float* out_score,
                                  int out_base, cudaStream_t st, uint32_t* thresh = nullptr,
-                                 int lim_shift = 0, int out_stride = 0) {
+                                 int lim_shift = 0, int out_stride = 0,
+                                 const SegTable* seg = nullptr, double work = -1.0) {
     SelectParams sp{};
+    if (seg) sp.seg = *seg;
     sp.lim_shift = lim_shift;
     sp.out_stride = out_stride;
     sp.split = split;
@@ -264,8 +269,8 @@ pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, in
             profiled(PK_SELECT, 0.0, st, [&] { return launch_row_threshold(sp, thresh, st); }));
         if (t != PIVOT_OK) return t;
     }
-    return from_cuda(profiled(PK_SELECT, scan_pairs(scan_kind, r0, r1, L, g), st,
-                              [&] { return launch_select(sp, st); }));
+    return from_cuda(profiled(PK_SELECT, work >= 0.0 ? work : scan_pairs(scan_kind, r0, r1, L, g),
+                              st, [&] { return launch_select(sp, st); }));
 }
 
 // Refine rows: S holds the scores without the key scale, which the
@@ -274,8 +279,10 @@ pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int 
                                const int32_t* cache_len, const float* S, const int32_t* cand,
                                int cand_base, int C, int K, int npos, int32_t* out,
                                float* out_score, int out_base, cudaStream_t st,
-                               const float* key_scale, int lim_shift = 0, int out_stride = 0) {
+                               const float* key_scale, int lim_shift = 0, int out_stride = 0,
+                               const SegTable* seg = nullptr) {
     SelectParams sp{};
+    if (seg) sp.seg = *seg;
     sp.npos = npos;
     sp.kind = SEL_CANDIDATES;
     sp.scan_kind = scan_kind;
@@ -457,6 +464,12 @@ pivot_status_t pivot_set_wait_limit_ns(uint64_t ns) {
                                                                             : PIVOT_ERR_CUDA;
 }
 
+pivot_status_t pivot_set_score_buffer_cap(size_t bytes) {
+    if (bytes != 0 && bytes < 4096) return PIVOT_ERR_INVALID_ARG;
+    g_score_buf_cap = bytes ? bytes : SCORE_BUF_DEFAULT;
+    return PIVOT_OK;
+}
+
 pivot_status_t pivot_selftest_wait_timeout(void* stream) {
     return launch_wait_selftest(static_cast<cudaStream_t>(stream)) == cudaSuccess ? PIVOT_OK
                                                                                   : PIVOT_ERR_CUDA;
@@ -469,7 +482,7 @@ size_t pivot_dense_index_workspace_size(const pivot_seq_t* seq, int32_t topk) {
     const int P = rows_per_block(seq->H, seq->D, seq->dtype);
     const size_t rb = dense_rowbytes(seq->L);
     long long rows = t1 - t0;
-    long long cap = (long long)(SCORE_BUF_CAP / rb) / P * P;
+    long long cap = (long long)(g_score_buf_cap / rb) / P * P;
     if (cap < 1) cap = 1;
     if (rows > cap) rows = cap;
     return align_up((size_t)rows * rb, WS_ALIGN);
@@ -548,7 +561,7 @@ size_t pivot_proxy_scan_workspace_size(const pivot_seq_t* seq, int32_t g, int32_
     const int P = rows_per_block(seq->H, seq->D, seq->dtype);
     const size_t rb = dense_rowbytes(seq->L);
     long long rows = ceil_div(t1 - t0, g);
-    long long cap = (long long)(SCORE_BUF_CAP / rb) / P * P;
+    long long cap = (long long)(g_score_buf_cap / rb) / P * P;
     if (cap < 1) cap = 1;
     if (rows > cap) rows = cap;
     return align_up((size_t)rows * rb, WS_ALIGN);
@@ -653,7 +666,7 @@ size_t pivot_refine_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C,
     if (check_seq(seq, &t0, &t1) != PIVOT_OK || g < 1 || C < 1 || topk < 1) return 0;
     long long rows = t1 - t0;
     const size_t rb = (size_t)C * 4;
-    long long cap = (long long)(SCORE_BUF_CAP / rb) / g * g;
+    long long cap = (long long)(g_score_buf_cap / rb) / g * g;
     if (cap < 1) cap = 1;
     if (rows > cap) rows = cap;
     return align_up((size_t)rows * rb, WS_ALIGN);
@@ -726,8 +739,8 @@ pivot_status_t check_varlen(const pivot_varlen_t* b, int mode, int g, int C, int
     return PIVOT_OK;
 }
 
-// Workspace: proxies and candidates of the longest sequence, then the inner
-// workspace the single-sequence calls need.
+// Workspace of the sequence-by-sequence path: proxies and candidates of the
+// longest sequence, then the inner workspace the single-sequence calls need.
 struct VarlenWs {
     size_t pq, pqs, pw, cand, inner, total;
 };
@@ -765,11 +778,341 @@ VarlenWs varlen_layout(const pivot_varlen_t* b, int mode, int g, int C, int topk
     return w;
 }
 
+// ---- one launch per stage over all sequences (tensor-core shapes)
+constexpr int VAR_TPI = 32;   // key tiles per scan work item, as in the single-sequence prefill
+
+// Host copies of the segment prefixes (segments.h): tokens, groups and the
+// scan work items of the dense (query rows) and proxy (group rows) scans.
+struct VarTabs {
+    int B = 0, T = 0, maxL = 0, G = 0;
+    std::vector<int32_t> tok, grp, itmD, itmP;
+};
+
+bool varlen_tabs(const pivot_varlen_t* b, int g, int P, VarTabs& t) {
+    const int B = b->nseq;
+    const int gg = g > 0 ? g : 1;
+    t.B = B;
+    t.tok.assign(b->cu_seqlens, b->cu_seqlens + B + 1);
+    t.grp.assign(B + 1, 0);
+    t.itmD.assign(B + 1, 0);
+    t.itmP.assign(B + 1, 0);
+    long long G = 0, ID = 0, IP = 0;
+    for (int i = 0; i < B; ++i) {
+        const int len = t.tok[i + 1] - t.tok[i];
+        if (len > t.maxL) t.maxL = len;
+        const int ng = ceil_div(len, gg);
+        const long long ch = seg_chunks(len, VAR_TPI);
+        G += ng;
+        ID += (long long)ceil_div(len, P) * ch;
+        IP += (long long)ceil_div(ng, P) * ch;
+        if (G > INT32_MAX || ID > INT32_MAX || IP > INT32_MAX) return false;
+        t.grp[i + 1] = (int32_t)G;
+        t.itmD[i + 1] = (int32_t)ID;
+        t.itmP[i + 1] = (int32_t)IP;
+    }
+    t.T = t.tok[B];
+    t.G = (int)G;
+    return true;
+}
+
+// Rows of the Refine tensor-core block for groups of g members.
+int refine_rows(int H, int g) {
+    const int P = umma_rows(H);
+    return P < g ? P : g;
+}
+
+// Whether the batch runs as one launch per stage: the tensor-core scan
+// shapes (and, for Refine, a member block the tensor cores take).
+bool varlen_single_ok(const pivot_varlen_t* b, int mode, int g) {
+    // inputs the single-sequence checks would refuse take that path and its errors
+    if (!dtype_ok(b->dtype) || !b->q || !b->w || !b->k) return false;
+    const bool fp8 = b->dtype == PIVOT_E4M3;
+    if (fp8 != (b->q_scale != nullptr) || fp8 != (b->k_scale != nullptr)) return false;
+    if (!umma_shape_ok(b->H, b->D, b->dtype)) return false;
+    if (!aligned16(b->q) || !aligned16(b->k)) return false;
+    if (mode == PIVOT_MODE_REFINE) {
+        const int N = refine_rows(b->H, g) * b->H;
+        if (N < 16 || N > 256 || N % 16) return false;
+    }
+    VarTabs t;
+    return varlen_tabs(b, g, umma_rows(b->H), t);
+}
+
+struct VarlenWs1 {
+    size_t tabs, pq, pqs, pw, cand, S, S_bytes, total;
+};
+
+VarlenWs1 varlen_layout1(const pivot_varlen_t* b, const VarTabs& t, int mode, int g, int C) {
+    VarlenWs1 w{};
+    size_t off = 0;
+    w.tabs = off;
+    off = align_up(off + (size_t)4 * (t.B + 1) * 4, WS_ALIGN);
+    const size_t G = mode != PIVOT_MODE_DENSE ? (size_t)t.G : 0;
+    if (G > 0) {
+        w.pq = off;
+        off = align_up(off + G * b->H * b->D * esize_of(b->dtype), WS_ALIGN);
+        w.pqs = off;
+        off = align_up(off + G * 4, WS_ALIGN);
+        w.pw = off;
+        off = align_up(off + G * b->H * 4, WS_ALIGN);
+        w.cand = off;
+        off = align_up(off + G * C * 4, WS_ALIGN);
+    }
+    const int P = umma_rows(b->H);
+    const size_t rb = dense_rowbytes(t.maxL);
+    long long cap = (long long)(g_score_buf_cap / rb) / P * P;
+    if (cap < P) cap = P;
+    const long long scan_rows = mode == PIVOT_MODE_DENSE ? t.T : t.G;
+    size_t sb = (size_t)(scan_rows < cap ? scan_rows : cap) * rb;
+    if (mode == PIVOT_MODE_REFINE) {
+        long long capr = (long long)(g_score_buf_cap / ((size_t)C * 4)) / g * g;
+        if (capr < g) capr = g;
+        const size_t rbytes = (size_t)(t.T < capr ? t.T : capr) * C * 4;
+        if (rbytes > sb) sb = rbytes;
+    }
+    w.S = off;
+    w.S_bytes = align_up(sb, WS_ALIGN);
+    w.total = align_up(off + w.S_bytes, WS_ALIGN);
+    return w;
+}
+
+// Causal (row, key) pairs of packed dense rows [r0, r1) and of packed proxy
+// rows [j0, j1); (member, candidate) pairs of Refine rows [r0, r1).
+double varlen_dense_pairs(const VarTabs& t, int r0, int r1) {
+    double s = 0.0;
+    for (int b = seg_find(t.tok.data(), t.B, r0); b < t.B && t.tok[b] < r1; ++b) {
+        const double a = (r0 > t.tok[b] ? r0 : t.tok[b]) - t.tok[b];
+        const double z = (r1 < t.tok[b + 1] ? r1 : t.tok[b + 1]) - t.tok[b];
+        if (z > a) s += 0.5 * (z * (z + 1) - a * (a + 1));
+    }
+    return s;
+}
+
+double varlen_proxy_pairs(const VarTabs& t, int g, int j0, int j1) {
+    double s = 0.0;
+    for (int b = seg_find(t.grp.data(), t.B, j0); b < t.B && t.grp[b] < j1; ++b) {
+        const int len = t.tok[b + 1] - t.tok[b];
+        const int ng = t.grp[b + 1] - t.grp[b];
+        const double a = (j0 > t.grp[b] ? j0 : t.grp[b]) - t.grp[b];
+        const double z = (j1 < t.grp[b + 1] ? j1 : t.grp[b + 1]) - t.grp[b];
+        if (z <= a) continue;
+        // groups x < ng - 1 end at (x + 1) g; the last one at len
+        s += (double)g * 0.5 * (z * (z + 1) - a * (a + 1));
+        if (z == ng) s += (double)len - (double)ng * g;
+    }
+    return s;
+}
+
+double varlen_refine_pairs(const VarTabs& t, int C, int r0, int r1) {
+    double s = 0.0;
+    for (int b = seg_find(t.tok.data(), t.B, r0); b < t.B && t.tok[b] < r1; ++b) {
+        const int a = (r0 > t.tok[b] ? r0 : t.tok[b]) - t.tok[b];
+        const int z = (r1 < t.tok[b + 1] ? r1 : t.tok[b + 1]) - t.tok[b];
+        if (z > a) s += refine_pairs(a, z, C);
+    }
+    return s;
+}
+
+// The scan of packed rows [r0, r1) (kind SCAN_VARLEN_DENSE: tokens of q;
+// SCAN_VARLEN_PROXY: groups of pq) against each row's sequence's keys.
+pivot_status_t run_scan_varlen(int kind, const pivot_varlen_t* b, int T, const void* qbase,
+                               long long q_rows, const float* w, const float* q_scale, int g,
+                               int P, const SegTable& seg, int nitems, int r0, int r1, float* S,
+                               long long stride, double work, cudaStream_t st) {
+    ScanParams p{};
+    p.kind = kind;
+    p.dtype = b->dtype;
+    p.esize = esize_of(b->dtype);
+    p.H = b->H;
+    p.D = b->D;
+    p.P = P;
+    p.row0 = r0;
+    p.nrows = r1 - r0;
+    p.qrow_base = 0;
+    p.g = g;
+    p.Gm = 1;
+    p.w = w;
+    p.q_scale = q_scale;
+    p.k_scale = b->k_scale;
+    p.S = S;
+    p.S_stride = stride;
+    p.tiles_per_item = seg.tpi;
+    p.items_per_block = 0;
+    p.nitems = nitems;
+    p.seg = seg;
+    CUtensorMap tk, tq;
+    if (!make_tmap(&tk, b->dtype, b->k, T, b->D, 128)) return PIVOT_ERR_CUDA;
+    if (!make_tmap(&tq, b->dtype, qbase, q_rows * b->H, b->D, P * b->H)) return PIVOT_ERR_CUDA;
+    const int grid = nitems < num_sms() ? nitems : num_sms();
+    return from_cuda(
+        profiled(PK_SCAN, work, st, [&] { return launch_scan_umma(tk, tq, p, grid, st); }));
+}
+
+pivot_status_t varlen_single(const pivot_varlen_t* b, int mode, int g, int C, int topk,
+                             int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t st) {
+    const int P = umma_rows(b->H);
+    VarTabs t;
+    if (!varlen_tabs(b, g, P, t)) return PIVOT_ERR_UNSUPPORTED;
+    const VarlenWs1 lay = varlen_layout1(b, t, mode, g, C);
+    if (ws_bytes < lay.total) return PIVOT_ERR_WORKSPACE;
+    if (t.T == 0) return PIVOT_OK;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    // the segment tables, carried to the device as launch parameters
+    int32_t* d_tab = reinterpret_cast<int32_t*>(base + lay.tabs);
+    const int n1 = t.B + 1;
+    const std::vector<int32_t>* tabs[4] = {&t.tok, &t.grp, &t.itmD, &t.itmP};
+    for (int a = 0; a < 4; ++a)
+        for (int i = 0; i < n1; i += 960) {
+            const int n = n1 - i < 960 ? n1 - i : 960;
+            cudaError_t e = launch_write_ints(d_tab + (size_t)a * n1 + i, tabs[a]->data() + i, n, st);
+            if (e != cudaSuccess) return from_cuda(e);
+            count_launch();
+        }
+    SegTable seg{};
+    seg.tok = d_tab;
+    seg.grp = d_tab + n1;
+    seg.nseq = t.B;
+    seg.tpi = VAR_TPI;
+    const int32_t* d_itmD = d_tab + 2 * n1;
+    const int32_t* d_itmP = d_tab + 3 * n1;
+    float* S = reinterpret_cast<float*>(base + lay.S);
+    const long long stride = score_stride(t.maxL);
+    const long long cap_scan = (long long)(lay.S_bytes / dense_rowbytes(t.maxL));
+    pivot_status_t res;
+
+    // the scan + selection of packed rows [r0, r1) in launches of at most
+    // cap_scan rows (a launch may cut a row block: rows outside it are dropped)
+    auto scan_select = [&](int kind, const std::vector<int32_t>& rowpre, const int32_t* d_itm,
+                           const std::vector<int32_t>& itm, int nrows_total, const void* qb,
+                           const float* w, const float* qs, int gg, int K, int split,
+                           int32_t* out) -> pivot_status_t {
+        for (long long c0 = 0; c0 < nrows_total; c0 += cap_scan) {
+            const int r0 = (int)c0;
+            const int r1 = (int)(c0 + cap_scan < nrows_total ? c0 + cap_scan : nrows_total);
+            int i0, n0, i1, n1b;
+            seg_block_items(t.tok.data(), rowpre.data(), itm.data(), t.B, P, VAR_TPI, r0, &i0, &n0);
+            seg_block_items(t.tok.data(), rowpre.data(), itm.data(), t.B, P, VAR_TPI, r1 - 1, &i1,
+                            &n1b);
+            SegTable sg = seg;
+            sg.itm = d_itm;
+            sg.item0 = i0;
+            const int nitems = i1 + n1b - i0;
+            const double work = kind == SCAN_VARLEN_DENSE ? varlen_dense_pairs(t, r0, r1)
+                                                          : varlen_proxy_pairs(t, gg, r0, r1);
+            uint32_t* thresh = reinterpret_cast<uint32_t*>(S + (size_t)(r1 - r0) * stride);
+            pivot_status_t r = run_scan_varlen(kind, b, t.T, qb, nrows_total, w, qs, gg, P, sg,
+                                               nitems, r0, r1, S, stride, work, st);
+            if (r != PIVOT_OK) return r;
+            r = run_select_prefix(kind, r0, r1, t.maxL, gg, 1, 0, nullptr, S, stride, K, split,
+                                  t.maxL, out, nullptr, 0, st, thresh, 0, 0, &sg, work);
+            if (r != PIVOT_OK) return r;
+        }
+        return PIVOT_OK;
+    };
+
+    if (mode == PIVOT_MODE_DENSE)
+        return scan_select(SCAN_VARLEN_DENSE, t.tok, d_itmD, t.itmD, t.T, b->q, b->w, b->q_scale,
+                           1, topk, 0, idx);
+
+    // proxies of every group of the batch
+    void* pq = base + lay.pq;
+    float* pqs = b->dtype == PIVOT_E4M3 ? reinterpret_cast<float*>(base + lay.pqs) : nullptr;
+    float* pw = reinterpret_cast<float*>(base + lay.pw);
+    int32_t* cand = reinterpret_cast<int32_t*>(base + lay.cand);
+    {
+        ReduceParams rp{};
+        rp.dtype = b->dtype;
+        rp.esize = esize_of(b->dtype);
+        rp.H = b->H;
+        rp.D = b->D;
+        rp.nmembers_total = t.T;
+        rp.g = g;
+        rp.ngroups = t.G;
+        rp.q = b->q;
+        rp.q_scale = b->q_scale;
+        rp.w = b->w;
+        rp.pq = pq;
+        rp.pq_scale = pqs;
+        rp.pw = pw;
+        rp.group_stride_members = g;
+        rp.seg = seg;
+        const double bytes = ((double)t.T + t.G) * b->H * (b->D * rp.esize + 4.0);
+        res = from_cuda(profiled(PK_REDUCE, bytes, st, [&] { return launch_proxy_reduce(rp, st); }));
+        if (res != PIVOT_OK) return res;
+    }
+    // one full-prefix scan per group, top-C with its top-k first
+    res = scan_select(SCAN_VARLEN_PROXY, t.grp, d_itmP, t.itmP, t.G, pq, pw, pqs, g, C, topk, cand);
+    if (res != PIVOT_OK) return res;
+
+    if (mode == PIVOT_MODE_REUSE) {
+        const double bytes = 4.0 * topk * ((double)t.T + t.G);
+        return from_cuda(profiled(PK_REUSE, bytes, st, [&] {
+            return launch_reuse_varlen(seg, t.T, g, cand, C, topk, idx, st);
+        }));
+    }
+
+    // Refine: members re-score their group's candidates, in launches of at
+    // most cap_ref member rows
+    const int Pr = refine_rows(b->H, g);
+    const int N = Pr * b->H;
+    CUtensorMap tq;
+    if (!make_tmap(&tq, b->dtype, b->q, (long long)t.T * b->H, b->D, N)) return PIVOT_ERR_CUDA;
+    const long long cap_ref = (long long)(lay.S_bytes / ((size_t)C * 4));
+    for (long long c0 = 0; c0 < t.T; c0 += cap_ref) {
+        const int r0 = (int)c0;
+        const int r1 = (int)(c0 + cap_ref < t.T ? c0 + cap_ref : t.T);
+        const int jA = seg_group_of(SegTable{t.tok.data(), t.grp.data(), nullptr, t.B, 0, 0}, g, r0);
+        const int jB = seg_group_of(SegTable{t.tok.data(), t.grp.data(), nullptr, t.B, 0, 0}, g,
+                                    r1 - 1) + 1;
+        ScanParams p{};
+        p.kind = SCAN_VARLEN_DENSE;
+        p.dtype = b->dtype;
+        p.esize = esize_of(b->dtype);
+        p.H = b->H;
+        p.D = b->D;
+        p.P = Pr;
+        p.row0 = r0;
+        p.nrows = r1 - r0;
+        p.qrow_base = 0;
+        p.g = g;
+        p.Gm = 1;
+        p.w = b->w;
+        p.q_scale = b->q_scale;
+        p.k_scale = b->k_scale;
+        p.S = S;
+        p.S_stride = C;
+        p.cand = cand + (size_t)jA * C;
+        p.cand_base = jA;
+        p.C = C;
+        p.gsize = g;
+        p.tiles_per_item = ceil_div(C, 128);
+        p.items_per_block = ceil_div(g, Pr);
+        p.nitems = (jB - jA) * p.items_per_block;
+        p.kbase = b->k;
+        p.seg = seg;
+        const double work = varlen_refine_pairs(t, C, r0, r1);
+        const int grid = p.nitems < num_sms() ? p.nitems : num_sms();
+        res = from_cuda(
+            profiled(PK_REFINE, work, st, [&] { return launch_refine_umma(tq, p, grid, st); }));
+        if (res != PIVOT_OK) return res;
+        res = run_select_cand(SCAN_VARLEN_DENSE, r0, r1, t.maxL, g, 1, 0, nullptr, S,
+                              cand + (size_t)jA * C, jA, C, topk, t.maxL, idx, nullptr, 0, st,
+                              b->k_scale, 0, 0, &seg);
+        if (res != PIVOT_OK) return res;
+    }
+    return PIVOT_OK;
+}
+
 }  // namespace
 
 size_t pivot_index_varlen_workspace_size(const pivot_varlen_t* batch, int32_t mode, int32_t g,
                                          int32_t C, int32_t topk) {
     if (check_varlen(batch, mode, g, C, topk) != PIVOT_OK) return 0;
+    if (varlen_single_ok(batch, mode, g)) {
+        VarTabs t;
+        varlen_tabs(batch, g, umma_rows(batch->H), t);
+        return varlen_layout1(batch, t, mode, g, C).total;
+    }
     return varlen_layout(batch, mode, g, C, topk).total;
 }
 
@@ -779,6 +1122,9 @@ pivot_status_t pivot_index_varlen(const pivot_varlen_t* batch, int32_t mode, int
     pivot_status_t st = check_varlen(batch, mode, g, C, topk);
     if (st != PIVOT_OK) return st;
     if (!idx || !ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
+    if (varlen_single_ok(batch, mode, g))
+        return varlen_single(batch, mode, g, C, topk, idx, ws, ws_bytes,
+                             static_cast<cudaStream_t>(stream));
     const VarlenWs lay = varlen_layout(batch, mode, g, C, topk);
     if (ws_bytes < lay.total) return PIVOT_ERR_WORKSPACE;
     uint8_t* base = static_cast<uint8_t*>(ws);

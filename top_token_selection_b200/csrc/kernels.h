@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "segments.h"
+
 namespace pivot {
 
 // Which rows a scan launch scores and how their causal limit is found.
@@ -14,6 +16,8 @@ enum ScanKind {
     SCAN_PREFILL_PROXY = 1,   // row r = group j, keys [0, min(L,(j+1)g) - 1]
     SCAN_DECODE_DENSE = 2,    // row r = b*Gm + m, keys [0, cache_len[b] - Gm + m] of seq b
     SCAN_DECODE_PROXY = 3,    // row r = b, keys [0, cache_len[b] - 1] of seq b
+    SCAN_VARLEN_DENSE = 4,    // packed token r of sequence b: keys [0, r - tok[b]] of b
+    SCAN_VARLEN_PROXY = 5,    // packed group r of sequence b: keys of b up to its last member
 };
 
 struct ScanParams {
@@ -39,6 +43,7 @@ struct ScanParams {
     int gsize;              // members per group (g in prefill, Gm in decode)
     int nkeys;              // key positions per sequence (L, or maxlen in decode)
     const void* kbase;      // gather mode: key rows (stored format), row stride D*esize
+    SegTable seg;           // SCAN_VARLEN_*: the batch's sequences (rows, keys packed)
 };
 
 int scan_smem_bytes(int row_bytes);
@@ -81,6 +86,9 @@ struct SelectParams {
                               // (kb = grp * maxlen for decode rows, else 0)
     const uint32_t* thresh;   // SEL_PREFIX: row r's lower bound at thresh[r - row0]
                               // (launch_row_threshold), or NULL: sampled in the select
+    SegTable seg;             // scan_kind SCAN_VARLEN_*: the batch's sequences; candidate
+                              // rows of packed token r: group seg_group_of(r), key scales
+                              // from the sequence's first token
 };
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
@@ -101,6 +109,7 @@ struct ReduceParams {
     float* pq_scale;
     float* pw;
     long long group_stride_members;  // members between consecutive groups
+    SegTable seg;          // seg.tok set: packed groups of a ragged batch (seg_group)
 };
 cudaError_t launch_proxy_reduce(const ReduceParams& p, cudaStream_t stream);
 
@@ -114,6 +123,13 @@ cudaError_t launch_reuse(int t_begin, int t_end, int g, const int32_t* cand, int
 cudaError_t launch_window_union(const int32_t* idx, int rows, int k, int t_begin,
                                 const int32_t* positions, int window, int32_t* out,
                                 cudaStream_t stream, int in_stride = 0);
+// Reuse over a ragged batch: packed token t takes the first topk entries of
+// its group's candidate row (seg_group_of) that are <= its position.
+cudaError_t launch_reuse_varlen(const SegTable& seg, int T, int g, const int32_t* cand, int C,
+                                int topk, int32_t* idx, cudaStream_t stream);
+// Copy n (<= 960) host integers, carried as launch parameters, to dst: a
+// host-to-device copy that stream capture records like any launch.
+cudaError_t launch_write_ints(int32_t* dst, const int32_t* host, int n, cudaStream_t stream);
 cudaError_t launch_decode_reuse(int B, int Gm, int maxlen, const int32_t* cache_len,
                                 const int32_t* cand, int C, int topk, int32_t* idx,
                                 cudaStream_t stream);

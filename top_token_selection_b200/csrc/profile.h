@@ -10,6 +10,8 @@ enum ProfKernel { PK_SCAN = 0, PK_SELECT = 1, PK_REFINE = 2, PK_REDUCE = 3, PK_R
 
 bool prof_begin(int kernel, cudaStream_t s, cudaEvent_t* a, cudaEvent_t* b);
 void prof_end(int kernel, cudaStream_t s, cudaEvent_t a, cudaEvent_t b, double work);
+// Count a launch that is not timed (pivot_launch_count).
+void count_launch();
 
 // Run `launch` (returning cudaError_t), counted and, when timing is on,
 // bracketed by events on stream `s` with `work` units attributed to it.

@@ -26,8 +26,16 @@ __global__ void __launch_bounds__(RED_THREADS) proxy_reduce_kernel(const ReduceP
     __shared__ float red_s[RED_THREADS / 32];
     const int j = blockIdx.x;
     const size_t HD = (size_t)p.H * p.D;
-    const long long m0 = (long long)j * p.group_stride_members;
-    const int n = (int)min((long long)p.g, (long long)p.nmembers_total - m0);
+    long long m0;
+    int n;
+    if (p.seg.tok) {   // packed group j of a ragged batch
+        const SegGroup sg = seg_group(p.seg, p.g, j);
+        m0 = sg.first;
+        n = sg.n;
+    } else {
+        m0 = (long long)j * p.group_stride_members;
+        n = (int)min((long long)p.g, (long long)p.nmembers_total - m0);
+    }
     if (n <= 0) return;
 
     if (n == 1) {   // a group of one is its member
@@ -145,6 +153,24 @@ __global__ void reuse_kernel(int t_begin, int t_end, int g, const int32_t* cand,
     reuse_row(cand + (size_t)j * C, topk, t - lim_shift, idx + (size_t)(t - t_begin) * out_stride);
 }
 
+__global__ void reuse_varlen_kernel(const SegTable seg, int T, int g, const int32_t* cand, int C,
+                                    int topk, int32_t* idx) {
+    const int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int b = seg_find(seg.tok, seg.nseq, t);
+    const int j = seg.grp[b] + (t - seg.tok[b]) / g;
+    reuse_row(cand + (size_t)j * C, topk, t - seg.tok[b], idx + (size_t)t * topk);
+}
+
+constexpr int WRITE_INTS_MAX = 960;
+struct IntBlock {
+    int32_t v[WRITE_INTS_MAX];
+};
+
+__global__ void write_ints_kernel(int32_t* dst, const IntBlock blk, int n) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = blk.v[i];
+}
+
 __global__ void decode_reuse_kernel(int B, int Gm, int maxlen, const int32_t* cache_len,
                                     const int32_t* cand, int C, int topk, int32_t* idx) {
     const int r = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
@@ -229,6 +255,23 @@ cudaError_t launch_reuse(int t_begin, int t_end, int g, const int32_t* cand, int
     const int wpb = 8;
     reuse_kernel<<<ceil_div(rows, wpb), wpb * 32, 0, stream>>>(
         t_begin, t_end, g, cand, C, topk, idx, lim_shift, out_stride ? out_stride : topk);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reuse_varlen(const SegTable& seg, int T, int g, const int32_t* cand, int C,
+                                int topk, int32_t* idx, cudaStream_t stream) {
+    if (T <= 0) return cudaSuccess;
+    const int wpb = 8;
+    reuse_varlen_kernel<<<ceil_div(T, wpb), wpb * 32, 0, stream>>>(seg, T, g, cand, C, topk, idx);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_write_ints(int32_t* dst, const int32_t* host, int n, cudaStream_t stream) {
+    if (n < 0 || n > WRITE_INTS_MAX) return cudaErrorInvalidValue;
+    if (n == 0) return cudaSuccess;
+    IntBlock blk;
+    for (int i = 0; i < n; ++i) blk.v[i] = host[i];
+    write_ints_kernel<<<1, 256, 0, stream>>>(dst, blk, n);
     return cudaGetLastError();
 }
 

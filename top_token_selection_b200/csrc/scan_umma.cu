@@ -55,6 +55,10 @@ __device__ __forceinline__ int scan_row_lim(const ScanParams& p, int r, bool& ok
             if (n < p.Gm || n > p.maxlen) { ok = false; return -1; }
             return n - p.Gm + m;
         }
+        case SCAN_VARLEN_DENSE:
+            return seg_dense_lim(p.seg, r);
+        case SCAN_VARLEN_PROXY:
+            return seg_proxy_lim(p.seg, p.g, r);
         default: {  // SCAN_DECODE_PROXY
             int n = p.cache_len[r];
             if (n < 1 || n > p.maxlen) { ok = false; return -1; }
@@ -71,6 +75,7 @@ __device__ __forceinline__ int scan_key_base(const ScanParams& p, int r) {
 
 struct ItemInfo {
     int rows, row_first, t0, t1, keybase, maxlim;
+    int nkeys;             // gather mode: key rows of the item's sequence
     const int32_t* cand;   // gather mode: this group's candidate row
     bool valid;
 };
@@ -83,15 +88,36 @@ template <bool GATHER>
 __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
     ItemInfo it;
     if constexpr (!GATHER) {
-        const int blk = item / p.items_per_block;
-        const int chunk = item % p.items_per_block;
-        it.row_first = p.row0 + blk * p.P;
-        const int rows = p.row0 + p.nrows - it.row_first;
-        it.rows = rows < p.P ? rows : p.P;
+        int chunk;
+        if (p.kind == SCAN_VARLEN_DENSE || p.kind == SCAN_VARLEN_PROXY) {
+            // blocks never straddle two sequences: each is one sequence's;
+            // rows outside the launch's [row0, row0 + nrows) are dropped
+            const SegItem si = seg_scan_item(
+                p.seg, p.kind == SCAN_VARLEN_DENSE ? p.seg.tok : p.seg.grp, p.P, p.row0, p.nrows, item);
+            chunk = si.chunk;
+            it.row_first = si.first;
+            it.rows = si.rows;
+            it.keybase = p.seg.tok[si.b];
+            if (it.rows <= 0) {
+                it.valid = false;
+                it.t0 = it.t1 = 0;
+                it.maxlim = -1;
+                it.nkeys = 0;
+                it.cand = nullptr;
+                return it;
+            }
+        } else {
+            const int blk = item / p.items_per_block;
+            chunk = item % p.items_per_block;
+            it.row_first = p.row0 + blk * p.P;
+            const int rows = p.row0 + p.nrows - it.row_first;
+            it.rows = rows < p.P ? rows : p.P;
+            it.keybase = scan_key_base(p, it.row_first);
+        }
         bool ok;
         const int maxlim = scan_row_lim(p, it.row_first + it.rows - 1, ok);
         it.maxlim = ok ? maxlim : -1;
-        it.keybase = scan_key_base(p, it.row_first);
+        it.nkeys = 0;
         const int nt = ok ? (maxlim + 1 + 127) / 128 : 0;
         it.t0 = chunk * p.tiles_per_item;
         it.t1 = it.t0 + p.tiles_per_item < nt ? it.t0 + p.tiles_per_item : nt;
@@ -100,16 +126,25 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
     } else {
         const int grp = p.cand_base + item / p.items_per_block;
         const int mb = item % p.items_per_block;
-        const int gstart = grp * p.gsize;
-        int first = gstart + mb * p.P;
-        int end = first + p.P;
-        if (end > gstart + p.gsize) end = gstart + p.gsize;
-        if (first < p.row0) first = p.row0;
-        if (end > p.row0 + p.nrows) end = p.row0 + p.nrows;
-        it.row_first = first;
-        it.rows = end - first;
-        it.keybase = p.kind == SCAN_DECODE_DENSE ? grp * p.maxlen : 0;
-        it.maxlim = p.nkeys - 1;
+        if (p.kind == SCAN_VARLEN_DENSE) {   // packed group of a ragged batch
+            const SegItem si = seg_refine_item(p.seg, p.gsize, p.P, grp, mb, p.row0, p.nrows);
+            it.row_first = si.first;
+            it.rows = si.rows;
+            it.keybase = p.seg.tok[si.b];
+            it.nkeys = p.seg.tok[si.b + 1] - p.seg.tok[si.b];
+        } else {
+            const int gstart = grp * p.gsize;
+            int first = gstart + mb * p.P;
+            int end = first + p.P;
+            if (end > gstart + p.gsize) end = gstart + p.gsize;
+            if (first < p.row0) first = p.row0;
+            if (end > p.row0 + p.nrows) end = p.row0 + p.nrows;
+            it.row_first = first;
+            it.rows = end - first;
+            it.keybase = p.kind == SCAN_DECODE_DENSE ? grp * p.maxlen : 0;
+            it.nkeys = p.nkeys;
+        }
+        it.maxlim = it.nkeys - 1;
         it.t0 = 0;
         it.t1 = (p.C + 127) / 128;
         it.valid = it.rows > 0;
@@ -304,7 +339,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                     for (int j = 0; j < 4; ++j) {
                         const int r = j * 32 + lane;
                         const int pos = cur[j];
-                        const size_t row = (size_t)(it.keybase + ((pos >= 0 && pos < p.nkeys) ? pos : 0));
+                        const size_t row = (size_t)(it.keybase + ((pos >= 0 && pos < it.nkeys) ? pos : 0));
                         const uint8_t* src = kbytes + row * ROWB;
                         const uint32_t x = (uint32_t)(r & 7);
                         const uint32_t rowbase = dst + (uint32_t)(r >> 3) * 1024u + x * 128u + (x << 4);

@@ -62,6 +62,14 @@ __device__ __forceinline__ int row_limit(int kind, int r, int L, int g, int Gm, 
     }
 }
 
+// Row r's causal limit for a select launch (ragged batches through the
+// launch's segment table).
+__device__ __forceinline__ int select_row_limit(const SelectParams& p, int r, bool& ok) {
+    if (p.scan_kind == SCAN_VARLEN_DENSE) { ok = true; return seg_dense_lim(p.seg, r); }
+    if (p.scan_kind == SCAN_VARLEN_PROXY) { ok = true; return seg_proxy_lim(p.seg, p.g, r); }
+    return row_limit(p.scan_kind, r, p.L, p.g, p.Gm, p.maxlen, p.cache_len, ok);
+}
+
 struct RowView {
     const float* S;
     const int32_t* cand;   // null: position = entry index
@@ -797,7 +805,7 @@ __global__ void __launch_bounds__(THR_WARPS * 32) row_threshold_kernel(const Sel
     const int r = p.row0 + rr;
     bool ok;
     const int lim =
-        row_limit(p.scan_kind, r, p.L, p.g, p.Gm, p.maxlen, p.cache_len, ok) - p.lim_shift;
+        select_row_limit(p, r, ok) - p.lim_shift;
     const int n = ok && lim >= 0 ? lim + 1 : 0;
     uint32_t T = 1;
     if (n > p.fast_cap) {
@@ -866,7 +874,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const SelectParams 
 
     bool ok;
     const int lim =
-        row_limit(p.scan_kind, r, p.L, p.g, p.Gm, p.maxlen, p.cache_len, ok) - p.lim_shift;
+        select_row_limit(p, r, ok) - p.lim_shift;
     RowView v;
     v.S = p.S + (size_t)(r - p.row0) * p.S_stride;
     v.lim = lim;
@@ -876,10 +884,14 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const SelectParams 
         v.n = ok && lim >= 0 ? lim + 1 : 0;
     } else {
         const bool dec = p.scan_kind == SCAN_DECODE_DENSE;
-        const int grp = dec ? r / p.Gm : r / p.g;
+        const bool var = p.scan_kind == SCAN_VARLEN_DENSE;
+        const int grp = dec ? r / p.Gm : (var ? seg_group_of(p.seg, p.g, r) : r / p.g);
         v.cand = p.cand + (size_t)(grp - p.cand_base) * p.C;
         v.n = ok ? p.C : 0;
-        if (p.key_scale) v.ksc = p.key_scale + (dec ? (size_t)grp * p.maxlen : 0);
+        if (p.key_scale)
+            v.ksc = p.key_scale + (dec ? (size_t)grp * p.maxlen
+                                       : (var ? (size_t)p.seg.tok[seg_find(p.seg.tok, p.seg.nseq, r)]
+                                              : 0));
         if (p.s_per_group) v.S = p.S + (size_t)(grp - p.cand_base) * p.S_stride;
     }
     if (!ok && threadIdx.x == 0) raise_error(ERRBIT_DATA);

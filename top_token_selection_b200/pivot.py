@@ -33,7 +33,7 @@ ABI_SYMBOLS = [
     "pivot_launch_count", "pivot_decode_noalloc", "pivot_last_error_detail",
     "pivot_reuse_backfill", "pivot_window_union", "pivot_index_varlen",
     "pivot_index_varlen_workspace_size", "pivot_index_window_outside",
-    "pivot_index_window_outside_workspace_size",
+    "pivot_index_window_outside_workspace_size", "pivot_set_score_buffer_cap",
 ]
 KERNELS = {0: "scan", 1: "select", 2: "refine", 3: "reduce", 4: "reuse"}
 
@@ -92,6 +92,7 @@ def load(path: str = LIB_PATH):
         "pivot_decode_workspace_size": ([P, I32, I32, I32], SZ),
         "pivot_get_device_error": ([P], I32),
         "pivot_set_wait_limit_ns": ([ctypes.c_uint64], I32),
+        "pivot_set_score_buffer_cap": ([SZ], I32),
         "pivot_selftest_wait_timeout": ([P], I32),
         "pivot_status_string": ([I32], ctypes.c_char_p),
         "pivot_version": ([], I32),
@@ -180,6 +181,10 @@ def pivot_get_device_error(stream):
 
 def pivot_set_wait_limit_ns(ns):
     return load().pivot_set_wait_limit_ns(ns)
+
+
+def pivot_set_score_buffer_cap(nbytes):
+    return load().pivot_set_score_buffer_cap(nbytes)
 
 
 def pivot_selftest_wait_timeout(stream):
