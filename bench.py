@@ -418,8 +418,8 @@ def measure_extra(run, wl, device, peaks, seed, reps=3):
     """Steps outside the headline step, each timed on its own (CUDA events,
     warm): the MTP decode step on its workload in the three modes, Reuse with
     backfill and the window union on this prefill, and this prefill's tokens
-    as a ragged batch of 2048-token sequences (one call, and Refine sequence
-    by sequence).  Not part of `value`."""
+    as ragged batches of 2048- and 256-token sequences (one call, and Refine
+    sequence by sequence).  Not part of `value`."""
     pv, s = run.pv, run.stream
     sp = pv._stream(s)
     hbm = peaks["hbm_gbs"]
@@ -445,48 +445,50 @@ def measure_extra(run, wl, device, peaks, seed, reps=3):
     nbytes = run.L * (2 * run.k + window) * 4
     out["window_union"] = {"window": window, "ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9,
                            "frac_hbm": nbytes / (ms / 1e3) / 1e9 / hbm, "bytes": nbytes}
-    # a ragged batch: the prefill's tokens cut into sequences of 2048 (each
-    # with its own keys), every step as one launch over all of them, against
-    # the same sequences through the single-sequence calls one after another
-    seg = 2048
-    nseq = run.L // seg
-    if nseq >= 2:
+    # ragged batches: the prefill's tokens cut into equal sequences (each with
+    # its own keys), every step as one launch over all of them, against the
+    # same sequences through the single-sequence calls one after another
+    def ragged(seg, C, topk):
+        nseq = run.L // seg
         T = nseq * seg
         cu = [i * seg for i in range(nseq + 1)]
         dv = run.dev
         cut = lambda t: None if t is None else t[:T]
         batch = pv.make_varlen(cu, cut(dv["q"]), cut(dv["q_scale"]), cut(dv["w"]), cut(dv["k"]),
                                cut(dv["k_scale"]))
-        rag = {"sequences": nseq, "tokens_each": seg, "g": run.g, "C": run.C, "topk": run.k}
-        idx = torch.empty(T, run.k, dtype=torch.int32, device=device)
+        rag = {"sequences": nseq, "tokens_each": seg, "g": run.g, "C": C, "topk": topk}
+        idx = torch.empty(T, topk, dtype=torch.int32, device=device)
         for name, mode in (("dense", pv.DENSE), ("reuse", pv.REUSE), ("refine", pv.REFINE)):
-            wsv = torch.empty(pv.pivot_index_varlen_workspace_size(batch, mode, run.g, run.C, run.k),
+            wsv = torch.empty(pv.pivot_index_varlen_workspace_size(batch, mode, run.g, C, topk),
                               dtype=torch.uint8, device=device)
             ms = _event_ms(lambda: pv._check(pv.pivot_index_varlen(
-                batch, mode, run.g, run.C, run.k, idx.data_ptr(), wsv.data_ptr(), wsv.numel(), sp),
+                batch, mode, run.g, C, topk, idx.data_ptr(), wsv.data_ptr(), wsv.numel(), sp),
                 "varlen"), s, reps)
             rag[name] = {"ms": ms, "queries_per_s": T / (ms / 1e3)}
-        # Refine, sequence by sequence through the single-sequence calls
         seqs = [pv.make_seq(*(None if t is None else t[a:a + seg] for t in
                               (dv["q"], dv["q_scale"], dv["w"], dv["k"], dv["k_scale"])))
                 for a in cu[:-1]]
-        Gs = -(-seg // run.g)
+        assert -(-seg // run.g) <= run.G and C <= run.C
 
-        def per_sequence():
+        def per_sequence():   # Refine, sequence by sequence
             for i, sq in enumerate(seqs):
                 pv._check(pv.pivot_proxy_reduce(sq, run.g, run.pq.data_ptr(), run._ptr(run.pqs),
                                                 run.pw.data_ptr(), sp), "reduce")
                 pv._check(pv.pivot_proxy_scan(sq, run.g, run.pq.data_ptr(), run._ptr(run.pqs),
-                                              run.pw.data_ptr(), run.C, run.k, run.cand.data_ptr(),
+                                              run.pw.data_ptr(), C, topk, run.cand.data_ptr(),
                                               None, run.ws.data_ptr(), run.ws.numel(), sp), "scan")
-                pv._check(pv.pivot_refine(sq, run.g, run.cand.data_ptr(), run.C, run.k,
+                pv._check(pv.pivot_refine(sq, run.g, run.cand.data_ptr(), C, topk,
                                           idx[i * seg:].data_ptr(), None, run.ws.data_ptr(),
                                           run.ws.numel(), sp), "refine")
-        assert Gs <= run.G
         ms = _event_ms(per_sequence, s, reps)
         rag["refine_sequence_by_sequence"] = {"ms": ms, "queries_per_s": T / (ms / 1e3)}
         rag["refine"]["speedup_vs_sequence_by_sequence"] = ms / rag["refine"]["ms"]
-        out["ragged_batch"] = rag
+        return rag
+
+    if run.L >= 2 * 2048:
+        out["ragged_batch"] = ragged(2048, run.C, run.k)
+    if run.L >= 2 * 256 and run.C >= 256 and run.k >= 64:
+        out["ragged_batch_short"] = ragged(256, 256, 64)
     # the MTP decode step (its own workload)
     dw = gen.WORKLOADS["mtp_decode_b32"]
     d = gen.make_decode(B=dw["B"], Gm=dw["Gm"], H=dw["H"], D=dw["D"], dtype=dw["dtype"],
