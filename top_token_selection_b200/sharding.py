@@ -35,3 +35,42 @@ def zigzag_ranges(L: int, g: int, world: int, rank: int):
 def causal_work(ranges):
     """Sum over rows t of (t + 1): the dense indexer's pairs for those rows."""
     return sum((b * (b + 1) - a * (a + 1)) // 2 for a, b in ranges)
+
+
+def varlen_shards(cu_seqlens, world: int):
+    """Whole sequences of a ragged batch per rank, balancing causal work.
+
+    Sequences are independent (each has its own keys), so a packed batch
+    shards by sequence with no exchange step.  Sequence i costs
+    len_i (len_i + 1) / 2 causal pairs; sequences are dealt longest first to
+    the rank with the least work so far (ties to the lower rank), which
+    keeps every rank within the longest sequence's cost of the mean.  A
+    sequence much longer than the rest is better split by rows with
+    ``zigzag_ranges`` and the single-sequence calls.  Returns one ascending
+    list of sequence indices per rank (empty sequences go nowhere)."""
+    n = len(cu_seqlens) - 1
+    if world < 1 or n < 0:
+        raise ValueError("bad arguments")
+    lens = [int(cu_seqlens[i + 1]) - int(cu_seqlens[i]) for i in range(n)]
+    if any(x < 0 for x in lens):
+        raise ValueError("cu_seqlens must not decrease")
+    order = sorted((i for i in range(n) if lens[i] > 0), key=lambda i: (-lens[i], i))
+    load = [0] * world
+    out = [[] for _ in range(world)]
+    for i in order:
+        r = min(range(world), key=lambda x: (load[x], x))
+        out[r].append(i)
+        load[r] += lens[i] * (lens[i] + 1) // 2
+    return [sorted(s) for s in out]
+
+
+def varlen_subbatch(cu_seqlens, seqs):
+    """A rank's sub-batch: its cu_seqlens and, per sequence, the token range
+    [a, b) of the full packed batch its rows come from (and go back to)."""
+    cu = [0]
+    spans = []
+    for i in seqs:
+        a, b = int(cu_seqlens[i]), int(cu_seqlens[i + 1])
+        spans.append((a, b))
+        cu.append(cu[-1] + b - a)
+    return cu, spans
