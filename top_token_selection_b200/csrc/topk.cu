@@ -409,33 +409,36 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
         // Entries are compared as floats: for finite scores, key >= T exactly
         // when score >= key_to_float(T) (-0 and +0 alike); a bound at or
         // below the key of -FLT_MAX keeps every finite score.  Each thread
-        // takes two float4 per step and reserves room for all its kept
-        // entries with one shared-memory atomic (a few entries in a hundred
-        // pass, so the atomics rarely collide).
+        // reserves room for all its kept entries of a step with one
+        // shared-memory atomic (a few entries in a hundred pass, so the
+        // atomics rarely collide).
         const float Tf = T <= 0x00800000u ? -INFINITY : key_to_float(T);
-        for (int i0 = 0; i0 < n4; i0 += 2 * SEL_THREADS) {
-            const int ia = i0 + threadIdx.x, ib = ia + SEL_THREADS;
-            const bool a = ia < n4, b = ib < n4;
-            const float4 xa = a ? __ldcs(S4 + ia) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 xb = b ? __ldcs(S4 + ib) : make_float4(0.f, 0.f, 0.f, 0.f);
-            uint32_t m = 0;
-            if (a) {
-                m |= (xa.x >= Tf ? 1u : 0u) | (xa.y >= Tf ? 2u : 0u) | (xa.z >= Tf ? 4u : 0u) |
-                     (xa.w >= Tf ? 8u : 0u);
-            }
-            if (b) {
-                m |= (xb.x >= Tf ? 16u : 0u) | (xb.y >= Tf ? 32u : 0u) | (xb.z >= Tf ? 64u : 0u) |
-                     (xb.w >= Tf ? 128u : 0u);
-            }
+        // four float4 per thread in flight per step: the loads of a step go
+        // out together, so a row pays one memory latency per 8192 scores
+        auto bits = [&](const float4& x, bool in) -> uint32_t {
+            return in ? ((x.x >= Tf ? 1u : 0u) | (x.y >= Tf ? 2u : 0u) | (x.z >= Tf ? 4u : 0u) |
+                         (x.w >= Tf ? 8u : 0u))
+                      : 0u;
+        };
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i0 = 0; i0 < n4; i0 += 4 * SEL_THREADS) {
+            const int ia = i0 + threadIdx.x, ib = ia + SEL_THREADS, ic = ib + SEL_THREADS,
+                      id = ic + SEL_THREADS;
+            const float4 xa = ia < n4 ? __ldcs(S4 + ia) : z4;
+            const float4 xb = ib < n4 ? __ldcs(S4 + ib) : z4;
+            const float4 xc = ic < n4 ? __ldcs(S4 + ic) : z4;
+            const float4 xd = id < n4 ? __ldcs(S4 + id) : z4;
+            uint32_t m = bits(xa, ia < n4) | (bits(xb, ib < n4) << 4) | (bits(xc, ic < n4) << 8) |
+                         (bits(xd, id < n4) << 12);
             if (m) {
                 uint32_t slot = atomicAdd(s_cnt, (uint32_t)__popc(m));
                 do {
                     const int e = __ffs(m) - 1;
                     m &= m - 1;
-                    const float4& x = e < 4 ? xa : xb;
-                    const int c = e & 3;
+                    const int j = e >> 2, c = e & 3;
+                    const float4 x = j == 0 ? xa : (j == 1 ? xb : (j == 2 ? xc : xd));
                     const float f = c == 0 ? x.x : (c == 1 ? x.y : (c == 2 ? x.z : x.w));
-                    const int pos = 4 * (e < 4 ? ia : ib) + c;
+                    const int pos = 4 * (ia + j * SEL_THREADS) + c;
                     if (slot < (uint32_t)cap) buf[slot] = make_key(ordered_key(f), pos);
                     ++slot;
                 } while (m);
