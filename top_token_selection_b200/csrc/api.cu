@@ -957,13 +957,14 @@ pivot_status_t varlen_single(const pivot_varlen_t* b, int mode, int g, int C, in
     if (ws_bytes < lay.total) return PIVOT_ERR_WORKSPACE;
     if (t.T == 0) return PIVOT_OK;
     uint8_t* base = static_cast<uint8_t*>(ws);
-    // the segment tables, carried to the device as launch parameters
+    // the segment tables, carried to the device as launch parameters (a
+    // pageable host copy could not be captured in a CUDA graph)
     int32_t* d_tab = reinterpret_cast<int32_t*>(base + lay.tabs);
     const int n1 = t.B + 1;
     const std::vector<int32_t>* tabs[4] = {&t.tok, &t.grp, &t.itmD, &t.itmP};
     for (int a = 0; a < 4; ++a)
-        for (int i = 0; i < n1; i += 960) {
-            const int n = n1 - i < 960 ? n1 - i : 960;
+        for (int i = 0; i < n1; i += WRITE_INTS_MAX) {
+            const int n = n1 - i < WRITE_INTS_MAX ? n1 - i : WRITE_INTS_MAX;
             cudaError_t e = launch_write_ints(d_tab + (size_t)a * n1 + i, tabs[a]->data() + i, n, st);
             if (e != cudaSuccess) return from_cuda(e);
             count_launch();
@@ -1058,12 +1059,12 @@ pivot_status_t varlen_single(const pivot_varlen_t* b, int mode, int g, int C, in
     CUtensorMap tq;
     if (!make_tmap(&tq, b->dtype, b->q, (long long)t.T * b->H, b->D, N)) return PIVOT_ERR_CUDA;
     const long long cap_ref = (long long)(lay.S_bytes / ((size_t)C * 4));
+    const SegTable host_seg{t.tok.data(), t.grp.data(), nullptr, t.B, 0, 0};
     for (long long c0 = 0; c0 < t.T; c0 += cap_ref) {
         const int r0 = (int)c0;
         const int r1 = (int)(c0 + cap_ref < t.T ? c0 + cap_ref : t.T);
-        const int jA = seg_group_of(SegTable{t.tok.data(), t.grp.data(), nullptr, t.B, 0, 0}, g, r0);
-        const int jB = seg_group_of(SegTable{t.tok.data(), t.grp.data(), nullptr, t.B, 0, 0}, g,
-                                    r1 - 1) + 1;
+        const int jA = seg_group_of(host_seg, g, r0);
+        const int jB = seg_group_of(host_seg, g, r1 - 1) + 1;
         ScanParams p{};
         p.kind = SCAN_VARLEN_DENSE;
         p.dtype = b->dtype;
