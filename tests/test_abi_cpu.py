@@ -160,3 +160,67 @@ def test_window_outside_rejects_bad_arguments(lib):
     assert pv.pivot_index_window_outside(seq, 0, 4, 16, 8, 4, FAKE, FAKE, 64, None) == 3
     assert pv.pivot_index_window_outside_workspace_size(seq, 2, 4, 16, 8, 4) > 0
     assert pv.pivot_index_window_outside_workspace_size(seq, 2, 4, 16, 8, 0) == 0
+
+
+def test_score_buffer_cap_shrinks_workspaces(lib):
+    """The score-buffer cap bounds what the workspace functions ask for (the
+    calls then work in several launches); 0 restores the default, and caps
+    below 4096 bytes are refused."""
+    import ctypes
+    seq = _seq(L=1000, H=4, D=32)
+    cu = [0, 700, 0 + 700, 1900]
+    arr = (ctypes.c_int32 * len(cu))(*cu)
+    batch = pv.PivotVarlen(pv.E4M3, len(cu) - 1, 64, 128, ctypes.addressof(arr), FAKE, FAKE,
+                           FAKE, FAKE, FAKE)
+    batch._keep = (arr,)
+    full = (pv.pivot_dense_index_workspace_size(seq, 64),
+            pv.pivot_index_varlen_workspace_size(batch, 0, 8, 256, 64),
+            pv.pivot_index_varlen_workspace_size(batch, 2, 8, 256, 64))
+    assert pv.pivot_set_score_buffer_cap(100) == 1
+    try:
+        assert pv.pivot_set_score_buffer_cap(1 << 16) == 0
+        small = (pv.pivot_dense_index_workspace_size(seq, 64),
+                 pv.pivot_index_varlen_workspace_size(batch, 0, 8, 256, 64),
+                 pv.pivot_index_varlen_workspace_size(batch, 2, 8, 256, 64))
+        for a, b in zip(small, full):
+            assert 0 < a < b and a % 256 == 0
+    finally:
+        assert pv.pivot_set_score_buffer_cap(0) == 0
+    assert (pv.pivot_dense_index_workspace_size(seq, 64),
+            pv.pivot_index_varlen_workspace_size(batch, 0, 8, 256, 64),
+            pv.pivot_index_varlen_workspace_size(batch, 2, 8, 256, 64)) == full
+
+
+def test_ragged_batch_workspace_layout(lib):
+    """One-launch ragged batch (tensor-core shape): the workspace holds the
+    four segment tables, proxies and candidates of every group, and one
+    score buffer at the longest sequence's stride; a shape outside the
+    tensor-core tiling sizes for the sequence-by-sequence path instead."""
+    import ctypes
+    lens = [700, 0, 1200, 1, 9]
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    arr = (ctypes.c_int32 * len(cu))(*cu)
+
+    def batch(H, D, dtype):
+        b = pv.PivotVarlen(dtype, len(lens), H, D, ctypes.addressof(arr), FAKE,
+                           FAKE if dtype == pv.E4M3 else None, FAKE, FAKE,
+                           FAKE if dtype == pv.E4M3 else None)
+        b._keep = (arr,)
+        return b
+    g, C, k = 8, 256, 64
+    T, G, maxL = sum(lens), sum(-(-n // g) for n in lens), max(lens)
+    up = lambda x: -(-x // 256) * 256
+    tabs = up(4 * (len(lens) + 1) * 4)
+    prox = up(G * 64 * 128) + up(G * 4) + up(G * 64 * 4) + up(G * C * 4)
+    stride = -(-maxL // 32) * 32
+    dense_rows = up(T * (stride * 4 + 4))
+    b = batch(64, 128, pv.E4M3)
+    assert pv.pivot_index_varlen_workspace_size(b, 0, g, C, k) == tabs + dense_rows
+    assert pv.pivot_index_varlen_workspace_size(b, 1, g, C, k) == tabs + prox + up(G * (stride * 4 + 4))
+    refine_s = max(G * (stride * 4 + 4), T * C * 4)
+    assert pv.pivot_index_varlen_workspace_size(b, 2, g, C, k) == tabs + prox + up(refine_s)
+    # H = 2 is not a tensor-core shape: the sequence-by-sequence layout
+    seq_path = pv.pivot_index_varlen_workspace_size(batch(2, 64, pv.F32), 0, g, C, k)
+    assert 0 < seq_path < T * (stride * 4 + 4)
