@@ -1,0 +1,92 @@
+"""The selection kernels on the CPU: csrc/topk.cu compiled for the host with
+the CUDA features it uses emulated (tests/emu: one thread per CUDA thread,
+block barriers, warp collectives, dynamic shared memory filled with junk),
+under AddressSanitizer and UndefinedBehaviorSanitizer.  Every row must equal
+a plain sort's top-k by (score desc, position asc), listed by position --
+the selection rule of the indexer tutorial (Fig. 1: the top-k positions of
+the scores) with the tie and order readings of this library.
+
+The kernel source is used as it is; only its launch syntax and shared-memory
+declarations are rewritten for the host, and the few helpers it takes from
+common.cuh are copied from there verbatim.
+"""
+import re
+import shutil
+import subprocess
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parents[1]
+CSRC = ROOT / "top_token_selection_b200" / "csrc"
+EMU = ROOT / "tests" / "emu"
+
+pytestmark = pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+
+
+def _rewrite(src, pairs):
+    for old, new in pairs:
+        assert src.count(old) == 1, f"kernel source changed shape: {old!r}"
+        src = src.replace(old, new)
+    return src
+
+
+@pytest.fixture(scope="module")
+def select_check(tmp_path_factory):
+    d = tmp_path_factory.mktemp("select_emu")
+    common = (CSRC / "common.cuh").read_text()
+    errbits = re.search(r"enum : uint32_t \{.*?\};", common, re.S).group(0)
+    helpers = re.search(r"// Order-preserving unsigned key.*?int ceil_div\(int a, int b\) \{[^}]*\}",
+                        common, re.S).group(0)
+    (d / "common.cuh").write_text(
+        "#pragma once\n#include \"emu.h\"\nnamespace pivot {\n" + errbits +
+        "\nextern uint32_t g_error_word;\n"
+        "inline void raise_error(uint32_t bit) { __atomic_fetch_or(&g_error_word, bit, "
+        "__ATOMIC_SEQ_CST); }\n" + helpers + "\n}  // namespace pivot\n")
+    kernels = (CSRC / "kernels.h").read_text()
+    kernels = _rewrite(kernels, [("#include <cuda.h>", "#include \"emu.h\""),
+                                 ("#include <cuda_runtime.h>\n", "")])
+    (d / "kernels.h").write_text(kernels)
+    shutil.copy(CSRC / "segments.h", d / "segments.h")
+    topk = _rewrite((CSRC / "topk.cu").read_text(), [
+        ("extern __shared__ __align__(16) uint8_t smem[];", "uint8_t* smem = emu_smem();"),
+        ("select_kernel<<<p.nrows, SEL_THREADS, lay.total, stream>>>(p);",
+         "emu_launch(p.nrows, SEL_THREADS, lay.total, [&] { select_kernel(p); });"),
+        ("extern __shared__ __align__(16) uint8_t smem_t[];", "uint8_t* smem_t = emu_smem();"),
+        ("row_threshold_kernel<<<grid, THR_WARPS * 32, smem, stream>>>(p, thresh);",
+         "emu_launch(grid, THR_WARPS * 32, smem, [&] { row_threshold_kernel(p, thresh); });"),
+    ])
+    (d / "topk_emu.cpp").write_text(topk)
+    exe = d / "select_check"
+    res = subprocess.run(
+        ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined",
+         "-fno-sanitize-recover=all", "-pthread", "-I", str(d), "-I", str(EMU),
+         str(EMU / "emu.cpp"), str(d / "topk_emu.cpp"), str(EMU / "select_check.cpp"),
+         "-o", str(exe)], capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-4000:]
+    return exe
+
+
+def _run(exe, *args):
+    res = subprocess.run([str(exe), *map(str, args)], capture_output=True, text=True,
+                         timeout=600)
+    assert res.returncode == 0, (res.stdout + res.stderr)[-4000:]
+    assert res.stdout.strip().endswith("0 bad rows, error word 0")
+
+
+@pytest.mark.parametrize("L,K,split,dist,rows,bound", [
+    (20000, 2048, 0, 0, 3, 1),      # sampled bound, buffer path
+    (20000, 2048, 1024, 0, 2, 1),   # a candidate row: the top 1024 listed first
+    (9000, 300, 0, 1, 3, 1),        # five distinct values: ties decided by position
+    (9000, 64, 0, 2, 3, 0),         # signed zeros, bound sampled inside the select
+    (20000, 1, 0, 3, 2, 1),         # k = 1 under a heavy tail
+])
+def test_prefix_rows_match_a_sort(select_check, L, K, split, dist, rows, bound):
+    _run(select_check, "prefix", L, K, split, dist, rows, bound)
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+def test_candidate_rows_match_a_sort(select_check, mode):
+    """Refine rows: cand[j] gives the positions, the member's limit masks later
+    ones; ties (1), -1 padded rows (2), per-key scales multiplied in (3)."""
+    _run(select_check, "cand", 4096, 2048, mode, 2)
