@@ -263,7 +263,7 @@ def neighbour_overlap(dense, rows_per_chunk=4096):
 # CPU oracle on a bounded sample (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_time(p, wl, budget_rows=None, seed=0):
+def oracle_sample_time(p, wl, sample_rows=None, seed=0):
     """Time the oracle on a stratified sample of the step and extrapolate.
 
     Dense rows, proxy-scan groups and Refine rows are sampled evenly over
@@ -275,7 +275,7 @@ def oracle_sample_time(p, wl, budget_rows=None, seed=0):
     L, H, D, g, C, k = p.L, p.H, p.D, wl["g"], wl["C"], wl["topk"]
     G = -(-L // g)
     q, qs, w, kk, ks = p.codes()
-    nd, ns, nr = budget_rows or (48, 24, 192)
+    nd, ns, nr = sample_rows or (48, 24, 192)
     rng = np.random.default_rng(seed)
     dense_rows = np.unique(np.linspace(0, L - 1, nd).astype(np.int64) +
                            rng.integers(0, max(1, L // nd), nd)).clip(0, L - 1).astype(np.int32)

@@ -63,7 +63,7 @@ extern "C" {
 typedef enum {
     PIVOT_OK = 0,
     PIVOT_ERR_INVALID_ARG = 1,   /* null pointer, bad size, C < k, misaligned ... */
-    PIVOT_ERR_UNSUPPORTED = 2,   /* a shape this build does not implement       */
+    PIVOT_ERR_UNSUPPORTED = 2,   /* a shape the library does not implement     */
     PIVOT_ERR_WORKSPACE = 3,     /* ws_bytes below the minimum for the call      */
     PIVOT_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed         */
     PIVOT_ERR_TIMEOUT = 5,       /* a kernel's bounded wait ran out              */

@@ -29,7 +29,7 @@
  *  head, w = 1 and non-negative dot products the form reduces to Fig. 1's
  *  plain dot product.
  *
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent:
  *  - causal prefix is inclusive: query t sees s in [0, t]        ([TUT] Fig. 2)
  *  - selection: the k highest scores, equal scores lower position first;
  *    -0 == +0; the selected positions are listed in ascending order (the
