@@ -780,6 +780,7 @@ VarlenWs varlen_layout(const pivot_varlen_t* b, int mode, int g, int C, int topk
 
 // ---- one launch per stage over all sequences (tensor-core shapes)
 constexpr int VAR_TPI = 32;   // key tiles per scan work item, as in the single-sequence prefill
+constexpr int TABLE_CHUNK = 960;   // integers per launch_write_ints call (its limit)
 
 // Host copies of the segment prefixes (segments.h): tokens, groups and the
 // scan work items of the dense (query rows) and proxy (group rows) scans.
@@ -963,8 +964,8 @@ pivot_status_t varlen_single(const pivot_varlen_t* b, int mode, int g, int C, in
     const int n1 = t.B + 1;
     const std::vector<int32_t>* tabs[4] = {&t.tok, &t.grp, &t.itmD, &t.itmP};
     for (int a = 0; a < 4; ++a)
-        for (int i = 0; i < n1; i += WRITE_INTS_MAX) {
-            const int n = n1 - i < WRITE_INTS_MAX ? n1 - i : WRITE_INTS_MAX;
+        for (int i = 0; i < n1; i += TABLE_CHUNK) {
+            const int n = n1 - i < TABLE_CHUNK ? n1 - i : TABLE_CHUNK;
             cudaError_t e = launch_write_ints(d_tab + (size_t)a * n1 + i, tabs[a]->data() + i, n, st);
             if (e != cudaSuccess) return from_cuda(e);
             count_launch();

@@ -127,9 +127,8 @@ cudaError_t launch_window_union(const int32_t* idx, int rows, int k, int t_begin
 // its group's candidate row (seg_group_of) that are <= its position.
 cudaError_t launch_reuse_varlen(const SegTable& seg, int T, int g, const int32_t* cand, int C,
                                 int topk, int32_t* idx, cudaStream_t stream);
-// Copy n (<= WRITE_INTS_MAX) host integers, carried as launch parameters,
-// to dst: a host-to-device copy that stream capture records like any launch.
-constexpr int WRITE_INTS_MAX = 960;   // 3840 bytes: under the 4 KB parameter limit
+// Copy n (<= 960) host integers, carried as launch parameters, to dst: a
+// host-to-device copy that stream capture records like any launch.
 cudaError_t launch_write_ints(int32_t* dst, const int32_t* host, int n, cudaStream_t stream);
 cudaError_t launch_decode_reuse(int B, int Gm, int maxlen, const int32_t* cache_len,
                                 const int32_t* cand, int C, int topk, int32_t* idx,

@@ -162,6 +162,7 @@ __global__ void reuse_varlen_kernel(const SegTable seg, int T, int g, const int3
     reuse_row(cand + (size_t)j * C, topk, t - seg.tok[b], idx + (size_t)t * topk);
 }
 
+constexpr int WRITE_INTS_MAX = 960;   // 3840 bytes: under the 4 KB parameter limit
 struct IntBlock {
     int32_t v[WRITE_INTS_MAX];
 };
