@@ -7,6 +7,7 @@
 //
 //   select_check prefix <L> <K> <split> <dist> <rows> <use_bound>
 //   select_check cand <C> <K> <mode> <rows>
+//   select_check varlen <kind> <g> <K> <C>     (ragged batch rows, see run_varlen)
 // dist: 0 normal, 1 few distinct values (heavy ties), 2 signed zeros and
 // small integers, 3 a heavy tail (a few huge scores); mode: 0 plain, 1 ties,
 // 2 rows padded with -1, 3 with per-key scales.
@@ -164,6 +165,119 @@ int run_cand(int C, int K, int mode, int nrows) {
     return bad;
 }
 
+// Ragged batch rows: packed rows of several sequences, mapped through the
+// segment tables.  kind 0: dense rows (token r, limit = its position);
+// kind 1: proxy rows (group j, limit = its last member, top-C with the top K
+// first); kind 2: candidate rows of members (their group's candidates,
+// positions <= the member's, key scales from the sequence's first token).
+int run_varlen(int kind, int g, int K, int C) {
+    const std::vector<int> lens = {0, 5, 1, 300, 0, 33, 26, 9};
+    const int B = (int)lens.size();
+    std::vector<int32_t> tok(B + 1, 0), grp(B + 1, 0);
+    int maxL = 0;
+    for (int b = 0; b < B; ++b) {
+        tok[b + 1] = tok[b] + lens[b];
+        grp[b + 1] = grp[b] + (lens[b] + g - 1) / g;
+        maxL = std::max(maxL, lens[b]);
+    }
+    const int T = tok[B], G = grp[B];
+    SegTable seg{tok.data(), grp.data(), nullptr, B, 0, 0};
+    std::mt19937 rng(23 + kind);
+    const int rows = kind == 1 ? G : T;
+    const int width = kind == 2 ? C : maxL;
+    const int Kout = kind == 1 ? C : K;
+    std::vector<float> S((size_t)rows * width), ksc(T);
+    for (auto& x : S) x = (rng() % 3 == 0) ? (float)(rng() % 4) : std::normal_distribution<float>(0.f, 1.f)(rng);
+    for (auto& x : ksc) x = std::uniform_real_distribution<float>(0.5f, 2.0f)(rng);
+    std::vector<int32_t> cand;
+    if (kind == 2) {   // each group's candidates: distinct positions of its sequence
+        cand.assign((size_t)G * C, -1);
+        for (int b = 0; b < B; ++b)
+            for (int j = grp[b]; j < grp[b + 1]; ++j) {
+                std::vector<int> all(lens[b]);
+                for (int i = 0; i < lens[b]; ++i) all[i] = i;
+                std::shuffle(all.begin(), all.end(), rng);
+                const int n = std::min(C, lens[b]);
+                std::sort(all.begin(), all.begin() + n);
+                for (int i = 0; i < n; ++i) cand[(size_t)j * C + i] = all[i];
+            }
+    }
+    std::vector<int32_t> out((size_t)rows * Kout, -7);
+    std::vector<float> outs((size_t)rows * Kout);
+    std::vector<uint32_t> bound(rows);
+    SelectParams sp{};
+    sp.kind = kind == 2 ? SEL_CANDIDATES : SEL_PREFIX;
+    sp.scan_kind = kind == 1 ? SCAN_VARLEN_PROXY : SCAN_VARLEN_DENSE;
+    sp.row0 = 0;
+    sp.nrows = rows;
+    sp.L = maxL;
+    sp.g = g;
+    sp.Gm = 1;
+    sp.S = S.data();
+    sp.S_stride = width;
+    sp.K = Kout;
+    sp.split = kind == 1 ? K : 0;
+    sp.out_idx = out.data();
+    sp.out_score = outs.data();
+    sp.out_base = 0;
+    sp.tail_cap = 4096;
+    sp.npos = maxL;
+    sp.seg = seg;
+    if (kind == 2) {
+        sp.cand = cand.data();
+        sp.cand_base = 0;
+        sp.C = C;
+        sp.key_scale = ksc.data();
+    }
+    // the rows at each sequence's edges (the first two and the last two), in
+    // one launch per contiguous range; rows start at row0 in S and thresh
+    const std::vector<int32_t>& pre = kind == 1 ? grp : tok;
+    std::vector<int> pick;
+    for (int b = 0; b < B; ++b)
+        for (int r = pre[b]; r < pre[b + 1]; ++r)
+            if (r < pre[b] + 2 || r >= pre[b + 1] - 2) pick.push_back(r);
+    for (size_t a = 0; a < pick.size();) {
+        size_t z = a + 1;
+        while (z < pick.size() && pick[z] == pick[z - 1] + 1) ++z;
+        SelectParams q = sp;
+        q.row0 = pick[a];
+        q.nrows = (int)(z - a);
+        q.S = S.data() + (size_t)q.row0 * width;
+        if (kind != 2) {
+            if (launch_row_threshold(q, bound.data() + q.row0, nullptr) != cudaSuccess) return 2;
+            q.thresh = bound.data() + q.row0;
+        }
+        if (launch_select(q, nullptr) != cudaSuccess) return 2;
+        a = z;
+    }
+    int bad = 0;
+    for (int r : pick) {
+        int b = 0;
+        while (!(pre[b] <= r && r < pre[b + 1])) ++b;
+        const int len = lens[b];
+        std::vector<std::pair<uint32_t, int>> e;
+        const float* row = S.data() + (size_t)r * width;
+        if (kind == 0) {
+            for (int i = 0; i <= r - tok[b]; ++i) e.push_back({okey(row[i]), i});
+        } else if (kind == 1) {
+            const int lim = std::min((r - grp[b] + 1) * g, len) - 1;
+            for (int i = 0; i <= lim; ++i) e.push_back({okey(row[i]), i});
+        } else {
+            const int t = r - tok[b], j = grp[b] + t / g;
+            for (int i = 0; i < C; ++i) {
+                const int pos = cand[(size_t)j * C + i];
+                if (pos >= 0 && pos <= t) e.push_back({okey(row[i] * ksc[tok[b] + pos]), pos});
+            }
+        }
+        const std::vector<int> want = reference(e, Kout, kind == 1 ? K : 0);
+        if (want != std::vector<int>(out.begin() + (size_t)r * Kout, out.begin() + (size_t)(r + 1) * Kout)) {
+            ++bad;
+            std::printf("ragged kind %d row %d (sequence %d): mismatch\n", kind, r, b);
+        }
+    }
+    return bad;
+}
+
 }  // namespace
 
 int main(int argc, char** argv) {
@@ -175,6 +289,8 @@ int main(int argc, char** argv) {
                          atoi(argv[7]) != 0);
     else if (what == "cand" && argc == 6)
         bad = run_cand(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]));
+    else if (what == "varlen" && argc == 6)
+        bad = run_varlen(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]));
     else
         return 2;
     std::printf("%d bad rows, error word %u\n", bad, g_error_word);

@@ -90,3 +90,13 @@ def test_candidate_rows_match_a_sort(select_check, mode):
     """Refine rows: cand[j] gives the positions, the member's limit masks later
     ones; ties (1), -1 padded rows (2), per-key scales multiplied in (3)."""
     _run(select_check, "cand", 4096, 2048, mode, 2)
+
+
+@pytest.mark.parametrize("kind,g,K,C", [(0, 8, 64, 0), (1, 8, 16, 96), (2, 8, 16, 96),
+                                        (0, 3, 1, 0), (2, 3, 40, 40)])
+def test_ragged_batch_rows_match_a_sort(select_check, kind, g, K, C):
+    """Rows of a packed ragged batch (sequences of 0 to 300 tokens) mapped
+    through the segment tables -- dense rows, proxy rows (top C, the top K
+    first) and member candidate rows with per-sequence key scales -- at each
+    sequence's edges, where a mapping error would show."""
+    _run(select_check, "varlen", kind, g, K, C)
