@@ -8,6 +8,7 @@
 //   select_check prefix <L> <K> <split> <dist> <rows> <use_bound>
 //   select_check cand <C> <K> <mode> <rows>
 //   select_check varlen <kind> <g> <K> <C>     (ragged batch rows, see run_varlen)
+//   select_check decode <kind> <K>             (MTP decode rows, see run_decode)
 // dist: 0 normal, 1 few distinct values (heavy ties), 2 signed zeros and
 // small integers, 3 a heavy tail (a few huge scores); mode: 0 plain, 1 ties,
 // 2 rows padded with -1, 3 with per-key scales.
@@ -19,6 +20,7 @@
 #include <string>
 #include <vector>
 
+#include "common.cuh"   // the error bits
 #include "kernels.h"
 
 namespace pivot {
@@ -278,6 +280,61 @@ int run_varlen(int kind, int g, int K, int C) {
     return bad;
 }
 
+// Decode rows (the MTP members of B sequences with cached keys): kind 0,
+// member m of sequence b sees [0, cache_len[b] - Gm + m]; kind 1, the proxy
+// of sequence b sees [0, cache_len[b] - 1].  Cache lengths outside the
+// valid range give an all -1 row and raise the data error.
+int run_decode(int kind, int K) {
+    const int B = 6, Gm = 3, maxlen = 700;
+    const std::vector<int32_t> cache_len = {3, 700, 41, 2, 900, 260};   // 2 and 900 invalid
+    const int rows = kind == 0 ? B * Gm : B;
+    std::mt19937 rng(31 + kind);
+    std::vector<float> S((size_t)rows * maxlen);
+    for (auto& x : S) x = (rng() % 4 == 0) ? (float)(rng() % 3) : std::normal_distribution<float>(0.f, 1.f)(rng);
+    std::vector<int32_t> out((size_t)rows * K, -7);
+    std::vector<float> outs((size_t)rows * K);
+    SelectParams sp{};
+    sp.kind = SEL_PREFIX;
+    sp.scan_kind = kind == 0 ? SCAN_DECODE_DENSE : SCAN_DECODE_PROXY;
+    sp.row0 = 0;
+    sp.nrows = rows;
+    sp.Gm = Gm;
+    sp.g = 1;
+    sp.maxlen = maxlen;
+    sp.cache_len = cache_len.data();
+    sp.S = S.data();
+    sp.S_stride = maxlen;
+    sp.K = K;
+    sp.out_idx = out.data();
+    sp.out_score = outs.data();
+    sp.out_base = 0;
+    sp.tail_cap = 4096;
+    sp.npos = maxlen;
+    if (launch_select(sp, nullptr) != cudaSuccess) return 2;
+    int bad = 0;
+    for (int r = 0; r < rows; ++r) {
+        const int b = kind == 0 ? r / Gm : r, m = kind == 0 ? r % Gm : 0;
+        const int n = cache_len[b];
+        const bool valid = kind == 0 ? (n >= Gm && n <= maxlen) : (n >= 1 && n <= maxlen);
+        std::vector<std::pair<uint32_t, int>> e;
+        if (valid) {
+            const int lim = kind == 0 ? n - Gm + m : n - 1;
+            for (int i = 0; i <= lim; ++i) e.push_back({okey(S[(size_t)r * maxlen + i]), i});
+        }
+        if (reference(e, K, 0) != std::vector<int>(out.begin() + (size_t)r * K, out.begin() + (size_t)(r + 1) * K)) {
+            ++bad;
+            std::printf("decode kind %d row %d: mismatch\n", kind, r);
+        }
+    }
+    // the invalid lengths must have raised the data error (and nothing else)
+    if (g_error_word != ERRBIT_DATA) {
+        std::printf("error word %u, expected the data error\n", g_error_word);
+        ++bad;
+    }
+    g_error_word = 0;
+    return bad;
+}
+
 }  // namespace
 
 int main(int argc, char** argv) {
@@ -289,6 +346,8 @@ int main(int argc, char** argv) {
                          atoi(argv[7]) != 0);
     else if (what == "cand" && argc == 6)
         bad = run_cand(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]));
+    else if (what == "decode" && argc == 4)
+        bad = run_decode(atoi(argv[2]), atoi(argv[3]));
     else if (what == "varlen" && argc == 6)
         bad = run_varlen(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]));
     else

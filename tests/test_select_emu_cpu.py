@@ -100,3 +100,11 @@ def test_ragged_batch_rows_match_a_sort(select_check, kind, g, K, C):
     first) and member candidate rows with per-sequence key scales -- at each
     sequence's edges, where a mapping error would show."""
     _run(select_check, "varlen", kind, g, K, C)
+
+
+@pytest.mark.parametrize("kind,K", [(0, 64), (1, 300)])
+def test_decode_rows_match_a_sort(select_check, kind, K):
+    """MTP decode rows over ragged cache lengths: member m of a sequence sees
+    [0, cache_len - Gm + m], the proxy [0, cache_len - 1]; a length outside
+    [Gm, maxlen] gives a -1 row and raises the data error."""
+    _run(select_check, "decode", kind, K)
