@@ -10,76 +10,26 @@ batches and decode; the window union (indexer tutorial Fig. 3).  The bf16 /
 e4m3 stores of the proxy are not emulated (their conversions would abort).
 """
 import ctypes
-import re
 import shutil
-import subprocess
-from pathlib import Path
 
 import numpy as np
 import pytest
 
 import oracle
-
-ROOT = Path(__file__).resolve().parents[1]
-CSRC = ROOT / "top_token_selection_b200" / "csrc"
-EMU = ROOT / "tests" / "emu"
+from emu_build import CSRC, EMU, compile_, prepare, rewrite, rewrite_launches
 
 pytestmark = pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
-
-SHIM_EXTRA = r"""
-struct alignas(16) uint4 { uint32_t x, y, z, w; };
-inline uint4 make_uint4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) { return {a, b, c, d}; }
-inline float __fadd_rn(float a, float b) { return a + b; }   // IEEE single, round to nearest
-inline float __fmul_rn(float a, float b) { return a * b; }
-inline float __fdiv_rn(float a, float b) { return a / b; }
-struct __nv_bfloat16 { uint16_t x; };
-inline __nv_bfloat16 __float2bfloat16_rn(float) { EMU_FAIL("bf16 store not emulated"); }
-inline uint16_t __bfloat16_as_ushort(__nv_bfloat16 v) { return v.x; }
-inline float e4m3_to_f32(uint8_t) { EMU_FAIL("e4m3 not emulated"); }
-inline uint8_t f32_to_e4m3_satfinite(float) { EMU_FAIL("e4m3 not emulated"); }
-inline float bf16_to_f32(uint16_t c) { return __uint_as_float((uint32_t)c << 16); }
-"""
-
-
-def _rewrite_launches(src):
-    """kernel<<<grid, block, smem, stream>>>(args); -> emu_launch(grid, block, smem, [&] {...});"""
-    pat = re.compile(r"([A-Za-z_][\w]*(?:<[^<>;]*>)?)<<<(.*?),(.*?),(.*?),\s*stream>>>\((.*?)\);",
-                     re.S)
-    out, n = pat.subn(lambda m: f"emu_launch({m.group(2)}, {m.group(3)}, {m.group(4)}, "
-                                f"[&] {{ {m.group(1)}({m.group(5)}); }});", src)
-    assert n == src.count("<<<"), "a launch was not rewritten"
-    return out
 
 
 @pytest.fixture(scope="module")
 def emu(tmp_path_factory):
     d = tmp_path_factory.mktemp("reuse_emu")
-    common = (CSRC / "common.cuh").read_text()
-    errbits = re.search(r"enum : uint32_t \{.*?\};", common, re.S).group(0)
-    helpers = re.search(r"// Order-preserving unsigned key.*?int ceil_div\(int a, int b\) \{[^}]*\}",
-                        common, re.S).group(0)
-    (d / "common.cuh").write_text(
-        "#pragma once\n#include \"emu.h\"\n#include \"pivot.h\"\nnamespace pivot {\n" + errbits +
-        "\nextern uint32_t g_error_word;\n"
-        "inline void raise_error(uint32_t bit) { __atomic_fetch_or(&g_error_word, bit, "
-        "__ATOMIC_SEQ_CST); }\n" + helpers + SHIM_EXTRA + "\n}  // namespace pivot\n")
-    kernels = (CSRC / "kernels.h").read_text()
-    assert kernels.count("#include <cuda.h>") == 1
-    kernels = kernels.replace("#include <cuda.h>", "#include \"emu.h\"").replace(
-        "#include <cuda_runtime.h>\n", "")
-    (d / "kernels.h").write_text(kernels)
-    shutil.copy(CSRC / "segments.h", d / "segments.h")
-    src = (CSRC / "proxy_reuse.cu").read_text()
-    assert src.count("extern __shared__ float qbar_s[];") == 1
-    src = src.replace("extern __shared__ float qbar_s[];", "float* qbar_s = (float*)emu_smem();")
-    (d / "proxy_reuse_emu.cpp").write_text(_rewrite_launches(src))
-    so = d / "libreuse_emu.so"
-    res = subprocess.run(
-        ["g++", "-std=c++20", "-O1", "-g", "-fPIC", "-shared", "-pthread", "-I", str(d),
-         "-I", str(EMU), "-I", str(ROOT / "include"), str(EMU / "emu.cpp"),
-         str(d / "proxy_reuse_emu.cpp"), str(EMU / "reuse_glue.cpp"), "-o", str(so)],
-        capture_output=True, text=True, timeout=600)
-    assert res.returncode == 0, res.stderr[-4000:]
+    prepare(d, extra=True)
+    src = rewrite((CSRC / "proxy_reuse.cu").read_text(),
+                  [("extern __shared__ float qbar_s[];", "float* qbar_s = (float*)emu_smem();")])
+    (d / "proxy_reuse_emu.cpp").write_text(rewrite_launches(src))
+    so = compile_(d, [d / "proxy_reuse_emu.cpp", EMU / "reuse_glue.cpp"], d / "libreuse_emu.so",
+                  shared=True)
     lib = ctypes.CDLL(str(so))
     lib.emu_error_word.restype = ctypes.c_uint32
     return lib

@@ -10,45 +10,21 @@ The kernel source is used as it is; only its launch syntax and shared-memory
 declarations are rewritten for the host, and the few helpers it takes from
 common.cuh are copied from there verbatim.
 """
-import re
 import shutil
 import subprocess
-from pathlib import Path
 
 import pytest
 
-ROOT = Path(__file__).resolve().parents[1]
-CSRC = ROOT / "top_token_selection_b200" / "csrc"
-EMU = ROOT / "tests" / "emu"
+from emu_build import CSRC, EMU, compile_, prepare, rewrite
 
 pytestmark = pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
-
-
-def _rewrite(src, pairs):
-    for old, new in pairs:
-        assert src.count(old) == 1, f"kernel source changed shape: {old!r}"
-        src = src.replace(old, new)
-    return src
 
 
 @pytest.fixture(scope="module")
 def select_check(tmp_path_factory):
     d = tmp_path_factory.mktemp("select_emu")
-    common = (CSRC / "common.cuh").read_text()
-    errbits = re.search(r"enum : uint32_t \{.*?\};", common, re.S).group(0)
-    helpers = re.search(r"// Order-preserving unsigned key.*?int ceil_div\(int a, int b\) \{[^}]*\}",
-                        common, re.S).group(0)
-    (d / "common.cuh").write_text(
-        "#pragma once\n#include \"emu.h\"\nnamespace pivot {\n" + errbits +
-        "\nextern uint32_t g_error_word;\n"
-        "inline void raise_error(uint32_t bit) { __atomic_fetch_or(&g_error_word, bit, "
-        "__ATOMIC_SEQ_CST); }\n" + helpers + "\n}  // namespace pivot\n")
-    kernels = (CSRC / "kernels.h").read_text()
-    kernels = _rewrite(kernels, [("#include <cuda.h>", "#include \"emu.h\""),
-                                 ("#include <cuda_runtime.h>\n", "")])
-    (d / "kernels.h").write_text(kernels)
-    shutil.copy(CSRC / "segments.h", d / "segments.h")
-    topk = _rewrite((CSRC / "topk.cu").read_text(), [
+    prepare(d)
+    topk = rewrite((CSRC / "topk.cu").read_text(), [
         ("extern __shared__ __align__(16) uint8_t smem[];", "uint8_t* smem = emu_smem();"),
         ("select_kernel<<<p.nrows, SEL_THREADS, lay.total, stream>>>(p);",
          "emu_launch(p.nrows, SEL_THREADS, lay.total, [&] { select_kernel(p); });"),
@@ -57,14 +33,8 @@ def select_check(tmp_path_factory):
          "emu_launch(grid, THR_WARPS * 32, smem, [&] { row_threshold_kernel(p, thresh); });"),
     ])
     (d / "topk_emu.cpp").write_text(topk)
-    exe = d / "select_check"
-    res = subprocess.run(
-        ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined",
-         "-fno-sanitize-recover=all", "-pthread", "-I", str(d), "-I", str(EMU),
-         str(EMU / "emu.cpp"), str(d / "topk_emu.cpp"), str(EMU / "select_check.cpp"),
-         "-o", str(exe)], capture_output=True, text=True, timeout=600)
-    assert res.returncode == 0, res.stderr[-4000:]
-    return exe
+    return compile_(d, [d / "topk_emu.cpp", EMU / "select_check.cpp"], d / "select_check",
+                    sanitize=True)
 
 
 def _run(exe, *args):

@@ -11,19 +11,13 @@ rows (limit = the group's last member), MTP decode rows over ragged cache
 lengths, and Refine rows over candidate keys.
 """
 import ctypes
-import re
 import shutil
-import subprocess
-from pathlib import Path
 
 import numpy as np
 import pytest
 
-from test_reuse_emu_cpu import SHIM_EXTRA, _rewrite_launches
+from emu_build import CSRC, EMU, compile_, prepare, rewrite, rewrite_launches
 
-ROOT = Path(__file__).resolve().parents[1]
-CSRC = ROOT / "top_token_selection_b200" / "csrc"
-EMU = ROOT / "tests" / "emu"
 F32, BF16 = 0, 1
 PREFILL_DENSE, PREFILL_PROXY, DECODE_DENSE, DECODE_PROXY = 0, 1, 2, 3
 SENTINEL = np.float32(-12345.0)
@@ -34,31 +28,13 @@ pytestmark = pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
 @pytest.fixture(scope="module")
 def emu(tmp_path_factory):
     d = tmp_path_factory.mktemp("simt_emu")
-    common = (CSRC / "common.cuh").read_text()
-    errbits = re.search(r"enum : uint32_t \{.*?\};", common, re.S).group(0)
-    helpers = re.search(r"// Order-preserving unsigned key.*?int ceil_div\(int a, int b\) \{[^}]*\}",
-                        common, re.S).group(0)
-    (d / "common.cuh").write_text(
-        "#pragma once\n#include <cmath>\n#include \"emu.h\"\n#include \"pivot.h\"\n"
-        "namespace pivot {\n" + errbits + "\nextern uint32_t g_error_word;\n"
-        "inline void raise_error(uint32_t bit) { __atomic_fetch_or(&g_error_word, bit, "
-        "__ATOMIC_SEQ_CST); }\n" + helpers + SHIM_EXTRA +
-        "\ninline float fmaf(float a, float b, float c) { return std::fma(a, b, c); }\n"
-        "}  // namespace pivot\n")
-    kernels = (CSRC / "kernels.h").read_text().replace("#include <cuda.h>", "#include \"emu.h\"")
-    (d / "kernels.h").write_text(kernels.replace("#include <cuda_runtime.h>\n", ""))
-    shutil.copy(CSRC / "segments.h", d / "segments.h")
+    prepare(d, extra=True)
     src = (CSRC / "simt.cu").read_text()
     assert src.count("extern __shared__ float sm[];") == 2
     src = src.replace("extern __shared__ float sm[];", "float* sm = (float*)emu_smem();")
-    (d / "simt_emu.cpp").write_text(_rewrite_launches(src))
-    so = d / "libsimt_emu.so"
-    res = subprocess.run(
-        ["g++", "-std=c++20", "-O1", "-g", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
-         "-I", str(d), "-I", str(EMU), "-I", str(ROOT / "include"), str(EMU / "emu.cpp"),
-         str(d / "simt_emu.cpp"), str(EMU / "simt_glue.cpp"), "-o", str(so)],
-        capture_output=True, text=True, timeout=600)
-    assert res.returncode == 0, res.stderr[-4000:]
+    (d / "simt_emu.cpp").write_text(rewrite_launches(src))
+    so = compile_(d, [d / "simt_emu.cpp", EMU / "simt_glue.cpp"], d / "libsimt_emu.so",
+                  shared=True)
     lib = ctypes.CDLL(str(so))
     lib.emu_error_word.restype = ctypes.c_uint32
     lib.emu_scan_simt.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 5 + \
