@@ -9,6 +9,7 @@
 //   select_check cand <C> <K> <mode> <rows>
 //   select_check varlen <kind> <g> <K> <C>     (ragged batch rows, see run_varlen)
 //   select_check decode <kind> <K>             (MTP decode rows, see run_decode)
+//   select_check backfill <L> <g> <C> <K>      (Reuse with backfill, see run_backfill)
 // dist: 0 normal, 1 few distinct values (heavy ties), 2 signed zeros and
 // small integers, 3 a heavy tail (a few huge scores); mode: 0 plain, 1 ties,
 // 2 rows padded with -1, 3 with per-key scales.
@@ -280,6 +281,61 @@ int run_varlen(int kind, int g, int K, int C) {
     return bad;
 }
 
+// Reuse with backfill: member t of group j = t / g takes the top K of the
+// group's candidates at or before t, ranked by the group's proxy scores
+// (one score row per group), lower position first on ties.
+int run_backfill(int L, int g, int C, int K) {
+    const int G = (L + g - 1) / g;
+    std::mt19937 rng(41 + g);
+    std::vector<int32_t> cand((size_t)G * C, -1);
+    std::vector<float> sc((size_t)G * C);
+    for (int j = 0; j < G; ++j) {
+        const int e = std::min(L, (j + 1) * g) - 1;
+        std::vector<int> all(e + 1);
+        for (int i = 0; i <= e; ++i) all[i] = i;
+        std::shuffle(all.begin(), all.end(), rng);
+        const int n = std::min(C, e + 1);
+        std::sort(all.begin(), all.begin() + n);
+        for (int i = 0; i < n; ++i) cand[(size_t)j * C + i] = all[i];
+        for (int i = 0; i < C; ++i) sc[(size_t)j * C + i] = (float)(rng() % 6);   // many ties
+    }
+    std::vector<int32_t> out((size_t)L * K, -7);
+    SelectParams sp{};
+    sp.kind = SEL_CANDIDATES;
+    sp.scan_kind = SCAN_PREFILL_DENSE;
+    sp.row0 = 0;
+    sp.nrows = L;
+    sp.L = L;
+    sp.g = g;
+    sp.Gm = 1;
+    sp.S = sc.data();
+    sp.S_stride = C;
+    sp.s_per_group = 1;
+    sp.cand = cand.data();
+    sp.cand_base = 0;
+    sp.C = C;
+    sp.K = K;
+    sp.out_idx = out.data();
+    sp.out_base = 0;
+    sp.tail_cap = 4096;
+    sp.npos = L;
+    if (launch_select(sp, nullptr) != cudaSuccess) return 2;
+    int bad = 0;
+    for (int t = 0; t < L; ++t) {
+        const int j = t / g;
+        std::vector<std::pair<uint32_t, int>> e;
+        for (int i = 0; i < C; ++i) {
+            const int pos = cand[(size_t)j * C + i];
+            if (pos >= 0 && pos <= t) e.push_back({okey(sc[(size_t)j * C + i]), pos});
+        }
+        if (reference(e, K, 0) != std::vector<int>(out.begin() + (size_t)t * K, out.begin() + (size_t)(t + 1) * K)) {
+            ++bad;
+            std::printf("backfill row %d: mismatch\n", t);
+        }
+    }
+    return bad;
+}
+
 // Decode rows (the MTP members of B sequences with cached keys): kind 0,
 // member m of sequence b sees [0, cache_len[b] - Gm + m]; kind 1, the proxy
 // of sequence b sees [0, cache_len[b] - 1].  Cache lengths outside the
@@ -346,6 +402,8 @@ int main(int argc, char** argv) {
                          atoi(argv[7]) != 0);
     else if (what == "cand" && argc == 6)
         bad = run_cand(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]));
+    else if (what == "backfill" && argc == 6)
+        bad = run_backfill(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]));
     else if (what == "decode" && argc == 4)
         bad = run_decode(atoi(argv[2]), atoi(argv[3]));
     else if (what == "varlen" && argc == 6)

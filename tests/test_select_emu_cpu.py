@@ -78,3 +78,12 @@ def test_decode_rows_match_a_sort(select_check, kind, K):
     [0, cache_len - Gm + m], the proxy [0, cache_len - 1]; a length outside
     [Gm, maxlen] gives a -1 row and raises the data error."""
     _run(select_check, "decode", kind, K)
+
+
+@pytest.mark.parametrize("L,g,C,K", [(40, 4, 12, 5), (33, 8, 30, 30)])
+def test_backfill_rows_match_a_sort(select_check, L, g, C, K):
+    """Reuse with backfill (the reading this library takes where the PIVOT
+    abstract's Reuse leaves masked slots open): member t takes the top K of
+    its group's candidates at or before t by proxy score, lower position
+    first on ties (scores drawn from six values, so ties are common)."""
+    _run(select_check, "backfill", L, g, C, K)
