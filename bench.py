@@ -7,9 +7,14 @@ One step is one pass of the whole hot path over one synthetic sequence:
 the dense indexer (every query scans its full causal prefix, keeps top-k),
 then PIVOT -- proxy reduce, one proxy scan per group (top-C candidates),
 PIVOT-Reuse and PIVOT-Refine -- so each step produces the dense, Reuse and
-Refine index sets of all L queries.  ``value`` = L * n_gpus / step time
-(queries/s, whole job).  Per-mode times, Reuse/Refine recall against dense
-and the neighbour overlap of dense are reported beside it.
+Refine index sets of all L queries.  ``value`` = L / step time (queries/s,
+whole job).  With N > 1 ranks the one sequence's query rows are split
+across the ranks by zig-zag group blocks (every rank holds all keys and
+indexes its own rows; no exchange), so the total work is fixed (strong
+scaling).  Per-mode times, Reuse/Refine recall against dense and the
+neighbour overlap of dense are reported beside it, and (rank 0, N = 1) the
+other prefill workloads -- dsa_prefill_16k and the dsa_prefill_64k sweep
+over g in {8, 16} and C in {4096, 8192} -- each timed on its own.
 
 Timing: W untimed warm-up steps, then K steps between CUDA events on the
 launching stream, bracketed by a barrier and a device synchronize; the max
@@ -44,6 +49,14 @@ DEFAULT_WORKLOAD = "long_prefill_128k_fp8"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
+# DRAM bytes per causal pair of the dense scan kernel, from one ncu capture
+# of the fp8_prefill_16k dense scan (dram__bytes_read.sum +
+# dram__bytes_write.sum over its causal pairs; the summary is under
+# profiles/).  Valid only for the kernel sources it was taken on: the bench
+# reports it while these files hash (sha1, first 12 hex digits) as listed,
+# and null otherwise.
+SCAN_TRAFFIC = {"bytes_per_pair": None, "sources": {}}
+
 
 # ---------------------------------------------------------------------------
 # distributed plumbing (host logic, testable on CPU with gloo)
@@ -54,9 +67,11 @@ def dist_env():
             int(os.environ.get("WORLD_SIZE", 1)))
 
 
-def rank_seed(base_seed: int, rank: int) -> int:
-    """Weak scaling: every rank indexes its own independent sequence."""
-    return base_seed + 1000003 * rank
+def rank_rows(L: int, g: int, world: int, rank: int):
+    """This rank's query row ranges of the one sequence: the whole sequence on
+    one GPU, else its zig-zag group blocks (balanced causal work)."""
+    from top_token_selection_b200.sharding import zigzag_ranges
+    return [(0, L)] if world == 1 else zigzag_ranges(L, g, world, rank)
 
 
 def max_over_ranks(x: float, device=None) -> float:
@@ -68,9 +83,10 @@ def max_over_ranks(x: float, device=None) -> float:
     return float(t.item())
 
 
-def aggregate_value(queries_per_rank: int, world: int, ms_max: float, steps: int) -> float:
-    """Whole-job queries/s: all ranks' queries over the slowest rank's time."""
-    return queries_per_rank * world * steps / (ms_max / 1e3)
+def job_value(total_queries: int, ms_max: float, steps: int) -> float:
+    """Whole-job queries/s: the sequence's queries per step over the slowest
+    rank's time (every rank holds a share of the same rows)."""
+    return total_queries * steps / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------------------
@@ -153,9 +169,10 @@ def make_inputs(wl, seed):
 
 
 class Runner:
-    """Device buffers and one step of the hot path through the C ABI."""
+    """Device buffers and one step of the hot path through the C ABI over
+    this rank's query row ranges (the whole sequence on one GPU)."""
 
-    def __init__(self, p, wl, device):
+    def __init__(self, p, wl, device, ranges=None):
         from top_token_selection_b200 import pivot as pv
         self.pv = pv
         pv.load()
@@ -163,6 +180,8 @@ class Runner:
         self.L, self.H, self.D = p.L, p.H, p.D
         self.g, self.C, self.k = wl["g"], wl["C"], wl["topk"]
         self.G = -(-self.L // self.g)
+        self.ranges = list(ranges) if ranges else [(0, self.L)]
+        self.rows = sum(b - a for a, b in self.ranges)
         d = device
         self.host = {"q": p.q, "q_scale": p.q_scale, "w": p.w, "k": p.k, "k_scale": p.k_scale}
         self.dev = {n: (None if t is None else torch.empty_like(t, device=d))
@@ -182,50 +201,74 @@ class Runner:
         self.pqs = (torch.empty(self.G, dtype=torch.float32, device=d)
                     if wl["dtype"] == gen.E4M3 else None)
         self.pw = torch.empty(self.G, self.H, dtype=torch.float32, device=d)
-        wsb = max(pv.pivot_dense_index_workspace_size(self.seq, self.k),
-                  pv.pivot_proxy_scan_workspace_size(self.seq, self.g, self.C),
-                  pv.pivot_refine_workspace_size(self.seq, self.g, self.C, self.k))
+        wsb = 0
+        for a, b in self.ranges:
+            sq = self.range_seq(self.seq, a, b)
+            wsb = max(wsb, pv.pivot_dense_index_workspace_size(sq, self.k),
+                      pv.pivot_proxy_scan_workspace_size(sq, self.g, self.C),
+                      pv.pivot_refine_workspace_size(sq, self.g, self.C, self.k))
         self.ws = torch.empty(wsb, dtype=torch.uint8, device=d)
         self.stream = torch.cuda.current_stream()
+
+    def range_seq(self, seq, a, b):
+        sq = self.pv.PivotSeq.from_buffer_copy(seq)
+        sq.t_begin, sq.t_end = a, b
+        return sq
 
     def _ptr(self, t):
         return None if t is None else t.data_ptr()
 
     def step(self, events=None, seq=None, outs=None):
         """One step on `seq` (default: this runner's sequence) into `outs` =
-        (dense, reuse, refine) index buffers (default: this runner's)."""
+        (dense, reuse, refine) index buffers (default: this runner's), for
+        every row range of this rank."""
         pv, s = self.pv, self.stream
         sp = pv._stream(s)
         ws, wsn = self.ws.data_ptr(), self.ws.numel()
         seq = self.seq if seq is None else seq
         dense, reu, ref = (self.dense, self.reu, self.ref) if outs is None else outs
+        seqs = [(a, b, self.range_seq(seq, a, b)) for a, b in self.ranges]
+        g, k, C = self.g, self.k, self.C
 
         def mark(i):
             if events is not None:
                 events[i].record(s)
+
+        def grp(a):   # this range's first group row in pq / pw / cand
+            return a // g
         mark(0)
-        pv._check(pv.pivot_dense_index(seq, self.k, dense.data_ptr(), None, ws, wsn, sp),
-                  "dense")
+        for a, b, sq in seqs:
+            pv._check(pv.pivot_dense_index(sq, k, dense[a].data_ptr(), None, ws, wsn, sp),
+                      "dense")
         mark(1)
-        pv._check(pv.pivot_proxy_reduce(seq, self.g, self.pq.data_ptr(), self._ptr(self.pqs),
-                                        self.pw.data_ptr(), sp), "reduce")
+        for a, b, sq in seqs:
+            pv._check(pv.pivot_proxy_reduce(sq, g, self.pq[grp(a)].data_ptr(),
+                                            None if self.pqs is None else
+                                            self.pqs[grp(a):].data_ptr(),
+                                            self.pw[grp(a)].data_ptr(), sp), "reduce")
         mark(2)
-        pv._check(pv.pivot_proxy_scan(seq, self.g, self.pq.data_ptr(), self._ptr(self.pqs),
-                                      self.pw.data_ptr(), self.C, self.k, self.cand.data_ptr(),
-                                      None, ws, wsn, sp), "scan")
+        for a, b, sq in seqs:
+            pv._check(pv.pivot_proxy_scan(sq, g, self.pq[grp(a)].data_ptr(),
+                                          None if self.pqs is None else
+                                          self.pqs[grp(a):].data_ptr(),
+                                          self.pw[grp(a)].data_ptr(), C, k,
+                                          self.cand[grp(a)].data_ptr(), None, ws, wsn, sp),
+                      "scan")
         mark(3)
-        pv._check(pv.pivot_reuse(0, self.L, self.g, self.cand.data_ptr(), self.C, self.k,
-                                 reu.data_ptr(), sp), "reuse")
+        for a, b, sq in seqs:
+            pv._check(pv.pivot_reuse(a, b, g, self.cand[grp(a)].data_ptr(), C, k,
+                                     reu[a].data_ptr(), sp), "reuse")
         mark(4)
-        pv._check(pv.pivot_refine(seq, self.g, self.cand.data_ptr(), self.C, self.k,
-                                  ref.data_ptr(), None, ws, wsn, sp), "refine")
+        for a, b, sq in seqs:
+            pv._check(pv.pivot_refine(sq, g, self.cand[grp(a)].data_ptr(), C, k,
+                                      ref[a].data_ptr(), None, ws, wsn, sp), "refine")
         mark(5)
 
     def h2d_bytes(self):
         return sum(t.numel() * t.element_size() for t in self.host.values() if t is not None)
 
     def d2h_bytes(self):
-        return 3 * self.L * self.k * 4
+        return 3 * self.rows * self.k * 4
 
 
 def recall_stats(dense, other, rows_per_chunk=4096):
@@ -353,7 +396,7 @@ def run_reference(args, wl):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
-    p = make_inputs(wl, rank_seed(args.seed, 0))
+    p = make_inputs(wl, args.seed)
     times = []
     desc, threads = "", 0
     for i in range(args.warmup + args.steps):
@@ -381,29 +424,65 @@ def config_of(wl, args):
             "q_k_format": gen.DTYPE_NAMES[wl["dtype"]] + (" + fp32 per-token scale"
                                                          if wl["dtype"] == gen.E4M3 else ""),
             "step": "dense index + proxy reduce + proxy scan + Reuse + Refine, all L queries",
-            "parallelism": f"replicas{dist_env()[2]}",
+            "parallelism": (f"zigzag{dist_env()[2]}: one sequence's query rows in 2N group "
+                            "blocks, rank r takes blocks r and 2N-1-r; keys replicated"
+                            if dist_env()[2] > 1 else "1 GPU, whole sequence"),
             "l2": "no flush: inputs and score buffers larger than L2 (q alone 1 GiB)"}
 
 
 def scan_traffic_per_pair():
-    """DRAM bytes per causal pair of the scan kernel from its committed ncu
-    summary, or None once the kernel sources differ from the captured ones."""
+    """DRAM bytes per causal pair of the scan kernel (SCAN_TRAFFIC), or None
+    once the kernel sources differ from the ones it was measured on."""
     import hashlib
-    import re
-    prof = os.path.join(ROOT, "profiles", "index_umma_dense_fp8_L16384.md")
-    try:
-        text = open(prof).read()
-    except OSError:
+    bpp = SCAN_TRAFFIC.get("bytes_per_pair")
+    if bpp is None or not SCAN_TRAFFIC.get("sources"):
         return None
-    m = re.search(r"traffic_bytes_per_pair=([0-9.]+) sources=(\S+)", text)
-    if not m:
-        return None
-    for item in m.group(2).split(","):
-        name, digest = item.split(":")
+    for name, digest in SCAN_TRAFFIC["sources"].items():
         src = os.path.join(ROOT, "top_token_selection_b200", "csrc", name)
-        if hashlib.sha1(open(src, "rb").read()).hexdigest()[:len(digest)] != digest:
+        try:
+            data = open(src, "rb").read()
+        except OSError:
             return None
-    return float(m.group(1))
+        if hashlib.sha1(data).hexdigest()[:len(digest)] != digest:
+            return None
+    return float(bpp)
+
+
+def measure_fp8_peak(device, n=8192, sustain_s=3.0):
+    """Dense FP8 (e4m3 x e4m3, fp32 accumulate, bf16 out) tensor throughput
+    of the library GEMM, torch._scaled_mm at n^3: best of 10 (burst) and
+    back to back for `sustain_s` seconds (sustained, the figure for kernels
+    timed inside a long step).  TFLOP/s."""
+    g = torch.Generator(device=device).manual_seed(0)
+    a = (torch.randn(n, n, device=device, generator=g) * 0.5).to(torch.float8_e4m3fn)
+    b = (torch.randn(n, n, device=device, generator=g) * 0.5).to(torch.float8_e4m3fn).t()
+    one = torch.tensor(1.0, device=device)
+
+    def mm():
+        return torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    for _ in range(3):
+        mm()
+    torch.cuda.synchronize()
+    flop = 2.0 * n ** 3
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    iters = max(10, int(sustain_s / (best * 1e-3)))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        mm()
+    e1.record()
+    torch.cuda.synchronize()
+    return {"burst": flop / (best * 1e-3) / 1e12,
+            "sustained": flop * iters / (e0.elapsed_time(e1) * 1e-3) / 1e12,
+            "how": f"torch._scaled_mm e4m3 {n}^3 (2 n^3 flop): best of 10, and {iters} back to "
+                   f"back (~{sustain_s:.0f} s), CUDA events"}
 
 
 def _event_ms(fn, stream, reps):
@@ -519,6 +598,64 @@ def measure_extra(run, wl, device, peaks, seed, reps=3):
     return out
 
 
+def time_modes(run, steps=3):
+    """Per-stage CUDA-event times of `steps` warm steps of `run`: dense,
+    Reuse (reduce + scan + Reuse) and Refine (reduce + scan + Refine)."""
+    run.step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    for e in ev:
+        run.step(e)
+    torch.cuda.synchronize()
+    st = np.zeros(5)
+    for e in ev:
+        for j in range(5):
+            st[j] += e[j].elapsed_time(e[j + 1])
+    dense, red, scan, reu, ref = st / steps
+    L = run.rows
+    out = {"dense": {"ms": dense, "queries_per_s": L / (dense / 1e3)},
+           "reuse": {"ms": red + scan + reu, "queries_per_s": L / ((red + scan + reu) / 1e3),
+                     "speedup_vs_dense": dense / (red + scan + reu)},
+           "refine": {"ms": red + scan + ref, "queries_per_s": L / ((red + scan + ref) / 1e3),
+                      "speedup_vs_dense": dense / (red + scan + ref)},
+           "stages_ms": {"dense": dense, "proxy_reduce": red, "proxy_scan": scan,
+                         "reuse": reu, "refine": ref}}
+    return out
+
+
+def measure_workloads(args, device, peaks, fp8_peak):
+    """The other prefill workloads, each timed on its own (not in `value`):
+    dsa_prefill_16k (bf16, g = 8, C = 4096) and dsa_prefill_64k (bf16) at
+    g in {8, 16} x C in {4096, 8192}; per mode queries/s and speedup over
+    dense, the scan's tensor throughput, and Reuse / Refine recall."""
+    from top_token_selection_b200 import pivot as pv
+    out = {}
+    points = [("dsa_prefill_16k", 8, 4096)] + [("dsa_prefill_64k", g, C)
+                                              for g in (8, 16) for C in (4096, 8192)]
+    made = {}
+    for name, g, C in points:
+        wl = dict(gen.WORKLOADS[name], g=g, C=C)
+        if name not in made:
+            made.clear()
+            made[name] = make_inputs(wl, args.seed)
+        run = Runner(made[name], wl, device)
+        pv.pivot_profile_enable(1)
+        res = time_modes(run)
+        pv.pivot_profile_enable(0)
+        n, kms, work = pv.profile_read(0)     # scan: dense + proxy rows of the timed steps
+        res["scan_tflops"] = work * 2.0 * run.H * run.D / (kms / 1e3) / 1e12 if kms else None
+        res["recall"] = {"reuse_vs_dense": recall_stats(run.dense, run.reu),
+                         "refine_vs_dense": recall_stats(run.dense, run.ref),
+                         "dense_neighbour_overlap": neighbour_overlap(run.dense)}
+        res.update({"L": wl["L"], "dtype": gen.DTYPE_NAMES[wl["dtype"]], "g": g, "C": C,
+                    "topk": wl["topk"]})
+        out[f"{name}_g{g}_C{C}"] = res
+        del run
+        torch.cuda.empty_cache()
+    assert pv.device_error() == 0, "a kernel reported an error in the workload sweep"
+    return out
+
+
 def run_ours(args, wl):
     import torch.distributed as dist
     rank, local_rank, world = dist_env()
@@ -527,9 +664,13 @@ def run_ours(args, wl):
     if world > 1 and not dist.is_initialized():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=device)
-    p = make_inputs(wl, rank_seed(args.seed, rank))
-    run = Runner(p, wl, device)
+    # one sequence for the whole job: every rank builds the same inputs (the
+    # keys are needed whole) and indexes its own zig-zag row ranges
+    p = make_inputs(wl, args.seed)
+    run = Runner(p, wl, device, rank_rows(wl["L"], wl["g"], world, rank))
     pv = run.pv
+    fp8 = wl["dtype"] == gen.E4M3
+    fp8_peak = measure_fp8_peak(device) if fp8 else None
 
     def barrier():
         if world > 1:
@@ -589,9 +730,12 @@ def run_ours(args, wl):
     for v in kern.values():
         v["share"] = v["ms"] / total_k
     flop_pair = 2.0 * run.H * run.D
-    fp8 = wl["dtype"] == gen.E4M3
-    tc_peak_burst = peaks["bf16_tflops"] * (FP8_OVER_BF16 if fp8 else 1.0)
-    tc_peak = peaks["bf16_tflops_sustained"] * (FP8_OVER_BF16 if fp8 else 1.0)
+    if fp8:   # the measured FP8 GEMM figures of this GPU
+        tc_peak_burst, tc_peak = fp8_peak["burst"], fp8_peak["sustained"]
+        tc_src = "measured fp8 sustained (" + fp8_peak["how"] + ")"
+    else:
+        tc_peak_burst, tc_peak = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+        tc_src = f"{peak_src} bf16 sustained"
     for name in ("scan", "refine"):
         v = kern[name]
         if v["ms"] > 0:
@@ -618,9 +762,10 @@ def run_ours(args, wl):
                 "traffic_source": None if bpp is None else
                     "ncu dram bytes of the dense scan at L=16384 (profiles/), per causal pair, "
                     "times this run's pairs per launch",
-                "peak_source": f"{peak_src} bf16 sustained x {FP8_OVER_BF16 if fp8 else 1.0} "
-                               f"({'fp8' if fp8 else 'bf16'} nominal ratio)",
+                "peak_source": tc_src,
                 "frac_of_burst": ach / tc_peak_burst,
+                "frac_of_nominal_x2_bf16": ach / (peaks["bf16_tflops_sustained"] *
+                                                  (FP8_OVER_BF16 if fp8 else 1.0)),
                 "per_launch": {"work_pairs": dv["work"] / max(dv["launches"], 1),
                                "ms": dv["ms"] / max(dv["launches"], 1)}}
     else:
@@ -630,10 +775,30 @@ def run_ours(args, wl):
                 "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
                 "peak_source": f"{peak_src} hbm"}
 
-    # quality
-    rec = {"reuse_vs_dense": recall_stats(run.dense, run.reu),
-           "refine_vs_dense": recall_stats(run.dense, run.ref),
-           "dense_neighbour_overlap": neighbour_overlap(run.dense)}
+    # Refine + its top-k against HBM (algorithmic bytes: every group's C
+    # candidate keys and scales gathered once, the members' queries and
+    # weights read, the candidate rows read, the index rows written) and
+    # against the tensor peak (member-candidate pairs x 2 H D)
+    esz = {gen.F32: 4, gen.BF16: 2, gen.E4M3: 1}[wl["dtype"]]
+    key_b = run.D * esz + (4 if fp8 else 0)
+    groups = sum(-(-b // run.g) - a // run.g for a, b in run.ranges)
+    gather = sum(min(run.C, min(run.L, (j + 1) * run.g)) for a, b in run.ranges
+                 for j in range(a // run.g, -(-b // run.g)))
+    ref_bytes = (gather * key_b + run.rows * (run.H * run.D * esz + run.H * 4 + 4)
+                 + groups * run.C * 4 + run.rows * run.k * 4)
+    ref_pairs = kern["refine"]["work"] / max(args.steps, 1)
+    modes["refine_stage"] = {
+        "ms": ref_ms, "algorithmic_bytes": ref_bytes,
+        "gbs": ref_bytes / (ref_ms / 1e3) / 1e9,
+        "frac_hbm": ref_bytes / (ref_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "tflops": ref_pairs * flop_pair / (ref_ms / 1e3) / 1e12,
+        "frac_tensor": ref_pairs * flop_pair / (ref_ms / 1e3) / 1e12 / tc_peak}
+
+    # quality (this rank's rows)
+    rows_of = lambda t: torch.cat([t[a:b] for a, b in run.ranges])  # noqa: E731
+    rec = {"reuse_vs_dense": recall_stats(rows_of(run.dense), rows_of(run.reu)),
+           "refine_vs_dense": recall_stats(rows_of(run.dense), rows_of(run.ref)),
+           "dense_neighbour_overlap": neighbour_overlap(rows_of(run.dense))}
 
     # end to end through host buffers (pinned), every step's copies inside the
     # timed region: step i's inputs go up while step i - 1 computes (two
@@ -681,14 +846,15 @@ def run_ours(args, wl):
                 with torch.cuda.stream(d2h):
                     for o, dsrc, e in zip(outs, dev_out[b], (ev[1], ev[4], ev[5])):
                         d2h.wait_event(e)
-                        o.copy_(dsrc, non_blocking=True)
+                        for ra, rb in run.ranges:        # this rank's rows
+                            o[ra:rb].copy_(dsrc[ra:rb], non_blocking=True)
                 back[b] = mk()
                 back[b].record(d2h)
             comp.wait_stream(h2d)
             comp.wait_stream(d2h)
         pipelined(2)
         barrier()
-        k_e2e = max(1, min(args.steps, 3))
+        k_e2e = args.steps
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(run.stream)
         pipelined(k_e2e)
@@ -697,15 +863,20 @@ def run_ours(args, wl):
         e_ms = max_over_ranks(a.elapsed_time(b), device)
         # the host copies are the device results of the last step
         last = dev_out[(k_e2e - 1) % 2]
+        ra, rb = run.ranges[0]
         for o, dsrc in zip(outs, last):
-            assert torch.equal(o[:1024], dsrc[:1024].cpu()), "host indices differ from the device's"
-        e2e = {"value": aggregate_value(L, world, e_ms, k_e2e), "unit": "queries/s",
+            assert torch.equal(o[ra:ra + 1024], dsrc[ra:ra + 1024].cpu()), \
+                "host indices differ from the device's"
+        e2e = {"value": job_value(L, e_ms, k_e2e), "unit": "queries/s",
                "h2d_bytes_per_step": run.h2d_bytes(), "d2h_bytes_per_step": run.d2h_bytes(),
                "ms_per_step": e_ms / k_e2e, "steps": k_e2e,
                "overlap": "inputs of step i+1 uploaded during step i; each stage's indices "
                           "copied back during the later stages"}
 
-    extra = None if args.no_extra else measure_extra(run, wl, device, peaks, args.seed)
+    extra = None
+    if not args.no_extra and world == 1:
+        extra = measure_extra(run, wl, device, peaks, args.seed)
+        extra["workloads"] = measure_workloads(args, device, peaks, fp8_peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -713,14 +884,15 @@ def run_ours(args, wl):
         cpu = {"value": L / total, "unit": "queries/s", "cores": threads, "kind": "oracle",
                "sample": desc, "extrapolated_step_s": total, "parts_s": parts}
 
-    value = aggregate_value(L, world, ms_max, args.steps)
+    value = job_value(L, ms_max, args.steps)      # the whole sequence's queries
     line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
             "dtype": gen.DTYPE_NAMES[wl["dtype"]], "data": "synthetic",
             "config": config_of(wl, args), "modes": modes, "recall": rec,
             "roofline": roof, "kernels": kern, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": int(n1 - n0), "clocks": clk, "extra": extra}
+            "gpu_launches": int(n1 - n0), "clocks": clk, "fp8_peak_tflops": fp8_peak,
+            "extra": extra}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -34,19 +34,25 @@
  *    bfloat16.  PIVOT_E4M3: OCP FP8 e4m3 codes with one float32 scale per
  *    token (value = code * scale).  w is float32 in every dtype.
  *  - Selection keeps the k highest scores; equal scores are taken lower
- *    position first; -0 equals +0.  Output index rows list the selected
- *    positions in ascending order (the indexer hands on a set of positions;
- *    the indexer tutorial's Fig. 1 lists them by position), padded with -1
- *    when fewer positions are eligible.  Optional score outputs are float32,
- *    aligned with the positions, -inf padding.
+ *    position first; -0 equals +0.  Index rows are padded with -1 when
+ *    fewer positions are eligible.  The input struct's `order` field says
+ *    how a row lists its positions:
+ *      PIVOT_ORDER_POSITION (0, what a zero-initialised struct asks for):
+ *        ascending positions (the indexer hands on a set of positions; the
+ *        indexer tutorial's Fig. 1 lists them by position);
+ *      PIVOT_ORDER_RANK: rank order -- score descending, then position
+ *        ascending -- so the best k' < k are a row's first k' entries.
+ *    Optional score outputs are float32, aligned with the positions, -inf
+ *    padding.
  *  - Argument errors are found before anything is enqueued and return
  *    PIVOT_ERR_INVALID_ARG / _UNSUPPORTED / _WORKSPACE; a failed launch
  *    returns PIVOT_ERR_CUDA.  Faults found by the kernels themselves (a
  *    bounded wait that ran out, a bad cache length) set a per-device error
  *    word read by pivot_get_device_error().
  *  - FP8 and bf16 scoring runs on the tensor cores with fp32 accumulation;
- *    PIVOT_F32 inputs are consumed at TF32 precision by the tensor cores
- *    (exact for integer-valued inputs of magnitude < 2048).
+ *    PIVOT_F32 inputs are scored on the CUDA cores in full fp32 (the tensor
+ *    cores have no fp32 operand kind; their tf32 kind would drop 13 of the
+ *    24 significand bits).
  */
 #ifndef PIVOT_H
 #define PIVOT_H
@@ -73,6 +79,11 @@ typedef enum {
 typedef enum { PIVOT_F32 = 0, PIVOT_BF16 = 1, PIVOT_E4M3 = 2 } pivot_dtype_t;
 
 typedef enum {
+    PIVOT_ORDER_POSITION = 0,    /* index rows ascending by position (default)   */
+    PIVOT_ORDER_RANK = 1         /* score descending, then position ascending    */
+} pivot_order_t;
+
+typedef enum {
     PIVOT_MODE_DENSE = 0,        /* per-query full-prefix scan                   */
     PIVOT_MODE_REUSE = 1,        /* the proxy's top-k shared by the group        */
     PIVOT_MODE_REFINE = 2        /* candidates re-scored per member              */
@@ -92,6 +103,7 @@ typedef struct {
     const void* k;               /* [L, D] one shared indexer key per token      */
     const float* k_scale;        /* [L] for PIVOT_E4M3, else NULL                */
     int32_t t_begin, t_end;      /* query rows of this call                      */
+    int32_t order;               /* pivot_order_t of the index rows written      */
 } pivot_seq_t;
 
 /* One MTP decode step over a batch of cached sequences.  cache_len[b]
@@ -108,6 +120,7 @@ typedef struct {
     const void* kc;              /* [B, maxlen, D]                               */
     const float* kc_scale;       /* [B, maxlen] for PIVOT_E4M3, else NULL        */
     const int32_t* cache_len;    /* [B] on the device, Gm <= cache_len <= maxlen */
+    int32_t order;               /* pivot_order_t of the index rows written      */
 } pivot_decode_t;
 
 /* A batch of prefill sequences packed row after row, the layout of ragged
@@ -125,6 +138,7 @@ typedef struct {
     const float* w;              /* [total, H]                                   */
     const void* k;               /* [total, D]                                   */
     const float* k_scale;        /* [total] for PIVOT_E4M3, else NULL            */
+    int32_t order;               /* pivot_order_t of the index rows written      */
 } pivot_varlen_t;
 
 /* Dense indexer (Fig. 1-2 of the indexer tutorial; the baseline the PIVOT
@@ -151,10 +165,11 @@ pivot_status_t pivot_proxy_reduce(const pivot_seq_t* seq, int32_t g, void* pq,
 
 /* One full-prefix scan per group (PIVOT abstract): proxy j scores keys
  * [0, e_j], e_j = min(L, (j+1)*g) - 1, with the dense score formula and
- * keeps its top-C.  cand [G, C] int32: the proxy's top-`topk` positions
- * (ascending), then the rest of its top-C (ascending) -- so the first topk
- * entries are what PIVOT-Reuse shares.  cand_score [G, C] or NULL.
- * 1 <= topk <= C <= 8192. */
+ * keeps its top-C.  cand [G, C] int32: with PIVOT_ORDER_POSITION the
+ * proxy's top-`topk` positions (ascending), then the rest of its top-C
+ * (ascending); with PIVOT_ORDER_RANK the whole top-C in rank order.  Either
+ * way the first topk entries are what PIVOT-Reuse shares.  cand_score
+ * [G, C] or NULL.  1 <= topk <= C <= 8192. */
 pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* pq,
                                  const float* pq_scale, const float* pw, int32_t C,
                                  int32_t topk, int32_t* cand, float* cand_score, void* ws,
@@ -163,7 +178,7 @@ size_t pivot_proxy_scan_workspace_size(const pivot_seq_t* seq, int32_t g, int32_
 
 /* PIVOT-Reuse (PIVOT abstract): member t of group j takes the first topk
  * entries of cand[j] (the proxy's top-k), keeps those <= t in their order
- * (ascending) and pads with -1.
+ * (the order pivot_proxy_scan wrote them in) and pads with -1.
  * Rows [t_begin, t_end) with t_begin a multiple of g; cand rows relative to
  * t_begin / g.  idx [rows, topk].  1 <= topk <= C. */
 pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int32_t* cand,
@@ -175,8 +190,9 @@ pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int3
  * reading refills the masked slots with the next proxy-ranked candidates:
  * member t of group j takes, among the entries of cand[j] at positions <= t,
  * the topk with the highest cand_score[j] (lower position first on equal
- * scores), listed in ascending position, -1 padded.  Where nothing of the
- * proxy's top-k is masked this is exactly pivot_reuse.
+ * scores), listed in ascending position (whatever the candidates' order),
+ * -1 padded.  Where nothing of the proxy's top-k is masked this is exactly
+ * pivot_reuse on position-ordered candidates.
  * cand, cand_score [G, C] device (rows relative to t_begin / g), as written
  * by pivot_proxy_scan; rows [t_begin, t_end), t_begin a multiple of g;
  * idx [rows, topk] device.  1 <= topk <= C <= 8192.  No workspace. */
@@ -229,10 +245,12 @@ size_t pivot_index_window_outside_workspace_size(const pivot_seq_t* seq, int32_t
  * variant where the window lies inside the indexer's candidates: row r's
  * output is its entries of idx below t - window + 1, then every position of
  * [max(0, t - window + 1), t], ascending, -1 padded.
- * idx [rows, topk] device, each row ascending with -1 padding (the layout
+ * idx [rows, topk] device, each row -1 padded (the layout
  * every index entry point writes); t = positions[r] (device [rows]) or,
  * when positions is NULL, t_begin + r; out [rows, topk + window] device.
- * window >= 1.  Rows whose t is negative come out all -1. */
+ * window >= 1.  Rows whose t is negative come out all -1.  The entries kept
+ * from idx stay in their order, so rank-ordered rows stay rank-ordered
+ * ahead of the window. */
 pivot_status_t pivot_window_union(const int32_t* idx, int32_t rows, int32_t topk, int32_t t_begin,
                                   const int32_t* positions, int32_t window, int32_t* out,
                                   void* stream);
@@ -257,6 +275,21 @@ pivot_status_t pivot_decode(const pivot_decode_t* batch, int32_t mode, int32_t C
 size_t pivot_decode_workspace_size(const pivot_decode_t* batch, int32_t mode, int32_t C,
                                    int32_t topk);
 
+/* The workspace, in bytes, of one whole indexer pass of `mode`, from sizes
+ * alone (no buffers needed): the largest that any call of the mode's chain
+ * asks for -- pivot_dense_index for PIVOT_MODE_DENSE; pivot_proxy_scan for
+ * PIVOT_MODE_REUSE (reduce and Reuse need none); the larger of
+ * pivot_proxy_scan and pivot_refine for PIVOT_MODE_REFINE.
+ *   B == 0: one prefill sequence of L_or_maxlen tokens, groups of g, all
+ *           rows in one call;
+ *   B >= 1: one MTP decode step (pivot_decode) of B sequences with key
+ *           caches of L_or_maxlen positions and g = Gm tokens per step.
+ * dtype is a pivot_dtype_t; H, D, C, topk as for the calls themselves
+ * (C unused in dense prefill).  Returns 0 for arguments the calls would
+ * refuse.  The caller's own buffers (pq, pw, cand, idx) are not included. */
+size_t pivot_workspace_size(int32_t mode, int32_t dtype, int32_t L_or_maxlen, int32_t B,
+                            int32_t H, int32_t D, int32_t g, int32_t C, int32_t topk);
+
 /* pivot_decode without a caller workspace, for callers that cannot allocate
  * device memory at the call site -- e.g. a plugin inside an inference engine
  * whose memory planner owns the whole device, or a per-token decode loop
@@ -264,16 +297,21 @@ size_t pivot_decode_workspace_size(const pivot_decode_t* batch, int32_t mode, in
  * counterpart on the pages; it is a packaging of pivot_decode.
  *
  * Arguments and results are those of pivot_decode (inputs and outputs are
- * still the caller's device buffers).  The scratch space is a fixed 64 MiB
- * array inside the library, one per device, held from when the library is
- * loaded until the process exits; the call allocates nothing.  A batch
- * whose pivot_decode_workspace_size() exceeds 64 MiB is rejected with
- * PIVOT_ERR_WORKSPACE before anything is enqueued.  The first call on each
- * device looks up that device's array address (with the device current);
- * make that first call before any stream capture.  Every call on a device
- * uses the same array and leaves its contents behind: calls that can
- * overlap on the GPU (different streams without ordering) race on it and
- * must be serialised by the caller. */
+ * still the caller's device buffers), and the argument checks are the same,
+ * so both return the same status for the same arguments.  The scratch
+ * space is a fixed 64 MiB array inside the library, one per device: with
+ * CUDA's default lazy module loading it is reserved on a device by the
+ * first call there (under CUDA_MODULE_LOADING=EAGER, when the library is
+ * loaded) and held until the process exits; the call itself allocates
+ * nothing.  A batch whose pivot_decode_workspace_size() exceeds 64 MiB is
+ * rejected with PIVOT_ERR_WORKSPACE before anything is enqueued.  Each call
+ * made outside stream capture looks up the array's address on the current
+ * device; a call made while `stream` is being captured reuses the address
+ * the last uncaptured call on that device found, so make one call on each
+ * device before capturing, and again after a device reset (which moves the
+ * array).  Every call on a device uses the same array and leaves its
+ * contents behind: calls that can overlap on the GPU (different streams
+ * without ordering) race on it and must be serialised by the caller. */
 pivot_status_t pivot_decode_noalloc(const pivot_decode_t* batch, int32_t mode, int32_t C,
                                     int32_t topk, int32_t* idx, int32_t* cand, void* stream);
 

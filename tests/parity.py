@@ -1,7 +1,8 @@
 """Shared helpers of the GPU parity tests: move seeded inputs to the device,
 run the library through its C ABI, compare with the oracle.
 
-Comparison rules (the indexer returns positions in rank order):
+Comparison rules (index rows list the selected positions in ascending
+order unless rank order is asked for):
 * integer-valued inputs: every score is exact in fp32 and fp64, so index
   rows must be identical, order and -1 padding included;
 * real-valued inputs: GPU scores accumulate in fp32 (tensor cores) while the
@@ -43,11 +44,8 @@ def assert_rows_exact(gpu, ref, what=""):
                              f"gpu {gpu[r][:16]} ref {ref[r][:16]}")
 
 
-def assert_rows_close(gpu_idx, ref_idx, ref_scores, score_fn, rows, what="", gpu_scores=None,
-                      abs_tol=None):
-    """Boundary-tolerant set comparison, row by row (see module doc).
-    `abs_tol(row)`, when given, replaces the relative tolerance by an
-    absolute bound derived for that row's arithmetic."""
+def assert_rows_close(gpu_idx, ref_idx, ref_scores, score_fn, rows, what="", gpu_scores=None):
+    """Boundary-tolerant set comparison, row by row (see module doc)."""
     gpu_idx = np.asarray(gpu_idx)
     ref_idx = np.asarray(ref_idx)
     nbad = 0
@@ -58,7 +56,7 @@ def assert_rows_close(gpu_idx, ref_idx, ref_scores, score_fn, rows, what="", gpu
         if not o:
             continue
         sk = float(np.min(ref_scores[i][:len(o)]))     # the k-th score: rows are listed by position
-        tol = REL_TOL * max(abs(sk), 1e-30) if abs_tol is None else abs_tol(r)
+        tol = REL_TOL * max(abs(sk), 1e-30)
         gs, os_ = set(g), set(o)
         only_g = sorted(gs - os_)
         only_o = sorted(os_ - gs)
@@ -78,22 +76,6 @@ def assert_rows_close(gpu_idx, ref_idx, ref_scores, score_fn, rows, what="", gpu
             err = np.abs(gsc - want).max()
             assert err <= tol, f"{what} row {r}: score error {err} > {tol}"
     return nbad
-
-
-def tf32_abs_tol(pq, pw, k):
-    """Error bound of one score when the tensor cores consume fp32 operands
-    at TF32 (10 explicit mantissa bits; truncation at worst): each product
-    q*k is off by at most 2^-9 |q||k| relative, plus fp32 accumulation, so
-    |err| <= 2^-8 * sum_h |w_h| sum_d |q_hd| |k_d|.  Returns a per-row bound
-    (max over the row's keys)."""
-    aq = np.abs(pq.astype(np.float64))                 # [G, H, D]
-    ak = np.abs(k.astype(np.float64))                  # [L, D]
-    bound = np.einsum("gh,ghd->gd", np.abs(pw.astype(np.float64)), aq) @ ak.T   # [G, L]
-    per_row = bound.max(axis=1) * 2.0 ** -8
-
-    def fn(j):
-        return per_row[j]
-    return fn
 
 
 def oracle_codes(p):

@@ -224,3 +224,44 @@ def test_ragged_batch_workspace_layout(lib):
     # H = 2 is not a tensor-core shape: the sequence-by-sequence layout
     seq_path = pv.pivot_index_varlen_workspace_size(batch(2, 64, pv.F32), 0, g, C, k)
     assert 0 < seq_path < T * (stride * 4 + 4)
+
+
+def test_one_workspace_size_for_a_whole_pass(lib):
+    """pivot_workspace_size from sizes alone equals the largest per-call
+    workspace of the mode's chain (prefill with B = 0, decode with B >= 1)."""
+    for dt, D, scale in ((pv.F32, 32, None), (pv.E4M3, 128, FAKE), (pv.BF16, 128, None)):
+        H = 4 if dt == pv.F32 else 64
+        seq = _seq(dtype=dt, L=5000, H=H, D=D, q_scale=scale, k_scale=scale)
+        dense = pv.pivot_dense_index_workspace_size(seq, 256)
+        scan = pv.pivot_proxy_scan_workspace_size(seq, 8, 1024)
+        ref = pv.pivot_refine_workspace_size(seq, 8, 1024, 256)
+        assert pv.pivot_workspace_size(pv.DENSE, dt, 5000, 0, H, D, 8, 1024, 256) == dense
+        assert pv.pivot_workspace_size(pv.REUSE, dt, 5000, 0, H, D, 8, 1024, 256) == scan
+        assert pv.pivot_workspace_size(pv.REFINE, dt, 5000, 0, H, D, 8, 1024, 256) == max(scan, ref)
+    dec = pv.PivotDecode(pv.E4M3, 4, 2, 64, 128, 4096, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    for mode in (pv.DENSE, pv.REUSE, pv.REFINE):
+        assert pv.pivot_workspace_size(mode, pv.E4M3, 4096, 4, 64, 128, 2, 256, 64) == \
+            pv.pivot_decode_workspace_size(dec, mode, 256, 64)
+    # arguments the calls refuse give 0
+    assert pv.pivot_workspace_size(3, pv.F32, 5000, 0, 4, 32, 8, 1024, 256) == 0
+    assert pv.pivot_workspace_size(pv.REUSE, pv.F32, 5000, 0, 4, 32, 8, 100, 256) == 0   # C < k
+    assert pv.pivot_workspace_size(pv.DENSE, 9, 5000, 0, 4, 32, 8, 1024, 256) == 0
+
+
+def test_output_order_field_is_validated(lib):
+    """order is PIVOT_ORDER_POSITION (0) or PIVOT_ORDER_RANK (1); anything
+    else is an invalid argument for every call that reads it."""
+    for order in (2, -1):
+        seq = _seq(order=order)
+        assert pv.pivot_dense_index(seq, 8, FAKE, None, FAKE, 1 << 20, None) == 1
+        assert pv.pivot_proxy_scan(seq, 4, FAKE, None, FAKE, 16, 8, FAKE, None, FAKE, 1 << 20,
+                                   None) == 1
+        assert pv.pivot_refine(seq, 4, FAKE, 16, 8, FAKE, None, FAKE, 1 << 20, None) == 1
+        dec = pv.PivotDecode(pv.E4M3, 4, 2, 64, 128, 4096, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                             order)
+        assert pv.pivot_decode(dec, pv.DENSE, 0, 64, FAKE, None, FAKE, 1 << 20, None) == 1
+        cu = (ctypes.c_int32 * 2)(0, 64)
+        vb = pv.PivotVarlen(pv.F32, 1, 4, 32, ctypes.addressof(cu), FAKE, None, FAKE, FAKE, None,
+                            order)
+        assert pv.pivot_index_varlen(vb, pv.DENSE, 4, 16, 8, FAKE, FAKE, 1 << 20, None) == 1
+    assert pv.pivot_dense_index_workspace_size(_seq(order=pv.ORDER_RANK), 8) > 0

@@ -25,7 +25,7 @@ def tiny():
 
 @pytest.mark.parametrize("g,C,kk", [(4, 256, 64), (8, 100, 37), (1, 64, 64), (2, 40, 9)])
 def test_reuse_backfill_exact(tiny, g, C, kk):
-    """Power-of-two member counts keep the integer proxy exact at TF32, so
+    """Power-of-two member counts keep the integer proxy dyadic (exact fp32 scores), so
     candidates and proxy scores are the oracle's bit for bit."""
     p, dev, _ = tiny
     seq = seq_of(dev)

@@ -13,7 +13,7 @@ from top_token_selection_b200 import inputs as gen
 from top_token_selection_b200 import pivot as pv
 
 from parity import (assert_rows_close, assert_rows_exact, proxy_score_fn, score_fn_for, seq_of,
-                    tf32_abs_tol, to_device)
+                    to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -122,7 +122,8 @@ def test_tiny_invariants_on_gpu(tiny):
 ])
 def test_edge_shapes_exact(L, g, C, kk):
     """Every group has a power-of-two member count, so the proxy mean of
-    integers is exact at TF32 and every comparison is bit for bit."""
+    integers is dyadic, every fp32 score is exact and every comparison is
+    bit for bit."""
     p = gen.make_prefill(L, 4, 32, F32, kind="int", seed=L)
     dev = to_device(p)
     q, qs, w, k, ks = p.codes()
@@ -180,10 +181,10 @@ def test_dsa_long_rows_within_tolerance(dtype):
 
 @pytest.mark.parametrize("L,g,C,kk", [(300, 5, 64, 64), (515, 3, 40, 9)])
 def test_edge_shapes_odd_groups(L, g, C, kk):
-    """g not a power of two: the proxy mean is not dyadic and the tensor
-    cores consume fp32 at TF32, so candidates compare within the TF32 error
-    bound; Reuse and Refine on the GPU's own candidates stay exact (members'
-    own integer queries)."""
+    """g not a power of two: the proxy mean of integers is not dyadic, so
+    proxy scores are fp32 sums of non-integers; the candidates compare
+    within the relative tolerance, and Reuse and Refine on the GPU's own
+    candidates stay exact (members' own integer queries)."""
     p = gen.make_prefill(L, 4, 32, F32, kind="int", seed=L + 1)
     dev = to_device(p)
     q, qs, w, k, ks = p.codes()
@@ -193,10 +194,38 @@ def test_edge_shapes_odd_groups(L, g, C, kk):
     groups = np.arange(opq.shape[0])
     ocand, ocs = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, L, g, C, kk)
     assert_rows_close(cand.cpu().numpy(), ocand, ocs, proxy_score_fn(p, opq, opqs, opw), groups,
-                      "cand", gpu_scores=cs.cpu().numpy(), abs_tol=tf32_abs_tol(opq, opw, k))
+                      "cand", gpu_scores=cs.cpu().numpy())
     gc = cand.cpu().numpy()
     assert_rows_exact(reu.cpu(), oracle.reuse(L, g, gc, kk), "reuse")
     assert_rows_exact(ref.cpu(), oracle.refine(F32, q, qs, w, k, ks, g, gc, kk)[0], "refine")
+
+
+def test_f32_real_valued_within_tolerance():
+    """Real-valued fp32 inputs (the DSA-shaped generator kept in fp32): the
+    fp32 scores meet the relative tolerance against the fp64 oracle for
+    dense, the proxy scan and Refine."""
+    L, H, D, g, C, kk = 700, 4, 32, 4, 256, 64
+    p = gen.make_prefill(L, H, D, F32, kind="dsa", seed=31)
+    dev = to_device(p)
+    q, qs, w, k, ks = p.codes()
+    rows = np.array(sorted(set(np.linspace(0, L - 1, 40).astype(int)) | {L - 1}))
+    idx, sc = pv.dense_index(seq_of(dev), kk, with_score=True)
+    oidx, osc = oracle.dense_index(F32, q, qs, w, k, ks, kk, rows=rows)
+    fn = score_fn_for(p)
+    assert_rows_close(idx.cpu().numpy()[rows], oidx, osc, fn, rows, "dense",
+                      gpu_scores=sc.cpu().numpy()[rows])
+    pq, pqs, pw, cand, cs, reu, ref, rs = _pivot_gpu(p, dev, g, C, kk)
+    opq, opqs, opw = oracle.proxy_reduce(F32, q, qs, w, g)
+    assert (pq.cpu().numpy() == opq).all() and (pw.cpu().numpy() == opw).all()
+    groups = np.arange(opq.shape[0])
+    ocand, ocs = oracle.proxy_scan(F32, opq, opqs, opw, k, ks, L, g, C, kk)
+    assert_rows_close(cand.cpu().numpy(), ocand, ocs, proxy_score_fn(p, opq, opqs, opw), groups,
+                      "cand", gpu_scores=cs.cpu().numpy())
+    gc = cand.cpu().numpy()
+    assert_rows_exact(reu.cpu(), oracle.reuse(L, g, gc, kk), "reuse")
+    oref, ors = oracle.refine(F32, q, qs, w, k, ks, g, gc, kk, rows=rows)
+    assert_rows_close(ref.cpu().numpy()[rows], oref, ors, fn, rows, "refine",
+                      gpu_scores=rs.cpu().numpy()[rows])
 
 
 def test_row_ranges_and_small_workspace_match_one_call(tiny):

@@ -1,8 +1,9 @@
 """The N > 1 host logic on CPU: world-size-2 gloo process groups.
 
 Covers the row sharding of one sequence across ranks (ranges cover every
-query once, causal work balanced) and the benchmark's rank plumbing (seeds
-differ per rank, timings reduce to the max over ranks, whole-job value)."""
+query once, causal work balanced) and the benchmark's rank plumbing (each
+rank's rows are its zig-zag ranges of the one sequence, timings reduce to
+the max over ranks, whole-job value)."""
 import os
 import socket
 
@@ -32,9 +33,9 @@ def _worker(rank, world, port, L, g, q):
         dist.all_gather_object(gathered, mine)
         t_mine = 10.0 + 5.0 * rank
         t_max = bench.max_over_ranks(t_mine)
-        seeds = [None] * world
-        dist.all_gather_object(seeds, bench.rank_seed(0, rank))
-        q.put((rank, gathered, t_max, seeds, bench.dist_env()))
+        rows = [None] * world
+        dist.all_gather_object(rows, bench.rank_rows(L, g, world, rank))
+        q.put((rank, gathered, t_max, rows, bench.dist_env()))
     finally:
         dist.destroy_process_group()
 
@@ -64,14 +65,15 @@ def test_two_rank_sharding_and_timing(L, g):
         w = [causal_work(r) for r in gathered]
         assert max(w) / min(w) < 1.05                          # balanced causal work
     assert res[0][2] == res[1][2] == 15.0                      # max over ranks
-    assert res[0][3][0] != res[0][3][1]                        # independent replicas
+    assert res[0][3] == gathered                               # the bench's rows are these
     assert res[0][4] == (0, 0, 2) and res[1][4] == (1, 1, 2)
 
 
-def test_aggregate_value_is_whole_job():
+def test_job_value_is_whole_job():
     import bench
-    # 2 ranks x 131072 queries x 5 steps in 1000 ms (slowest rank)
-    assert bench.aggregate_value(131072, 2, 1000.0, 5) == pytest.approx(2 * 131072 * 5)
+    # one sequence of 131072 queries x 5 steps in 1000 ms (slowest rank)
+    assert bench.job_value(131072, 1000.0, 5) == pytest.approx(131072 * 5)
+    assert bench.rank_rows(1000, 8, 1, 0) == [(0, 1000)]
 
 
 def test_single_rank_ranges_are_the_whole_sequence():

@@ -272,22 +272,87 @@ def test_proxy_integer_mean_is_exact_and_partial_group_uses_member_count():
         assert (pw[j] == w[a:b].astype(np.float64).mean(axis=0)).all()
 
 
-def test_proxy_e4m3_requantisation():
-    p = gen.make_prefill(64, 4, 16, E4M3, kind="dsa", seed=12)
+def _f32_nearest(fr):
+    """The float32 nearest to the exact rational `fr`, ties to even: an
+    IEEE-754 correctly rounded division, computed without float division
+    (exact Fraction comparisons among the float32 neighbours)."""
+    from fractions import Fraction
+    f = np.float32(float(fr))
+    cands = [np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))]
+    best = min(abs(Fraction(float(c)) - fr) for c in cands)
+    near = [c for c in cands if abs(Fraction(float(c)) - fr) == best]
+    if len(near) > 1:
+        near = [c for c in near if (np.array(c).view(np.uint32) & 1) == 0]
+    return np.float32(near[0])
+
+
+@pytest.mark.parametrize("dtype", [F32, BF16])
+@pytest.mark.parametrize("g", [3, 5, 7])
+def test_proxy_odd_group_mean_is_the_correctly_rounded_quotient(dtype, g):
+    """Integer inputs make every member sum exact; the proxy is then that sum
+    divided by the member count and rounded once to fp32 (the IEEE divide),
+    for full and partial groups.  A reciprocal multiply (sum * (1/n)) rounds
+    twice and differs on some of these values, so this pins the divide."""
+    from fractions import Fraction
+    L = 23
+    p = gen.make_prefill(L, 3, 8, dtype, kind="int", seed=40 + g)
+    q, _, w, _, _ = p.codes()
+    pq, _, pw = oracle.proxy_reduce(dtype, q, None, w, g)
+    qv = q.astype(np.float64) if dtype == F32 else oracle.bf16_to_float(q).astype(np.float64)
+    recip_differs = False
+    for j in range(-(-L // g)):
+        a, b = j * g, min(L, (j + 1) * g)
+        n = b - a
+        sq = qv[a:b].sum(axis=0)           # exact: small integers
+        sw = w[a:b].astype(np.float64).sum(axis=0)
+        want_q = np.array([_f32_nearest(Fraction(int(x), n)) for x in sq.ravel()],
+                          dtype=np.float32).reshape(sq.shape)
+        want_w = np.array([_f32_nearest(Fraction(int(x), n)) for x in sw], dtype=np.float32)
+        if dtype == F32:
+            got_q = pq[j]
+        else:   # stored bf16: the fp32 quotient rounded to nearest even by torch's cast
+            got_q = pq[j]
+            want_q = torch.from_numpy(want_q).to(torch.bfloat16).view(torch.int16).numpy()
+            got_q = got_q.view(np.int16)
+        assert (got_q == want_q).all(), (g, j)
+        assert (pw[j] == want_w).all(), (g, j)
+        recip = sq.astype(np.float32) * (np.float32(1) / np.float32(n))
+        if n > 1 and (recip != np.float32(sq) / np.float32(n)).any():
+            recip_differs = True
+    assert recip_differs or g == 1
+
+
+@pytest.mark.parametrize("g,L", [(8, 64), (3, 31), (5, 40)])
+def test_proxy_e4m3_requantisation(g, L):
+    """The FP8 proxy, recomputed with numpy float32 arithmetic and torch's
+    float8 cast (neither shares code with the oracle's C codec): each member
+    value = code * scale rounded to fp32, summed left to right in member
+    order in fp32, divided by the member count (IEEE); scale = amax / 448;
+    codes = the saturating round-to-nearest-even of mean / scale.  Every
+    code, scale and weight must match bit for bit."""
+    p = gen.make_prefill(L, 4, 16, E4M3, kind="dsa", seed=12 + g)
     q, qs, w, _, _ = p.codes()
-    g = 8
     pq, pqs, pw = oracle.proxy_reduce(E4M3, q, qs, w, g)
-    deq = oracle.e4m3_to_float(q) * qs[:, None, None]
-    for j in range(8):
-        mean = deq[j * g:(j + 1) * g].mean(axis=0)
-        amax = np.abs(mean).max()
-        assert abs(pqs[j] - amax / 448.0) <= 1e-6 * amax / 448.0
-        # codes are the saturating round-to-nearest-even of mean / scale
-        y = torch.from_numpy((mean / pqs[j]).astype(np.float32))
-        ref = y.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
-        mism = (pq[j] != ref)
-        # fp32 vs fp64 summation can move a value across a rounding midpoint
-        assert mism.mean() < 0.01
+    dq = torch.from_numpy(q.copy()).view(torch.float8_e4m3fn).float().numpy()   # exact decode
+    for j in range(-(-L // g)):
+        a, b = j * g, min(L, (j + 1) * g)
+        n = b - a
+        if n == 1:
+            assert (pq[j] == q[a]).all() and pqs[j] == qs[a]
+            continue
+        acc = dq[a] * np.float32(qs[a])
+        wacc = w[a].copy()
+        for m in range(a + 1, b):
+            acc = acc + dq[m] * np.float32(qs[m])
+            wacc = wacc + w[m]
+        mean = acc / np.float32(n)
+        amax = np.float32(np.abs(mean).max())
+        s = amax / np.float32(448.0) if amax > 0 else np.float32(1.0)
+        y = mean / s
+        ref = torch.from_numpy(y).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+        assert np.float32(pqs[j]) == s, (j, pqs[j], s)
+        assert (pq[j] == ref.numpy()).all(), (j, int((pq[j] != ref.numpy()).sum()))
+        assert (pw[j] == wacc / np.float32(n)).all()
         assert (pq[j] & 0x7F).max() == 0x7E            # the largest magnitude maps to 448
 
 

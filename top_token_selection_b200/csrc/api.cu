@@ -85,9 +85,12 @@ bool dtype_ok(int dt) { return dt == PIVOT_F32 || dt == PIVOT_BF16 || dt == PIVO
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// Tensor-core tiling: N = P*H <= 256 with H in {4..64}; key rows of 128 or
-// 256 bytes (two 128-byte swizzle atoms).
+// Tensor-core tiling: FP8 and bf16 codes (the tensor cores have no fp32
+// kind, and their tf32 kind keeps 10 mantissa bits, so PIVOT_F32 is scored
+// on the CUDA cores in full fp32); N = P*H <= 256 with H in {4..64}; key rows
+// of 128 or 256 bytes (two 128-byte swizzle atoms).
 bool umma_shape_ok(int H, int D, int dtype) {
+    if (dtype == PIVOT_F32) return false;
     const int rb = D * esize_of(dtype);
     return (H == 4 || H == 8 || H == 16 || H == 32 || H == 64) && (rb == 128 || rb == 256);
 }
@@ -97,8 +100,22 @@ bool simt_shape_ok(int H, int D) {
     return smem <= 200 * 1024;
 }
 
+bool order_ok(int order) { return order == PIVOT_ORDER_POSITION || order == PIVOT_ORDER_RANK; }
+
+// The output order of the entry point running on this host thread: set for
+// the duration of a call from its input struct, read by every selection
+// launch the call makes.
+thread_local int t_rank_order = 0;
+struct OrderScope {
+    int prev;
+    explicit OrderScope(int order) : prev(t_rank_order) {
+        t_rank_order = order == PIVOT_ORDER_RANK ? 1 : 0;
+    }
+    ~OrderScope() { t_rank_order = prev; }
+};
+
 pivot_status_t check_seq(const pivot_seq_t* s, int* t0, int* t1) {
-    if (!s || !dtype_ok(s->dtype)) return PIVOT_ERR_INVALID_ARG;
+    if (!s || !dtype_ok(s->dtype) || !order_ok(s->order)) return PIVOT_ERR_INVALID_ARG;
     if (s->L < 1 || s->H < 1 || s->D < 1) return PIVOT_ERR_INVALID_ARG;
     if (!s->q || !s->w || !s->k) return PIVOT_ERR_INVALID_ARG;
     const bool fp8 = s->dtype == PIVOT_E4M3;
@@ -263,6 +280,7 @@ pivot_status_t run_select_prefix(int scan_kind, int r0, int r1, int L, int g, in
     sp.out_score = out_score;
     sp.out_base = out_base;
     sp.tail_cap = TAIL_CAP;
+    sp.rank_order = t_rank_order;
     sp.thresh = thresh;
     if (thresh) {   // a launch of its own (no work of its own: the select's bytes count once)
         const pivot_status_t t = from_cuda(
@@ -306,6 +324,7 @@ pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int 
     sp.out_score = out_score;
     sp.out_base = out_base;
     sp.tail_cap = TAIL_CAP;
+    sp.rank_order = t_rank_order;
     return from_cuda(profiled(PK_SELECT, (double)(r1 - r0) * C, st,
                               [&] { return launch_select(sp, st); }));
 }
@@ -425,6 +444,11 @@ cudaError_t launch_wait_selftest(cudaStream_t stream) {
 
 }  // namespace pivot
 
+namespace pivot {
+pivot_status_t decode_check_args(const pivot_decode_t* b, int32_t mode, int32_t C, int32_t topk,
+                                 const int32_t* idx);
+}  // namespace pivot
+
 using namespace pivot;
 
 extern "C" {
@@ -522,6 +546,7 @@ static pivot_status_t dense_index_impl(const pivot_seq_t* seq, int32_t topk, int
 
 pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* idx, float* score,
                                  void* ws, size_t ws_bytes, void* stream) {
+    OrderScope order_scope(seq ? seq->order : 0);
     return dense_index_impl(seq, topk, idx, score, ws, ws_bytes, stream, 0, 0);
 }
 
@@ -571,6 +596,7 @@ pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* p
                                  const float* pq_scale, const float* pw, int32_t C, int32_t topk,
                                  int32_t* cand, float* cand_score, void* ws, size_t ws_bytes,
                                  void* stream) {
+    OrderScope order_scope(seq ? seq->order : 0);
     int t0, t1;
     pivot_status_t st = check_seq(seq, &t0, &t1);
     if (st != PIVOT_OK) return st;
@@ -706,6 +732,7 @@ static pivot_status_t refine_impl(const pivot_seq_t* seq, int32_t g, const int32
 pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* cand, int32_t C,
                             int32_t topk, int32_t* idx, float* score, void* ws, size_t ws_bytes,
                             void* stream) {
+    OrderScope order_scope(seq ? seq->order : 0);
     return refine_impl(seq, g, cand, C, topk, idx, score, ws, ws_bytes, stream, 0, 0);
 }
 
@@ -726,11 +753,13 @@ pivot_seq_t varlen_seq(const pivot_varlen_t* b, int i) {
     s.w = b->w + off * b->H;
     s.k = static_cast<const uint8_t*>(b->k) + off * b->D * es;
     s.k_scale = b->k_scale ? b->k_scale + off : nullptr;
+    s.order = b->order;
     return s;
 }
 
 pivot_status_t check_varlen(const pivot_varlen_t* b, int mode, int g, int C, int topk) {
     if (!b || b->nseq < 1 || !b->cu_seqlens || b->cu_seqlens[0] != 0) return PIVOT_ERR_INVALID_ARG;
+    if (!order_ok(b->order)) return PIVOT_ERR_INVALID_ARG;
     if (mode < PIVOT_MODE_DENSE || mode > PIVOT_MODE_REFINE || topk < 1) return PIVOT_ERR_INVALID_ARG;
     if (mode != PIVOT_MODE_DENSE && (g < 1 || C < topk)) return PIVOT_ERR_INVALID_ARG;
     if (topk > MAX_K || (mode != PIVOT_MODE_DENSE && C > MAX_K)) return PIVOT_ERR_UNSUPPORTED;
@@ -1121,6 +1150,7 @@ size_t pivot_index_varlen_workspace_size(const pivot_varlen_t* batch, int32_t mo
 pivot_status_t pivot_index_varlen(const pivot_varlen_t* batch, int32_t mode, int32_t g, int32_t C,
                                   int32_t topk, int32_t* idx, void* ws, size_t ws_bytes,
                                   void* stream) {
+    OrderScope order_scope(batch ? batch->order : 0);
     pivot_status_t st = check_varlen(batch, mode, g, C, topk);
     if (st != PIVOT_OK) return st;
     if (!idx || !ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
@@ -1218,6 +1248,7 @@ size_t pivot_index_window_outside_workspace_size(const pivot_seq_t* seq, int32_t
 pivot_status_t pivot_index_window_outside(const pivot_seq_t* seq, int32_t mode, int32_t g,
                                           int32_t C, int32_t topk, int32_t window, int32_t* idx,
                                           void* ws, size_t ws_bytes, void* stream) {
+    OrderScope order_scope(seq ? seq->order : 0);
     int t0, t1;
     pivot_status_t st = check_window(seq, mode, g, C, topk, window, &t0, &t1);
     if (st != PIVOT_OK) return st;
@@ -1260,7 +1291,7 @@ pivot_status_t pivot_index_window_outside(const pivot_seq_t* seq, int32_t mode, 
 
 // ------------------------------------------------------------------ decode
 static pivot_status_t check_decode(const pivot_decode_t* b) {
-    if (!b || !dtype_ok(b->dtype)) return PIVOT_ERR_INVALID_ARG;
+    if (!b || !dtype_ok(b->dtype) || !order_ok(b->order)) return PIVOT_ERR_INVALID_ARG;
     if (b->B < 1 || b->Gm < 1 || b->H < 1 || b->D < 1 || b->maxlen < b->Gm)
         return PIVOT_ERR_INVALID_ARG;
     if (!b->q || !b->w || !b->kc || !b->cache_len) return PIVOT_ERR_INVALID_ARG;
@@ -1310,13 +1341,54 @@ size_t pivot_decode_workspace_size(const pivot_decode_t* b, int32_t mode, int32_
     return decode_layout(b, mode, C, nullptr, nullptr, 0);
 }
 
+// The workspace of a whole indexer pass, from sizes alone (no buffers): the
+// largest workspace any call of the mode's call chain needs.
+size_t pivot_workspace_size(int32_t mode, int32_t dtype, int32_t L_or_maxlen, int32_t B,
+                            int32_t H, int32_t D, int32_t g, int32_t C, int32_t topk) {
+    if (mode < PIVOT_MODE_DENSE || mode > PIVOT_MODE_REFINE || !dtype_ok(dtype)) return 0;
+    // stand-in addresses: only checked for presence and alignment, never read
+    const void* dummy = reinterpret_cast<const void*>(uintptr_t(WS_ALIGN));
+    const float* fdummy = static_cast<const float*>(dummy);
+    const bool fp8 = dtype == PIVOT_E4M3;
+    if (B == 0) {
+        pivot_seq_t s{};
+        s.dtype = dtype;
+        s.L = L_or_maxlen;
+        s.H = H;
+        s.D = D;
+        s.q = dummy;
+        s.w = fdummy;
+        s.k = dummy;
+        s.q_scale = fp8 ? fdummy : nullptr;
+        s.k_scale = fp8 ? fdummy : nullptr;
+        if (mode == PIVOT_MODE_DENSE) return pivot_dense_index_workspace_size(&s, topk);
+        if (topk < 1 || C < topk) return 0;
+        const size_t scan = pivot_proxy_scan_workspace_size(&s, g, C);
+        if (scan == 0 || mode == PIVOT_MODE_REUSE) return scan;
+        const size_t ref = pivot_refine_workspace_size(&s, g, C, topk);
+        return ref == 0 ? 0 : (scan > ref ? scan : ref);
+    }
+    pivot_decode_t b{};
+    b.dtype = dtype;
+    b.B = B;
+    b.Gm = g;
+    b.H = H;
+    b.D = D;
+    b.maxlen = L_or_maxlen;
+    b.q = dummy;
+    b.w = fdummy;
+    b.kc = dummy;
+    b.q_scale = fp8 ? fdummy : nullptr;
+    b.kc_scale = fp8 ? fdummy : nullptr;
+    b.cache_len = static_cast<const int32_t*>(dummy);
+    return pivot_decode_workspace_size(&b, mode, C, topk);
+}
+
 pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, int32_t topk,
                             int32_t* idx, int32_t* cand, void* ws, size_t ws_bytes, void* stream) {
-    pivot_status_t st = check_decode(b);
+    OrderScope order_scope(b ? b->order : 0);
+    pivot_status_t st = decode_check_args(b, mode, C, topk, idx);
     if (st != PIVOT_OK) return st;
-    if (mode < 0 || mode > 2 || topk < 1 || !idx) return PIVOT_ERR_INVALID_ARG;
-    if (mode != PIVOT_MODE_DENSE && C < topk) return PIVOT_ERR_INVALID_ARG;
-    if (topk > MAX_K || C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
     DecodeWs w;
     if (decode_layout(b, mode, C, &w, ws, ws_bytes) == 0) return PIVOT_ERR_WORKSPACE;
@@ -1377,3 +1449,19 @@ pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, in
 }
 
 }  // extern "C"
+
+namespace pivot {
+
+// The argument checks of pivot_decode, shared with pivot_decode_noalloc so
+// that both report the same status for the same arguments.
+pivot_status_t decode_check_args(const pivot_decode_t* b, int32_t mode, int32_t C, int32_t topk,
+                                 const int32_t* idx) {
+    pivot_status_t st = check_decode(b);
+    if (st != PIVOT_OK) return st;
+    if (mode < 0 || mode > 2 || topk < 1 || !idx) return PIVOT_ERR_INVALID_ARG;
+    if (mode != PIVOT_MODE_DENSE && C < topk) return PIVOT_ERR_INVALID_ARG;
+    if (topk > MAX_K || C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
+    return PIVOT_OK;
+}
+
+}  // namespace pivot

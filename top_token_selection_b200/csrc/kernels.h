@@ -89,6 +89,8 @@ struct SelectParams {
     SegTable seg;             // scan_kind SCAN_VARLEN_*: the batch's sequences; candidate
                               // rows of packed token r: group seg_group_of(r), key scales
                               // from the sequence's first token
+    int rank_order;           // 1: rows in rank order (score descending, then position
+                              // ascending; `split` is then moot); 0: ascending positions
 };
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);

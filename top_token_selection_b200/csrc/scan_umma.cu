@@ -647,7 +647,7 @@ static cudaError_t launch_any(const CUtensorMap& tk, const CUtensorMap& tq, cons
     switch (p.dtype) {
         case PIVOT_E4M3: return launch_kind<KIND_F8, GATHER>(tk, tq, p, row_bytes, grid, stream);
         case PIVOT_BF16: return launch_kind<KIND_F16, GATHER>(tk, tq, p, row_bytes, grid, stream);
-        default: return launch_kind<KIND_TF32, GATHER>(tk, tq, p, row_bytes, grid, stream);
+        default: return cudaErrorInvalidValue;   // fp32 inputs are scored on the CUDA cores
     }
 }
 

@@ -357,6 +357,30 @@ __device__ void pad_row(uint32_t from, int K, int32_t* out, float* outs) {
     }
 }
 
+template <class Less>
+__device__ void bitonic_sort(uint64_t* buf, int n, uint64_t pad, Less less);
+
+// Rank order: the kept entries whose positions are marked in `bm` (exactly
+// Kp of them), sorted by key descending -- score descending, then position
+// ascending -- into out[0, Kp), then -1 padding to K.  Unmarked entries are
+// cleared to the padding key 0 (which sorts last) and everything is sorted
+// in place.
+__device__ void write_rank_order(uint64_t* buf, int n, const uint32_t* bm, uint32_t Kp, int K,
+                                 int32_t* out, float* outs) {
+    for (int i = threadIdx.x; i < n; i += SEL_THREADS) {
+        const uint64_t k = buf[i];
+        if (k != 0 && !bit_of(bm, key_pos(k))) buf[i] = 0;
+    }
+    __syncthreads();
+    bitonic_sort(buf, n, 0ull, [](uint64_t a, uint64_t b) { return a > b; });
+    for (int i = threadIdx.x; i < (int)Kp; i += SEL_THREADS) {
+        const uint64_t k = buf[i];
+        out[i] = key_pos(k);
+        if (outs) outs[i] = key_to_float(key_u(k));
+    }
+    pad_row(Kp, K, out, outs);
+}
+
 struct FastSmem {
     uint32_t* hist;     // HIST_BINS: samples, then linear bins
     uint32_t* scratch;  // 64
@@ -508,13 +532,17 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
     auto uval = [&](int i) { return key_u(buf[i]); };
     uint32_t aboveK, aboveS = 0;
     const uint32_t TuK = kth_largest_linear(uval, n, Kp, hist, scratch, &aboveK);
-    const int split = (p.split > 0 && (uint32_t)p.split < Kp) ? p.split : 0;
+    const int split = (!p.rank_order && p.split > 0 && (uint32_t)p.split < Kp) ? p.split : 0;
     uint32_t TuS = 0;
     if (split) TuS = kth_largest_linear(uval, n, (uint32_t)split, hist, scratch, &aboveS);
     // selected set (the linear bins are no longer needed, so pref may alias them)
     for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmS[w] = 0;
     __syncthreads();
     mark_top(buf, n, TuK, Kp - aboveK, sm.bmS, sm.bmT, sm.pref, W, scratch);
+    if (p.rank_order) {
+        write_rank_order(buf, n, sm.bmS, Kp, K, out, outs);
+        return true;
+    }
     if (!split) {
         write_marked(buf, n, sm.bmS, sm.pref, W, 0, scratch, out, outs);
     } else {
@@ -676,8 +704,10 @@ __device__ void select_exact(const SelectParams& p, const RowView& v, uint32_t* 
 
     // 5. order: by key (to split off the top `split`), then by position
     auto by_pos = [](uint64_t a, uint64_t b) { return key_upos(a) < key_upos(b); };
-    const int split = (p.split > 0 && (uint32_t)p.split < Kp) ? p.split : 0;
-    if (split) {
+    const int split = (!p.rank_order && p.split > 0 && (uint32_t)p.split < Kp) ? p.split : 0;
+    if (p.rank_order) {
+        bitonic_sort(sel, (int)Kp, 0ull, [](uint64_t a, uint64_t b) { return a > b; });
+    } else if (split) {
         bitonic_sort(sel, (int)Kp, 0ull, [](uint64_t a, uint64_t b) { return a > b; });
         uint64_t* rest = sel + M2;
         for (int i = threadIdx.x; i < (int)Kp - split; i += SEL_THREADS) rest[i] = sel[split + i];

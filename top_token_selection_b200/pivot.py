@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(HERE, "libpivot.so")
 
 F32, BF16, E4M3 = 0, 1, 2
 DENSE, REUSE, REFINE = 0, 1, 2
+ORDER_POSITION, ORDER_RANK = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "workspace too small",
           4: "CUDA error", 5: "a kernel wait timed out", 6: "bad device-side data"}
 
@@ -34,6 +35,7 @@ ABI_SYMBOLS = [
     "pivot_reuse_backfill", "pivot_window_union", "pivot_index_varlen",
     "pivot_index_varlen_workspace_size", "pivot_index_window_outside",
     "pivot_index_window_outside_workspace_size", "pivot_set_score_buffer_cap",
+    "pivot_workspace_size",
 ]
 KERNELS = {0: "scan", 1: "select", 2: "refine", 3: "reduce", 4: "reuse"}
 
@@ -48,14 +50,15 @@ class PivotSeq(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int32), ("L", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("q", ctypes.c_void_p), ("q_scale", ctypes.c_void_p),
                 ("w", ctypes.c_void_p), ("k", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
-                ("t_begin", ctypes.c_int32), ("t_end", ctypes.c_int32)]
+                ("t_begin", ctypes.c_int32), ("t_end", ctypes.c_int32),
+                ("order", ctypes.c_int32)]
 
 
 class PivotVarlen(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int32), ("nseq", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p), ("q", ctypes.c_void_p),
                 ("q_scale", ctypes.c_void_p), ("w", ctypes.c_void_p), ("k", ctypes.c_void_p),
-                ("k_scale", ctypes.c_void_p)]
+                ("k_scale", ctypes.c_void_p), ("order", ctypes.c_int32)]
 
 
 class PivotDecode(ctypes.Structure):
@@ -63,7 +66,7 @@ class PivotDecode(ctypes.Structure):
                 ("H", ctypes.c_int32), ("D", ctypes.c_int32), ("maxlen", ctypes.c_int32),
                 ("q", ctypes.c_void_p), ("q_scale", ctypes.c_void_p), ("w", ctypes.c_void_p),
                 ("kc", ctypes.c_void_p), ("kc_scale", ctypes.c_void_p),
-                ("cache_len", ctypes.c_void_p)]
+                ("cache_len", ctypes.c_void_p), ("order", ctypes.c_int32)]
 
 
 _lib = None
@@ -107,6 +110,7 @@ def load(path: str = LIB_PATH):
         "pivot_index_varlen_workspace_size": ([P, I32, I32, I32, I32], SZ),
         "pivot_index_window_outside": ([P, I32, I32, I32, I32, I32, P, P, SZ, P], I32),
         "pivot_index_window_outside_workspace_size": ([P, I32, I32, I32, I32, I32], SZ),
+        "pivot_workspace_size": ([I32, I32, I32, I32, I32, I32, I32, I32, I32], SZ),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -169,6 +173,10 @@ def pivot_decode(batch, mode, C, topk, idx, cand, ws, ws_bytes, stream):
 
 def pivot_decode_workspace_size(batch, mode, C, topk):
     return load().pivot_decode_workspace_size(ctypes.byref(batch), mode, C, topk)
+
+
+def pivot_workspace_size(mode, dtype, L_or_maxlen, B, H, D, g, C, topk):
+    return load().pivot_workspace_size(mode, dtype, L_or_maxlen, B, H, D, g, C, topk)
 
 
 def pivot_decode_noalloc(batch, mode, C, topk, idx, cand, stream):
@@ -263,22 +271,22 @@ def _workspace(nbytes, device):
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def make_seq(q, q_scale, w, k, k_scale, t_begin=0, t_end=0) -> PivotSeq:
+def make_seq(q, q_scale, w, k, k_scale, t_begin=0, t_end=0, order=ORDER_POSITION) -> PivotSeq:
     """Describe one prefill sequence; the struct keeps the tensors alive."""
     L, H, D = q.shape
     s = PivotSeq(_dtype_code(q), L, H, D, _p(q), _p(q_scale), _p(w), _p(k), _p(k_scale),
-                 t_begin, t_end)
+                 t_begin, t_end, order)
     s._keep = (q, q_scale, w, k, k_scale)
     return s
 
 
-def make_varlen(cu_seqlens, q, q_scale, w, k, k_scale) -> PivotVarlen:
+def make_varlen(cu_seqlens, q, q_scale, w, k, k_scale, order=ORDER_POSITION) -> PivotVarlen:
     """Describe a ragged batch: cu_seqlens is a host sequence of nseq + 1
     row offsets; the struct keeps it and the tensors alive."""
     cu = (ctypes.c_int32 * len(cu_seqlens))(*[int(x) for x in cu_seqlens])
     _, H, D = q.shape
     s = PivotVarlen(_dtype_code(q), len(cu_seqlens) - 1, H, D, ctypes.addressof(cu), _p(q),
-                    _p(q_scale), _p(w), _p(k), _p(k_scale))
+                    _p(q_scale), _p(w), _p(k), _p(k_scale), order)
     s._keep = (cu, q, q_scale, w, k, k_scale)
     return s
 
@@ -323,11 +331,11 @@ def index_varlen(batch: PivotVarlen, mode, g, C, topk, ws=None, stream=None, dev
     return idx
 
 
-def make_decode(q, q_scale, w, kc, kc_scale, cache_len) -> PivotDecode:
+def make_decode(q, q_scale, w, kc, kc_scale, cache_len, order=ORDER_POSITION) -> PivotDecode:
     """Describe one decode batch; the struct keeps the tensors alive."""
     B, Gm, H, D = q.shape
     s = PivotDecode(_dtype_code(q), B, Gm, H, D, kc.shape[1], _p(q), _p(q_scale), _p(w),
-                    _p(kc), _p(kc_scale), _p(cache_len))
+                    _p(kc), _p(kc_scale), _p(cache_len), order)
     s._keep = (q, q_scale, w, kc, kc_scale, cache_len)
     return s
 
@@ -361,7 +369,7 @@ def proxy_reduce(seq: PivotSeq, g, stream=None, device="cuda"):
 def proxy_scan(seq: PivotSeq, g, pq, pqs, pw, C, topk, with_score=False, ws=None, stream=None,
                device="cuda"):
     """Candidates [G, C]: each proxy's top-topk positions, then the rest of
-    its top-C, each ascending."""
+    its top-C, each ascending (rank order throughout if seq.order asks)."""
     G = pq.shape[0]
     cand = torch.empty(G, C, dtype=torch.int32, device=device)
     cs = torch.empty(G, C, dtype=torch.float32, device=device) if with_score else None
