@@ -6,13 +6,14 @@
 // AddressSanitizer and UndefinedBehaviorSanitizer.
 //
 //   select_check prefix <L> <K> <split> <dist> <rows> <use_bound>
-//   select_check cand <C> <K> <mode> <rows>
+//   select_check cand <C> <K> <mode> <rows> <order> <layout>
 //   select_check varlen <kind> <g> <K> <C>     (ragged batch rows, see run_varlen)
 //   select_check decode <kind> <K>             (MTP decode rows, see run_decode)
 //   select_check backfill <L> <g> <C> <K>      (Reuse with backfill, see run_backfill)
 // dist: 0 normal, 1 few distinct values (heavy ties), 2 signed zeros and
 // small integers, 3 a heavy tail (a few huge scores); mode: 0 plain, 1 ties,
-// 2 rows padded with -1, 3 with per-key scales.
+// 2 rows padded with -1, 3 with per-key scales; order: 0 ascending positions,
+// 1 rank order; layout: 0 the proxy scan's two ascending runs, 1 shuffled.
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
@@ -110,59 +111,99 @@ int run_prefix(int L, int K, int split, int dist, int nrows, bool use_bound) {
     return bad;
 }
 
-int run_cand(int C, int K, int mode, int nrows) {
+// Top K of the entries (score desc, position asc), in that rank order,
+// -1 padded.
+std::vector<int> reference_rank(std::vector<std::pair<uint32_t, int>> e, int K) {
+    std::sort(e.begin(), e.end(), [](const auto& a, const auto& b) {
+        return a.first != b.first ? a.first > b.first : a.second < b.second;
+    });
+    std::vector<int> A;
+    for (int i = 0; i < std::min<int>(K, (int)e.size()); ++i) A.push_back(e[i].second);
+    while ((int)A.size() < K) A.push_back(-1);
+    return A;
+}
+
+// Candidate rows of `nrows` consecutive members (one launch; each member its
+// own group, g = 1), member t seeing positions <= t.  layout 0: the proxy
+// scan's rows (its top-K ascending, then the rest ascending, -1 padded);
+// layout 1: the same positions shuffled.  order 0: positions ascending;
+// order 1: rank order.
+int run_cand(int C, int K, int mode, int nrows, int order, int layout) {
     const int L = 20000;
-    std::mt19937 rng(7 + mode);
-    std::vector<int32_t> cand(C), out(K);
-    std::vector<float> S(C), outs(K), ksc(L);
+    std::mt19937 rng(7 + mode + 13 * layout + 29 * order);
+    std::vector<int32_t> cand((size_t)nrows * C), out((size_t)nrows * K);
+    std::vector<float> S((size_t)nrows * C), outs((size_t)nrows * K), ksc(L);
     for (auto& x : ksc) x = std::uniform_real_distribution<float>(0.5f, 2.0f)(rng);
     std::vector<int> all(L);
-    int bad = 0;
+    const int t0 = (int)(rng() % (L - nrows));
     for (int r = 0; r < nrows; ++r) {
-        // the proxy's top-K (ascending), then the rest (ascending), -1 padded
         for (int i = 0; i < L; ++i) all[i] = i;
         std::shuffle(all.begin(), all.end(), rng);
-        const int nreal = mode == 2 ? C / 2 + (int)(rng() % (C / 2)) : C;
+        const int nreal = mode == 2 ? C / 2 + (int)(rng() % (C / 2 + 1)) : C;
         const int s = std::min(K, nreal);
         std::vector<int> A(all.begin(), all.begin() + s), B(all.begin() + s, all.begin() + nreal);
         std::sort(A.begin(), A.end());
         std::sort(B.begin(), B.end());
-        for (int i = 0; i < C; ++i) cand[i] = i < s ? A[i] : (i < nreal ? B[i - s] : -1);
+        int32_t* c = cand.data() + (size_t)r * C;
+        for (int i = 0; i < C; ++i) c[i] = i < s ? A[i] : (i < nreal ? B[i - s] : -1);
+        if (layout == 1) std::shuffle(c, c + C, rng);
         for (int i = 0; i < C; ++i)
-            S[i] = mode == 1 ? (float)(rng() % 7) : std::normal_distribution<float>(1.f, 3.f)(rng);
-        const int t = (int)(rng() % L);   // the member's position
-        SelectParams sp{};
-        sp.kind = SEL_CANDIDATES;
-        sp.scan_kind = SCAN_PREFILL_DENSE;
-        sp.row0 = t;
-        sp.nrows = 1;
-        sp.L = L;
-        sp.g = 1;
-        sp.Gm = 1;
-        sp.S = S.data();
-        sp.S_stride = C;
-        sp.cand = cand.data();
-        sp.cand_base = t;
-        sp.C = C;
-        sp.K = K;
-        sp.out_idx = out.data();
-        sp.out_score = outs.data();
-        sp.out_base = t;
-        sp.tail_cap = 2048;
-        sp.npos = L;
-        sp.key_scale = mode == 3 ? ksc.data() : nullptr;
-        std::fill(out.begin(), out.end(), -7);
-        if (launch_select(sp, nullptr) != cudaSuccess) return 2;
+            S[(size_t)r * C + i] =
+                mode == 1 ? (float)(rng() % 7) : std::normal_distribution<float>(1.f, 3.f)(rng);
+    }
+    SelectParams sp{};
+    sp.kind = SEL_CANDIDATES;
+    sp.scan_kind = SCAN_PREFILL_DENSE;
+    sp.row0 = t0;
+    sp.nrows = nrows;
+    sp.L = L;
+    sp.g = 1;
+    sp.Gm = 1;
+    sp.S = S.data();
+    sp.S_stride = C;
+    sp.cand = cand.data();
+    sp.cand_base = t0;
+    sp.C = C;
+    sp.K = K;
+    sp.out_idx = out.data();
+    sp.out_score = outs.data();
+    sp.out_base = t0;
+    sp.tail_cap = 2048;
+    sp.npos = L;
+    sp.rank_order = order;
+    sp.key_scale = mode == 3 ? ksc.data() : nullptr;
+    std::fill(out.begin(), out.end(), -7);
+    if (launch_select(sp, nullptr) != cudaSuccess) return 2;
+    int bad = 0;
+    for (int r = 0; r < nrows; ++r) {
+        const int t = t0 + r;
+        const int32_t* c = cand.data() + (size_t)r * C;
         std::vector<std::pair<uint32_t, int>> e;
         for (int i = 0; i < C; ++i)
-            if (cand[i] >= 0 && cand[i] <= t) {
-                float x = S[i];
-                if (mode == 3) x = x * ksc[cand[i]];
-                e.push_back({okey(x), cand[i]});
+            if (c[i] >= 0 && c[i] <= t) {
+                float x = S[(size_t)r * C + i];
+                if (mode == 3) x = x * ksc[c[i]];
+                e.push_back({okey(x), c[i]});
             }
-        if (reference(e, K, 0) != std::vector<int>(out.begin(), out.end())) {
+        const std::vector<int> want = order ? reference_rank(e, K) : reference(e, K, 0);
+        if (want != std::vector<int>(out.begin() + (size_t)r * K,
+                                     out.begin() + (size_t)(r + 1) * K)) {
             ++bad;
             std::printf("candidate row %d (t = %d): mismatch\n", r, t);
+        }
+        // scores line up with the positions
+        for (int i = 0; i < K && out[(size_t)r * K + i] >= 0; ++i) {
+            const int pos = out[(size_t)r * K + i];
+            int at = -1;
+            for (int j = 0; j < C; ++j)
+                if (c[j] == pos) at = j;
+            float x = S[(size_t)r * C + at];
+            if (mode == 3) x = x * ksc[pos];
+            if (okey(x) != okey(outs[(size_t)r * K + i])) {
+                ++bad;
+                std::printf("candidate row %d: score of slot %d\n", r, i);
+                break;
+            }
         }
     }
     return bad;
@@ -400,8 +441,9 @@ int main(int argc, char** argv) {
     if (what == "prefix" && argc == 8)
         bad = run_prefix(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]), atoi(argv[6]),
                          atoi(argv[7]) != 0);
-    else if (what == "cand" && argc == 6)
-        bad = run_cand(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]));
+    else if (what == "cand" && argc == 8)
+        bad = run_cand(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]), atoi(argv[6]),
+                       atoi(argv[7]));
     else if (what == "backfill" && argc == 6)
         bad = run_backfill(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]));
     else if (what == "decode" && argc == 4)

@@ -31,6 +31,9 @@ def select_check(tmp_path_factory):
         ("extern __shared__ __align__(16) uint8_t smem_t[];", "uint8_t* smem_t = emu_smem();"),
         ("row_threshold_kernel<<<grid, THR_WARPS * 32, smem, stream>>>(p, thresh);",
          "emu_launch(grid, THR_WARPS * 32, smem, [&] { row_threshold_kernel(p, thresh); });"),
+        ("extern __shared__ __align__(16) uint8_t smem_c[];", "uint8_t* smem_c = emu_smem();"),
+        ("select_cand_kernel<<<grid, warps * 32, smem, stream>>>(p, warps);",
+         "emu_launch(grid, warps * 32, smem, [&] { select_cand_kernel(p, warps); });"),
     ])
     (d / "topk_emu.cpp").write_text(topk)
     return compile_(d, [d / "topk_emu.cpp", EMU / "select_check.cpp"], d / "select_check",
@@ -57,9 +60,24 @@ def test_prefix_rows_match_a_sort(select_check, L, K, split, dist, rows, bound):
 
 @pytest.mark.parametrize("mode", [0, 1, 2, 3])
 def test_candidate_rows_match_a_sort(select_check, mode):
-    """Refine rows: cand[j] gives the positions, the member's limit masks later
-    ones; ties (1), -1 padded rows (2), per-key scales multiplied in (3)."""
-    _run(select_check, "cand", 4096, 2048, mode, 2)
+    """Refine rows (one warp each, several warps per block): cand[j] gives the
+    positions, the member's limit masks later ones; ties (1), -1 padded rows
+    (2), per-key scales multiplied in (3)."""
+    _run(select_check, "cand", 4096, 2048, mode, 9, 0, 0)
+
+
+@pytest.mark.parametrize("C,K,mode,order,layout", [
+    (4096, 2048, 1, 1, 0),   # rank order with heavy ties
+    (4096, 2048, 3, 1, 0),   # rank order, per-key scales
+    (4096, 2048, 0, 0, 1),   # shuffled candidate rows: sorted by position, not merged
+    (300, 300, 1, 0, 0),     # C = k, ties
+    (40, 9, 2, 0, 0),        # tiny rows, -1 padding
+    (8192, 2048, 0, 0, 0),   # the largest C (three warps a block)
+    (8192, 8192, 1, 1, 1),   # k = C = 8192, rank order, shuffled
+    (1, 1, 0, 0, 0),         # one candidate
+])
+def test_candidate_rows_orders_and_sizes(select_check, C, K, mode, order, layout):
+    _run(select_check, "cand", C, K, mode, 7, order, layout)
 
 
 @pytest.mark.parametrize("kind,g,K,C", [(0, 8, 64, 0), (1, 8, 16, 96), (2, 8, 16, 96),

@@ -79,12 +79,12 @@ def test_noalloc_decode_matches_decode_with_workspace(dtype):
 
 
 def test_noalloc_rejects_a_batch_beyond_its_scratch():
-    # One sequence with an 8M-key cache: two dense score rows need 64 MiB
-    # plus their selection bounds, more than the array holds, so the call is
-    # refused before anything is enqueued.  The buffers are real and the
-    # cached length is short, so nothing could read out of bounds even if
-    # the size guard were lost.
-    maxlen = 1 << 23
+    # One sequence with an (8M + 4096)-key cache: two dense score rows need
+    # just over 64 MiB, more than the array holds, so the call is refused
+    # before anything is enqueued.  The buffers are real and the cached
+    # length is short, so nothing could read out of bounds even if the size
+    # guard were lost.
+    maxlen = (1 << 23) + 4096
     dev = "cuda"
     q = torch.zeros((1, 2, 64, 128), dtype=torch.float8_e4m3fn, device=dev)
     qs = torch.ones((1, 2), dtype=torch.float32, device=dev)

@@ -529,18 +529,25 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                         uint64_t a[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) a[j] = 0ull;
+                        // the row's columns in 16-column chunks, software-
+                        // pipelined: chunk c + 1 is loaded from TMEM while
+                        // chunk c's math runs
+                        constexpr int NCH = HEADS / 16;
+                        float v[2][16];
+                        tmem_ld16(taddr + (uint32_t)(pr * HEADS), v[0]);
 #pragma unroll
-                        for (int c = 0; c < HEADS / 32; ++c) {
-                            float v[32];
-                            tmem_ld32(taddr + (uint32_t)(pr * HEADS + c * 32), v);
-                            tmem_ld_wait();
+                        for (int c = 0; c < NCH; ++c) {
+                            tmem_ld_wait16(v[c & 1]);
+                            if (c + 1 < NCH)
+                                tmem_ld16(taddr + (uint32_t)(pr * HEADS + (c + 1) * 16),
+                                          v[(c + 1) & 1]);
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const int wi = lr * HEADS + c * 32 + 2 * i;
+                            for (int i = 0; i < 8; ++i) {
+                                const int wi = lr * HEADS + c * 16 + 2 * i;
+                                const float x0 = v[c & 1][2 * i], x1 = v[c & 1][2 * i + 1];
                                 // x + |x| = 2 max(0, x): one add on the FMA pipe
                                 // instead of a half-rate max on the ALU pipe
-                                a[i & 3] = ffma2(pack2(v[2 * i] + fabsf(v[2 * i]),
-                                                       v[2 * i + 1] + fabsf(v[2 * i + 1])),
+                                a[i & 3] = ffma2(pack2(x0 + fabsf(x0), x1 + fabsf(x1)),
                                                  pack2(wr[wi], wr[wi + 1]), a[i & 3]);
                             }
                         }

@@ -755,13 +755,14 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t x) {
     return x;
 }
 
-// The m-th largest of the nonzero values v[0..n), 1 <= m <= their count, by
-// one warp; v and hist (THR_BINS words) in this warp's shared memory.
-__device__ uint32_t warp_kth_largest(const uint32_t* v, int n, uint32_t m, uint32_t* hist) {
+// The m-th largest of the nonzero values get(0..n), 1 <= m <= their count,
+// by one warp; hist (THR_BINS words) in this warp's shared memory.
+template <class F>
+__device__ uint32_t warp_kth_largest_f(F get, int n, uint32_t m, uint32_t* hist) {
     const int lane = threadIdx.x & 31;
     uint32_t lo = 0xFFFFFFFFu, hi = 0;
     for (int i = lane; i < n; i += 32) {
-        const uint32_t u = v[i];
+        const uint32_t u = get(i);
         if (u) { lo = min(lo, u); hi = max(hi, u); }
     }
     lo = warp_min_u32(lo);
@@ -776,7 +777,7 @@ __device__ uint32_t warp_kth_largest(const uint32_t* v, int n, uint32_t m, uint3
         for (int b = 0; b < THR_BINS / 32; ++b) hist[b * 32 + lane] = 0;
         __syncwarp();
         for (int i = lane; i < n; i += 32) {
-            const uint32_t u = v[i];
+            const uint32_t u = get(i);
             if (u && u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> sh], 1u);
         }
         __syncwarp();
@@ -827,6 +828,10 @@ __device__ uint32_t warp_kth_largest(const uint32_t* v, int n, uint32_t m, uint3
     return lo;
 }
 
+__device__ uint32_t warp_kth_largest(const uint32_t* v, int n, uint32_t m, uint32_t* hist) {
+    return warp_kth_largest_f([&](int i) { return v[i]; }, n, m, hist);
+}
+
 __global__ void __launch_bounds__(THR_WARPS * 32) row_threshold_kernel(const SelectParams p,
                                                                         uint32_t* thresh) {
     extern __shared__ __align__(16) uint8_t smem_t[];
@@ -860,10 +865,215 @@ __global__ void __launch_bounds__(THR_WARPS * 32) row_threshold_kernel(const Sel
     if (lane == 0) thresh[rr] = T;
 }
 
+// ------------------------------------------------------------ candidate rows
+//
+// Candidate rows (Refine, Reuse with backfill: C entries, positions from the
+// group's candidate row) are short, so each is selected by ONE warp with no
+// block barriers: its C entries, as 64-bit keys, sit in the warp's slice of
+// shared memory; the k-th largest score key comes from warp histograms over
+// the remaining key range (then, when the k-th score is tied, the same search
+// over the tied entries' positions); unselected entries are cleared and the
+// selected ones compacted in place, keeping their order.  In position order a
+// candidate row written by the proxy scan is two ascending runs (the proxy's
+// top-k, then the rest), so each selected entry's output slot is its rank in
+// its own run plus the number of selected entries of the other run at lower
+// positions (a binary search).  Rank order, and candidate rows of any other
+// layout, sort the selected keys in the warp (bitonic).
+
 __host__ __device__ int pow2_at_least(int x) {
     int m = 1;
     while (m < x) m <<= 1;
     return m;
+}
+
+constexpr int CW_MAX_WARPS = 8;
+constexpr size_t CW_SMEM_LIMIT = 200 * 1024;
+
+__host__ __device__ int cw_slots(int C) { return pow2_at_least(C < 32 ? 32 : C); }
+__host__ __device__ size_t cw_warp_bytes(int C) {
+    return (size_t)cw_slots(C) * 8 + (size_t)THR_BINS * 4;
+}
+
+// Sort e[0, M) (M a power of two, whole warp) so that before(a, b) holds for
+// every earlier a and later b.
+template <class Before>
+__device__ void warp_bitonic(uint64_t* e, int M, Before before) {
+    const int lane = threadIdx.x & 31;
+    for (int kk = 2; kk <= M; kk <<= 1) {
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+            for (int i = lane; i < M; i += 32) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const uint64_t a = e[i], b = e[ixj];
+                    const bool up = (i & kk) == 0;
+                    if (up ? before(b, a) : before(a, b)) {
+                        e[i] = b;
+                        e[ixj] = a;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+}
+
+// Compacts the nonzero entries of e[a, b) to the front of that range, in
+// order; returns their count.  Whole warp.
+__device__ int warp_compact(uint64_t* e, int a, int b) {
+    const int lane = threadIdx.x & 31;
+    int n = 0;
+    for (int i0 = a; i0 < b; i0 += 32) {
+        const int i = i0 + lane;
+        const uint64_t x = i < b ? e[i] : 0ull;
+        const unsigned m = __ballot_sync(0xffffffffu, x != 0);
+        __syncwarp();   // every read of this chunk precedes its writes
+        if (x != 0) e[a + n + __popc(m & ((1u << lane) - 1u))] = x;
+        n += __popc(m);
+        __syncwarp();
+    }
+    return n;
+}
+
+// Entries of sorted e[0, n) (ascending position: key_upos) at positions < pos.
+__device__ __forceinline__ int count_below(const uint64_t* e, int n, uint32_t pos) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (key_upos(e[mid]) < pos) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(CW_MAX_WARPS * 32) select_cand_kernel(const SelectParams p,
+                                                                        int warps) {
+    extern __shared__ __align__(16) uint8_t smem_c[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rr = blockIdx.x * warps + warp;
+    if (warp >= warps || rr >= p.nrows) return;   // whole warps; no block barriers below
+    const int C = p.C, K = p.K;
+    const int M = cw_slots(C);
+    uint64_t* e = reinterpret_cast<uint64_t*>(smem_c + (size_t)warp * cw_warp_bytes(C));
+    uint32_t* hist = reinterpret_cast<uint32_t*>(e + M);
+
+    // row r: its causal limit, candidate row, score row and key scales (as
+    // select_kernel reads a candidate row)
+    const int r = p.row0 + rr;
+    const size_t ostride = p.out_stride ? (size_t)p.out_stride : (size_t)K;
+    int32_t* out = p.out_idx + (size_t)(r - p.out_base) * ostride;
+    float* outs = p.out_score ? p.out_score + (size_t)(r - p.out_base) * ostride : nullptr;
+    bool ok;
+    const int lim = select_row_limit(p, r, ok) - p.lim_shift;
+    if (!ok && lane == 0) raise_error(ERRBIT_DATA);
+    const bool dec = p.scan_kind == SCAN_DECODE_DENSE;
+    const bool var = p.scan_kind == SCAN_VARLEN_DENSE;
+    const int grp = dec ? r / p.Gm : (var ? seg_group_of(p.seg, p.g, r) : r / p.g);
+    const int32_t* cand = p.cand + (size_t)(grp - p.cand_base) * C;
+    const float* S = p.s_per_group ? p.S + (size_t)(grp - p.cand_base) * p.S_stride
+                                   : p.S + (size_t)(r - p.row0) * p.S_stride;
+    const float* ksc = nullptr;
+    if (p.key_scale)
+        ksc = p.key_scale + (dec ? (size_t)grp * p.maxlen
+                                 : (var ? (size_t)p.seg.tok[seg_find(p.seg.tok, p.seg.nseq, r)]
+                                        : 0));
+
+    // 1. keys; descents between consecutive candidate positions (0 or 1:
+    //    at most two ascending runs, split where the descent is)
+    uint32_t nvalid = 0, ndesc = 0;
+    int split = C;
+    int prev_last = -1;   // position of the entry before this chunk
+    for (int i0 = 0; i0 < C; i0 += 32) {
+        const int i = i0 + lane;
+        const int pos = (ok && i < C) ? cand[i] : -1;
+        const bool valid = pos >= 0 && pos <= lim;
+        float x = 0.0f;
+        if (valid) {
+            x = S[i];
+            if (ksc) x = x * ksc[pos];
+        }
+        e[i] = valid ? make_key(ordered_key(x), pos) : 0ull;
+        nvalid += valid;
+        int before = __shfl_up_sync(0xffffffffu, pos, 1);
+        if (lane == 0) before = prev_last;
+        const unsigned dm = __ballot_sync(0xffffffffu, before >= 0 && pos >= 0 && pos < before);
+        if (dm && ndesc == 0) split = i0 + __ffs(dm) - 1;
+        ndesc += __popc(dm);
+        prev_last = __shfl_sync(0xffffffffu, pos, 31);
+    }
+    for (int i = C + lane; i < M; i += 32) e[i] = 0ull;
+    for (int o = 16; o > 0; o >>= 1) nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
+    __syncwarp();
+    const uint32_t Kp = nvalid < (uint32_t)K ? nvalid : (uint32_t)K;
+
+    // 2. keep exactly the top Kp keys (score, then lower position)
+    if (Kp < nvalid) {
+        const uint32_t T = warp_kth_largest_f([&](int i) { return key_u(e[i]); }, C, Kp, hist);
+        uint32_t above = 0, eq = 0;
+        for (int i = lane; i < C; i += 32) {
+            const uint32_t u = key_u(e[i]);
+            above += u > T;
+            eq += u == T;
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            above += __shfl_xor_sync(0xffffffffu, above, o);
+            eq += __shfl_xor_sync(0xffffffffu, eq, o);
+        }
+        const uint32_t need = Kp - above;   // 1 <= need <= eq
+        uint32_t Lmin = 0;                  // tied entries kept: low key half >= Lmin
+        if (eq > need)
+            Lmin = warp_kth_largest_f(
+                [&](int i) { return key_u(e[i]) == T ? (uint32_t)e[i] : 0u; }, C, need, hist);
+        __syncwarp();
+        for (int i = lane; i < C; i += 32) {
+            const uint64_t k = e[i];
+            const uint32_t u = key_u(k);
+            if (u < T || (u == T && (uint32_t)k < Lmin)) e[i] = 0ull;
+        }
+        __syncwarp();
+    }
+
+    // 3. output.  Position order: merge the two runs when each run's
+    //    selected entries are strictly ascending (always, for the proxy
+    //    scan's candidate rows; checked, since any row may be passed in).
+    bool merged = false;
+    if (!p.rank_order && ndesc <= 1) {
+        const int a = warp_compact(e, 0, split);
+        const int b = warp_compact(e, split, C);
+        const uint64_t* eb = e + split;
+        bool asc = true;
+        for (int i = lane; i + 1 < a; i += 32) asc = asc && key_upos(e[i]) < key_upos(e[i + 1]);
+        for (int i = lane; i + 1 < b; i += 32) asc = asc && key_upos(eb[i]) < key_upos(eb[i + 1]);
+        if (__all_sync(0xffffffffu, asc)) {
+            for (int i = lane; i < a + b; i += 32) {
+                const bool in_a = i < a;
+                const uint64_t k = in_a ? e[i] : eb[i - a];
+                const int own = in_a ? i : i - a;
+                const uint32_t pos = key_upos(k);
+                const int slot = own + (in_a ? count_below(eb, b, pos) : count_below(e, a, pos));
+                out[slot] = (int32_t)pos;
+                if (outs) outs[slot] = key_to_float(key_u(k));
+            }
+            merged = true;
+        }
+    }
+    if (!merged) {
+        const int n = warp_compact(e, 0, C);
+        const int Mn = pow2_at_least(n < 1 ? 1 : n);
+        for (int i = n + lane; i < Mn; i += 32) e[i] = 0ull;
+        __syncwarp();
+        if (p.rank_order)
+            warp_bitonic(e, Mn, [](uint64_t x, uint64_t y) { return x > y; });
+        else   // ascending position; the zero padding (position 0xFFFFFFFF) last
+            warp_bitonic(e, Mn, [](uint64_t x, uint64_t y) { return key_upos(x) < key_upos(y); });
+        for (int i = lane; i < n; i += 32) {
+            out[i] = key_pos(e[i]);
+            if (outs) outs[i] = key_to_float(key_u(e[i]));
+        }
+    }
+    for (int i = (int)Kp + lane; i < K; i += 32) {
+        out[i] = -1;
+        if (outs) outs[i] = -INFINITY;
+    }
 }
 
 }  // namespace
@@ -977,8 +1187,24 @@ size_t select_smem_bytes(int K, int tail_cap) {
     return select_layout(K, tail_cap, 0, 0, false).total;
 }
 
+// Candidate rows: one warp each, as many warps per CTA as the slices fit.
+static cudaError_t launch_select_cand(const SelectParams& p, cudaStream_t stream) {
+    const size_t per = cw_warp_bytes(p.C);
+    int warps = (int)(CW_SMEM_LIMIT / per);
+    if (warps > CW_MAX_WARPS) warps = CW_MAX_WARPS;
+    if (warps < 1) return cudaErrorInvalidValue;
+    const size_t smem = per * (size_t)warps;
+    cudaError_t e = cudaFuncSetAttribute(select_cand_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (p.nrows + warps - 1) / warps;
+    select_cand_kernel<<<grid, warps * 32, smem, stream>>>(p, warps);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_select(const SelectParams& p_in, cudaStream_t stream) {
     if (p_in.nrows <= 0) return cudaSuccess;
+    if (p_in.kind == SEL_CANDIDATES) return launch_select_cand(p_in, stream);
     SelectParams p = p_in;
     p.bitmap_words = (p.npos + 31) / 32;
     p.fast_cap = select_fast_cap(p.K);
