@@ -333,6 +333,20 @@ pivot_status_t pivot_set_wait_limit_ns(uint64_t ns);
  * thread-safe against concurrent calls. */
 pivot_status_t pivot_set_score_buffer_cap(size_t bytes);
 
+/* Test hook for the selection fused into the scan.  Prefix rows (dense
+ * queries and proxies, H >= 32 on the tensor cores) are selected without
+ * writing their scores: a sample scan over every 32nd key tile gives each
+ * row a bound, the scan keeps only the scores at or above it, and a row
+ * whose survivors fall outside what the in-scan selection holds is rescanned
+ * keeping everything.  on = 0 writes every score and selects afterwards (the
+ * results are identical); margin_sigmas (default 4.5) sets how far below the
+ * expected K-th score the bound sits, in standard deviations of the kept
+ * count: a large negative margin makes every long row miss low, a large
+ * positive one every long row miss high, which exercises the rescan.
+ * Process-wide, not thread-safe against concurrent calls; it changes what
+ * the *_workspace_size calls return. */
+pivot_status_t pivot_set_fused_selection(int32_t on, float margin_sigmas);
+
 /* Test hook: enqueue one kernel whose single wait is on a barrier nothing
  * arrives on.  With the wait limit lowered, a following
  * pivot_get_device_error() returns PIVOT_ERR_TIMEOUT and the device stays

@@ -10,6 +10,8 @@
 //   select_check varlen <kind> <g> <K> <C>     (ragged batch rows, see run_varlen)
 //   select_check decode <kind> <K>             (MTP decode rows, see run_decode)
 //   select_check backfill <L> <g> <C> <K>      (Reuse with backfill, see run_backfill)
+//   select_check fused <L> <K> <split> <dist> <rows> <r0> <order> <sigmas> <kind>
+//                                              (selection fused into the scan, see run_fused)
 // dist: 0 normal, 1 few distinct values (heavy ties), 2 signed zeros and
 // small integers, 3 a heavy tail (a few huge scores); mode: 0 plain, 1 ties,
 // 2 rows padded with -1, 3 with per-key scales; order: 0 ascending positions,
@@ -432,6 +434,120 @@ int run_decode(int kind, int K) {
     return bad;
 }
 
+// The selection fused into the scan, on prefix rows [r0, r0 + nrows) of a
+// dense (kind 0) or proxy (kind 1, groups of g = 8) scan: sample scores as
+// the sample scan writes them, the bound kernel, the filter scan's appends
+// emulated here (every score at or above the row's bound, shuffled within
+// each 4096-key chunk, as the scan's atomics may leave them), the warp
+// finish, then for the rows it listed the keep-everything regions and the
+// block select on keys.  Every row must equal the plain sort.  Prints the
+// number of rows that took the fallback.
+int run_fused(int L, int K, int split, int dist, int nrows, int r0, int order, float sigmas,
+              int kind) {
+    const int g = kind == 1 ? 8 : 1;
+    const int KTS = 32, CK = 32 * 128;
+    const int tiles = (L + 127) / 128;
+    const long long ss = (long long)((tiles + KTS - 1) / KTS) * 128;
+    const int nch = (tiles + 31) / 32;
+    const long long sv = (long long)nch * CK;
+    std::mt19937 rng(31 + 7 * dist + K + r0);
+    std::vector<float> samp((size_t)nrows * ss, 0.0f);
+    std::vector<uint64_t> surv((size_t)nrows * sv, 0);
+    std::vector<uint32_t> cnt((size_t)nrows * nch, 0xDEADu), bound(nrows);
+    std::vector<int32_t> miss(nrows, -9), out((size_t)nrows * K, -7);
+    std::vector<float> outs((size_t)nrows * K);
+    uint32_t nmiss = 12345;
+    std::vector<std::vector<float>> S(nrows);
+    auto lim_of = [&](int r) { return kind == 1 ? std::min(L, (r + 1) * g) - 1 : r; };
+    for (int i = 0; i < nrows; ++i) {
+        const int lim = lim_of(r0 + i);
+        S[i].resize(lim + 1);
+        for (auto& x : S[i]) x = draw(rng, dist);
+        for (long long j = 0; j < ss; ++j) {
+            const long long pos = (j / 128) * KTS * 128 + j % 128;
+            if (pos <= lim) samp[(size_t)i * ss + j] = S[i][pos];
+        }
+    }
+    FusedSelectParams fp{};
+    fp.scan_kind = kind == 1 ? SCAN_PREFILL_PROXY : SCAN_PREFILL_DENSE;
+    fp.row0 = r0;
+    fp.nrows = nrows;
+    fp.L = L;
+    fp.g = g;
+    fp.K = K;
+    fp.split = split;
+    fp.rank_order = order;
+    fp.samp = samp.data();
+    fp.samp_stride = ss;
+    fp.kts = KTS;
+    fp.sigmas = sigmas;
+    fp.bound = bound.data();
+    fp.cap = fused_cap(K);
+    fp.surv = surv.data();
+    fp.surv_stride = sv;
+    fp.surv_count = cnt.data();
+    fp.nchunks = nch;
+    fp.chunk_keys = CK;
+    fp.out_idx = out.data();
+    fp.out_score = outs.data();
+    fp.out_base = r0;
+    fp.miss_list = miss.data();
+    fp.miss_count = &nmiss;
+    if (launch_sample_bound(fp, nullptr) != cudaSuccess) return 2;
+    if (nmiss != 0) { std::printf("miss count not cleared\n"); return 3; }
+    // the filter scan: appends, then each chunk's count
+    auto fill = [&](int i, uint32_t T) {
+        const float tf = T <= 0x00800000u ? -INFINITY : key_to_float(T);
+        const int lim = lim_of(r0 + i);
+        for (int c = 0; c * CK <= lim; ++c) {
+            std::vector<uint64_t> kept;
+            for (int pos = c * CK; pos <= std::min(lim, (c + 1) * CK - 1); ++pos)
+                if (S[i][pos] >= tf)
+                    kept.push_back(((uint64_t)okey(S[i][pos]) << 32) | (0xFFFFFFFFu - (uint32_t)pos));
+            std::shuffle(kept.begin(), kept.end(), rng);
+            std::copy(kept.begin(), kept.end(), surv.begin() + (size_t)i * sv + (size_t)c * CK);
+            cnt[(size_t)i * nch + c] = (uint32_t)kept.size();
+        }
+    };
+    for (int i = 0; i < nrows; ++i) fill(i, bound[i]);
+    if (launch_fused_finish(fp, nullptr) != cudaSuccess) return 2;
+    // the fallback: listed rows keep everything, then the block select on keys
+    for (uint32_t m = 0; m < nmiss; ++m) fill(miss[m] - r0, 1u);
+    SelectParams sp{};
+    sp.kind = SEL_PREFIX;
+    sp.scan_kind = fp.scan_kind;
+    sp.row0 = r0;
+    sp.nrows = nrows;
+    sp.L = L;
+    sp.g = g;
+    sp.Gm = 1;
+    sp.keys = surv.data();
+    sp.S_stride = sv;
+    sp.K = K;
+    sp.split = split;
+    sp.npos = L;
+    sp.out_idx = out.data();
+    sp.out_score = outs.data();
+    sp.out_base = r0;
+    sp.tail_cap = 4096;
+    sp.rank_order = order;
+    sp.row_list = miss.data();
+    sp.row_count = &nmiss;
+    if (launch_select(sp, nullptr) != cudaSuccess) return 2;
+    int bad = 0;
+    for (int i = 0; i < nrows; ++i) {
+        std::vector<std::pair<uint32_t, int>> e;
+        for (int pos = 0; pos < (int)S[i].size(); ++pos) e.push_back({okey(S[i][pos]), pos});
+        const std::vector<int> want = order ? reference_rank(e, K) : reference(e, K, split);
+        if (want != std::vector<int>(out.begin() + (size_t)i * K, out.begin() + (size_t)(i + 1) * K)) {
+            ++bad;
+            std::printf("fused row %d: mismatch\n", r0 + i);
+        }
+    }
+    std::printf("fallback rows %u of %d\n", nmiss, nrows);
+    return bad;
+}
+
 }  // namespace
 
 int main(int argc, char** argv) {
@@ -444,6 +560,9 @@ int main(int argc, char** argv) {
     else if (what == "cand" && argc == 8)
         bad = run_cand(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]), atoi(argv[6]),
                        atoi(argv[7]));
+    else if (what == "fused" && argc == 11)
+        bad = run_fused(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]), atoi(argv[6]),
+                        atoi(argv[7]), atoi(argv[8]), (float)atof(argv[9]), atoi(argv[10]));
     else if (what == "backfill" && argc == 6)
         bad = run_backfill(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]));
     else if (what == "decode" && argc == 4)

@@ -265,3 +265,19 @@ def test_output_order_field_is_validated(lib):
                             order)
         assert pv.pivot_index_varlen(vb, pv.DENSE, 4, 16, 8, FAKE, FAKE, 1 << 20, None) == 1
     assert pv.pivot_dense_index_workspace_size(_seq(order=pv.ORDER_RANK), 8) > 0
+
+
+def test_fused_selection_hook(lib):
+    """The fused-selection switch takes 0 or 1 and a finite margin; switching
+    it off sizes the score buffer path's workspace instead."""
+    seq = _seq(dtype=pv.E4M3, L=20000, H=64, D=128, q_scale=FAKE, k_scale=FAKE)
+    try:
+        assert pv.pivot_set_fused_selection(2, 4.5) == 1
+        assert pv.pivot_set_fused_selection(1, float("nan")) == 1
+        assert pv.pivot_set_fused_selection(1, 4.5) == 0
+        fused = pv.pivot_dense_index_workspace_size(seq, 2048)
+        assert pv.pivot_set_fused_selection(0, 4.5) == 0
+        plain = pv.pivot_dense_index_workspace_size(seq, 2048)
+        assert fused > 0 and plain > 0 and fused != plain
+    finally:
+        assert pv.pivot_set_fused_selection(1, 4.5) == 0

@@ -10,6 +10,7 @@ The kernel source is used as it is; only its launch syntax and shared-memory
 declarations are rewritten for the host, and the few helpers it takes from
 common.cuh are copied from there verbatim.
 """
+import re
 import shutil
 import subprocess
 
@@ -34,6 +35,14 @@ def select_check(tmp_path_factory):
         ("extern __shared__ __align__(16) uint8_t smem_c[];", "uint8_t* smem_c = emu_smem();"),
         ("select_cand_kernel<<<grid, warps * 32, smem, stream>>>(p, warps);",
          "emu_launch(grid, warps * 32, smem, [&] { select_cand_kernel(p, warps); });"),
+        ("extern __shared__ __align__(16) uint8_t smem_b[];", "uint8_t* smem_b = emu_smem();"),
+        ("sample_bound_kernel<<<(p.nrows + FB_WARPS - 1) / FB_WARPS, FB_WARPS * 32, smem, stream>>>(p);",
+         "emu_launch((p.nrows + FB_WARPS - 1) / FB_WARPS, FB_WARPS * 32, smem, "
+         "[&] { sample_bound_kernel(p); });"),
+        ("extern __shared__ __align__(16) uint8_t smem_f[];", "uint8_t* smem_f = emu_smem();"),
+        ("fused_finish_kernel<<<(p.nrows + warps - 1) / warps, warps * 32, smem, stream>>>(p, warps);",
+         "emu_launch((p.nrows + warps - 1) / warps, warps * 32, smem, "
+         "[&] { fused_finish_kernel(p, warps); });"),
     ])
     (d / "topk_emu.cpp").write_text(topk)
     return compile_(d, [d / "topk_emu.cpp", EMU / "select_check.cpp"], d / "select_check",
@@ -105,3 +114,31 @@ def test_backfill_rows_match_a_sort(select_check, L, g, C, K):
     its group's candidates at or before t by proxy score, lower position
     first on ties (scores drawn from six values, so ties are common)."""
     _run(select_check, "backfill", L, g, C, K)
+
+
+@pytest.mark.parametrize("L,K,split,dist,rows,r0,order,sigmas,kind,want_fallback", [
+    (20000, 2048, 0, 0, 6, 19990, 0, 4.5, 0, "none"),    # long dense rows, normal scores
+    (20000, 2048, 0, 0, 5, 3000, 0, 4.5, 0, "none"),     # rows within the capacity keep all
+    (20000, 2048, 0, 3, 5, 19000, 1, 4.5, 0, "none"),    # heavy tail, rank order
+    (20000, 100, 0, 1, 6, 15000, 0, 4.5, 0, "any"),      # five values: ties at the bound
+    (20000, 2048, 0, 0, 4, 19000, 0, -40.0, 0, "all"),   # bound too high: every row falls back
+    (20000, 2048, 0, 0, 4, 19000, 1, 400.0, 0, "all"),   # bound too low: every row falls back
+    (40000, 4096, 2048, 0, 4, 4990, 0, 4.5, 1, "none"),  # proxy rows: top-k first, then the rest
+    (40000, 4096, 2048, 0, 3, 4990, 0, -40.0, 1, "all"), # the same through the fallback
+    (40000, 4096, 2048, 2, 3, 4990, 1, -40.0, 1, "any"), # signed zeros and small integers
+])
+def test_fused_selection_matches_a_sort(select_check, L, K, split, dist, rows, r0, order, sigmas,
+                                        kind, want_fallback):
+    """The selection fused into the scan: sample bound, warp select of the
+    survivors and, for rows that miss it, the keep-everything fallback --
+    every row equals a plain sort."""
+    res = subprocess.run([str(select_check), "fused", *map(str, (L, K, split, dist, rows, r0, order,
+                                                                  sigmas, kind))],
+                         capture_output=True, text=True, timeout=900)
+    assert res.returncode == 0, (res.stdout + res.stderr)[-4000:]
+    m = re.search(r"fallback rows (\d+) of (\d+)", res.stdout)
+    n_fb, n = int(m.group(1)), int(m.group(2))
+    if want_fallback == "none":
+        assert n_fb == 0
+    elif want_fallback == "all":
+        assert n_fb == n

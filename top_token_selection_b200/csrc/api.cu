@@ -20,6 +20,10 @@ constexpr size_t WS_ALIGN = 256;
 constexpr size_t SCORE_BUF_DEFAULT = size_t(4) << 30;   // preferred score buffer, 4 GiB
 size_t g_score_buf_cap = SCORE_BUF_DEFAULT;             // pivot_set_score_buffer_cap
 constexpr int MAX_K = 8192;   // the select's exact path holds 2 pow2(K) keys in shared memory
+// Fused selection: the sample scan scores every FUSED_KTS-th key tile; a scan
+// work item covers FUSED_TILES key tiles (its chunk of 4096 keys).
+constexpr int FUSED_KTS = 32;
+constexpr int FUSED_TILES = 32;
 constexpr int TAIL_CAP = 4096;
 constexpr int MAX_SMS = 1024;
 
@@ -184,12 +188,40 @@ double refine_pairs(int r0, int r1, int C) {
 
 // ------------------------------------------------------------------ scans
 // Rows [r0, r1) of kind `kind` into S (row r at S + (r - r0)*stride).
+// Modes of a tensor-core scan beyond plain scores (see ScanParams).
+struct ScanExtra {
+    int key_tile_stride = 0;            // sample scan
+    const uint32_t* bound = nullptr;    // filter mode
+    uint64_t* surv = nullptr;
+    long long surv_stride = 0;
+    uint32_t* surv_count = nullptr;
+    int nchunks = 0;
+    int lim_shift = 0;
+    const int32_t* row_list = nullptr;  // row-list mode (P = 1)
+    const uint32_t* row_count = nullptr;
+    double work = -1.0;                 // the launch's algorithmic pairs (profiling)
+};
+
 pivot_status_t run_scan(int kind, int dtype, int H, int D, const void* qbase, long long q_rows,
                         int qrow_base, const float* w, const float* q_scale, const void* kbase,
                         long long k_rows, const float* k_scale, int L, int g, int Gm, int maxlen,
                         const int32_t* cache_len, int P, int r0, int r1, int maxlim_total,
-                        float* S, long long stride, cudaStream_t st) {
+                        float* S, long long stride, cudaStream_t st,
+                        const ScanExtra* x = nullptr) {
     ScanParams p{};
+    if (x) {
+        p.key_tile_stride = x->key_tile_stride;
+        p.bound = x->bound;
+        p.surv = x->surv;
+        p.surv_stride = x->surv_stride;
+        p.surv_count = x->surv_count;
+        p.nchunks = x->nchunks;
+        p.lim_shift = x->lim_shift;
+        p.row_list = x->row_list;
+        p.row_count = x->row_count;
+        if (x->row_list) P = 1;
+    }
+    const double work = (x && x->work >= 0.0) ? x->work : scan_pairs(kind, r0, r1, L, g);
     p.kind = kind;
     p.dtype = dtype;
     p.esize = esize_of(dtype);
@@ -210,20 +242,22 @@ pivot_status_t run_scan(int kind, int dtype, int H, int D, const void* qbase, lo
     p.S = S;
     p.S_stride = stride;
     const int nblocks = ceil_div(p.nrows, P);
-    const int nt = ceil_div(maxlim_total + 1, 128);
+    const int kts = p.key_tile_stride > 1 ? p.key_tile_stride : 1;
+    const int nt = ceil_div(ceil_div(maxlim_total + 1, 128), kts);
     const int N = P * H;
     if (umma_shape_ok(H, D, dtype) && N >= 16 && N <= 256 && N % 16 == 0) {
         const bool decode = kind == SCAN_DECODE_DENSE || kind == SCAN_DECODE_PROXY;
-        p.tiles_per_item = decode ? 8 : 32;
+        p.tiles_per_item = decode ? 8 : FUSED_TILES;
         p.items_per_block = ceil_div(nt, p.tiles_per_item);
         p.nitems = nblocks * p.items_per_block;
         CUtensorMap tk, tq;
         if (!make_tmap(&tk, dtype, kbase, k_rows, D, 128)) return PIVOT_ERR_CUDA;
         if (!make_tmap(&tq, dtype, qbase, q_rows * H, D, P * H)) return PIVOT_ERR_CUDA;
         const int grid = p.nitems < num_sms() ? p.nitems : num_sms();
-        return from_cuda(profiled(PK_SCAN, scan_pairs(kind, r0, r1, L, g), st,
+        return from_cuda(profiled(PK_SCAN, work, st,
                                   [&] { return launch_scan_umma(tk, tq, p, grid, st); }));
     }
+    if (x && (x->surv || x->key_tile_stride > 1 || x->row_list)) return PIVOT_ERR_UNSUPPORTED;
     p.tiles_per_item = 1;
     p.items_per_block = nt;
     p.nitems = nblocks * nt;
@@ -423,6 +457,155 @@ struct Carver {
 // after all score rows of the chunk).
 size_t dense_rowbytes(int L) { return (size_t)score_stride(L) * 4 + 4; }
 
+// ------------------------------------------------------------ fused selection
+// Prefix rows (dense queries, proxies) whose top-K is taken inside the scan:
+// a sample scan over every FUSED_KTS-th key tile, a bound per row, the
+// filter-mode scan appending the scores at or above it, one warp per row
+// selecting among them, and -- for rows whose survivors miss the warp
+// select's range -- a keep-everything rescan of just those rows and the
+// block select on their keys.  The scores themselves never reach memory.
+bool g_fused_on = true;
+float g_fused_sigmas = 4.5f;
+
+bool fused_ok(int H, int D, int dtype, int K) {
+    return g_fused_on && umma_shape_ok(H, D, dtype) && H >= 32 && K <= MAX_K;
+}
+int fused_tiles(int L) { return ceil_div(L, 128); }
+long long fused_samp_stride(int L) { return (long long)ceil_div(fused_tiles(L), FUSED_KTS) * 128; }
+int fused_nchunks(int L) { return ceil_div(fused_tiles(L), FUSED_TILES); }
+long long fused_surv_stride(int L) { return (long long)fused_nchunks(L) * FUSED_TILES * 128; }
+// per row: samples, survivor regions, chunk counts, the bound, a miss slot
+size_t fused_rowbytes(int L) {
+    return (size_t)fused_samp_stride(L) * 4 + (size_t)fused_surv_stride(L) * 8 +
+           (size_t)fused_nchunks(L) * 4 + 4 + 4;
+}
+constexpr size_t FUSED_FIXED = 8 * WS_ALIGN;   // alignment of the six arrays, the miss count
+
+struct FusedWs {
+    float* samp;
+    uint64_t* surv;
+    uint32_t* count;
+    uint32_t* bound;
+    int32_t* miss;
+    uint32_t* nmiss;
+};
+
+bool fused_carve(void* ws, size_t bytes, long long rows, int L, FusedWs* w) {
+    Carver c{static_cast<uint8_t*>(ws), bytes};
+    w->samp = static_cast<float*>(c.take((size_t)rows * fused_samp_stride(L) * 4));
+    w->surv = static_cast<uint64_t*>(c.take((size_t)rows * fused_surv_stride(L) * 8));
+    w->count = static_cast<uint32_t*>(c.take((size_t)rows * fused_nchunks(L) * 4));
+    w->bound = static_cast<uint32_t*>(c.take((size_t)rows * 4));
+    w->miss = static_cast<int32_t*>(c.take((size_t)rows * 4));
+    w->nmiss = static_cast<uint32_t*>(c.take(4));
+    return c.ok;
+}
+
+// Rows a launch of the fused path takes from `bytes` of workspace.
+long long fused_chunk_rows(size_t bytes, int L, long long total, int P) {
+    return chunk_rows(bytes > FUSED_FIXED ? bytes - FUSED_FIXED : 0, fused_rowbytes(L), total, P);
+}
+
+// The top K of prefix rows [r0, r1) of `kind` (SCAN_PREFILL_DENSE: rows of
+// seq->q; SCAN_PREFILL_PROXY: rows of the proxies `qbase`), written like
+// run_select_prefix writes them.
+pivot_status_t run_prefix_fused(int kind, const pivot_seq_t* seq, const void* qbase,
+                                long long q_rows, int qrow_base, const float* w,
+                                const float* q_scale, int g, int P, int r0, int r1, int maxlim,
+                                int K, int split, int32_t* out, float* out_score, int out_base,
+                                int lim_shift, int out_stride, const FusedWs& fw,
+                                cudaStream_t s) {
+    const int L = seq->L;
+    const double pairs = scan_pairs(kind, r0, r1, L, g);
+    // 1. samples
+    ScanExtra xs;
+    xs.key_tile_stride = FUSED_KTS;
+    xs.work = pairs / FUSED_KTS;
+    pivot_status_t st =
+        run_scan(kind, seq->dtype, seq->H, seq->D, qbase, q_rows, qrow_base, w, q_scale, seq->k,
+                 L, seq->k_scale, L, g, 1, 0, nullptr, P, r0, r1, maxlim, fw.samp,
+                 fused_samp_stride(L), s, &xs);
+    if (st != PIVOT_OK) return st;
+    // 2. bounds
+    FusedSelectParams fp{};
+    fp.scan_kind = kind;
+    fp.row0 = r0;
+    fp.nrows = r1 - r0;
+    fp.L = L;
+    fp.g = g;
+    fp.lim_shift = lim_shift;
+    fp.K = K;
+    fp.split = split;
+    fp.rank_order = t_rank_order;
+    fp.samp = fw.samp;
+    fp.samp_stride = fused_samp_stride(L);
+    fp.kts = FUSED_KTS;
+    fp.sigmas = g_fused_sigmas;
+    fp.bound = fw.bound;
+    fp.cap = fused_cap(K);
+    fp.surv = fw.surv;
+    fp.surv_stride = fused_surv_stride(L);
+    fp.surv_count = fw.count;
+    fp.nchunks = fused_nchunks(L);
+    fp.chunk_keys = FUSED_TILES * 128;
+    fp.out_idx = out;
+    fp.out_score = out_score;
+    fp.out_base = out_base;
+    fp.out_stride = out_stride;
+    fp.miss_list = fw.miss;
+    fp.miss_count = fw.nmiss;
+    st = from_cuda(profiled(PK_SELECT, 0.0, s, [&] { return launch_sample_bound(fp, s); }));
+    if (st != PIVOT_OK) return st;
+    // 3. the scan, keeping the scores at or above each row's bound
+    ScanExtra xf;
+    xf.bound = fw.bound;
+    xf.surv = fw.surv;
+    xf.surv_stride = fused_surv_stride(L);
+    xf.surv_count = fw.count;
+    xf.nchunks = fused_nchunks(L);
+    xf.lim_shift = lim_shift;
+    xf.work = pairs;
+    st = run_scan(kind, seq->dtype, seq->H, seq->D, qbase, q_rows, qrow_base, w, q_scale, seq->k,
+                  L, seq->k_scale, L, g, 1, 0, nullptr, P, r0, r1, maxlim, nullptr, 0, s, &xf);
+    if (st != PIVOT_OK) return st;
+    // 4. the top K of every row's survivors
+    st = from_cuda(profiled(PK_SELECT, 0.0, s, [&] { return launch_fused_finish(fp, s); }));
+    if (st != PIVOT_OK) return st;
+    // 5. rows that missed: rescan keeping every score (one row a block) ...
+    ScanExtra xr = xf;
+    xr.bound = nullptr;
+    xr.row_list = fw.miss;
+    xr.row_count = fw.nmiss;
+    xr.work = 0.0;
+    st = run_scan(kind, seq->dtype, seq->H, seq->D, qbase, q_rows, qrow_base, w, q_scale, seq->k,
+                  L, seq->k_scale, L, g, 1, 0, nullptr, 1, r0, r1, maxlim, nullptr, 0, s, &xr);
+    if (st != PIVOT_OK) return st;
+    // 6. ... and select on their keys
+    SelectParams sp{};
+    sp.kind = SEL_PREFIX;
+    sp.scan_kind = kind;
+    sp.row0 = r0;
+    sp.nrows = r1 - r0;
+    sp.L = L;
+    sp.g = g;
+    sp.Gm = 1;
+    sp.keys = fw.surv;
+    sp.S_stride = fused_surv_stride(L);
+    sp.K = K;
+    sp.split = split;
+    sp.npos = L;
+    sp.out_idx = out;
+    sp.out_score = out_score;
+    sp.out_base = out_base;
+    sp.out_stride = out_stride;
+    sp.lim_shift = lim_shift;
+    sp.tail_cap = TAIL_CAP;
+    sp.rank_order = t_rank_order;
+    sp.row_list = fw.miss;
+    sp.row_count = fw.nmiss;
+    return from_cuda(profiled(PK_SELECT, 0.0, s, [&] { return launch_select(sp, s); }));
+}
+
 // One thread waits on an mbarrier that nothing arrives on: the bounded wait
 // must run out, raise the timeout bit and let the kernel return.
 __global__ void wait_selftest_kernel() {
@@ -488,6 +671,14 @@ pivot_status_t pivot_set_wait_limit_ns(uint64_t ns) {
                                                                             : PIVOT_ERR_CUDA;
 }
 
+pivot_status_t pivot_set_fused_selection(int32_t on, float margin_sigmas) {
+    if ((on != 0 && on != 1) || !(margin_sigmas > -1e6f && margin_sigmas < 1e6f))
+        return PIVOT_ERR_INVALID_ARG;
+    g_fused_on = on != 0;
+    g_fused_sigmas = margin_sigmas;
+    return PIVOT_OK;
+}
+
 pivot_status_t pivot_set_score_buffer_cap(size_t bytes) {
     if (bytes != 0 && bytes < 4096) return PIVOT_ERR_INVALID_ARG;
     g_score_buf_cap = bytes ? bytes : SCORE_BUF_DEFAULT;
@@ -504,6 +695,14 @@ size_t pivot_dense_index_workspace_size(const pivot_seq_t* seq, int32_t topk) {
     int t0, t1;
     if (check_seq(seq, &t0, &t1) != PIVOT_OK || topk < 1) return 0;
     const int P = rows_per_block(seq->H, seq->D, seq->dtype);
+    if (fused_ok(seq->H, seq->D, seq->dtype, topk)) {
+        const size_t rb = fused_rowbytes(seq->L);
+        long long rows = t1 - t0;
+        long long cap = (long long)(g_score_buf_cap / rb) / P * P;
+        if (cap < 1) cap = 1;
+        if (rows > cap) rows = cap;
+        return align_up((size_t)rows * rb + FUSED_FIXED, WS_ALIGN);
+    }
     const size_t rb = dense_rowbytes(seq->L);
     long long rows = t1 - t0;
     long long cap = (long long)(g_score_buf_cap / rb) / P * P;
@@ -524,10 +723,24 @@ static pivot_status_t dense_index_impl(const pivot_seq_t* seq, int32_t topk, int
     if (topk > MAX_K) return PIVOT_ERR_UNSUPPORTED;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
     const int P = rows_per_block(seq->H, seq->D, seq->dtype);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (fused_ok(seq->H, seq->D, seq->dtype, topk)) {
+        const long long chunk = fused_chunk_rows(ws_bytes, seq->L, t1 - t0, P);
+        FusedWs fw;
+        if (chunk < 1 || !fused_carve(ws, ws_bytes, chunk, seq->L, &fw)) return PIVOT_ERR_WORKSPACE;
+        for (long long c0 = t0; c0 < t1; c0 += chunk) {
+            const int r0 = (int)c0;
+            const int r1 = (int)(c0 + chunk < t1 ? c0 + chunk : t1);
+            st = run_prefix_fused(SCAN_PREFILL_DENSE, seq, seq->q, seq->L, 0, seq->w, seq->q_scale,
+                                  1, P, r0, r1, r1 - 1, topk, 0, idx, score, t0, lim_shift,
+                                  out_stride, fw, s);
+            if (st != PIVOT_OK) return st;
+        }
+        return PIVOT_OK;
+    }
     const long long stride = score_stride(seq->L);
     const long long chunk = chunk_rows(ws_bytes, dense_rowbytes(seq->L), t1 - t0, P);
     if (chunk < 1) return PIVOT_ERR_WORKSPACE;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* S = static_cast<float*>(ws);
     uint32_t* thresh = reinterpret_cast<uint32_t*>(S + chunk * stride);
     for (long long c0 = t0; c0 < t1; c0 += chunk) {
@@ -584,6 +797,14 @@ size_t pivot_proxy_scan_workspace_size(const pivot_seq_t* seq, int32_t g, int32_
     int t0, t1;
     if (check_seq(seq, &t0, &t1) != PIVOT_OK || g < 1 || C < 1) return 0;
     const int P = rows_per_block(seq->H, seq->D, seq->dtype);
+    if (fused_ok(seq->H, seq->D, seq->dtype, C)) {
+        const size_t rb = fused_rowbytes(seq->L);
+        long long rows = ceil_div(t1 - t0, g);
+        long long cap = (long long)(g_score_buf_cap / rb) / P * P;
+        if (cap < 1) cap = 1;
+        if (rows > cap) rows = cap;
+        return align_up((size_t)rows * rb + FUSED_FIXED, WS_ALIGN);
+    }
     const size_t rb = dense_rowbytes(seq->L);
     long long rows = ceil_div(t1 - t0, g);
     long long cap = (long long)(g_score_buf_cap / rb) / P * P;
@@ -609,10 +830,24 @@ pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* p
     const int P = rows_per_block(seq->H, seq->D, seq->dtype);
     const long long stride = score_stride(seq->L);
     const int j0 = t0 / g, j1 = ceil_div(t1, g);
-    const long long chunk = chunk_rows(ws_bytes, dense_rowbytes(seq->L), j1 - j0, P);
-    if (chunk < 1) return PIVOT_ERR_WORKSPACE;
     const int G = j1 - j0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (fused_ok(seq->H, seq->D, seq->dtype, C)) {
+        const long long chunk = fused_chunk_rows(ws_bytes, seq->L, j1 - j0, P);
+        FusedWs fw;
+        if (chunk < 1 || !fused_carve(ws, ws_bytes, chunk, seq->L, &fw)) return PIVOT_ERR_WORKSPACE;
+        for (long long c0 = j0; c0 < j1; c0 += chunk) {
+            const int r0 = (int)c0;
+            const int r1 = (int)(c0 + chunk < j1 ? c0 + chunk : j1);
+            const int e_last = (r1 * g < seq->L ? r1 * g : seq->L) - 1;
+            st = run_prefix_fused(SCAN_PREFILL_PROXY, seq, pq, G, j0, pw, pq_scale, g, P, r0, r1,
+                                  e_last, C, topk, cand, cand_score, j0, 0, 0, fw, s);
+            if (st != PIVOT_OK) return st;
+        }
+        return PIVOT_OK;
+    }
+    const long long chunk = chunk_rows(ws_bytes, dense_rowbytes(seq->L), j1 - j0, P);
+    if (chunk < 1) return PIVOT_ERR_WORKSPACE;
     float* S = static_cast<float*>(ws);
     uint32_t* thresh = reinterpret_cast<uint32_t*>(S + chunk * stride);
     for (long long c0 = j0; c0 < j1; c0 += chunk) {

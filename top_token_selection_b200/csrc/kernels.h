@@ -44,6 +44,26 @@ struct ScanParams {
     int nkeys;              // key positions per sequence (L, or maxlen in decode)
     const void* kbase;      // gather mode: key rows (stored format), row stride D*esize
     SegTable seg;           // SCAN_VARLEN_*: the batch's sequences (rows, keys packed)
+    // Sample scan: key tile t of a row is key tile t * key_tile_stride of its
+    // prefix; its scores go to columns t*128 + (key in tile).  0 or 1: every tile.
+    int key_tile_stride;
+    // Filter mode (surv set; the selection fused into the scan): a score
+    // >= its row's bound is appended, as a 64-bit key (ordered score << 32 |
+    // ~position), to the row's region for the item's key chunk -- row r,
+    // chunk c at surv + (r - row0) * surv_stride + c * tiles_per_item * 128 --
+    // and the chunk's count goes to surv_count[(r - row0) * nchunks + c].  No
+    // score is written to S.
+    const uint32_t* bound;  // [nrows]: row r's bound (an ordered key) at bound[r - row0];
+                            // keys <= 0x00800000 keep every score; NULL keeps every score
+    uint64_t* surv;
+    long long surv_stride;
+    uint32_t* surv_count;
+    int nchunks;
+    int lim_shift;          // filter mode: positions kept are <= lim(r) - lim_shift
+    // Row-list mode (row_list set): the launch's rows are row_list[0, *row_count),
+    // one row a block (P = 1); prefill kinds only.
+    const int32_t* row_list;
+    const uint32_t* row_count;
 };
 
 int scan_smem_bytes(int row_bytes);
@@ -91,7 +111,52 @@ struct SelectParams {
                               // from the sequence's first token
     int rank_order;           // 1: rows in rank order (score descending, then position
                               // ascending; `split` is then moot); 0: ascending positions
+    // SEL_PREFIX rows whose entries are 64-bit keys (ordered score << 32 |
+    // ~position) instead of scores: row r's n = lim + 1 keys at
+    // keys + (r - row0) * S_stride (the fused scan's regions, every key kept)
+    const uint64_t* keys;
+    // Row list: block b selects row row_list[b] when b < *row_count (and
+    // does nothing otherwise)
+    const int32_t* row_list;
+    const uint32_t* row_count;
 };
+
+// The selection fused into the scan (prefill dense and proxy rows): a sample
+// scan gives each row a bound, the filter-mode scan keeps the scores at or
+// above it, and one warp per row selects the top K among them.
+struct FusedSelectParams {
+    int scan_kind;            // SCAN_PREFILL_DENSE or SCAN_PREFILL_PROXY
+    int row0, nrows, L, g;
+    int lim_shift;            // positions considered are <= lim(r) - lim_shift
+    int K, split, rank_order;
+    // samples: row r's sample scores at samp + (r - row0) * samp_stride,
+    // column j = key position (j / 128) * kts * 128 + j % 128
+    const float* samp;
+    long long samp_stride;
+    int kts;
+    float sigmas;             // margin of the bound, in standard deviations of the count
+    uint32_t* bound;          // [nrows] out: row r's bound (an ordered key; 1 keeps all)
+    int cap;                  // survivors a row may have for the warp select
+    // survivors: row r, chunk c at surv + (r - row0) * surv_stride + c * chunk_keys,
+    // surv_count[(r - row0) * nchunks + c] of them
+    const uint64_t* surv;
+    long long surv_stride;
+    const uint32_t* surv_count;
+    int nchunks, chunk_keys;
+    int32_t* out_idx;         // row r at out_idx + (r - out_base) * (out_stride or K)
+    float* out_score;         // or NULL
+    int out_base, out_stride;
+    int32_t* miss_list;       // rows whose survivors fell outside [min(K, n), cap]
+    uint32_t* miss_count;     // zeroed by the bound kernel
+};
+// Bound of every row (one warp per row) and a zeroed miss count.
+cudaError_t launch_sample_bound(const FusedSelectParams& p, cudaStream_t stream);
+// Top K of every row's survivors (one warp per row); rows that miss go to the
+// list for the fallback (a keep-everything rescan and launch_select on keys).
+cudaError_t launch_fused_finish(const FusedSelectParams& p, cudaStream_t stream);
+// Survivor capacity a row may have for K (entries), and the shared memory
+// that needs per warp.
+int fused_cap(int K);
 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
 // SEL_PREFIX rows: per-row lower bound for the select's fast path, written

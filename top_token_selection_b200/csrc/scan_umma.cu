@@ -75,6 +75,7 @@ __device__ __forceinline__ int scan_key_base(const ScanParams& p, int r) {
 
 struct ItemInfo {
     int rows, row_first, t0, t1, keybase, maxlim;
+    int chunk;             // scan mode: the item's chunk of key tiles
     int nkeys;             // gather mode: key rows of the item's sequence
     const int32_t* cand;   // gather mode: this group's candidate row
     bool valid;
@@ -89,7 +90,26 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
     ItemInfo it;
     if constexpr (!GATHER) {
         int chunk;
-        if (p.kind == SCAN_VARLEN_DENSE || p.kind == SCAN_VARLEN_PROXY) {
+        if (p.row_list) {
+            // one listed row per block; slots past the device count are empty
+            const int slot = item / p.items_per_block;
+            chunk = item % p.items_per_block;
+            if ((uint32_t)slot >= *p.row_count) {
+                it.valid = false;
+                it.rows = 0;
+                it.row_first = p.row0;
+                it.t0 = it.t1 = 0;
+                it.maxlim = -1;
+                it.nkeys = 0;
+                it.keybase = 0;
+                it.chunk = chunk;
+                it.cand = nullptr;
+                return it;
+            }
+            it.row_first = p.row_list[slot];
+            it.rows = 1;
+            it.keybase = 0;
+        } else if (p.kind == SCAN_VARLEN_DENSE || p.kind == SCAN_VARLEN_PROXY) {
             // blocks never straddle two sequences: each is one sequence's;
             // rows outside the launch's [row0, row0 + nrows) are dropped
             const SegItem si = seg_scan_item(
@@ -103,6 +123,7 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
                 it.t0 = it.t1 = 0;
                 it.maxlim = -1;
                 it.nkeys = 0;
+                it.chunk = chunk;
                 it.cand = nullptr;
                 return it;
             }
@@ -118,7 +139,11 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
         const int maxlim = scan_row_lim(p, it.row_first + it.rows - 1, ok);
         it.maxlim = ok ? maxlim : -1;
         it.nkeys = 0;
-        const int nt = ok ? (maxlim + 1 + 127) / 128 : 0;
+        it.chunk = chunk;
+        // key tiles of the block's longest prefix (sample scan: every
+        // key_tile_stride-th of them)
+        const int kts = p.key_tile_stride > 1 ? p.key_tile_stride : 1;
+        const int nt = ok ? ((maxlim + 1 + 127) / 128 + kts - 1) / kts : 0;
         it.t0 = chunk * p.tiles_per_item;
         it.t1 = it.t0 + p.tiles_per_item < nt ? it.t0 + p.tiles_per_item : nt;
         it.valid = it.t0 < nt;
@@ -145,6 +170,7 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
             it.nkeys = p.nkeys;
         }
         it.maxlim = it.nkeys - 1;
+        it.chunk = 0;
         it.t0 = 0;
         it.t1 = (p.C + 127) / 128;
         it.valid = it.rows > 0;
@@ -153,7 +179,7 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
     return it;
 }
 
-template <int KIND, int HEADS, int ROWB, bool GATHER>
+template <int KIND, int HEADS, int ROWB, bool GATHER, bool FILTER>
 __global__ void __maxnreg__(SCAN_MAXREG)
     index_umma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
@@ -183,11 +209,15 @@ __global__ void __maxnreg__(SCAN_MAXREG)
     float* w_s = reinterpret_cast<float*>(tmem_holder + 4);   // [256], 16-byte aligned
     float* sq_s = w_s + 256;                                   // [PMAX]
     int* lim_s = reinterpret_cast<int*>(sq_s + PMAX);          // [PMAX]
+    // filter mode: survivors of each row of the current item, double-
+    // buffered by the epilogue's item parity
+    uint32_t* cnt_s = reinterpret_cast<uint32_t*>(lim_s + PMAX);   // [2][PMAX]
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const int N = p.P * HEADS;
 
+    for (int i = threadIdx.x; i < 2 * PMAX; i += blockDim.x) cnt_s[i] = 0;
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&full[i], 1);
@@ -242,9 +272,10 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                         if (!mbar_wait(&empty[stage], phase ^ 1)) { aborted = true; break; }
                         mbar_arrive_expect_tx(&full[stage], (uint32_t)A_BYTES);
                         last_a[stage] = (int)phase;
+                        const int kt = p.key_tile_stride > 1 ? t * p.key_tile_stride : t;
                         for (int kb = 0; kb < KBLK; ++kb)
                             tma_load_2d(sA + stage * A_BYTES + kb * (128 * 128), &tmap_k,
-                                        &full[stage], kb * (128 / p.esize), it.keybase + t * 128);
+                                        &full[stage], kb * (128 / p.esize), it.keybase + kt * 128);
                         if (++stage == STAGES) { stage = 0; phase ^= 1; }
                     }
                     ++nit;
@@ -435,7 +466,11 @@ __global__ void __maxnreg__(SCAN_MAXREG)
         float wr[HEADS >= 32 ? 64 : 1];
         int lim_r[RROWS];
         float sq_r[RROWS];
+        float tf_r[RROWS];    // filter mode: scores >= tf_r are kept
         int ntile = 0;
+        int nit_e = 0;        // valid items this CTA's epilogue has walked
+        const int kts = p.key_tile_stride > 1 ? p.key_tile_stride : 1;
+        constexpr bool filter = FILTER && !GATHER && HEADS >= 32;
         // Once a wait runs out the warp stops touching TMEM and memory but
         // keeps walking the items, so the named barriers shared by the
         // epilogue warps are always reached.
@@ -475,6 +510,11 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                     }
                     lim_r[lr] = pr < r_hi ? row_lim(pr) : -1;
                     sq_r[lr] = row_sq(pr);
+                    tf_r[lr] = -INFINITY;
+                    if (filter && live && p.bound) {
+                        const uint32_t T = p.bound[it.row_first + pr - p.row0];
+                        if (T > 0x00800000u) tf_r[lr] = key_to_float(T);
+                    }
                 }
             } else {
                 named_bar_sync(1, EPI_WARPS * 32);
@@ -500,9 +540,10 @@ __global__ void __maxnreg__(SCAN_MAXREG)
             // loads on every tile and halved the rate.
             auto key_scale = [&](int t) -> float {
                 if (GATHER || !p.k_scale) return 1.0f;
-                const int s_t = t * 128 + key_in_tile;
+                const int s_t = t * kts * 128 + key_in_tile;
                 return s_t <= it.maxlim ? ld_nc_early(p.k_scale + it.keybase + s_t) : 1.0f;
             };
+            uint32_t* cnt_cur = cnt_s + (nit_e & 1) * PMAX;
             float sk_next = key_scale(it.t0);
             for (int t = it.t0; t < it.t1; ++t) {
                 const int acc = ntile & 1;
@@ -514,9 +555,11 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 const bool got = mbar_wait(&accfull[acc], aph);
                 if (!__all_sync(0xffffffffu, got)) { aborted = true; continue; }
                 tc_fence_after();
-                // s: the output column (key position in scan mode, candidate
-                // slot in gather mode)
+                // s: the output column (key position in scan mode, sample
+                // index in the sample scan, candidate slot in gather mode);
+                // spos: the key position the causal limit applies to
                 const int s = t * 128 + key_in_tile;
+                const int spos = kts > 1 ? t * kts * 128 + key_in_tile : s;
                 const bool col_ok = GATHER ? (s < p.C) : true;
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * 256);
@@ -556,9 +599,31 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                         for (int j = 0; j < 4; ++j) unpack2(a[j], lo[j], hi[j]);
                         const float rowsum = ((lo[0] + hi[0]) + (lo[1] + hi[1])) +
                                              ((lo[2] + hi[2]) + (lo[3] + hi[3]));
-                        if (col_ok && s <= lim_r[lr])   // streaming store: keep L2 for the keys
+                        const float score = rowsum * sq_r[lr] * sk;
+                        if constexpr (filter) {
+                            // survivors only: warp-aggregated append to the
+                            // row's region for this chunk
+                            const bool keep = spos <= lim_r[lr] - p.lim_shift &&
+                                              score >= tf_r[lr];
+                            const unsigned m = __ballot_sync(0xffffffffu, keep);
+                            if (m) {
+                                const int leader = __ffs(m) - 1;
+                                uint32_t base = 0;
+                                if (lane == leader) base = atomicAdd(&cnt_cur[pr], (uint32_t)__popc(m));
+                                base = __shfl_sync(0xffffffffu, base, leader);
+                                if (keep) {
+                                    const uint32_t u = ordered_key(score);
+                                    p.surv[(size_t)(it.row_first + pr - p.row0) * p.surv_stride +
+                                           (size_t)it.chunk * (p.tiles_per_item * 128) + base +
+                                           __popc(m & ((1u << lane) - 1u))] =
+                                        ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)spos);
+                                }
+                            }
+                        } else if (col_ok && spos <= lim_r[lr]) {
+                            // streaming store: keep L2 for the keys
                             __stcs(p.S + (size_t)(it.row_first + pr - p.row0) * p.S_stride + s,
-                                   rowsum * sq_r[lr] * sk);
+                                   score);
+                        }
                     }
                 } else {
                     if (r_hi > 0) {
@@ -573,7 +638,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                                 rowacc = fmaf(w_s[c0 + i], fmaxf(v[i], 0.0f), rowacc);
                                 if ((i + 1) % HEADS == 0) {
                                     const int pr = (c0 + i) / HEADS;
-                                    if (col_ok && s <= lim_s[pr])
+                                    if (col_ok && spos <= lim_s[pr])
                                         __stcs(p.S + (size_t)(it.row_first + pr - p.row0) *
                                                          p.S_stride + s,
                                                rowacc * sq_s[pr] * sk);
@@ -587,6 +652,17 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&accempty[acc]);
             }
+            if constexpr (filter) {
+                // every append of this item has counted: publish the rows'
+                // counts, and clear this buffer for item nit_e + 2 (the next
+                // item uses the other one)
+                named_bar_sync(2, EPI_WARPS * 32);
+                if (et < it.rows && !aborted)
+                    p.surv_count[(size_t)(it.row_first + et - p.row0) * p.nchunks + it.chunk] =
+                        cnt_cur[et];
+                if (et < PMAX) cnt_cur[et] = 0;
+            }
+            ++nit_e;
         }
     }
 
@@ -602,7 +678,7 @@ int scan_smem_bytes(int row_bytes) {
     const int stages = row_bytes == 128 ? 6 : 3;
     const int pmax = 64;
     return 1024 /*align slack*/ + 2 * 256 * row_bytes + stages * 128 * row_bytes +
-           256 /*barriers*/ + 16 /*TMEM address*/ + 256 * 4 + pmax * 8;
+           256 /*barriers*/ + 16 /*TMEM address*/ + 256 * 4 + pmax * 8 + 2 * pmax * 4;
 }
 
 // The epilogue's three warp groups take ceil(P / 3) rows each, with room
@@ -613,24 +689,31 @@ inline bool epilogue_fits(int P, int heads) {
     return heads >= 32 ? (P + 2) / 3 <= 64 / heads : true;
 }
 
+template <int KIND, int HEADS, int ROWB, bool GATHER, bool FILTER>
+static cudaError_t launch_one(const CUtensorMap& tk, const CUtensorMap& tq, const ScanParams& p,
+                              int grid, cudaStream_t stream) {
+    auto kfn = index_umma_kernel<KIND, HEADS, ROWB, GATHER, FILTER>;
+    const int smem = scan_smem_bytes(ROWB);
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kfn<<<grid, SCAN_THREADS, smem, stream>>>(tk, tq, p);
+    return cudaGetLastError();
+}
+
 template <int KIND, int HEADS, bool GATHER>
 static cudaError_t launch_heads(const CUtensorMap& tk, const CUtensorMap& tq, const ScanParams& p,
                                 int row_bytes, int grid, cudaStream_t stream) {
     if (!epilogue_fits(p.P, HEADS)) return cudaErrorInvalidValue;
-    if (row_bytes == 128) {
-        auto kfn = index_umma_kernel<KIND, HEADS, 128, GATHER>;
-        const int smem = scan_smem_bytes(128);
-        cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        kfn<<<grid, SCAN_THREADS, smem, stream>>>(tk, tq, p);
-    } else {
-        auto kfn = index_umma_kernel<KIND, HEADS, 256, GATHER>;
-        const int smem = scan_smem_bytes(256);
-        cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        kfn<<<grid, SCAN_THREADS, smem, stream>>>(tk, tq, p);
+    // the fused selection runs in the register-resident epilogue (H >= 32)
+    const bool filter = !GATHER && p.surv != nullptr;
+    if (filter && HEADS < 32) return cudaErrorInvalidValue;
+    if constexpr (!GATHER && HEADS >= 32) {
+        if (filter)
+            return row_bytes == 128 ? launch_one<KIND, HEADS, 128, false, true>(tk, tq, p, grid, stream)
+                                    : launch_one<KIND, HEADS, 256, false, true>(tk, tq, p, grid, stream);
     }
-    return cudaGetLastError();
+    return row_bytes == 128 ? launch_one<KIND, HEADS, 128, GATHER, false>(tk, tq, p, grid, stream)
+                            : launch_one<KIND, HEADS, 256, GATHER, false>(tk, tq, p, grid, stream);
 }
 
 template <int KIND, bool GATHER>

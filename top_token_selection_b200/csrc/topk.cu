@@ -74,6 +74,7 @@ struct RowView {
     const float* S;
     const int32_t* cand;   // null: position = entry index
     const float* ksc;      // candidate rows: score = S[i] * ksc[position], or null
+    const uint64_t* keys;  // or: entry i is the full key keys[i] (S, cand unused)
     int n;                 // entries
     int lim;               // valid positions are <= lim
 };
@@ -91,7 +92,16 @@ __device__ __forceinline__ uint32_t key_upos(uint64_t k) {
 }
 
 // Key of entry i, or 0 when the entry is not eligible.
+// A key whose position lies outside [0, lim] is an empty entry (the keep-
+// everything rescan writes none; only a rescan that gave up leaves them).
+__device__ __forceinline__ uint64_t listed_key(const RowView& v, int i) {
+    const uint64_t k = v.keys[i];
+    const int pos = key_pos(k);
+    return (pos >= 0 && pos <= v.lim) ? k : 0ull;
+}
+
 __device__ __forceinline__ uint64_t entry_key(const RowView& v, int i) {
+    if (v.keys) return listed_key(v, i);
     int pos = i;
     float x = v.S[i];
     if (v.cand) {
@@ -102,6 +112,7 @@ __device__ __forceinline__ uint64_t entry_key(const RowView& v, int i) {
     return make_key(ordered_key(x), pos);
 }
 __device__ __forceinline__ uint32_t entry_key32(const RowView& v, int i) {
+    if (v.keys) return key_u(listed_key(v, i));
     float x = v.S[i];
     if (v.cand) {
         const int pos = v.cand[i];
@@ -426,7 +437,8 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
     __syncthreads();
     // filtering pass
     uint32_t nvalid_local = 0;
-    const bool vec = (v.cand == nullptr) && ((reinterpret_cast<uintptr_t>(v.S) & 15) == 0);
+    const bool vec = (v.cand == nullptr) && !v.keys &&
+                     ((reinterpret_cast<uintptr_t>(v.S) & 15) == 0);
     if (vec) {
         const int n4 = v.n / 4;
         const float4* S4 = reinterpret_cast<const float4*>(v.S);
@@ -507,8 +519,14 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
             uint32_t u = 0;
             int pos = i;
             if (i < v.n) {
-                u = entry_key32(v, i);
-                if (v.cand) pos = v.cand[i];
+                if (v.keys) {
+                    const uint64_t k = listed_key(v, i);
+                    u = key_u(k);
+                    pos = k ? key_pos(k) : 0;
+                } else {
+                    u = entry_key32(v, i);
+                    if (v.cand) pos = v.cand[i];
+                }
             }
             nvalid_local += (u != 0);
             warp_append(buf, s_cnt, cap, make_key(u, pos), u != 0 && u >= T);
@@ -1076,6 +1094,209 @@ __global__ void __launch_bounds__(CW_MAX_WARPS * 32) select_cand_kernel(const Se
     }
 }
 
+// ------------------------------------------------------------ fused selection
+//
+// Prefix rows whose scan ran in filter mode.  A sample scan scored every
+// kts-th key tile of each row; the bound of a row is the m-th largest of its
+// samples, m = m0 + 4.5 sqrt(m0) with m0 = K * (samples) / (row length) the
+// samples expected at or above the row's K-th score (4.5 is the default
+// margin) -- so, for keys in random order, at least K and about
+// K (1 + 4.5 / sqrt(m0)) entries of the row lie
+// at or above it, far from the warp select's capacity.  Rows no longer than
+// the capacity keep everything (bound 1).  The filter-mode scan appended every
+// score at or above the bound; one warp per row then takes the exact top K of
+// those survivors -- provided at least min(K, n) and at most `cap` survived
+// (else the row goes on the miss list, and the fallback rescans it keeping
+// everything and selects with the block select).  Every row that passes holds
+// all of its entries at or above its K-th score among the survivors, so its
+// answer is exact.
+
+constexpr int FB_WARPS = 8;              // bound kernel: rows a block
+constexpr int FB_MAX_SAMPLES = 4096;     // samples a bound reads at most
+constexpr int FF_MAX_WARPS = 8;
+
+__device__ __forceinline__ int prefill_lim(int kind, int r, int L, int g) {
+    if (kind == SCAN_PREFILL_PROXY) {
+        const int e = (r + 1) * g;
+        return (e < L ? e : L) - 1;
+    }
+    return r;
+}
+
+// Sample columns at positions <= lim (sample j sits at position
+// (j / 128) * kts * 128 + j % 128).
+__device__ __forceinline__ int samples_upto(int lim, int kts) {
+    if (lim < 0) return 0;
+    const int span = kts * 128;
+    const int full = lim / span;
+    const int rem = lim - full * span;
+    return full * 128 + (rem < 128 ? rem + 1 : 128);
+}
+
+__global__ void __launch_bounds__(FB_WARPS * 32) sample_bound_kernel(const FusedSelectParams p) {
+    extern __shared__ __align__(16) uint8_t smem_b[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.miss_count = 0;
+    const int rr = blockIdx.x * FB_WARPS + warp;
+    if (rr >= p.nrows) return;
+    uint32_t* v = reinterpret_cast<uint32_t*>(smem_b) + (size_t)warp * (FB_MAX_SAMPLES + THR_BINS);
+    uint32_t* hist = v + FB_MAX_SAMPLES;
+    const int lim = prefill_lim(p.scan_kind, p.row0 + rr, p.L, p.g) - p.lim_shift;
+    const int n = lim + 1;
+    uint32_t T = 1;
+    if (n > p.cap) {
+        const int ns = samples_upto(lim, p.kts);
+        const int step = (ns + FB_MAX_SAMPLES - 1) / FB_MAX_SAMPLES;
+        const int nt = (ns + step - 1) / step;
+        const float* row = p.samp + (size_t)rr * p.samp_stride;
+        for (int j = lane; j < nt; j += 32) v[j] = ordered_key(row[(size_t)j * step]);
+        __syncwarp();
+        const double m0 = (double)p.K * nt / n;
+        long long m = (long long)ceil(m0 + (double)p.sigmas * sqrt(m0));
+        if (m < 1) m = 1;
+        if (m <= nt) T = warp_kth_largest(v, nt, (uint32_t)m, hist);
+        // else: too few samples to bound the row; it keeps everything and
+        // takes the fallback
+    }
+    if (lane == 0) p.bound[rr] = T;
+}
+
+// Among the nonzero keys e[0, n), keep exactly the `keep` largest (score,
+// then lower position) and clear the rest.  Whole warp; keep <= nonzero count.
+__device__ void warp_keep_top(uint64_t* e, int n, uint32_t keep, uint32_t* hist) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t T = warp_kth_largest_f([&](int i) { return key_u(e[i]); }, n, keep, hist);
+    uint32_t above = 0, eq = 0;
+    for (int i = lane; i < n; i += 32) {
+        const uint32_t u = key_u(e[i]);
+        above += u > T;
+        eq += u == T;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        above += __shfl_xor_sync(0xffffffffu, above, o);
+        eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    const uint32_t need = keep - above;
+    uint32_t Lmin = 0;
+    if (eq > need)
+        Lmin = warp_kth_largest_f([&](int i) { return key_u(e[i]) == T ? (uint32_t)e[i] : 0u; },
+                                  n, need, hist);
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+        const uint64_t k = e[i];
+        const uint32_t u = key_u(k);
+        if (u < T || (u == T && (uint32_t)k < Lmin)) e[i] = 0ull;
+    }
+    __syncwarp();
+}
+
+__global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const FusedSelectParams p,
+                                                                         int warps) {
+    extern __shared__ __align__(16) uint8_t smem_f[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rr = blockIdx.x * warps + warp;
+    if (warp >= warps || rr >= p.nrows) return;   // whole warps; no block barriers
+    const int M = p.cap;
+    uint64_t* e = reinterpret_cast<uint64_t*>(smem_f + (size_t)warp * ((size_t)M * 8 + THR_BINS * 4));
+    uint32_t* hist = reinterpret_cast<uint32_t*>(e + M);
+    const int r = p.row0 + rr;
+    const int lim = prefill_lim(p.scan_kind, r, p.L, p.g) - p.lim_shift;
+    const int n = lim >= 0 ? lim + 1 : 0;
+    const int K = p.K;
+    const size_t ostride = p.out_stride ? (size_t)p.out_stride : (size_t)K;
+    int32_t* out = p.out_idx + (size_t)(r - p.out_base) * ostride;
+    float* outs = p.out_score ? p.out_score + (size_t)(r - p.out_base) * ostride : nullptr;
+    const uint32_t Kp = n < K ? (uint32_t)n : (uint32_t)K;
+
+    const int nch = n > 0 ? (n + p.chunk_keys - 1) / p.chunk_keys : 0;
+    const uint32_t* cnt = p.surv_count + (size_t)rr * p.nchunks;
+    // a count above its chunk's size (a scan that gave up left it stale)
+    // counts as a miss, so the gather below stays inside the regions
+    uint32_t total = 0, over = 0;
+    for (int c = lane; c < nch; c += 32) {
+        const uint32_t k = cnt[c];
+        if (k > (uint32_t)p.chunk_keys) over = 1;
+        else total += k;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        total += __shfl_xor_sync(0xffffffffu, total, o);
+        over |= __shfl_xor_sync(0xffffffffu, over, o);
+    }
+    if (over || total < Kp || total > (uint32_t)M) {
+        if (lane == 0) p.miss_list[atomicAdd(p.miss_count, 1u)] = r;
+        return;
+    }
+    if (Kp > 0) {
+        // the row's survivors, chunk after chunk
+        int off = 0;
+        const uint64_t* src = p.surv + (size_t)rr * p.surv_stride;
+        for (int c = 0; c < nch; ++c) {
+            const int k = (int)cnt[c];
+            for (int i = lane; i < k; i += 32) e[off + i] = src[(size_t)c * p.chunk_keys + i];
+            off += k;
+        }
+        __syncwarp();
+        const int nt = (int)total;
+        if (Kp < total) warp_keep_top(e, nt, Kp, hist);
+        // class A (position order with a split): the top `split`
+        const int split = (!p.rank_order && p.split > 0 && (uint32_t)p.split < Kp) ? p.split : 0;
+        uint32_t TA = 0xFFFFFFFFu, LA = 0xFFFFFFFFu;
+        if (split) {
+            TA = warp_kth_largest_f([&](int i) { return key_u(e[i]); }, nt, (uint32_t)split, hist);
+            uint32_t above = 0, eq = 0;
+            for (int i = lane; i < nt; i += 32) {
+                const uint32_t u = key_u(e[i]);
+                above += u > TA;
+                eq += u == TA;
+            }
+            for (int o = 16; o > 0; o >>= 1) {
+                above += __shfl_xor_sync(0xffffffffu, above, o);
+                eq += __shfl_xor_sync(0xffffffffu, eq, o);
+            }
+            const uint32_t need = (uint32_t)split - above;
+            LA = 0;
+            if (eq > need)
+                LA = warp_kth_largest_f(
+                    [&](int i) { return key_u(e[i]) == TA ? (uint32_t)e[i] : 0u; }, nt, need, hist);
+            __syncwarp();
+        }
+        const int kept = warp_compact(e, 0, nt);   // == Kp
+        const int Mk = pow2_at_least(kept);
+        if (p.rank_order) {
+            for (int i = kept + lane; i < Mk; i += 32) e[i] = 0ull;
+            __syncwarp();
+            warp_bitonic(e, Mk, [](uint64_t x, uint64_t y) { return x > y; });
+            for (int i = lane; i < kept; i += 32) {
+                out[i] = key_pos(e[i]);
+                if (outs) outs[i] = key_to_float(key_u(e[i]));
+            }
+        } else {
+            // sort key: class (A first), then position, with the score kept
+            for (int i = lane; i < Mk; i += 32) {
+                if (i < kept) {
+                    const uint64_t k = e[i];
+                    const uint32_t u = key_u(k);
+                    const bool inA = split && (u > TA || (u == TA && (uint32_t)k >= LA));
+                    const uint64_t cls = (split && !inA) ? 1ull : 0ull;
+                    e[i] = (cls << 63) | ((uint64_t)(uint32_t)key_pos(k) << 32) | u;
+                } else {
+                    e[i] = ~0ull;
+                }
+            }
+            __syncwarp();
+            warp_bitonic(e, Mk, [](uint64_t x, uint64_t y) { return x < y; });
+            for (int i = lane; i < kept; i += 32) {
+                out[i] = (int32_t)((e[i] >> 32) & 0x7FFFFFFFu);
+                if (outs) outs[i] = key_to_float((uint32_t)e[i]);
+            }
+        }
+    }
+    for (int i = (int)Kp + lane; i < K; i += 32) {
+        out[i] = -1;
+        if (outs) outs[i] = -INFINITY;
+    }
+}
+
 }  // namespace
 
 // Shared-memory layout, in bytes from the start of the dynamic buffer:
@@ -1110,7 +1331,11 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const SelectParams 
     const int M2 = pow2_at_least(p.K);
     __shared__ uint32_t s_a, s_b;
 
-    const int r = p.row0 + blockIdx.x;
+    int r = p.row0 + blockIdx.x;
+    if (p.row_list) {
+        if (blockIdx.x >= *p.row_count) return;
+        r = p.row_list[blockIdx.x];
+    }
     const size_t ostride = p.out_stride ? (size_t)p.out_stride : (size_t)p.K;
     int32_t* out = p.out_idx + (size_t)(r - p.out_base) * ostride;
     float* outs = p.out_score ? p.out_score + (size_t)(r - p.out_base) * ostride : nullptr;
@@ -1119,7 +1344,8 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const SelectParams 
     const int lim =
         select_row_limit(p, r, ok) - p.lim_shift;
     RowView v;
-    v.S = p.S + (size_t)(r - p.row0) * p.S_stride;
+    v.S = p.keys ? nullptr : p.S + (size_t)(r - p.row0) * p.S_stride;
+    v.keys = p.keys ? p.keys + (size_t)(r - p.row0) * p.S_stride : nullptr;
     v.lim = lim;
     v.ksc = nullptr;
     if (p.kind == SEL_PREFIX) {
@@ -1180,6 +1406,32 @@ cudaError_t launch_row_threshold(const SelectParams& p_in, uint32_t* thresh, cud
     if (e != cudaSuccess) return e;
     const int grid = (p.nrows + THR_WARPS - 1) / THR_WARPS;
     row_threshold_kernel<<<grid, THR_WARPS * 32, smem, stream>>>(p, thresh);
+    return cudaGetLastError();
+}
+
+int fused_cap(int K) { return K <= 4096 ? 8192 : 16384; }
+
+cudaError_t launch_sample_bound(const FusedSelectParams& p, cudaStream_t stream) {
+    if (p.nrows <= 0) return cudaSuccess;
+    const size_t smem = (size_t)FB_WARPS * (FB_MAX_SAMPLES + THR_BINS) * 4;
+    cudaError_t e = cudaFuncSetAttribute(sample_bound_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    sample_bound_kernel<<<(p.nrows + FB_WARPS - 1) / FB_WARPS, FB_WARPS * 32, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fused_finish(const FusedSelectParams& p, cudaStream_t stream) {
+    if (p.nrows <= 0) return cudaSuccess;
+    const size_t per = (size_t)p.cap * 8 + THR_BINS * 4;
+    int warps = (int)(CW_SMEM_LIMIT / per);
+    if (warps > FF_MAX_WARPS) warps = FF_MAX_WARPS;
+    if (warps < 1) return cudaErrorInvalidValue;
+    const size_t smem = per * (size_t)warps;
+    cudaError_t e = cudaFuncSetAttribute(fused_finish_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    fused_finish_kernel<<<(p.nrows + warps - 1) / warps, warps * 32, smem, stream>>>(p, warps);
     return cudaGetLastError();
 }
 

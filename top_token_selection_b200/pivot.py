@@ -35,7 +35,7 @@ ABI_SYMBOLS = [
     "pivot_reuse_backfill", "pivot_window_union", "pivot_index_varlen",
     "pivot_index_varlen_workspace_size", "pivot_index_window_outside",
     "pivot_index_window_outside_workspace_size", "pivot_set_score_buffer_cap",
-    "pivot_workspace_size",
+    "pivot_workspace_size", "pivot_set_fused_selection",
 ]
 KERNELS = {0: "scan", 1: "select", 2: "refine", 3: "reduce", 4: "reuse"}
 
@@ -111,6 +111,7 @@ def load(path: str = LIB_PATH):
         "pivot_index_window_outside": ([P, I32, I32, I32, I32, I32, P, P, SZ, P], I32),
         "pivot_index_window_outside_workspace_size": ([P, I32, I32, I32, I32, I32], SZ),
         "pivot_workspace_size": ([I32, I32, I32, I32, I32, I32, I32, I32, I32], SZ),
+        "pivot_set_fused_selection": ([I32, ctypes.c_float], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -193,6 +194,10 @@ def pivot_set_wait_limit_ns(ns):
 
 def pivot_set_score_buffer_cap(nbytes):
     return load().pivot_set_score_buffer_cap(nbytes)
+
+
+def pivot_set_fused_selection(on, margin_sigmas=4.5):
+    return load().pivot_set_fused_selection(on, margin_sigmas)
 
 
 def pivot_selftest_wait_timeout(stream):
