@@ -740,10 +740,6 @@ def run_ours(args, wl):
         v = kern[name]
         if v["ms"] > 0:
             v["tflops"] = v["work"] * flop_pair / (v["ms"] / 1e3) / 1e12
-    for name in ("select",):
-        v = kern[name]
-        if v["ms"] > 0:
-            v["gbs_scores"] = v["work"] * 4 / (v["ms"] / 1e3) / 1e9
     for name in ("reduce", "reuse"):
         v = kern[name]
         if v["ms"] > 0:
@@ -768,12 +764,13 @@ def run_ours(args, wl):
                                                   (FP8_OVER_BF16 if fp8 else 1.0)),
                 "per_launch": {"work_pairs": dv["work"] / max(dv["launches"], 1),
                                "ms": dv["ms"] / max(dv["launches"], 1)}}
-    else:
-        key = "gbs_scores" if dom == "select" else "gbs"
-        ach = dv[key]
+    elif dom in ("reduce", "reuse"):
+        ach = dv["gbs"]
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
                 "peak_source": f"{peak_src} hbm"}
+    else:   # the selection: its work is per row, not per byte
+        roof = None
 
     # Refine + its top-k against HBM (algorithmic bytes: every group's C
     # candidate keys and scales gathered once, the members' queries and

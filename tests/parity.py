@@ -44,8 +44,11 @@ def assert_rows_exact(gpu, ref, what=""):
                              f"gpu {gpu[r][:16]} ref {ref[r][:16]}")
 
 
-def assert_rows_close(gpu_idx, ref_idx, ref_scores, score_fn, rows, what="", gpu_scores=None):
-    """Boundary-tolerant set comparison, row by row (see module doc)."""
+def assert_rows_close(gpu_idx, ref_idx, ref_scores, score_fn, rows, what="", gpu_scores=None,
+                      abs_tol=None):
+    """Boundary-tolerant set comparison, row by row (see module doc).
+    `abs_tol(row)`, when given, is a floor on every tolerance of that row:
+    the error bound of its fp32 arithmetic (fp32_abs_tol)."""
     gpu_idx = np.asarray(gpu_idx)
     ref_idx = np.asarray(ref_idx)
     nbad = 0
@@ -57,6 +60,8 @@ def assert_rows_close(gpu_idx, ref_idx, ref_scores, score_fn, rows, what="", gpu
             continue
         sk = float(np.min(ref_scores[i][:len(o)]))     # the k-th score: rows are listed by position
         tol = REL_TOL * max(abs(sk), 1e-30)
+        if abs_tol is not None:
+            tol = max(tol, abs_tol(r))
         gs, os_ = set(g), set(o)
         only_g = sorted(gs - os_)
         only_o = sorted(os_ - gs)
@@ -81,6 +86,26 @@ def assert_rows_close(gpu_idx, ref_idx, ref_scores, score_fn, rows, what="", gpu
             assert not bad.any(), (f"{what} row {r}: score error "
                                    f"{np.abs(gsc - want)[bad].max()} > {stol[bad].min()}")
     return nbad
+
+
+def fp32_abs_tol(pq, pw, k):
+    """The error bound of a score computed in fp32 on the CUDA cores (each
+    head's dot product a chain of D fused multiply-adds, then a chain of H
+    weighted adds): |err| <= (D + H + 2) u sum_h |w_h| sum_d |q_hd| |k_d|,
+    u = 2^-24 (the standard bound on recursive summation, Higham, Accuracy
+    and Stability of Numerical Algorithms, ch. 3), taken twice for margin.
+    It matters where a row's boundary sits among near-zero scores that come
+    from cancelling dot products, which no relative tolerance can scale.
+    Returns a per-row bound (max over the row's keys)."""
+    pq = np.asarray(pq, dtype=np.float64)
+    H, D = pq.shape[1], pq.shape[2]
+    bound = np.einsum("gh,ghd->gd", np.abs(np.asarray(pw, dtype=np.float64)), np.abs(pq)) @ \
+        np.abs(np.asarray(k, dtype=np.float64)).T
+    per_row = bound.max(axis=1) * 2.0 * (D + H + 2) * 2.0 ** -24
+
+    def fn(j):
+        return per_row[j]
+    return fn
 
 
 def oracle_codes(p):

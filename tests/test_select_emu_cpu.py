@@ -126,6 +126,7 @@ def test_backfill_rows_match_a_sort(select_check, L, g, C, K):
     (40000, 4096, 2048, 0, 4, 4990, 0, 4.5, 1, "none"),  # proxy rows: top-k first, then the rest
     (40000, 4096, 2048, 0, 3, 4990, 0, -40.0, 1, "all"), # the same through the fallback
     (40000, 4096, 2048, 2, 3, 4990, 1, -40.0, 1, "any"), # signed zeros and small integers
+    (262144, 2048, 0, 0, 2, 262142, 0, 4.5, 0, "none"),  # rows too long for the bitmap: sorted
 ])
 def test_fused_selection_matches_a_sort(select_check, L, K, split, dist, rows, r0, order, sigmas,
                                         kind, want_fallback):

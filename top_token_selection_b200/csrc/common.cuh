@@ -275,31 +275,6 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// 16 consecutive fp32 columns of this thread's TMEM lane (the load is
-// asynchronous: the registers are valid after tmem_ld_wait16 on them).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-    uint32_t* r = reinterpret_cast<uint32_t*>(v);
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-
-// Waits for this thread's TMEM loads; the 16 registers of the load being
-// waited for pass through the wait, so no use of them can be scheduled
-// before it (a later load may already be in flight into other registers).
-__device__ __forceinline__ void tmem_ld_wait16(float* v) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
-                   "+f"(v[6]), "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]),
-                   "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15])
-                 :
-                 : "memory");
-}
-
 // ---------------------------------------------------------------------------
 // number formats
 // ---------------------------------------------------------------------------

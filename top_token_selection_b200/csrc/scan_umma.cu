@@ -35,9 +35,12 @@ namespace pivot {
 
 constexpr int EPI_GROUPS = 3;                       // epilogue warps per TMEM lane quarter
 constexpr int EPI_WARPS = 4 * EPI_GROUPS;           // 12
-constexpr int SCAN_THREADS = 64 + EPI_WARPS * 32;   // + producer warp + MMA warp = 448
+// producer warp 0, MMA warp 1, epilogue warps 2-13, and warp 14: the second
+// candidate-gathering warp of gather mode (idle in scan mode)
+constexpr int GATHER_WARP2 = 2 + EPI_WARPS;         // 14
+constexpr int SCAN_THREADS = (GATHER_WARP2 + 1) * 32;   // 480
 // Register files are per SM sub-partition (16K each); warp w runs on
-// sub-partition w % 4, so 14 warps put at most 4 on one: 128 registers.
+// sub-partition w % 4, so 15 warps put at most 4 on one: 128 registers.
 constexpr int SCAN_MAXREG = 128;
 
 __device__ __forceinline__ int scan_row_lim(const ScanParams& p, int r, bool& ok) {
@@ -209,18 +212,27 @@ __global__ void __maxnreg__(SCAN_MAXREG)
     float* w_s = reinterpret_cast<float*>(tmem_holder + 4);   // [256], 16-byte aligned
     float* sq_s = w_s + 256;                                   // [PMAX]
     int* lim_s = reinterpret_cast<int*>(sq_s + PMAX);          // [PMAX]
-    // filter mode: survivors of each row of the current item, double-
-    // buffered by the epilogue's item parity
-    uint32_t* cnt_s = reinterpret_cast<uint32_t*>(lim_s + PMAX);   // [2][PMAX]
+    // filter mode (H >= 32, where the weight table is unused): survivors of
+    // each row of the current item, double-buffered by the epilogue's item
+    // parity, in the weight table's space
+    uint32_t* cnt_s = reinterpret_cast<uint32_t*>(w_s);   // [2][PMAX], PMAX <= 8 here
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const int N = p.P * HEADS;
+    // row-list mode: only the listed rows' items (the count is read once)
+    int nitems = p.nitems;
+    if (p.row_list) {
+        const long long lim = (long long)(*p.row_count) * p.items_per_block;
+        if (lim < nitems) nitems = (int)lim;
+    }
 
-    for (int i = threadIdx.x; i < 2 * PMAX; i += blockDim.x) cnt_s[i] = 0;
+    if (FILTER && HEADS >= 32)
+        for (int i = threadIdx.x; i < 2 * PMAX; i += blockDim.x) cnt_s[i] = 0;
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&full[i], 1);
+            // gather mode: both gathering warps publish each tile
+            mbar_init(&full[i], GATHER ? 2 : 1);
             mbar_init(&empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -243,9 +255,10 @@ __global__ void __maxnreg__(SCAN_MAXREG)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    if (warp == 0) {
+    if (warp == 0 || warp == GATHER_WARP2) {
         // ------------------------------------------------------- producer
         if constexpr (!GATHER) {
+            if (warp == 0) {
             // Scan mode: lane 0 streams contiguous key tiles with tiled TMA.
             if (lane == 0) {
                 int stage = 0;
@@ -256,7 +269,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 int last_a[STAGES], last_b[2] = {-1, -1};
                 for (int i = 0; i < STAGES; ++i) last_a[i] = -1;
                 bool aborted = false;
-                for (int item = blockIdx.x; item < p.nitems && !aborted; item += gridDim.x) {
+                for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
                     ItemInfo it = scan_item<GATHER>(p, item);
                     if (!it.valid) continue;
                     const int slot = nit & 1;
@@ -287,12 +300,21 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 for (int i = 0; i < 2; ++i)
                     if (last_b[i] >= 0) mbar_wait(&bfull[i], (uint32_t)last_b[i]);
             }
+            }
         } else {
-            // Gather mode: the whole warp copies each tile's 128 candidate
-            // key rows with 16-byte cp.async straight into the swizzled tile
-            // layout.  A tile is published (full[stage] arrive) once its
-            // copies have landed and been fenced for the tensor cores; up to
-            // GDEPTH tiles are in flight.
+            // Gather mode: two warps copy each tile's 128 candidate key rows
+            // (warp 0 rows 0-63, warp 14 rows 64-127) with 16-byte cp.async
+            // straight into the swizzled tile layout.  Each publishes its half
+            // of a tile (an arrive on full[stage], which expects both) once
+            // its copies have landed and been fenced for the tensor cores; up
+            // to GDEPTH tiles are in flight per warp.  Warp 0 alone loads the
+            // query blocks.  Neither warp blocks while holding an unpublished
+            // tile older than the one it waits for: warp 0 publishes the
+            // tiles of item nit - 2 before waiting for its query slot, and a
+            // ring stage a warp waits on was last used by a tile older than
+            // all of that warp's pending ones (STAGES > GDEPTH).
+            const bool lead = warp == 0;
+            const int jb = lead ? 0 : 2;   // row groups j of this warp (rows j * 32 + lane)
             constexpr int GDEPTH = STAGES > 3 ? 3 : STAGES - 1;   // deeper was slower
             static_assert(STAGES > GDEPTH && GDEPTH >= 1, "the ring must outrun the copies");
             const uint8_t* kbytes = static_cast<const uint8_t*>(p.kbase);
@@ -314,7 +336,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 }
                 --npend;
             };
-            for (int item = blockIdx.x; item < p.nitems && !aborted; item += gridDim.x) {
+            for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
                 ItemInfo it = scan_item<GATHER>(p, item);
                 if (!it.valid) continue;
                 const int slot = nit & 1;
@@ -323,43 +345,46 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 // which needs every tile of that item published: land and
                 // publish what is in flight if any of it is that old (items
                 // shorter than the copy depth).
-                if (npend > 0 && pend_it[0] <= nit - 2) {
-                    cp_async_wait<0>();
-                    while (npend > 0) publish_oldest();
+                if (lead) {
+                    if (npend > 0 && pend_it[0] <= nit - 2) {
+                        cp_async_wait<0>();
+                        while (npend > 0) publish_oldest();
+                    }
+                    if (!__all_sync(0xffffffffu, mbar_wait(&bempty[slot], bph ^ 1))) {
+                        aborted = true;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&bfull[slot], (uint32_t)(N * ROWB));
+                        const int qrow = (it.row_first - p.qrow_base) * HEADS;
+                        for (int kb = 0; kb < KBLK; ++kb)
+                            tma_load_2d(sB + slot * B_SLOT + kb * (N * 128), &tmap_q, &bfull[slot],
+                                        kb * (128 / p.esize), qrow);
+                    }
+                    last_b[slot] = (int)bph;
                 }
-                if (!__all_sync(0xffffffffu, mbar_wait(&bempty[slot], bph ^ 1))) {
-                    aborted = true;
-                    break;
-                }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&bfull[slot], (uint32_t)(N * ROWB));
-                    const int qrow = (it.row_first - p.qrow_base) * HEADS;
-                    for (int kb = 0; kb < KBLK; ++kb)
-                        tma_load_2d(sB + slot * B_SLOT + kb * (N * 128), &tmap_q, &bfull[slot],
-                                    kb * (128 / p.esize), qrow);
-                }
-                last_b[slot] = (int)bph;
-                // candidate positions of a tile: lane l holds slots l + 32 j
-                // (j < 4), read one tile ahead so no copy waits on them
-                auto tile_pos = [&](int t, int (&pp)[4]) {
+                // candidate positions of this warp's rows of a tile: lane l
+                // holds slots l + 32 (jb + j), read one tile ahead so no copy
+                // waits on them
+                auto tile_pos = [&](int t, int (&pp)[2]) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int slot_r = t * 128 + j * 32 + lane;
+                    for (int j = 0; j < 2; ++j) {
+                        const int slot_r = t * 128 + (jb + j) * 32 + lane;
                         pp[j] = slot_r < p.C ? ld_nc_early(it.cand + slot_r) : -1;
                     }
                 };
-                int cur[4], nxt[4];
+                int cur[2], nxt[2];
                 tile_pos(it.t0, nxt);
                 for (int t = it.t0; t < it.t1; ++t) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
+                    for (int j = 0; j < 2; ++j) cur[j] = nxt[j];
                     if (t + 1 < it.t1) tile_pos(t + 1, nxt);
                     if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1))) {
                         aborted = true;
                         break;
                     }
                     const uint32_t dst = smem_u32(sA + stage * A_BYTES);
-                    // Lane l copies tile rows l + 32 j (j < 4), its own
+                    // Lane l copies tile rows l + 32 (jb + j), its own
                     // positions, 16 bytes at a time.  Chunk c of row r sits at
                     // (r / 8) 1024 + (r % 8) 128 + ((c ^ r % 8) 16): with the
                     // tile 1024-byte aligned that is rowbase XOR (c 16), where
@@ -367,8 +392,8 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                     // out in consecutive instructions, so after the first the
                     // line is in L1 (.ca); the loop is two instructions a chunk.
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int r = j * 32 + lane;
+                    for (int j = 0; j < 2; ++j) {
+                        const int r = (jb + j) * 32 + lane;
                         const int pos = cur[j];
                         const size_t row = (size_t)(it.keybase + ((pos >= 0 && pos < it.nkeys) ? pos : 0));
                         const uint8_t* src = kbytes + row * ROWB;
@@ -396,7 +421,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
             // publish (or, after an abort, just land) every tile still in flight
             cp_async_wait<0>();
             while (npend > 0) publish_oldest();
-            if (lane == 0)
+            if (lead && lane == 0)
                 for (int i = 0; i < 2; ++i)
                     if (last_b[i] >= 0) mbar_wait(&bfull[i], (uint32_t)last_b[i]);
         }
@@ -408,7 +433,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
             uint32_t phase = 0;
             int nit = 0, ntile = 0;
             bool aborted = false;
-            for (int item = blockIdx.x; item < p.nitems && !aborted; item += gridDim.x) {
+            for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
                 ItemInfo it = scan_item<GATHER>(p, item);
                 if (!it.valid) continue;
                 const int slot = nit & 1;
@@ -475,7 +500,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
         // keeps walking the items, so the named barriers shared by the
         // epilogue warps are always reached.
         bool aborted = false;
-        for (int item = blockIdx.x; item < p.nitems; item += gridDim.x) {
+        for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
             ItemInfo it = scan_item<GATHER>(p, item);
             if (!it.valid) continue;
             // gather mode: every candidate slot is written (the selection
@@ -572,25 +597,18 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                         uint64_t a[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) a[j] = 0ull;
-                        // the row's columns in 16-column chunks, software-
-                        // pipelined: chunk c + 1 is loaded from TMEM while
-                        // chunk c's math runs
-                        constexpr int NCH = HEADS / 16;
-                        float v[2][16];
-                        tmem_ld16(taddr + (uint32_t)(pr * HEADS), v[0]);
 #pragma unroll
-                        for (int c = 0; c < NCH; ++c) {
-                            tmem_ld_wait16(v[c & 1]);
-                            if (c + 1 < NCH)
-                                tmem_ld16(taddr + (uint32_t)(pr * HEADS + (c + 1) * 16),
-                                          v[(c + 1) & 1]);
+                        for (int c = 0; c < HEADS / 32; ++c) {
+                            float v[32];
+                            tmem_ld32(taddr + (uint32_t)(pr * HEADS + c * 32), v);
+                            tmem_ld_wait();
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int wi = lr * HEADS + c * 16 + 2 * i;
-                                const float x0 = v[c & 1][2 * i], x1 = v[c & 1][2 * i + 1];
+                            for (int i = 0; i < 16; ++i) {
+                                const int wi = lr * HEADS + c * 32 + 2 * i;
                                 // x + |x| = 2 max(0, x): one add on the FMA pipe
                                 // instead of a half-rate max on the ALU pipe
-                                a[i & 3] = ffma2(pack2(x0 + fabsf(x0), x1 + fabsf(x1)),
+                                a[i & 3] = ffma2(pack2(v[2 * i] + fabsf(v[2 * i]),
+                                                       v[2 * i + 1] + fabsf(v[2 * i + 1])),
                                                  pack2(wr[wi], wr[wi + 1]), a[i & 3]);
                             }
                         }
@@ -678,7 +696,7 @@ int scan_smem_bytes(int row_bytes) {
     const int stages = row_bytes == 128 ? 6 : 3;
     const int pmax = 64;
     return 1024 /*align slack*/ + 2 * 256 * row_bytes + stages * 128 * row_bytes +
-           256 /*barriers*/ + 16 /*TMEM address*/ + 256 * 4 + pmax * 8 + 2 * pmax * 4;
+           256 /*barriers*/ + 16 /*TMEM address*/ + 256 * 4 + pmax * 8;
 }
 
 // The epilogue's three warp groups take ceil(P / 3) rows each, with room

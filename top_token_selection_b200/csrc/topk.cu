@@ -794,9 +794,15 @@ __device__ uint32_t warp_kth_largest_f(F get, int n, uint32_t m, uint32_t* hist)
 #pragma unroll
         for (int b = 0; b < THR_BINS / 32; ++b) hist[b * 32 + lane] = 0;
         __syncwarp();
-        for (int i = lane; i < n; i += 32) {
-            const uint32_t u = get(i);
-            if (u && u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> sh], 1u);
+        // lanes landing in one bin add once (the keys of a row cluster in
+        // few bins, and same-address shared atomics serialise)
+        for (int i0 = 0; i0 < n; i0 += 32) {
+            const int i = i0 + lane;
+            const uint32_t u = i < n ? get(i) : 0u;
+            const bool in = u && u >= lo && u <= hi;
+            const uint32_t bin = in ? (u - lo) >> sh : 0xFFFFFFFFu;
+            const unsigned peers = __match_any_sync(0xffffffffu, bin);
+            if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
         }
         __syncwarp();
         // lane l owns the 8 bins [THR_BINS - 8 (l + 1), THR_BINS - 8 l)
@@ -1269,6 +1275,58 @@ __global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const F
             for (int i = lane; i < kept; i += 32) {
                 out[i] = key_pos(e[i]);
                 if (outs) outs[i] = key_to_float(key_u(e[i]));
+            }
+        } else if ((size_t)kept * 8 + (size_t)((lim >> 5) + 1) * 8 <= (size_t)M * 8) {
+            // position order by a bitmap of the row's positions: each kept
+            // entry's slot is its class's base plus its rank among the
+            // class's marked positions (per-word prefix counts)
+            const int W = (lim >> 5) + 1;
+            uint32_t* bm = reinterpret_cast<uint32_t*>(e + kept);
+            uint32_t* pref = bm + W;
+            uint32_t base = 0;
+            for (int cls = 0; cls < (split ? 2 : 1); ++cls) {
+                for (int w = lane; w < W; w += 32) bm[w] = 0u;
+                __syncwarp();
+                for (int i = lane; i < kept; i += 32) {
+                    const uint64_t k = e[i];
+                    const uint32_t u = key_u(k);
+                    const bool inA = !split || u > TA || (u == TA && (uint32_t)k >= LA);
+                    if (inA == (cls == 0)) {
+                        const int pos = key_pos(k);
+                        atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+                    }
+                }
+                __syncwarp();
+                const int per = (W + 31) / 32;
+                const int w0 = lane * per, w1 = min(W, w0 + per);
+                uint32_t local = 0;
+                for (int w = w0; w < w1; ++w) local += __popc(bm[w]);
+                uint32_t inc = local;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += y;
+                }
+                uint32_t acc = inc - local;
+                for (int w = w0; w < w1; ++w) {
+                    pref[w] = acc;
+                    acc += __popc(bm[w]);
+                }
+                const uint32_t ncls = __shfl_sync(0xffffffffu, inc, 31);
+                __syncwarp();
+                for (int i = lane; i < kept; i += 32) {
+                    const uint64_t k = e[i];
+                    const uint32_t u = key_u(k);
+                    const bool inA = !split || u > TA || (u == TA && (uint32_t)k >= LA);
+                    if (inA == (cls == 0)) {
+                        const int pos = key_pos(k);
+                        const uint32_t slot =
+                            base + pref[pos >> 5] + __popc(bm[pos >> 5] & ((1u << (pos & 31)) - 1u));
+                        out[slot] = pos;
+                        if (outs) outs[slot] = key_to_float(u);
+                    }
+                }
+                base += ncls;
+                __syncwarp();
             }
         } else {
             // sort key: class (A first), then position, with the score kept
