@@ -10,6 +10,7 @@
 //   select_check varlen <kind> <g> <K> <C>     (ragged batch rows, see run_varlen)
 //   select_check decode <kind> <K>             (MTP decode rows, see run_decode)
 //   select_check backfill <L> <g> <C> <K>      (Reuse with backfill, see run_backfill)
+//   select_check planted <L> <K> <npos>        (bitmap too small; debug build only)
 //   select_check fused <L> <K> <split> <dist> <rows> <r0> <order> <sigmas> <kind>
 //                                              (selection fused into the scan, see run_fused)
 // dist: 0 normal, 1 few distinct values (heavy ties), 2 signed zeros and
@@ -548,6 +549,35 @@ int run_fused(int L, int K, int split, int dist, int nrows, int r0, int order, f
     return bad;
 }
 
+// A planted mistake in the launch parameters: the bitmap sized for only
+// `npos` positions while the rows reach L - 1.  Without PIVOT_DEBUG this
+// would write past the bitmap; with it every such access is skipped and the
+// error word carries the bounds bit.
+int run_planted(int L, int K, int npos) {
+    std::mt19937 rng(99);
+    std::vector<float> S(L);
+    for (auto& x : S) x = draw(rng, 0);
+    std::vector<int32_t> out(K);
+    std::vector<float> outs(K);
+    SelectParams sp{};
+    sp.kind = SEL_PREFIX;
+    sp.scan_kind = SCAN_PREFILL_DENSE;
+    sp.row0 = L - 1;
+    sp.nrows = 1;
+    sp.L = L;
+    sp.g = 1;
+    sp.Gm = 1;
+    sp.S = S.data();
+    sp.S_stride = L;
+    sp.K = K;
+    sp.out_idx = out.data();
+    sp.out_score = outs.data();
+    sp.out_base = L - 1;
+    sp.tail_cap = 4096;
+    sp.npos = npos;
+    return launch_select(sp, nullptr) == cudaSuccess ? 0 : 2;
+}
+
 }  // namespace
 
 int main(int argc, char** argv) {
@@ -563,6 +593,8 @@ int main(int argc, char** argv) {
     else if (what == "fused" && argc == 11)
         bad = run_fused(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]), atoi(argv[6]),
                         atoi(argv[7]), atoi(argv[8]), (float)atof(argv[9]), atoi(argv[10]));
+    else if (what == "planted" && argc == 5)
+        bad = run_planted(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]));
     else if (what == "backfill" && argc == 6)
         bad = run_backfill(atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]));
     else if (what == "decode" && argc == 4)

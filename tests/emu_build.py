@@ -56,13 +56,15 @@ def prepare(d: Path, extra=False):
     helpers copied from the real one), kernels.h and segments.h."""
     common = (CSRC / "common.cuh").read_text()
     errbits = re.search(r"enum : uint32_t \{.*?\};", common, re.S).group(0)
+    # the debug-build checks (used as they are; on when compiled with PIVOT_DEBUG)
+    checks = re.search(r"#ifdef PIVOT_DEBUG\n.*?#endif\n", common, re.S).group(0)
     helpers = re.search(r"// Order-preserving unsigned key.*?int ceil_div\(int a, int b\) \{[^}]*\}",
                         common, re.S).group(0)
     (d / "common.cuh").write_text(
         "#pragma once\n#include <cmath>\n#include \"emu.h\"\n#include \"pivot.h\"\n"
         "namespace pivot {\n" + errbits + "\nextern uint32_t g_error_word;\n"
         "inline void raise_error(uint32_t bit) { __atomic_fetch_or(&g_error_word, bit, "
-        "__ATOMIC_SEQ_CST); }\n" + helpers + (EXTRA if extra else "") +
+        "__ATOMIC_SEQ_CST); }\n" + checks + helpers + (EXTRA if extra else "") +
         "\n}  // namespace pivot\n")
     kernels = rewrite((CSRC / "kernels.h").read_text(),
                       [("#include <cuda.h>", "#include \"emu.h\""), ("#include <cuda_runtime.h>\n", "")])
@@ -70,9 +72,10 @@ def prepare(d: Path, extra=False):
     shutil.copy(CSRC / "segments.h", d / "segments.h")
 
 
-def compile_(d: Path, sources, out: Path, shared=False, sanitize=False):
+def compile_(d: Path, sources, out: Path, shared=False, sanitize=False, defines=()):
     cmd = ["g++", "-std=c++20", "-O1", "-g", "-pthread", "-ffp-contract=off",
            "-I", str(d), "-I", str(EMU), "-I", str(ROOT / "include")]
+    cmd += [f"-D{x}" for x in defines]
     if shared:
         cmd += ["-fPIC", "-shared"]
     if sanitize:

@@ -125,3 +125,34 @@ def test_fused_row_ranges_and_small_workspace():
     torch.cuda.synchronize()
     assert pv.device_error() == 0
     assert torch.equal(c, full)
+
+
+@pytest.mark.parametrize("dtype,Gm", [(E4M3, 2), (BF16, 3)])
+def test_fused_decode_equals_writing_every_score(dtype, Gm):
+    """MTP decode over ragged cache lengths: dense and
+    proxy rows through the fused selection equal the rows written from every
+    score, in both output orders and through the forced rescan."""
+    d = gen.make_decode(B=6, Gm=Gm, H=64, D=128, dtype=dtype, len_lo=3000, len_hi=20000, seed=17)
+    c = "cuda"
+    C, kk = 4096, 2048
+    try:
+        for order in (pv.ORDER_POSITION, pv.ORDER_RANK):
+            batch = pv.make_decode(d.q.to(c), None if d.q_scale is None else d.q_scale.to(c),
+                                   d.w.to(c), d.kc.to(c),
+                                   None if d.kc_scale is None else d.kc_scale.to(c),
+                                   d.cache_len.to(c), order=order)
+            want = {}
+            assert pv.pivot_set_fused_selection(0, 4.5) == 0
+            for mode in (pv.DENSE, pv.REUSE, pv.REFINE):
+                want[mode] = pv.decode(batch, mode, C, kk, want_cand=True)
+            for sig in (4.5, -60.0, 600.0):
+                assert pv.pivot_set_fused_selection(1, sig) == 0
+                for mode in (pv.DENSE, pv.REUSE, pv.REFINE):
+                    idx, cand = pv.decode(batch, mode, C, kk, want_cand=True)
+                    torch.cuda.synchronize()
+                    assert pv.device_error() == 0
+                    assert torch.equal(idx, want[mode][0]), (order, sig, mode)
+                    if mode != pv.DENSE:
+                        assert torch.equal(cand, want[mode][1]), (order, sig, mode)
+    finally:
+        pv.pivot_set_fused_selection(1, 4.5)

@@ -49,6 +49,15 @@ def select_check(tmp_path_factory):
                     sanitize=True)
 
 
+@pytest.fixture(scope="module")
+def select_check_debug(tmp_path_factory, select_check):
+    """The same harness with PIVOT_DEBUG defined: the kernels' own index
+    checks are on."""
+    d = select_check.parent
+    return compile_(d, [d / "topk_emu.cpp", EMU / "select_check.cpp"], d / "select_check_debug",
+                    sanitize=True, defines=("PIVOT_DEBUG",))
+
+
 def _run(exe, *args):
     res = subprocess.run([str(exe), *map(str, args)], capture_output=True, text=True,
                          timeout=600)
@@ -143,3 +152,22 @@ def test_fused_selection_matches_a_sort(select_check, L, K, split, dist, rows, r
         assert n_fb == 0
     elif want_fallback == "all":
         assert n_fb == n
+
+
+@pytest.mark.parametrize("args", [("prefix", 20000, 2048, 0, 0, 3, 1), ("cand", 4096, 2048, 1, 5, 0, 0),
+                                  ("fused", 20000, 2048, 0, 0, 4, 19000, 0, 4.5, 0),
+                                  ("fused", 40000, 4096, 2048, 0, 3, 4990, 0, -40.0, 1)])
+def test_debug_build_raises_nothing_on_valid_rows(select_check_debug, args):
+    """PIVOT_DEBUG build: valid rows pass every check (error word 0) and
+    select exactly as the normal build does."""
+    _run(select_check_debug, *args)
+
+
+def test_debug_build_flags_a_planted_bitmap_overrun(select_check_debug):
+    """A launch whose bitmap is sized for 64 positions while the row reaches
+    20000: the debug build skips every out-of-range bitmap access (no
+    sanitizer report) and raises the bounds bit (4) in the error word."""
+    res = subprocess.run([str(select_check_debug), "planted", "20000", "2048", "64"],
+                         capture_output=True, text=True, timeout=600)
+    assert "ERROR: AddressSanitizer" not in res.stderr, res.stderr[-3000:]
+    assert res.stdout.strip().endswith("error word 4"), res.stdout + res.stderr[-2000:]

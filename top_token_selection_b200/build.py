@@ -1,6 +1,6 @@
 """Build libpivot.so in-tree with nvcc for sm_100a (B200).
 
-    python -m top_token_selection_b200.build [--force]
+    python -m top_token_selection_b200.build [--force] [--debug]
 
 Compiles every ``csrc/*.cu`` with relocatable device code (the per-device
 error word is shared across translation units) and links one shared
@@ -41,27 +41,37 @@ def stale() -> bool:
     return any(os.path.getmtime(d) > t for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+LIB_DEBUG = os.path.join(HERE, "libpivot_debug.so")
+
+
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Build libpivot.so; with debug=True, libpivot_debug.so instead: the same
+    sources with PIVOT_DEBUG defined, so every kernel checks its own index
+    invariants and reports a failed check through the device error word
+    (pivot_get_device_error returns PIVOT_ERR_DEVICE) instead of trapping."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and os.path.exists(lib) and \
+            not any(os.path.getmtime(d) > os.path.getmtime(lib) for d in _deps()):
+        return lib
+    bdir = BUILD + ("_debug" if debug else "")
+    os.makedirs(bdir, exist_ok=True)
+    extra = ["-DPIVOT_DEBUG"] if debug else []
     objs = []
     for src in _sources():
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-        cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
+        cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [NVCC, *ARCH, "-rdc=true", "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv))

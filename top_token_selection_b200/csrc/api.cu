@@ -470,14 +470,21 @@ float g_fused_sigmas = 4.5f;
 bool fused_ok(int H, int D, int dtype, int K) {
     return g_fused_on && umma_shape_ok(H, D, dtype) && H >= 32 && K <= MAX_K;
 }
+// Key tiles of one scan work item: prefill items take FUSED_TILES, decode
+// items (few, long rows) 8.
+int scan_tiles_per_item(int kind) {
+    return (kind == SCAN_DECODE_DENSE || kind == SCAN_DECODE_PROXY) ? 8 : FUSED_TILES;
+}
 int fused_tiles(int L) { return ceil_div(L, 128); }
 long long fused_samp_stride(int L) { return (long long)ceil_div(fused_tiles(L), FUSED_KTS) * 128; }
-int fused_nchunks(int L) { return ceil_div(fused_tiles(L), FUSED_TILES); }
-long long fused_surv_stride(int L) { return (long long)fused_nchunks(L) * FUSED_TILES * 128; }
+int fused_nchunks(int L, int tpi = FUSED_TILES) { return ceil_div(fused_tiles(L), tpi); }
+long long fused_surv_stride(int L, int tpi = FUSED_TILES) {
+    return (long long)fused_nchunks(L, tpi) * tpi * 128;
+}
 // per row: samples, survivor regions, chunk counts, the bound, a miss slot
-size_t fused_rowbytes(int L) {
-    return (size_t)fused_samp_stride(L) * 4 + (size_t)fused_surv_stride(L) * 8 +
-           (size_t)fused_nchunks(L) * 4 + 4 + 4;
+size_t fused_rowbytes(int L, int tpi = FUSED_TILES) {
+    return (size_t)fused_samp_stride(L) * 4 + (size_t)fused_surv_stride(L, tpi) * 8 +
+           (size_t)fused_nchunks(L, tpi) * 4 + 4 + 4;
 }
 constexpr size_t FUSED_FIXED = 8 * WS_ALIGN;   // alignment of the six arrays, the miss count
 
@@ -490,11 +497,12 @@ struct FusedWs {
     uint32_t* nmiss;
 };
 
-bool fused_carve(void* ws, size_t bytes, long long rows, int L, FusedWs* w) {
+bool fused_carve(void* ws, size_t bytes, long long rows, int L, FusedWs* w,
+                 int tpi = FUSED_TILES) {
     Carver c{static_cast<uint8_t*>(ws), bytes};
     w->samp = static_cast<float*>(c.take((size_t)rows * fused_samp_stride(L) * 4));
-    w->surv = static_cast<uint64_t*>(c.take((size_t)rows * fused_surv_stride(L) * 8));
-    w->count = static_cast<uint32_t*>(c.take((size_t)rows * fused_nchunks(L) * 4));
+    w->surv = static_cast<uint64_t*>(c.take((size_t)rows * fused_surv_stride(L, tpi) * 8));
+    w->count = static_cast<uint32_t*>(c.take((size_t)rows * fused_nchunks(L, tpi) * 4));
     w->bound = static_cast<uint32_t*>(c.take((size_t)rows * 4));
     w->miss = static_cast<int32_t*>(c.take((size_t)rows * 4));
     w->nmiss = static_cast<uint32_t*>(c.take(4));
@@ -506,33 +514,54 @@ long long fused_chunk_rows(size_t bytes, int L, long long total, int P) {
     return chunk_rows(bytes > FUSED_FIXED ? bytes - FUSED_FIXED : 0, fused_rowbytes(L), total, P);
 }
 
-// The top K of prefix rows [r0, r1) of `kind` (SCAN_PREFILL_DENSE: rows of
-// seq->q; SCAN_PREFILL_PROXY: rows of the proxies `qbase`), written like
+// The keys a fused selection scans: one prefill sequence, or the caches of
+// a decode batch.
+struct KeySrc {
+    int dtype, H, D;
+    const void* k;
+    long long k_rows;
+    const float* k_scale;
+    int L;                 // prefill length, or the cache capacity (maxlen) in decode
+    int Gm, maxlen;
+    const int32_t* cache_len;
+};
+
+KeySrc key_src(const pivot_seq_t* s) {
+    return KeySrc{s->dtype, s->H, s->D, s->k, s->L, s->k_scale, s->L, 1, 0, nullptr};
+}
+
+// The top K of rows [r0, r1) of `kind` (prefill: rows of queries or
+// proxies; decode: members or proxies of the batch), written like
 // run_select_prefix writes them.
-pivot_status_t run_prefix_fused(int kind, const pivot_seq_t* seq, const void* qbase,
+pivot_status_t run_prefix_fused(int kind, const KeySrc& ks, const void* qbase,
                                 long long q_rows, int qrow_base, const float* w,
                                 const float* q_scale, int g, int P, int r0, int r1, int maxlim,
                                 int K, int split, int32_t* out, float* out_score, int out_base,
                                 int lim_shift, int out_stride, const FusedWs& fw,
                                 cudaStream_t s) {
-    const int L = seq->L;
-    const double pairs = scan_pairs(kind, r0, r1, L, g);
+    const int L = ks.L;
+    const int tpi = scan_tiles_per_item(kind);
+    const bool dec = kind == SCAN_DECODE_DENSE || kind == SCAN_DECODE_PROXY;
+    const double pairs = dec ? 0.0 : scan_pairs(kind, r0, r1, L, g);
     // 1. samples
     ScanExtra xs;
     xs.key_tile_stride = FUSED_KTS;
     xs.work = pairs / FUSED_KTS;
     pivot_status_t st =
-        run_scan(kind, seq->dtype, seq->H, seq->D, qbase, q_rows, qrow_base, w, q_scale, seq->k,
-                 L, seq->k_scale, L, g, 1, 0, nullptr, P, r0, r1, maxlim, fw.samp,
-                 fused_samp_stride(L), s, &xs);
+        run_scan(kind, ks.dtype, ks.H, ks.D, qbase, q_rows, qrow_base, w, q_scale, ks.k,
+                 ks.k_rows, ks.k_scale, dec ? 0 : L, g, ks.Gm, ks.maxlen, ks.cache_len, P, r0,
+                 r1, maxlim, fw.samp, fused_samp_stride(L), s, &xs);
     if (st != PIVOT_OK) return st;
     // 2. bounds
     FusedSelectParams fp{};
     fp.scan_kind = kind;
     fp.row0 = r0;
     fp.nrows = r1 - r0;
-    fp.L = L;
+    fp.L = dec ? 0 : L;
     fp.g = g;
+    fp.Gm = ks.Gm;
+    fp.maxlen = ks.maxlen;
+    fp.cache_len = ks.cache_len;
     fp.lim_shift = lim_shift;
     fp.K = K;
     fp.split = split;
@@ -544,10 +573,10 @@ pivot_status_t run_prefix_fused(int kind, const pivot_seq_t* seq, const void* qb
     fp.bound = fw.bound;
     fp.cap = fused_cap(K);
     fp.surv = fw.surv;
-    fp.surv_stride = fused_surv_stride(L);
+    fp.surv_stride = fused_surv_stride(L, tpi);
     fp.surv_count = fw.count;
-    fp.nchunks = fused_nchunks(L);
-    fp.chunk_keys = FUSED_TILES * 128;
+    fp.nchunks = fused_nchunks(L, tpi);
+    fp.chunk_keys = tpi * 128;
     fp.out_idx = out;
     fp.out_score = out_score;
     fp.out_base = out_base;
@@ -560,13 +589,14 @@ pivot_status_t run_prefix_fused(int kind, const pivot_seq_t* seq, const void* qb
     ScanExtra xf;
     xf.bound = fw.bound;
     xf.surv = fw.surv;
-    xf.surv_stride = fused_surv_stride(L);
+    xf.surv_stride = fused_surv_stride(L, tpi);
     xf.surv_count = fw.count;
-    xf.nchunks = fused_nchunks(L);
+    xf.nchunks = fused_nchunks(L, tpi);
     xf.lim_shift = lim_shift;
     xf.work = pairs;
-    st = run_scan(kind, seq->dtype, seq->H, seq->D, qbase, q_rows, qrow_base, w, q_scale, seq->k,
-                  L, seq->k_scale, L, g, 1, 0, nullptr, P, r0, r1, maxlim, nullptr, 0, s, &xf);
+    st = run_scan(kind, ks.dtype, ks.H, ks.D, qbase, q_rows, qrow_base, w, q_scale, ks.k,
+                  ks.k_rows, ks.k_scale, dec ? 0 : L, g, ks.Gm, ks.maxlen, ks.cache_len, P, r0, r1,
+                  maxlim, nullptr, 0, s, &xf);
     if (st != PIVOT_OK) return st;
     // 4. the top K of every row's survivors
     st = from_cuda(profiled(PK_SELECT, 0.0, s, [&] { return launch_fused_finish(fp, s); }));
@@ -577,8 +607,9 @@ pivot_status_t run_prefix_fused(int kind, const pivot_seq_t* seq, const void* qb
     xr.row_list = fw.miss;
     xr.row_count = fw.nmiss;
     xr.work = 0.0;
-    st = run_scan(kind, seq->dtype, seq->H, seq->D, qbase, q_rows, qrow_base, w, q_scale, seq->k,
-                  L, seq->k_scale, L, g, 1, 0, nullptr, 1, r0, r1, maxlim, nullptr, 0, s, &xr);
+    st = run_scan(kind, ks.dtype, ks.H, ks.D, qbase, q_rows, qrow_base, w, q_scale, ks.k,
+                  ks.k_rows, ks.k_scale, dec ? 0 : L, g, ks.Gm, ks.maxlen, ks.cache_len, 1, r0, r1,
+                  maxlim, nullptr, 0, s, &xr);
     if (st != PIVOT_OK) return st;
     // 6. ... and select on their keys
     SelectParams sp{};
@@ -586,11 +617,13 @@ pivot_status_t run_prefix_fused(int kind, const pivot_seq_t* seq, const void* qb
     sp.scan_kind = kind;
     sp.row0 = r0;
     sp.nrows = r1 - r0;
-    sp.L = L;
+    sp.L = dec ? 0 : L;
     sp.g = g;
-    sp.Gm = 1;
+    sp.Gm = dec ? ks.Gm : 1;
+    sp.maxlen = ks.maxlen;
+    sp.cache_len = ks.cache_len;
     sp.keys = fw.surv;
-    sp.S_stride = fused_surv_stride(L);
+    sp.S_stride = fused_surv_stride(L, tpi);
     sp.K = K;
     sp.split = split;
     sp.npos = L;
@@ -661,7 +694,7 @@ pivot_status_t pivot_get_device_error(void* stream) {
     const uint32_t zero = 0;
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return PIVOT_ERR_CUDA;
     if (w & ERRBIT_TIMEOUT) return PIVOT_ERR_TIMEOUT;
-    if (w & ERRBIT_DATA) return PIVOT_ERR_DEVICE;
+    if (w & (ERRBIT_DATA | ERRBIT_BOUNDS)) return PIVOT_ERR_DEVICE;
     return PIVOT_OK;
 }
 
@@ -731,9 +764,9 @@ static pivot_status_t dense_index_impl(const pivot_seq_t* seq, int32_t topk, int
         for (long long c0 = t0; c0 < t1; c0 += chunk) {
             const int r0 = (int)c0;
             const int r1 = (int)(c0 + chunk < t1 ? c0 + chunk : t1);
-            st = run_prefix_fused(SCAN_PREFILL_DENSE, seq, seq->q, seq->L, 0, seq->w, seq->q_scale,
-                                  1, P, r0, r1, r1 - 1, topk, 0, idx, score, t0, lim_shift,
-                                  out_stride, fw, s);
+            st = run_prefix_fused(SCAN_PREFILL_DENSE, key_src(seq), seq->q, seq->L, 0, seq->w,
+                                  seq->q_scale, 1, P, r0, r1, r1 - 1, topk, 0, idx, score, t0,
+                                  lim_shift, out_stride, fw, s);
             if (st != PIVOT_OK) return st;
         }
         return PIVOT_OK;
@@ -840,8 +873,8 @@ pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* p
             const int r0 = (int)c0;
             const int r1 = (int)(c0 + chunk < j1 ? c0 + chunk : j1);
             const int e_last = (r1 * g < seq->L ? r1 * g : seq->L) - 1;
-            st = run_prefix_fused(SCAN_PREFILL_PROXY, seq, pq, G, j0, pw, pq_scale, g, P, r0, r1,
-                                  e_last, C, topk, cand, cand_score, j0, 0, 0, fw, s);
+            st = run_prefix_fused(SCAN_PREFILL_PROXY, key_src(seq), pq, G, j0, pw, pq_scale, g, P,
+                                  r0, r1, e_last, C, topk, cand, cand_score, j0, 0, 0, fw, s);
             if (st != PIVOT_OK) return st;
         }
         return PIVOT_OK;
@@ -1542,7 +1575,8 @@ static pivot_status_t check_decode(const pivot_decode_t* b) {
 }
 
 struct DecodeWs {
-    float* S;       // [B*Gm or B, stride]
+    FusedWs f;      // fused selection (dense or proxy rows), when the shape takes it
+    float* S;       // [B*Gm or B, stride] otherwise
     void* pq;       // [B, H, D]
     float* pqs;     // [B]
     float* pw;      // [B, H]
@@ -1550,14 +1584,26 @@ struct DecodeWs {
     float* R;       // [B*Gm, C]
 };
 
-static size_t decode_layout(const pivot_decode_t* b, int mode, int C, DecodeWs* out, void* base,
-                            size_t cap) {
+static size_t decode_layout(const pivot_decode_t* b, int mode, int C, int topk, DecodeWs* out,
+                            void* base, size_t cap) {
     Carver c{static_cast<uint8_t*>(base), base ? cap : ~size_t(0) / 2};
     if (!base) c.base = reinterpret_cast<uint8_t*>(WS_ALIGN);   // size query only
     const long long stride = score_stride(b->maxlen);
     const int rows = mode == PIVOT_MODE_DENSE ? b->B * b->Gm : b->B;
     DecodeWs w{};
-    w.S = static_cast<float*>(c.take((size_t)rows * stride * 4));
+    const int K = mode == PIVOT_MODE_DENSE ? topk : C;
+    if (fused_ok(b->H, b->D, b->dtype, K)) {
+        const int tpi = scan_tiles_per_item(SCAN_DECODE_DENSE);
+        const int L = b->maxlen;
+        w.f.samp = static_cast<float*>(c.take((size_t)rows * fused_samp_stride(L) * 4));
+        w.f.surv = static_cast<uint64_t*>(c.take((size_t)rows * fused_surv_stride(L, tpi) * 8));
+        w.f.count = static_cast<uint32_t*>(c.take((size_t)rows * fused_nchunks(L, tpi) * 4));
+        w.f.bound = static_cast<uint32_t*>(c.take((size_t)rows * 4));
+        w.f.miss = static_cast<int32_t*>(c.take((size_t)rows * 4));
+        w.f.nmiss = static_cast<uint32_t*>(c.take(4));
+    } else {
+        w.S = static_cast<float*>(c.take((size_t)rows * stride * 4));
+    }
     if (mode != PIVOT_MODE_DENSE) {
         w.pq = c.take((size_t)b->B * b->H * b->D * esize_of(b->dtype));
         w.pqs = static_cast<float*>(c.take((size_t)b->B * 4));
@@ -1573,7 +1619,7 @@ static size_t decode_layout(const pivot_decode_t* b, int mode, int C, DecodeWs* 
 size_t pivot_decode_workspace_size(const pivot_decode_t* b, int32_t mode, int32_t C, int32_t topk) {
     if (check_decode(b) != PIVOT_OK || mode < 0 || mode > 2 || topk < 1) return 0;
     if (mode != PIVOT_MODE_DENSE && C < topk) return 0;
-    return decode_layout(b, mode, C, nullptr, nullptr, 0);
+    return decode_layout(b, mode, C, topk, nullptr, nullptr, 0);
 }
 
 // The workspace of a whole indexer pass, from sizes alone (no buffers): the
@@ -1626,13 +1672,18 @@ pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, in
     if (st != PIVOT_OK) return st;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
     DecodeWs w;
-    if (decode_layout(b, mode, C, &w, ws, ws_bytes) == 0) return PIVOT_ERR_WORKSPACE;
+    if (decode_layout(b, mode, C, topk, &w, ws, ws_bytes) == 0) return PIVOT_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const long long stride = score_stride(b->maxlen);
     const long long krows = (long long)b->B * b->maxlen;
+    const KeySrc ks{b->dtype, b->H, b->D, b->kc, krows, b->kc_scale, b->maxlen, b->Gm, b->maxlen,
+                    b->cache_len};
     if (mode == PIVOT_MODE_DENSE) {
         const int rows = b->B * b->Gm;
         const int P = decode_dense_rows(b->Gm, b->H, b->D, b->dtype);
+        if (w.f.surv)
+            return run_prefix_fused(SCAN_DECODE_DENSE, ks, b->q, rows, 0, b->w, b->q_scale, 1, P, 0,
+                                    rows, b->maxlen - 1, topk, 0, idx, nullptr, 0, 0, 0, w.f, s);
         st = run_scan(SCAN_DECODE_DENSE, b->dtype, b->H, b->D, b->q, rows, 0, b->w, b->q_scale,
                       b->kc, krows, b->kc_scale, 0, 1, b->Gm, b->maxlen, b->cache_len, P, 0, rows,
                       b->maxlen - 1, w.S, stride, s);
@@ -1659,12 +1710,18 @@ pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, in
     if ((st = from_cuda(profiled(PK_REDUCE, 0.0, s, [&] { return launch_proxy_reduce(rp, s); }))) !=
         PIVOT_OK)
         return st;
-    st = run_scan(SCAN_DECODE_PROXY, b->dtype, b->H, b->D, w.pq, b->B, 0, w.pw,
-                  b->dtype == PIVOT_E4M3 ? w.pqs : nullptr, b->kc, krows, b->kc_scale, 0, 1, b->Gm,
-                  b->maxlen, b->cache_len, 1, 0, b->B, b->maxlen - 1, w.S, stride, s);
-    if (st != PIVOT_OK) return st;
-    st = run_select_prefix(SCAN_DECODE_PROXY, 0, b->B, 0, 1, b->Gm, b->maxlen, b->cache_len, w.S,
-                           stride, C, topk, b->maxlen, w.cand, nullptr, 0, s);
+    if (w.f.surv) {
+        st = run_prefix_fused(SCAN_DECODE_PROXY, ks, w.pq, b->B, 0, w.pw,
+                              b->dtype == PIVOT_E4M3 ? w.pqs : nullptr, 1, 1, 0, b->B,
+                              b->maxlen - 1, C, topk, w.cand, nullptr, 0, 0, 0, w.f, s);
+    } else {
+        st = run_scan(SCAN_DECODE_PROXY, b->dtype, b->H, b->D, w.pq, b->B, 0, w.pw,
+                      b->dtype == PIVOT_E4M3 ? w.pqs : nullptr, b->kc, krows, b->kc_scale, 0, 1,
+                      b->Gm, b->maxlen, b->cache_len, 1, 0, b->B, b->maxlen - 1, w.S, stride, s);
+        if (st != PIVOT_OK) return st;
+        st = run_select_prefix(SCAN_DECODE_PROXY, 0, b->B, 0, 1, b->Gm, b->maxlen, b->cache_len,
+                               w.S, stride, C, topk, b->maxlen, w.cand, nullptr, 0, s);
+    }
     if (st != PIVOT_OK) return st;
     if (cand)
         if (cudaMemcpyAsync(cand, w.cand, (size_t)b->B * C * 4, cudaMemcpyDeviceToDevice, s) !=

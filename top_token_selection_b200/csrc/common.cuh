@@ -22,6 +22,7 @@ namespace pivot {
 enum : uint32_t {
     ERRBIT_TIMEOUT = 1u,     // a bounded wait ran out
     ERRBIT_DATA = 2u,        // bad device-side data (e.g. a cache length)
+    ERRBIT_BOUNDS = 4u,      // a debug-build check of a kernel's own indexing failed
 };
 
 // One word per device (a __device__ variable lives once per GPU that loads
@@ -31,6 +32,20 @@ extern __device__ uint32_t g_error_word;
 extern __device__ uint64_t g_wait_limit_ns;
 
 __device__ __forceinline__ void raise_error(uint32_t bit) { atomicOr(&g_error_word, bit); }
+
+// Checks of the kernels' own index invariants, on in the debug build
+// (PIVOT_DEBUG defined): a false condition raises ERRBIT_BOUNDS and the
+// access it guards is skipped -- never a trap.  In the normal build the
+// check is the constant true and costs nothing.
+#ifdef PIVOT_DEBUG
+__device__ __forceinline__ bool pivot_check(bool ok) {
+    if (!ok) raise_error(ERRBIT_BOUNDS);
+    return ok;
+}
+#define PIVOT_CHECK(cond) ::pivot::pivot_check(cond)
+#else
+#define PIVOT_CHECK(cond) true
+#endif
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;

@@ -125,8 +125,10 @@ struct SelectParams {
 // scan gives each row a bound, the filter-mode scan keeps the scores at or
 // above it, and one warp per row selects the top K among them.
 struct FusedSelectParams {
-    int scan_kind;            // SCAN_PREFILL_DENSE or SCAN_PREFILL_PROXY
+    int scan_kind;            // SCAN_PREFILL_* or SCAN_DECODE_*
     int row0, nrows, L, g;
+    int Gm, maxlen;           // decode rows: limits from the device cache lengths
+    const int32_t* cache_len;
     int lim_shift;            // positions considered are <= lim(r) - lim_shift
     int K, split, rank_order;
     // samples: row r's sample scores at samp + (r - row0) * samp_stride,

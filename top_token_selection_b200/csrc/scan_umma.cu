@@ -111,7 +111,7 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
             }
             it.row_first = p.row_list[slot];
             it.rows = 1;
-            it.keybase = 0;
+            it.keybase = scan_key_base(p, it.row_first);
         } else if (p.kind == SCAN_VARLEN_DENSE || p.kind == SCAN_VARLEN_PROXY) {
             // blocks never straddle two sequences: each is one sequence's;
             // rows outside the launch's [row0, row0 + nrows) are dropped
@@ -629,7 +629,8 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                                 uint32_t base = 0;
                                 if (lane == leader) base = atomicAdd(&cnt_cur[pr], (uint32_t)__popc(m));
                                 base = __shfl_sync(0xffffffffu, base, leader);
-                                if (keep) {
+                                if (keep && PIVOT_CHECK(base + __popc(m & ((1u << lane) - 1u)) <
+                                                        (uint32_t)(p.tiles_per_item * 128))) {
                                     const uint32_t u = ordered_key(score);
                                     p.surv[(size_t)(it.row_first + pr - p.row0) * p.surv_stride +
                                            (size_t)it.chunk * (p.tiles_per_item * 128) + base +
@@ -637,7 +638,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                                         ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)spos);
                                 }
                             }
-                        } else if (col_ok && spos <= lim_r[lr]) {
+                        } else if (col_ok && spos <= lim_r[lr] && PIVOT_CHECK(s < p.S_stride)) {
                             // streaming store: keep L2 for the keys
                             __stcs(p.S + (size_t)(it.row_first + pr - p.row0) * p.S_stride + s,
                                    score);

@@ -307,8 +307,11 @@ __device__ void mark_top(const uint64_t* buf, int cnt, uint32_t Tu, uint32_t nee
         const uint64_t k = buf[i];
         const uint32_t u = key_u(k);
         const int pos = key_pos(k);
-        if (u > Tu) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
-        else if (u == Tu) ++nties;
+        if (u > Tu) {
+            if (PIVOT_CHECK(pos >= 0 && (pos >> 5) < W)) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+        } else if (u == Tu) {
+            ++nties;
+        }
     }
     nties = block_sum_u32(nties, scratch);   // also orders the marks above
     if (nties <= need) {
@@ -316,7 +319,7 @@ __device__ void mark_top(const uint64_t* buf, int cnt, uint32_t Tu, uint32_t nee
             const uint64_t k = buf[i];
             if (key_u(k) == Tu) {
                 const int pos = key_pos(k);
-                atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+                if (PIVOT_CHECK(pos >= 0 && (pos >> 5) < W)) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
             }
         }
         __syncthreads();
@@ -328,7 +331,7 @@ __device__ void mark_top(const uint64_t* buf, int cnt, uint32_t Tu, uint32_t nee
         const uint64_t k = buf[i];
         if (key_u(k) == Tu) {
             const int pos = key_pos(k);
-            atomicOr(&tie[pos >> 5], 1u << (pos & 31));
+            if (PIVOT_CHECK(pos >= 0 && (pos >> 5) < W)) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
         }
     }
     __syncthreads();
@@ -337,7 +340,8 @@ __device__ void mark_top(const uint64_t* buf, int cnt, uint32_t Tu, uint32_t nee
         const uint64_t k = buf[i];
         if (key_u(k) == Tu) {
             const int pos = key_pos(k);
-            if (rank_of(tie, pref, pos) < need) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+            if (PIVOT_CHECK(pos >= 0 && (pos >> 5) < W) && rank_of(tie, pref, pos) < need)
+                atomicOr(&bm[pos >> 5], 1u << (pos & 31));
         }
     }
     __syncthreads();
@@ -346,14 +350,17 @@ __device__ void mark_top(const uint64_t* buf, int cnt, uint32_t Tu, uint32_t nee
 // Write every kept entry whose position is marked in `bm` at slot
 // base + (its rank among the marked positions).
 __device__ void write_marked(const uint64_t* buf, int cnt, const uint32_t* bm, uint32_t* pref,
-                             int W, uint32_t base, uint32_t* scratch, int32_t* out, float* outs) {
+                             int W, uint32_t base, uint32_t* scratch, int32_t* out, float* outs,
+                             int kmax) {
     bitmap_prefix(bm, pref, W, scratch);
     for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
         const uint64_t k = buf[i];
         if (k == 0) continue;   // an empty slot (candidate rows keep them in place)
         const int pos = key_pos(k);
+        if (!PIVOT_CHECK(pos >= 0 && (pos >> 5) < W)) continue;
         if (bit_of(bm, pos)) {
             const uint32_t slot = base + rank_of(bm, pref, pos);
+            if (!PIVOT_CHECK(slot < (uint32_t)kmax)) continue;
             out[slot] = pos;
             if (outs) outs[slot] = key_to_float(key_u(k));
         }
@@ -562,16 +569,16 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
         return true;
     }
     if (!split) {
-        write_marked(buf, n, sm.bmS, sm.pref, W, 0, scratch, out, outs);
+        write_marked(buf, n, sm.bmS, sm.pref, W, 0, scratch, out, outs, K);
     } else {
         // class A: the top `split`; class B: the rest of the selected set
         for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmA[w] = 0;
         __syncthreads();
         mark_top(buf, n, TuS, (uint32_t)split - aboveS, sm.bmA, sm.bmT, sm.pref, W, scratch);
-        write_marked(buf, n, sm.bmA, sm.pref, W, 0, scratch, out, outs);
+        write_marked(buf, n, sm.bmA, sm.pref, W, 0, scratch, out, outs, K);
         for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmT[w] = sm.bmS[w] & ~sm.bmA[w];
         __syncthreads();
-        write_marked(buf, n, sm.bmT, sm.pref, W, (uint32_t)split, scratch, out, outs);
+        write_marked(buf, n, sm.bmT, sm.pref, W, (uint32_t)split, scratch, out, outs, K);
     }
     pad_row(Kp, K, out, outs);
     return true;
@@ -1074,6 +1081,7 @@ __global__ void __launch_bounds__(CW_MAX_WARPS * 32) select_cand_kernel(const Se
                 const int own = in_a ? i : i - a;
                 const uint32_t pos = key_upos(k);
                 const int slot = own + (in_a ? count_below(eb, b, pos) : count_below(e, a, pos));
+                if (!PIVOT_CHECK(slot >= 0 && slot < (int)Kp)) continue;
                 out[slot] = (int32_t)pos;
                 if (outs) outs[slot] = key_to_float(key_u(k));
             }
@@ -1121,12 +1129,9 @@ constexpr int FB_WARPS = 8;              // bound kernel: rows a block
 constexpr int FB_MAX_SAMPLES = 4096;     // samples a bound reads at most
 constexpr int FF_MAX_WARPS = 8;
 
-__device__ __forceinline__ int prefill_lim(int kind, int r, int L, int g) {
-    if (kind == SCAN_PREFILL_PROXY) {
-        const int e = (r + 1) * g;
-        return (e < L ? e : L) - 1;
-    }
-    return r;
+// Row r's causal limit (-1 with ok = false for a bad cache length).
+__device__ __forceinline__ int fused_lim(const FusedSelectParams& p, int r, bool& ok) {
+    return row_limit(p.scan_kind, r, p.L, p.g, p.Gm, p.maxlen, p.cache_len, ok);
 }
 
 // Sample columns at positions <= lim (sample j sits at position
@@ -1147,10 +1152,11 @@ __global__ void __launch_bounds__(FB_WARPS * 32) sample_bound_kernel(const Fused
     if (rr >= p.nrows) return;
     uint32_t* v = reinterpret_cast<uint32_t*>(smem_b) + (size_t)warp * (FB_MAX_SAMPLES + THR_BINS);
     uint32_t* hist = v + FB_MAX_SAMPLES;
-    const int lim = prefill_lim(p.scan_kind, p.row0 + rr, p.L, p.g) - p.lim_shift;
+    bool ok;
+    const int lim = fused_lim(p, p.row0 + rr, ok) - p.lim_shift;
     const int n = lim + 1;
     uint32_t T = 1;
-    if (n > p.cap) {
+    if (ok && n > p.cap) {
         const int ns = samples_upto(lim, p.kts);
         const int step = (ns + FB_MAX_SAMPLES - 1) / FB_MAX_SAMPLES;
         const int nt = (ns + step - 1) / step;
@@ -1206,8 +1212,10 @@ __global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const F
     uint64_t* e = reinterpret_cast<uint64_t*>(smem_f + (size_t)warp * ((size_t)M * 8 + THR_BINS * 4));
     uint32_t* hist = reinterpret_cast<uint32_t*>(e + M);
     const int r = p.row0 + rr;
-    const int lim = prefill_lim(p.scan_kind, r, p.L, p.g) - p.lim_shift;
-    const int n = lim >= 0 ? lim + 1 : 0;
+    bool ok;
+    const int lim = fused_lim(p, r, ok) - p.lim_shift;
+    if (!ok && lane == 0) raise_error(ERRBIT_DATA);
+    const int n = (ok && lim >= 0) ? lim + 1 : 0;
     const int K = p.K;
     const size_t ostride = p.out_stride ? (size_t)p.out_stride : (size_t)K;
     int32_t* out = p.out_idx + (size_t)(r - p.out_base) * ostride;
@@ -1233,13 +1241,41 @@ __global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const F
         return;
     }
     if (Kp > 0) {
-        // the row's survivors, chunk after chunk
-        int off = 0;
+        // the row's survivors, chunk after chunk: an exclusive prefix of the
+        // chunk counts (in the histogram's space), then every lane copies
+        // entries, finding each one's chunk by binary search
         const uint64_t* src = p.surv + (size_t)rr * p.surv_stride;
-        for (int c = 0; c < nch; ++c) {
-            const int k = (int)cnt[c];
-            for (int i = lane; i < k; i += 32) e[off + i] = src[(size_t)c * p.chunk_keys + i];
-            off += k;
+        if (nch <= THR_BINS) {
+            uint32_t carry = 0;
+            for (int c0 = 0; c0 < nch; c0 += 32) {
+                const int c = c0 + lane;
+                const uint32_t k = c < nch ? cnt[c] : 0u;
+                uint32_t inc = k;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += y;
+                }
+                if (c < nch) hist[c] = carry + inc - k;
+                carry += __shfl_sync(0xffffffffu, inc, 31);
+            }
+            __syncwarp();
+            for (int i = lane; i < (int)total; i += 32) {
+                int lo = 0, hi = nch - 1;   // the last chunk whose start is <= i
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (hist[mid] <= (uint32_t)i) lo = mid;
+                    else hi = mid - 1;
+                }
+                if (PIVOT_CHECK(i < M && i - hist[lo] < (uint32_t)p.chunk_keys))
+                    e[i] = src[(size_t)lo * p.chunk_keys + (i - hist[lo])];
+            }
+        } else {
+            int off = 0;
+            for (int c = 0; c < nch; ++c) {
+                const int k = (int)cnt[c];
+                for (int i = lane; i < k; i += 32) e[off + i] = src[(size_t)c * p.chunk_keys + i];
+                off += k;
+            }
         }
         __syncwarp();
         const int nt = (int)total;
@@ -1293,7 +1329,8 @@ __global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const F
                     const bool inA = !split || u > TA || (u == TA && (uint32_t)k >= LA);
                     if (inA == (cls == 0)) {
                         const int pos = key_pos(k);
-                        atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+                        if (PIVOT_CHECK(pos >= 0 && (pos >> 5) < W))
+                            atomicOr(&bm[pos >> 5], 1u << (pos & 31));
                     }
                 }
                 __syncwarp();
@@ -1319,8 +1356,10 @@ __global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const F
                     const bool inA = !split || u > TA || (u == TA && (uint32_t)k >= LA);
                     if (inA == (cls == 0)) {
                         const int pos = key_pos(k);
+                        if (!PIVOT_CHECK(pos >= 0 && (pos >> 5) < W)) continue;
                         const uint32_t slot =
                             base + pref[pos >> 5] + __popc(bm[pos >> 5] & ((1u << (pos & 31)) - 1u));
+                        if (!PIVOT_CHECK(slot < Kp)) continue;
                         out[slot] = pos;
                         if (outs) outs[slot] = key_to_float(u);
                     }
