@@ -454,7 +454,7 @@ int run_fused(int L, int K, int split, int dist, int nrows, int r0, int order, f
     std::mt19937 rng(31 + 7 * dist + K + r0);
     std::vector<float> samp((size_t)nrows * ss, 0.0f);
     std::vector<uint64_t> surv((size_t)nrows * sv, 0);
-    std::vector<uint32_t> cnt((size_t)nrows * nch, 0xDEADu), bound(nrows);
+    std::vector<uint32_t> cnt((size_t)nrows * nch * 4, 0xDEADu), bound(nrows);
     std::vector<int32_t> miss(nrows, -9), out((size_t)nrows * K, -7);
     std::vector<float> outs((size_t)nrows * K);
     uint32_t nmiss = 12345;
@@ -489,6 +489,8 @@ int run_fused(int L, int K, int split, int dist, int nrows, int r0, int order, f
     fp.surv_count = cnt.data();
     fp.nchunks = nch;
     fp.chunk_keys = CK;
+    fp.nsub = 4;
+    fp.sub_keys = CK / 4;
     fp.out_idx = out.data();
     fp.out_score = outs.data();
     fp.out_base = r0;
@@ -496,24 +498,36 @@ int run_fused(int L, int K, int split, int dist, int nrows, int r0, int order, f
     fp.miss_count = &nmiss;
     if (launch_sample_bound(fp, nullptr) != cudaSuccess) return 2;
     if (nmiss != 0) { std::printf("miss count not cleared\n"); return 3; }
-    // the filter scan: appends, then each chunk's count
+    // the filter scan: each epilogue warp appends the survivors among its
+    // TMEM lane quarter's keys (32 of every 128-key tile) to its own
+    // sub-region of the chunk, in an order the emulation shuffles, and
+    // writes the count
+    auto key_of = [&](int i, int pos) {
+        return ((uint64_t)okey(S[i][pos]) << 32) | (0xFFFFFFFFu - (uint32_t)pos);
+    };
     auto fill = [&](int i, uint32_t T) {
         const float tf = T <= 0x00800000u ? -INFINITY : key_to_float(T);
         const int lim = lim_of(r0 + i);
         for (int c = 0; c * CK <= lim; ++c) {
-            std::vector<uint64_t> kept;
-            for (int pos = c * CK; pos <= std::min(lim, (c + 1) * CK - 1); ++pos)
-                if (S[i][pos] >= tf)
-                    kept.push_back(((uint64_t)okey(S[i][pos]) << 32) | (0xFFFFFFFFu - (uint32_t)pos));
-            std::shuffle(kept.begin(), kept.end(), rng);
-            std::copy(kept.begin(), kept.end(), surv.begin() + (size_t)i * sv + (size_t)c * CK);
-            cnt[(size_t)i * nch + c] = (uint32_t)kept.size();
+            for (int q = 0; q < 4; ++q) {
+                std::vector<uint64_t> kept;
+                for (int pos = c * CK; pos <= std::min(lim, (c + 1) * CK - 1); ++pos)
+                    if ((pos % 128) / 32 == q && S[i][pos] >= tf) kept.push_back(key_of(i, pos));
+                std::shuffle(kept.begin(), kept.end(), rng);
+                std::copy(kept.begin(), kept.end(),
+                          surv.begin() + (size_t)i * sv + (size_t)c * CK + (size_t)q * (CK / 4));
+                cnt[((size_t)i * nch + c) * 4 + q] = (uint32_t)kept.size();
+            }
         }
     };
     for (int i = 0; i < nrows; ++i) fill(i, bound[i]);
     if (launch_fused_finish(fp, nullptr) != cudaSuccess) return 2;
-    // the fallback: listed rows keep everything, then the block select on keys
-    for (uint32_t m = 0; m < nmiss; ++m) fill(miss[m] - r0, 1u);
+    // the fallback: the listed rows' rescan keeps every key, each at its own
+    // position, then the block select reads them as keys
+    for (uint32_t m = 0; m < nmiss; ++m) {
+        const int i = miss[m] - r0;
+        for (int pos = 0; pos <= lim_of(r0 + i); ++pos) surv[(size_t)i * sv + pos] = key_of(i, pos);
+    }
     SelectParams sp{};
     sp.kind = SEL_PREFIX;
     sp.scan_kind = fp.scan_kind;

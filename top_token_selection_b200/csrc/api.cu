@@ -484,7 +484,7 @@ long long fused_surv_stride(int L, int tpi = FUSED_TILES) {
 // per row: samples, survivor regions, chunk counts, the bound, a miss slot
 size_t fused_rowbytes(int L, int tpi = FUSED_TILES) {
     return (size_t)fused_samp_stride(L) * 4 + (size_t)fused_surv_stride(L, tpi) * 8 +
-           (size_t)fused_nchunks(L, tpi) * 4 + 4 + 4;
+           (size_t)fused_nchunks(L, tpi) * 4 * 4 + 4 + 4;
 }
 constexpr size_t FUSED_FIXED = 8 * WS_ALIGN;   // alignment of the six arrays, the miss count
 
@@ -502,7 +502,7 @@ bool fused_carve(void* ws, size_t bytes, long long rows, int L, FusedWs* w,
     Carver c{static_cast<uint8_t*>(ws), bytes};
     w->samp = static_cast<float*>(c.take((size_t)rows * fused_samp_stride(L) * 4));
     w->surv = static_cast<uint64_t*>(c.take((size_t)rows * fused_surv_stride(L, tpi) * 8));
-    w->count = static_cast<uint32_t*>(c.take((size_t)rows * fused_nchunks(L, tpi) * 4));
+    w->count = static_cast<uint32_t*>(c.take((size_t)rows * fused_nchunks(L, tpi) * 4 * 4));
     w->bound = static_cast<uint32_t*>(c.take((size_t)rows * 4));
     w->miss = static_cast<int32_t*>(c.take((size_t)rows * 4));
     w->nmiss = static_cast<uint32_t*>(c.take(4));
@@ -577,6 +577,8 @@ pivot_status_t run_prefix_fused(int kind, const KeySrc& ks, const void* qbase,
     fp.surv_count = fw.count;
     fp.nchunks = fused_nchunks(L, tpi);
     fp.chunk_keys = tpi * 128;
+    fp.nsub = 4;                 // one sub-region per TMEM lane quarter
+    fp.sub_keys = tpi * 32;
     fp.out_idx = out;
     fp.out_score = out_score;
     fp.out_base = out_base;
@@ -1597,7 +1599,7 @@ static size_t decode_layout(const pivot_decode_t* b, int mode, int C, int topk, 
         const int L = b->maxlen;
         w.f.samp = static_cast<float*>(c.take((size_t)rows * fused_samp_stride(L) * 4));
         w.f.surv = static_cast<uint64_t*>(c.take((size_t)rows * fused_surv_stride(L, tpi) * 8));
-        w.f.count = static_cast<uint32_t*>(c.take((size_t)rows * fused_nchunks(L, tpi) * 4));
+        w.f.count = static_cast<uint32_t*>(c.take((size_t)rows * fused_nchunks(L, tpi) * 4 * 4));
         w.f.bound = static_cast<uint32_t*>(c.take((size_t)rows * 4));
         w.f.miss = static_cast<int32_t*>(c.take((size_t)rows * 4));
         w.f.nmiss = static_cast<uint32_t*>(c.take(4));

@@ -48,11 +48,14 @@ struct ScanParams {
     // prefix; its scores go to columns t*128 + (key in tile).  0 or 1: every tile.
     int key_tile_stride;
     // Filter mode (surv set; the selection fused into the scan): a score
-    // >= its row's bound is appended, as a 64-bit key (ordered score << 32 |
-    // ~position), to the row's region for the item's key chunk -- row r,
-    // chunk c at surv + (r - row0) * surv_stride + c * tiles_per_item * 128 --
-    // and the chunk's count goes to surv_count[(r - row0) * nchunks + c].  No
-    // score is written to S.
+    // >= its row's bound is kept as a 64-bit key (ordered score << 32 |
+    // ~position).  Row r's region is surv + (r - row0) * surv_stride; chunk c
+    // of it (tiles_per_item * 128 keys) holds four sub-regions of
+    // tiles_per_item * 32, one per TMEM lane quarter, each filled by one
+    // epilogue warp from the front, its count at
+    // surv_count[((r - row0) * nchunks + c) * 4 + quarter].  In row-list mode
+    // (the keep-everything rescan) every key goes to its own position in the
+    // region instead, and no count is written.  No score is written to S.
     const uint32_t* bound;  // [nrows]: row r's bound (an ordered key) at bound[r - row0];
                             // keys <= 0x00800000 keep every score; NULL keeps every score
     uint64_t* surv;
@@ -139,12 +142,13 @@ struct FusedSelectParams {
     float sigmas;             // margin of the bound, in standard deviations of the count
     uint32_t* bound;          // [nrows] out: row r's bound (an ordered key; 1 keeps all)
     int cap;                  // survivors a row may have for the warp select
-    // survivors: row r, chunk c at surv + (r - row0) * surv_stride + c * chunk_keys,
-    // surv_count[(r - row0) * nchunks + c] of them
+    // survivors: row r's segment s = chunk * nsub + sub at surv + (r - row0) *
+    // surv_stride + chunk * chunk_keys + sub * sub_keys, with
+    // surv_count[(r - row0) * nchunks * nsub + s] of them
     const uint64_t* surv;
     long long surv_stride;
     const uint32_t* surv_count;
-    int nchunks, chunk_keys;
+    int nchunks, chunk_keys, nsub, sub_keys;
     int32_t* out_idx;         // row r at out_idx + (r - out_base) * (out_stride or K)
     float* out_score;         // or NULL
     int out_base, out_stride;

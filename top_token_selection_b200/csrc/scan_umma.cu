@@ -212,10 +212,6 @@ __global__ void __maxnreg__(SCAN_MAXREG)
     float* w_s = reinterpret_cast<float*>(tmem_holder + 4);   // [256], 16-byte aligned
     float* sq_s = w_s + 256;                                   // [PMAX]
     int* lim_s = reinterpret_cast<int*>(sq_s + PMAX);          // [PMAX]
-    // filter mode (H >= 32, where the weight table is unused): survivors of
-    // each row of the current item, double-buffered by the epilogue's item
-    // parity, in the weight table's space
-    uint32_t* cnt_s = reinterpret_cast<uint32_t*>(w_s);   // [2][PMAX], PMAX <= 8 here
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -227,8 +223,6 @@ __global__ void __maxnreg__(SCAN_MAXREG)
         if (lim < nitems) nitems = (int)lim;
     }
 
-    if (FILTER && HEADS >= 32)
-        for (int i = threadIdx.x; i < 2 * PMAX; i += blockDim.x) cnt_s[i] = 0;
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             // gather mode: both gathering warps publish each tile
@@ -492,8 +486,8 @@ __global__ void __maxnreg__(SCAN_MAXREG)
         int lim_r[RROWS];
         float sq_r[RROWS];
         float tf_r[RROWS];    // filter mode: scores >= tf_r are kept
+        uint32_t nkept[RROWS];  // filter mode: this warp's survivors of the item, per row
         int ntile = 0;
-        int nit_e = 0;        // valid items this CTA's epilogue has walked
         const int kts = p.key_tile_stride > 1 ? p.key_tile_stride : 1;
         constexpr bool filter = FILTER && !GATHER && HEADS >= 32;
         // Once a wait runs out the warp stops touching TMEM and memory but
@@ -536,6 +530,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                     lim_r[lr] = pr < r_hi ? row_lim(pr) : -1;
                     sq_r[lr] = row_sq(pr);
                     tf_r[lr] = -INFINITY;
+                    nkept[lr] = 0;
                     if (filter && live && p.bound) {
                         const uint32_t T = p.bound[it.row_first + pr - p.row0];
                         if (T > 0x00800000u) tf_r[lr] = key_to_float(T);
@@ -568,7 +563,6 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 const int s_t = t * kts * 128 + key_in_tile;
                 return s_t <= it.maxlim ? ld_nc_early(p.k_scale + it.keybase + s_t) : 1.0f;
             };
-            uint32_t* cnt_cur = cnt_s + (nit_e & 1) * PMAX;
             float sk_next = key_scale(it.t0);
             for (int t = it.t0; t < it.t1; ++t) {
                 const int acc = ntile & 1;
@@ -619,25 +613,30 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                                              ((lo[2] + hi[2]) + (lo[3] + hi[3]));
                         const float score = rowsum * sq_r[lr] * sk;
                         if constexpr (filter) {
-                            // survivors only: warp-aggregated append to the
-                            // row's region for this chunk
+                            // survivors only, appended to this warp's own
+                            // sub-region of the row's chunk (its TMEM lane
+                            // quarter: 32 keys of every tile of the item),
+                            // counted in a register; the keep-everything
+                            // rescan of listed rows writes each key at its
+                            // own position instead
                             const bool keep = spos <= lim_r[lr] - p.lim_shift &&
                                               score >= tf_r[lr];
                             const unsigned m = __ballot_sync(0xffffffffu, keep);
-                            if (m) {
-                                const int leader = __ffs(m) - 1;
-                                uint32_t base = 0;
-                                if (lane == leader) base = atomicAdd(&cnt_cur[pr], (uint32_t)__popc(m));
-                                base = __shfl_sync(0xffffffffu, base, leader);
-                                if (keep && PIVOT_CHECK(base + __popc(m & ((1u << lane) - 1u)) <
-                                                        (uint32_t)(p.tiles_per_item * 128))) {
-                                    const uint32_t u = ordered_key(score);
-                                    p.surv[(size_t)(it.row_first + pr - p.row0) * p.surv_stride +
-                                           (size_t)it.chunk * (p.tiles_per_item * 128) + base +
-                                           __popc(m & ((1u << lane) - 1u))] =
-                                        ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)spos);
+                            if (keep) {
+                                const uint32_t at = nkept[lr] + __popc(m & ((1u << lane) - 1u));
+                                const uint64_t key =
+                                    ((uint64_t)ordered_key(score) << 32) |
+                                    (uint64_t)(0xFFFFFFFFu - (uint32_t)spos);
+                                uint64_t* row = p.surv + (size_t)(it.row_first + pr - p.row0) *
+                                                             p.surv_stride;
+                                if (p.row_list) {
+                                    if (PIVOT_CHECK(spos < p.surv_stride)) row[spos] = key;
+                                } else if (PIVOT_CHECK(at < (uint32_t)(p.tiles_per_item * 32))) {
+                                    row[(size_t)it.chunk * (p.tiles_per_item * 128) +
+                                        (size_t)quarter * (p.tiles_per_item * 32) + at] = key;
                                 }
                             }
+                            nkept[lr] += __popc(m);
                         } else if (col_ok && spos <= lim_r[lr] && PIVOT_CHECK(s < p.S_stride)) {
                             // streaming store: keep L2 for the keys
                             __stcs(p.S + (size_t)(it.row_first + pr - p.row0) * p.S_stride + s,
@@ -672,16 +671,17 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 if (lane == 0) mbar_arrive(&accempty[acc]);
             }
             if constexpr (filter) {
-                // every append of this item has counted: publish the rows'
-                // counts, and clear this buffer for item nit_e + 2 (the next
-                // item uses the other one)
-                named_bar_sync(2, EPI_WARPS * 32);
-                if (et < it.rows && !aborted)
-                    p.surv_count[(size_t)(it.row_first + et - p.row0) * p.nchunks + it.chunk] =
-                        cnt_cur[et];
-                if (et < PMAX) cnt_cur[et] = 0;
+                // this warp's survivor counts of the item, one per row it owns
+                if (lane == 0 && !aborted && !p.row_list) {
+#pragma unroll
+                    for (int lr = 0; lr < RROWS; ++lr) {
+                        const int pr = r_lo + lr;
+                        if (pr < r_hi && pr < it.rows)
+                            p.surv_count[((size_t)(it.row_first + pr - p.row0) * p.nchunks +
+                                          it.chunk) * 4 + quarter] = nkept[lr];
+                    }
+                }
             }
-            ++nit_e;
         }
     }
 

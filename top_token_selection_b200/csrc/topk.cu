@@ -801,15 +801,9 @@ __device__ uint32_t warp_kth_largest_f(F get, int n, uint32_t m, uint32_t* hist)
 #pragma unroll
         for (int b = 0; b < THR_BINS / 32; ++b) hist[b * 32 + lane] = 0;
         __syncwarp();
-        // lanes landing in one bin add once (the keys of a row cluster in
-        // few bins, and same-address shared atomics serialise)
-        for (int i0 = 0; i0 < n; i0 += 32) {
-            const int i = i0 + lane;
-            const uint32_t u = i < n ? get(i) : 0u;
-            const bool in = u && u >= lo && u <= hi;
-            const uint32_t bin = in ? (u - lo) >> sh : 0xFFFFFFFFu;
-            const unsigned peers = __match_any_sync(0xffffffffu, bin);
-            if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+        for (int i = lane; i < n; i += 32) {
+            const uint32_t u = get(i);
+            if (u && u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> sh], 1u);
         }
         __syncwarp();
         // lane l owns the 8 bins [THR_BINS - 8 (l + 1), THR_BINS - 8 l)
@@ -918,6 +912,7 @@ __host__ __device__ int pow2_at_least(int x) {
 }
 
 constexpr int CW_MAX_WARPS = 8;
+constexpr int CW_BATCH = 8;              // independent loads a lane issues at once
 constexpr size_t CW_SMEM_LIMIT = 200 * 1024;
 
 __host__ __device__ int cw_slots(int C) { return pow2_at_least(C < 32 ? 32 : C); }
@@ -1008,32 +1003,57 @@ __global__ void __launch_bounds__(CW_MAX_WARPS * 32) select_cand_kernel(const Se
                                  : (var ? (size_t)p.seg.tok[seg_find(p.seg.tok, p.seg.nseq, r)]
                                         : 0));
 
-    // 1. keys; descents between consecutive candidate positions (0 or 1:
-    //    at most two ascending runs, split where the descent is)
-    uint32_t nvalid = 0, ndesc = 0;
-    int split = C;
-    int prev_last = -1;   // position of the entry before this chunk
-    for (int i0 = 0; i0 < C; i0 += 32) {
-        const int i = i0 + lane;
-        const int pos = (ok && i < C) ? cand[i] : -1;
-        const bool valid = pos >= 0 && pos <= lim;
-        float x = 0.0f;
-        if (valid) {
-            x = S[i];
-            if (ksc) x = x * ksc[pos];
+    // 1. keys: each lane issues CW_BATCH independent loads of positions and
+    //    scores, then their key scales, before using any of them (a warp has
+    //    few threads to hide a row's memory latency with)
+    uint32_t nvalid = 0;
+    for (int i0 = 0; i0 < C; i0 += 32 * CW_BATCH) {
+        int pos[CW_BATCH];
+        float x[CW_BATCH];
+#pragma unroll
+        for (int u = 0; u < CW_BATCH; ++u) {
+            const int i = i0 + u * 32 + lane;
+            pos[u] = (ok && i < C) ? cand[i] : -1;
+            x[u] = i < C ? S[i] : 0.0f;
         }
-        e[i] = valid ? make_key(ordered_key(x), pos) : 0ull;
-        nvalid += valid;
-        int before = __shfl_up_sync(0xffffffffu, pos, 1);
-        if (lane == 0) before = prev_last;
-        const unsigned dm = __ballot_sync(0xffffffffu, before >= 0 && pos >= 0 && pos < before);
-        if (dm && ndesc == 0) split = i0 + __ffs(dm) - 1;
-        ndesc += __popc(dm);
-        prev_last = __shfl_sync(0xffffffffu, pos, 31);
+        if (ksc) {
+            float sc[CW_BATCH];
+#pragma unroll
+            for (int u = 0; u < CW_BATCH; ++u)
+                sc[u] = (pos[u] >= 0 && pos[u] <= lim) ? ksc[pos[u]] : 1.0f;
+#pragma unroll
+            for (int u = 0; u < CW_BATCH; ++u) x[u] = x[u] * sc[u];
+        }
+#pragma unroll
+        for (int u = 0; u < CW_BATCH; ++u) {
+            const int i = i0 + u * 32 + lane;
+            const bool valid = pos[u] >= 0 && pos[u] <= lim;
+            if (i < C) e[i] = valid ? make_key(ordered_key(x[u]), pos[u]) : 0ull;
+            nvalid += valid;
+        }
     }
     for (int i = C + lane; i < M; i += 32) e[i] = 0ull;
     for (int o = 16; o > 0; o >>= 1) nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
     __syncwarp();
+    // descents between consecutive valid positions (0 or 1: at most two
+    // ascending runs, split where the descent is), from shared memory
+    uint32_t ndesc = 0;
+    int split = C;
+    int carry = -1;   // the last valid position before this chunk
+    for (int i0 = 0; i0 < C; i0 += 32) {
+        const int i = i0 + lane;
+        const uint64_t k = i < C ? e[i] : 0ull;
+        const int pos = k ? key_pos(k) : -1;
+        const unsigned vm = __ballot_sync(0xffffffffu, pos >= 0);
+        const unsigned below = vm & ((1u << lane) - 1u);
+        const int src = below ? 31 - __clz(below) : lane;
+        int prev = __shfl_sync(0xffffffffu, pos, src);
+        if (!below) prev = carry;
+        const unsigned dm = __ballot_sync(0xffffffffu, pos >= 0 && prev >= 0 && pos < prev);
+        if (dm && ndesc == 0) split = i0 + __ffs(dm) - 1;
+        ndesc += __popc(dm);
+        if (vm) carry = __shfl_sync(0xffffffffu, pos, 31 - __clz(vm));
+    }
     const uint32_t Kp = nvalid < (uint32_t)K ? nvalid : (uint32_t)K;
 
     // 2. keep exactly the top Kp keys (score, then lower position)
@@ -1128,6 +1148,7 @@ __global__ void __launch_bounds__(CW_MAX_WARPS * 32) select_cand_kernel(const Se
 constexpr int FB_WARPS = 8;              // bound kernel: rows a block
 constexpr int FB_MAX_SAMPLES = 4096;     // samples a bound reads at most
 constexpr int FF_MAX_WARPS = 8;
+constexpr int FF_AUX = 1024;             // warp-select words beside its entries: histogram, prefix
 
 // Row r's causal limit (-1 with ok = false for a bad cache length).
 __device__ __forceinline__ int fused_lim(const FusedSelectParams& p, int r, bool& ok) {
@@ -1209,8 +1230,8 @@ __global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const F
     const int rr = blockIdx.x * warps + warp;
     if (warp >= warps || rr >= p.nrows) return;   // whole warps; no block barriers
     const int M = p.cap;
-    uint64_t* e = reinterpret_cast<uint64_t*>(smem_f + (size_t)warp * ((size_t)M * 8 + THR_BINS * 4));
-    uint32_t* hist = reinterpret_cast<uint32_t*>(e + M);
+    uint64_t* e = reinterpret_cast<uint64_t*>(smem_f + (size_t)warp * ((size_t)M * 8 + FF_AUX * 4));
+    uint32_t* hist = reinterpret_cast<uint32_t*>(e + M);   // FF_AUX words: histogram / prefix
     const int r = p.row0 + rr;
     bool ok;
     const int lim = fused_lim(p, r, ok) - p.lim_shift;
@@ -1222,14 +1243,16 @@ __global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const F
     float* outs = p.out_score ? p.out_score + (size_t)(r - p.out_base) * ostride : nullptr;
     const uint32_t Kp = n < K ? (uint32_t)n : (uint32_t)K;
 
+    // segments (chunk, sub-region) of the row's survivors
     const int nch = n > 0 ? (n + p.chunk_keys - 1) / p.chunk_keys : 0;
-    const uint32_t* cnt = p.surv_count + (size_t)rr * p.nchunks;
-    // a count above its chunk's size (a scan that gave up left it stale)
+    const int nseg = nch * p.nsub;
+    const uint32_t* cnt = p.surv_count + (size_t)rr * p.nchunks * p.nsub;
+    // a count above its segment's size (a scan that gave up left it stale)
     // counts as a miss, so the gather below stays inside the regions
     uint32_t total = 0, over = 0;
-    for (int c = lane; c < nch; c += 32) {
+    for (int c = lane; c < nseg; c += 32) {
         const uint32_t k = cnt[c];
-        if (k > (uint32_t)p.chunk_keys) over = 1;
+        if (k > (uint32_t)p.sub_keys) over = 1;
         else total += k;
     }
     for (int o = 16; o > 0; o >>= 1) {
@@ -1241,39 +1264,56 @@ __global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const F
         return;
     }
     if (Kp > 0) {
-        // the row's survivors, chunk after chunk: an exclusive prefix of the
-        // chunk counts (in the histogram's space), then every lane copies
-        // entries, finding each one's chunk by binary search
+        // the row's survivors, segment after segment: an exclusive prefix of
+        // the segment counts (in the auxiliary space), then every lane copies
+        // entries, finding each one's segment by binary search
         const uint64_t* src = p.surv + (size_t)rr * p.surv_stride;
-        if (nch <= THR_BINS) {
+        if (nseg <= FF_AUX) {
             uint32_t carry = 0;
-            for (int c0 = 0; c0 < nch; c0 += 32) {
+            for (int c0 = 0; c0 < nseg; c0 += 32) {
                 const int c = c0 + lane;
-                const uint32_t k = c < nch ? cnt[c] : 0u;
+                const uint32_t k = c < nseg ? cnt[c] : 0u;
                 uint32_t inc = k;
                 for (int o = 1; o < 32; o <<= 1) {
                     const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
                     if (lane >= o) inc += y;
                 }
-                if (c < nch) hist[c] = carry + inc - k;
+                if (c < nseg) hist[c] = carry + inc - k;
                 carry += __shfl_sync(0xffffffffu, inc, 31);
             }
             __syncwarp();
-            for (int i = lane; i < (int)total; i += 32) {
-                int lo = 0, hi = nch - 1;   // the last chunk whose start is <= i
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (hist[mid] <= (uint32_t)i) lo = mid;
-                    else hi = mid - 1;
+            for (int i0 = 0; i0 < (int)total; i0 += 32 * CW_BATCH) {
+                // CW_BATCH independent loads a lane before any store
+                uint64_t v[CW_BATCH];
+#pragma unroll
+                for (int u = 0; u < CW_BATCH; ++u) {
+                    const int i = i0 + u * 32 + lane;
+                    v[u] = 0ull;
+                    if (i < (int)total) {
+                        int lo = 0, hi = nseg - 1;   // the last segment whose start is <= i
+                        while (lo < hi) {
+                            const int mid = (lo + hi + 1) >> 1;
+                            if (hist[mid] <= (uint32_t)i) lo = mid;
+                            else hi = mid - 1;
+                        }
+                        if (PIVOT_CHECK(i < M && i - hist[lo] < (uint32_t)p.sub_keys))
+                            v[u] = src[(size_t)(lo / p.nsub) * p.chunk_keys +
+                                       (size_t)(lo % p.nsub) * p.sub_keys + (i - hist[lo])];
+                    }
                 }
-                if (PIVOT_CHECK(i < M && i - hist[lo] < (uint32_t)p.chunk_keys))
-                    e[i] = src[(size_t)lo * p.chunk_keys + (i - hist[lo])];
+#pragma unroll
+                for (int u = 0; u < CW_BATCH; ++u) {
+                    const int i = i0 + u * 32 + lane;
+                    if (i < (int)total) e[i] = v[u];
+                }
             }
         } else {
             int off = 0;
-            for (int c = 0; c < nch; ++c) {
+            for (int c = 0; c < nseg; ++c) {
                 const int k = (int)cnt[c];
-                for (int i = lane; i < k; i += 32) e[off + i] = src[(size_t)c * p.chunk_keys + i];
+                const uint64_t* sg =
+                    src + (size_t)(c / p.nsub) * p.chunk_keys + (size_t)(c % p.nsub) * p.sub_keys;
+                for (int i = lane; i < k; i += 32) e[off + i] = sg[i];
                 off += k;
             }
         }
@@ -1520,7 +1560,7 @@ cudaError_t launch_sample_bound(const FusedSelectParams& p, cudaStream_t stream)
 
 cudaError_t launch_fused_finish(const FusedSelectParams& p, cudaStream_t stream) {
     if (p.nrows <= 0) return cudaSuccess;
-    const size_t per = (size_t)p.cap * 8 + THR_BINS * 4;
+    const size_t per = (size_t)p.cap * 8 + FF_AUX * 4;
     int warps = (int)(CW_SMEM_LIMIT / per);
     if (warps > FF_MAX_WARPS) warps = FF_MAX_WARPS;
     if (warps < 1) return cudaErrorInvalidValue;
