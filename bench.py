@@ -598,6 +598,31 @@ def measure_extra(run, wl, device, peaks, seed, reps=3):
     return out
 
 
+def measure_layers(device, seed, nlayers=4, L=16384, rho=0.9, period=2, reps=3):
+    """Cross-layer reuse of index rows (not in `value`): `nlayers` correlated
+    layers of the 16K FP8 prefill; every layer runs the dense indexer
+    (period 1) against every `period`-th layer running it and the others
+    reusing its rows; the recall of each layer's rows against its own dense
+    rows."""
+    from top_token_selection_b200 import pivot as pv
+    lay = gen.make_layers(nlayers, L, 64, 128, gen.E4M3, rho=rho, seed=seed + 29)
+    seqs = []
+    for p in lay:
+        dev = [None if t is None else t.to(device) for t in (p.q, p.q_scale, p.w, p.k, p.k_scale)]
+        seqs.append(pv.make_seq(*dev))
+    own = pv.index_layers(seqs, pv.DENSE, 8, 4096, 2048, period=1)
+    out = {"layers": nlayers, "L": L, "rho": rho, "period": period, "mode": "dense"}
+    for per in (1, period):
+        ms = _event_ms(lambda: pv.index_layers(seqs, pv.DENSE, 8, 4096, 2048, period=per),
+                       torch.cuda.current_stream(), reps)
+        out[f"period{per}_ms"] = ms
+    got = pv.index_layers(seqs, pv.DENSE, 8, 4096, 2048, period=period)
+    out["recall_per_layer"] = [recall_stats(o, r) for o, r in zip(own, got)]
+    out["speedup"] = out["period1_ms"] / out[f"period{period}_ms"]
+    assert pv.device_error() == 0
+    return out
+
+
 def time_modes(run, steps=3):
     """Per-stage CUDA-event times of `steps` warm steps of `run`: dense,
     Reuse (reduce + scan + Reuse) and Refine (reduce + scan + Refine)."""
@@ -874,6 +899,7 @@ def run_ours(args, wl):
     if not args.no_extra and world == 1:
         extra = measure_extra(run, wl, device, peaks, args.seed)
         extra["workloads"] = measure_workloads(args, device, peaks, fp8_peak)
+        extra["cross_layer_reuse"] = measure_layers(device, args.seed)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -264,6 +264,25 @@ pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* ca
                             size_t ws_bytes, void* stream);
 size_t pivot_refine_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C, int32_t topk);
 
+/* PIVOT-Refine with a per-group adaptive candidate count.  The pages fix C
+ * per run ("PIVOT in 10 minutes", Gotchas: no adaptive strategy); this is a
+ * design choice of this library, not a reading of the pages: group j
+ * re-scores only its first C_j candidates, those whose proxy score is at
+ * least rho times the proxy's k-th score, clamped to [min(topk, valid), C]
+ * -- groups whose proxy scores fall steeply past the k-th score re-score
+ * fewer candidates.  rho = 0 keeps all C (exactly pivot_refine); rho in
+ * [0, 1].  cand and cand_score [G, C] must come from pivot_proxy_scan with
+ * seq->order = PIVOT_ORDER_RANK (scores descending along each row), so that
+ * C_j candidates are a row's first C_j entries.  cand_count [G] receives
+ * the C_j, or is NULL.  idx / score as pivot_refine; ws of
+ * pivot_refine_adaptive_workspace_size bytes, 256-byte aligned. */
+pivot_status_t pivot_refine_adaptive(const pivot_seq_t* seq, int32_t g, const int32_t* cand,
+                                     const float* cand_score, int32_t C, int32_t topk, float rho,
+                                     int32_t* cand_count, int32_t* idx, float* score, void* ws,
+                                     size_t ws_bytes, void* stream);
+size_t pivot_refine_adaptive_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C,
+                                            int32_t topk);
+
 /* One MTP decode step (PIVOT abstract: the tokens decoded together form the
  * group).  PIVOT_MODE_DENSE: each member scans its own prefix.  REUSE /
  * REFINE: the Gm members' proxy scans [0, cache_len[b] - 1] for its top-C,

@@ -281,3 +281,16 @@ def test_fused_selection_hook(lib):
         assert fused > 0 and plain > 0 and fused != plain
     finally:
         assert pv.pivot_set_fused_selection(1, 4.5) == 0
+
+
+def test_adaptive_refine_rejects_bad_arguments(lib):
+    seq = _seq()
+    ws = pv.pivot_refine_adaptive_workspace_size(seq, 4, 16, 8)
+    assert ws > pv.pivot_refine_workspace_size(seq, 4, 16, 8)
+    for rho in (-0.1, 1.5, float("nan")):
+        assert pv.pivot_refine_adaptive(seq, 4, FAKE, FAKE, 16, 8, rho, None, FAKE, None, FAKE,
+                                        1 << 20, None) == 1
+    assert pv.pivot_refine_adaptive(seq, 4, FAKE, None, 16, 8, 0.5, None, FAKE, None, FAKE,
+                                    1 << 20, None) == 1           # no candidate scores
+    assert pv.pivot_refine_adaptive(seq, 4, FAKE, FAKE, 8, 16, 0.5, None, FAKE, None, FAKE,
+                                    1 << 20, None) == 1           # C < k

@@ -9,6 +9,8 @@
 #include "kernels.h"
 #include "profile.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace pivot {
 
 __device__ uint32_t g_error_word = 0;
@@ -332,8 +334,9 @@ pivot_status_t run_select_cand(int scan_kind, int r0, int r1, int L, int g, int 
                                int cand_base, int C, int K, int npos, int32_t* out,
                                float* out_score, int out_base, cudaStream_t st,
                                const float* key_scale, int lim_shift = 0, int out_stride = 0,
-                               const SegTable* seg = nullptr) {
+                               const SegTable* seg = nullptr, const int32_t* cand_count = nullptr) {
     SelectParams sp{};
+    sp.cand_count = cand_count;
     if (seg) sp.seg = *seg;
     sp.npos = npos;
     sp.kind = SEL_CANDIDATES;
@@ -368,7 +371,8 @@ pivot_status_t run_refine_scores(int kind, int dtype, int H, int D, const void* 
                                  const float* w, const void* k, long long k_rows,
                                  const float* k_scale, int L, int g, int Gm, int maxlen,
                                  const int32_t* cache_len, const int32_t* cand, int cand_base,
-                                 int C, int r0, int r1, float* S, cudaStream_t st) {
+                                 int C, int r0, int r1, float* S, cudaStream_t st,
+                                 const int32_t* cand_count = nullptr) {
     const double work = kind == SCAN_PREFILL_DENSE ? refine_pairs(r0, r1, C) : 0.0;
     const int gsize = kind == SCAN_DECODE_DENSE ? Gm : g;
     int P = umma_shape_ok(H, D, dtype) ? umma_rows(H) : 0;
@@ -406,6 +410,7 @@ pivot_status_t run_refine_scores(int kind, int dtype, int H, int D, const void* 
         const int ngroups = (r1 - 1) / gsize - cand_base + 1;
         p.nitems = ngroups * p.items_per_block;
         p.kbase = k;
+        p.cand_count = cand_count;
         (void)k_rows;
         CUtensorMap tq;
         if (!make_tmap(&tq, dtype, q, q_rows * H, D, N)) return PIVOT_ERR_CUDA;
@@ -436,6 +441,7 @@ pivot_status_t run_refine_scores(int kind, int dtype, int H, int D, const void* 
     rp.cand_base = cand_base;
     rp.C = C;
     rp.S = S;
+    // (CUDA-core shapes score all C; the selection drops what the counts exclude)
     return from_cuda(profiled(PK_REFINE, work, st, [&] { return launch_refine_simt(rp, st); }));
 }
 
@@ -547,10 +553,12 @@ pivot_status_t run_prefix_fused(int kind, const KeySrc& ks, const void* qbase,
     ScanExtra xs;
     xs.key_tile_stride = FUSED_KTS;
     xs.work = pairs / FUSED_KTS;
+    nvtxRangePushA("fused: sample scan");
     pivot_status_t st =
         run_scan(kind, ks.dtype, ks.H, ks.D, qbase, q_rows, qrow_base, w, q_scale, ks.k,
                  ks.k_rows, ks.k_scale, dec ? 0 : L, g, ks.Gm, ks.maxlen, ks.cache_len, P, r0,
                  r1, maxlim, fw.samp, fused_samp_stride(L), s, &xs);
+    nvtxRangePop();
     if (st != PIVOT_OK) return st;
     // 2. bounds
     FusedSelectParams fp{};
@@ -585,7 +593,9 @@ pivot_status_t run_prefix_fused(int kind, const KeySrc& ks, const void* qbase,
     fp.out_stride = out_stride;
     fp.miss_list = fw.miss;
     fp.miss_count = fw.nmiss;
+    nvtxRangePushA("fused: bounds");
     st = from_cuda(profiled(PK_SELECT, 0.0, s, [&] { return launch_sample_bound(fp, s); }));
+    nvtxRangePop();
     if (st != PIVOT_OK) return st;
     // 3. the scan, keeping the scores at or above each row's bound
     ScanExtra xf;
@@ -596,12 +606,16 @@ pivot_status_t run_prefix_fused(int kind, const KeySrc& ks, const void* qbase,
     xf.nchunks = fused_nchunks(L, tpi);
     xf.lim_shift = lim_shift;
     xf.work = pairs;
+    nvtxRangePushA("fused: filter scan");
     st = run_scan(kind, ks.dtype, ks.H, ks.D, qbase, q_rows, qrow_base, w, q_scale, ks.k,
                   ks.k_rows, ks.k_scale, dec ? 0 : L, g, ks.Gm, ks.maxlen, ks.cache_len, P, r0, r1,
                   maxlim, nullptr, 0, s, &xf);
+    nvtxRangePop();
     if (st != PIVOT_OK) return st;
     // 4. the top K of every row's survivors
+    nvtxRangePushA("fused: warp select");
     st = from_cuda(profiled(PK_SELECT, 0.0, s, [&] { return launch_fused_finish(fp, s); }));
+    nvtxRangePop();
     if (st != PIVOT_OK) return st;
     // 5. rows that missed: rescan keeping every score (one row a block) ...
     ScanExtra xr = xf;
@@ -609,10 +623,14 @@ pivot_status_t run_prefix_fused(int kind, const KeySrc& ks, const void* qbase,
     xr.row_list = fw.miss;
     xr.row_count = fw.nmiss;
     xr.work = 0.0;
+    nvtxRangePushA("fused: rescan of missed rows");
     st = run_scan(kind, ks.dtype, ks.H, ks.D, qbase, q_rows, qrow_base, w, q_scale, ks.k,
                   ks.k_rows, ks.k_scale, dec ? 0 : L, g, ks.Gm, ks.maxlen, ks.cache_len, 1, r0, r1,
                   maxlim, nullptr, 0, s, &xr);
-    if (st != PIVOT_OK) return st;
+    if (st != PIVOT_OK) {
+        nvtxRangePop();
+        return st;
+    }
     // 6. ... and select on their keys
     SelectParams sp{};
     sp.kind = SEL_PREFIX;
@@ -638,7 +656,9 @@ pivot_status_t run_prefix_fused(int kind, const KeySrc& ks, const void* qbase,
     sp.rank_order = t_rank_order;
     sp.row_list = fw.miss;
     sp.row_count = fw.nmiss;
-    return from_cuda(profiled(PK_SELECT, 0.0, s, [&] { return launch_select(sp, s); }));
+    st = from_cuda(profiled(PK_SELECT, 0.0, s, [&] { return launch_select(sp, s); }));
+    nvtxRangePop();
+    return st;
 }
 
 // One thread waits on an mbarrier that nothing arrives on: the bounded wait
@@ -665,6 +685,17 @@ cudaError_t launch_wait_selftest(cudaStream_t stream) {
 namespace pivot {
 pivot_status_t decode_check_args(const pivot_decode_t* b, int32_t mode, int32_t C, int32_t topk,
                                  const int32_t* idx);
+
+// A named NVTX range around an entry point or a stage of it: the profilers'
+// timelines show which call (and which step of the fused selection) each
+// kernel belongs to.  Header-only NVTX: without a profiler attached a range
+// costs a branch.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 }  // namespace pivot
 
 using namespace pivot;
@@ -794,6 +825,7 @@ static pivot_status_t dense_index_impl(const pivot_seq_t* seq, int32_t topk, int
 
 pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* idx, float* score,
                                  void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange nvtx_range("pivot_dense_index");
     OrderScope order_scope(seq ? seq->order : 0);
     return dense_index_impl(seq, topk, idx, score, ws, ws_bytes, stream, 0, 0);
 }
@@ -801,6 +833,7 @@ pivot_status_t pivot_dense_index(const pivot_seq_t* seq, int32_t topk, int32_t* 
 // ------------------------------------------------------------ proxy reduce
 pivot_status_t pivot_proxy_reduce(const pivot_seq_t* seq, int32_t g, void* pq, float* pq_scale,
                                   float* pw, void* stream) {
+    NvtxRange nvtx_range("pivot_proxy_reduce");
     int t0, t1;
     pivot_status_t st = check_seq(seq, &t0, &t1);
     if (st != PIVOT_OK) return st;
@@ -852,6 +885,7 @@ pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* p
                                  const float* pq_scale, const float* pw, int32_t C, int32_t topk,
                                  int32_t* cand, float* cand_score, void* ws, size_t ws_bytes,
                                  void* stream) {
+    NvtxRange nvtx_range("pivot_proxy_scan");
     OrderScope order_scope(seq ? seq->order : 0);
     int t0, t1;
     pivot_status_t st = check_seq(seq, &t0, &t1);
@@ -903,6 +937,7 @@ pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* p
 // ------------------------------------------------------------------- reuse
 pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int32_t* cand,
                            int32_t C, int32_t topk, int32_t* idx, void* stream) {
+    NvtxRange nvtx_range("pivot_reuse");
     if (g < 1 || t_begin < 0 || t_end <= t_begin || t_begin % g) return PIVOT_ERR_INVALID_ARG;
     if (!cand || !idx || topk < 1 || C < topk) return PIVOT_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -915,6 +950,7 @@ pivot_status_t pivot_reuse(int32_t t_begin, int32_t t_end, int32_t g, const int3
 pivot_status_t pivot_reuse_backfill(int32_t t_begin, int32_t t_end, int32_t g,
                                     const int32_t* cand, const float* cand_score, int32_t C,
                                     int32_t topk, int32_t* idx, void* stream) {
+    NvtxRange nvtx_range("pivot_reuse_backfill");
     if (g < 1 || t_begin < 0 || t_end <= t_begin || t_begin % g) return PIVOT_ERR_INVALID_ARG;
     if (!cand || !cand_score || !idx || topk < 1 || C < topk) return PIVOT_ERR_INVALID_ARG;
     if (C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
@@ -946,6 +982,7 @@ pivot_status_t pivot_reuse_backfill(int32_t t_begin, int32_t t_end, int32_t g,
 pivot_status_t pivot_window_union(const int32_t* idx, int32_t rows, int32_t topk, int32_t t_begin,
                                   const int32_t* positions, int32_t window, int32_t* out,
                                   void* stream) {
+    NvtxRange nvtx_range("pivot_window_union");
     if (rows < 0 || topk < 1 || window < 1 || !idx || !out) return PIVOT_ERR_INVALID_ARG;
     if (!positions && t_begin < 0) return PIVOT_ERR_INVALID_ARG;
     if (rows == 0) return PIVOT_OK;
@@ -970,7 +1007,8 @@ size_t pivot_refine_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C,
 
 static pivot_status_t refine_impl(const pivot_seq_t* seq, int32_t g, const int32_t* cand,
                                   int32_t C, int32_t topk, int32_t* idx, float* score, void* ws,
-                                  size_t ws_bytes, void* stream, int lim_shift, int out_stride) {
+                                  size_t ws_bytes, void* stream, int lim_shift, int out_stride,
+                                  const int32_t* cand_count = nullptr) {
     int t0, t1;
     pivot_status_t st = check_seq(seq, &t0, &t1);
     if (st != PIVOT_OK) return st;
@@ -989,11 +1027,13 @@ static pivot_status_t refine_impl(const pivot_seq_t* seq, int32_t g, const int32
         const int jc = r0 / g;
         st = run_refine_scores(SCAN_PREFILL_DENSE, seq->dtype, seq->H, seq->D, seq->q, seq->L, 0,
                                seq->q_scale, seq->w, seq->k, seq->L, seq->k_scale, seq->L, g, 1,
-                               0, nullptr, cand + (size_t)(jc - j0) * C, jc, C, r0, r1, S, s);
+                               0, nullptr, cand + (size_t)(jc - j0) * C, jc, C, r0, r1, S, s,
+                               cand_count ? cand_count + (jc - j0) : nullptr);
         if (st != PIVOT_OK) return st;
         st = run_select_cand(SCAN_PREFILL_DENSE, r0, r1, seq->L, g, 1, 0, nullptr, S,
                              cand + (size_t)(jc - j0) * C, jc, C, topk, seq->L, idx, score, t0, s,
-                             seq->k_scale, lim_shift, out_stride);
+                             seq->k_scale, lim_shift, out_stride, nullptr,
+                             cand_count ? cand_count + (jc - j0) : nullptr);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;
@@ -1002,8 +1042,46 @@ static pivot_status_t refine_impl(const pivot_seq_t* seq, int32_t g, const int32
 pivot_status_t pivot_refine(const pivot_seq_t* seq, int32_t g, const int32_t* cand, int32_t C,
                             int32_t topk, int32_t* idx, float* score, void* ws, size_t ws_bytes,
                             void* stream) {
+    NvtxRange nvtx_range("pivot_refine");
     OrderScope order_scope(seq ? seq->order : 0);
     return refine_impl(seq, g, cand, C, topk, idx, score, ws, ws_bytes, stream, 0, 0);
+}
+
+size_t pivot_refine_adaptive_workspace_size(const pivot_seq_t* seq, int32_t g, int32_t C,
+                                            int32_t topk) {
+    const size_t inner = pivot_refine_workspace_size(seq, g, C, topk);
+    if (inner == 0) return 0;
+    int t0, t1;
+    check_seq(seq, &t0, &t1);
+    return inner + align_up((size_t)ceil_div(t1 - t0, g) * 4, WS_ALIGN);
+}
+
+pivot_status_t pivot_refine_adaptive(const pivot_seq_t* seq, int32_t g, const int32_t* cand,
+                                     const float* cand_score, int32_t C, int32_t topk, float rho,
+                                     int32_t* cand_count, int32_t* idx, float* score, void* ws,
+                                     size_t ws_bytes, void* stream) {
+    NvtxRange nvtx_range("pivot_refine_adaptive");
+    OrderScope order_scope(seq ? seq->order : 0);
+    int t0, t1;
+    pivot_status_t st = check_seq(seq, &t0, &t1);
+    if (st != PIVOT_OK) return st;
+    if ((st = check_group_range(seq, g, t0, t1)) != PIVOT_OK) return st;
+    if (!cand || !cand_score || !idx || topk < 1 || C < topk) return PIVOT_ERR_INVALID_ARG;
+    if (!(rho >= 0.0f && rho <= 1.0f)) return PIVOT_ERR_INVALID_ARG;
+    if (C > MAX_K) return PIVOT_ERR_UNSUPPORTED;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) % WS_ALIGN)) return PIVOT_ERR_INVALID_ARG;
+    const int G = ceil_div(t1 - t0, g);
+    const size_t cnt_bytes = align_up((size_t)G * 4, WS_ALIGN);
+    if (ws_bytes <= cnt_bytes) return PIVOT_ERR_WORKSPACE;
+    int32_t* counts = cand_count ? cand_count : static_cast<int32_t*>(ws);
+    void* inner = static_cast<uint8_t*>(ws) + cnt_bytes;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = from_cuda(profiled(PK_REUSE, 0.0, s, [&] {
+        return launch_adaptive_count(cand_score, G, C, topk, rho, counts, s);
+    }));
+    if (st != PIVOT_OK) return st;
+    return refine_impl(seq, g, cand, C, topk, idx, score, inner, ws_bytes - cnt_bytes, stream, 0,
+                       0, counts);
 }
 
 // ------------------------------------------------------------------ ragged batch
@@ -1420,6 +1498,7 @@ size_t pivot_index_varlen_workspace_size(const pivot_varlen_t* batch, int32_t mo
 pivot_status_t pivot_index_varlen(const pivot_varlen_t* batch, int32_t mode, int32_t g, int32_t C,
                                   int32_t topk, int32_t* idx, void* ws, size_t ws_bytes,
                                   void* stream) {
+    NvtxRange nvtx_range("pivot_index_varlen");
     OrderScope order_scope(batch ? batch->order : 0);
     pivot_status_t st = check_varlen(batch, mode, g, C, topk);
     if (st != PIVOT_OK) return st;
@@ -1518,6 +1597,7 @@ size_t pivot_index_window_outside_workspace_size(const pivot_seq_t* seq, int32_t
 pivot_status_t pivot_index_window_outside(const pivot_seq_t* seq, int32_t mode, int32_t g,
                                           int32_t C, int32_t topk, int32_t window, int32_t* idx,
                                           void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange nvtx_range("pivot_index_window_outside");
     OrderScope order_scope(seq ? seq->order : 0);
     int t0, t1;
     pivot_status_t st = check_window(seq, mode, g, C, topk, window, &t0, &t1);
@@ -1669,6 +1749,7 @@ size_t pivot_workspace_size(int32_t mode, int32_t dtype, int32_t L_or_maxlen, in
 
 pivot_status_t pivot_decode(const pivot_decode_t* b, int32_t mode, int32_t C, int32_t topk,
                             int32_t* idx, int32_t* cand, void* ws, size_t ws_bytes, void* stream) {
+    NvtxRange nvtx_range("pivot_decode");
     OrderScope order_scope(b ? b->order : 0);
     pivot_status_t st = decode_check_args(b, mode, C, topk, idx);
     if (st != PIVOT_OK) return st;

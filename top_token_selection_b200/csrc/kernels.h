@@ -43,6 +43,8 @@ struct ScanParams {
     int gsize;              // members per group (g in prefill, Gm in decode)
     int nkeys;              // key positions per sequence (L, or maxlen in decode)
     const void* kbase;      // gather mode: key rows (stored format), row stride D*esize
+    const int32_t* cand_count;  // gather mode: group g's first cand_count[g - cand_base]
+                                // candidates only (adaptive C), or NULL: all C
     SegTable seg;           // SCAN_VARLEN_*: the batch's sequences (rows, keys packed)
     // Sample scan: key tile t of a row is key tile t * key_tile_stride of its
     // prefix; its scores go to columns t*128 + (key in tile).  0 or 1: every tile.
@@ -92,6 +94,8 @@ struct SelectParams {
     const float* S;       // row r at S + (r - row0)*S_stride
     long long S_stride;
     const int32_t* cand;  // SEL_CANDIDATES: group rows at cand + (grp - cand_base)*C
+    const int32_t* cand_count;  // SEL_CANDIDATES: only the group's first cand_count[grp -
+                                // cand_base] entries (adaptive C), or NULL: all C
     int cand_base, C;
     int K;
     int32_t* out_idx;     // row r at out_idx + (r - out_base)*K
@@ -196,6 +200,11 @@ cudaError_t launch_reuse(int t_begin, int t_end, int g, const int32_t* cand, int
 cudaError_t launch_window_union(const int32_t* idx, int rows, int k, int t_begin,
                                 const int32_t* positions, int window, int32_t* out,
                                 cudaStream_t stream, int in_stride = 0);
+// Adaptive C: group j keeps its first count[j] candidates -- those whose
+// proxy score is at least rho times its k-th (the rows rank-ordered, scores
+// descending), clamped to [min(topk, valid), C].
+cudaError_t launch_adaptive_count(const float* cand_score, int G, int C, int topk, float rho,
+                                  int32_t* count, cudaStream_t stream);
 // Reuse over a ragged batch: packed token t takes the first topk entries of
 // its group's candidate row (seg_group_of) that are <= its position.
 cudaError_t launch_reuse_varlen(const SegTable& seg, int T, int g, const int32_t* cand, int C,

@@ -217,6 +217,47 @@ __global__ void window_union_kernel(const int32_t* idx, int rows, int k, int t_b
 
 }  // namespace
 
+namespace {
+
+// One thread a group: the rank-ordered scores fall along the row (-inf
+// padding last), so the count is one binary search for the last score at
+// or above rho times the k-th.
+__global__ void adaptive_count_kernel(const float* cs, int G, int C, int topk, float rho,
+                                      int32_t* count) {
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= G) return;
+    const float* row = cs + (size_t)j * C;
+    int valid = 0, hi = C;   // valid = entries with a finite score
+    while (valid < hi) {
+        const int mid = (valid + hi) >> 1;
+        if (row[mid] > -INFINITY) valid = mid + 1;
+        else hi = mid;
+    }
+    const int kk = topk < valid ? topk : valid;
+    int n = C;
+    if (kk > 0 && row[kk - 1] > 0.0f) {
+        const float T = rho * row[kk - 1];
+        int lo = kk;
+        hi = valid;
+        while (lo < hi) {   // the first entry below T, from the k-th on
+            const int mid = (lo + hi) >> 1;
+            if (row[mid] >= T) lo = mid + 1;
+            else hi = mid;
+        }
+        n = lo;
+    }
+    count[j] = n < kk ? kk : n;
+}
+
+}  // namespace
+
+cudaError_t launch_adaptive_count(const float* cand_score, int G, int C, int topk, float rho,
+                                  int32_t* count, cudaStream_t stream) {
+    if (G <= 0) return cudaSuccess;
+    adaptive_count_kernel<<<ceil_div(G, 256), 256, 0, stream>>>(cand_score, G, C, topk, rho, count);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_window_union(const int32_t* idx, int rows, int k, int t_begin,
                                 const int32_t* positions, int window, int32_t* out,
                                 cudaStream_t stream, int in_stride) {

@@ -79,6 +79,7 @@ __device__ __forceinline__ int scan_key_base(const ScanParams& p, int r) {
 struct ItemInfo {
     int rows, row_first, t0, t1, keybase, maxlim;
     int chunk;             // scan mode: the item's chunk of key tiles
+    int ncand;             // gather mode: candidates scored (C, or the group's adaptive count)
     int nkeys;             // gather mode: key rows of the item's sequence
     const int32_t* cand;   // gather mode: this group's candidate row
     bool valid;
@@ -175,8 +176,14 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
         it.maxlim = it.nkeys - 1;
         it.chunk = 0;
         it.t0 = 0;
-        it.t1 = (p.C + 127) / 128;
-        it.valid = it.rows > 0;
+        // adaptive C: only the group's first ncand candidates are scored
+        it.ncand = p.C;
+        if (p.cand_count) {
+            const int c = p.cand_count[grp - p.cand_base];
+            it.ncand = c < 0 ? 0 : (c < p.C ? c : p.C);
+        }
+        it.t1 = (it.ncand + 127) / 128;
+        it.valid = it.rows > 0 && it.t1 > 0;
         it.cand = p.cand + (size_t)(grp - p.cand_base) * p.C;
     }
     return it;
@@ -364,7 +371,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         const int slot_r = t * 128 + (jb + j) * 32 + lane;
-                        pp[j] = slot_r < p.C ? ld_nc_early(it.cand + slot_r) : -1;
+                        pp[j] = slot_r < it.ncand ? ld_nc_early(it.cand + slot_r) : -1;
                     }
                 };
                 int cur[2], nxt[2];
@@ -579,7 +586,7 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                 // spos: the key position the causal limit applies to
                 const int s = t * 128 + key_in_tile;
                 const int spos = kts > 1 ? t * kts * 128 + key_in_tile : s;
-                const bool col_ok = GATHER ? (s < p.C) : true;
+                const bool col_ok = GATHER ? (s < it.ncand) : true;
                 const uint32_t taddr =
                     tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * 256);
                 if constexpr (HEADS >= 32) {

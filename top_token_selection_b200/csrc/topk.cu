@@ -995,6 +995,12 @@ __global__ void __launch_bounds__(CW_MAX_WARPS * 32) select_cand_kernel(const Se
     const bool var = p.scan_kind == SCAN_VARLEN_DENSE;
     const int grp = dec ? r / p.Gm : (var ? seg_group_of(p.seg, p.g, r) : r / p.g);
     const int32_t* cand = p.cand + (size_t)(grp - p.cand_base) * C;
+    // adaptive C: entries past the group's count are not candidates
+    int Cg = C;
+    if (p.cand_count) {
+        const int c = p.cand_count[grp - p.cand_base];
+        Cg = c < 0 ? 0 : (c < C ? c : C);
+    }
     const float* S = p.s_per_group ? p.S + (size_t)(grp - p.cand_base) * p.S_stride
                                    : p.S + (size_t)(r - p.row0) * p.S_stride;
     const float* ksc = nullptr;
@@ -1013,8 +1019,8 @@ __global__ void __launch_bounds__(CW_MAX_WARPS * 32) select_cand_kernel(const Se
 #pragma unroll
         for (int u = 0; u < CW_BATCH; ++u) {
             const int i = i0 + u * 32 + lane;
-            pos[u] = (ok && i < C) ? cand[i] : -1;
-            x[u] = i < C ? S[i] : 0.0f;
+            pos[u] = (ok && i < Cg) ? cand[i] : -1;
+            x[u] = i < Cg ? S[i] : 0.0f;
         }
         if (ksc) {
             float sc[CW_BATCH];

@@ -204,6 +204,33 @@ def make_decode(B: int, Gm: int, H: int, D: int, dtype: int, len_lo: int, len_hi
                   cache_len.to(torch.int32))
 
 
+def make_layers(nlayers: int, L: int, H: int, D: int, dtype: int, rho: float,
+                seed: int = 0) -> list[Prefill]:
+    """Indexer inputs of `nlayers` consecutive layers over one sequence, with
+    layer-to-layer correlation rho: layer 0 from the DSA-shaped generator;
+    layer l + 1's queries, keys and weight logits are rho * layer l's plus
+    sqrt(1 - rho^2) * an independent draw of the same generator, so each layer
+    keeps the generator's marginals while neighbouring layers' selections
+    overlap more as rho grows.  (A synthetic stand-in: the pages give no
+    cross-layer statistics.)"""
+    gen = torch.Generator().manual_seed(seed)
+    mix = float(np.sqrt(max(0.0, 1.0 - rho * rho)))
+    k = _dsa_keys(L, D, gen)
+    q, _ = _ar1_queries(L, H, D, gen, out_dtype=F32)
+    z = torch.randn(L, H, generator=gen, dtype=torch.float32)
+    out = []
+    for layer in range(nlayers):
+        if layer:
+            k = rho * k + mix * _dsa_keys(L, D, gen)
+            q = rho * q + mix * _ar1_queries(L, H, D, gen, out_dtype=F32)[0]
+            z = rho * z + mix * torch.randn(L, H, generator=gen, dtype=torch.float32)
+        qs, q_scale = _store(q, dtype)
+        ks, k_scale = _store(k, dtype)
+        w = torch.nn.functional.softplus(z).contiguous()
+        out.append(Prefill(dtype, qs, q_scale, w, ks, k_scale))
+    return out
+
+
 # Named workloads (sizes as the benchmark and the parity tests use them).
 WORKLOADS = {
     "tiny_int_prefill": dict(L=1024, H=4, D=32, dtype=F32, kind="int", topk=64, g=4, C=256),

@@ -35,7 +35,8 @@ ABI_SYMBOLS = [
     "pivot_reuse_backfill", "pivot_window_union", "pivot_index_varlen",
     "pivot_index_varlen_workspace_size", "pivot_index_window_outside",
     "pivot_index_window_outside_workspace_size", "pivot_set_score_buffer_cap",
-    "pivot_workspace_size", "pivot_set_fused_selection",
+    "pivot_workspace_size", "pivot_set_fused_selection", "pivot_refine_adaptive",
+    "pivot_refine_adaptive_workspace_size",
 ]
 KERNELS = {0: "scan", 1: "select", 2: "refine", 3: "reduce", 4: "reuse"}
 
@@ -112,6 +113,9 @@ def load(path: str = LIB_PATH):
         "pivot_index_window_outside_workspace_size": ([P, I32, I32, I32, I32, I32], SZ),
         "pivot_workspace_size": ([I32, I32, I32, I32, I32, I32, I32, I32, I32], SZ),
         "pivot_set_fused_selection": ([I32, ctypes.c_float], I32),
+        "pivot_refine_adaptive": ([P, I32, P, P, I32, I32, ctypes.c_float, P, P, P, P, SZ, P],
+                                  I32),
+        "pivot_refine_adaptive_workspace_size": ([P, I32, I32, I32], SZ),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -419,6 +423,32 @@ def refine(seq: PivotSeq, g, cand, topk, with_score=False, ws=None, stream=None,
     return idx, score
 
 
+def pivot_refine_adaptive(seq, g, cand, cand_score, C, topk, rho, cand_count, idx, score, ws,
+                          ws_bytes, stream):
+    return load().pivot_refine_adaptive(ctypes.byref(seq), g, cand, cand_score, C, topk, rho,
+                                        cand_count, idx, score, ws, ws_bytes, stream)
+
+
+def pivot_refine_adaptive_workspace_size(seq, g, C, topk):
+    return load().pivot_refine_adaptive_workspace_size(ctypes.byref(seq), g, C, topk)
+
+
+def refine_adaptive(seq: PivotSeq, g, cand, cand_score, topk, rho, ws=None, stream=None,
+                    device="cuda"):
+    """Refine over each group's adaptive count of rank-ordered candidates;
+    returns (idx, counts)."""
+    n = _rows(seq)
+    C = cand.shape[1]
+    idx = torch.empty(n, topk, dtype=torch.int32, device=device)
+    counts = torch.empty(cand.shape[0], dtype=torch.int32, device=device)
+    if ws is None:
+        ws = _workspace(pivot_refine_adaptive_workspace_size(seq, g, C, topk), device)
+    _check(pivot_refine_adaptive(seq, g, _p(cand), _p(cand_score), C, topk, rho, _p(counts),
+                                 _p(idx), None, _p(ws), ws.numel(), _stream(stream)),
+           "pivot_refine_adaptive")
+    return idx, counts
+
+
 def decode(batch: PivotDecode, mode, C, topk, want_cand=False, ws=None, stream=None,
            device="cuda"):
     idx = torch.empty(batch.B, batch.Gm, topk, dtype=torch.int32, device=device)
@@ -433,3 +463,42 @@ def decode(batch: PivotDecode, mode, C, topk, want_cand=False, ws=None, stream=N
 
 def device_error(stream=None) -> int:
     return pivot_get_device_error(_stream(stream))
+
+
+# ---------------------------------------------------------------------------
+# cross-layer reuse of index rows
+# ---------------------------------------------------------------------------
+
+def layer_anchors(nlayers: int, period: int):
+    """Which layer's index rows each of `nlayers` layers uses when every
+    `period`-th layer runs the indexer and the layers after it reuse its rows
+    (in the style of IndexCache, which the PIVOT blog post names as stacking
+    with PIVOT; the pages give none of its method, so the schedule is a plain
+    fixed period): anchors[l] = l - l % period."""
+    if nlayers < 1 or period < 1:
+        raise ValueError("nlayers and period must be >= 1")
+    return [layer - layer % period for layer in range(nlayers)]
+
+
+def index_layers(layer_seqs, mode, g, C, topk, period, stream=None, device="cuda"):
+    """Index rows for every layer of a model's consecutive layers: the anchor
+    layers (layer_anchors) run the indexer -- dense (mode DENSE) or PIVOT
+    with Reuse or Refine -- through the library; every other layer is handed
+    its anchor's rows (the same tensor: nothing is recomputed or copied).
+    Returns one [rows, topk] int32 tensor per layer."""
+    anchors = layer_anchors(len(layer_seqs), period)
+    rows = {}
+    for layer, seq in enumerate(layer_seqs):
+        if anchors[layer] != layer:
+            continue
+        if mode == DENSE:
+            rows[layer], _ = dense_index(seq, topk, stream=stream, device=device)
+        else:
+            pq, pqs, pw = proxy_reduce(seq, g, stream=stream, device=device)
+            cand, _ = proxy_scan(seq, g, pq, pqs, pw, C, topk, stream=stream, device=device)
+            t0 = seq.t_begin
+            t1 = seq.t_end or seq.L
+            rows[layer] = (reuse(t0, t1, g, cand, topk, stream=stream, device=device)
+                           if mode == REUSE else
+                           refine(seq, g, cand, topk, stream=stream, device=device)[0])
+    return [rows[a] for a in anchors]
