@@ -427,7 +427,8 @@ def config_of(wl, args):
             "parallelism": (f"zigzag{dist_env()[2]}: one sequence's query rows in 2N group "
                             "blocks, rank r takes blocks r and 2N-1-r; keys replicated"
                             if dist_env()[2] > 1 else "1 GPU, whole sequence"),
-            "l2": "no flush: inputs and score buffers larger than L2 (q alone 1 GiB)"}
+            "l2": "no flush: inputs and score buffers larger than L2 (q alone 1 GiB)",
+            "selection": getattr(args, "selection", "library")}
 
 
 def scan_traffic_per_pair():
@@ -694,6 +695,9 @@ def run_ours(args, wl):
     p = make_inputs(wl, args.seed)
     run = Runner(p, wl, device, rank_rows(wl["L"], wl["g"], world, rank))
     pv = run.pv
+    if args.selection != "library":
+        pv._check(pv.pivot_set_fused_selection(1 if args.selection == "fused" else 0, 4.5),
+                  "selection mode")
     fp8 = wl["dtype"] == gen.E4M3
     fp8_peak = measure_fp8_peak(device) if fp8 else None
 
@@ -937,6 +941,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the decode / backfill / window-union measurements")
+    ap.add_argument("--selection", choices=["library", "fused", "scores"], default="library",
+                    help="top-k of prefix rows: the library's default, fused into the scan, "
+                         "or from every score written to the workspace")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -352,13 +352,16 @@ pivot_status_t pivot_set_wait_limit_ns(uint64_t ns);
  * thread-safe against concurrent calls. */
 pivot_status_t pivot_set_score_buffer_cap(size_t bytes);
 
-/* Test hook for the selection fused into the scan.  Prefix rows (dense
- * queries and proxies, H >= 32 on the tensor cores) are selected without
- * writing their scores: a sample scan over every 32nd key tile gives each
- * row a bound, the scan keeps only the scores at or above it, and a row
- * whose survivors fall outside what the in-scan selection holds is rescanned
- * keeping everything.  on = 0 writes every score and selects afterwards (the
- * results are identical); margin_sigmas (default 4.5) sets how far below the
+/* Selection of prefix rows (dense queries and proxies, H >= 32 on the tensor
+ * cores): on = 1 fuses it into the scan -- a sample scan over every 32nd key
+ * tile gives each row a bound, the scan keeps only the scores at or above
+ * it (the score matrix never reaches memory), and a row whose survivors
+ * fall outside what the in-scan selection holds is rescanned keeping
+ * everything; on = 0 (the default) writes every score to the workspace and
+ * selects afterwards.  The results are identical.  On B200 at L = 128K the
+ * default is the faster of the two: the scan is bound by its epilogue's
+ * FP32 instruction stream, to which the filter adds more than the separate
+ * selection costs.  margin_sigmas (default 4.5) sets how far below the
  * expected K-th score the bound sits, in standard deviations of the kept
  * count: a large negative margin makes every long row miss low, a large
  * positive one every long row miss high, which exercises the rescan.

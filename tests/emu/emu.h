@@ -30,6 +30,8 @@ typedef void* cudaStream_t;
 constexpr int cudaSuccess = 0;
 constexpr int cudaErrorInvalidValue = 1;
 constexpr int cudaFuncAttributeMaxDynamicSharedMemorySize = 8;
+constexpr int cudaFuncAttributePreferredSharedMemoryCarveout = 9;
+constexpr int cudaSharedmemCarveoutMaxShared = 100;
 struct CUtensorMap { char b[128]; };
 template <class F> inline cudaError_t cudaFuncSetAttribute(F, int, int) { return cudaSuccess; }
 inline cudaError_t cudaGetLastError() { return cudaSuccess; }
@@ -83,6 +85,7 @@ template <class T> inline T emu_unpack(uint64_t r) { T v; memcpy(&v, &r, sizeof(
 inline unsigned emu_lane() { return threadIdx.x & 31; }
 inline void __syncwarp(unsigned mask = 0xffffffffu) { uint64_t v[32]; emu_exchange(mask, 0, v); }
 inline int __clz(unsigned x) { return x ? __builtin_clz(x) : 32; }
+inline int __clzll(long long x) { return x ? __builtin_clzll((unsigned long long)x) : 64; }
 inline void emu_check_mask(unsigned mask) {
     if (!((mask >> emu_lane()) & 1)) EMU_FAIL("lane %u not in its own mask %08x", emu_lane(), mask);
 }

@@ -280,7 +280,7 @@ def test_fused_selection_hook(lib):
         plain = pv.pivot_dense_index_workspace_size(seq, 2048)
         assert fused > 0 and plain > 0 and fused != plain
     finally:
-        assert pv.pivot_set_fused_selection(1, 4.5) == 0
+        assert pv.pivot_set_fused_selection(0, 4.5) == 0   # the default
 
 
 def test_adaptive_refine_rejects_bad_arguments(lib):

@@ -44,7 +44,7 @@ def dbg():
     lib.pivot_set_fused_selection.argtypes = [I32, ctypes.c_float]
     assert os.path.basename(path) == "libpivot_debug.so"
     yield lib
-    lib.pivot_set_fused_selection(1, 4.5)
+    lib.pivot_set_fused_selection(0, 4.5)
 
 
 def _ws(n):
@@ -83,7 +83,7 @@ def test_debug_build_matches_and_raises_nothing(dbg, sig):
         assert pv.device_error() == 0
         assert torch.equal(got_d, want_d) and torch.equal(got_c, want_c)
         assert torch.equal(got_r, want_r)
-    dbg.pivot_set_fused_selection(1, 4.5)
+    dbg.pivot_set_fused_selection(0, 4.5)
 
 
 def test_debug_build_decode(dbg):

@@ -31,7 +31,7 @@ def _lib():
         pytest.skip("no CUDA device")
     pv.load()
     yield
-    pv.pivot_set_fused_selection(1, 4.5)
+    pv.pivot_set_fused_selection(0, 4.5)   # the default
 
 
 def _dense_and_cand(dev, L, g, C, kk, order=pv.ORDER_POSITION):
@@ -71,7 +71,7 @@ def test_fused_equals_writing_every_score(dtype, L, kk, C):
         for a, b, what in zip(got_r, ref_r, ("dense", "dense scores", "cand", "cand scores")):
             assert torch.equal(a, b), ("rank", what)
     finally:
-        pv.pivot_set_fused_selection(1, 4.5)
+        pv.pivot_set_fused_selection(0, 4.5)
 
 
 @pytest.mark.parametrize("sig", [4.5, -60.0])
@@ -106,7 +106,7 @@ def test_fused_integer_rows_exact(sig):
         assert_rows_exact(ref.cpu().numpy()[rows],
                           oracle.refine(BF16, q, qs, w, k, ks, g, gc, kk, rows=rows)[0], "refine")
     finally:
-        pv.pivot_set_fused_selection(1, 4.5)
+        pv.pivot_set_fused_selection(0, 4.5)
 
 
 def test_fused_row_ranges_and_small_workspace():
@@ -115,6 +115,7 @@ def test_fused_row_ranges_and_small_workspace():
     L, kk = 7000, 512
     p = gen.make_prefill(L, 64, 128, E4M3, kind="dsa", seed=3)
     dev = to_device(p)
+    assert pv.pivot_set_fused_selection(1, 4.5) == 0
     full, _ = pv.dense_index(seq_of(dev), kk)
     a, _ = pv.dense_index(seq_of(dev, 0, 3000), kk)
     b, _ = pv.dense_index(seq_of(dev, 3000, L), kk)
@@ -125,6 +126,8 @@ def test_fused_row_ranges_and_small_workspace():
     torch.cuda.synchronize()
     assert pv.device_error() == 0
     assert torch.equal(c, full)
+    assert pv.pivot_set_fused_selection(0, 4.5) == 0
+    assert torch.equal(pv.dense_index(seq_of(dev), kk)[0], full)
 
 
 @pytest.mark.parametrize("dtype,Gm", [(E4M3, 2), (BF16, 3)])
@@ -155,4 +158,4 @@ def test_fused_decode_equals_writing_every_score(dtype, Gm):
                     if mode != pv.DENSE:
                         assert torch.equal(cand, want[mode][1]), (order, sig, mode)
     finally:
-        pv.pivot_set_fused_selection(1, 4.5)
+        pv.pivot_set_fused_selection(0, 4.5)

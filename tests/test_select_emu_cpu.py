@@ -32,9 +32,6 @@ def select_check(tmp_path_factory):
         ("extern __shared__ __align__(16) uint8_t smem_t[];", "uint8_t* smem_t = emu_smem();"),
         ("row_threshold_kernel<<<grid, THR_WARPS * 32, smem, stream>>>(p, thresh);",
          "emu_launch(grid, THR_WARPS * 32, smem, [&] { row_threshold_kernel(p, thresh); });"),
-        ("extern __shared__ __align__(16) uint8_t smem_c[];", "uint8_t* smem_c = emu_smem();"),
-        ("select_cand_kernel<<<grid, warps * 32, smem, stream>>>(p, warps);",
-         "emu_launch(grid, warps * 32, smem, [&] { select_cand_kernel(p, warps); });"),
         ("extern __shared__ __align__(16) uint8_t smem_b[];", "uint8_t* smem_b = emu_smem();"),
         ("sample_bound_kernel<<<(p.nrows + FB_WARPS - 1) / FB_WARPS, FB_WARPS * 32, smem, stream>>>(p);",
          "emu_launch((p.nrows + FB_WARPS - 1) / FB_WARPS, FB_WARPS * 32, smem, "
@@ -78,7 +75,7 @@ def test_prefix_rows_match_a_sort(select_check, L, K, split, dist, rows, bound):
 
 @pytest.mark.parametrize("mode", [0, 1, 2, 3])
 def test_candidate_rows_match_a_sort(select_check, mode):
-    """Refine rows (one warp each, several warps per block): cand[j] gives the
+    """Refine rows (the block select, candidate rows in place): cand[j] gives the
     positions, the member's limit masks later ones; ties (1), -1 padded rows
     (2), per-key scales multiplied in (3)."""
     _run(select_check, "cand", 4096, 2048, mode, 9, 0, 0)
@@ -90,8 +87,10 @@ def test_candidate_rows_match_a_sort(select_check, mode):
     (4096, 2048, 0, 0, 1),   # shuffled candidate rows: sorted by position, not merged
     (300, 300, 1, 0, 0),     # C = k, ties
     (40, 9, 2, 0, 0),        # tiny rows, -1 padding
-    (8192, 2048, 0, 0, 0),   # the largest C (three warps a block)
+    (8192, 2048, 0, 0, 0),   # C = 8192 > twice k: compacted above the sampled bound
     (8192, 8192, 1, 1, 1),   # k = C = 8192, rank order, shuffled
+    (10000, 2048, 1, 0, 0),  # C = 10000: above the in-place capacity, compacted
+    (10000, 2048, 3, 1, 1),  # the same in rank order, shuffled, per-key scales
     (1, 1, 0, 0, 0),         # one candidate
 ])
 def test_candidate_rows_orders_and_sizes(select_check, C, K, mode, order, layout):
@@ -135,7 +134,9 @@ def test_backfill_rows_match_a_sort(select_check, L, g, C, K):
     (40000, 4096, 2048, 0, 4, 4990, 0, 4.5, 1, "none"),  # proxy rows: top-k first, then the rest
     (40000, 4096, 2048, 0, 3, 4990, 0, -40.0, 1, "all"), # the same through the fallback
     (40000, 4096, 2048, 2, 3, 4990, 1, -40.0, 1, "any"), # signed zeros and small integers
-    (262144, 2048, 0, 0, 2, 262142, 0, 4.5, 0, "none"),  # rows too long for the bitmap: sorted
+    (262144, 2048, 0, 0, 2, 262142, 0, 4.5, 0, "none"),  # rows spanning four bitmap windows
+    (40000, 8192, 0, 0, 2, 39990, 0, 4.5, 0, "none"),    # k = 8192: capacity 16384
+    (40000, 8192, 0, 1, 2, 39990, 1, -40.0, 0, "all"),   # the same through the fallback
 ])
 def test_fused_selection_matches_a_sort(select_check, L, K, split, dist, rows, r0, order, sigmas,
                                         kind, want_fallback):

@@ -267,9 +267,9 @@ pivot_status_t run_scan(int kind, int dtype, int H, int D, const void* qbase, lo
                               [&] { return launch_scan_simt(qbase, kbase, p, st); }));
 }
 
-// Rows of a tensor-core block: N = rows * H columns, 192 for H >= 32 (one
-// row per epilogue warp at H = 64), 256 for smaller H.
-int umma_rows(int H) { return (H >= 32 ? 192 : 256) / H; }
+// Rows of a tensor-core block (scan and Refine): N = rows * H = 256 columns
+// (one row per epilogue warp at H = 64: four warps per TMEM lane quarter).
+int umma_rows(int H) { return 256 / H; }
 
 int rows_per_block(int H, int D, int dtype) {
     return umma_shape_ok(H, D, dtype) ? umma_rows(H) : 8;
@@ -277,7 +277,7 @@ int rows_per_block(int H, int D, int dtype) {
 
 // Decode dense rows: a row block must not straddle two sequences (its keys
 // are one sequence's), so its row count divides Gm; on the tensor cores it is
-// also at most umma_rows(H) (the epilogue gives each of its three warp groups
+// also at most umma_rows(H) (the epilogue gives each of its four warp groups
 // at most 64 / H rows at H >= 32).
 int decode_dense_rows(int Gm, int H, int D, int dtype) {
     if (!umma_shape_ok(H, D, dtype)) return Gm;
@@ -470,7 +470,9 @@ size_t dense_rowbytes(int L) { return (size_t)score_stride(L) * 4 + 4; }
 // selecting among them, and -- for rows whose survivors miss the warp
 // select's range -- a keep-everything rescan of just those rows and the
 // block select on their keys.  The scores themselves never reach memory.
-bool g_fused_on = true;
+// Off by default (pivot_set_fused_selection): the separate selection is
+// faster where the scan's epilogue is the bound.
+bool g_fused_on = false;
 float g_fused_sigmas = 4.5f;
 
 bool fused_ok(int H, int D, int dtype, int K) {

@@ -21,27 +21,34 @@
 // through a TMA ring.  Accumulators are double-buffered in TMEM (2 x 256
 // columns) so the epilogue of tile i overlaps the MMAs of tile i+1.
 //
-// Warp roles (448 threads): warp 0 loads (one lane issuing TMA in scan mode;
-// all 32 lanes copying in gather mode), warp 1 allocates TMEM and issues
-// tcgen05.mma, warps 2-13 run the epilogue (three warps per TMEM lane
-// quarter, each reducing a third of the rows; at H = 64 the block has 3
-// rows, N = 192, and every epilogue warp owns one row whose 64 head weights
-// stay in registers -- reloading them from shared memory every tile competed
-// with the tensor cores' operand reads).
+// Warp roles.  Warp 0 loads (one lane issuing TMA in scan mode; all 32 lanes
+// copying in gather mode, with warp 14 as a second copier), warp 1 allocates
+// TMEM and issues tcgen05.mma, and the epilogue warps reduce: in scan mode
+// warps 4-19, four per TMEM lane quarter (a block of 256 / H rows, N = 256:
+// at H = 64 each epilogue warp owns one row, whose 64 head weights stay in
+// registers -- reloading them from shared memory every tile competed with the
+// tensor cores' operand reads); in gather mode warps 2-13, three per quarter
+// (N = 192 at H >= 32).
 #include "common.cuh"
 #include "kernels.h"
 
 namespace pivot {
 
-constexpr int EPI_GROUPS = 3;                       // epilogue warps per TMEM lane quarter
-constexpr int EPI_WARPS = 4 * EPI_GROUPS;           // 12
-// producer warp 0, MMA warp 1, epilogue warps 2-13, and warp 14: the second
-// candidate-gathering warp of gather mode (idle in scan mode)
-constexpr int GATHER_WARP2 = 2 + EPI_WARPS;         // 14
-constexpr int SCAN_THREADS = (GATHER_WARP2 + 1) * 32;   // 480
-// Register files are per SM sub-partition (16K each); warp w runs on
-// sub-partition w % 4, so 15 warps put at most 4 on one: 128 registers.
-constexpr int SCAN_MAXREG = 128;
+// Warp layout: warp 0 loads, warp 1 issues the MMAs, warps 2-17 run the
+// epilogue -- four per TMEM lane quarter, blocks of 256 / H rows (one row a
+// warp at H = 64), the rows' halved head weights in shared memory -- and in
+// gather mode warp 18 copies candidates beside warp 0.  Registers are per SM
+// sub-partition (16K each; warp w runs on sub-partition w % 4): 18 or 19
+// warps put five on one, so 96 registers a thread.
+template <bool GATHER> struct EpiShape {
+    static constexpr int GROUPS = 4;
+    static constexpr int WARPS = 4 * GROUPS;                  // 16
+    static constexpr int WARP2 = GATHER ? 2 + WARPS : -1;     // second copying warp
+    static constexpr int THREADS = (2 + WARPS + (GATHER ? 1 : 0)) * 32;   // 576 / 608
+    static constexpr int MAXREG = 96;
+};
+static_assert(5 * 32 * EpiShape<false>::MAXREG <= 16384 && 5 * 32 * EpiShape<true>::MAXREG <= 16384,
+              "register file of a sub-partition");
 
 __device__ __forceinline__ int scan_row_lim(const ScanParams& p, int r, bool& ok) {
     ok = true;
@@ -190,7 +197,7 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
 }
 
 template <int KIND, int HEADS, int ROWB, bool GATHER, bool FILTER>
-__global__ void __maxnreg__(SCAN_MAXREG)
+__global__ void __maxnreg__(EpiShape<GATHER>::MAXREG)
     index_umma_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_q, const ScanParams p) {
     constexpr int KBLK = ROWB / 128;           // 128-byte K blocks per row
@@ -199,6 +206,11 @@ __global__ void __maxnreg__(SCAN_MAXREG)
     constexpr int B_SLOT = 256 * ROWB;         // query block, N <= 256 rows
     constexpr int STAGES = ROWB == 128 ? 6 : 3;
     constexpr int PMAX = 256 / HEADS;
+    constexpr int EPI_GROUPS = EpiShape<GATHER>::GROUPS;
+    constexpr int EPI_WARPS = EpiShape<GATHER>::WARPS;
+    constexpr int GATHER_WARP2 = EpiShape<GATHER>::WARP2;
+    constexpr int FIRST_EPI = 2;
+    constexpr int TCOLS = 32;                   // TMEM columns a load at H >= 32
     constexpr uint32_t FMT = KIND == KIND_F8 ? 0u : (KIND == KIND_F16 ? 1u : 2u);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -256,226 +268,229 @@ __global__ void __maxnreg__(SCAN_MAXREG)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    if (warp == 0 || warp == GATHER_WARP2) {
-        // ------------------------------------------------------- producer
-        if constexpr (!GATHER) {
-            if (warp == 0) {
-            // Scan mode: lane 0 streams contiguous key tiles with tiled TMA.
-            if (lane == 0) {
+    if (warp < FIRST_EPI || (GATHER && warp == GATHER_WARP2)) {
+        if (warp == 0 || (GATHER && warp == GATHER_WARP2)) {
+            // ------------------------------------------------------- producer
+            if constexpr (!GATHER) {
+                if (warp == 0) {
+                // Scan mode: lane 0 streams contiguous key tiles with tiled TMA.
+                if (lane == 0) {
+                    int stage = 0;
+                    uint32_t phase = 0;
+                    int nit = 0;
+                    // parity of the last load issued per stage / query slot (-1:
+                    // none), so every load can be waited for before the CTA exits
+                    int last_a[STAGES], last_b[2] = {-1, -1};
+                    for (int i = 0; i < STAGES; ++i) last_a[i] = -1;
+                    bool aborted = false;
+                    for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
+                        ItemInfo it = scan_item<GATHER>(p, item);
+                        if (!it.valid) continue;
+                        const int slot = nit & 1;
+                        const uint32_t bph = (nit >> 1) & 1;
+                        if (!mbar_wait(&bempty[slot], bph ^ 1)) { aborted = true; break; }
+                        mbar_arrive_expect_tx(&bfull[slot], (uint32_t)(N * ROWB));
+                        last_b[slot] = (int)bph;
+                        const int qrow = (it.row_first - p.qrow_base) * HEADS;
+                        for (int kb = 0; kb < KBLK; ++kb)
+                            tma_load_2d(sB + slot * B_SLOT + kb * (N * 128), &tmap_q, &bfull[slot],
+                                        kb * (128 / p.esize), qrow);
+                        for (int t = it.t0; t < it.t1; ++t) {
+                            if (!mbar_wait(&empty[stage], phase ^ 1)) { aborted = true; break; }
+                            mbar_arrive_expect_tx(&full[stage], (uint32_t)A_BYTES);
+                            last_a[stage] = (int)phase;
+                            const int kt = p.key_tile_stride > 1 ? t * p.key_tile_stride : t;
+                            for (int kb = 0; kb < KBLK; ++kb)
+                                tma_load_2d(sA + stage * A_BYTES + kb * (128 * 128), &tmap_k,
+                                            &full[stage], kb * (128 / p.esize), it.keybase + kt * 128);
+                            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                        }
+                        ++nit;
+                    }
+                    // Every load issued lands before the CTA may exit (only the
+                    // producer arrives on these barriers, so the last phase stays).
+                    for (int i = 0; i < STAGES; ++i)
+                        if (last_a[i] >= 0) mbar_wait(&full[i], (uint32_t)last_a[i]);
+                    for (int i = 0; i < 2; ++i)
+                        if (last_b[i] >= 0) mbar_wait(&bfull[i], (uint32_t)last_b[i]);
+                }
+                }
+            } else {
+                // Gather mode: two warps copy each tile's 128 candidate key rows
+                // (warp 0 rows 0-63, warp 14 rows 64-127) with 16-byte cp.async
+                // straight into the swizzled tile layout.  Each publishes its half
+                // of a tile (an arrive on full[stage], which expects both) once
+                // its copies have landed and been fenced for the tensor cores; up
+                // to GDEPTH tiles are in flight per warp.  Warp 0 alone loads the
+                // query blocks.  Neither warp blocks while holding an unpublished
+                // tile older than the one it waits for: warp 0 publishes the
+                // tiles of item nit - 2 before waiting for its query slot, and a
+                // ring stage a warp waits on was last used by a tile older than
+                // all of that warp's pending ones (STAGES > GDEPTH).
+                const bool lead = warp == 0;
+                const int jb = lead ? 0 : 2;   // row groups j of this warp (rows j * 32 + lane)
+                constexpr int GDEPTH = STAGES > 3 ? 3 : STAGES - 1;   // deeper was slower
+                static_assert(STAGES > GDEPTH && GDEPTH >= 1, "the ring must outrun the copies");
+                const uint8_t* kbytes = static_cast<const uint8_t*>(p.kbase);
                 int stage = 0;
                 uint32_t phase = 0;
                 int nit = 0;
-                // parity of the last load issued per stage / query slot (-1:
-                // none), so every load can be waited for before the CTA exits
-                int last_a[STAGES], last_b[2] = {-1, -1};
-                for (int i = 0; i < STAGES; ++i) last_a[i] = -1;
+                int pend[GDEPTH] = {0};       // stages of the tiles in flight, oldest first
+                int pend_it[GDEPTH] = {0};    // and the item (in this CTA's order) of each
+                int npend = 0;
+                int last_b[2] = {-1, -1};
+                bool aborted = false;
+                auto publish_oldest = [&]() {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&full[pend[0]]);
+                    for (int i = 1; i < npend; ++i) {
+                        pend[i - 1] = pend[i];
+                        pend_it[i - 1] = pend_it[i];
+                    }
+                    --npend;
+                };
+                for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
+                    ItemInfo it = scan_item<GATHER>(p, item);
+                    if (!it.valid) continue;
+                    const int slot = nit & 1;
+                    const uint32_t bph = (nit >> 1) & 1;
+                    // The query slot frees once the MMAs of item nit - 2 are done,
+                    // which needs every tile of that item published: land and
+                    // publish what is in flight if any of it is that old (items
+                    // shorter than the copy depth).
+                    if (lead) {
+                        if (npend > 0 && pend_it[0] <= nit - 2) {
+                            cp_async_wait<0>();
+                            while (npend > 0) publish_oldest();
+                        }
+                        if (!__all_sync(0xffffffffu, mbar_wait(&bempty[slot], bph ^ 1))) {
+                            aborted = true;
+                            break;
+                        }
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&bfull[slot], (uint32_t)(N * ROWB));
+                            const int qrow = (it.row_first - p.qrow_base) * HEADS;
+                            for (int kb = 0; kb < KBLK; ++kb)
+                                tma_load_2d(sB + slot * B_SLOT + kb * (N * 128), &tmap_q, &bfull[slot],
+                                            kb * (128 / p.esize), qrow);
+                        }
+                        last_b[slot] = (int)bph;
+                    }
+                    // candidate positions of this warp's rows of a tile: lane l
+                    // holds slots l + 32 (jb + j), read one tile ahead so no copy
+                    // waits on them
+                    auto tile_pos = [&](int t, int (&pp)[2]) {
+    #pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const int slot_r = t * 128 + (jb + j) * 32 + lane;
+                            pp[j] = slot_r < it.ncand ? ld_nc_early(it.cand + slot_r) : -1;
+                        }
+                    };
+                    int cur[2], nxt[2];
+                    tile_pos(it.t0, nxt);
+                    for (int t = it.t0; t < it.t1; ++t) {
+    #pragma unroll
+                        for (int j = 0; j < 2; ++j) cur[j] = nxt[j];
+                        if (t + 1 < it.t1) tile_pos(t + 1, nxt);
+                        if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1))) {
+                            aborted = true;
+                            break;
+                        }
+                        const uint32_t dst = smem_u32(sA + stage * A_BYTES);
+                        // Lane l copies tile rows l + 32 (jb + j), its own
+                        // positions, 16 bytes at a time.  Chunk c of row r sits at
+                        // (r / 8) 1024 + (r % 8) 128 + ((c ^ r % 8) 16): with the
+                        // tile 1024-byte aligned that is rowbase XOR (c 16), where
+                        // rowbase holds r % 8 in bits 4-6.  The chunks of a row go
+                        // out in consecutive instructions, so after the first the
+                        // line is in L1 (.ca); the loop is two instructions a chunk.
+    #pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const int r = (jb + j) * 32 + lane;
+                            const int pos = cur[j];
+                            const size_t row = (size_t)(it.keybase + ((pos >= 0 && pos < it.nkeys) ? pos : 0));
+                            const uint8_t* src = kbytes + row * ROWB;
+                            const uint32_t x = (uint32_t)(r & 7);
+                            const uint32_t rowbase = dst + (uint32_t)(r >> 3) * 1024u + x * 128u + (x << 4);
+    #pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+    #pragma unroll
+                                for (int kb = 0; kb < KBLK; ++kb)
+                                    cp_async16_ca((rowbase ^ ((uint32_t)c << 4)) + kb * (128 * 128),
+                                                  src + kb * 128 + c * 16);
+                            }
+                        }
+                        cp_async_commit();
+                        pend_it[npend] = nit;
+                        pend[npend++] = stage;
+                        if (npend == GDEPTH) {
+                            cp_async_wait<GDEPTH - 1>();
+                            publish_oldest();
+                        }
+                        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    }
+                    ++nit;
+                }
+                // publish (or, after an abort, just land) every tile still in flight
+                cp_async_wait<0>();
+                while (npend > 0) publish_oldest();
+                if (lead && lane == 0)
+                    for (int i = 0; i < 2; ++i)
+                        if (last_b[i] >= 0) mbar_wait(&bfull[i], (uint32_t)last_b[i]);
+            }
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ MMA
+            if (lane == 0) {
+                const uint32_t idesc = make_idesc(FMT, 128, (uint32_t)N);
+                int stage = 0;
+                uint32_t phase = 0;
+                int nit = 0, ntile = 0;
                 bool aborted = false;
                 for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
                     ItemInfo it = scan_item<GATHER>(p, item);
                     if (!it.valid) continue;
                     const int slot = nit & 1;
                     const uint32_t bph = (nit >> 1) & 1;
-                    if (!mbar_wait(&bempty[slot], bph ^ 1)) { aborted = true; break; }
-                    mbar_arrive_expect_tx(&bfull[slot], (uint32_t)(N * ROWB));
-                    last_b[slot] = (int)bph;
-                    const int qrow = (it.row_first - p.qrow_base) * HEADS;
-                    for (int kb = 0; kb < KBLK; ++kb)
-                        tma_load_2d(sB + slot * B_SLOT + kb * (N * 128), &tmap_q, &bfull[slot],
-                                    kb * (128 / p.esize), qrow);
+                    if (!mbar_wait(&bfull[slot], bph)) { aborted = true; break; }
+                    const uint32_t bbase = smem_u32(sB + slot * B_SLOT);
                     for (int t = it.t0; t < it.t1; ++t) {
-                        if (!mbar_wait(&empty[stage], phase ^ 1)) { aborted = true; break; }
-                        mbar_arrive_expect_tx(&full[stage], (uint32_t)A_BYTES);
-                        last_a[stage] = (int)phase;
-                        const int kt = p.key_tile_stride > 1 ? t * p.key_tile_stride : t;
-                        for (int kb = 0; kb < KBLK; ++kb)
-                            tma_load_2d(sA + stage * A_BYTES + kb * (128 * 128), &tmap_k,
-                                        &full[stage], kb * (128 / p.esize), it.keybase + kt * 128);
+                        const int acc = ntile & 1;
+                        const uint32_t aph = (ntile >> 1) & 1;
+                        if (!mbar_wait(&accempty[acc], aph ^ 1)) { aborted = true; break; }
+                        if (!mbar_wait(&full[stage], phase)) { aborted = true; break; }
+                        tc_fence_after();
+                        const uint32_t abase = smem_u32(sA + stage * A_BYTES);
+                        const uint32_t dcol = tmem_base + (uint32_t)(acc * 256);
+    #pragma unroll
+                        for (int ks = 0; ks < KSTEPS; ++ks) {
+                            const int kb = ks / 4, kin = ks % 4;
+                            const uint64_t ad = smem_desc_k_sw128(abase + kb * (128 * 128) + kin * 32);
+                            const uint64_t bd = smem_desc_k_sw128(bbase + kb * (N * 128) + kin * 32);
+                            umma_ss<KIND>(dcol, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&empty[stage]);
+                        umma_commit(&accfull[acc]);
                         if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                        ++ntile;
                     }
+                    umma_commit(&bempty[slot]);
                     ++nit;
                 }
-                // Every load issued lands before the CTA may exit (only the
-                // producer arrives on these barriers, so the last phase stays).
-                for (int i = 0; i < STAGES; ++i)
-                    if (last_a[i] >= 0) mbar_wait(&full[i], (uint32_t)last_a[i]);
-                for (int i = 0; i < 2; ++i)
-                    if (last_b[i] >= 0) mbar_wait(&bfull[i], (uint32_t)last_b[i]);
+                // Drain: wait until every MMA issued has completed.
+                umma_commit(drain);
+                mbar_wait(drain, 0);
             }
-            }
-        } else {
-            // Gather mode: two warps copy each tile's 128 candidate key rows
-            // (warp 0 rows 0-63, warp 14 rows 64-127) with 16-byte cp.async
-            // straight into the swizzled tile layout.  Each publishes its half
-            // of a tile (an arrive on full[stage], which expects both) once
-            // its copies have landed and been fenced for the tensor cores; up
-            // to GDEPTH tiles are in flight per warp.  Warp 0 alone loads the
-            // query blocks.  Neither warp blocks while holding an unpublished
-            // tile older than the one it waits for: warp 0 publishes the
-            // tiles of item nit - 2 before waiting for its query slot, and a
-            // ring stage a warp waits on was last used by a tile older than
-            // all of that warp's pending ones (STAGES > GDEPTH).
-            const bool lead = warp == 0;
-            const int jb = lead ? 0 : 2;   // row groups j of this warp (rows j * 32 + lane)
-            constexpr int GDEPTH = STAGES > 3 ? 3 : STAGES - 1;   // deeper was slower
-            static_assert(STAGES > GDEPTH && GDEPTH >= 1, "the ring must outrun the copies");
-            const uint8_t* kbytes = static_cast<const uint8_t*>(p.kbase);
-            int stage = 0;
-            uint32_t phase = 0;
-            int nit = 0;
-            int pend[GDEPTH] = {0};       // stages of the tiles in flight, oldest first
-            int pend_it[GDEPTH] = {0};    // and the item (in this CTA's order) of each
-            int npend = 0;
-            int last_b[2] = {-1, -1};
-            bool aborted = false;
-            auto publish_oldest = [&]() {
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full[pend[0]]);
-                for (int i = 1; i < npend; ++i) {
-                    pend[i - 1] = pend[i];
-                    pend_it[i - 1] = pend_it[i];
-                }
-                --npend;
-            };
-            for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
-                ItemInfo it = scan_item<GATHER>(p, item);
-                if (!it.valid) continue;
-                const int slot = nit & 1;
-                const uint32_t bph = (nit >> 1) & 1;
-                // The query slot frees once the MMAs of item nit - 2 are done,
-                // which needs every tile of that item published: land and
-                // publish what is in flight if any of it is that old (items
-                // shorter than the copy depth).
-                if (lead) {
-                    if (npend > 0 && pend_it[0] <= nit - 2) {
-                        cp_async_wait<0>();
-                        while (npend > 0) publish_oldest();
-                    }
-                    if (!__all_sync(0xffffffffu, mbar_wait(&bempty[slot], bph ^ 1))) {
-                        aborted = true;
-                        break;
-                    }
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&bfull[slot], (uint32_t)(N * ROWB));
-                        const int qrow = (it.row_first - p.qrow_base) * HEADS;
-                        for (int kb = 0; kb < KBLK; ++kb)
-                            tma_load_2d(sB + slot * B_SLOT + kb * (N * 128), &tmap_q, &bfull[slot],
-                                        kb * (128 / p.esize), qrow);
-                    }
-                    last_b[slot] = (int)bph;
-                }
-                // candidate positions of this warp's rows of a tile: lane l
-                // holds slots l + 32 (jb + j), read one tile ahead so no copy
-                // waits on them
-                auto tile_pos = [&](int t, int (&pp)[2]) {
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int slot_r = t * 128 + (jb + j) * 32 + lane;
-                        pp[j] = slot_r < it.ncand ? ld_nc_early(it.cand + slot_r) : -1;
-                    }
-                };
-                int cur[2], nxt[2];
-                tile_pos(it.t0, nxt);
-                for (int t = it.t0; t < it.t1; ++t) {
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) cur[j] = nxt[j];
-                    if (t + 1 < it.t1) tile_pos(t + 1, nxt);
-                    if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1))) {
-                        aborted = true;
-                        break;
-                    }
-                    const uint32_t dst = smem_u32(sA + stage * A_BYTES);
-                    // Lane l copies tile rows l + 32 (jb + j), its own
-                    // positions, 16 bytes at a time.  Chunk c of row r sits at
-                    // (r / 8) 1024 + (r % 8) 128 + ((c ^ r % 8) 16): with the
-                    // tile 1024-byte aligned that is rowbase XOR (c 16), where
-                    // rowbase holds r % 8 in bits 4-6.  The chunks of a row go
-                    // out in consecutive instructions, so after the first the
-                    // line is in L1 (.ca); the loop is two instructions a chunk.
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int r = (jb + j) * 32 + lane;
-                        const int pos = cur[j];
-                        const size_t row = (size_t)(it.keybase + ((pos >= 0 && pos < it.nkeys) ? pos : 0));
-                        const uint8_t* src = kbytes + row * ROWB;
-                        const uint32_t x = (uint32_t)(r & 7);
-                        const uint32_t rowbase = dst + (uint32_t)(r >> 3) * 1024u + x * 128u + (x << 4);
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-#pragma unroll
-                            for (int kb = 0; kb < KBLK; ++kb)
-                                cp_async16_ca((rowbase ^ ((uint32_t)c << 4)) + kb * (128 * 128),
-                                              src + kb * 128 + c * 16);
-                        }
-                    }
-                    cp_async_commit();
-                    pend_it[npend] = nit;
-                    pend[npend++] = stage;
-                    if (npend == GDEPTH) {
-                        cp_async_wait<GDEPTH - 1>();
-                        publish_oldest();
-                    }
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-                ++nit;
-            }
-            // publish (or, after an abort, just land) every tile still in flight
-            cp_async_wait<0>();
-            while (npend > 0) publish_oldest();
-            if (lead && lane == 0)
-                for (int i = 0; i < 2; ++i)
-                    if (last_b[i] >= 0) mbar_wait(&bfull[i], (uint32_t)last_b[i]);
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc(FMT, 128, (uint32_t)N);
-            int stage = 0;
-            uint32_t phase = 0;
-            int nit = 0, ntile = 0;
-            bool aborted = false;
-            for (int item = blockIdx.x; item < nitems && !aborted; item += gridDim.x) {
-                ItemInfo it = scan_item<GATHER>(p, item);
-                if (!it.valid) continue;
-                const int slot = nit & 1;
-                const uint32_t bph = (nit >> 1) & 1;
-                if (!mbar_wait(&bfull[slot], bph)) { aborted = true; break; }
-                const uint32_t bbase = smem_u32(sB + slot * B_SLOT);
-                for (int t = it.t0; t < it.t1; ++t) {
-                    const int acc = ntile & 1;
-                    const uint32_t aph = (ntile >> 1) & 1;
-                    if (!mbar_wait(&accempty[acc], aph ^ 1)) { aborted = true; break; }
-                    if (!mbar_wait(&full[stage], phase)) { aborted = true; break; }
-                    tc_fence_after();
-                    const uint32_t abase = smem_u32(sA + stage * A_BYTES);
-                    const uint32_t dcol = tmem_base + (uint32_t)(acc * 256);
-#pragma unroll
-                    for (int ks = 0; ks < KSTEPS; ++ks) {
-                        const int kb = ks / 4, kin = ks % 4;
-                        const uint64_t ad = smem_desc_k_sw128(abase + kb * (128 * 128) + kin * 32);
-                        const uint64_t bd = smem_desc_k_sw128(bbase + kb * (N * 128) + kin * 32);
-                        umma_ss<KIND>(dcol, ad, bd, idesc, ks > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&empty[stage]);
-                    umma_commit(&accfull[acc]);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                    ++ntile;
-                }
-                umma_commit(&bempty[slot]);
-                ++nit;
-            }
-            // Drain: wait until every MMA issued has completed.
-            umma_commit(drain);
-            mbar_wait(drain, 0);
         }
     } else {
         // ------------------------------------------------------- epilogue
         // EPI_GROUPS warps per TMEM lane quarter.  With H >= 32 the rows of
         // the block are split between the groups (each row's H columns are
-        // reduced by one thread, weights in registers); with H < 32 the first
+        // reduced by one thread; the halved head weights in registers in
+        // gather mode, in shared memory in scan mode); with H < 32 the first
         // group does all rows in 32-column chunks (weights from shared
         // memory) and the others only keep step.
-        const int e = warp - 2;                   // 0..EPI_WARPS-1
+        const int e = warp - FIRST_EPI;           // 0..EPI_WARPS-1
         const int quarter = warp & 3;             // TMEM lane quarter of this warp
         const int grp = e >> 2;                   // 0..EPI_GROUPS-1
         const int key_in_tile = quarter * 32 + lane;
@@ -489,7 +504,6 @@ __global__ void __maxnreg__(SCAN_MAXREG)
             r_hi = grp == 0 ? p.P : 0;
         }
         constexpr int RROWS = HEADS >= 32 ? 64 / HEADS : 1;      // rows per warp at most
-        float wr[HEADS >= 32 ? 64 : 1];
         int lim_r[RROWS];
         float sq_r[RROWS];
         float tf_r[RROWS];    // filter mode: scores >= tf_r are kept
@@ -518,22 +532,22 @@ __global__ void __maxnreg__(SCAN_MAXREG)
                                                    : 1.0f;
             };
             if constexpr (HEADS >= 32) {
-                // this warp's rows: weights, limits and query scales in registers
+                // the block's halved head weights, P x H <= 256 floats
+                // (w * max(0, x) == (w / 2) * (x + |x|) exactly)
+                named_bar_sync(1, EPI_WARPS * 32);
+                for (int i = et; i < p.P * HEADS; i += EPI_WARPS * 32) {
+                    const int pr = i / HEADS;
+                    w_s[i] = pr < it.rows
+                                 ? 0.5f * p.w[(size_t)(it.row_first + pr - p.qrow_base) * HEADS +
+                                              i % HEADS]
+                                 : 0.0f;
+                }
+                named_bar_sync(1, EPI_WARPS * 32);
+                // this warp's rows: limits and query scales in registers
 #pragma unroll
                 for (int lr = 0; lr < RROWS; ++lr) {
                     const int pr = r_lo + lr;
                     const bool live = pr < r_hi && pr < it.rows;
-                    const float4* w4 = reinterpret_cast<const float4*>(
-                        p.w + (size_t)(it.row_first + pr - p.qrow_base) * HEADS);
-#pragma unroll
-                    for (int i4 = 0; i4 < HEADS / 4; ++i4) {
-                        const float4 wv = live ? __ldg(w4 + i4) : make_float4(0.f, 0.f, 0.f, 0.f);
-                        // halved: w * max(0, x) == (w / 2) * (x + |x|) exactly
-                        wr[lr * HEADS + 4 * i4 + 0] = 0.5f * wv.x;
-                        wr[lr * HEADS + 4 * i4 + 1] = 0.5f * wv.y;
-                        wr[lr * HEADS + 4 * i4 + 2] = 0.5f * wv.z;
-                        wr[lr * HEADS + 4 * i4 + 3] = 0.5f * wv.w;
-                    }
                     lim_r[lr] = pr < r_hi ? row_lim(pr) : -1;
                     sq_r[lr] = row_sq(pr);
                     tf_r[lr] = -INFINITY;
@@ -599,18 +613,26 @@ __global__ void __maxnreg__(SCAN_MAXREG)
 #pragma unroll
                         for (int j = 0; j < 4; ++j) a[j] = 0ull;
 #pragma unroll
-                        for (int c = 0; c < HEADS / 32; ++c) {
-                            float v[32];
-                            tmem_ld32(taddr + (uint32_t)(pr * HEADS + c * 32), v);
+                        for (int c = 0; c < HEADS / TCOLS; ++c) {
+                            float v[TCOLS];
+                            tmem_ld32(taddr + (uint32_t)(pr * HEADS + c * TCOLS), v);
                             tmem_ld_wait();
+                            // x + |x| = 2 max(0, x): one add on the FMA pipe
+                            // instead of a half-rate max on the ALU pipe; four
+                            // weights a broadcast load (every lane the same row)
+                            const float4* w4 =
+                                reinterpret_cast<const float4*>(w_s + pr * HEADS + c * TCOLS);
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const int wi = lr * HEADS + c * 32 + 2 * i;
-                                // x + |x| = 2 max(0, x): one add on the FMA pipe
-                                // instead of a half-rate max on the ALU pipe
-                                a[i & 3] = ffma2(pack2(v[2 * i] + fabsf(v[2 * i]),
-                                                       v[2 * i + 1] + fabsf(v[2 * i + 1])),
-                                                 pack2(wr[wi], wr[wi + 1]), a[i & 3]);
+                            for (int i = 0; i < TCOLS / 4; ++i) {
+                                const float4 wv = w4[i];
+                                a[(2 * i) & 3] =
+                                    ffma2(pack2(v[4 * i] + fabsf(v[4 * i]),
+                                                v[4 * i + 1] + fabsf(v[4 * i + 1])),
+                                          pack2(wv.x, wv.y), a[(2 * i) & 3]);
+                                a[(2 * i + 1) & 3] =
+                                    ffma2(pack2(v[4 * i + 2] + fabsf(v[4 * i + 2]),
+                                                v[4 * i + 3] + fabsf(v[4 * i + 3])),
+                                          pack2(wv.z, wv.w), a[(2 * i + 1) & 3]);
                             }
                         }
                         float lo[4], hi[4];
@@ -707,12 +729,13 @@ int scan_smem_bytes(int row_bytes) {
            256 /*barriers*/ + 16 /*TMEM address*/ + 256 * 4 + pmax * 8;
 }
 
-// The epilogue's three warp groups take ceil(P / 3) rows each, with room
-// for 64 / HEADS rows' weights in registers at HEADS >= 32, and PMAX rows'
-// tables in shared memory below: larger blocks are refused.
-inline bool epilogue_fits(int P, int heads) {
+// The epilogue's warp groups (four in scan mode, three in gather mode) take
+// ceil(P / groups) rows each, with room for 64 / HEADS rows' weights in
+// registers at HEADS >= 32, and PMAX rows' tables in shared memory below:
+// larger blocks are refused.
+inline bool epilogue_fits(int P, int heads, int groups) {
     if (P < 1 || P * heads > 256) return false;
-    return heads >= 32 ? (P + 2) / 3 <= 64 / heads : true;
+    return heads >= 32 ? (P + groups - 1) / groups <= 64 / heads : true;
 }
 
 template <int KIND, int HEADS, int ROWB, bool GATHER, bool FILTER>
@@ -722,14 +745,14 @@ static cudaError_t launch_one(const CUtensorMap& tk, const CUtensorMap& tq, cons
     const int smem = scan_smem_bytes(ROWB);
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kfn<<<grid, SCAN_THREADS, smem, stream>>>(tk, tq, p);
+    kfn<<<grid, EpiShape<GATHER>::THREADS, smem, stream>>>(tk, tq, p);
     return cudaGetLastError();
 }
 
 template <int KIND, int HEADS, bool GATHER>
 static cudaError_t launch_heads(const CUtensorMap& tk, const CUtensorMap& tq, const ScanParams& p,
                                 int row_bytes, int grid, cudaStream_t stream) {
-    if (!epilogue_fits(p.P, HEADS)) return cudaErrorInvalidValue;
+    if (!epilogue_fits(p.P, HEADS, EpiShape<GATHER>::GROUPS)) return cudaErrorInvalidValue;
     // the fused selection runs in the register-resident epilogue (H >= 32)
     const bool filter = !GATHER && p.surv != nullptr;
     if (filter && HEADS < 32) return cudaErrorInvalidValue;

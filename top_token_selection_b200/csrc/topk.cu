@@ -892,18 +892,8 @@ __global__ void __launch_bounds__(THR_WARPS * 32) row_threshold_kernel(const Sel
 
 // ------------------------------------------------------------ candidate rows
 //
-// Candidate rows (Refine, Reuse with backfill: C entries, positions from the
-// group's candidate row) are short, so each is selected by ONE warp with no
-// block barriers: its C entries, as 64-bit keys, sit in the warp's slice of
-// shared memory; the k-th largest score key comes from warp histograms over
-// the remaining key range (then, when the k-th score is tied, the same search
-// over the tied entries' positions); unselected entries are cleared and the
-// selected ones compacted in place, keeping their order.  In position order a
-// candidate row written by the proxy scan is two ascending runs (the proxy's
-// top-k, then the rest), so each selected entry's output slot is its rank in
-// its own run plus the number of selected entries of the other run at lower
-// positions (a binary search).  Rank order, and candidate rows of any other
-// layout, sort the selected keys in the warp (bitonic).
+// Warp-level helpers of the fused selection's finish (one warp a row): the
+// k-th largest key by warp histograms, stable compaction, bitonic sort.
 
 __host__ __device__ int pow2_at_least(int x) {
     int m = 1;
@@ -911,14 +901,8 @@ __host__ __device__ int pow2_at_least(int x) {
     return m;
 }
 
-constexpr int CW_MAX_WARPS = 8;
 constexpr int CW_BATCH = 8;              // independent loads a lane issues at once
 constexpr size_t CW_SMEM_LIMIT = 200 * 1024;
-
-__host__ __device__ int cw_slots(int C) { return pow2_at_least(C < 32 ? 32 : C); }
-__host__ __device__ size_t cw_warp_bytes(int C) {
-    return (size_t)cw_slots(C) * 8 + (size_t)THR_BINS * 4;
-}
 
 // Sort e[0, M) (M a power of two, whole warp) so that before(a, b) holds for
 // every earlier a and later b.
@@ -960,180 +944,6 @@ __device__ int warp_compact(uint64_t* e, int a, int b) {
     return n;
 }
 
-// Entries of sorted e[0, n) (ascending position: key_upos) at positions < pos.
-__device__ __forceinline__ int count_below(const uint64_t* e, int n, uint32_t pos) {
-    int lo = 0, hi = n;
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (key_upos(e[mid]) < pos) lo = mid + 1;
-        else hi = mid;
-    }
-    return lo;
-}
-
-__global__ void __launch_bounds__(CW_MAX_WARPS * 32) select_cand_kernel(const SelectParams p,
-                                                                        int warps) {
-    extern __shared__ __align__(16) uint8_t smem_c[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rr = blockIdx.x * warps + warp;
-    if (warp >= warps || rr >= p.nrows) return;   // whole warps; no block barriers below
-    const int C = p.C, K = p.K;
-    const int M = cw_slots(C);
-    uint64_t* e = reinterpret_cast<uint64_t*>(smem_c + (size_t)warp * cw_warp_bytes(C));
-    uint32_t* hist = reinterpret_cast<uint32_t*>(e + M);
-
-    // row r: its causal limit, candidate row, score row and key scales (as
-    // select_kernel reads a candidate row)
-    const int r = p.row0 + rr;
-    const size_t ostride = p.out_stride ? (size_t)p.out_stride : (size_t)K;
-    int32_t* out = p.out_idx + (size_t)(r - p.out_base) * ostride;
-    float* outs = p.out_score ? p.out_score + (size_t)(r - p.out_base) * ostride : nullptr;
-    bool ok;
-    const int lim = select_row_limit(p, r, ok) - p.lim_shift;
-    if (!ok && lane == 0) raise_error(ERRBIT_DATA);
-    const bool dec = p.scan_kind == SCAN_DECODE_DENSE;
-    const bool var = p.scan_kind == SCAN_VARLEN_DENSE;
-    const int grp = dec ? r / p.Gm : (var ? seg_group_of(p.seg, p.g, r) : r / p.g);
-    const int32_t* cand = p.cand + (size_t)(grp - p.cand_base) * C;
-    // adaptive C: entries past the group's count are not candidates
-    int Cg = C;
-    if (p.cand_count) {
-        const int c = p.cand_count[grp - p.cand_base];
-        Cg = c < 0 ? 0 : (c < C ? c : C);
-    }
-    const float* S = p.s_per_group ? p.S + (size_t)(grp - p.cand_base) * p.S_stride
-                                   : p.S + (size_t)(r - p.row0) * p.S_stride;
-    const float* ksc = nullptr;
-    if (p.key_scale)
-        ksc = p.key_scale + (dec ? (size_t)grp * p.maxlen
-                                 : (var ? (size_t)p.seg.tok[seg_find(p.seg.tok, p.seg.nseq, r)]
-                                        : 0));
-
-    // 1. keys: each lane issues CW_BATCH independent loads of positions and
-    //    scores, then their key scales, before using any of them (a warp has
-    //    few threads to hide a row's memory latency with)
-    uint32_t nvalid = 0;
-    for (int i0 = 0; i0 < C; i0 += 32 * CW_BATCH) {
-        int pos[CW_BATCH];
-        float x[CW_BATCH];
-#pragma unroll
-        for (int u = 0; u < CW_BATCH; ++u) {
-            const int i = i0 + u * 32 + lane;
-            pos[u] = (ok && i < Cg) ? cand[i] : -1;
-            x[u] = i < Cg ? S[i] : 0.0f;
-        }
-        if (ksc) {
-            float sc[CW_BATCH];
-#pragma unroll
-            for (int u = 0; u < CW_BATCH; ++u)
-                sc[u] = (pos[u] >= 0 && pos[u] <= lim) ? ksc[pos[u]] : 1.0f;
-#pragma unroll
-            for (int u = 0; u < CW_BATCH; ++u) x[u] = x[u] * sc[u];
-        }
-#pragma unroll
-        for (int u = 0; u < CW_BATCH; ++u) {
-            const int i = i0 + u * 32 + lane;
-            const bool valid = pos[u] >= 0 && pos[u] <= lim;
-            if (i < C) e[i] = valid ? make_key(ordered_key(x[u]), pos[u]) : 0ull;
-            nvalid += valid;
-        }
-    }
-    for (int i = C + lane; i < M; i += 32) e[i] = 0ull;
-    for (int o = 16; o > 0; o >>= 1) nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
-    __syncwarp();
-    // descents between consecutive valid positions (0 or 1: at most two
-    // ascending runs, split where the descent is), from shared memory
-    uint32_t ndesc = 0;
-    int split = C;
-    int carry = -1;   // the last valid position before this chunk
-    for (int i0 = 0; i0 < C; i0 += 32) {
-        const int i = i0 + lane;
-        const uint64_t k = i < C ? e[i] : 0ull;
-        const int pos = k ? key_pos(k) : -1;
-        const unsigned vm = __ballot_sync(0xffffffffu, pos >= 0);
-        const unsigned below = vm & ((1u << lane) - 1u);
-        const int src = below ? 31 - __clz(below) : lane;
-        int prev = __shfl_sync(0xffffffffu, pos, src);
-        if (!below) prev = carry;
-        const unsigned dm = __ballot_sync(0xffffffffu, pos >= 0 && prev >= 0 && pos < prev);
-        if (dm && ndesc == 0) split = i0 + __ffs(dm) - 1;
-        ndesc += __popc(dm);
-        if (vm) carry = __shfl_sync(0xffffffffu, pos, 31 - __clz(vm));
-    }
-    const uint32_t Kp = nvalid < (uint32_t)K ? nvalid : (uint32_t)K;
-
-    // 2. keep exactly the top Kp keys (score, then lower position)
-    if (Kp < nvalid) {
-        const uint32_t T = warp_kth_largest_f([&](int i) { return key_u(e[i]); }, C, Kp, hist);
-        uint32_t above = 0, eq = 0;
-        for (int i = lane; i < C; i += 32) {
-            const uint32_t u = key_u(e[i]);
-            above += u > T;
-            eq += u == T;
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-            above += __shfl_xor_sync(0xffffffffu, above, o);
-            eq += __shfl_xor_sync(0xffffffffu, eq, o);
-        }
-        const uint32_t need = Kp - above;   // 1 <= need <= eq
-        uint32_t Lmin = 0;                  // tied entries kept: low key half >= Lmin
-        if (eq > need)
-            Lmin = warp_kth_largest_f(
-                [&](int i) { return key_u(e[i]) == T ? (uint32_t)e[i] : 0u; }, C, need, hist);
-        __syncwarp();
-        for (int i = lane; i < C; i += 32) {
-            const uint64_t k = e[i];
-            const uint32_t u = key_u(k);
-            if (u < T || (u == T && (uint32_t)k < Lmin)) e[i] = 0ull;
-        }
-        __syncwarp();
-    }
-
-    // 3. output.  Position order: merge the two runs when each run's
-    //    selected entries are strictly ascending (always, for the proxy
-    //    scan's candidate rows; checked, since any row may be passed in).
-    bool merged = false;
-    if (!p.rank_order && ndesc <= 1) {
-        const int a = warp_compact(e, 0, split);
-        const int b = warp_compact(e, split, C);
-        const uint64_t* eb = e + split;
-        bool asc = true;
-        for (int i = lane; i + 1 < a; i += 32) asc = asc && key_upos(e[i]) < key_upos(e[i + 1]);
-        for (int i = lane; i + 1 < b; i += 32) asc = asc && key_upos(eb[i]) < key_upos(eb[i + 1]);
-        if (__all_sync(0xffffffffu, asc)) {
-            for (int i = lane; i < a + b; i += 32) {
-                const bool in_a = i < a;
-                const uint64_t k = in_a ? e[i] : eb[i - a];
-                const int own = in_a ? i : i - a;
-                const uint32_t pos = key_upos(k);
-                const int slot = own + (in_a ? count_below(eb, b, pos) : count_below(e, a, pos));
-                if (!PIVOT_CHECK(slot >= 0 && slot < (int)Kp)) continue;
-                out[slot] = (int32_t)pos;
-                if (outs) outs[slot] = key_to_float(key_u(k));
-            }
-            merged = true;
-        }
-    }
-    if (!merged) {
-        const int n = warp_compact(e, 0, C);
-        const int Mn = pow2_at_least(n < 1 ? 1 : n);
-        for (int i = n + lane; i < Mn; i += 32) e[i] = 0ull;
-        __syncwarp();
-        if (p.rank_order)
-            warp_bitonic(e, Mn, [](uint64_t x, uint64_t y) { return x > y; });
-        else   // ascending position; the zero padding (position 0xFFFFFFFF) last
-            warp_bitonic(e, Mn, [](uint64_t x, uint64_t y) { return key_upos(x) < key_upos(y); });
-        for (int i = lane; i < n; i += 32) {
-            out[i] = key_pos(e[i]);
-            if (outs) outs[i] = key_to_float(key_u(e[i]));
-        }
-    }
-    for (int i = (int)Kp + lane; i < K; i += 32) {
-        out[i] = -1;
-        if (outs) outs[i] = -INFINITY;
-    }
-}
-
 // ------------------------------------------------------------ fused selection
 //
 // Prefix rows whose scan ran in filter mode.  A sample scan scored every
@@ -1152,7 +962,6 @@ __global__ void __launch_bounds__(CW_MAX_WARPS * 32) select_cand_kernel(const Se
 // answer is exact.
 
 constexpr int FB_WARPS = 8;              // bound kernel: rows a block
-constexpr int FB_MAX_SAMPLES = 4096;     // samples a bound reads at most
 constexpr int FF_MAX_WARPS = 8;
 constexpr int FF_AUX = 1024;             // warp-select words beside its entries: histogram, prefix
 
@@ -1177,23 +986,22 @@ __global__ void __launch_bounds__(FB_WARPS * 32) sample_bound_kernel(const Fused
     if (blockIdx.x == 0 && threadIdx.x == 0) *p.miss_count = 0;
     const int rr = blockIdx.x * FB_WARPS + warp;
     if (rr >= p.nrows) return;
-    uint32_t* v = reinterpret_cast<uint32_t*>(smem_b) + (size_t)warp * (FB_MAX_SAMPLES + THR_BINS);
-    uint32_t* hist = v + FB_MAX_SAMPLES;
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem_b) + (size_t)warp * THR_BINS;
     bool ok;
     const int lim = fused_lim(p, p.row0 + rr, ok) - p.lim_shift;
     const int n = lim + 1;
     uint32_t T = 1;
     if (ok && n > p.cap) {
+        // every sample of the row, read in place (each pass of the warp
+        // select re-reads the row, written just before and still in L2)
         const int ns = samples_upto(lim, p.kts);
-        const int step = (ns + FB_MAX_SAMPLES - 1) / FB_MAX_SAMPLES;
-        const int nt = (ns + step - 1) / step;
         const float* row = p.samp + (size_t)rr * p.samp_stride;
-        for (int j = lane; j < nt; j += 32) v[j] = ordered_key(row[(size_t)j * step]);
-        __syncwarp();
-        const double m0 = (double)p.K * nt / n;
+        const double m0 = (double)p.K * ns / n;
         long long m = (long long)ceil(m0 + (double)p.sigmas * sqrt(m0));
         if (m < 1) m = 1;
-        if (m <= nt) T = warp_kth_largest(v, nt, (uint32_t)m, hist);
+        if (m <= ns)
+            T = warp_kth_largest_f([&](int j) { return ordered_key(row[j]); }, ns, (uint32_t)m,
+                                   hist);
         // else: too few samples to bound the row; it keeps everything and
         // takes the fallback
     }
@@ -1358,60 +1166,62 @@ __global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const F
                 out[i] = key_pos(e[i]);
                 if (outs) outs[i] = key_to_float(key_u(e[i]));
             }
-        } else if ((size_t)kept * 8 + (size_t)((lim >> 5) + 1) * 8 <= (size_t)M * 8) {
-            // position order by a bitmap of the row's positions: each kept
-            // entry's slot is its class's base plus its rank among the
-            // class's marked positions (per-word prefix counts)
+        } else if ((M - kept) >= 32) {
+            // position order by a bitmap of the row's positions, a window of
+            // WW words at a time in the space past the kept entries (bitmap,
+            // then per-word prefix counts): each kept entry's slot is its
+            // class's base plus its rank among the class's marked positions
             const int W = (lim >> 5) + 1;
+            const int WW = min(W, (M - kept) & ~31);
             uint32_t* bm = reinterpret_cast<uint32_t*>(e + kept);
-            uint32_t* pref = bm + W;
+            uint32_t* pref = bm + WW;
             uint32_t base = 0;
             for (int cls = 0; cls < (split ? 2 : 1); ++cls) {
-                for (int w = lane; w < W; w += 32) bm[w] = 0u;
-                __syncwarp();
-                for (int i = lane; i < kept; i += 32) {
-                    const uint64_t k = e[i];
-                    const uint32_t u = key_u(k);
-                    const bool inA = !split || u > TA || (u == TA && (uint32_t)k >= LA);
-                    if (inA == (cls == 0)) {
-                        const int pos = key_pos(k);
-                        if (PIVOT_CHECK(pos >= 0 && (pos >> 5) < W))
-                            atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+                for (int w0 = 0; w0 < W; w0 += WW) {
+                    const int nw = min(WW, W - w0);
+                    for (int w = lane; w < nw; w += 32) bm[w] = 0u;
+                    __syncwarp();
+                    for (int i = lane; i < kept; i += 32) {
+                        const uint64_t k = e[i];
+                        const uint32_t u = key_u(k);
+                        const bool inA = !split || u > TA || (u == TA && (uint32_t)k >= LA);
+                        const int wd = (key_pos(k) >> 5) - w0;
+                        if (inA == (cls == 0) && wd >= 0 && wd < nw)
+                            atomicOr(&bm[wd], 1u << (key_pos(k) & 31));
                     }
-                }
-                __syncwarp();
-                const int per = (W + 31) / 32;
-                const int w0 = lane * per, w1 = min(W, w0 + per);
-                uint32_t local = 0;
-                for (int w = w0; w < w1; ++w) local += __popc(bm[w]);
-                uint32_t inc = local;
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-                    if (lane >= o) inc += y;
-                }
-                uint32_t acc = inc - local;
-                for (int w = w0; w < w1; ++w) {
-                    pref[w] = acc;
-                    acc += __popc(bm[w]);
-                }
-                const uint32_t ncls = __shfl_sync(0xffffffffu, inc, 31);
-                __syncwarp();
-                for (int i = lane; i < kept; i += 32) {
-                    const uint64_t k = e[i];
-                    const uint32_t u = key_u(k);
-                    const bool inA = !split || u > TA || (u == TA && (uint32_t)k >= LA);
-                    if (inA == (cls == 0)) {
+                    __syncwarp();
+                    const int per = (nw + 31) / 32;
+                    const int v0 = lane * per, v1 = min(nw, v0 + per);
+                    uint32_t local = 0;
+                    for (int w = v0; w < v1; ++w) local += __popc(bm[w]);
+                    uint32_t inc = local;
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+                        if (lane >= o) inc += y;
+                    }
+                    uint32_t acc = inc - local;
+                    for (int w = v0; w < v1; ++w) {
+                        pref[w] = acc;
+                        acc += __popc(bm[w]);
+                    }
+                    const uint32_t nwin = __shfl_sync(0xffffffffu, inc, 31);
+                    __syncwarp();
+                    for (int i = lane; i < kept; i += 32) {
+                        const uint64_t k = e[i];
+                        const uint32_t u = key_u(k);
+                        const bool inA = !split || u > TA || (u == TA && (uint32_t)k >= LA);
                         const int pos = key_pos(k);
-                        if (!PIVOT_CHECK(pos >= 0 && (pos >> 5) < W)) continue;
+                        const int wd = (pos >> 5) - w0;
+                        if (inA != (cls == 0) || wd < 0 || wd >= nw) continue;
                         const uint32_t slot =
-                            base + pref[pos >> 5] + __popc(bm[pos >> 5] & ((1u << (pos & 31)) - 1u));
+                            base + pref[wd] + __popc(bm[wd] & ((1u << (pos & 31)) - 1u));
                         if (!PIVOT_CHECK(slot < Kp)) continue;
                         out[slot] = pos;
                         if (outs) outs[slot] = key_to_float(u);
                     }
+                    base += nwin;
+                    __syncwarp();
                 }
-                base += ncls;
-                __syncwarp();
             }
         } else {
             // sort key: class (A first), then position, with the score kept
@@ -1465,7 +1275,9 @@ static SelectLayout select_layout(int K, int tail_cap, int fast_cap, int W, bool
     return L;
 }
 
-__global__ void __launch_bounds__(SEL_THREADS) select_kernel(const SelectParams p) {
+// Two CTAs an SM (64 registers a thread): a row's barrier-separated phases
+// leave the SM idle unless another row fills the gaps.
+__global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelectParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem);
     uint32_t* scratch = hist + HIST_BINS;
@@ -1499,7 +1311,13 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const SelectParams 
         const bool var = p.scan_kind == SCAN_VARLEN_DENSE;
         const int grp = dec ? r / p.Gm : (var ? seg_group_of(p.seg, p.g, r) : r / p.g);
         v.cand = p.cand + (size_t)(grp - p.cand_base) * p.C;
-        v.n = ok ? p.C : 0;
+        // adaptive C: entries past the group's count are not candidates
+        int Cg = p.C;
+        if (p.cand_count) {
+            const int c = p.cand_count[grp - p.cand_base];
+            Cg = c < 0 ? 0 : (c < p.C ? c : p.C);
+        }
+        v.n = ok ? Cg : 0;
         if (p.key_scale)
             v.ksc = p.key_scale + (dec ? (size_t)grp * p.maxlen
                                        : (var ? (size_t)p.seg.tok[seg_find(p.seg.tok, p.seg.nseq, r)]
@@ -1547,16 +1365,23 @@ cudaError_t launch_row_threshold(const SelectParams& p_in, uint32_t* thresh, cud
     cudaError_t e = cudaFuncSetAttribute(row_threshold_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(row_threshold_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     const int grid = (p.nrows + THR_WARPS - 1) / THR_WARPS;
     row_threshold_kernel<<<grid, THR_WARPS * 32, smem, stream>>>(p, thresh);
     return cudaGetLastError();
 }
 
-int fused_cap(int K) { return K <= 4096 ? 8192 : 16384; }
+// Survivor capacity of a fused row: 2 pow2(K) keys (K = 2048: 4096 keys,
+// 36 KB of shared memory a warp with its auxiliary words, six warps an SM).
+// The bound leaves about K (1 + 4.5 / sqrt(m0)) survivors, m0 >= 64 samples
+// for rows longer than the capacity: 1.6 K at most on average.
+int fused_cap(int K) { return 2 * pow2_at_least(K < 128 ? 128 : K); }
 
 cudaError_t launch_sample_bound(const FusedSelectParams& p, cudaStream_t stream) {
     if (p.nrows <= 0) return cudaSuccess;
-    const size_t smem = (size_t)FB_WARPS * (FB_MAX_SAMPLES + THR_BINS) * 4;
+    const size_t smem = (size_t)FB_WARPS * THR_BINS * 4;
     cudaError_t e = cudaFuncSetAttribute(sample_bound_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -1567,12 +1392,16 @@ cudaError_t launch_sample_bound(const FusedSelectParams& p, cudaStream_t stream)
 cudaError_t launch_fused_finish(const FusedSelectParams& p, cudaStream_t stream) {
     if (p.nrows <= 0) return cudaSuccess;
     const size_t per = (size_t)p.cap * 8 + FF_AUX * 4;
-    int warps = (int)(CW_SMEM_LIMIT / per);
-    if (warps > FF_MAX_WARPS) warps = FF_MAX_WARPS;
-    if (warps < 1) return cudaErrorInvalidValue;
+    // one or two warps a block: blocks pack the SM's shared memory more
+    // tightly than one large block would
+    int warps = per * 2 <= CW_SMEM_LIMIT / 2 ? 2 : 1;
+    if (per > CW_SMEM_LIMIT) return cudaErrorInvalidValue;
     const size_t smem = per * (size_t)warps;
     cudaError_t e = cudaFuncSetAttribute(fused_finish_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(fused_finish_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     fused_finish_kernel<<<(p.nrows + warps - 1) / warps, warps * 32, smem, stream>>>(p, warps);
     return cudaGetLastError();
@@ -1583,23 +1412,8 @@ size_t select_smem_bytes(int K, int tail_cap) {
 }
 
 // Candidate rows: one warp each, as many warps per CTA as the slices fit.
-static cudaError_t launch_select_cand(const SelectParams& p, cudaStream_t stream) {
-    const size_t per = cw_warp_bytes(p.C);
-    int warps = (int)(CW_SMEM_LIMIT / per);
-    if (warps > CW_MAX_WARPS) warps = CW_MAX_WARPS;
-    if (warps < 1) return cudaErrorInvalidValue;
-    const size_t smem = per * (size_t)warps;
-    cudaError_t e = cudaFuncSetAttribute(select_cand_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int grid = (p.nrows + warps - 1) / warps;
-    select_cand_kernel<<<grid, warps * 32, smem, stream>>>(p, warps);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_select(const SelectParams& p_in, cudaStream_t stream) {
     if (p_in.nrows <= 0) return cudaSuccess;
-    if (p_in.kind == SEL_CANDIDATES) return launch_select_cand(p_in, stream);
     SelectParams p = p_in;
     p.bitmap_words = (p.npos + 31) / 32;
     p.fast_cap = select_fast_cap(p.K);
@@ -1611,6 +1425,10 @@ cudaError_t launch_select(const SelectParams& p_in, cudaStream_t stream) {
     if (lay.total > SELECT_SMEM_LIMIT) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)lay.total);
+    if (e != cudaSuccess) return e;
+    // the whole carveout as shared memory, so two CTAs fit where their buffers allow
+    e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     select_kernel<<<p.nrows, SEL_THREADS, lay.total, stream>>>(p);
     return cudaGetLastError();
