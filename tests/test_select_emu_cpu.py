@@ -68,6 +68,7 @@ def _run(exe, *args):
     (9000, 300, 0, 1, 3, 1),        # five distinct values: ties decided by position
     (9000, 64, 0, 2, 3, 0),         # signed zeros, bound sampled inside the select
     (20000, 1, 0, 3, 2, 1),         # k = 1 under a heavy tail
+    (20000, 4096, 2048, 1, 3, 1),   # k = 4096 with a split: the trimmed boundary buffer, ties
 ])
 def test_prefix_rows_match_a_sort(select_check, L, K, split, dist, rows, bound):
     _run(select_check, "prefix", L, K, split, dist, rows, bound)

@@ -818,8 +818,10 @@ static pivot_status_t dense_index_impl(const pivot_seq_t* seq, int32_t topk, int
                       seq->q_scale, seq->k, seq->L, seq->k_scale, seq->L, 1, 1, 0, nullptr, P, r0,
                       r1, r1 - 1, S, stride, s);
         if (st != PIVOT_OK) return st;
+        // positions of these rows are < r1: bitmaps of r1 bits (smaller
+        // shared memory for the early chunks, more CTAs an SM)
         st = run_select_prefix(SCAN_PREFILL_DENSE, r0, r1, seq->L, 1, 1, 0, nullptr, S, stride,
-                               topk, 0, seq->L, idx, score, t0, s, thresh, lim_shift, out_stride);
+                               topk, 0, r1, idx, score, t0, s, thresh, lim_shift, out_stride);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;
@@ -930,7 +932,7 @@ pivot_status_t pivot_proxy_scan(const pivot_seq_t* seq, int32_t g, const void* p
                       stride, s);
         if (st != PIVOT_OK) return st;
         st = run_select_prefix(SCAN_PREFILL_PROXY, r0, r1, seq->L, g, 1, 0, nullptr, S, stride, C,
-                               topk, seq->L, cand, cand_score, j0, s, thresh);
+                               topk, e_last + 1, cand, cand_score, j0, s, thresh);
         if (st != PIVOT_OK) return st;
     }
     return PIVOT_OK;

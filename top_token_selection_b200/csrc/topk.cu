@@ -1411,13 +1411,26 @@ size_t select_smem_bytes(int K, int tail_cap) {
     return select_layout(K, tail_cap, 0, 0, false).total;
 }
 
-// Candidate rows: one warp each, as many warps per CTA as the slices fit.
+// Shared memory a CTA may take for two to fit an SM (228 KB, less 1 KB
+// reserved a CTA and the kernel's static words).
+constexpr size_t SELECT_TWO_CTAS = 233472 / 2 - 1024 - 64;
+
 cudaError_t launch_select(const SelectParams& p_in, cudaStream_t stream) {
     if (p_in.nrows <= 0) return cudaSuccess;
     SelectParams p = p_in;
     p.bitmap_words = (p.npos + 31) / 32;
     p.fast_cap = select_fast_cap(p.K);
     SelectLayout lay = select_layout(p.K, p.tail_cap, p.fast_cap, p.bitmap_words, p.split > 0);
+    // Where the exact path's boundary buffer is what keeps a second CTA off
+    // the SM (k = 4096: 2 x 4096 + 4096 keys), trim it a little: a fuller
+    // boundary bin is then searched from global memory, with the same result.
+    if (lay.total > SELECT_TWO_CTAS && lay.exact_bytes >= lay.fast_bytes) {
+        const int trim = (int)((lay.total - SELECT_TWO_CTAS + 7) / 8);
+        if (trim <= p.tail_cap / 4) {
+            p.tail_cap -= trim;
+            lay = select_layout(p.K, p.tail_cap, p.fast_cap, p.bitmap_words, p.split > 0);
+        }
+    }
     if (lay.total > SELECT_SMEM_LIMIT) {   // rows too long for the bitmaps: exact path only
         p.fast_cap = 0;
         lay = select_layout(p.K, p.tail_cap, 0, p.bitmap_words, p.split > 0);
