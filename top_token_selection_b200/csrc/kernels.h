@@ -172,7 +172,6 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
 // SEL_PREFIX rows: per-row lower bound for the select's fast path, written
 // to thresh[r - row0] (one warp per row; p.thresh is ignored).
 cudaError_t launch_row_threshold(const SelectParams& p, uint32_t* thresh, cudaStream_t stream);
-size_t select_smem_bytes(int K, int tail_cap);
 
 struct ReduceParams {
     int dtype, esize, H, D;

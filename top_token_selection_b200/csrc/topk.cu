@@ -1407,9 +1407,6 @@ cudaError_t launch_fused_finish(const FusedSelectParams& p, cudaStream_t stream)
     return cudaGetLastError();
 }
 
-size_t select_smem_bytes(int K, int tail_cap) {
-    return select_layout(K, tail_cap, 0, 0, false).total;
-}
 
 // Shared memory a CTA may take for two to fit an SM (228 KB, less 1 KB
 // reserved a CTA and the kernel's static words).
