@@ -409,7 +409,7 @@ def run_reference(args, wl):
     value = p.L / t
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": gen.DTYPE_NAMES[wl["dtype"]], "data": "synthetic",
             "config": config_of(wl, args),
             "cpu_baseline": {"value": value, "unit": "queries/s", "cores": threads,
