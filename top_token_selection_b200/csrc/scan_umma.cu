@@ -22,13 +22,12 @@
 // columns) so the epilogue of tile i overlaps the MMAs of tile i+1.
 //
 // Warp roles.  Warp 0 loads (one lane issuing TMA in scan mode; all 32 lanes
-// copying in gather mode, with warp 14 as a second copier), warp 1 allocates
-// TMEM and issues tcgen05.mma, and the epilogue warps reduce: in scan mode
-// warps 4-19, four per TMEM lane quarter (a block of 256 / H rows, N = 256:
-// at H = 64 each epilogue warp owns one row, whose 64 head weights stay in
-// registers -- reloading them from shared memory every tile competed with the
-// tensor cores' operand reads); in gather mode warps 2-13, three per quarter
-// (N = 192 at H >= 32).
+// copying in gather mode, with warp 18 as a second copier), warp 1 allocates
+// TMEM and issues tcgen05.mma, and warps 2-17 reduce, four per TMEM lane
+// quarter: a block of 256 / H rows (N = 256), so at H = 64 each epilogue
+// warp owns one row.  The block's halved head weights sit in shared memory
+// (read as float4 broadcasts): four warps per quarter with 64 weights each in
+// registers do not fit the 96 registers five warps a sub-partition leave.
 #include "common.cuh"
 #include "kernels.h"
 
