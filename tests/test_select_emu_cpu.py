@@ -69,6 +69,11 @@ def _run(exe, *args):
     (9000, 64, 0, 2, 3, 0),         # signed zeros, bound sampled inside the select
     (20000, 1, 0, 3, 2, 1),         # k = 1 under a heavy tail
     (20000, 4096, 2048, 1, 3, 1),   # k = 4096 with a split: the trimmed boundary buffer, ties
+    # rows to 128K (4096 bitmap words): proxy rows (k = 4096, the top 2048
+    # first) in two CTAs' shared memory, with and without ties at the k-th
+    (131072, 4096, 2048, 0, 2, 1),
+    (131072, 4096, 2048, 4, 2, 1),
+    (131072, 2048, 0, 4, 2, 1),
 ])
 def test_prefix_rows_match_a_sort(select_check, L, K, split, dist, rows, bound):
     _run(select_check, "prefix", L, K, split, dist, rows, bound)

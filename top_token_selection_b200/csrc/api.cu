@@ -1055,8 +1055,8 @@ size_t pivot_refine_adaptive_workspace_size(const pivot_seq_t* seq, int32_t g, i
                                             int32_t topk) {
     const size_t inner = pivot_refine_workspace_size(seq, g, C, topk);
     if (inner == 0) return 0;
-    int t0, t1;
-    check_seq(seq, &t0, &t1);
+    int t0 = 0, t1 = 0;
+    if (check_seq(seq, &t0, &t1) != PIVOT_OK) return 0;
     return inner + align_up((size_t)ceil_div(t1 - t0, g) * 4, WS_ALIGN);
 }
 

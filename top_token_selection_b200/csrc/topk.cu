@@ -296,12 +296,27 @@ __device__ __forceinline__ uint32_t rank_of(const uint32_t* bm, const uint32_t* 
     return pref[pos >> 5] + __popc(bm[pos >> 5] & ((1u << (pos & 31)) - 1u));
 }
 
+// The need-th largest low key word among the entries whose score key is Tu
+// (1 <= need < their count): lower positions have larger low words, and no
+// two are equal.  Kept out of line: only rows with many tied scores take it.
+__device__ __noinline__ uint32_t tie_bound(const uint64_t* buf, int cnt, uint32_t Tu,
+                                           uint32_t need, uint32_t* hist, uint32_t* scratch) {
+    uint32_t above;
+    return kth_largest_linear(
+        [&](int i) {
+            const uint64_t k = buf[i];
+            return key_u(k) == Tu ? (uint32_t)(k & 0xFFFFFFFFu) : 0u;
+        },
+        cnt, need, hist, scratch, &above);
+}
+
 // Mark in `bm` the kept entries with u > Tu, plus the `need` lowest-position
-// entries with u == Tu.  `tie` is a scratch bitmap, `pref` scratch prefixes.
-// When every entry equal to Tu is taken (the usual case: one of them), the
-// ranking of the ties is skipped.
+// entries with u == Tu.  When more entries than that equal Tu, the lowest
+// positions among them are found by the linear-bin search over the keys'
+// low words (larger for lower positions, and distinct), in `hist`; when every
+// entry equal to Tu is taken (the usual case: one of them), that is skipped.
 __device__ void mark_top(const uint64_t* buf, int cnt, uint32_t Tu, uint32_t need, uint32_t* bm,
-                         uint32_t* tie, uint32_t* pref, int W, uint32_t* scratch) {
+                         int W, uint32_t* hist, uint32_t* scratch) {
     uint32_t nties = 0;
     for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
         const uint64_t k = buf[i];
@@ -314,34 +329,13 @@ __device__ void mark_top(const uint64_t* buf, int cnt, uint32_t Tu, uint32_t nee
         }
     }
     nties = block_sum_u32(nties, scratch);   // also orders the marks above
-    if (nties <= need) {
-        for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
-            const uint64_t k = buf[i];
-            if (key_u(k) == Tu) {
-                const int pos = key_pos(k);
-                if (PIVOT_CHECK(pos >= 0 && (pos >> 5) < W)) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
-            }
-        }
-        __syncthreads();
-        return;
-    }
-    for (int w = threadIdx.x; w < W; w += SEL_THREADS) tie[w] = 0;
-    __syncthreads();
+    // tied entries with a low key word >= lowmin are taken
+    const uint32_t lowmin = nties > need ? tie_bound(buf, cnt, Tu, need, hist, scratch) : 0u;
     for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
         const uint64_t k = buf[i];
-        if (key_u(k) == Tu) {
+        if (key_u(k) == Tu && (uint32_t)(k & 0xFFFFFFFFu) >= lowmin) {
             const int pos = key_pos(k);
-            if (PIVOT_CHECK(pos >= 0 && (pos >> 5) < W)) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
-        }
-    }
-    __syncthreads();
-    bitmap_prefix(tie, pref, W, scratch);
-    for (int i = threadIdx.x; i < cnt; i += SEL_THREADS) {
-        const uint64_t k = buf[i];
-        if (key_u(k) == Tu) {
-            const int pos = key_pos(k);
-            if (PIVOT_CHECK(pos >= 0 && (pos >> 5) < W) && rank_of(tie, pref, pos) < need)
-                atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+            if (PIVOT_CHECK(pos >= 0 && (pos >> 5) < W)) atomicOr(&bm[pos >> 5], 1u << (pos & 31));
         }
     }
     __syncthreads();
@@ -404,7 +398,6 @@ struct FastSmem {
     uint32_t* scratch;  // 64
     uint64_t* buf;      // fast_cap kept entries
     uint32_t* bmS;      // selected positions (W words)
-    uint32_t* bmT;      // ties / class-B scratch (W words)
     uint32_t* bmA;      // class A, only when split (W words)
     uint32_t* pref;     // W prefix counts (aliases hist when W <= HIST_BINS)
 };
@@ -560,10 +553,11 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
     const int split = (!p.rank_order && p.split > 0 && (uint32_t)p.split < Kp) ? p.split : 0;
     uint32_t TuS = 0;
     if (split) TuS = kth_largest_linear(uval, n, (uint32_t)split, hist, scratch, &aboveS);
-    // selected set (the linear bins are no longer needed, so pref may alias them)
+    // selected set (mark_top may take the linear bins again for ties; pref,
+    // which may alias them, is used only after it)
     for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmS[w] = 0;
     __syncthreads();
-    mark_top(buf, n, TuK, Kp - aboveK, sm.bmS, sm.bmT, sm.pref, W, scratch);
+    mark_top(buf, n, TuK, Kp - aboveK, sm.bmS, W, hist, scratch);
     if (p.rank_order) {
         write_rank_order(buf, n, sm.bmS, Kp, K, out, outs);
         return true;
@@ -572,13 +566,14 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
         write_marked(buf, n, sm.bmS, sm.pref, W, 0, scratch, out, outs, K);
     } else {
         // class A: the top `split`; class B: the rest of the selected set
+        // (bmS less class A, in place)
         for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmA[w] = 0;
         __syncthreads();
-        mark_top(buf, n, TuS, (uint32_t)split - aboveS, sm.bmA, sm.bmT, sm.pref, W, scratch);
+        mark_top(buf, n, TuS, (uint32_t)split - aboveS, sm.bmA, W, hist, scratch);
         write_marked(buf, n, sm.bmA, sm.pref, W, 0, scratch, out, outs, K);
-        for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmT[w] = sm.bmS[w] & ~sm.bmA[w];
+        for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmS[w] &= ~sm.bmA[w];
         __syncthreads();
-        write_marked(buf, n, sm.bmT, sm.pref, W, (uint32_t)split, scratch, out, outs, K);
+        write_marked(buf, n, sm.bmS, sm.pref, W, (uint32_t)split, scratch, out, outs, K);
     }
     pad_row(Kp, K, out, outs);
     return true;
@@ -1253,25 +1248,30 @@ __global__ void __launch_bounds__(FF_MAX_WARPS * 32) fused_finish_kernel(const F
 }  // namespace
 
 // Shared-memory layout, in bytes from the start of the dynamic buffer:
-//   hist [HIST_BINS] u32 | scratch [64] u32 | hist256 [256] u32 | region
-// region (8-byte aligned) is either the exact path's sel [2 * pow2(K)] +
-// tail [tail_cap] keys, or the fast path's buf [fast_cap] keys followed by
-// the bitmaps bmS, bmT (and bmA when split) and, when W > HIST_BINS, pref.
+//   hist [HIST_BINS] u32 | scratch [64] u32 | hist256 [256] u32 | exact region
+// The exact path's region (after hist256) holds sel [2 * pow2(K)] + tail
+// [tail_cap] keys.  The fast path, which has no use for hist256, starts its
+// region there: buf [fast_cap] keys, then the bitmaps bmS (and bmA when
+// split) and, when W > HIST_BINS, pref.  All offsets are multiples of 16
+// bytes up to the bitmaps, which take 32-bit accesses only.
 struct SelectLayout {
-    size_t region_off, exact_bytes, fast_bytes, total;
+    size_t exact_total, fast_total, total;
 };
+
+constexpr size_t SEL_FAST_OFF = (size_t)(HIST_BINS + 64) * 4;
+constexpr size_t SEL_EXACT_OFF = SEL_FAST_OFF + 256 * 4;
 
 static SelectLayout select_layout(int K, int tail_cap, int fast_cap, int W, bool split) {
     SelectLayout L{};
-    L.region_off = (size_t)(HIST_BINS + 64 + 256) * 4;
     const size_t m2 = (size_t)pow2_at_least(K);
-    L.exact_bytes = (2 * m2 + (size_t)tail_cap) * 8;
-    L.fast_bytes = 0;
+    L.exact_total = SEL_EXACT_OFF + (2 * m2 + (size_t)tail_cap) * 8;
+    L.fast_total = 0;
     if (fast_cap > 0) {
-        const int nbm = split ? 3 : 2;
-        L.fast_bytes = (size_t)fast_cap * 8 + (size_t)(nbm + (W > HIST_BINS ? 1 : 0)) * W * 4;
+        const int nbm = split ? 2 : 1;
+        L.fast_total = SEL_FAST_OFF + (size_t)fast_cap * 8 +
+                       (size_t)(nbm + (W > HIST_BINS ? 1 : 0)) * W * 4;
     }
-    L.total = L.region_off + (L.exact_bytes > L.fast_bytes ? L.exact_bytes : L.fast_bytes);
+    L.total = L.exact_total > L.fast_total ? L.exact_total : L.fast_total;
     return L;
 }
 
@@ -1282,7 +1282,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelectPara
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem);
     uint32_t* scratch = hist + HIST_BINS;
     uint32_t* hist256 = scratch + 64;
-    uint64_t* region = reinterpret_cast<uint64_t*>(hist256 + 256);
+    uint64_t* region = reinterpret_cast<uint64_t*>(hist256 + 256);   // exact path
     const int M2 = pow2_at_least(p.K);
     __shared__ uint32_t s_a, s_b;
 
@@ -1331,12 +1331,11 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelectPara
         FastSmem sm;
         sm.hist = hist;
         sm.scratch = scratch;
-        sm.buf = region;
-        uint32_t* bms = reinterpret_cast<uint32_t*>(region + p.fast_cap);
+        sm.buf = reinterpret_cast<uint64_t*>(hist256);   // fast path: from hist256 on
+        uint32_t* bms = reinterpret_cast<uint32_t*>(sm.buf + p.fast_cap);
         sm.bmS = bms;
-        sm.bmT = bms + W;
-        sm.bmA = p.split > 0 ? bms + 2 * W : nullptr;
-        sm.pref = W > HIST_BINS ? bms + (p.split > 0 ? 3 : 2) * W : hist;
+        sm.bmA = p.split > 0 ? bms + W : nullptr;
+        sm.pref = W > HIST_BINS ? bms + (p.split > 0 ? 2 : 1) * W : hist;
         if (select_fast(p, v, sm, &s_a, &s_b, out, outs)) return;
         __syncthreads();
     }
@@ -1421,8 +1420,8 @@ cudaError_t launch_select(const SelectParams& p_in, cudaStream_t stream) {
     // Where the exact path's boundary buffer is what keeps a second CTA off
     // the SM (k = 4096: 2 x 4096 + 4096 keys), trim it a little: a fuller
     // boundary bin is then searched from global memory, with the same result.
-    if (lay.total > SELECT_TWO_CTAS && lay.exact_bytes >= lay.fast_bytes) {
-        const int trim = (int)((lay.total - SELECT_TWO_CTAS + 7) / 8);
+    if (lay.exact_total > SELECT_TWO_CTAS && lay.fast_total <= SELECT_TWO_CTAS) {
+        const int trim = (int)((lay.exact_total - SELECT_TWO_CTAS + 7) / 8);
         if (trim <= p.tail_cap / 4) {
             p.tail_cap -= trim;
             lay = select_layout(p.K, p.tail_cap, p.fast_cap, p.bitmap_words, p.split > 0);
