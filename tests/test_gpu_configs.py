@@ -6,7 +6,8 @@ Each test names the workload it stands for:
 * dsa_prefill_16k: L = 16384, bf16, g = 8, C = 4096;
 * fp8_prefill_16k: the same with FP8 e4m3 codes and per-token scales;
 * dsa_prefill_64k at g = 16, C = 8192 (the sweep's widest point);
-* long_prefill_128k_fp8: L = 131072, FP8, g = 8, C = 4096 (the headline);
+* long_prefill_128k_fp8: L = 131072, FP8, g = 8, C = 4096 (the headline),
+  and the same sizes with integer-valued bf16 codes (exact scores, ties);
 * mtp_decode_b32: 32 cached sequences of 32768..131072 FP8 keys, two MTP
   tokens per step, C = 4096, k = 2048.
 
@@ -116,6 +117,39 @@ def test_dsa_prefill_64k_g16_c8192():
 def test_long_prefill_128k_fp8_sampled():
     p, cfg = _workload("long_prefill_128k_fp8")
     _check_prefill(p, cfg["g"], cfg["C"], cfg["topk"], nrows=16, ngroups=12)
+
+
+def test_long_prefill_128k_integer_exact():
+    """Integer-valued bf16 codes at the headline's sizes (L = 131072, H = 64,
+    D = 128, g = 8, C = 4096, k = 2048): every score is exact in fp32 and
+    equal scores are common, so sampled dense rows, candidate rows (the
+    proxy's top-k first), Reuse and Refine rows equal the oracle's bit for
+    bit -- the long rows' selection in two CTAs an SM, and its search among
+    tied scores, included."""
+    L, g, C, kk = 131072, 8, 4096, 2048
+    p = gen.make_prefill(L, 64, 128, BF16, kind="int", seed=9)
+    dev = to_device(p)
+    seq = seq_of(dev)
+    q, qs, w, k, ks = p.codes()
+    rows = _sample(L, 12, extra=(kk - 1, kk, C))
+    groups = _sample(L // g, 10, extra=(C // g - 1, C // g))
+    idx, _ = pv.dense_index(seq, kk)
+    got = idx[rows].cpu().numpy()
+    del idx
+    assert_rows_exact(got, oracle.dense_index(BF16, q, qs, w, k, ks, kk, rows=rows)[0], "dense")
+    pq, pqs, pw = pv.proxy_reduce(seq, g)
+    cand, _ = pv.proxy_scan(seq, g, pq, pqs, pw, C, kk)
+    reu = pv.reuse(0, L, g, cand, kk)
+    ref, _ = pv.refine(seq, g, cand, kk)
+    torch.cuda.synchronize()
+    assert pv.device_error() == 0
+    opq, opqs, opw = oracle.proxy_reduce(BF16, q, qs, w, g)
+    ocand, _ = oracle.proxy_scan(BF16, opq, opqs, opw, k, ks, L, g, C, kk, groups=groups)
+    assert_rows_exact(cand[groups].cpu().numpy(), ocand, "cand")
+    gc = cand.cpu().numpy()
+    assert_rows_exact(reu[rows].cpu().numpy(), oracle.reuse(L, g, gc, kk, rows=rows), "reuse")
+    assert_rows_exact(ref[rows].cpu().numpy(),
+                      oracle.refine(BF16, q, qs, w, k, ks, g, gc, kk, rows=rows)[0], "refine")
 
 
 def test_mtp_decode_b32_sampled():
