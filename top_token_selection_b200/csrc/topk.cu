@@ -20,7 +20,8 @@
 //      memory (warp-aggregated);
 //   3. if between K and the buffer capacity entries were kept, they hold the
 //      top K exactly; the exact K-th score is found by radix passes over
-//      linear bins (no sort); ties at it are resolved by position rank;
+//      linear bins (no sort); of the entries tied at it, the lowest
+//      positions are taken (the same search over their position words);
 //   4. positions go into a bitmap; prefix popcounts give every selected
 //      entry its output slot, so rows come out in position order unsorted.
 // Otherwise (threshold missed, K > 8192, rows too long for the bitmaps) the
