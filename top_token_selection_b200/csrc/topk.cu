@@ -13,9 +13,11 @@
 // K largest keys" is exactly the answer.
 //
 // One CTA per row.  Fast path:
-//   1. a lower bound T for the kept scores: the m-th largest of 4096 evenly
-//      spaced sampled scores, m chosen so about 1.4 K entries of the row
-//      should lie at or above it (all entries when the row is short);
+//   1. a lower bound T for the kept scores: the m-th largest of sampled
+//      scores (prefix rows: 2048, in 64 runs of 32, by row_threshold_kernel
+//      ahead of the select; other long rows: 4096 evenly spaced, inside it),
+//      m chosen so about 1.4 K entries of the row should lie at or above it
+//      (all entries when the row is short);
 //   2. one vectorised pass appends every eligible entry >= T to shared
 //      memory (warp-aggregated);
 //   3. if between K and the buffer capacity entries were kept, they hold the
