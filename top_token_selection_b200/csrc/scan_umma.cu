@@ -92,7 +92,14 @@ struct ItemInfo {
 };
 
 // Scan mode: item i = (row block, chunk of key tiles); items whose chunk
-// starts beyond the block's causal extent are empty.
+// starts beyond the block's causal extent are empty.  Prefill launches number
+// their items chunk by chunk (every row block's first chunk, then every
+// block's second, ...): item i runs on CTA i mod grid, so numbering block by
+// block gave CTA c only the chunks congruent to c modulo gcd(grid, chunks a
+// block), and at L = 16384 (four chunks a block, 148 CTAs) a quarter of the
+// CTAs got every block's first chunk while another quarter only got the
+// fourth chunks of the longest rows.  Decode launches (few row blocks of
+// ragged lengths) keep the block-by-block numbering.
 // Gather mode: item i = (group, block of that group's member rows); the
 // tiles cover the C candidates.  Every role walks the same item sequence.
 template <bool GATHER>
@@ -138,8 +145,15 @@ __device__ __forceinline__ ItemInfo scan_item(const ScanParams& p, int item) {
                 return it;
             }
         } else {
-            const int blk = item / p.items_per_block;
-            chunk = item % p.items_per_block;
+            int blk;
+            if (p.kind == SCAN_PREFILL_DENSE || p.kind == SCAN_PREFILL_PROXY) {
+                const int nblocks = p.nitems / p.items_per_block;   // items_per_block >= 1
+                chunk = item / nblocks;
+                blk = item % nblocks;
+            } else {
+                blk = item / p.items_per_block;
+                chunk = item % p.items_per_block;
+            }
             it.row_first = p.row0 + blk * p.P;
             const int rows = p.row0 + p.nrows - it.row_first;
             it.rows = rows < p.P ? rows : p.P;
