@@ -52,12 +52,14 @@ FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 # DRAM bytes per causal pair of the dense scan kernel, from one ncu capture
 # of the fp8_prefill_16k dense scan (dram__bytes_read.sum +
 # dram__bytes_write.sum over its causal pairs; the summary is under
-# profiles/).  Valid only for the kernel sources it was taken on: the bench
-# reports it while these files hash (sha1, first 12 hex digits) as listed,
-# and null otherwise.
-SCAN_TRAFFIC = {"bytes_per_pair": 5.932,
-                "sources": {"scan_umma.cu": "3f398271ab66", "common.cuh": "e15e822467cd",
-                            "segments.h": "fbc71176c053", "kernels.h": "cd53f91c3deb"}}
+# profiles/).  Valid only for the kernel sources and launch code it was
+# taken on (api.cu sets the work items, whose query-block loads are part of
+# the traffic): the bench reports it while these files hash (sha1, first 12
+# hex digits) as listed, and null otherwise.
+SCAN_TRAFFIC = {"bytes_per_pair": 5.119,
+                "sources": {"scan_umma.cu": "61f46778e241", "common.cuh": "e15e822467cd",
+                            "segments.h": "fbc71176c053", "kernels.h": "cd53f91c3deb",
+                            "api.cu": "7ab9d36de145"}}
 
 
 # ---------------------------------------------------------------------------

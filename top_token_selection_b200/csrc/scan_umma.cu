@@ -96,9 +96,9 @@ struct ItemInfo {
 // their items chunk by chunk (every row block's first chunk, then every
 // block's second, ...): item i runs on CTA i mod grid, so numbering block by
 // block gave CTA c only the chunks congruent to c modulo gcd(grid, chunks a
-// block), and at L = 16384 (four chunks a block, 148 CTAs) a quarter of the
-// CTAs got every block's first chunk while another quarter only got the
-// fourth chunks of the longest rows.  Decode launches (few row blocks of
+// block): with four chunks a block and 148 CTAs, a quarter of the CTAs got
+// every block's first chunk while another quarter only got the fourth
+// chunks of the longest rows.  Decode launches (few row blocks of
 // ragged lengths) keep the block-by-block numbering.
 // Gather mode: item i = (group, block of that group's member rows); the
 // tiles cover the C candidates.  Every role walks the same item sequence.
