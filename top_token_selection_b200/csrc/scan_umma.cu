@@ -330,7 +330,7 @@ __global__ void __maxnreg__(EpiShape<GATHER>::MAXREG)
                 }
             } else {
                 // Gather mode: two warps copy each tile's 128 candidate key rows
-                // (warp 0 rows 0-63, warp 14 rows 64-127) with 16-byte cp.async
+                // (warp 0 rows 0-63, warp 18 rows 64-127) with 16-byte cp.async
                 // straight into the swizzled tile layout.  Each publishes its half
                 // of a tile (an arrive on full[stage], which expects both) once
                 // its copies have landed and been fenced for the tensor cores; up
@@ -411,27 +411,30 @@ __global__ void __maxnreg__(EpiShape<GATHER>::MAXREG)
                             break;
                         }
                         const uint32_t dst = smem_u32(sA + stage * A_BYTES);
-                        // Lane l copies tile rows l + 32 (jb + j), its own
-                        // positions, 16 bytes at a time.  Chunk c of row r sits at
-                        // (r / 8) 1024 + (r % 8) 128 + ((c ^ r % 8) 16): with the
-                        // tile 1024-byte aligned that is rowbase XOR (c 16), where
-                        // rowbase holds r % 8 in bits 4-6.  The chunks of a row go
-                        // out in consecutive instructions, so after the first the
-                        // line is in L1 (.ca); the loop is two instructions a chunk.
+                        // Eight lanes copy one row together: in instruction i
+                        // lanes 8q .. 8q + 7 take the 16-byte chunks c = lane % 8
+                        // of this warp's row 4i + q, whose position the lane that
+                        // read it passes by a shuffle, so each instruction reads
+                        // four whole 128-byte lines (one line a chunk per lane had
+                        // each instruction touch 32 lines: 256-byte bf16 rows took
+                        // 18.1 ms of Refine scan at L = 64K, C = 8192, now 11.4).
+                        // Chunk c of row r sits at (r / 8) 1024 + (r % 8) 128 +
+                        // ((c ^ r % 8) 16), the 128-byte swizzle of a 1024-byte
+                        // aligned tile.
+                        {
+                            const uint32_t c = (uint32_t)(lane & 7);
     #pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const int r = (jb + j) * 32 + lane;
-                            const int pos = cur[j];
-                            const size_t row = (size_t)(it.keybase + ((pos >= 0 && pos < it.nkeys) ? pos : 0));
-                            const uint8_t* src = kbytes + row * ROWB;
-                            const uint32_t x = (uint32_t)(r & 7);
-                            const uint32_t rowbase = dst + (uint32_t)(r >> 3) * 1024u + x * 128u + (x << 4);
-    #pragma unroll
-                            for (int c = 0; c < 8; ++c) {
+                            for (int i = 0; i < 16; ++i) {
+                                const int rl = 4 * i + (lane >> 3);
+                                const int pos = __shfl_sync(0xffffffffu, cur[i >> 3], rl & 31);
+                                const int r = jb * 32 + rl;
+                                const size_t row = (size_t)(it.keybase + ((pos >= 0 && pos < it.nkeys) ? pos : 0));
+                                const uint8_t* src = kbytes + row * ROWB + c * 16;
+                                const uint32_t x = (uint32_t)(r & 7);
+                                const uint32_t d = dst + (uint32_t)(r >> 3) * 1024u + x * 128u + ((c ^ x) << 4);
     #pragma unroll
                                 for (int kb = 0; kb < KBLK; ++kb)
-                                    cp_async16_ca((rowbase ^ ((uint32_t)c << 4)) + kb * (128 * 128),
-                                                  src + kb * 128 + c * 16);
+                                    cp_async16_ca(d + kb * (128 * 128), src + kb * 128);
                             }
                         }
                         cp_async_commit();
