@@ -219,6 +219,63 @@ __device__ int find_threshold_bin(const uint32_t* hist, int nbins, uint32_t need
     return r;
 }
 
+// One pass of the linear-bin search: hist[b] = the count of values u in
+// [lo, hi] with floor((u - lo) LBINS / (hi - lo + 1)) == b.
+template <class F>
+__device__ void linear_histogram(F vals, int n, uint32_t lo, uint32_t hi, uint32_t* hist) {
+    const uint64_t range = (uint64_t)hi - lo + 1;
+    for (int b = threadIdx.x; b < LBINS; b += SEL_THREADS) hist[b] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += SEL_THREADS) {
+        const uint32_t u = vals(i);
+        if (u && u >= lo && u <= hi) {
+            const uint32_t b = (uint32_t)(((uint64_t)(u - lo) * LBINS) / range);
+            atomicAdd(&hist[b], 1u);
+        }
+    }
+    __syncthreads();
+}
+
+// [lo, hi] narrowed to the values of bin b of that pass.
+__device__ __forceinline__ void narrow_to_bin(int b, uint32_t& lo, uint32_t& hi) {
+    const uint64_t range = (uint64_t)hi - lo + 1;
+    const uint32_t nlo = lo + (uint32_t)(((uint64_t)b * range + LBINS - 1) / LBINS);
+    const uint32_t nhi = lo + (uint32_t)(((uint64_t)(b + 1) * range + LBINS - 1) / LBINS) - 1;
+    lo = nlo;
+    hi = nhi;
+}
+
+// The search from a range [lo, hi] that holds the wanted value, `remaining`
+// the rank still wanted inside it and `above_total` the values counted above
+// it so far.
+template <class F>
+__device__ uint32_t kth_in_range(F vals, int n, uint32_t remaining, uint32_t lo, uint32_t hi,
+                                 uint32_t above_total, uint32_t* hist, uint32_t* scratch,
+                                 uint32_t* above_out) {
+    while (lo < hi) {
+        linear_histogram(vals, n, lo, hi, hist);
+        uint32_t above;
+        const int b = find_threshold_bin(hist, LBINS, remaining, scratch, &above);
+        remaining -= above;
+        above_total += above;
+        narrow_to_bin(b, lo, hi);
+    }
+    *above_out = above_total;
+    return lo;
+}
+
+// The smallest and largest values >= 1 (lo > hi when there are none).
+template <class F>
+__device__ void value_range(F vals, int n, uint32_t* scratch, uint32_t& lo, uint32_t& hi) {
+    uint32_t lo_l = 0xFFFFFFFFu, hi_l = 0;
+    for (int i = threadIdx.x; i < n; i += SEL_THREADS) {
+        const uint32_t u = vals(i);
+        if (u) { lo_l = min(lo_l, u); hi_l = max(hi_l, u); }
+    }
+    lo = block_min_u32(lo_l, scratch);
+    hi = block_max_u32(hi_l, scratch);
+}
+
 // The m-th largest value among n uint32 values >= 1 (values 0 are ignored),
 // 1 <= m <= the count of such values: repeated histograms over LBINS linear
 // bins of the remaining value range.  *above_out = the count of values
@@ -226,38 +283,35 @@ __device__ int find_threshold_bin(const uint32_t* hist, int nbins, uint32_t need
 template <class F>
 __device__ uint32_t kth_largest_linear(F vals, int n, uint32_t m, uint32_t* hist,
                                        uint32_t* scratch, uint32_t* above_out) {
-    uint32_t lo_l = 0xFFFFFFFFu, hi_l = 0;
-    for (int i = threadIdx.x; i < n; i += SEL_THREADS) {
-        const uint32_t u = vals(i);
-        if (u) { lo_l = min(lo_l, u); hi_l = max(hi_l, u); }
+    uint32_t lo, hi;
+    value_range(vals, n, scratch, lo, hi);
+    return kth_in_range(vals, n, m, lo, hi, 0u, hist, scratch, above_out);
+}
+
+// The m1-th and the m2-th largest of the same values (1 <= m1, m2 <= their
+// count): exactly the two searches above, with the range and the first
+// pass's histogram shared.  Returns the m1-th; the m2-th goes to *t2.
+template <class F>
+__device__ uint32_t kth_largest_linear_pair(F vals, int n, uint32_t m1, uint32_t m2,
+                                            uint32_t* hist, uint32_t* scratch,
+                                            uint32_t* above1, uint32_t* above2, uint32_t* t2) {
+    uint32_t lo, hi;
+    value_range(vals, n, scratch, lo, hi);
+    if (!(lo < hi)) {
+        *above1 = 0;
+        *above2 = 0;
+        *t2 = lo;
+        return lo;
     }
-    uint32_t lo = block_min_u32(lo_l, scratch);
-    uint32_t hi = block_max_u32(hi_l, scratch);
-    uint32_t remaining = m, above_total = 0;
-    while (lo < hi) {
-        const uint64_t range = (uint64_t)hi - lo + 1;
-        for (int b = threadIdx.x; b < LBINS; b += SEL_THREADS) hist[b] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < n; i += SEL_THREADS) {
-            const uint32_t u = vals(i);
-            if (u && u >= lo && u <= hi) {
-                const uint32_t b = (uint32_t)(((uint64_t)(u - lo) * LBINS) / range);
-                atomicAdd(&hist[b], 1u);
-            }
-        }
-        __syncthreads();
-        uint32_t above;
-        const int b = find_threshold_bin(hist, LBINS, remaining, scratch, &above);
-        remaining -= above;
-        above_total += above;
-        // bin b holds the u with floor((u - lo) * LBINS / range) == b
-        const uint32_t nlo = lo + (uint32_t)(((uint64_t)b * range + LBINS - 1) / LBINS);
-        const uint32_t nhi = lo + (uint32_t)(((uint64_t)(b + 1) * range + LBINS - 1) / LBINS) - 1;
-        lo = nlo;
-        hi = nhi;
-    }
-    *above_out = above_total;
-    return lo;
+    linear_histogram(vals, n, lo, hi, hist);
+    uint32_t a1, a2;
+    const int b1 = find_threshold_bin(hist, LBINS, m1, scratch, &a1);
+    const int b2 = find_threshold_bin(hist, LBINS, m2, scratch, &a2);
+    uint32_t lo1 = lo, hi1 = hi, lo2 = lo, hi2 = hi;
+    narrow_to_bin(b1, lo1, hi1);
+    narrow_to_bin(b2, lo2, hi2);
+    *t2 = kth_in_range(vals, n, m2 - a2, lo2, hi2, a2, hist, scratch, above2);
+    return kth_in_range(vals, n, m1 - a1, lo1, hi1, a1, hist, scratch, above1);
 }
 
 // Warp-aggregated append of `key` (where pred) to buf[*cnt++]; entries past
@@ -552,10 +606,11 @@ __device__ bool select_fast(const SelectParams& p, const RowView& v, const FastS
     const int n = (int)cnt;
     auto uval = [&](int i) { return key_u(buf[i]); };
     uint32_t aboveK, aboveS = 0;
-    const uint32_t TuK = kth_largest_linear(uval, n, Kp, hist, scratch, &aboveK);
     const int split = (!p.rank_order && p.split > 0 && (uint32_t)p.split < Kp) ? p.split : 0;
     uint32_t TuS = 0;
-    if (split) TuS = kth_largest_linear(uval, n, (uint32_t)split, hist, scratch, &aboveS);
+    const uint32_t TuK = split ? kth_largest_linear_pair(uval, n, Kp, (uint32_t)split, hist,
+                                                          scratch, &aboveK, &aboveS, &TuS)
+                               : kth_largest_linear(uval, n, Kp, hist, scratch, &aboveK);
     // selected set (mark_top may take the linear bins again for ties; pref,
     // which may alias them, is used only after it)
     for (int w = threadIdx.x; w < W; w += SEL_THREADS) sm.bmS[w] = 0;
