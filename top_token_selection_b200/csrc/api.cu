@@ -162,13 +162,18 @@ pivot_status_t from_cuda(cudaError_t e) {
 long long score_stride(int nkeys) { return (long long)align_up((size_t)nkeys, 32); }
 
 // Rows per chunk for `total` rows of `rowbytes` each in `bytes` of
-// workspace: all of them if they fit, else a multiple of `unit` when at
-// least one unit fits, else as many as fit (0 if not even one row fits).
+// workspace: all of them if they fit; else, when at least one unit fits, a
+// multiple of `unit` that splits the rows into as few chunks as fit, of
+// about equal size (a last chunk of a few rows would cost a scan pass and a
+// selection wave of its own: 64 of 131072 rows, 8 of 16384 groups, at the
+// default workspace); else as many as fit (0 if not even one row fits).
 long long chunk_rows(size_t bytes, size_t rowbytes, long long total, int unit) {
     const long long fit = (long long)(bytes / rowbytes);
     if (fit >= total) return total;
-    if (fit >= unit) return fit / unit * unit;
-    return fit;
+    if (fit < unit) return fit;
+    const long long most = fit / unit * unit;
+    const long long n = (total + most - 1) / most;
+    return ((total + n - 1) / n + unit - 1) / unit * unit;   // <= most
 }
 
 // Causal (row, key) pairs of rows [r0, r1): the algorithmic work of a scan.
