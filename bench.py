@@ -59,7 +59,7 @@ FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 SCAN_TRAFFIC = {"bytes_per_pair": 5.121,
                 "sources": {"scan_umma.cu": "3e8b3e987d59", "common.cuh": "e15e822467cd",
                             "segments.h": "fbc71176c053", "kernels.h": "cd53f91c3deb",
-                            "api.cu": "2d80058cd2e7"}}
+                            "api.cu": "2223bc936ec0"}}
 
 
 # ---------------------------------------------------------------------------

@@ -490,8 +490,9 @@ float g_fused_sigmas = 4.5f;
 bool fused_ok(int H, int D, int dtype, int K) {
     return g_fused_on && umma_shape_ok(H, D, dtype) && H >= 32 && K <= MAX_K;
 }
-// Key tiles of one scan work item: prefill items take FUSED_TILES, decode
-// items (few, long rows) 8.
+// Key tiles of one work item of the fused selection's scans (their survivor
+// regions are laid out per item): prefill FUSED_TILES, decode (few, long
+// rows) 8.
 int scan_tiles_per_item(int kind) {
     return (kind == SCAN_DECODE_DENSE || kind == SCAN_DECODE_PROXY) ? 8 : FUSED_TILES;
 }
