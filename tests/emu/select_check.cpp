@@ -15,7 +15,8 @@
 //                                              (selection fused into the scan, see run_fused)
 // dist: 0 normal, 1 few distinct values (heavy ties), 2 signed zeros and
 // small integers, 3 a heavy tail (a few huge scores), 4 normal scores rounded
-// to eighths (a few hundred to a thousand ties at the k-th score); mode: 0 plain, 1 ties,
+// to eighths (a few hundred to a thousand ties at the k-th score), 5 one
+// value everywhere (every entry tied); mode: 0 plain, 1 ties,
 // 2 rows padded with -1, 3 with per-key scales; order: 0 ascending positions,
 // 1 rank order; layout: 0 the proxy scan's two ascending runs, 1 shuffled.
 #include <algorithm>
@@ -69,6 +70,7 @@ float draw(std::mt19937& rng, int dist) {
         case 3: return (rng() % 997 == 0) ? 1e6f * (1 + (float)(rng() % 9))
                                           : std::normal_distribution<float>(0.f, 1.f)(rng);
         case 4: return std::round(std::normal_distribution<float>(0.f, 1.f)(rng) * 8.f) / 8.f;
+        case 5: return 1.5f;
         default: return std::normal_distribution<float>(0.f, 1.f)(rng);
     }
 }

@@ -74,6 +74,7 @@ def _run(exe, *args):
     (131072, 4096, 2048, 0, 2, 1),
     (131072, 4096, 2048, 4, 2, 1),
     (131072, 2048, 0, 4, 2, 1),
+    (20000, 4096, 2048, 5, 3, 1),   # one value everywhere: both split searches see one value
 ])
 def test_prefix_rows_match_a_sort(select_check, L, K, split, dist, rows, bound):
     _run(select_check, "prefix", L, K, split, dist, rows, bound)
